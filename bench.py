@@ -1,0 +1,461 @@
+"""Benchmark of the paged decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+A step is one pass of the whole hot path over one batch: copy-on-write block
+copies (when the workload has any), the cache write of each sequence's new
+token, and the paged decode attention of every sequence.  Default workload:
+the Llama-3-8B-shaped GQA layer (32 q / 8 kv heads, head_dim 128, bf16,
+block 16, 256 sequences, lognormal lengths with median 1024 in [16, 8192]).
+
+Metric: algorithmic HBM bytes of the step / step time (GB/s), with tokens/s
+beside it.  Algorithmic bytes of a decode: every (block, kv head) tile pair
+the tables reach (2 * B * D * 2 bytes each) + q + out + block-table entries +
+seq_lens; of a cache write: new K/V read + written + slots; of a copy: block
+bytes read + written + pairs.
+
+Timing: W untimed steps, then K steps between barriers and device syncs,
+measured with CUDA events on the launching stream (max over ranks for N>1).
+Per-step K/V (1.4 GB here) is far larger than the 126 MB L2, so no flush is
+needed between steps.  The decode kernel's own time comes from events around
+each launch inside the timed region.  The e2e figure repeats the step through
+``PagedDecodeStep`` from pinned host buffers: host->device copies of the
+step's inputs and the device->host copy of the output are inside its timed
+region.  N>1 runs independent sequence shards per GPU (weak scaling); the
+path has no exchange step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode-attention HBM GB/s and % of roofline; tokens/s at Llama-3-8B GQA"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "pa_decode_llama3_8b.md")
+KERNEL_SOURCES = [
+    os.path.join(ROOT, "paged_kv_cache_357_b200", "csrc", "pa_decode.cu"),
+    os.path.join(ROOT, "paged_kv_cache_357_b200", "csrc", "pa_device.cuh"),
+]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description="paged decode step benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="llama3_8b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--num-ctas", type=int, default=0)
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# byte accounting
+# ---------------------------------------------------------------------------
+
+
+def step_bytes(L) -> dict:
+    import numpy as np
+
+    es = 2
+    B, D, Hq, Hkv, S = L.block_size, L.head_dim, L.num_q_heads, L.num_kv_heads, L.num_seqs
+    nb = L.total_blocks_touched()
+    tile_pair = 2 * B * D * es
+    small = 2 * S * Hq * D * es + nb * 4 + S * 4
+    decode = nb * Hkv * tile_pair + small
+    exact = int(L.seq_lens.astype(np.int64).sum()) * Hkv * 2 * D * es + small
+    unique = L.unique_blocks_touched() * Hkv * tile_pair + small
+    T = L.num_new_tokens
+    write = T * Hkv * D * es * 2 * 2 + T * 8
+    n = L.copy_pairs.shape[0]
+    copy = n * 2 * Hkv * B * D * es * 2 + n * 16
+    return dict(decode=decode, decode_token_exact=exact, decode_unique_blocks=unique, write=write, copy=copy,
+                step=decode + write + copy, tile_pair=tile_pair, tiles=nb * Hkv)
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(decode_bytes_per_launch):
+    """dram read+write bytes per decode launch from the committed ncu summary,
+    or None when there is none or the kernel source changed since."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    m_traf = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_traf or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_traf.group(1))
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100", "-i",
+                 gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for(device_index: int) -> str:
+    import torch
+
+    try:
+        u = str(torch.cuda.get_device_properties(device_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(device_index)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+
+def oracle_sample_step(L, seqs):
+    """Build a bounded sample (untimed), then time one oracle step on it."""
+    import oracle
+    from workloads import fill_values_numpy, restrict_layout
+
+    R = restrict_layout(L, seqs)
+    V = fill_values_numpy(R)
+    t0 = time.perf_counter()
+    kp, vp = V.k_pool, V.v_pool
+    if R.copy_pairs.shape[0] > 0:
+        kp, vp = oracle.copy_blocks(kp, vp, R.copy_pairs)
+    if R.num_new_tokens > 0:
+        kp, vp = oracle.cache_write(kp, vp, V.new_k, V.new_v, R.slot_mapping)
+    oracle.decode(V.q, kp, vp, R.block_tables, R.seq_lens, R.scale, R.num_kv_heads, R.dtype)
+    dt = time.perf_counter() - t0
+    return dt, step_bytes(R)["step"]
+
+
+def cpu_baseline(L, budget_s: float) -> dict:
+    """The oracle as it stands on a bounded sample of the workload: whole
+    sequences in a seeded order until ~budget_s of oracle time."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    order = np.random.default_rng(0).permutation(L.num_seqs)
+    t_tot, b_tot, n = 0.0, 0, 0
+    with threadpool_limits(1):
+        for s in order:
+            dt, nbytes = oracle_sample_step(L, [int(s)])
+            t_tot += dt
+            b_tot += nbytes
+            n += 1
+            if t_tot >= budget_s:
+                break
+    return {"value": b_tot / t_tot / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {L.num_seqs} sequences (seeded order), all heads, full step, float64 NumPy, "
+                      f"1 thread, {t_tot:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle, as it stands, timed on the host cores on bounded samples."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from workloads import CONFIGS
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    L = CONFIGS[args.config]()
+    order = np.random.default_rng(0).permutation(L.num_seqs)
+    with threadpool_limits(1):
+        t_one, _ = oracle_sample_step(L, [int(order[0])])
+        per_step_budget = max(0.02, 150.0 / max(1, args.steps + args.warmup))
+        k = int(max(1, min(L.num_seqs, per_step_budget / max(t_one, 1e-6))))
+        times, nbytes = [], 0
+        for i in range(args.warmup + args.steps):
+            seqs = [int(order[(i * k + j) % L.num_seqs]) for j in range(k)]
+            dt, b = oracle_sample_step(L, seqs)
+            if i >= args.warmup:
+                times.append(dt)
+                nbytes += b
+    total = sum(times)
+    value = nbytes / total / 1e9
+    sample = f"{k} sequence(s) of {L.num_seqs} per step (seeded order), all heads, full step, float64 NumPy, 1 thread"
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": L.name, "note": L.note},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_357_b200 as pa
+    from workloads import CONFIGS, fill_values_torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    pa.load()
+    L = CONFIGS[args.config]()
+    V = fill_values_torch(L, dev, value_seed=L.seed + 7 * rank)
+    nbytes = step_bytes(L)
+    tables = torch.from_numpy(L.block_tables).to(dev)
+    lens = torch.from_numpy(L.seq_lens).to(dev)
+    slots = torch.from_numpy(L.slot_mapping).to(dev)
+    pairs = torch.from_numpy(L.copy_pairs.reshape(-1, 2)).to(dev)
+    out = torch.empty_like(V.q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, V.k_pool, args.num_ctas)
+    stream = torch.cuda.Stream(device=dev)
+    has_copy, has_write = L.copy_pairs.shape[0] > 0, L.num_new_tokens > 0
+    launches_per_step = 1 + int(has_copy) + int(has_write)
+
+    def prologue():
+        if has_copy:
+            pa.pa_copy_blocks(pairs, V.k_pool, V.v_pool, status, stream=stream)
+        if has_write:
+            pa.pa_cache_write(V.new_k, V.new_v, slots, V.k_pool, V.v_pool, status, stream=stream)
+
+    def decode():
+        pa.pa_decode(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status, num_ctas=args.num_ctas,
+                     stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            prologue()
+            decode()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_id_for(local))
+    barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for k in range(K):
+            ev[k][0].record(stream)
+            prologue()
+            ev[k][1].record(stream)
+            decode()
+            ev[k][2].record(stream)
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    decode_ms = sorted(ev[k][1].elapsed_time(ev[k][2]) for k in range(K))
+    decode_mean_ms = sum(decode_ms) / K
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} in the timed region")
+
+    # ---- end to end through the public step API, from pinned host buffers
+    host = dict(
+        q=V.q.cpu().pin_memory(), tables=tables.cpu().pin_memory(), lens=lens.cpu().pin_memory(),
+        new_k=V.new_k.cpu().pin_memory(), new_v=V.new_v.cpu().pin_memory(), slots=slots.cpu().pin_memory(),
+        pairs=pairs.cpu().pin_memory() if has_copy else None,
+    )
+    step = pa.PagedDecodeStep(V.k_pool, V.v_pool, L.num_seqs, L.num_q_heads, L.max_blocks_per_seq,
+                              max_new_tokens=L.num_new_tokens, max_copy_pairs=L.copy_pairs.shape[0],
+                              scale=L.scale, num_ctas=args.num_ctas)
+
+    def e2e_step():
+        return step.run(host["q"], host["tables"], host["lens"], host["new_k"], host["new_v"],
+                        host["slots"] if has_write else None, host["pairs"])
+
+    for _ in range(args.warmup):
+        e2e_step()
+    step.stream.synchronize()
+    K2 = max(1, min(K, 500))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(step.stream)
+    for _ in range(K2):
+        e2e_step()
+    e1.record(step.stream)
+    step.stream.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / K2
+    if step.device_status() != 0:
+        raise SystemExit("device status set in the e2e loop")
+
+    # ---- max over ranks
+    t = torch.tensor([elapsed_ms, e2e_ms, decode_mean_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms, decode_mean_ms = (float(x) for x in t.tolist())
+    ms_per_step = elapsed_ms / K
+    value = world * nbytes["step"] / (ms_per_step * 1e-3) / 1e9
+    tokens_per_s = world * L.num_seqs / (ms_per_step * 1e-3)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = nbytes["decode"] / (decode_mean_ms * 1e-3) / 1e9
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": L.dtype,
+            "data": "synthetic",
+            "config": {
+                "workload": L.name,
+                "note": L.note,
+                "global_batch": L.num_seqs * world,
+                "seq_len": {"mean": float(np.mean(L.seq_lens)), "min": int(L.seq_lens.min()),
+                            "max": int(L.seq_lens.max())},
+                "step": "+".join((["pa_copy_blocks"] if has_copy else []) + (["pa_cache_write"] if has_write
+                                                                             else []) + ["pa_decode"]),
+                "l2": f"no flush: per-step K/V {nbytes['decode'] / 1e9:.2f} GB > 126 MB L2",
+                "parallelism": f"dp{world} (independent sequence shards, no collective)",
+            },
+            "tokens_per_s": tokens_per_s,
+            "tokens_per_s_note": "one new token per sequence per single-layer step",
+            "decode_ms": decode_mean_ms,
+            "decode_ms_p50": decode_ms[K // 2],
+            "bytes": nbytes,
+            "roofline": {
+                "kernel": "pa_decode_kernel",
+                "bound": "hbm",
+                "achieved": achieved,
+                "peak": peak,
+                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind,
+                "unit": "GB/s",
+                "frac": achieved / peak,
+                "frac_of_8000_nominal": achieved / 8000.0,
+                "traffic": profiled_traffic(nbytes["decode"]),
+                "algorithmic_bytes_per_launch": nbytes["decode"],
+            },
+            "e2e": {
+                "value": world * nbytes["step"] / (e2e_ms * 1e-3) / 1e9,
+                "unit": "GB/s",
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": step.last_h2d_bytes,
+                "d2h_bytes_per_step": step.last_d2h_bytes,
+                "steps": K2,
+            },
+            "gpu_launches": K * launches_per_step,
+            "clocks": clocks,
+        }
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(L, args.cpu_budget)
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

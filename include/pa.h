@@ -1,0 +1,193 @@
+/*
+ * pa.h — C ABI of libpa, the paged KV-cache decode hot path for NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (PagedAttention): each sequence's keys and values live in
+ * fixed-size physical blocks of `block_size` tokens scattered through one
+ * shared pool and are reached only through a per-sequence block table and a
+ * sequence length ("PagedAttention 与 KV 显存管理" study notes ch.05 §3; vLLM
+ * blog "vLLM 是什么" §2).  Attention over those blocks is merged across
+ * blocks with online softmax (study notes §4); new tokens are stored into
+ * their slots (vLLM blog §1); blocks shared by several outputs are copied
+ * before a write (copy on write, study notes §6.1 and §12 exercise 4).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers to caller-owned memory on the
+ *   current CUDA device; the library allocates and frees nothing.
+ * - Dense row-major layouts, no strides:
+ *     k_pool, v_pool : [num_blocks][num_kv_heads][block_size][head_dim]
+ *     q, out         : [num_seqs][num_q_heads][head_dim]
+ *     k, v (new)     : [num_tokens][num_kv_heads][head_dim]
+ *   Element type fp16 or bf16 (pa_pool_desc.dtype) for q, out, k, v and the
+ *   pools alike.  Every tensor pointer must be 16-byte aligned.
+ * - Token t of a sequence is row (t % block_size) of physical block
+ *   block_tables[s][t / block_size]; a slot is  block * block_size + row.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Every call only enqueues work and returns; results and the
+ *   device status are valid after the stream is synchronised.
+ * - The return value reports what the host can see (bad arguments,
+ *   unsupported shapes, a failed launch).  Errors that depend on device data
+ *   (a block id or slot out of range, a wait that ran out) are written to
+ *   `*dev_status` (int32, device memory, nullable): the first error wins via
+ *   compare-and-swap from PA_DEV_OK, the kernel skips the offending access
+ *   and carries on or returns; it never traps.  Outputs are unspecified
+ *   after a non-zero device status.  With dev_status == NULL such errors
+ *   are still skipped but not reported.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host-side return codes. */
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1, /* null or misaligned pointer, negative or zero size */
+  PA_ERR_UNSUPPORTED = 2, /* no kernel for this block_size/head_dim/group/dtype */
+  PA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+  PA_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+} pa_status;
+
+/* Device-side status codes written to *dev_status (a range of their own,
+ * so pa_status_string names either kind). */
+#define PA_DEV_OK 0
+#define PA_DEV_BAD_BLOCK_ID 101 /* a block_tables entry outside [0, num_blocks) */
+#define PA_DEV_BAD_SEQ_LEN 102 /* seq_lens[s] < 0 or > max_blocks_per_seq * block_size */
+#define PA_DEV_BAD_SLOT 103    /* slot_mapping entry >= num_blocks * block_size */
+#define PA_DEV_BAD_PAIR 104    /* copy pair with src or dst outside [0, num_blocks) */
+#define PA_DEV_TIMEOUT 105     /* a bounded pipeline wait ran out (kernel returned early) */
+
+typedef enum pa_dtype { PA_FP16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Shape of the physical block pool (the same for the K and the V pool). */
+typedef struct pa_pool_desc {
+  int32_t num_blocks;   /* physical blocks in each pool */
+  int32_t block_size;   /* tokens per block: 8, 16 or 32 */
+  int32_t num_kv_heads; /* key/value heads */
+  int32_t head_dim;     /* 64 or 128 */
+  int32_t dtype;        /* pa_dtype */
+} pa_pool_desc;
+
+/* Tuning/test options for pa_decode_ex; zero-initialise for the defaults. */
+typedef struct pa_decode_opts {
+  int32_t num_ctas; /* persistent CTAs; 0 = SM count x resident CTAs per SM */
+  int32_t flags;    /* 0, or PA_DECODE_TEST_WITHHOLD_COPIES */
+} pa_decode_opts;
+
+/* Failure-detection test hook for pa_decode_opts.flags: the producer warp
+ * issues no copies, every consumer wait runs out after about 20 ms, and the
+ * kernel returns early with PA_DEV_TIMEOUT in *dev_status and the GPU context
+ * still usable.  Output is not written.  Never set it outside such tests. */
+#define PA_DECODE_TEST_WITHHOLD_COPIES 1
+
+/*
+ * pa_decode_workspace_bytes — bytes of device scratch pa_decode needs.
+ *
+ * The scratch holds per-CTA partial softmax states (running max, running
+ * sum and unnormalised output of each query head of a kv head) and one
+ * arrival counter per (sequence, kv head).  It depends on the current
+ * device's SM count, so query it with the device current that will run the
+ * decode.  The caller allocates it and must ZERO it once before the first
+ * pa_decode; every pa_decode that ends with PA_DEV_OK leaves the counters at
+ * zero again, so the same workspace serves any number of later calls on the
+ * same stream.  After a non-zero device status, zero it again.  Two decodes
+ * that may run at the same time need separate workspaces.
+ * Returns 0 for invalid arguments.
+ */
+PA_API size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, const pa_pool_desc* pool);
+PA_API size_t pa_decode_workspace_bytes_ex(int32_t num_seqs, int32_t num_q_heads, const pa_pool_desc* pool,
+                                    const pa_decode_opts* opts);
+
+/*
+ * pa_decode — one decode step of paged attention.
+ *
+ * For each sequence s and query head h (kv head h / (num_q_heads /
+ * num_kv_heads), contiguous GQA groups), with n = seq_lens[s]:
+ *   out[s][h] = sum_t softmax_t(scale * q[s][h] . K_t) V_t,  t = 0..n-1,
+ * where K_t / V_t are row t % B of block block_tables[s][t / B] of the
+ * pools (vLLM blog §2: softmax(QK^T/sqrt(d))V through block_table; study
+ * notes ch.05 §4: blocks merged with a running max and running sum).
+ * A sequence with n == 0 gets a zero output.  Rows of a partly filled last
+ * block past n are never read into the result (they may hold anything).
+ *
+ * Arguments
+ *   q               [num_seqs][num_q_heads][head_dim], fp16/bf16
+ *   k_pool, v_pool  [num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_tables    int32 [num_seqs][max_blocks_per_seq]; only the first
+ *                   ceil(n / B) entries of each row are read
+ *   seq_lens        int32 [num_seqs]
+ *   num_q_heads     multiple of pool->num_kv_heads; the group size
+ *                   num_q_heads / num_kv_heads must be 1, 2, 4 or 8
+ *   scale           multiplier of q.K (typically 1/sqrt(head_dim))
+ *   out             [num_seqs][num_q_heads][head_dim], same dtype as q
+ *   workspace       device scratch of at least pa_decode_workspace_bytes()
+ *                   bytes, zeroed before first use (see above)
+ *   dev_status      nullable int32 device pointer (see the conventions)
+ * Accumulation is fp32; the output is rounded to the input dtype.
+ * Device errors: PA_DEV_BAD_SEQ_LEN (that sequence is treated as empty),
+ * PA_DEV_BAD_BLOCK_ID (block 0 is read instead), PA_DEV_TIMEOUT.
+ */
+PA_API pa_status pa_decode(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                    float scale, void* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                    const pa_pool_desc* pool, void* stream);
+
+/* pa_decode with explicit options (e.g. a fixed CTA count; num_ctas = 1
+ * processes every block in one CTA, without any cross-CTA merge). */
+PA_API pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                       int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
+                       int32_t num_q_heads, float scale, void* out, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_status, const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream);
+
+/*
+ * pa_cache_write — store the K/V of new tokens into their slots
+ * (vLLM blog §1: each generated token's K/V is written to the cache;
+ * study notes ch.05 §5 item 2: a token goes to the next free slot).
+ *
+ * For each token t with slot = slot_mapping[t] >= 0:
+ *   k_pool[slot / B][h][slot % B][:] = k[t][h][:]   for every kv head h
+ *   v_pool[slot / B][h][slot % B][:] = v[t][h][:]
+ * A bit copy: no rounding.  Negative slots skip the token (padding).  Two
+ * tokens with the same slot in one call: undefined which one lands.
+ *   k, v          [num_tokens][num_kv_heads][head_dim]
+ *   slot_mapping  int64 [num_tokens]
+ * num_tokens == 0 is a no-op.  Device error: PA_DEV_BAD_SLOT (token skipped).
+ */
+PA_API pa_status pa_cache_write(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                         void* k_pool, void* v_pool, int32_t* dev_status, const pa_pool_desc* pool,
+                         void* stream);
+
+/*
+ * pa_copy_blocks — copy-on-write block copies (study notes ch.05 §6.1: a
+ * writer to a shared block copies it first; §12 exercise 4).
+ *
+ * For each pair i: block src_dst_pairs[2i+1] of both pools becomes a bit
+ * copy of block src_dst_pairs[2i] (all kv heads, all rows).  src == dst is
+ * a no-op.  Pairs run in parallel: a dst that appears twice, or that is
+ * also a src in the same call, is undefined.
+ *   src_dst_pairs int64 [num_pairs][2] (src, dst)
+ * num_pairs == 0 is a no-op.  Device error: PA_DEV_BAD_PAIR (pair skipped).
+ */
+PA_API pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs, void* k_pool, void* v_pool,
+                         int32_t* dev_status, const pa_pool_desc* pool, void* stream);
+
+/* Static string for a pa_status or PA_DEV_* code. */
+PA_API const char* pa_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

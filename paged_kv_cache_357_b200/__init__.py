@@ -1,0 +1,33 @@
+"""paged_kv_cache_357_b200 — PagedAttention's decode hot path on B200 (sm_100a).
+
+The kernels live in ``libpa.so`` (C ABI: ``include/pa.h``), built in-tree by
+``python -m paged_kv_cache_357_b200.build``.  This package is a thin binding:
+
+* ``pa_decode``       paged decode attention with online softmax
+* ``pa_cache_write``  slot-mapped write of new tokens' K/V
+* ``pa_copy_blocks``  copy-on-write block copies
+* ``PagedDecodeStep`` one whole step (copy, write, decode) from host buffers
+
+PyTorch supplies device memory and streams only.
+"""
+
+from ._lib import (  # noqa: F401
+    DEV_STATUS,
+    EXPORTED,
+    LIB_PATH,
+    PA_BF16,
+    PA_DECODE_TEST_WITHHOLD_COPIES,
+    PA_FP16,
+    DecodeOpts,
+    PaError,
+    PoolDesc,
+    alloc_decode_workspace,
+    decode_workspace_bytes,
+    load,
+    pa_cache_write,
+    pa_copy_blocks,
+    pa_decode,
+    pool_desc,
+    status_string,
+)
+from .step import PagedDecodeStep  # noqa: F401

@@ -1,0 +1,238 @@
+"""ctypes binding of libpa (C ABI declared in include/pa.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, their device pointers and sizes are passed to the C entry points,
+and non-zero return codes become ``PaError``.  Every step of the hot path runs
+in libpa's CUDA kernels; there is no fallback of any kind — if libpa.so is
+missing the import of the functions below raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpa.so")
+
+PA_FP16, PA_BF16 = 0, 1
+PA_DECODE_TEST_WITHHOLD_COPIES = 1
+DEV_STATUS = {
+    0: "PA_DEV_OK",
+    101: "PA_DEV_BAD_BLOCK_ID",
+    102: "PA_DEV_BAD_SEQ_LEN",
+    103: "PA_DEV_BAD_SLOT",
+    104: "PA_DEV_BAD_PAIR",
+    105: "PA_DEV_TIMEOUT",
+}
+EXPORTED = (
+    "pa_decode_workspace_bytes",
+    "pa_decode_workspace_bytes_ex",
+    "pa_decode",
+    "pa_decode_ex",
+    "pa_cache_write",
+    "pa_copy_blocks",
+    "pa_status_string",
+)
+
+
+class PoolDesc(ctypes.Structure):
+    _fields_ = [
+        ("num_blocks", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class DecodeOpts(ctypes.Structure):
+    _fields_ = [("num_ctas", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+
+class PaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: libpa returned {code} ({status_string(code)})")
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libpa.so and declare its signatures (raises if it is not built)."""
+    global _LIB
+    if _LIB is not None and path == LIB_PATH:
+        return _LIB
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libpa.so not found at {path}; build it with `python -m paged_kv_cache_357_b200.build` "
+            "(there is no fallback implementation)"
+        )
+    lib = ctypes.CDLL(path)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    pdesc, popts = ctypes.POINTER(PoolDesc), ctypes.POINTER(DecodeOpts)
+    lib.pa_decode_workspace_bytes.argtypes = [i32, i32, pdesc]
+    lib.pa_decode_workspace_bytes.restype = sz
+    lib.pa_decode_workspace_bytes_ex.argtypes = [i32, i32, pdesc, popts]
+    lib.pa_decode_workspace_bytes_ex.restype = sz
+    lib.pa_decode.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, f32, vp, vp, sz, vp, pdesc, vp]
+    lib.pa_decode.restype = i32
+    lib.pa_decode_ex.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, f32, vp, vp, sz, vp, pdesc, popts, vp]
+    lib.pa_decode_ex.restype = i32
+    lib.pa_cache_write.argtypes = [vp, vp, vp, i32, vp, vp, vp, pdesc, vp]
+    lib.pa_cache_write.restype = i32
+    lib.pa_copy_blocks.argtypes = [vp, i32, vp, vp, vp, pdesc, vp]
+    lib.pa_copy_blocks.restype = i32
+    lib.pa_status_string.argtypes = [i32]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    if path == LIB_PATH:
+        _LIB = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().pa_status_string(int(code)).decode()
+
+
+# ---------------------------------------------------------------------------
+# torch-facing helpers (device memory and streams come from PyTorch)
+# ---------------------------------------------------------------------------
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float16:
+        return PA_FP16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"expected fp16 or bf16, got {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _need(t, name, *, dtype=None, ndim=None, device=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def pool_desc(k_pool) -> PoolDesc:
+    """Descriptor of a [num_blocks, num_kv_heads, block_size, head_dim] pool."""
+    nb, hkv, bs, d = k_pool.shape
+    return PoolDesc(nb, bs, hkv, d, _dtype_code(k_pool))
+
+
+def decode_workspace_bytes(num_seqs: int, num_q_heads: int, k_pool, num_ctas: int = 0) -> int:
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, 0)
+    n = load().pa_decode_workspace_bytes_ex(num_seqs, num_q_heads, ctypes.byref(desc), ctypes.byref(opts))
+    if n == 0:
+        raise PaError(1, "pa_decode_workspace_bytes")
+    return int(n)
+
+
+def alloc_decode_workspace(num_seqs: int, num_q_heads: int, k_pool, num_ctas: int = 0):
+    """Zeroed device workspace for pa_decode (see include/pa.h)."""
+    torch = _torch()
+    n = decode_workspace_bytes(num_seqs, num_q_heads, k_pool, num_ctas)
+    return torch.zeros(n, dtype=torch.uint8, device=k_pool.device)
+
+
+def pa_decode(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, workspace, dev_status=None,
+              num_ctas: int = 0, flags: int = 0, stream=None) -> None:
+    """out[s, h] = softmax(scale * q[s, h] . K^T) V over seq_lens[s] paged tokens (pa_decode_ex)."""
+    torch = _torch()
+    _need(k_pool, "k_pool", ndim=4)
+    dev = k_pool.device
+    _need(v_pool, "v_pool", dtype=k_pool.dtype, ndim=4, device=dev)
+    if v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool and v_pool shapes differ")
+    _need(q, "q", dtype=k_pool.dtype, ndim=3, device=dev)
+    _need(out, "out", dtype=k_pool.dtype, ndim=3, device=dev)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2, device=dev)
+    _need(seq_lens, "seq_lens", dtype=torch.int32, ndim=1, device=dev)
+    _need(workspace, "workspace", device=dev)
+    S, Hq, D = q.shape
+    if block_tables.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_tables / seq_lens must have num_seqs rows")
+    if D != k_pool.shape[3]:
+        raise ValueError("head_dim of q and the pools differ")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", dtype=torch.int32, device=dev)
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    rc = load().pa_decode_ex(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), S, Hq,
+        float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+        ctypes.byref(desc), ctypes.byref(opts), _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode")
+
+
+def pa_cache_write(k, v, slot_mapping, k_pool, v_pool, dev_status=None, stream=None) -> None:
+    """Store new tokens' K/V ([T, Hkv, D]) into their slots (pa_cache_write)."""
+    torch = _torch()
+    _need(k_pool, "k_pool", ndim=4)
+    dev = k_pool.device
+    _need(v_pool, "v_pool", dtype=k_pool.dtype, ndim=4, device=dev)
+    _need(k, "k", dtype=k_pool.dtype, ndim=3, device=dev)
+    _need(v, "v", dtype=k_pool.dtype, ndim=3, device=dev)
+    _need(slot_mapping, "slot_mapping", dtype=torch.int64, ndim=1, device=dev)
+    T = k.shape[0]
+    if v.shape != k.shape or slot_mapping.shape[0] != T:
+        raise ValueError("k, v and slot_mapping disagree on the token count")
+    if k.shape[1:] != (k_pool.shape[1], k_pool.shape[3]):
+        raise ValueError("new tokens must be [T, num_kv_heads, head_dim]")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", dtype=torch.int32, device=dev)
+    desc = pool_desc(k_pool)
+    rc = load().pa_cache_write(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_pool), _ptr(v_pool),
+                               _ptr(dev_status), ctypes.byref(desc), _stream(stream))
+    if rc != 0:
+        raise PaError(rc, "pa_cache_write")
+
+
+def pa_copy_blocks(src_dst_pairs, k_pool, v_pool, dev_status=None, stream=None) -> None:
+    """Copy-on-write block copies: block dst of both pools <- block src (pa_copy_blocks)."""
+    torch = _torch()
+    _need(k_pool, "k_pool", ndim=4)
+    dev = k_pool.device
+    _need(v_pool, "v_pool", dtype=k_pool.dtype, ndim=4, device=dev)
+    _need(src_dst_pairs, "src_dst_pairs", dtype=torch.int64, ndim=2, device=dev)
+    if src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [n, 2]")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", dtype=torch.int32, device=dev)
+    desc = pool_desc(k_pool)
+    rc = load().pa_copy_blocks(_ptr(src_dst_pairs), src_dst_pairs.shape[0], _ptr(k_pool), _ptr(v_pool),
+                               _ptr(dev_status), ctypes.byref(desc), _stream(stream))
+    if rc != 0:
+        raise PaError(rc, "pa_copy_blocks")

@@ -1,0 +1,810 @@
+// pa_decode — paged decode attention for sm_100a.
+//
+// What it computes (vLLM blog §2; PagedAttention study notes ch.05 §4):
+//   out[s][h] = softmax(scale * q[s][h] . K^T) V over the seq_lens[s] tokens
+//   of sequence s, K/V reached block by block through block_tables, the
+//   softmax normalisation merged across blocks with a running max and sum.
+//
+// How (B200 design):
+//   * Work list.  All (sequence, kv head, logical block) triples are laid end
+//     to end — sequence-major, kv head next, block innermost — and cut into
+//     gridDim.x equal contiguous ranges, one per persistent CTA (grid = SMs x
+//     resident CTAs).  Every CTA gets the same number of 8 KB K+V tile pairs
+//     whatever the length mix, so ragged batches and long sequences
+//     (split-KV) are one mechanism.  Each CTA derives its range from
+//     seq_lens on the device; the host never reads lengths.
+//   * Producer warp: walks the range, resolves each block's physical id once
+//     (32 table entries per coalesced load), and issues one 1-D bulk copy
+//     (TMA, cp.async.bulk) per K tile and per V tile into a ring of
+//     shared-memory stages signalled by mbarriers; q of each (sequence, kv
+//     head) unit comes the same way into a double-buffered slot.
+//   * Four consumer warps: each owns B/4 rows of every block, computes the
+//     scores of all G query heads of the GQA group with fp32 FMAs, keeps its
+//     own running max / sum / output (online softmax) and accumulates P.V.
+//     At the end of a unit the four states are merged through shared memory.
+//   * Split units (a range boundary inside a unit): the CTA stores its
+//     partial state (max, sum, unnormalised output) in the workspace and
+//     bumps the unit's arrival counter; the last CTA to arrive merges all
+//     partial states with the same rescaling rule and writes the output,
+//     then resets the counter.  No second kernel, no host round trip.
+//   * Masking: rows of the last block past seq_len get a score of -inf by
+//     selection and are skipped in P.V, so whatever those rows hold (NaN
+//     included) never reaches the result.
+//   * Every wait is bounded (pa_device.cuh); a timeout raises the CTA's abort
+//     flag, records PA_DEV_TIMEOUT, drains copies still in flight and returns.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
+constexpr int kRingBytes = 64 * 1024;             // K+V bytes staged per CTA
+constexpr int kMergeBarrier = 1;                  // named barrier of the consumer warps
+
+template <int D, int B, int G>
+struct Cfg {
+  static constexpr int kTileElems = B * D;
+  static constexpr int kTileBytes = kTileElems * 2;
+  static constexpr int kStagesRaw = kRingBytes / (2 * kTileBytes);
+  static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
+  static constexpr int TPW = B / kConsumerWarps;        // rows of a block per consumer warp
+  static constexpr int LPT = (TPW >= 4) ? 8 : 32 / TPW;  // lanes sharing one row in q.k
+  static constexpr int PT = 32 / LPT;                    // rows per q.k pass
+  static constexpr int NPASS = TPW / PT;
+  static constexpr int DPL = D / LPT;  // dims per lane in q.k
+  static constexpr int VEC = DPL >= 8 ? 8 : DPL;
+  static constexpr int NCHUNK = DPL / VEC;
+  static constexpr int DPV = D / 32;                 // dims per lane in p.V
+  static constexpr int kPartStride = G * (D + 2);    // floats per partial slot: m[G], l[G], acc[G][D]
+  static_assert(B % kConsumerWarps == 0, "block size");
+  static_assert(TPW % PT == 0, "rows per pass");
+  static_assert(DPL % VEC == 0 && (VEC == 2 || VEC == 4 || VEC == 8), "q.k vector width");
+  static_assert(DPV == 2 || DPV == 4, "p.V vector width");
+};
+
+template <int D, int B, int G>
+struct __align__(128) DecodeSmem {
+  using C = Cfg<D, B, G>;
+  uint16_t k[C::kStages][C::kTileElems];
+  uint16_t v[C::kStages][C::kTileElems];
+  uint16_t q[2][G * D];
+  float merge_acc[kConsumerWarps][G * D];
+  float merge_m[kConsumerWarps][G];
+  float merge_l[kConsumerWarps][G];
+  float pbuf[kConsumerWarps][C::TPW][G];
+  uint64_t full[C::kStages];
+  uint64_t empty[C::kStages];
+  uint64_t qfull[2];
+  uint64_t qempty[2];
+  long long scan[kThreads / 32];
+  long long total;
+  long long pre0;
+  int s0;
+  int found;
+  int abort;
+  int is_last;
+  int issued;
+  int consumed;
+  int q_issued;
+  int q_consumed;
+};
+
+struct DecodeParams {
+  const uint16_t* q;
+  const uint16_t* k_pool;
+  const uint16_t* v_pool;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  uint16_t* out;
+  float* partials;
+  int32_t* counters;
+  int32_t* status;
+  int max_nb;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int num_blocks;
+  float scale_log2;
+  unsigned long long wait_limit_ns;
+  int test_flags;
+};
+
+constexpr int kFlagTestWithholdCopies = PA_DECODE_TEST_WITHHOLD_COPIES;  // producer issues nothing
+
+__device__ __forceinline__ int checked_len(const DecodeParams& p, int s, int B) {
+  const int n = __ldg(p.seq_lens + s);
+  return (n < 0 || n > p.max_nb * B) ? 0 : n;
+}
+
+struct Cursor {
+  int s, h, j, nb, len;
+  long long x, remaining;
+};
+
+struct Seg {
+  int s, h, j0, n, nb, len;
+  long long unit_first;  // flattened index of block 0 of unit (s, h)
+};
+
+template <int B>
+__device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams& p) {
+  if (c.remaining <= 0) return false;
+  const long long left = c.nb - c.j;
+  const int n = static_cast<int>(left < c.remaining ? left : c.remaining);
+  sg.s = c.s;
+  sg.h = c.h;
+  sg.j0 = c.j;
+  sg.n = n;
+  sg.nb = c.nb;
+  sg.len = c.len;
+  sg.unit_first = c.x - c.j;
+  c.remaining -= n;
+  c.x += n;
+  c.j += n;
+  if (c.j == c.nb) {
+    c.j = 0;
+    if (++c.h == p.num_kv_heads) {
+      c.h = 0;
+      if (c.remaining > 0) {
+        do {
+          if (++c.s >= p.num_seqs) {  // inconsistent lengths: stop cleanly
+            c.remaining = 0;
+            break;
+          }
+          c.len = checked_len(p, c.s, B);
+          c.nb = (c.len + B - 1) / B;
+        } while (c.nb == 0);
+      }
+    }
+  }
+  return true;
+}
+
+// CTA whose range [c*N/C, (c+1)*N/C) holds flattened block x.
+__device__ __forceinline__ long long cta_of(long long x, long long N, long long C) {
+  return ((x + 1) * C - 1) / N;
+}
+
+__device__ __forceinline__ long long range_start(long long c, long long N, long long C) { return c * N / C; }
+
+// Block-wide inclusive scan of one long long per thread (all kThreads threads).
+template <typename Smem>
+__device__ __forceinline__ long long block_inclusive_scan(long long v, Smem& sm, long long& block_total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) sm.scan[warp] = v;
+  __syncthreads();
+  long long before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) {
+    const long long t = sm.scan[w];
+    if (w < warp) before += t;
+    total += t;
+  }
+  __syncthreads();
+  block_total = total;
+  return v + before;
+}
+
+template <bool kBf16, int D, int B, int G>
+__global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams p) {
+  using C = Cfg<D, B, G>;
+  using Smem = DecodeSmem<D, B, G>;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const long long nctas = gridDim.x, cta = blockIdx.x;
+  const int Hkv = p.num_kv_heads, Hq = p.num_q_heads;
+
+  // ---- prologue: total work, zero outputs of empty sequences -------------
+  long long mine = 0;
+  for (int s = tid; s < p.num_seqs; s += kThreads) {
+    const int raw = __ldg(p.seq_lens + s);
+    int n = raw;
+    if (raw < 0 || raw > p.max_nb * B) {
+      if (cta == 0) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
+      n = 0;
+    }
+    if (n == 0 && (s % nctas) == cta) {
+      uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(s) * Hq * D);
+      for (int i = 0; i < Hq * D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+    }
+    mine += (n + B - 1) / B;
+  }
+  long long seq_blocks;
+  (void)block_inclusive_scan(mine, sm, seq_blocks);
+  const long long NBT = seq_blocks * Hkv;
+  // Partition over at most NBT CTAs so that every range is non-empty; the
+  // CTAs that split a unit are then exactly cta_of(first)..cta_of(last).
+  const long long nparts = NBT < nctas ? NBT : nctas;
+  if (cta >= nparts) return;  // uniform across the CTA (also covers NBT == 0)
+  const long long start = range_start(cta, NBT, nparts);
+  const long long end = range_start(cta + 1, NBT, nparts);
+
+  // ---- locate the sequence holding `start` ---------------------------------
+  const long long target = start / Hkv;  // in per-sequence block units
+  if (tid == 0) sm.found = 0;
+  __syncthreads();
+  long long base = 0;
+  for (int chunk = 0; chunk < p.num_seqs; chunk += kThreads) {
+    const int s = chunk + tid;
+    const long long nb = (s < p.num_seqs) ? (checked_len(p, s, B) + B - 1) / B : 0;
+    long long chunk_total;
+    const long long incl = block_inclusive_scan(nb, sm, chunk_total);
+    const long long excl = incl - nb;
+    if (nb > 0 && base + excl <= target && target < base + incl) {
+      sm.s0 = s;
+      sm.pre0 = base + excl;
+      sm.found = 1;
+    }
+    base += chunk_total;
+    __syncthreads();
+    if (sm.found) break;
+  }
+
+  if (tid == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], kConsumerWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.qfull[i], 1);
+      mbar_init(&sm.qempty[i], kConsumerWarps);
+    }
+    sm.abort = 0;
+    sm.issued = 0;
+    sm.consumed = 0;
+    sm.q_issued = 0;
+    sm.q_consumed = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (!sm.found) return;  // only with lengths changing under the kernel
+
+  Cursor cur;
+  cur.s = sm.s0;
+  cur.len = checked_len(p, cur.s, B);
+  cur.nb = (cur.len + B - 1) / B;
+  {
+    const long long off = start - sm.pre0 * Hkv;
+    cur.h = static_cast<int>(off / cur.nb);
+    cur.j = static_cast<int>(off % cur.nb);
+  }
+  cur.x = start;
+  cur.remaining = end - start;
+  const volatile int* abort_flag = &sm.abort;
+
+  if (warp == kConsumerWarps) {
+    // ===================== producer warp ======================================
+    const uint64_t pol_stream = l2_policy_evict_first();
+    int stage = 0, qslot = 0;
+    uint32_t phase = 0, qphase = 0;
+    int issued = 0, q_issued = 0;
+    bool ok = true;
+    if (p.test_flags & kFlagTestWithholdCopies) {
+      // Test hook: issue nothing; the consumers' bounded waits must run out.
+      if (lane == 0) {
+        const uint64_t t0 = global_timer_ns();
+        while (*abort_flag == 0 && global_timer_ns() - t0 < 4 * p.wait_limit_ns) {
+        }
+      }
+      __syncwarp();
+    } else {
+      Seg sg;
+      while (ok && next_seg<B>(cur, sg, p)) {
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&sm.qempty[qslot], qphase ^ 1u, abort_flag, p.wait_limit_ns);
+          if (ok) {
+            mbar_arrive_expect_tx(&sm.qfull[qslot], G * D * 2);
+            const uint16_t* src = p.q + (static_cast<size_t>(sg.s) * Hq + static_cast<size_t>(sg.h) * G) * D;
+            bulk_copy_g2s(sm.q[qslot], src, G * D * 2, &sm.qfull[qslot], pol_stream);
+            ++q_issued;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        qslot ^= 1;
+        if (qslot == 0) qphase ^= 1u;
+        const int32_t* trow = p.block_tables + static_cast<size_t>(sg.s) * p.max_nb;
+        for (int jb = sg.j0; jb < sg.j0 + sg.n && ok; jb += 32) {
+          const int cnt = min(32, sg.j0 + sg.n - jb);
+          int e = 0;
+          if (lane < cnt) {
+            e = __ldg(trow + jb + lane);
+            if (e < 0 || e >= p.num_blocks) {
+              record_status(p.status, PA_DEV_BAD_BLOCK_ID);
+              e = 0;
+            }
+          }
+          for (int k = 0; k < cnt; ++k) {
+            const int phys = __shfl_sync(0xffffffffu, e, k);
+            if (lane == 0) {
+              ok = mbar_wait_bounded(&sm.empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns);
+              if (ok) {
+                const size_t tile = (static_cast<size_t>(phys) * Hkv + sg.h) * C::kTileElems;
+                mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
+                bulk_copy_g2s(sm.k[stage], p.k_pool + tile, C::kTileBytes, &sm.full[stage], pol_stream);
+                bulk_copy_g2s(sm.v[stage], p.v_pool + tile, C::kTileBytes, &sm.full[stage], pol_stream);
+                ++issued;
+              }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+      sm.issued = issued;
+      sm.q_issued = q_issued;
+      if (!ok) {
+        sm.abort = 1;
+        record_status(p.status, PA_DEV_TIMEOUT);
+      }
+    }
+  } else {
+    // ===================== consumer warps =====================================
+    const int ctid = tid;  // 0..127
+    const int c = lane % C::LPT;        // lane's column group inside its row
+    const int rsub = lane / C::LPT;     // row inside a pass
+    int stage = 0, qslot = 0;
+    uint32_t phase = 0, qphase = 0;
+    int consumed = 0, q_consumed = 0;
+    bool ok = true;
+    Seg sg;
+    while (ok && next_seg<B>(cur, sg, p)) {
+      // ---- q of this unit, pre-multiplied by scale*log2(e)
+      ok = mbar_wait_bounded(&sm.qfull[qslot], qphase, abort_flag, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      float qr[G][C::DPL];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int k = 0; k < C::NCHUNK; ++k) {
+          load_f32<kBf16, C::VEC>(&sm.q[qslot][g * D + (k * C::LPT + c) * C::VEC], &qr[g][k * C::VEC]);
+        }
+#pragma unroll
+        for (int i = 0; i < C::DPL; ++i) qr[g][i] *= p.scale_log2;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.qempty[qslot]);
+      ++q_consumed;
+      qslot ^= 1;
+      if (qslot == 0) qphase ^= 1u;
+
+      float m[G], l[G], acc[G][C::DPV];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.f;
+#pragma unroll
+        for (int i = 0; i < C::DPV; ++i) acc[g][i] = 0.f;
+      }
+
+      for (int i = 0; i < sg.n; ++i) {
+        ok = mbar_wait_bounded(&sm.full[stage], phase, abort_flag, p.wait_limit_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const int j = sg.j0 + i;
+        const int valid = (j == sg.nb - 1) ? sg.len - j * B : B;
+        const uint16_t* Kt = sm.k[stage];
+        const uint16_t* Vt = sm.v[stage];
+
+        // ---- scores of this warp's rows for the G heads (log2 domain)
+        float sc[C::NPASS][G];
+#pragma unroll
+        for (int ps = 0; ps < C::NPASS; ++ps) {
+          const int r = warp * C::TPW + ps * C::PT + rsub;
+          float dot[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) dot[g] = 0.f;
+#pragma unroll
+          for (int k = 0; k < C::NCHUNK; ++k) {
+            float kf[C::VEC];
+            load_f32<kBf16, C::VEC>(Kt + r * D + (k * C::LPT + c) * C::VEC, kf);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+#pragma unroll
+              for (int e = 0; e < C::VEC; ++e) dot[g] = fmaf(qr[g][k * C::VEC + e], kf[e], dot[g]);
+            }
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int o = C::LPT / 2; o >= 1; o >>= 1) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], o);
+            sc[ps][g] = (r < valid) ? dot[g] : -INFINITY;
+          }
+        }
+
+        // ---- online softmax update (running max m, running sum l)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float bm = sc[0][g];
+#pragma unroll
+          for (int ps = 1; ps < C::NPASS; ++ps) bm = fmaxf(bm, sc[ps][g]);
+#pragma unroll
+          for (int o = C::LPT; o < 32; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+          const float m_new = fmaxf(m[g], bm);
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          const float alpha = fast_exp2(m[g] - m_use);
+          m[g] = m_new;
+          float psum = 0.f;
+#pragma unroll
+          for (int ps = 0; ps < C::NPASS; ++ps) {
+            const float pr = fast_exp2(sc[ps][g] - m_use);
+            psum += pr;
+            if (c == 0) sm.pbuf[warp][ps * C::PT + rsub][g] = pr;
+          }
+          l[g] = l[g] * alpha + psum;
+#pragma unroll
+          for (int e = 0; e < C::DPV; ++e) acc[g][e] *= alpha;
+        }
+        __syncwarp();
+
+        // ---- P.V over this warp's valid rows
+        int nv = valid - warp * C::TPW;
+        nv = nv < 0 ? 0 : (nv > C::TPW ? C::TPW : nv);
+#pragma unroll
+        for (int t = 0; t < C::TPW; ++t) {
+          if (t < nv) {
+            const int r = warp * C::TPW + t;
+            float vf[C::DPV];
+            load_f32<kBf16, C::DPV>(Vt + r * D + lane * C::DPV, vf);
+            float pt[G];
+            if constexpr (G == 4) {
+              const float4 pv = *reinterpret_cast<const float4*>(&sm.pbuf[warp][t][0]);
+              pt[0] = pv.x;
+              pt[1] = pv.y;
+              pt[2] = pv.z;
+              pt[3] = pv.w;
+            } else {
+#pragma unroll
+              for (int g = 0; g < G; ++g) pt[g] = sm.pbuf[warp][t][g];
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+#pragma unroll
+              for (int e = 0; e < C::DPV; ++e) acc[g][e] = fmaf(pt[g], vf[e], acc[g][e]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        ++consumed;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+
+      // ---- merge the four warps' states of this segment
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int o = C::LPT; o < 32; o <<= 1) l[g] += __shfl_xor_sync(0xffffffffu, l[g], o);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          sm.merge_m[warp][g] = m[g];
+          sm.merge_l[warp][g] = l[g];
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float* dst = &sm.merge_acc[warp][g * D + lane * C::DPV];
+        if constexpr (C::DPV == 4) {
+          *reinterpret_cast<float4*>(dst) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+        } else {
+          *reinterpret_cast<float2*>(dst) = make_float2(acc[g][0], acc[g][1]);
+        }
+      }
+      named_barrier_sync(kMergeBarrier, kConsumerThreads);
+
+      const bool whole_unit = (sg.j0 == 0 && sg.n == sg.nb);
+      const long long F = sg.unit_first;
+      float* my_part = nullptr;
+      if (!whole_unit) {
+        const int slot = (start >= F) ? 0 : 1;
+        my_part = p.partials + (static_cast<size_t>(cta) * 2 + slot) * C::kPartStride;
+      }
+      uint16_t* out_row = p.out + (static_cast<size_t>(sg.s) * Hq + static_cast<size_t>(sg.h) * G) * D;
+      for (int idx = ctid; idx < G * D / 2; idx += kConsumerThreads) {
+        const int g = (2 * idx) / D, d = (2 * idx) % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.merge_m[w][g]);
+        float L = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float sc_w = fast_exp2(sm.merge_m[w][g] - M);
+          L = fmaf(sm.merge_l[w][g], sc_w, L);
+          a0 = fmaf(sm.merge_acc[w][g * D + d], sc_w, a0);
+          a1 = fmaf(sm.merge_acc[w][g * D + d + 1], sc_w, a1);
+        }
+        if (whole_unit) {
+          const float inv = 1.f / L;
+          *reinterpret_cast<uint32_t*>(out_row + g * D + d) = pack2<kBf16>(a0 * inv, a1 * inv);
+        } else {
+          if (d == 0) {
+            my_part[g] = M;
+            my_part[G + g] = L;
+          }
+          *reinterpret_cast<float2*>(&my_part[2 * G + g * D + d]) = make_float2(a0, a1);
+        }
+      }
+      if (!whole_unit) {
+        __threadfence();
+        named_barrier_sync(kMergeBarrier, kConsumerThreads);
+        const long long first = cta_of(F, NBT, nparts);
+        const long long last = cta_of(F + sg.nb - 1, NBT, nparts);
+        int32_t* counter = p.counters + static_cast<size_t>(sg.s) * Hkv + sg.h;
+        if (ctid == 0) {
+          const int prev = atomicAdd(counter, 1);
+          sm.is_last = (prev == static_cast<int>(last - first));
+        }
+        named_barrier_sync(kMergeBarrier, kConsumerThreads);
+        if (sm.is_last) {
+          __threadfence();
+          for (int idx = ctid; idx < G * D / 2; idx += kConsumerThreads) {
+            const int g = (2 * idx) / D, d = (2 * idx) % D;
+            float M = -INFINITY;
+            for (long long cc = first; cc <= last; ++cc) {
+              const int sl = (range_start(cc, NBT, nparts) >= F) ? 0 : 1;
+              const float* pp = p.partials + (static_cast<size_t>(cc) * 2 + sl) * C::kPartStride;
+              M = fmaxf(M, __ldcg(pp + g));
+            }
+            float L = 0.f, a0 = 0.f, a1 = 0.f;
+            for (long long cc = first; cc <= last; ++cc) {
+              const int sl = (range_start(cc, NBT, nparts) >= F) ? 0 : 1;
+              const float* pp = p.partials + (static_cast<size_t>(cc) * 2 + sl) * C::kPartStride;
+              const float sc_p = fast_exp2(__ldcg(pp + g) - M);
+              L = fmaf(__ldcg(pp + G + g), sc_p, L);
+              const float2 av = __ldcg(reinterpret_cast<const float2*>(pp + 2 * G + g * D + d));
+              a0 = fmaf(av.x, sc_p, a0);
+              a1 = fmaf(av.y, sc_p, a1);
+            }
+            const float inv = 1.f / L;
+            *reinterpret_cast<uint32_t*>(out_row + g * D + d) = pack2<kBf16>(a0 * inv, a1 * inv);
+          }
+          if (ctid == 0) *counter = 0;
+        }
+      }
+      named_barrier_sync(kMergeBarrier, kConsumerThreads);
+    }
+    if (tid == 0) {
+      sm.consumed = consumed;
+      sm.q_consumed = q_consumed;
+    }
+    if (!ok && lane == 0) {
+      sm.abort = 1;
+      record_status(p.status, PA_DEV_TIMEOUT);
+    }
+  }
+
+  // ---- epilogue: after an abort, wait (bounded) for copies still in flight
+  __syncthreads();
+  if (tid == 0 && sm.abort) {
+    for (int k = sm.consumed; k < sm.issued; ++k) {
+      (void)mbar_wait_bounded(&sm.full[k % C::kStages], (k / C::kStages) & 1, nullptr, p.wait_limit_ns);
+    }
+    for (int k = sm.q_consumed; k < sm.q_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.qfull[k & 1], (k >> 1) & 1, nullptr, p.wait_limit_ns);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+using KernelFn = void (*)(DecodeParams);
+
+struct Variant {
+  KernelFn fn;
+  int smem_bytes;
+  int part_stride;  // floats per partial slot
+};
+
+template <bool kBf16, int D, int B, int G>
+Variant make_variant() {
+  return Variant{pa_decode_kernel<kBf16, D, B, G>, static_cast<int>(sizeof(DecodeSmem<D, B, G>)),
+                 Cfg<D, B, G>::kPartStride};
+}
+
+template <bool kBf16, int D, int B>
+bool pick_g(int G, Variant& v) {
+  switch (G) {
+    case 1: v = make_variant<kBf16, D, B, 1>(); return true;
+    case 2: v = make_variant<kBf16, D, B, 2>(); return true;
+    case 4: v = make_variant<kBf16, D, B, 4>(); return true;
+    case 8: v = make_variant<kBf16, D, B, 8>(); return true;
+    default: return false;
+  }
+}
+
+template <bool kBf16, int D>
+bool pick_b(int B, int G, Variant& v) {
+  switch (B) {
+    case 8: return pick_g<kBf16, D, 8>(G, v);
+    case 16: return pick_g<kBf16, D, 16>(G, v);
+    case 32: return pick_g<kBf16, D, 32>(G, v);
+    default: return false;
+  }
+}
+
+template <bool kBf16>
+bool pick_d(int D, int B, int G, Variant& v) {
+  switch (D) {
+    case 64: return pick_b<kBf16, 64>(B, G, v);
+    case 128: return pick_b<kBf16, 128>(B, G, v);
+    default: return false;
+  }
+}
+
+static bool select_variant(const pa_pool_desc& pool, int num_q_heads, Variant& v) {
+  if (pool.num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % pool.num_kv_heads != 0) return false;
+  const int G = num_q_heads / pool.num_kv_heads;
+  if (pool.dtype == PA_BF16) return pick_d<true>(pool.head_dim, pool.block_size, G, v);
+  if (pool.dtype == PA_FP16) return pick_d<false>(pool.head_dim, pool.block_size, G, v);
+  return false;
+}
+
+// Resident CTAs per SM and SM count for a variant on the current device
+// (cached per device and kernel).
+static bool grid_size_for(const Variant& v, int& ctas) {
+  struct Entry {
+    int device;
+    KernelFn fn;
+    int ctas;
+  };
+  static std::mutex mu;
+  static Entry cache[256];
+  static int n_cache = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_cache; ++i) {
+      if (cache[i].device == dev && cache[i].fn == v.fn) {
+        ctas = cache[i].ctas;
+        return true;
+      }
+    }
+  }
+  if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem_bytes) != cudaSuccess)
+    return false;
+  int per_sm = 0, sms = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, kThreads, v.smem_bytes) != cudaSuccess)
+    return false;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+  if (per_sm < 1) return false;
+  ctas = per_sm * sms;
+  std::lock_guard<std::mutex> lock(mu);
+  if (n_cache < 256) cache[n_cache++] = Entry{dev, v.fn, ctas};
+  return true;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static size_t workspace_bytes_for(int num_seqs, int num_kv_heads, int ctas, int part_stride) {
+  const size_t parts = align_up(static_cast<size_t>(ctas) * 2 * part_stride * sizeof(float), 256);
+  const size_t counters = align_up(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t), 256);
+  return parts + counters;
+}
+
+static bool pool_shape_ok(const pa_pool_desc* pool) {
+  return pool != nullptr && pool->num_blocks > 0 && pool->block_size > 0 && pool->num_kv_heads > 0 &&
+         pool->head_dim > 0 && (pool->dtype == PA_FP16 || pool->dtype == PA_BF16);
+}
+
+static int resolve_ctas(const Variant& v, const pa_decode_opts* opts) {
+  if (opts != nullptr && opts->num_ctas > 0) return opts->num_ctas;
+  int ctas = 0;
+  return grid_size_for(v, ctas) ? ctas : 0;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" size_t pa_decode_workspace_bytes_ex(int32_t num_seqs, int32_t num_q_heads, const pa_pool_desc* pool,
+                                               const pa_decode_opts* opts) {
+  if (num_seqs < 0 || !pool_shape_ok(pool)) return 0;
+  Variant v;
+  if (!select_variant(*pool, num_q_heads, v)) return 0;
+  const int ctas = resolve_ctas(v, opts);
+  if (ctas <= 0) return 0;
+  return workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
+}
+
+extern "C" size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, const pa_pool_desc* pool) {
+  return pa_decode_workspace_bytes_ex(num_seqs, num_q_heads, pool, nullptr);
+}
+
+extern "C" pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_pool,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                  int32_t num_seqs, int32_t num_q_heads, float scale, void* out, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                                  const pa_decode_opts* opts, void* stream) {
+  if (!pool_shape_ok(pool) || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (num_seqs == 0) return PA_OK;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || block_tables == nullptr || seq_lens == nullptr ||
+      out == nullptr) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) || !std::isfinite(scale)) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (opts != nullptr && (opts->num_ctas < 0 || (opts->flags & ~kFlagTestWithholdCopies) != 0)) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(max_blocks_per_seq) * pool->block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  Variant v;
+  if (!select_variant(*pool, num_q_heads, v)) return PA_ERR_UNSUPPORTED;
+  const int ctas = resolve_ctas(v, opts);
+  if (ctas <= 0) return PA_ERR_CUDA;
+  const size_t need = workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+  if (opts != nullptr && opts->num_ctas > 0) {
+    if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem_bytes) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.k_pool = static_cast<const uint16_t*>(k_pool);
+  prm.v_pool = static_cast<const uint16_t*>(v_pool);
+  prm.block_tables = block_tables;
+  prm.seq_lens = seq_lens;
+  prm.out = static_cast<uint16_t*>(out);
+  prm.partials = static_cast<float*>(workspace);
+  prm.counters = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
+                                            align_up(static_cast<size_t>(ctas) * 2 * v.part_stride * sizeof(float),
+                                                     256));
+  prm.status = dev_status;
+  prm.max_nb = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = pool->num_kv_heads;
+  prm.num_blocks = pool->num_blocks;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const bool test_timeout = opts != nullptr && (opts->flags & kFlagTestWithholdCopies) != 0;
+  prm.wait_limit_ns = test_timeout ? 20ull * 1000 * 1000 : 2ull * 1000 * 1000 * 1000;
+  prm.test_flags = test_timeout ? kFlagTestWithholdCopies : 0;
+
+  v.fn<<<ctas, kThreads, v.smem_bytes, static_cast<cudaStream_t>(stream)>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" pa_status pa_decode(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                               int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
+                               int32_t num_q_heads, float scale, void* out, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                               void* stream) {
+  return pa_decode_ex(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads, scale,
+                      out, workspace, workspace_bytes, dev_status, pool, nullptr, stream);
+}

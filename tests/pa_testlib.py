@@ -1,0 +1,164 @@
+"""Helpers shared by the GPU parity tests: move generator bits to the device,
+run one step through the C-ABI binding, run the oracle step on the same bits,
+and compare.
+
+Tolerance (the reading used throughout): a decode output element passes when
+|gpu - oracle| <= 2e-3 + 1e-2 * |oracle| — max-abs 2e-3 near zero, max-rel
+1e-2 elsewhere, the allclose form; see the design notes for why the two
+bounds combine this way (rounding the output to bf16 alone moves a value of
+magnitude 1 by up to 2^-9 = 1.95e-3).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from workloads import PagedLayout, PagedValues, bits_to_torch
+
+ATOL = 2e-3
+RTOL = 1e-2
+
+
+def to_device(layout: PagedLayout, values: PagedValues, device):
+    """Torch device tensors for one layout (numpy bit arrays or torch tensors)."""
+    import torch
+
+    def t16(x):
+        if isinstance(x, np.ndarray):
+            return bits_to_torch(x, layout.dtype).to(device)
+        return x.to(device)
+
+    return dict(
+        q=t16(values.q),
+        k_pool=t16(values.k_pool).contiguous(),
+        v_pool=t16(values.v_pool).contiguous(),
+        new_k=t16(values.new_k),
+        new_v=t16(values.new_v),
+        tables=torch.from_numpy(layout.block_tables).to(device),
+        lens=torch.from_numpy(layout.seq_lens).to(device),
+        slots=torch.from_numpy(layout.slot_mapping).to(device),
+        pairs=torch.from_numpy(layout.copy_pairs.reshape(-1, 2)).to(device),
+    )
+
+
+def torch_bits(t) -> np.ndarray:
+    """uint16 bit array of a 16-bit torch tensor (any device)."""
+    import torch
+
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def torch_f64(t) -> np.ndarray:
+    return t.detach().cpu().double().numpy()
+
+
+def gpu_step(dev_t, layout: PagedLayout, *, num_ctas: int = 0, do_copy=True, do_write=True, status=None,
+             workspace=None):
+    """copy -> write -> decode through the C ABI; returns (out tensor, status tensor)."""
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    d = dev_t
+    st = torch.zeros(1, dtype=torch.int32, device=d["q"].device) if status is None else status
+    if do_copy and layout.copy_pairs.shape[0] > 0:
+        pa.pa_copy_blocks(d["pairs"], d["k_pool"], d["v_pool"], st)
+    if do_write and layout.num_new_tokens > 0:
+        pa.pa_cache_write(d["new_k"], d["new_v"], d["slots"], d["k_pool"], d["v_pool"], st)
+    out = torch.full_like(d["q"], float("nan"))
+    ws = workspace
+    if ws is None:
+        ws = pa.alloc_decode_workspace(layout.num_seqs, layout.num_q_heads, d["k_pool"], num_ctas)
+    pa.pa_decode(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], layout.scale, out, ws, st,
+                 num_ctas=num_ctas)
+    torch.cuda.synchronize()
+    return out, st
+
+
+def oracle_step(layout: PagedLayout, values: PagedValues, *, do_copy=True, do_write=True):
+    """The same step on the host in float64: returns (out, k_pool, v_pool)."""
+    kp, vp = values.k_pool, values.v_pool
+    if do_copy and layout.copy_pairs.shape[0] > 0:
+        kp, vp = oracle.copy_blocks(kp, vp, layout.copy_pairs)
+    if do_write and layout.num_new_tokens > 0:
+        kp, vp = oracle.cache_write(kp, vp, values.new_k, values.new_v, layout.slot_mapping)
+    out = oracle.decode(values.q, kp, vp, layout.block_tables, layout.seq_lens, layout.scale,
+                        layout.num_kv_heads, layout.dtype)
+    return out, kp, vp
+
+
+def attention_errors(got: np.ndarray, ref: np.ndarray):
+    err = np.abs(got - ref)
+    big = np.abs(ref) >= 0.1
+    max_rel = float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0
+    return float(err.max()) if err.size else 0.0, max_rel
+
+
+def assert_attention_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    bad = err > ATOL + RTOL * np.abs(ref)
+    if bad.any():
+        idx = np.argwhere(bad)[:5].tolist()
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} elements outside 2e-3 + 1e-2*|ref|; "
+            f"max abs err {err.max():.3e}; first bad {idx}; got {got[bad][:5]} ref {ref[bad][:5]}"
+        )
+
+
+def subproblem(layout: PagedLayout, values_dev, seqs):
+    """Host bits (pre-step state) of the blocks that sequences `seqs` read,
+    plus the copy sources feeding them, renumbered into a compact pool.
+    values_dev are the generator's torch device tensors, captured before any
+    kernel runs.  Returns (compact layout fields, compact values)."""
+    import torch
+
+    B = layout.block_size
+    seqs = list(seqs)
+    ids = []
+    for s in seqs:
+        ids.extend(layout.block_tables[s, : layout.blocks_of(s)].tolist())
+    dst_set = set(ids)
+    pairs = [(int(a), int(b)) for a, b in layout.copy_pairs.reshape(-1, 2) if int(b) in dst_set]
+    ids.extend(a for a, _ in pairs)
+    uniq = sorted(set(ids))
+    remap = {b: i for i, b in enumerate(uniq)}
+    idx = torch.tensor(uniq, dtype=torch.long, device=values_dev.k_pool.device)
+    kp = torch_bits(values_dev.k_pool.index_select(0, idx))
+    vp = torch_bits(values_dev.v_pool.index_select(0, idx))
+    max_nb = max(layout.blocks_of(s) for s in seqs)
+    tables = np.full((len(seqs), max_nb), -1, np.int32)
+    for i, s in enumerate(seqs):
+        nb = layout.blocks_of(s)
+        tables[i, :nb] = [remap[int(b)] for b in layout.block_tables[s, :nb]]
+    cpairs = np.array([(remap[a], remap[b]) for a, b in pairs], np.int64).reshape(-1, 2)
+    q = torch_bits(values_dev.q[seqs])
+    slots, nk, nv = [], [], []
+    if layout.num_new_tokens > 0:
+        for s in seqs:
+            slot = int(layout.slot_mapping[s])
+            blk, row = slot // B, slot % B
+            slots.append(remap[blk] * B + row)
+        nk = torch_bits(values_dev.new_k[seqs])
+        nv = torch_bits(values_dev.new_v[seqs])
+    return dict(q=q, k_pool=kp, v_pool=vp, tables=tables, lens=layout.seq_lens[seqs].copy(), pairs=cpairs,
+                slots=np.asarray(slots, np.int64), new_k=nk, new_v=nv)
+
+
+def oracle_subproblem(layout: PagedLayout, sub, heads=None) -> np.ndarray:
+    """Oracle outputs [len(seqs), len(heads), D] of a subproblem after its
+    copies and writes (heads: the q heads to compute, default all)."""
+    kp, vp = sub["k_pool"], sub["v_pool"]
+    if sub["pairs"].shape[0] > 0:
+        kp, vp = oracle.copy_blocks(kp, vp, sub["pairs"])
+    if sub["slots"].shape[0] > 0:
+        kp, vp = oracle.cache_write(kp, vp, sub["new_k"], sub["new_v"], sub["slots"])
+    heads = list(range(layout.num_q_heads)) if heads is None else list(heads)
+    out = np.zeros((sub["q"].shape[0], len(heads), layout.head_dim))
+    for i in range(sub["q"].shape[0]):
+        for k, h in enumerate(heads):
+            out[i, k] = oracle.decode_one(i, h, sub["q"], kp, vp, sub["tables"], sub["lens"], layout.scale,
+                                          layout.num_kv_heads, layout.dtype)
+    return out

@@ -20,6 +20,7 @@ from .generate import (  # noqa: F401
     config_llama2_70b_shared,
     config_opt13b_long,
     random_layout,
+    restrict_layout,
     fill_values_numpy,
     fill_values_torch,
     CONFIGS,

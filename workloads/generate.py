@@ -376,3 +376,41 @@ def fill_values_torch(layout: PagedLayout, device, value_seed: Optional[int] = N
     new_k = torch.randn((T, Hkv, D), generator=g, device=device, dtype=torch.float32).to(tdt)
     new_v = torch.randn((T, Hkv, D), generator=g, device=device, dtype=torch.float32).to(tdt)
     return PagedValues(q=q, k_pool=pools[0], v_pool=pools[1], new_k=new_k, new_v=new_v)
+
+
+def restrict_layout(layout: PagedLayout, seqs) -> PagedLayout:
+    """The same workload limited to sequences ``seqs``: their blocks (and the
+    copy sources feeding them) renumbered into a compact pool, the tables,
+    lengths, slots and copy pairs remapped.  Used to draw bounded samples of
+    a large workload for the CPU baseline."""
+    L = layout
+    B = L.block_size
+    seqs = [int(s) for s in seqs]
+    ids = []
+    for s in seqs:
+        ids.extend(int(b) for b in L.block_tables[s, : L.blocks_of(s)])
+    dst = set(ids)
+    pairs = [(int(a), int(b)) for a, b in L.copy_pairs.reshape(-1, 2) if int(b) in dst]
+    ids.extend(a for a, _ in pairs)
+    uniq = sorted(set(ids))
+    remap = {b: i for i, b in enumerate(uniq)}
+    max_nb = max([L.blocks_of(s) for s in seqs] + [1])
+    tables = np.full((len(seqs), max_nb), PAD_ENTRY, np.int32)
+    for i, s in enumerate(seqs):
+        nb = L.blocks_of(s)
+        tables[i, :nb] = [remap[int(b)] for b in L.block_tables[s, :nb]]
+    slots = []
+    if L.num_new_tokens > 0:
+        for s in seqs:
+            slot = int(L.slot_mapping[s])
+            slots.append(remap[slot // B] * B + slot % B)
+    fill = np.zeros(len(uniq), np.int32)
+    for b, i in remap.items():
+        fill[i] = L.block_fill[b]
+    return PagedLayout(
+        name=f"{L.name}[{len(seqs)} seqs]", seed=L.seed, dtype=L.dtype, block_size=B, num_blocks=len(uniq),
+        num_q_heads=L.num_q_heads, num_kv_heads=L.num_kv_heads, head_dim=L.head_dim, scale=L.scale,
+        seq_lens=L.seq_lens[seqs].astype(np.int32), block_tables=tables, slot_mapping=np.asarray(slots, np.int64),
+        copy_pairs=np.asarray([(remap[a], remap[b]) for a, b in pairs], np.int64).reshape(-1, 2),
+        block_fill=fill, note=f"sample of {L.name}",
+    )
