@@ -55,7 +55,9 @@ def test_config_full_size(cuda_device, name):
     seqs = _sample(L, 2 if long_ctx else 8, seed=len(name))
     heads = [0, 7, 21, 39] if long_ctx else None
     sub = subproblem(L, V, seqs)  # pre-step state, captured before any kernel runs
-    vmax = float(max(V.v_pool.float().nan_to_num(0).abs().max(), V.new_v.float().abs().max()))
+    vmax = float(V.v_pool.float().nan_to_num(0).abs().max())
+    if V.new_v.numel() > 0:
+        vmax = max(vmax, float(V.new_v.float().abs().max()))
     d = _device_inputs(L, V, cuda_device)
     out, st = gpu_step(d, L)
     assert int(st.item()) == 0
