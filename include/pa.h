@@ -8,7 +8,7 @@
  * sequence length ("PagedAttention 与 KV 显存管理" study notes ch.05 §3; vLLM
  * blog "vLLM 是什么" §2).  Attention over those blocks is merged across
  * blocks with online softmax (study notes §4); new tokens are stored into
- * their slots (vLLM blog §1); blocks shared by several outputs are copied
+ * their slots (vLLM blog, plain-language section); blocks shared by several outputs are copied
  * before a write (copy on write, study notes §6.1 and §12 exercise 4).
  *
  * Conventions shared by every entry point
@@ -117,7 +117,7 @@ PA_API size_t pa_decode_workspace_bytes_ex(int32_t num_seqs, int32_t num_q_heads
  * num_kv_heads), contiguous GQA groups), with n = seq_lens[s]:
  *   out[s][h] = sum_t softmax_t(scale * q[s][h] . K_t) V_t,  t = 0..n-1,
  * where K_t / V_t are row t % B of block block_tables[s][t / B] of the
- * pools (vLLM blog §2: softmax(QK^T/sqrt(d))V through block_table; study
+ * pools (vLLM blog §"关键细节" 2): softmax(QK^T/sqrt(d))V through block_table; study
  * notes ch.05 §4: blocks merged with a running max and running sum).
  * A sequence with n == 0 gets a zero output.  Rows of a partly filled last
  * block past n are never read into the result (they may hold anything).
@@ -153,7 +153,8 @@ PA_API pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_p
 
 /*
  * pa_cache_write — store the K/V of new tokens into their slots
- * (vLLM blog §1: each generated token's K/V is written to the cache;
+ * (vLLM blog, plain-language section: each generated token's K/V is
+ * written to the cache;
  * study notes ch.05 §5 item 2: a token goes to the next free slot).
  *
  * For each token t with slot = slot_mapping[t] >= 0:

@@ -4,7 +4,7 @@
   takes ceil(n / B) blocks and only the last one may be partly filled
   (study notes ch.05 §5 item 2, §9.2, §12 exercise 1).
 * kv_bytes_per_token: 2 (K and V) x layers x kv heads x head_dim x dtype
-  bytes (vLLM blog §1 KV-size formula; study notes ch.05 §2 for OPT-13B).
+  bytes (vLLM blog §"关键细节" 1) KV-size formula; study notes ch.05 §2 for OPT-13B).
 * BlockManager: free set, reference counts, fork by sharing, copy on write
   when a writer's target block is shared, free at ref count zero
   (study notes ch.05 §5, §6.1, §6.2, §12 exercise 4).

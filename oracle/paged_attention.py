@@ -3,7 +3,7 @@
 Written from the pages, slow and literal:
 
 * decode = softmax(q K^T * scale) V over the gathered sequence
-  (vLLM blog §2 "PagedAttention 算子": Attn(Q,K,V) = softmax(QK^T/sqrt(d))V,
+  (vLLM blog §"关键细节" 2) "PagedAttention 算子": Attn(Q,K,V) = softmax(QK^T/sqrt(d))V,
   K/V reached block by block through block_table).
 * the blockwise form with a running max and running sum merged block by block
   (PagedAttention study notes ch.05 §4: S_ij = Q_i K_j^T, O_i = sum_j P_ij V_j,
@@ -11,7 +11,8 @@ Written from the pages, slow and literal:
 * the partition-then-merge form used for long sequences: each partition keeps
   (max, sum, unnormalised output) and the merge rescales them to a common max
   — the same online-softmax merge rule as ch.05 §4, applied to partitions.
-* cache write (vLLM blog §1: each new token's K/V is stored in its slot) and
+* cache write (vLLM blog, plain-language section: each generated token's
+  K/V is written down for later steps) and
   block copy for copy-on-write (study notes ch.05 §6.1, §12 exercise 4).
 
 Readings where the pages are silent (each listed in the design notes):
@@ -39,7 +40,7 @@ def bits_to_f64(bits: np.ndarray, dtype: str) -> np.ndarray:
 def gather_kv(pool: np.ndarray, table_row: np.ndarray, n: int, kv_head: int, block_size: int) -> np.ndarray:
     """Rows of tokens 0..n-1 of one sequence for one kv head, reached through
     the block table: token t lives in row t % B of block table_row[t // B]
-    (study notes ch.05 §3 and §9.2; vLLM blog §2).  pool is [NB, Hkv, B, D]."""
+    (study notes ch.05 §3 and §9.2; vLLM blog §"关键细节" 2)).  pool is [NB, Hkv, B, D]."""
     t = np.arange(n)
     blocks = np.asarray(table_row, dtype=np.int64)[t // block_size]
     rows = t % block_size
@@ -48,7 +49,7 @@ def gather_kv(pool: np.ndarray, table_row: np.ndarray, n: int, kv_head: int, blo
 
 def attention_dense(q_vec: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> np.ndarray:
     """softmax(scale * K q) V for one query vector over contiguous K, V [n, D]
-    (vLLM blog §2).  n == 0 gives zeros."""
+    (vLLM blog §"关键细节" 2)).  n == 0 gives zeros."""
     if K.shape[0] == 0:
         return np.zeros(V.shape[1], dtype=np.float64)
     z = scale * (K @ q_vec)
@@ -145,7 +146,7 @@ def merge_partition_states(states) -> np.ndarray:
 
 def cache_write(k_pool: np.ndarray, v_pool: np.ndarray, new_k: np.ndarray, new_v: np.ndarray,
                 slot_mapping: np.ndarray):
-    """Store each new token's K/V rows in its slot (vLLM blog §1: each
+    """Store each new token's K/V rows in its slot (vLLM blog, plain-language section: each
     generated token's K/V is written to the cache).  slot = block * B + row;
     a negative slot skips the token.  Returns new pool arrays (bit copies)."""
     k_out, v_out = k_pool.copy(), v_pool.copy()

@@ -1,6 +1,6 @@
 // pa_decode — paged decode attention for sm_100a.
 //
-// What it computes (vLLM blog §2; PagedAttention study notes ch.05 §4):
+// What it computes (vLLM blog §"关键细节" 2); PagedAttention study notes ch.05 §4):
 //   out[s][h] = softmax(scale * q[s][h] . K^T) V over the seq_lens[s] tokens
 //   of sequence s, K/V reached block by block through block_tables, the
 //   softmax normalisation merged across blocks with a running max and sum.

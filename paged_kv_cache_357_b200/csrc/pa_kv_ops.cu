@@ -1,5 +1,5 @@
 // pa_cache_write and pa_copy_blocks — the two bit-copy kernels beside the
-// decode: storing each new token's K/V in its slot (vLLM blog §1; study
+// decode: storing each new token's K/V in its slot (vLLM blog, plain-language section; study
 // notes ch.05 §5 item 2) and copying whole blocks for copy on write (study
 // notes ch.05 §6.1, §12 exercise 4).
 //

@@ -10,8 +10,8 @@ step enqueues, on one stream:
 
 matching the order of the method: a shared block is copied before a sample
 writes into it (study notes ch.05 §6.1), the new token is stored before the
-decode reads it (vLLM blog §1), and the decode reads every block through the
-table (vLLM blog §2).
+decode reads it (vLLM blog, plain-language section), and the decode reads every block through the
+table (vLLM blog §"关键细节" 2)).
 """
 
 from __future__ import annotations

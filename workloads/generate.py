@@ -4,7 +4,7 @@ Conventions (the same on both sides of every comparison):
 
 * A sequence of ``n`` tokens keeps token ``t`` in row ``t % B`` of the physical
   block ``block_tables[s, t // B]`` (block table indirection, PagedAttention
-  notes ch.05 §3 and §9.2; vLLM blog §2 "PagedAttention 算子").
+  notes ch.05 §3 and §9.2; vLLM blog §"关键细节" 2) "PagedAttention 算子").
 * ``seq_lens[s]`` counts every token the decode step attends, the newest one
   included.  When a layout writes new tokens, token ``seq_lens[s] - 1`` of each
   sequence is the one written this step: its row is NaN in the pool until the
