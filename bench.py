@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per GPU for the llama7b / llama3_8b workloads (0 = the workload's own)")
     return ap.parse_args(argv)
 
 
@@ -221,16 +223,25 @@ def cpu_baseline(L, budget_s: float) -> dict:
                       f"1 thread, {t_tot:.1f} s"}
 
 
+def make_layout(args):
+    from workloads import CONFIGS, config_llama3_8b, config_llama7b
+
+    if args.batch:
+        makers = {"llama3_8b": config_llama3_8b, "llama7b": config_llama7b}
+        if args.config not in makers:
+            raise SystemExit(f"--batch applies to {sorted(makers)} only")
+        return makers[args.config](batch=args.batch)
+    return CONFIGS[args.config]()
+
+
 def run_reference(args):
     """The oracle, as it stands, timed on the host cores on bounded samples."""
     import numpy as np
     from threadpoolctl import threadpool_limits
 
-    from workloads import CONFIGS
-
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
-    L = CONFIGS[args.config]()
+    L = make_layout(args)
     order = np.random.default_rng(0).permutation(L.num_seqs)
     with threadpool_limits(1):
         t_one, _ = oracle_sample_step(L, [int(order[0])])
@@ -270,7 +281,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     import paged_kv_cache_357_b200 as pa
-    from workloads import CONFIGS, fill_values_torch
+    from workloads import fill_values_torch
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -285,7 +296,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     pa.load()
-    L = CONFIGS[args.config]()
+    L = make_layout(args)
     V = fill_values_torch(L, dev, value_seed=L.seed + 7 * rank)
     nbytes = step_bytes(L)
     tables = torch.from_numpy(L.block_tables).to(dev)
