@@ -57,7 +57,8 @@ typedef enum pa_status {
   PA_ERR_INVALID_ARG = 1, /* null or misaligned pointer, negative or zero size */
   PA_ERR_UNSUPPORTED = 2, /* no kernel for this block_size/head_dim/group/dtype */
   PA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
-  PA_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+  PA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  PA_ERR_SCRATCH_LIMIT = 5 /* pa_decode_no_alloc: the batch needs more scratch than its fixed array */
 } pa_status;
 
 /* Device-side status codes written to *dev_status (a range of their own,
@@ -150,6 +151,39 @@ PA_API pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_p
                        int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
                        int32_t num_q_heads, float scale, void* out, void* workspace, size_t workspace_bytes,
                        int32_t* dev_status, const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream);
+
+/*
+ * pa_decode_no_alloc — pa_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is a calling convention of
+ * this library, not part of the method.
+ *
+ * Who needs it: code that is handed its inputs and outputs and may not call
+ * cudaMalloc or any routine that allocates — for example a plug-in run by a
+ * host engine that has already claimed nearly all device memory for its KV
+ * pool and gives the plug-in nothing else, or a latency-critical loop where
+ * an allocation (and the device synchronisation it can imply) is not allowed.
+ *
+ * It takes pa_decode's arguments minus the workspace and computes the same
+ * result with the same kernel.  Its scratch is a fixed array of
+ * PA_DECODE_NO_ALLOC_SCRATCH_BYTES (8 MiB) in libpa's own device memory; every
+ * GPU that loads the library holds that array until the process exits.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it.  Make
+ *     that first call on a device before any stream capture.
+ *   - Each call clears the arrival counters it needs (cudaMemsetAsync on
+ *     `stream`) and launches the decode.  Nothing is allocated or freed.
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     calls that can overlap on the GPU (other streams, or unordered work on
+ *     one stream) race and give wrong results.  Order them.
+ *   - Returns PA_ERR_SCRATCH_LIMIT, doing nothing, when the batch needs more
+ *     scratch than the array holds (what pa_decode_workspace_bytes reports for
+ *     the same arguments must not exceed PA_DECODE_NO_ALLOC_SCRATCH_BYTES).
+ */
+#define PA_DECODE_NO_ALLOC_SCRATCH_BYTES (8u << 20)
+PA_API pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const void* v_pool,
+                                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                    int32_t num_seqs, int32_t num_q_heads, float scale, void* out,
+                                    int32_t* dev_status, const pa_pool_desc* pool, void* stream);
 
 /*
  * pa_cache_write — store the K/V of new tokens into their slots

@@ -27,6 +27,7 @@ from ._lib import (  # noqa: F401
     pa_cache_write,
     pa_copy_blocks,
     pa_decode,
+    pa_decode_no_alloc,
     pool_desc,
     status_string,
 )

@@ -31,6 +31,7 @@ EXPORTED = (
     "pa_decode_workspace_bytes_ex",
     "pa_decode",
     "pa_decode_ex",
+    "pa_decode_no_alloc",
     "pa_cache_write",
     "pa_copy_blocks",
     "pa_status_string",
@@ -81,6 +82,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode.restype = i32
     lib.pa_decode_ex.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, f32, vp, vp, sz, vp, pdesc, popts, vp]
     lib.pa_decode_ex.restype = i32
+    lib.pa_decode_no_alloc.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, f32, vp, vp, pdesc, vp]
+    lib.pa_decode_no_alloc.restype = i32
     lib.pa_cache_write.argtypes = [vp, vp, vp, i32, vp, vp, vp, pdesc, vp]
     lib.pa_cache_write.restype = i32
     lib.pa_copy_blocks.argtypes = [vp, i32, vp, vp, vp, pdesc, vp]
@@ -195,6 +198,35 @@ def pa_decode(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, work
     )
     if rc != 0:
         raise PaError(rc, "pa_decode")
+
+
+def pa_decode_no_alloc(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, dev_status=None,
+                       stream=None) -> None:
+    """pa_decode without a caller workspace, for callers that may not
+    allocate device memory: the scratch is libpa's own fixed device array
+    (8 MiB per device).  Calls that may overlap on the GPU race; order them.
+    The first call on a device looks up the array's address, so make it
+    before any stream capture."""
+    torch = _torch()
+    _need(k_pool, "k_pool", ndim=4)
+    dev = k_pool.device
+    _need(v_pool, "v_pool", dtype=k_pool.dtype, ndim=4, device=dev)
+    _need(q, "q", dtype=k_pool.dtype, ndim=3, device=dev)
+    _need(out, "out", dtype=k_pool.dtype, ndim=3, device=dev)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2, device=dev)
+    _need(seq_lens, "seq_lens", dtype=torch.int32, ndim=1, device=dev)
+    S, Hq, D = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != S or seq_lens.shape[0] != S or D != k_pool.shape[3]:
+        raise ValueError("shapes of q, out, block_tables, seq_lens and the pools disagree")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", dtype=torch.int32, device=dev)
+    desc = pool_desc(k_pool)
+    rc = load().pa_decode_no_alloc(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), S, Hq,
+        float(scale), _ptr(out), _ptr(dev_status), ctypes.byref(desc), _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode_no_alloc")
 
 
 def pa_cache_write(k, v, slot_mapping, k_pool, v_pool, dev_status=None, stream=None) -> None:

@@ -808,3 +808,94 @@ extern "C" pa_status pa_decode(const void* q, const void* k_pool, const void* v_
   return pa_decode_ex(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads, scale,
                       out, workspace, workspace_bytes, dev_status, pool, nullptr, stream);
 }
+
+// ---------------------------------------------------------------------------
+// pa_decode_no_alloc: the same decode kernel with its scratch (partial states
+// and arrival counters) in a fixed array of libpa's own device memory, for
+// callers that cannot allocate device memory themselves.
+// ---------------------------------------------------------------------------
+
+namespace pa {
+
+constexpr size_t kNoAllocScratchBytes = PA_DECODE_NO_ALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+// Held by every GPU that loads libpa, until the process exits.  Host code must
+// not pass this name to a kernel: on the host it is only a stand-in for the
+// symbol, so its device address is looked up below.
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+// Device address of g_decode_scratch on the current device, looked up on the
+// first call per device (with that device current) and cached.
+static bool no_alloc_scratch_address(void** addr) {
+  static std::mutex mu;
+  static void* cached[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return false;
+    cached[dev] = p;
+  }
+  *addr = cached[dev];
+  return true;
+}
+
+}  // namespace pa
+
+extern "C" pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const void* v_pool,
+                                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
+                                        void* out, int32_t* dev_status, const pa_pool_desc* pool, void* stream) {
+  if (!pool_shape_ok(pool) || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (num_seqs == 0) return PA_OK;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || block_tables == nullptr || seq_lens == nullptr ||
+      out == nullptr) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) || !std::isfinite(scale)) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(max_blocks_per_seq) * pool->block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  Variant v;
+  if (!select_variant(*pool, num_q_heads, v)) return PA_ERR_UNSUPPORTED;
+  const int ctas = resolve_ctas(v, nullptr);
+  if (ctas <= 0) return PA_ERR_CUDA;
+  if (workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride) > kNoAllocScratchBytes) {
+    return PA_ERR_SCRATCH_LIMIT;
+  }
+  void* scratch = nullptr;
+  if (!no_alloc_scratch_address(&scratch)) return PA_ERR_CUDA;
+  const size_t parts_bytes = align_up(static_cast<size_t>(ctas) * 2 * v.part_stride * sizeof(float), 256);
+  int32_t* counters = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + parts_bytes);
+  // The array keeps whatever the previous call left; the arrival counters
+  // must start at zero, so clear them on the caller's stream first.
+  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(num_seqs) * pool->num_kv_heads * sizeof(int32_t),
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    return PA_ERR_CUDA;
+  }
+
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.k_pool = static_cast<const uint16_t*>(k_pool);
+  prm.v_pool = static_cast<const uint16_t*>(v_pool);
+  prm.block_tables = block_tables;
+  prm.seq_lens = seq_lens;
+  prm.out = static_cast<uint16_t*>(out);
+  prm.partials = static_cast<float*>(scratch);
+  prm.counters = counters;
+  prm.status = dev_status;
+  prm.max_nb = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = pool->num_kv_heads;
+  prm.num_blocks = pool->num_blocks;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_limit_ns = 2ull * 1000 * 1000 * 1000;
+  prm.test_flags = 0;
+  v.fn<<<ctas, kThreads, v.smem_bytes, static_cast<cudaStream_t>(stream)>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}

@@ -116,6 +116,7 @@ extern "C" const char* pa_status_string(int32_t status) {
     case PA_ERR_UNSUPPORTED: return "unsupported block_size/head_dim/group/dtype combination";
     case PA_ERR_WORKSPACE: return "workspace missing or too small";
     case PA_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+    case PA_ERR_SCRATCH_LIMIT: return "batch needs more scratch than pa_decode_no_alloc's fixed array";
     case PA_DEV_BAD_BLOCK_ID: return "device: block table entry outside [0, num_blocks)";
     case PA_DEV_BAD_SEQ_LEN: return "device: seq_len negative or beyond the block table";
     case PA_DEV_BAD_SLOT: return "device: slot_mapping entry beyond the pool";
