@@ -84,7 +84,7 @@ typedef struct pa_pool_desc {
 /* Tuning/test options for pa_decode_ex; zero-initialise for the defaults. */
 typedef struct pa_decode_opts {
   int32_t num_ctas; /* persistent CTAs; 0 = SM count x resident CTAs per SM */
-  int32_t flags;    /* 0, or PA_DECODE_TEST_WITHHOLD_COPIES */
+  int32_t flags;    /* 0, or PA_DECODE_CUDA_CORES_ONLY and/or PA_DECODE_TEST_WITHHOLD_COPIES */
 } pa_decode_opts;
 
 /* Failure-detection test hook for pa_decode_opts.flags: the producer warp
@@ -92,6 +92,12 @@ typedef struct pa_decode_opts {
  * kernel returns early with PA_DEV_TIMEOUT in *dev_status and the GPU context
  * still usable.  Output is not written.  Never set it outside such tests. */
 #define PA_DECODE_TEST_WITHHOLD_COPIES 1
+
+/* pa_decode_opts.flags bit: use the CUDA-core kernel even where the
+ * tensor-core kernel applies (group size 4 or 8 with head_dim 128 and
+ * block_size 16); for comparisons and tests.  Same results within the
+ * documented tolerance. */
+#define PA_DECODE_CUDA_CORES_ONLY 2
 
 /*
  * pa_decode_workspace_bytes — bytes of device scratch pa_decode needs.
@@ -104,7 +110,8 @@ typedef struct pa_decode_opts {
  * pa_decode; every pa_decode that ends with PA_DEV_OK leaves the counters at
  * zero again, so the same workspace serves any number of later calls on the
  * same stream.  After a non-zero device status, zero it again.  Two decodes
- * that may run at the same time need separate workspaces.
+ * that may run at the same time need separate workspaces.  The size depends
+ * on the kernel variant, so query with the opts the decode will use.
  * Returns 0 for invalid arguments.
  */
 PA_API size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, const pa_pool_desc* pool);

@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     EXPORTED,
     LIB_PATH,
     PA_BF16,
+    PA_DECODE_CUDA_CORES_ONLY,
     PA_DECODE_TEST_WITHHOLD_COPIES,
     PA_FP16,
     DecodeOpts,

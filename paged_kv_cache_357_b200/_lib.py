@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(HERE, "libpa.so")
 
 PA_FP16, PA_BF16 = 0, 1
 PA_DECODE_TEST_WITHHOLD_COPIES = 1
+PA_DECODE_CUDA_CORES_ONLY = 2
 DEV_STATUS = {
     0: "PA_DEV_OK",
     101: "PA_DEV_BAD_BLOCK_ID",
@@ -150,19 +151,21 @@ def pool_desc(k_pool) -> PoolDesc:
     return PoolDesc(nb, bs, hkv, d, _dtype_code(k_pool))
 
 
-def decode_workspace_bytes(num_seqs: int, num_q_heads: int, k_pool, num_ctas: int = 0) -> int:
+def decode_workspace_bytes(num_seqs: int, num_q_heads: int, k_pool, num_ctas: int = 0, flags: int = 0) -> int:
+    """Workspace bytes for pa_decode with the same num_ctas and flags."""
     desc = pool_desc(k_pool)
-    opts = DecodeOpts(num_ctas, 0)
+    opts = DecodeOpts(num_ctas, flags)
     n = load().pa_decode_workspace_bytes_ex(num_seqs, num_q_heads, ctypes.byref(desc), ctypes.byref(opts))
     if n == 0:
         raise PaError(1, "pa_decode_workspace_bytes")
     return int(n)
 
 
-def alloc_decode_workspace(num_seqs: int, num_q_heads: int, k_pool, num_ctas: int = 0):
-    """Zeroed device workspace for pa_decode (see include/pa.h)."""
+def alloc_decode_workspace(num_seqs: int, num_q_heads: int, k_pool, num_ctas: int = 0, flags: int = 0):
+    """Zeroed device workspace for pa_decode with the same num_ctas and flags
+    (see include/pa.h)."""
     torch = _torch()
-    n = decode_workspace_bytes(num_seqs, num_q_heads, k_pool, num_ctas)
+    n = decode_workspace_bytes(num_seqs, num_q_heads, k_pool, num_ctas, flags)
     return torch.zeros(n, dtype=torch.uint8, device=k_pool.device)
 
 

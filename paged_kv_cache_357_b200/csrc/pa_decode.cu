@@ -39,6 +39,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "pa_decode_host.h"
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -85,11 +86,7 @@ struct __align__(128) DecodeSmem {
   uint64_t empty[C::kStages];
   uint64_t qfull[2];
   uint64_t qempty[2];
-  long long scan[kThreads / 32];
-  long long total;
-  long long pre0;
-  int s0;
-  int found;
+  RangeSmem range;
   int abort;
   int is_last;
   int issued;
@@ -97,107 +94,6 @@ struct __align__(128) DecodeSmem {
   int q_issued;
   int q_consumed;
 };
-
-struct DecodeParams {
-  const uint16_t* q;
-  const uint16_t* k_pool;
-  const uint16_t* v_pool;
-  const int32_t* block_tables;
-  const int32_t* seq_lens;
-  uint16_t* out;
-  float* partials;
-  int32_t* counters;
-  int32_t* status;
-  int max_nb;
-  int num_seqs;
-  int num_q_heads;
-  int num_kv_heads;
-  int num_blocks;
-  float scale_log2;
-  unsigned long long wait_limit_ns;
-  int test_flags;
-};
-
-constexpr int kFlagTestWithholdCopies = PA_DECODE_TEST_WITHHOLD_COPIES;  // producer issues nothing
-
-__device__ __forceinline__ int checked_len(const DecodeParams& p, int s, int B) {
-  const int n = __ldg(p.seq_lens + s);
-  return (n < 0 || n > p.max_nb * B) ? 0 : n;
-}
-
-struct Cursor {
-  int s, h, j, nb, len;
-  long long x, remaining;
-};
-
-struct Seg {
-  int s, h, j0, n, nb, len;
-  long long unit_first;  // flattened index of block 0 of unit (s, h)
-};
-
-template <int B>
-__device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams& p) {
-  if (c.remaining <= 0) return false;
-  const long long left = c.nb - c.j;
-  const int n = static_cast<int>(left < c.remaining ? left : c.remaining);
-  sg.s = c.s;
-  sg.h = c.h;
-  sg.j0 = c.j;
-  sg.n = n;
-  sg.nb = c.nb;
-  sg.len = c.len;
-  sg.unit_first = c.x - c.j;
-  c.remaining -= n;
-  c.x += n;
-  c.j += n;
-  if (c.j == c.nb) {
-    c.j = 0;
-    if (++c.h == p.num_kv_heads) {
-      c.h = 0;
-      if (c.remaining > 0) {
-        do {
-          if (++c.s >= p.num_seqs) {  // inconsistent lengths: stop cleanly
-            c.remaining = 0;
-            break;
-          }
-          c.len = checked_len(p, c.s, B);
-          c.nb = (c.len + B - 1) / B;
-        } while (c.nb == 0);
-      }
-    }
-  }
-  return true;
-}
-
-// CTA whose range [c*N/C, (c+1)*N/C) holds flattened block x.
-__device__ __forceinline__ long long cta_of(long long x, long long N, long long C) {
-  return ((x + 1) * C - 1) / N;
-}
-
-__device__ __forceinline__ long long range_start(long long c, long long N, long long C) { return c * N / C; }
-
-// Block-wide inclusive scan of one long long per thread (all kThreads threads).
-template <typename Smem>
-__device__ __forceinline__ long long block_inclusive_scan(long long v, Smem& sm, long long& block_total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long t = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += t;
-  }
-  if (lane == 31) sm.scan[warp] = v;
-  __syncthreads();
-  long long before = 0, total = 0;
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) {
-    const long long t = sm.scan[w];
-    if (w < warp) before += t;
-    total += t;
-  }
-  __syncthreads();
-  block_total = total;
-  return v + before;
-}
 
 template <bool kBf16, int D, int B, int G>
 __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams p) {
@@ -208,54 +104,13 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const long long nctas = gridDim.x, cta = blockIdx.x;
-  const int Hkv = p.num_kv_heads, Hq = p.num_q_heads;
+  const long long cta = blockIdx.x;
+  const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
 
-  // ---- prologue: total work, zero outputs of empty sequences -------------
-  long long mine = 0;
-  for (int s = tid; s < p.num_seqs; s += kThreads) {
-    const int raw = __ldg(p.seq_lens + s);
-    int n = raw;
-    if (raw < 0 || raw > p.max_nb * B) {
-      if (cta == 0) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
-      n = 0;
-    }
-    if (n == 0 && (s % nctas) == cta) {
-      uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(s) * Hq * D);
-      for (int i = 0; i < Hq * D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
-    }
-    mine += (n + B - 1) / B;
-  }
-  long long seq_blocks;
-  (void)block_inclusive_scan(mine, sm, seq_blocks);
-  const long long NBT = seq_blocks * Hkv;
-  // Partition over at most NBT CTAs so that every range is non-empty; the
-  // CTAs that split a unit are then exactly cta_of(first)..cta_of(last).
-  const long long nparts = NBT < nctas ? NBT : nctas;
-  if (cta >= nparts) return;  // uniform across the CTA (also covers NBT == 0)
-  const long long start = range_start(cta, NBT, nparts);
-  const long long end = range_start(cta + 1, NBT, nparts);
-
-  // ---- locate the sequence holding `start` ---------------------------------
-  const long long target = start / Hkv;  // in per-sequence block units
-  if (tid == 0) sm.found = 0;
-  __syncthreads();
-  long long base = 0;
-  for (int chunk = 0; chunk < p.num_seqs; chunk += kThreads) {
-    const int s = chunk + tid;
-    const long long nb = (s < p.num_seqs) ? (checked_len(p, s, B) + B - 1) / B : 0;
-    long long chunk_total;
-    const long long incl = block_inclusive_scan(nb, sm, chunk_total);
-    const long long excl = incl - nb;
-    if (nb > 0 && base + excl <= target && target < base + incl) {
-      sm.s0 = s;
-      sm.pre0 = base + excl;
-      sm.found = 1;
-    }
-    base += chunk_total;
-    __syncthreads();
-    if (sm.found) break;
-  }
+  zero_empty_outputs<kThreads, B>(p, D);
+  WorkRange wr;
+  Cursor cur;
+  if (!decode_prologue<kThreads, B>(p, sm.range, wr, cur)) return;  // uniform across the CTA
 
   if (tid == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -274,19 +129,6 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
     fence_barrier_init();
   }
   __syncthreads();
-  if (!sm.found) return;  // only with lengths changing under the kernel
-
-  Cursor cur;
-  cur.s = sm.s0;
-  cur.len = checked_len(p, cur.s, B);
-  cur.nb = (cur.len + B - 1) / B;
-  {
-    const long long off = start - sm.pre0 * Hkv;
-    cur.h = static_cast<int>(off / cur.nb);
-    cur.j = static_cast<int>(off % cur.nb);
-  }
-  cur.x = start;
-  cur.remaining = end - start;
   const volatile int* abort_flag = &sm.abort;
 
   if (warp == kConsumerWarps) {
@@ -526,8 +368,7 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
       const long long F = sg.unit_first;
       float* my_part = nullptr;
       if (!whole_unit) {
-        const int slot = (start >= F) ? 0 : 1;
-        my_part = p.partials + (static_cast<size_t>(cta) * 2 + slot) * C::kPartStride;
+        my_part = p.partials + partial_slot(cta, F, wr) * C::kPartStride;
       }
       uint16_t* out_row = p.out + (static_cast<size_t>(sg.s) * Hq + static_cast<size_t>(sg.h) * G) * D;
       for (int idx = ctid; idx < G * D / 2; idx += kConsumerThreads) {
@@ -556,40 +397,8 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
       }
       if (!whole_unit) {
         __threadfence();
-        named_barrier_sync(kMergeBarrier, kConsumerThreads);
-        const long long first = cta_of(F, NBT, nparts);
-        const long long last = cta_of(F + sg.nb - 1, NBT, nparts);
-        int32_t* counter = p.counters + static_cast<size_t>(sg.s) * Hkv + sg.h;
-        if (ctid == 0) {
-          const int prev = atomicAdd(counter, 1);
-          sm.is_last = (prev == static_cast<int>(last - first));
-        }
-        named_barrier_sync(kMergeBarrier, kConsumerThreads);
-        if (sm.is_last) {
-          __threadfence();
-          for (int idx = ctid; idx < G * D / 2; idx += kConsumerThreads) {
-            const int g = (2 * idx) / D, d = (2 * idx) % D;
-            float M = -INFINITY;
-            for (long long cc = first; cc <= last; ++cc) {
-              const int sl = (range_start(cc, NBT, nparts) >= F) ? 0 : 1;
-              const float* pp = p.partials + (static_cast<size_t>(cc) * 2 + sl) * C::kPartStride;
-              M = fmaxf(M, __ldcg(pp + g));
-            }
-            float L = 0.f, a0 = 0.f, a1 = 0.f;
-            for (long long cc = first; cc <= last; ++cc) {
-              const int sl = (range_start(cc, NBT, nparts) >= F) ? 0 : 1;
-              const float* pp = p.partials + (static_cast<size_t>(cc) * 2 + sl) * C::kPartStride;
-              const float sc_p = fast_exp2(__ldcg(pp + g) - M);
-              L = fmaf(__ldcg(pp + G + g), sc_p, L);
-              const float2 av = __ldcg(reinterpret_cast<const float2*>(pp + 2 * G + g * D + d));
-              a0 = fmaf(av.x, sc_p, a0);
-              a1 = fmaf(av.y, sc_p, a1);
-            }
-            const float inv = 1.f / L;
-            *reinterpret_cast<uint32_t*>(out_row + g * D + d) = pack2<kBf16>(a0 * inv, a1 * inv);
-          }
-          if (ctid == 0) *counter = 0;
-        }
+        finish_split_unit<kBf16, D, G>(p, sg, wr, ctid, kConsumerThreads, &sm.is_last,
+                                       [] { named_barrier_sync(kMergeBarrier, kConsumerThreads); });
       }
       named_barrier_sync(kMergeBarrier, kConsumerThreads);
     }
@@ -619,18 +428,17 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
 // host side
 // ---------------------------------------------------------------------------
 
-using KernelFn = void (*)(DecodeParams);
-
-struct Variant {
-  KernelFn fn;
-  int smem_bytes;
-  int part_stride;  // floats per partial slot
-};
+template <bool kBf16, int D, int B, int G>
+static cudaError_t launch_cuda_cores(const Variant& v, const DecodeParams& prm, int ctas, cudaStream_t stream) {
+  pa_decode_kernel<kBf16, D, B, G><<<ctas, kThreads, v.smem_bytes, stream>>>(prm);
+  return cudaGetLastError();
+}
 
 template <bool kBf16, int D, int B, int G>
 Variant make_variant() {
-  return Variant{pa_decode_kernel<kBf16, D, B, G>, static_cast<int>(sizeof(DecodeSmem<D, B, G>)),
-                 Cfg<D, B, G>::kPartStride};
+  return Variant{reinterpret_cast<const void*>(&pa_decode_kernel<kBf16, D, B, G>), kThreads,
+                 static_cast<int>(sizeof(DecodeSmem<D, B, G>)), Cfg<D, B, G>::kPartStride,
+                 &launch_cuda_cores<kBf16, D, B, G>};
 }
 
 template <bool kBf16, int D, int B>
@@ -663,55 +471,62 @@ bool pick_d(int D, int B, int G, Variant& v) {
   }
 }
 
-static bool select_variant(const pa_pool_desc& pool, int num_q_heads, Variant& v) {
+// The tensor-core kernel where one applies (unless the caller asks for CUDA
+// cores only), else the CUDA-core kernel.
+static bool select_variant(const pa_pool_desc& pool, int num_q_heads, int flags, Variant& v) {
   if (pool.num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % pool.num_kv_heads != 0) return false;
   const int G = num_q_heads / pool.num_kv_heads;
+  if ((flags & PA_DECODE_CUDA_CORES_ONLY) == 0 && select_tc_variant(pool, G, v)) return true;
   if (pool.dtype == PA_BF16) return pick_d<true>(pool.head_dim, pool.block_size, G, v);
   if (pool.dtype == PA_FP16) return pick_d<false>(pool.head_dim, pool.block_size, G, v);
   return false;
 }
 
-// Resident CTAs per SM and SM count for a variant on the current device
-// (cached per device and kernel).
+// Resident CTAs per SM times the SM count for a variant on the current
+// device; also raises the kernel's dynamic shared memory limit.  Cached per
+// device and kernel.
 static bool grid_size_for(const Variant& v, int& ctas) {
   struct Entry {
     int device;
-    KernelFn fn;
+    const void* fn;
     int ctas;
   };
   static std::mutex mu;
-  static Entry cache[256];
+  static Entry cache[512];
   static int n_cache = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   {
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < n_cache; ++i) {
-      if (cache[i].device == dev && cache[i].fn == v.fn) {
+      if (cache[i].device == dev && cache[i].fn == v.kernel) {
         ctas = cache[i].ctas;
         return true;
       }
     }
   }
-  if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem_bytes) != cudaSuccess)
+  if (cudaFuncSetAttribute(v.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem_bytes) != cudaSuccess)
     return false;
   int per_sm = 0, sms = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, kThreads, v.smem_bytes) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.kernel, v.threads, v.smem_bytes) != cudaSuccess)
     return false;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
   if (per_sm < 1) return false;
   ctas = per_sm * sms;
   std::lock_guard<std::mutex> lock(mu);
-  if (n_cache < 256) cache[n_cache++] = Entry{dev, v.fn, ctas};
+  if (n_cache < 512) cache[n_cache++] = Entry{dev, v.kernel, ctas};
   return true;
 }
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+static size_t partials_bytes(int ctas, int part_stride) {
+  return align_up(static_cast<size_t>(ctas) * 2 * part_stride * sizeof(float), 256);
+}
+
 static size_t workspace_bytes_for(int num_seqs, int num_kv_heads, int ctas, int part_stride) {
-  const size_t parts = align_up(static_cast<size_t>(ctas) * 2 * part_stride * sizeof(float), 256);
   const size_t counters = align_up(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t), 256);
-  return parts + counters;
+  return partials_bytes(ctas, part_stride) + counters;
 }
 
 static bool pool_shape_ok(const pa_pool_desc* pool) {
@@ -719,10 +534,63 @@ static bool pool_shape_ok(const pa_pool_desc* pool) {
          pool->head_dim > 0 && (pool->dtype == PA_FP16 || pool->dtype == PA_BF16);
 }
 
+// CTA count: an explicit request, else the resident maximum.  Either way the
+// kernel's shared-memory attribute is set.
 static int resolve_ctas(const Variant& v, const pa_decode_opts* opts) {
-  if (opts != nullptr && opts->num_ctas > 0) return opts->num_ctas;
   int ctas = 0;
-  return grid_size_for(v, ctas) ? ctas : 0;
+  if (!grid_size_for(v, ctas)) return 0;
+  if (opts != nullptr && opts->num_ctas > 0) return opts->num_ctas;
+  return ctas;
+}
+
+static int opts_flags(const pa_decode_opts* opts) { return opts != nullptr ? opts->flags : 0; }
+
+constexpr int kKnownFlags = PA_DECODE_TEST_WITHHOLD_COPIES | PA_DECODE_CUDA_CORES_ONLY;
+
+// Shared argument checks of the decode entry points.
+static pa_status check_decode_args(const void* q, const void* k_pool, const void* v_pool,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                   int32_t num_seqs, int32_t num_q_heads, float scale, const void* out,
+                                   const pa_pool_desc* pool) {
+  if (!pool_shape_ok(pool) || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (num_seqs == 0) return PA_OK;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || block_tables == nullptr || seq_lens == nullptr ||
+      out == nullptr) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) || !std::isfinite(scale)) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(max_blocks_per_seq) * pool->block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+static DecodeParams make_params(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                                int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
+                                int32_t num_q_heads, float scale, void* out, void* scratch, int ctas,
+                                int part_stride, int32_t* dev_status, const pa_pool_desc* pool, int flags) {
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.k_pool = static_cast<const uint16_t*>(k_pool);
+  prm.v_pool = static_cast<const uint16_t*>(v_pool);
+  prm.block_tables = block_tables;
+  prm.seq_lens = seq_lens;
+  prm.out = static_cast<uint16_t*>(out);
+  prm.partials = static_cast<float*>(scratch);
+  prm.counters = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + partials_bytes(ctas, part_stride));
+  prm.status = dev_status;
+  prm.max_nb = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = pool->num_kv_heads;
+  prm.num_blocks = pool->num_blocks;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const bool test_timeout = (flags & PA_DECODE_TEST_WITHHOLD_COPIES) != 0;
+  prm.wait_limit_ns = test_timeout ? 20ull * 1000 * 1000 : 2ull * 1000 * 1000 * 1000;
+  prm.test_flags = test_timeout ? kFlagTestWithholdCopies : 0;
+  return prm;
 }
 
 }  // namespace pa
@@ -733,9 +601,13 @@ extern "C" size_t pa_decode_workspace_bytes_ex(int32_t num_seqs, int32_t num_q_h
                                                const pa_decode_opts* opts) {
   if (num_seqs < 0 || !pool_shape_ok(pool)) return 0;
   Variant v;
-  if (!select_variant(*pool, num_q_heads, v)) return 0;
-  const int ctas = resolve_ctas(v, opts);
-  if (ctas <= 0) return 0;
+  if (!select_variant(*pool, num_q_heads, opts_flags(opts), v)) return 0;
+  int ctas = 0;
+  if (opts != nullptr && opts->num_ctas > 0) {
+    ctas = opts->num_ctas;  // no device query needed
+  } else if (!grid_size_for(v, ctas)) {
+    return 0;
+  }
   return workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
 }
 
@@ -748,56 +620,20 @@ extern "C" pa_status pa_decode_ex(const void* q, const void* k_pool, const void*
                                   int32_t num_seqs, int32_t num_q_heads, float scale, void* out, void* workspace,
                                   size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
                                   const pa_decode_opts* opts, void* stream) {
-  if (!pool_shape_ok(pool) || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) {
-    return PA_ERR_INVALID_ARG;
-  }
-  if (num_seqs == 0) return PA_OK;
-  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || block_tables == nullptr || seq_lens == nullptr ||
-      out == nullptr) {
-    return PA_ERR_INVALID_ARG;
-  }
-  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) || !std::isfinite(scale)) {
-    return PA_ERR_INVALID_ARG;
-  }
-  if (opts != nullptr && (opts->num_ctas < 0 || (opts->flags & ~kFlagTestWithholdCopies) != 0)) {
-    return PA_ERR_INVALID_ARG;
-  }
-  if (static_cast<long long>(max_blocks_per_seq) * pool->block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  pa_status st = check_decode_args(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                                    num_q_heads, scale, out, pool);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (opts != nullptr && (opts->num_ctas < 0 || (opts->flags & ~kKnownFlags) != 0)) return PA_ERR_INVALID_ARG;
   Variant v;
-  if (!select_variant(*pool, num_q_heads, v)) return PA_ERR_UNSUPPORTED;
+  if (!select_variant(*pool, num_q_heads, opts_flags(opts), v)) return PA_ERR_UNSUPPORTED;
   const int ctas = resolve_ctas(v, opts);
   if (ctas <= 0) return PA_ERR_CUDA;
   const size_t need = workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
-  if (opts != nullptr && opts->num_ctas > 0) {
-    if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem_bytes) != cudaSuccess)
-      return PA_ERR_CUDA;
-  }
-
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.k_pool = static_cast<const uint16_t*>(k_pool);
-  prm.v_pool = static_cast<const uint16_t*>(v_pool);
-  prm.block_tables = block_tables;
-  prm.seq_lens = seq_lens;
-  prm.out = static_cast<uint16_t*>(out);
-  prm.partials = static_cast<float*>(workspace);
-  prm.counters = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
-                                            align_up(static_cast<size_t>(ctas) * 2 * v.part_stride * sizeof(float),
-                                                     256));
-  prm.status = dev_status;
-  prm.max_nb = max_blocks_per_seq;
-  prm.num_seqs = num_seqs;
-  prm.num_q_heads = num_q_heads;
-  prm.num_kv_heads = pool->num_kv_heads;
-  prm.num_blocks = pool->num_blocks;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  const bool test_timeout = opts != nullptr && (opts->flags & kFlagTestWithholdCopies) != 0;
-  prm.wait_limit_ns = test_timeout ? 20ull * 1000 * 1000 : 2ull * 1000 * 1000 * 1000;
-  prm.test_flags = test_timeout ? kFlagTestWithholdCopies : 0;
-
-  v.fn<<<ctas, kThreads, v.smem_bytes, static_cast<cudaStream_t>(stream)>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                                       num_q_heads, scale, out, workspace, ctas, v.part_stride, dev_status, pool,
+                                       opts_flags(opts));
+  return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" pa_status pa_decode(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
@@ -810,8 +646,8 @@ extern "C" pa_status pa_decode(const void* q, const void* k_pool, const void* v_
 }
 
 // ---------------------------------------------------------------------------
-// pa_decode_no_alloc: the same decode kernel with its scratch (partial states
-// and arrival counters) in a fixed array of libpa's own device memory, for
+// pa_decode_no_alloc: the same decode with its scratch (partial states and
+// arrival counters) in a fixed array of libpa's own device memory, for
 // callers that cannot allocate device memory themselves.
 // ---------------------------------------------------------------------------
 
@@ -848,20 +684,11 @@ extern "C" pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const
                                         const int32_t* block_tables, int32_t max_blocks_per_seq,
                                         const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
                                         void* out, int32_t* dev_status, const pa_pool_desc* pool, void* stream) {
-  if (!pool_shape_ok(pool) || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) {
-    return PA_ERR_INVALID_ARG;
-  }
-  if (num_seqs == 0) return PA_OK;
-  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || block_tables == nullptr || seq_lens == nullptr ||
-      out == nullptr) {
-    return PA_ERR_INVALID_ARG;
-  }
-  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) || !std::isfinite(scale)) {
-    return PA_ERR_INVALID_ARG;
-  }
-  if (static_cast<long long>(max_blocks_per_seq) * pool->block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  pa_status st = check_decode_args(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                                    num_q_heads, scale, out, pool);
+  if (st != PA_OK || num_seqs == 0) return st;
   Variant v;
-  if (!select_variant(*pool, num_q_heads, v)) return PA_ERR_UNSUPPORTED;
+  if (!select_variant(*pool, num_q_heads, 0, v)) return PA_ERR_UNSUPPORTED;
   const int ctas = resolve_ctas(v, nullptr);
   if (ctas <= 0) return PA_ERR_CUDA;
   if (workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride) > kNoAllocScratchBytes) {
@@ -869,33 +696,13 @@ extern "C" pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const
   }
   void* scratch = nullptr;
   if (!no_alloc_scratch_address(&scratch)) return PA_ERR_CUDA;
-  const size_t parts_bytes = align_up(static_cast<size_t>(ctas) * 2 * v.part_stride * sizeof(float), 256);
-  int32_t* counters = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + parts_bytes);
+  const DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                                       num_q_heads, scale, out, scratch, ctas, v.part_stride, dev_status, pool, 0);
   // The array keeps whatever the previous call left; the arrival counters
   // must start at zero, so clear them on the caller's stream first.
-  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(num_seqs) * pool->num_kv_heads * sizeof(int32_t),
+  if (cudaMemsetAsync(prm.counters, 0, static_cast<size_t>(num_seqs) * pool->num_kv_heads * sizeof(int32_t),
                       static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     return PA_ERR_CUDA;
   }
-
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.k_pool = static_cast<const uint16_t*>(k_pool);
-  prm.v_pool = static_cast<const uint16_t*>(v_pool);
-  prm.block_tables = block_tables;
-  prm.seq_lens = seq_lens;
-  prm.out = static_cast<uint16_t*>(out);
-  prm.partials = static_cast<float*>(scratch);
-  prm.counters = counters;
-  prm.status = dev_status;
-  prm.max_nb = max_blocks_per_seq;
-  prm.num_seqs = num_seqs;
-  prm.num_q_heads = num_q_heads;
-  prm.num_kv_heads = pool->num_kv_heads;
-  prm.num_blocks = pool->num_blocks;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.wait_limit_ns = 2ull * 1000 * 1000 * 1000;
-  prm.test_flags = 0;
-  v.fn<<<ctas, kThreads, v.smem_bytes, static_cast<cudaStream_t>(stream)>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -1,0 +1,262 @@
+// Pieces shared by the two decode kernels (CUDA-core and tensor-core):
+// kernel parameters, the balanced work partition over persistent CTAs, and
+// the merge of split units through the workspace.
+//
+// Work partition.  All (sequence, kv head, logical block) triples are laid
+// end to end — sequence-major, kv head next, block innermost — and cut into
+// `nparts` contiguous ranges of equal size, one per CTA, where nparts is the
+// grid size or the total block count if that is smaller (so no range is
+// empty).  A CTA's range falls into segments, one per (sequence, kv head)
+// "unit" it touches.  A unit covered by one CTA is finished there; a unit
+// split between CTAs is finished by whichever of them arrives last.
+//
+// Merge rule (study notes ch.05 §4, the online-softmax merge applied to
+// partitions): a partial state is (m, l, acc) in the log2 domain — running
+// max m, sum l of 2^(score - m), unnormalised output acc.  Combining states
+// rescales each by 2^(m_p - M) with M = max m_p; out = sum acc' / sum l'.
+#pragma once
+
+#include <cstdint>
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+struct DecodeParams {
+  const uint16_t* q;
+  const uint16_t* k_pool;
+  const uint16_t* v_pool;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  uint16_t* out;
+  float* partials;
+  int32_t* counters;
+  int32_t* status;
+  int max_nb;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int num_blocks;
+  float scale_log2;
+  unsigned long long wait_limit_ns;
+  int test_flags;
+};
+
+constexpr int kFlagTestWithholdCopies = PA_DECODE_TEST_WITHHOLD_COPIES;  // producer issues nothing
+
+__device__ __forceinline__ int checked_len(const DecodeParams& p, int s, int B) {
+  const int n = __ldg(p.seq_lens + s);
+  return (n < 0 || n > p.max_nb * B) ? 0 : n;
+}
+
+struct Cursor {
+  int s, h, j, nb, len;
+  long long x, remaining;
+};
+
+struct Seg {
+  int s, h, j0, n, nb, len;
+  long long unit_first;  // flattened index of block 0 of unit (s, h)
+};
+
+// Next segment of the CTA's range; advances the cursor past it.
+template <int B>
+__device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams& p) {
+  if (c.remaining <= 0) return false;
+  const long long left = c.nb - c.j;
+  const int n = static_cast<int>(left < c.remaining ? left : c.remaining);
+  sg.s = c.s;
+  sg.h = c.h;
+  sg.j0 = c.j;
+  sg.n = n;
+  sg.nb = c.nb;
+  sg.len = c.len;
+  sg.unit_first = c.x - c.j;
+  c.remaining -= n;
+  c.x += n;
+  c.j += n;
+  if (c.j == c.nb) {
+    c.j = 0;
+    if (++c.h == p.num_kv_heads) {
+      c.h = 0;
+      if (c.remaining > 0) {
+        do {
+          if (++c.s >= p.num_seqs) {  // inconsistent lengths: stop cleanly
+            c.remaining = 0;
+            break;
+          }
+          c.len = checked_len(p, c.s, B);
+          c.nb = (c.len + B - 1) / B;
+        } while (c.nb == 0);
+      }
+    }
+  }
+  return true;
+}
+
+// CTA whose range [c*N/C, (c+1)*N/C) holds flattened block x.
+__device__ __forceinline__ long long cta_of(long long x, long long N, long long C) { return ((x + 1) * C - 1) / N; }
+
+__device__ __forceinline__ long long range_start(long long c, long long N, long long C) { return c * N / C; }
+
+struct RangeSmem {
+  long long scan[32];
+  long long pre0;
+  int s0;
+  int found;
+};
+
+// Block-wide inclusive scan of one value per thread (NT threads, all call).
+template <int NT>
+__device__ __forceinline__ long long block_inclusive_scan(long long v, RangeSmem& rs, long long& block_total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) rs.scan[warp] = v;
+  __syncthreads();
+  long long before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const long long t = rs.scan[w];
+    if (w < warp) before += t;
+    total += t;
+  }
+  __syncthreads();
+  block_total = total;
+  return v + before;
+}
+
+struct WorkRange {
+  long long NBT;     // total (sequence, kv head, block) triples
+  long long nparts;  // CTAs that own a non-empty range
+  long long start, end;
+};
+
+// Every thread of the CTA calls this.  Writes zero outputs of empty
+// sequences (each by one CTA), computes this CTA's range and positions the
+// cursor at its first block.  Returns false when the CTA has no work.
+template <int NT, int B>
+__device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange& wr, Cursor& cur) {
+  const int tid = threadIdx.x;
+  const long long nctas = gridDim.x, cta = blockIdx.x;
+  const int Hkv = p.num_kv_heads;
+  long long mine = 0;
+  for (int s = tid; s < p.num_seqs; s += NT) {
+    const int raw = __ldg(p.seq_lens + s);
+    int n = raw;
+    if (raw < 0 || raw > p.max_nb * B) {
+      if (cta == 0) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
+      n = 0;
+    }
+    mine += (n + B - 1) / B;
+  }
+  long long seq_blocks;
+  (void)block_inclusive_scan<NT>(mine, rs, seq_blocks);
+  wr.NBT = seq_blocks * Hkv;
+  wr.nparts = wr.NBT < nctas ? wr.NBT : nctas;
+  if (cta >= wr.nparts) return false;  // uniform across the CTA (also covers NBT == 0)
+  wr.start = range_start(cta, wr.NBT, wr.nparts);
+  wr.end = range_start(cta + 1, wr.NBT, wr.nparts);
+
+  // locate the sequence holding `start`
+  const long long target = wr.start / Hkv;  // in per-sequence block units
+  if (tid == 0) rs.found = 0;
+  __syncthreads();
+  long long base = 0;
+  for (int chunk = 0; chunk < p.num_seqs; chunk += NT) {
+    const int s = chunk + tid;
+    const long long nb = (s < p.num_seqs) ? (checked_len(p, s, B) + B - 1) / B : 0;
+    long long chunk_total;
+    const long long incl = block_inclusive_scan<NT>(nb, rs, chunk_total);
+    const long long excl = incl - nb;
+    if (nb > 0 && base + excl <= target && target < base + incl) {
+      rs.s0 = s;
+      rs.pre0 = base + excl;
+      rs.found = 1;
+    }
+    base += chunk_total;
+    __syncthreads();
+    if (rs.found) break;
+  }
+  if (!rs.found) return false;  // only with lengths changing under the kernel
+  cur.s = rs.s0;
+  cur.len = checked_len(p, cur.s, B);
+  cur.nb = (cur.len + B - 1) / B;
+  const long long off = wr.start - rs.pre0 * Hkv;
+  cur.h = static_cast<int>(off / cur.nb);
+  cur.j = static_cast<int>(off % cur.nb);
+  cur.x = wr.start;
+  cur.remaining = wr.end - wr.start;
+  return true;
+}
+
+// Zero the outputs of sequences whose length is 0 (or invalid): sequence s
+// is written by CTA s % gridDim.x.  Called by all NT threads of every CTA
+// before any early return.
+template <int NT, int B>
+__device__ __forceinline__ void zero_empty_outputs(const DecodeParams& p, int D) {
+  const long long nctas = gridDim.x, cta = blockIdx.x;
+  for (int s = threadIdx.x; s < p.num_seqs; s += NT) {
+    if ((s % nctas) != cta) continue;
+    if (checked_len(p, s, B) != 0) continue;
+    uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(s) * p.num_q_heads * D);
+    for (int i = 0; i < p.num_q_heads * D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Partial slot of CTA c for a unit whose block 0 is flattened index F: slot 0
+// if c's range starts inside the unit, else slot 1 (the unit where it ends).
+__device__ __forceinline__ size_t partial_slot(long long c, long long F, const WorkRange& wr) {
+  const int sl = (range_start(c, wr.NBT, wr.nparts) >= F) ? 0 : 1;
+  return static_cast<size_t>(c) * 2 + sl;
+}
+
+// Called by the `nthreads` threads that own a split unit's partial after it
+// is written and fenced: bumps the unit's arrival counter; the last arrival
+// merges every partial of the unit and writes the output.  `sync` is a
+// barrier over exactly those threads; `is_last` is a shared int.
+template <bool kBf16, int D, int G, typename Sync>
+__device__ void finish_split_unit(const DecodeParams& p, const Seg& sg, const WorkRange& wr, int ctid,
+                                  int nthreads, int* is_last, Sync sync) {
+  constexpr int kStride = G * (D + 2);
+  const long long F = sg.unit_first;
+  const long long first = cta_of(F, wr.NBT, wr.nparts);
+  const long long last = cta_of(F + sg.nb - 1, wr.NBT, wr.nparts);
+  int32_t* counter = p.counters + static_cast<size_t>(sg.s) * p.num_kv_heads + sg.h;
+  sync();
+  if (ctid == 0) {
+    const int prev = atomicAdd(counter, 1);
+    *is_last = (prev == static_cast<int>(last - first));
+  }
+  sync();
+  if (*is_last) {
+    __threadfence();
+    uint16_t* out_row =
+        p.out + (static_cast<size_t>(sg.s) * p.num_q_heads + static_cast<size_t>(sg.h) * G) * D;
+    for (int idx = ctid; idx < G * D / 2; idx += nthreads) {
+      const int g = (2 * idx) / D, d = (2 * idx) % D;
+      float M = -INFINITY;
+      for (long long cc = first; cc <= last; ++cc) {
+        const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
+        M = fmaxf(M, __ldcg(pp + g));
+      }
+      float L = 0.f, a0 = 0.f, a1 = 0.f;
+      for (long long cc = first; cc <= last; ++cc) {
+        const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
+        const float sc = fast_exp2(__ldcg(pp + g) - M);
+        L = fmaf(__ldcg(pp + G + g), sc, L);
+        const float2 av = __ldcg(reinterpret_cast<const float2*>(pp + 2 * G + g * D + d));
+        a0 = fmaf(av.x, sc, a0);
+        a1 = fmaf(av.y, sc, a1);
+      }
+      const float inv = 1.f / L;
+      *reinterpret_cast<uint32_t*>(out_row + g * D + d) = pack2<kBf16>(a0 * inv, a1 * inv);
+    }
+    if (ctid == 0) *counter = 0;
+  }
+}
+
+}  // namespace pa

@@ -11,15 +11,16 @@ from workloads import fill_values_numpy, random_layout
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
+@pytest.mark.parametrize("G,D", [(2, 64), (4, 128)], ids=["cuda-core", "tensor-core"])
+def test_bounded_wait_reports_timeout_and_context_survives(cuda_device, G, D):
     import time
 
     import torch
 
     import paged_kv_cache_357_b200 as pa
 
-    L = random_layout(31, [40, 70, 5], dtype="bf16", block_size=16, num_q_heads=4, num_kv_heads=2, head_dim=64,
-                      write_new_token=False)
+    L = random_layout(31, [40, 70, 5], dtype="bf16", block_size=16, num_q_heads=2 * G, num_kv_heads=2,
+                      head_dim=D, write_new_token=False)
     V = fill_values_numpy(L)
     d = to_device(L, V, cuda_device)
     st = torch.zeros(1, dtype=torch.int32, device=cuda_device)

@@ -209,3 +209,34 @@ def test_device_errors_are_reported_not_trapped(pa_mod, cuda_device):
     # the context is still usable
     L3 = config_tiny()
     _run_and_check(L3, fill_values_numpy(L3), cuda_device, what="after errors")
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("G", [4, 8])
+def test_tensor_core_and_cuda_core_paths_agree(pa_mod, cuda_device, dtype, G):
+    """Groups of 4 and 8 at head_dim 128 / block 16 run on the tensor-core
+    kernel by default; the CUDA-core kernel is forced with a flag.  Both must
+    match the oracle, and each other to within the combined tolerance."""
+    import torch
+
+    lens = [1, 2, 15, 16, 17, 127, 128, 129, 300, 1000, 2049, 5]
+    L = random_layout(4000 + G, lens, dtype=dtype, block_size=16, num_q_heads=2 * G, num_kv_heads=2,
+                      head_dim=128, write_new_token=True)
+    V = fill_values_numpy(L)
+    ref, _, _ = oracle_step(L, V)
+    outs = {}
+    for name, flags in (("tensor", 0), ("cuda", pa_mod.PA_DECODE_CUDA_CORES_ONLY)):
+        d = to_device(L, V, cuda_device)
+        st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+        pa_mod.pa_cache_write(d["new_k"], d["new_v"], d["slots"], d["k_pool"], d["v_pool"], st)
+        out = torch.full_like(d["q"], float("nan"))
+        ws = pa_mod.alloc_decode_workspace(L.num_seqs, L.num_q_heads, d["k_pool"], flags=flags)
+        pa_mod.pa_decode(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], L.scale, out, ws, st,
+                         flags=flags)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0, name
+        outs[name] = torch_f64(out)
+        assert_attention_close(outs[name], ref, f"{name} G={G} {dtype}")
+    # both sit within the tolerance of the oracle, so they differ by at most twice it
+    diff = np.abs(outs["tensor"] - outs["cuda"])
+    assert (diff <= 2 * (2e-3 + 1e-2 * np.abs(ref))).all(), diff.max()
