@@ -45,8 +45,8 @@ METRIC = "paged decode-attention HBM GB/s and % of roofline; tokens/s at Llama-3
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "pa_decode_llama3_8b.md")
 KERNEL_SOURCES = [
-    os.path.join(ROOT, "paged_kv_cache_357_b200", "csrc", "pa_decode.cu"),
-    os.path.join(ROOT, "paged_kv_cache_357_b200", "csrc", "pa_device.cuh"),
+    os.path.join(ROOT, "paged_kv_cache_357_b200", "csrc", name)
+    for name in ("pa_decode.cu", "pa_decode_tc.cu", "pa_decode_common.cuh", "pa_device.cuh")
 ]
 
 
@@ -104,6 +104,13 @@ def kernel_source_hash() -> str:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def decode_kernel_name(L) -> str:
+    """Which decode kernel the library runs for this workload by default."""
+    if L.head_dim == 128 and L.block_size == 16 and L.group in (4, 8):
+        return "pa_decode_tc_kernel (tcgen05)"
+    return "pa_decode_kernel (CUDA cores)"
 
 
 def profiled_traffic(decode_bytes_per_launch):
@@ -429,7 +436,7 @@ def run_ours(args):
             "decode_ms_p50": decode_ms[K // 2],
             "bytes": nbytes,
             "roofline": {
-                "kernel": "pa_decode_kernel",
+                "kernel": decode_kernel_name(L),
                 "bound": "hbm",
                 "achieved": achieved,
                 "peak": peak,
