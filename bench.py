@@ -127,6 +127,24 @@ def profiled_traffic(decode_bytes_per_launch):
     return float(m_traf.group(1))
 
 
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of per-rank timings over the default process group
+    (identity with one rank).  NCCL needs a CUDA device, gloo runs on CPU."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_gbs(world: int, bytes_per_step_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank moves its own shard's bytes in the
+    slowest rank's step time (weak scaling)."""
+    return world * bytes_per_step_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -395,12 +413,9 @@ def run_ours(args):
         raise SystemExit("device status set in the e2e loop")
 
     # ---- max over ranks
-    t = torch.tensor([elapsed_ms, e2e_ms, decode_mean_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, decode_mean_ms = (float(x) for x in t.tolist())
+    elapsed_ms, e2e_ms, decode_mean_ms = max_over_ranks([elapsed_ms, e2e_ms, decode_mean_ms], dev)
     ms_per_step = elapsed_ms / K
-    value = world * nbytes["step"] / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbs(world, nbytes["step"], ms_per_step)
     tokens_per_s = world * L.num_seqs / (ms_per_step * 1e-3)
     peak, peak_kind = measured_hbm_peak()
     achieved = nbytes["decode"] / (decode_mean_ms * 1e-3) / 1e9
@@ -448,7 +463,7 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": nbytes["decode"],
             },
             "e2e": {
-                "value": world * nbytes["step"] / (e2e_ms * 1e-3) / 1e9,
+                "value": whole_job_gbs(world, nbytes["step"], e2e_ms),
                 "unit": "GB/s",
                 "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": step.last_h2d_bytes,
