@@ -15,15 +15,18 @@
 //
 // Roles (192 threads, one CTA per SM):
 //   warp 0      producer: resolves block ids, issues 2-D TMA loads of the K and
-//               V tiles (64-column boxes, 128-byte swizzle) into a 3-stage ring
-//               of 64 KB chunk stages, and of the group's q rows.
+//               V tiles (64-column boxes, 128-byte swizzle) into separate rings
+//               of 32 KB chunk stages — 2 for K, released when its QK is done,
+//               4 for V, released when its PV is done — and of the q rows.
 //   warp 1      allocates 64 TMEM columns; lane 0 issues every tcgen05.mma and
-//               tcgen05.commit: QK of chunk i+1 is issued before PV of chunk i.
+//               tcgen05.commit, polling which of QK(next) and PV(oldest
+//               pending) is ready and issuing it.
 //   warps 2-5   softmax + epilogue, one TMEM lane (token row, then head_dim
 //               index) per thread: read S^T from TMEM, online softmax with a
 //               cross-warp max per chunk, write P^T (bf16/fp16) into a swizzled
 //               shared buffer, zero V rows past the sequence end inside the
 //               last 16-token step, then read O^T and rescale-accumulate.
+//               The epilogue of chunk i runs after the softmax of chunk i+1.
 // The swizzled layouts written by TMA serve both products directly: the K
 // tile is a K-major A operand for QK, the V tile an MN-major A operand for PV.
 #include <cuda.h>
@@ -46,10 +49,11 @@ constexpr int B = 16;
 constexpr int kChunkTok = 128;             // tokens per chunk = MMA M of QK
 constexpr int CB = kChunkTok / B;          // blocks per chunk
 constexpr int N = 16;                      // MMA N (query heads, padded)
-constexpr int kStages = 3;
+constexpr int kKStages = 2;  // K is released as soon as its QK completes
+constexpr int kVStages = 4;  // V is held until its PV completes
 constexpr int kRowBytes = 128;             // one swizzle row: 64 elements
 constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 tokens
-constexpr int kStageBytes = 4 * kHalfBytes;        // K[0:64) K[64:128) V[0:64) V[64:128)
+constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
 constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
 constexpr int kQSlotBytes = 2 * N * kRowBytes;     // two halves of 16 rows
 constexpr int kPSlotBytes = 2 * N * kRowBytes;     // tokens [0,64) and [64,128), 16 rows each
@@ -59,13 +63,16 @@ constexpr int kSoftmaxBarrier = 1;
 constexpr uint32_t kTmemCols = 64;  // S[0], S[1], O[0], O[1]: 16 fp32 columns each
 
 struct TcSmem {
-  uint8_t stage[kStages][kStageBytes];  // 1024-aligned regions
+  uint8_t kbuf[kKStages][kOperandBytes];  // 1024-aligned regions
+  uint8_t vbuf[kVStages][kOperandBytes];
   uint8_t q[2][kQSlotBytes];
   uint8_t p[2][kPSlotBytes];
   float red[2][4][8];
   float lred[4][8];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t kfull[kKStages];
+  uint64_t kempty[kKStages];
+  uint64_t vfull[kVStages];
+  uint64_t vempty[kVStages];
   uint64_t qfull[2];
   uint64_t qempty[2];
   uint64_t s_full[2];
@@ -78,8 +85,10 @@ struct TcSmem {
   uint32_t tmem_base;
   int abort;
   int is_last;
-  int issued;
-  int consumed;
+  int k_issued;
+  int k_consumed;
+  int v_issued;
+  int v_consumed;
   int q_issued;
   int q_consumed;
 };
@@ -205,9 +214,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!decode_prologue<kThreads, B>(p, sm.range, wr, cur)) return;  // uniform across the CTA
 
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm.full[i], 1);
-      mbar_init(&sm.empty[i], 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sm.kfull[i], 1);
+      mbar_init(&sm.kempty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sm.vfull[i], 1);
+      mbar_init(&sm.vempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.qfull[i], 1);
@@ -220,8 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.mma_done, 1);
     sm.abort = 0;
-    sm.issued = 0;
-    sm.consumed = 0;
+    sm.k_issued = 0;
+    sm.k_consumed = 0;
+    sm.v_issued = 0;
+    sm.v_consumed = 0;
     sm.q_issued = 0;
     sm.q_consumed = 0;
     fence_barrier_init();
@@ -242,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t pol_stream = l2_policy_evict_first();
     const uint64_t pol_keep = l2_policy_evict_last();
     bool ok = true;
-    int ci = 0, qi = 0, issued = 0, q_issued = 0;
+    int ci = 0, qi = 0, k_issued = 0, v_issued = 0, q_issued = 0;
     if (lane == 0) {
       prefetch_tensormap(&map_q);
       prefetch_tensormap(&map_k);
@@ -272,40 +287,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         ++qi;
-        const int32_t* trow = p.block_tables + static_cast<size_t>(sg.s) * p.max_nb;
-        for (int c0 = 0; c0 < sg.n; c0 += CB) {
-          const ChunkInfo ch = chunk_at(sg, c0);
-          int e = 0;
-          if (lane < ch.nblk) {
-            e = __ldg(trow + ch.j + lane);
-            if (e < 0 || e >= p.num_blocks) {
-              record_status(p.status, PA_DEV_BAD_BLOCK_ID);
-              e = 0;
-            }
+        // Block-table entries 32 at a time (lane l holds entry b0 + l); the
+        // next batch is in flight while the current one is issued.
+        const int32_t* trow = p.block_tables + static_cast<size_t>(sg.s) * p.max_nb + sg.j0;
+        int e_cur = (lane < sg.n) ? __ldg(trow + lane) : 0;
+        for (int b0 = 0; ok && b0 < sg.n; b0 += 32) {
+          const int e_next = (b0 + 32 + lane < sg.n) ? __ldg(trow + b0 + 32 + lane) : 0;
+          if (b0 + lane < sg.n && (e_cur < 0 || e_cur >= p.num_blocks)) {
+            record_status(p.status, PA_DEV_BAD_BLOCK_ID);
+            e_cur = 0;
           }
-          const int st = ci % kStages;
-          if (lane == 0) {
-            ok = mbar_wait_bounded(&sm.empty[st], ((ci / kStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
-            if (ok) mbar_arrive_expect_tx(&sm.full[st], ch.nblk * 4 * kBlockBytes);
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
-          if (lane < ch.nblk) {
+          const int b_end = min(b0 + 32, sg.n);
+          for (int c0 = b0; c0 < b_end; c0 += CB) {
+            const ChunkInfo ch = chunk_at(sg, c0);
+            const int e = __shfl_sync(0xffffffffu, e_cur, (c0 - b0) + (lane & (CB - 1)));
+            const int ks = ci % kKStages, vs = ci % kVStages;
             const int y = (e * Hkv + sg.h) * B;
-            uint8_t* base = sm.stage[st] + lane * kBlockBytes;
-            tma_load_2d(base, &map_k, 0, y, &sm.full[st], pol_stream);
-            tma_load_2d(base + kHalfBytes, &map_k, 64, y, &sm.full[st], pol_stream);
-            tma_load_2d(base + 2 * kHalfBytes, &map_v, 0, y, &sm.full[st], pol_stream);
-            tma_load_2d(base + 3 * kHalfBytes, &map_v, 64, y, &sm.full[st], pol_stream);
+            if (lane == 0) {
+              ok = mbar_wait_bounded(&sm.kempty[ks], ((ci / kKStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+              if (ok) mbar_arrive_expect_tx(&sm.kfull[ks], ch.nblk * 2 * kBlockBytes);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane < ch.nblk) {
+              uint8_t* base = sm.kbuf[ks] + lane * kBlockBytes;
+              tma_load_2d(base, &map_k, 0, y, &sm.kfull[ks], pol_stream);
+              tma_load_2d(base + kHalfBytes, &map_k, 64, y, &sm.kfull[ks], pol_stream);
+            }
+            __syncwarp();
+            ++k_issued;
+            if (lane == 0) {
+              ok = mbar_wait_bounded(&sm.vempty[vs], ((ci / kVStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+              if (ok) mbar_arrive_expect_tx(&sm.vfull[vs], ch.nblk * 2 * kBlockBytes);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane < ch.nblk) {
+              uint8_t* base = sm.vbuf[vs] + lane * kBlockBytes;
+              tma_load_2d(base, &map_v, 0, y, &sm.vfull[vs], pol_stream);
+              tma_load_2d(base + kHalfBytes, &map_v, 64, y, &sm.vfull[vs], pol_stream);
+            }
+            __syncwarp();
+            ++v_issued;
+            ++ci;
           }
-          __syncwarp();
-          ++issued;
-          ++ci;
+          e_cur = e_next;
         }
       }
     }
     if (lane == 0) {
-      sm.issued = issued;
+      sm.k_issued = k_issued;
+      sm.v_issued = v_issued;
       sm.q_issued = q_issued;
       if (!ok) {
         sm.abort = 1;
@@ -314,74 +346,101 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ===================== MMA issuer ========================================
+    // A non-blocking scheduler: each pass tests whether QK of the next chunk
+    // (its K/V landed, its S buffer free, its q ready) or PV of the oldest
+    // chunk still waiting (its P written, its O buffer free) can go, and
+    // issues whichever can, so PV of chunk i never waits for chunk i+1's data.
     if (lane == 0) {
       constexpr uint32_t kIdescQK = make_idesc(kBf16, false);
       constexpr uint32_t kIdescPV = make_idesc(kBf16, true);
       bool ok = true;
-      int ci = 0, qi = 0, consumed = 0, q_consumed = 0;
-      bool have_prev = false;
-      int prev_ci = 0, prev_st = 0, prev_ntok = 0;
-      auto issue_pv = [&](int c, int st, int ntok) -> bool {
-        const int pb = c & 1;
-        const uint32_t par = (c >> 1) & 1;
-        if (!mbar_wait_bounded(&sm.p_full[pb], par, abort_flag, p.wait_limit_ns)) return false;
-        if (!mbar_wait_bounded(&sm.o_free[pb], par ^ 1u, abort_flag, p.wait_limit_ns)) return false;
-        tc_fence_after();
-        const uint32_t v0 = smem_u32(sm.stage[st] + 2 * kHalfBytes);
-        const uint32_t p0 = smem_u32(sm.p[pb]);
-        const int nks = (ntok + 15) / 16;
-        for (int k = 0; k < nks; ++k) {
-          const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
-          const uint64_t b = sw128_desc(p0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-          umma(tmem + kColO + pb * N, a, b, kIdescPV, k > 0 ? 1u : 0u);
-        }
-        umma_commit(&sm.o_full[pb]);
-        umma_commit(&sm.empty[st]);
-        return true;
-      };
+      int qk = 0, pv = 0, seg_i = 0, q_consumed = 0;
+      uint32_t ring = 0;  // valid tokens of each pending chunk (index & 3), 8 bits each
+      bool have_seg = false, q_ready = false, walk_done = false;
+      int c0 = 0;
       Seg sg;
-      while (ok && next_seg<B>(cur, sg, p)) {
-        const int qs = qi & 1;
-        ok = mbar_wait_bounded(&sm.qfull[qs], (qi >> 1) & 1, abort_flag, p.wait_limit_ns);
-        if (!ok) break;
-        ++q_consumed;
-        ++qi;
-        const uint32_t q0 = smem_u32(sm.q[qs]);
-        for (int c0 = 0; c0 < sg.n; c0 += CB) {
-          const ChunkInfo ch = chunk_at(sg, c0);
-          const int st = ci % kStages;
-          ok = mbar_wait_bounded(&sm.full[st], (ci / kStages) & 1, abort_flag, p.wait_limit_ns);
-          if (!ok) break;
-          ++consumed;
-          const int sb = ci & 1;
-          ok = mbar_wait_bounded(&sm.s_free[sb], ((ci >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t k0 = smem_u32(sm.stage[st]);
+      uint64_t t_idle = 0;
+      uint32_t idle = 0;
+      while (ok) {
+        bool progress = false;
+        if (!walk_done && !have_seg) {
+          if (next_seg<B>(cur, sg, p)) {
+            have_seg = true;
+            c0 = 0;
+          } else {
+            walk_done = true;
+          }
+        }
+        if (have_seg) {
+          const int qs = seg_i & 1;
+          if (!q_ready && mbar_test_wait(&sm.qfull[qs], (seg_i >> 1) & 1)) {
+            q_ready = true;
+            ++q_consumed;
+          }
+          const int ks = qk % kKStages;
+          if (q_ready && qk - pv < 4 && mbar_test_wait(&sm.kfull[ks], (qk / kKStages) & 1) &&
+              mbar_test_wait(&sm.s_free[qk & 1], ((qk >> 1) & 1) ^ 1u)) {
+            tc_fence_after();
+            const uint32_t k0 = smem_u32(sm.kbuf[ks]);
+            const uint32_t q0 = smem_u32(sm.q[qs]);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t a = sw128_desc(k0 + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-            const uint64_t b = sw128_desc(q0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-            umma(tmem + kColS + sb * N, a, b, kIdescQK, k > 0 ? 1u : 0u);
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t a = sw128_desc(k0 + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              const uint64_t b = sw128_desc(q0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              umma(tmem + kColS + (qk & 1) * N, a, b, kIdescQK, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[qk & 1]);
+            umma_commit(&sm.kempty[ks]);
+            const int slot_shift = (qk & 3) * 8;
+            ring = (ring & ~(0xFFu << slot_shift)) | (static_cast<uint32_t>(chunk_at(sg, c0).ntok) << slot_shift);
+            c0 += CB;
+            if (c0 >= sg.n) {  // last chunk of the segment: q may be reloaded after this QK
+              umma_commit(&sm.qempty[qs]);
+              have_seg = false;
+              q_ready = false;
+              ++seg_i;
+            }
+            ++qk;
+            progress = true;
           }
-          umma_commit(&sm.s_full[sb]);
-          if (c0 + CB >= sg.n) umma_commit(&sm.qempty[qs]);
-          if (have_prev) {
-            ok = issue_pv(prev_ci, prev_st, prev_ntok);
-            if (!ok) break;
+        }
+        if (pv < qk) {
+          const int pb = pv & 1;
+          const uint32_t par = (pv >> 1) & 1;
+          const int vs = pv % kVStages;
+          if (mbar_test_wait(&sm.p_full[pb], par) && mbar_test_wait(&sm.o_free[pb], par ^ 1u) &&
+              mbar_test_wait(&sm.vfull[vs], (pv / kVStages) & 1)) {
+            tc_fence_after();
+            const int ntok = static_cast<int>((ring >> ((pv & 3) * 8)) & 0xFFu);
+            const uint32_t v0 = smem_u32(sm.vbuf[vs]);
+            const uint32_t p0 = smem_u32(sm.p[pb]);
+            const int nks = (ntok + 15) / 16;
+            for (int k = 0; k < nks; ++k) {
+              const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
+              const uint64_t b = sw128_desc(p0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              umma(tmem + kColO + pb * N, a, b, kIdescPV, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.o_full[pb]);
+            umma_commit(&sm.vempty[vs]);
+            ++pv;
+            progress = true;
           }
-          have_prev = true;
-          prev_ci = ci;
-          prev_st = st;
-          prev_ntok = ch.ntok;
-          ++ci;
+        } else if (walk_done) {
+          break;  // every chunk has had its QK and its PV
+        }
+        if (progress) {
+          idle = 0;
+        } else if ((++idle & 63u) == 0) {
+          const uint64_t now = global_timer_ns();
+          if (idle == 64) t_idle = now;
+          if (*abort_flag != 0 || now - t_idle > p.wait_limit_ns) ok = false;
         }
       }
-      if (ok && have_prev) ok = issue_pv(prev_ci, prev_st, prev_ntok);
       // every MMA issued above completes before TMEM is released
       umma_commit(&sm.mma_done);
       (void)mbar_wait_bounded(&sm.mma_done, 0, nullptr, p.wait_limit_ns);
-      sm.consumed = consumed;
+      sm.k_consumed = qk;
+      sm.v_consumed = pv;
       sm.q_consumed = q_consumed;
       if (!ok) {
         sm.abort = 1;
@@ -391,6 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ===================== softmax + epilogue (warps 2-5) ====================
+    // Per chunk i: softmax(i) then the epilogue of chunk i-1, so the PV of
+    // chunk i-1 runs on the tensor core while the softmax of chunk i runs here.
     const int quad = warp & 3;           // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;      // token row of the chunk; head_dim index in the epilogue
     const int ctid = tid - 64;           // 0..127
@@ -398,95 +459,114 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int ci = 0;
     Seg sg;
+    float m[G], lthr[G], acc[G], a_pend[G];
+
+    // Online softmax of chunk ci; writes its P^T and returns the rescale
+    // factor of the running output in alpha.
+    auto softmax_chunk = [&](int ci, const ChunkInfo& ch, float* alpha) -> bool {
+      const int vs = ci % kVStages;
+      const int sb = ci & 1;
+      const uint32_t par = (ci >> 1) & 1;
+      bool w = mbar_wait_bounded(&sm.s_full[sb], par, abort_flag, p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      float s16[16];
+      tmem_ld16(tmem + lane_base + kColS + sb * N, s16);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[sb]);
+
+      const bool valid = r < ch.ntok;
+      float sc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        sc[g] = valid ? s16[g] * p.scale_log2 : -INFINITY;
+        float wm = sc[g];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+        if (lane == 0) sm.red[sb][quad][g] = wm;
+      }
+      named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+      float pr[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float cm = fmaxf(fmaxf(sm.red[sb][0][g], sm.red[sb][1][g]), fmaxf(sm.red[sb][2][g], sm.red[sb][3][g]));
+        const float m_new = fmaxf(m[g], cm);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha[g] = fast_exp2(m[g] - m_use);
+        m[g] = m_new;
+        pr[g] = fast_exp2(sc[g] - m_use);
+        lthr[g] = fmaf(lthr[g], alpha[g], pr[g]);
+      }
+      // P^T into the swizzled B operand: row = head, column = token
+      const int pb = ci & 1;
+      {
+        uint8_t* pbase = sm.p[pb] + (r >> 6) * (N * kRowBytes);
+        const int c = r & 63;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const int off = (g >> 3) * (8 * kRowBytes) + (g & 7) * kRowBytes + ((((c >> 3) ^ (g & 7)) & 7) << 4) +
+                          (c & 7) * 2;
+          const uint32_t two = pack2<kBf16>(pr[g], 0.f);
+          *reinterpret_cast<uint16_t*>(pbase + off) = static_cast<uint16_t>(two & 0xffffu);
+        }
+      }
+      // V rows past the sequence end inside the last 16-token step are zeroed
+      // so that 0 * (whatever they hold) cannot reach the output
+      if ((ch.ntok & 15) != 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
+        (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
+        uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + r * kRowBytes);
+        uint4* v1 = reinterpret_cast<uint4*>(sm.vbuf[vs] + kHalfBytes + r * kRowBytes);
+#pragma unroll
+        for (int i = 0; i < kRowBytes / 16; ++i) {
+          v0[i] = make_uint4(0, 0, 0, 0);
+          v1[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[pb]);
+      return true;
+    };
+
+    // acc = acc * alpha + O^T row r of chunk ci.
+    auto epilogue_chunk = [&](int ci, const float* alpha) -> bool {
+      const int pb = ci & 1;
+      bool w = mbar_wait_bounded(&sm.o_full[pb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      float o16[16];
+      tmem_ld16(tmem + lane_base + kColO + pb * N, o16);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free[pb]);
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = fmaf(acc[g], alpha[g], o16[g]);
+      return true;
+    };
+
     while (ok && next_seg<B>(cur, sg, p)) {
-      float m[G], lthr[G], acc[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
         lthr[g] = 0.f;
         acc[g] = 0.f;
       }
+      bool pending = false;
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
-        const ChunkInfo ch = chunk_at(sg, c0);
-        const int st = ci % kStages;
-        const int sb = ci & 1;
-        const uint32_t par = (ci >> 1) & 1;
-        ok = mbar_wait_bounded(&sm.s_full[sb], par, abort_flag, p.wait_limit_ns);
-        ok = __all_sync(0xffffffffu, ok);
+        float alpha[G];
+        ok = softmax_chunk(ci, chunk_at(sg, c0), alpha);
         if (!ok) break;
-        tc_fence_after();
-        float s16[16];
-        tmem_ld16(tmem + lane_base + kColS + sb * N, s16);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_free[sb]);
-
-        // ---- online softmax over the chunk (log2 domain)
-        const bool valid = r < ch.ntok;
-        float sc[G], alpha[G], pr[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          sc[g] = valid ? s16[g] * p.scale_log2 : -INFINITY;
-          float wm = sc[g];
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
-          if (lane == 0) sm.red[sb][quad][g] = wm;
+        if (pending) {
+          ok = epilogue_chunk(ci - 1, a_pend);
+          if (!ok) break;
         }
-        named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float cm = fmaxf(fmaxf(sm.red[sb][0][g], sm.red[sb][1][g]), fmaxf(sm.red[sb][2][g], sm.red[sb][3][g]));
-          const float m_new = fmaxf(m[g], cm);
-          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          alpha[g] = fast_exp2(m[g] - m_use);
-          m[g] = m_new;
-          pr[g] = fast_exp2(sc[g] - m_use);
-          lthr[g] = fmaf(lthr[g], alpha[g], pr[g]);
-        }
-
-        // ---- P^T into the swizzled B operand: row = head, column = token
-        const int pb = ci & 1;
-        {
-          uint8_t* pbase = sm.p[pb] + (r >> 6) * (N * kRowBytes);
-          const int c = r & 63;
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const int off = (g >> 3) * (8 * kRowBytes) + (g & 7) * kRowBytes + ((((c >> 3) ^ (g & 7)) & 7) << 4) +
-                            (c & 7) * 2;
-            const uint32_t two = pack2<kBf16>(pr[g], 0.f);
-            *reinterpret_cast<uint16_t*>(pbase + off) = static_cast<uint16_t>(two & 0xffffu);
-          }
-        }
-        // ---- V rows past the sequence end inside the last 16-token step are
-        // zeroed so that 0 * (whatever they hold) cannot reach the output
-        if ((ch.ntok & 15) != 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
-          (void)mbar_wait_bounded(&sm.full[st], (ci / kStages) & 1, abort_flag, p.wait_limit_ns);
-          uint4* v0 = reinterpret_cast<uint4*>(sm.stage[st] + 2 * kHalfBytes + r * kRowBytes);
-          uint4* v1 = reinterpret_cast<uint4*>(sm.stage[st] + 3 * kHalfBytes + r * kRowBytes);
-#pragma unroll
-          for (int i = 0; i < kRowBytes / 16; ++i) {
-            v0[i] = make_uint4(0, 0, 0, 0);
-            v1[i] = make_uint4(0, 0, 0, 0);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[pb]);
-
-        // ---- epilogue of the chunk: O^T row r (head_dim index r)
-        ok = mbar_wait_bounded(&sm.o_full[pb], par, abort_flag, p.wait_limit_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        float o16[16];
-        tmem_ld16(tmem + lane_base + kColO + pb * N, o16);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.o_free[pb]);
-#pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] = fmaf(acc[g], alpha[g], o16[g]);
+        for (int g = 0; g < G; ++g) a_pend[g] = alpha[g];
+        pending = true;
         ++ci;
       }
+      if (ok && pending) ok = epilogue_chunk(ci - 1, a_pend);
       if (!ok) break;
 
       // ---- end of the segment: total sums, then output or partial state
@@ -536,8 +616,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (tid == 0 && sm.abort) {
-    for (int k = sm.consumed; k < sm.issued; ++k) {
-      (void)mbar_wait_bounded(&sm.full[k % kStages], (k / kStages) & 1, nullptr, p.wait_limit_ns);
+    for (int k = sm.k_consumed; k < sm.k_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.kfull[k % kKStages], (k / kKStages) & 1, nullptr, p.wait_limit_ns);
+    }
+    for (int k = sm.v_consumed; k < sm.v_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.vfull[k % kVStages], (k / kVStages) & 1, nullptr, p.wait_limit_ns);
     }
     for (int k = sm.q_consumed; k < sm.q_issued; ++k) {
       (void)mbar_wait_bounded(&sm.qfull[k & 1], (k >> 1) & 1, nullptr, p.wait_limit_ns);

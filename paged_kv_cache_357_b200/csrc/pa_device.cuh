@@ -14,7 +14,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
-#include "../../include/pa.h"
+#include "pa.h"
 
 namespace pa {
 
@@ -46,6 +46,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       "{\n"
       "  .reg .pred p;\n"
       "  mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "  selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Non-blocking test of the phase with the given parity (acquire on success).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
       "  selp.u32 %0, 1, 0, p;\n"
       "}\n"
       : "=r"(done)
