@@ -4,14 +4,22 @@ The K/V pools are the cache state: they stay resident in device memory
 across steps.  What changes every step arrives from the host — q, the block
 tables and lengths, the new tokens' K/V with their slots, and any
 copy-on-write pairs — and the attention output goes back to the host.  A
-step enqueues, on one stream:
+step runs, in the order the method needs:
 
     H2D copies -> pa_copy_blocks -> pa_cache_write -> pa_decode -> D2H copy
 
-matching the order of the method: a shared block is copied before a sample
-writes into it (study notes ch.05 §6.1), the new token is stored before the
-decode reads it (vLLM blog, plain-language section), and the decode reads every block through the
-table (vLLM blog §"关键细节" 2)).
+a shared block is copied before a sample writes into it (study notes ch.05
+§6.1), the new token is stored before the decode reads it (vLLM blog,
+plain-language section), and the decode reads every block through the table
+(vLLM blog §"关键细节" 2).
+
+Consecutive steps overlap their copies with each other's kernels: the
+per-step device buffers come in two sets used alternately, uploads run on
+one stream, kernels on a second and downloads on a third.  Events order the
+work: a step's kernels wait for its uploads and for the previous step's
+kernels (they share the pools); its download waits for its kernels; the
+upload into a buffer set waits until the kernels that read that set two
+steps earlier are done.
 """
 
 from __future__ import annotations
@@ -21,10 +29,27 @@ from typing import Optional
 from . import _lib
 
 
+class _BufferSet:
+    def __init__(self, torch, dev, dt, S, Hq, D, Hkv, max_nb, T, P):
+        self.q = torch.empty((S, Hq, D), dtype=dt, device=dev)
+        self.out = torch.empty_like(self.q)
+        self.tables = torch.empty((S, max_nb), dtype=torch.int32, device=dev)
+        self.lens = torch.empty((S,), dtype=torch.int32, device=dev)
+        self.new_k = torch.empty((max(T, 1), Hkv, D), dtype=dt, device=dev)
+        self.new_v = torch.empty_like(self.new_k)
+        self.slots = torch.empty((max(T, 1),), dtype=torch.int64, device=dev)
+        self.pairs = torch.empty((max(P, 1), 2), dtype=torch.int64, device=dev)
+        self.out_host = torch.empty(self.out.shape, dtype=dt, pin_memory=True)
+        self.uploaded = torch.cuda.Event()
+        self.computed = torch.cuda.Event()
+        self.downloaded = torch.cuda.Event()
+        self.used = False
+
+
 class PagedDecodeStep:
     def __init__(self, k_pool, v_pool, num_seqs: int, num_q_heads: int, max_blocks_per_seq: int,
                  max_new_tokens: int = 0, max_copy_pairs: int = 0, scale: Optional[float] = None,
-                 stream=None, num_ctas: int = 0):
+                 num_ctas: int = 0):
         import torch
 
         self.torch = torch
@@ -33,53 +58,82 @@ class PagedDecodeStep:
         NB, Hkv, B, D = k_pool.shape
         self.S, self.Hq, self.D, self.Hkv = num_seqs, num_q_heads, D, Hkv
         self.scale = (1.0 / D**0.5) if scale is None else float(scale)
-        self.stream = torch.cuda.Stream(device=dev) if stream is None else stream
         self.num_ctas = num_ctas
-        dt = k_pool.dtype
-        self.q = torch.empty((num_seqs, num_q_heads, D), dtype=dt, device=dev)
-        self.out = torch.empty_like(self.q)
-        self.tables = torch.empty((num_seqs, max_blocks_per_seq), dtype=torch.int32, device=dev)
-        self.lens = torch.empty((num_seqs,), dtype=torch.int32, device=dev)
-        self.new_k = torch.empty((max(max_new_tokens, 1), Hkv, D), dtype=dt, device=dev)
-        self.new_v = torch.empty_like(self.new_k)
-        self.slots = torch.empty((max(max_new_tokens, 1),), dtype=torch.int64, device=dev)
-        self.pairs = torch.empty((max(max_copy_pairs, 1), 2), dtype=torch.int64, device=dev)
+        self.h2d_stream = torch.cuda.Stream(device=dev)
+        self.compute_stream = torch.cuda.Stream(device=dev)
+        self.d2h_stream = torch.cuda.Stream(device=dev)
+        self.sets = [_BufferSet(torch, dev, k_pool.dtype, num_seqs, num_q_heads, D, Hkv, max_blocks_per_seq,
+                                max_new_tokens, max_copy_pairs) for _ in range(2)]
         self.workspace = _lib.alloc_decode_workspace(num_seqs, num_q_heads, k_pool, num_ctas)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
-        self.out_host = torch.empty(self.out.shape, dtype=dt, pin_memory=True)
+        self.steps = 0
         self.last_h2d_bytes = 0
         self.last_d2h_bytes = 0
 
     def run(self, q, block_tables, seq_lens, new_k=None, new_v=None, slot_mapping=None, copy_pairs=None):
-        """Enqueue one step from host tensors (pinned for overlap); returns the
-        pinned host output tensor, valid after ``self.stream`` synchronises."""
+        """Enqueue one step from host tensors (pinned, so the copies run
+        asynchronously; leave them unchanged until the step completes).
+        Returns the pinned host output of this step, valid once
+        ``wait(result)`` or ``synchronize()`` returns and until the step after
+        next reuses it."""
         torch = self.torch
+        bs = self.sets[self.steps % 2]
         h2d = 0
-        with torch.cuda.stream(self.stream):
-            for dst, src in ((self.q, q), (self.tables, block_tables), (self.lens, seq_lens)):
+        with torch.cuda.stream(self.h2d_stream):
+            if bs.used:
+                self.h2d_stream.wait_event(bs.computed)  # kernels of two steps ago read this set
+            for dst, src in ((bs.q, q), (bs.tables, block_tables), (bs.lens, seq_lens)):
                 dst.copy_(src, non_blocking=True)
                 h2d += src.numel() * src.element_size()
-            if copy_pairs is not None and copy_pairs.shape[0] > 0:
-                n = copy_pairs.shape[0]
-                self.pairs[:n].copy_(copy_pairs, non_blocking=True)
+            n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
+            if n_pairs > 0:
+                bs.pairs[:n_pairs].copy_(copy_pairs, non_blocking=True)
                 h2d += copy_pairs.numel() * copy_pairs.element_size()
-                _lib.pa_copy_blocks(self.pairs[:n], self.k_pool, self.v_pool, self.status, stream=self.stream)
-            if slot_mapping is not None and slot_mapping.shape[0] > 0:
-                T = slot_mapping.shape[0]
-                self.new_k[:T].copy_(new_k, non_blocking=True)
-                self.new_v[:T].copy_(new_v, non_blocking=True)
-                self.slots[:T].copy_(slot_mapping, non_blocking=True)
+            T = 0 if slot_mapping is None else slot_mapping.shape[0]
+            if T > 0:
+                bs.new_k[:T].copy_(new_k, non_blocking=True)
+                bs.new_v[:T].copy_(new_v, non_blocking=True)
+                bs.slots[:T].copy_(slot_mapping, non_blocking=True)
                 h2d += sum(t.numel() * t.element_size() for t in (new_k, new_v, slot_mapping))
-                _lib.pa_cache_write(self.new_k[:T], self.new_v[:T], self.slots[:T], self.k_pool, self.v_pool,
-                                    self.status, stream=self.stream)
-            _lib.pa_decode(self.q, self.k_pool, self.v_pool, self.tables, self.lens, self.scale, self.out,
-                           self.workspace, self.status, num_ctas=self.num_ctas, stream=self.stream)
-            self.out_host.copy_(self.out, non_blocking=True)
+            bs.uploaded.record(self.h2d_stream)
+        with torch.cuda.stream(self.compute_stream):
+            # the compute stream is in order, so the previous step's kernels
+            # (which read the pools this step writes) are already ahead of us
+            self.compute_stream.wait_event(bs.uploaded)
+            if bs.used:
+                self.compute_stream.wait_event(bs.downloaded)  # out of this set was read back
+            if n_pairs > 0:
+                _lib.pa_copy_blocks(bs.pairs[:n_pairs], self.k_pool, self.v_pool, self.status,
+                                    stream=self.compute_stream)
+            if T > 0:
+                _lib.pa_cache_write(bs.new_k[:T], bs.new_v[:T], bs.slots[:T], self.k_pool, self.v_pool, self.status,
+                                    stream=self.compute_stream)
+            _lib.pa_decode(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out, self.workspace,
+                           self.status, num_ctas=self.num_ctas, stream=self.compute_stream)
+            bs.computed.record(self.compute_stream)
+        with torch.cuda.stream(self.d2h_stream):
+            self.d2h_stream.wait_event(bs.computed)
+            bs.out_host.copy_(bs.out, non_blocking=True)
+            bs.downloaded.record(self.d2h_stream)
+        bs.used = True
+        self.steps += 1
         self.last_h2d_bytes = h2d
-        self.last_d2h_bytes = self.out.numel() * self.out.element_size()
-        return self.out_host
+        self.last_d2h_bytes = bs.out.numel() * bs.out.element_size()
+        return bs.out_host
+
+    def wait(self, result) -> None:
+        """Block until the step that returned ``result`` has been read back."""
+        for bs in self.sets:
+            if bs.out_host is result:
+                bs.downloaded.synchronize()
+                return
+        raise ValueError("not a result of this PagedDecodeStep")
+
+    def synchronize(self) -> None:
+        for s in (self.h2d_stream, self.compute_stream, self.d2h_stream):
+            s.synchronize()
 
     def device_status(self) -> int:
-        """Synchronise the step's stream and return the device status code."""
-        self.stream.synchronize()
+        """Synchronise every stream of the step and return the device status."""
+        self.synchronize()
         return int(self.status.item())
