@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
   zero_empty_outputs<kThreads, B>(p, D);
   WorkRange wr;
   Cursor cur;
-  if (!decode_prologue<kThreads, B>(p, sm.range, wr, cur)) return;  // uniform across the CTA
+  if (!decode_prologue<kThreads, B, 1>(p, sm.range, wr, cur)) return;  // uniform across the CTA
 
   if (tid == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
       __syncwarp();
     } else {
       Seg sg;
-      while (ok && next_seg<B>(cur, sg, p)) {
+      while (ok && next_seg<B, 1>(cur, sg, p)) {
         if (lane == 0) {
           ok = mbar_wait_bounded(&sm.qempty[qslot], qphase ^ 1u, abort_flag, p.wait_limit_ns);
           if (ok) {
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
     int consumed = 0, q_consumed = 0;
     bool ok = true;
     Seg sg;
-    while (ok && next_seg<B>(cur, sg, p)) {
+    while (ok && next_seg<B, 1>(cur, sg, p)) {
       // ---- q of this unit, pre-multiplied by scale*log2(e)
       ok = mbar_wait_bounded(&sm.qfull[qslot], qphase, abort_flag, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);

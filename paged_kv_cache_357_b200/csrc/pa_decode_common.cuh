@@ -2,13 +2,17 @@
 // kernel parameters, the balanced work partition over persistent CTAs, and
 // the merge of split units through the workspace.
 //
-// Work partition.  All (sequence, kv head, logical block) triples are laid
-// end to end — sequence-major, kv head next, block innermost — and cut into
-// `nparts` contiguous ranges of equal size, one per CTA, where nparts is the
-// grid size or the total block count if that is smaller (so no range is
-// empty).  A CTA's range falls into segments, one per (sequence, kv head)
-// "unit" it touches.  A unit covered by one CTA is finished there; a unit
-// split between CTAs is finished by whichever of them arrives last.
+// Work partition.  Each (sequence, kv head) "unit" is cut into granules of
+// CB consecutive logical blocks (the last one may be shorter); all granules
+// are laid end to end — sequence-major, kv head next, granule innermost —
+// and cut into `nparts` contiguous ranges of equal count, one per CTA, where
+// nparts is the grid size or the total granule count if that is smaller (so
+// no range is empty).  CB is the kernel's processing chunk (1 block for the
+// CUDA-core kernel, 8 for the tensor-core kernel), so every CTA gets the same
+// number of chunks and no range boundary splits a chunk.  A CTA's range
+// falls into segments, one per unit it touches.  A unit covered by one CTA is
+// finished there; a unit split between CTAs is finished by whichever of them
+// arrives last.
 //
 // Merge rule (study notes ch.05 §4, the online-softmax merge applied to
 // partitions): a partial state is (m, l, acc) in the log2 domain — running
@@ -50,33 +54,50 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, int B) 
 }
 
 struct Cursor {
-  int s, h, j, nb, len;
-  long long x, remaining;
+  int s, h;
+  int jg;   // next granule of unit (s, h)
+  int ng;   // granules of sequence s's units
+  int nb;   // blocks of sequence s's units
+  int len;  // tokens of sequence s
+  long long x, remaining;  // flattened granule index; granules left in the range
 };
 
 struct Seg {
-  int s, h, j0, n, nb, len;
-  long long unit_first;  // flattened index of block 0 of unit (s, h)
+  int s, h;
+  int j0, n;  // logical blocks [j0, j0 + n) of unit (s, h)
+  int nb;     // blocks of the unit
+  int ng;     // granules of the unit
+  int len;    // tokens of the sequence
+  long long unit_first;  // flattened index of the unit's granule 0
 };
 
+template <int B, int CB>
+__device__ __forceinline__ void load_seq(Cursor& c, const DecodeParams& p) {
+  c.len = checked_len(p, c.s, B);
+  c.nb = (c.len + B - 1) / B;
+  c.ng = (c.nb + CB - 1) / CB;
+}
+
 // Next segment of the CTA's range; advances the cursor past it.
-template <int B>
+template <int B, int CB>
 __device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams& p) {
   if (c.remaining <= 0) return false;
-  const long long left = c.nb - c.j;
-  const int n = static_cast<int>(left < c.remaining ? left : c.remaining);
+  const long long left = c.ng - c.jg;
+  const int k = static_cast<int>(left < c.remaining ? left : c.remaining);
   sg.s = c.s;
   sg.h = c.h;
-  sg.j0 = c.j;
-  sg.n = n;
+  sg.j0 = c.jg * CB;
+  const int j1 = (c.jg + k) * CB;
+  sg.n = (j1 < c.nb ? j1 : c.nb) - sg.j0;
   sg.nb = c.nb;
+  sg.ng = c.ng;
   sg.len = c.len;
-  sg.unit_first = c.x - c.j;
-  c.remaining -= n;
-  c.x += n;
-  c.j += n;
-  if (c.j == c.nb) {
-    c.j = 0;
+  sg.unit_first = c.x - c.jg;
+  c.remaining -= k;
+  c.x += k;
+  c.jg += k;
+  if (c.jg == c.ng) {
+    c.jg = 0;
     if (++c.h == p.num_kv_heads) {
       c.h = 0;
       if (c.remaining > 0) {
@@ -85,16 +106,15 @@ __device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams&
             c.remaining = 0;
             break;
           }
-          c.len = checked_len(p, c.s, B);
-          c.nb = (c.len + B - 1) / B;
-        } while (c.nb == 0);
+          load_seq<B, CB>(c, p);
+        } while (c.ng == 0);
       }
     }
   }
   return true;
 }
 
-// CTA whose range [c*N/C, (c+1)*N/C) holds flattened block x.
+// CTA whose range [c*N/C, (c+1)*N/C) holds flattened granule x.
 __device__ __forceinline__ long long cta_of(long long x, long long N, long long C) { return ((x + 1) * C - 1) / N; }
 
 __device__ __forceinline__ long long range_start(long long c, long long N, long long C) { return c * N / C; }
@@ -130,7 +150,7 @@ __device__ __forceinline__ long long block_inclusive_scan(long long v, RangeSmem
 }
 
 struct WorkRange {
-  long long NBT;     // total (sequence, kv head, block) triples
+  long long total;   // granules over all units
   long long nparts;  // CTAs that own a non-empty range
   long long start, end;
 };
@@ -138,7 +158,7 @@ struct WorkRange {
 // Every thread of the CTA calls this.  Writes zero outputs of empty
 // sequences (each by one CTA), computes this CTA's range and positions the
 // cursor at its first block.  Returns false when the CTA has no work.
-template <int NT, int B>
+template <int NT, int B, int CB>
 __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange& wr, Cursor& cur) {
   const int tid = threadIdx.x;
   const long long nctas = gridDim.x, cta = blockIdx.x;
@@ -151,28 +171,28 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
       if (cta == 0) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
       n = 0;
     }
-    mine += (n + B - 1) / B;
+    mine += ((n + B - 1) / B + CB - 1) / CB;
   }
-  long long seq_blocks;
-  (void)block_inclusive_scan<NT>(mine, rs, seq_blocks);
-  wr.NBT = seq_blocks * Hkv;
-  wr.nparts = wr.NBT < nctas ? wr.NBT : nctas;
-  if (cta >= wr.nparts) return false;  // uniform across the CTA (also covers NBT == 0)
-  wr.start = range_start(cta, wr.NBT, wr.nparts);
-  wr.end = range_start(cta + 1, wr.NBT, wr.nparts);
+  long long seq_granules;
+  (void)block_inclusive_scan<NT>(mine, rs, seq_granules);
+  wr.total = seq_granules * Hkv;
+  wr.nparts = wr.total < nctas ? wr.total : nctas;
+  if (cta >= wr.nparts) return false;  // uniform across the CTA (also covers total == 0)
+  wr.start = range_start(cta, wr.total, wr.nparts);
+  wr.end = range_start(cta + 1, wr.total, wr.nparts);
 
   // locate the sequence holding `start`
-  const long long target = wr.start / Hkv;  // in per-sequence block units
+  const long long target = wr.start / Hkv;  // in per-sequence granule units
   if (tid == 0) rs.found = 0;
   __syncthreads();
   long long base = 0;
   for (int chunk = 0; chunk < p.num_seqs; chunk += NT) {
     const int s = chunk + tid;
-    const long long nb = (s < p.num_seqs) ? (checked_len(p, s, B) + B - 1) / B : 0;
+    const long long ng = (s < p.num_seqs) ? ((checked_len(p, s, B) + B - 1) / B + CB - 1) / CB : 0;
     long long chunk_total;
-    const long long incl = block_inclusive_scan<NT>(nb, rs, chunk_total);
-    const long long excl = incl - nb;
-    if (nb > 0 && base + excl <= target && target < base + incl) {
+    const long long incl = block_inclusive_scan<NT>(ng, rs, chunk_total);
+    const long long excl = incl - ng;
+    if (ng > 0 && base + excl <= target && target < base + incl) {
       rs.s0 = s;
       rs.pre0 = base + excl;
       rs.found = 1;
@@ -183,11 +203,10 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
   }
   if (!rs.found) return false;  // only with lengths changing under the kernel
   cur.s = rs.s0;
-  cur.len = checked_len(p, cur.s, B);
-  cur.nb = (cur.len + B - 1) / B;
+  load_seq<B, CB>(cur, p);
   const long long off = wr.start - rs.pre0 * Hkv;
-  cur.h = static_cast<int>(off / cur.nb);
-  cur.j = static_cast<int>(off % cur.nb);
+  cur.h = static_cast<int>(off / cur.ng);
+  cur.jg = static_cast<int>(off % cur.ng);
   cur.x = wr.start;
   cur.remaining = wr.end - wr.start;
   return true;
@@ -207,10 +226,10 @@ __device__ __forceinline__ void zero_empty_outputs(const DecodeParams& p, int D)
   }
 }
 
-// Partial slot of CTA c for a unit whose block 0 is flattened index F: slot 0
+// Partial slot of CTA c for a unit whose granule 0 is flattened index F: slot 0
 // if c's range starts inside the unit, else slot 1 (the unit where it ends).
 __device__ __forceinline__ size_t partial_slot(long long c, long long F, const WorkRange& wr) {
-  const int sl = (range_start(c, wr.NBT, wr.nparts) >= F) ? 0 : 1;
+  const int sl = (range_start(c, wr.total, wr.nparts) >= F) ? 0 : 1;
   return static_cast<size_t>(c) * 2 + sl;
 }
 
@@ -223,8 +242,8 @@ __device__ void finish_split_unit(const DecodeParams& p, const Seg& sg, const Wo
                                   int nthreads, int* is_last, Sync sync) {
   constexpr int kStride = G * (D + 2);
   const long long F = sg.unit_first;
-  const long long first = cta_of(F, wr.NBT, wr.nparts);
-  const long long last = cta_of(F + sg.nb - 1, wr.NBT, wr.nparts);
+  const long long first = cta_of(F, wr.total, wr.nparts);
+  const long long last = cta_of(F + sg.ng - 1, wr.total, wr.nparts);
   int32_t* counter = p.counters + static_cast<size_t>(sg.s) * p.num_kv_heads + sg.h;
   sync();
   if (ctid == 0) {

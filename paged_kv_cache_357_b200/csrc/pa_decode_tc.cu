@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   zero_empty_outputs<kThreads, B>(p, D);
   WorkRange wr;
   Cursor cur;
-  if (!decode_prologue<kThreads, B>(p, sm.range, wr, cur)) return;  // uniform across the CTA
+  if (!decode_prologue<kThreads, B, CB>(p, sm.range, wr, cur)) return;  // uniform across the CTA
 
   if (tid == 0) {
     for (int i = 0; i < kKStages; ++i) {
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else {
       Seg sg;
-      while (ok && next_seg<B>(cur, sg, p)) {
+      while (ok && next_seg<B, CB>(cur, sg, p)) {
         const int qs = qi & 1;
         if (lane == 0) {
           ok = mbar_wait_bounded(&sm.qempty[qs], ((qi >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok) {
         bool progress = false;
         if (!walk_done && !have_seg) {
-          if (next_seg<B>(cur, sg, p)) {
+          if (next_seg<B, CB>(cur, sg, p)) {
             have_seg = true;
             c0 = 0;
           } else {
@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    while (ok && next_seg<B>(cur, sg, p)) {
+    while (ok && next_seg<B, CB>(cur, sg, p)) {
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
