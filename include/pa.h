@@ -58,7 +58,8 @@ typedef enum pa_status {
   PA_ERR_UNSUPPORTED = 2, /* no kernel for this block_size/head_dim/group/dtype */
   PA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
   PA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
-  PA_ERR_SCRATCH_LIMIT = 5 /* pa_decode_no_alloc: the batch needs more scratch than its fixed array */
+  PA_ERR_SCRATCH_LIMIT = 5, /* pa_decode_no_alloc: the batch needs more scratch than its fixed array */
+  PA_ERR_OUT_OF_BLOCKS = 6  /* block manager: not enough free blocks (nothing was changed) */
 } pa_status;
 
 /* Device-side status codes written to *dev_status (a range of their own,
@@ -224,6 +225,80 @@ PA_API pa_status pa_cache_write(const void* k, const void* v, const int64_t* slo
  */
 PA_API pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs, void* k_pool, void* v_pool,
                          int32_t* dev_status, const pa_pool_desc* pool, void* stream);
+
+/*
+ * Host block manager — the bookkeeping half of the method (study notes
+ * ch.05 §3 block table, §5 ② on-demand allocation, §6.1 sharing and copy on
+ * write, §6.2 reference counts, §12 exercise 4).  Plain C++ on the host; it
+ * produces the block tables, lengths, slot mappings and copy-on-write pairs
+ * that pa_copy_blocks / pa_cache_write / pa_decode consume.
+ *
+ * Blocks are handed out first-in first-out from a free set that starts as
+ * 0..num_blocks-1.  Sequences are named by caller-chosen int64 ids.  A
+ * manager is not thread safe.  Calls that fail return an error and change
+ * nothing.
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+typedef struct pa_bm_stats {
+  int32_t num_blocks;     /* pool size */
+  int32_t free_blocks;    /* in the free set */
+  int32_t used_blocks;    /* referenced by at least one sequence */
+  int32_t shared_blocks;  /* referenced by two or more sequences */
+  int32_t num_sequences;
+  int64_t logical_blocks; /* sum over sequences of table lengths (what unshared storage would need) */
+  int64_t tokens;         /* sum over sequences of token counts */
+  int64_t slots_filled;   /* rows of used blocks that hold a token */
+} pa_bm_stats;
+
+/* A manager over num_blocks blocks of block_size tokens; NULL on bad sizes. */
+PA_API pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size);
+PA_API void pa_bm_destroy(pa_block_manager* bm);
+
+/* Register sequence seq_id holding num_tokens tokens (its prompt):
+ * ceil(num_tokens / block_size) fresh blocks.  PA_ERR_INVALID_ARG for a
+ * known id, PA_ERR_OUT_OF_BLOCKS when the free set is too small. */
+PA_API pa_status pa_bm_add(pa_block_manager* bm, int64_t seq_id, int32_t num_tokens);
+
+/* child_id starts as a copy of parent_id's table: every block gains one
+ * reference (parallel sampling / beam search share, study notes §6.1, §6.2). */
+PA_API pa_status pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id);
+
+/* Reserve the slot of the sequence's next token: a fresh block when the
+ * last one is full; when the target block is shared, a fresh block becomes
+ * the sequence's private copy first (*cow_src, *cow_dst receive the pair,
+ * else -1; the source loses one reference).  Pointers may be NULL. */
+PA_API pa_status pa_bm_append(pa_block_manager* bm, int64_t seq_id, int64_t* slot, int64_t* cow_src,
+                              int64_t* cow_dst);
+
+/* Drop the sequence: one reference off each of its blocks; blocks that reach
+ * zero return to the end of the free set. */
+PA_API pa_status pa_bm_free(pa_block_manager* bm, int64_t seq_id);
+
+/* Free blocks, or -1 for a NULL manager. */
+PA_API int32_t pa_bm_num_free_blocks(const pa_block_manager* bm);
+/* Reference count of one physical block, or -1 if out of range. */
+PA_API int32_t pa_bm_ref_count(const pa_block_manager* bm, int32_t block);
+/* The sequence's block table (first *num_blocks entries of `blocks`) and
+ * token count.  PA_ERR_INVALID_ARG if capacity is too small (the counts are
+ * still written). */
+PA_API pa_status pa_bm_table(const pa_block_manager* bm, int64_t seq_id, int32_t* blocks, int32_t capacity,
+                             int32_t* num_blocks, int32_t* num_tokens);
+PA_API void pa_bm_get_stats(const pa_block_manager* bm, pa_bm_stats* out);
+
+/* One decode step for a batch: append one token to each of the n distinct
+ * sequences in order, then fill the arrays the kernels take —
+ *   block_tables [n][max_blocks_per_seq] (rows padded with -1),
+ *   seq_lens [n] (token counts after the append),
+ *   slot_mapping [n] (the new tokens' slots),
+ *   copy_pairs [max_pairs][2] with *num_pairs copy-on-write pairs to run
+ *   (pa_copy_blocks) before the cache write.
+ * Checks ids, table width, free blocks and pair room first; on any error
+ * nothing changes. */
+PA_API pa_status pa_bm_prepare_step(pa_block_manager* bm, const int64_t* seq_ids, int32_t n,
+                                    int32_t max_blocks_per_seq, int32_t* block_tables, int32_t* seq_lens,
+                                    int64_t* slot_mapping, int64_t* copy_pairs, int32_t max_pairs,
+                                    int32_t* num_pairs);
 
 /* Static string for a pa_status or PA_DEV_* code. */
 PA_API const char* pa_status_string(int32_t status);

@@ -7,6 +7,7 @@ The kernels live in ``libpa.so`` (C ABI: ``include/pa.h``), built in-tree by
 * ``pa_cache_write``  slot-mapped write of new tokens' K/V
 * ``pa_copy_blocks``  copy-on-write block copies
 * ``PagedDecodeStep`` one whole step (copy, write, decode) from host buffers
+* ``BlockManager``    host block manager (free set, ref counts, copy on write)
 
 PyTorch supplies device memory and streams only.
 """
@@ -32,4 +33,5 @@ from ._lib import (  # noqa: F401
     pool_desc,
     status_string,
 )
+from .block_manager import BlockManager  # noqa: F401
 from .step import PagedDecodeStep  # noqa: F401

@@ -36,6 +36,17 @@ EXPORTED = (
     "pa_cache_write",
     "pa_copy_blocks",
     "pa_status_string",
+    "pa_bm_create",
+    "pa_bm_destroy",
+    "pa_bm_add",
+    "pa_bm_fork",
+    "pa_bm_append",
+    "pa_bm_free",
+    "pa_bm_num_free_blocks",
+    "pa_bm_ref_count",
+    "pa_bm_table",
+    "pa_bm_get_stats",
+    "pa_bm_prepare_step",
 )
 
 

@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
   const long long cta = blockIdx.x;
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
 
+  grid_dependency_wait();
+  grid_launch_dependents();
   zero_empty_outputs<kThreads, B>(p, D);
   WorkRange wr;
   Cursor cur;
@@ -430,8 +432,8 @@ __global__ void __launch_bounds__(kThreads) pa_decode_kernel(const DecodeParams 
 
 template <bool kBf16, int D, int B, int G>
 static cudaError_t launch_cuda_cores(const Variant& v, const DecodeParams& prm, int ctas, cudaStream_t stream) {
-  pa_decode_kernel<kBf16, D, B, G><<<ctas, kThreads, v.smem_bytes, stream>>>(prm);
-  return cudaGetLastError();
+  return launch_overlapped(pa_decode_kernel<kBf16, D, B, G>, dim3(ctas), dim3(kThreads),
+                           static_cast<size_t>(v.smem_bytes), stream, prm);
 }
 
 template <bool kBf16, int D, int B, int G>

@@ -208,11 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long cta = blockIdx.x;
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
 
-  zero_empty_outputs<kThreads, B>(p, D);
-  WorkRange wr;
-  Cursor cur;
-  if (!decode_prologue<kThreads, B, CB>(p, sm.range, wr, cur)) return;  // uniform across the CTA
-
+  // ---- set-up that reads no input (barriers, TMEM, tensor-map prefetch);
+  // with programmatic dependent launch it overlaps the previous kernel
   if (tid == 0) {
     for (int i = 0; i < kKStages; ++i) {
       mbar_init(&sm.kfull[i], 1);
@@ -245,6 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  if (tid == 0) {
+    prefetch_tensormap(&map_q);
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_v);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -252,17 +254,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const volatile int* abort_flag = &sm.abort;
   constexpr uint32_t kColS = 0, kColO = 32;
 
-  if (warp == 0) {
+  // ---- inputs may come from the previous kernel in the stream
+  grid_dependency_wait();
+  grid_launch_dependents();
+  zero_empty_outputs<kThreads, B>(p, D);
+  WorkRange wr;
+  Cursor cur;
+  const bool has_work = decode_prologue<kThreads, B, CB>(p, sm.range, wr, cur);  // uniform across the CTA
+
+  if (!has_work) {
+    // nothing to stream: straight to teardown
+  } else if (warp == 0) {
     // ===================== producer =========================================
     const uint64_t pol_stream = l2_policy_evict_first();
     const uint64_t pol_keep = l2_policy_evict_last();
     bool ok = true;
     int ci = 0, qi = 0, k_issued = 0, v_issued = 0, q_issued = 0;
-    if (lane == 0) {
-      prefetch_tensormap(&map_q);
-      prefetch_tensormap(&map_k);
-      prefetch_tensormap(&map_v);
-    }
     if (p.test_flags & kFlagTestWithholdCopies) {
       if (lane == 0) {
         const uint64_t t0 = global_timer_ns();
@@ -671,8 +678,8 @@ static cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas
       !make_map(&mv, prm.v_pool, kv_rows, kBf16, B)) {
     return cudaErrorInvalidValue;
   }
-  pa_decode_tc_kernel<kBf16, G><<<ctas, kThreads, v.smem_bytes, stream>>>(prm, mq, mk, mv);
-  return cudaGetLastError();
+  return launch_overlapped(pa_decode_tc_kernel<kBf16, G>, dim3(ctas), dim3(kThreads),
+                           static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
 }
 
 template <bool kBf16, int G>

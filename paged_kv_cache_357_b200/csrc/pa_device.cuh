@@ -114,6 +114,14 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   return pol;
 }
 
+// Programmatic dependent launch: wait until the previous kernel in the
+// stream has completed and its writes are visible (a no-op when the kernel
+// was launched without the attribute), and let the next kernel start its
+// own set-up early.  Every libpa kernel waits before reading any input.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

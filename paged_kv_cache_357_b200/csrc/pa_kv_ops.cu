@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(kCopyThreads)
     cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, const int64_t* __restrict__ slots,
                        long long total_chunks, int Hkv, int chunks_per_row, int B, long long num_slots,
                        uint4* __restrict__ k_pool, uint4* __restrict__ v_pool, int32_t* status) {
+  grid_dependency_wait();
+  grid_launch_dependents();
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks; i += stride) {
     const int chunk = static_cast<int>(i % chunks_per_row);
@@ -45,6 +47,8 @@ __global__ void __launch_bounds__(kCopyThreads)
 __global__ void __launch_bounds__(kCopyThreads)
     copy_blocks_kernel(const int64_t* __restrict__ pairs, long long total_chunks, long long chunks_per_block,
                        long long num_blocks, uint4* k_pool, uint4* v_pool, int32_t* status) {
+  grid_dependency_wait();
+  grid_launch_dependents();
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks; i += stride) {
     const long long chunk = i % chunks_per_block;
@@ -89,10 +93,11 @@ extern "C" pa_status pa_cache_write(const void* k, const void* v, const int64_t*
   const int cpr = pool->head_dim / 8;
   const long long total = static_cast<long long>(num_tokens) * pool->num_kv_heads * cpr;
   const long long num_slots = static_cast<long long>(pool->num_blocks) * pool->block_size;
-  cache_write_kernel<<<copy_grid(total), kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+  const cudaError_t e = launch_overlapped(
+      cache_write_kernel, dim3(copy_grid(total)), dim3(kCopyThreads), 0, static_cast<cudaStream_t>(stream),
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, total, pool->num_kv_heads, cpr,
       pool->block_size, num_slots, static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), dev_status);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs, void* k_pool, void* v_pool,
@@ -103,10 +108,11 @@ extern "C" pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pa
   if (!aligned16(k_pool) || !aligned16(v_pool)) return PA_ERR_INVALID_ARG;
   const long long cpb = static_cast<long long>(pool->num_kv_heads) * pool->block_size * pool->head_dim / 8;
   const long long total = static_cast<long long>(num_pairs) * 2 * cpb;
-  copy_blocks_kernel<<<copy_grid(total), kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      src_dst_pairs, total, cpb, pool->num_blocks, static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool),
-      dev_status);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = launch_overlapped(copy_blocks_kernel, dim3(copy_grid(total)), dim3(kCopyThreads), 0,
+                                          static_cast<cudaStream_t>(stream), src_dst_pairs, total, cpb,
+                                          static_cast<long long>(pool->num_blocks), static_cast<uint4*>(k_pool),
+                                          static_cast<uint4*>(v_pool), dev_status);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" const char* pa_status_string(int32_t status) {
@@ -117,6 +123,7 @@ extern "C" const char* pa_status_string(int32_t status) {
     case PA_ERR_WORKSPACE: return "workspace missing or too small";
     case PA_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
     case PA_ERR_SCRATCH_LIMIT: return "batch needs more scratch than pa_decode_no_alloc's fixed array";
+    case PA_ERR_OUT_OF_BLOCKS: return "block manager: not enough free blocks";
     case PA_DEV_BAD_BLOCK_ID: return "device: block table entry outside [0, num_blocks)";
     case PA_DEV_BAD_SEQ_LEN: return "device: seq_len negative or beyond the block table";
     case PA_DEV_BAD_SLOT: return "device: slot_mapping entry beyond the pool";

@@ -49,7 +49,7 @@ def test_library_exports_nothing_else(lib):
 
 
 def test_status_strings(lib):
-    for code in [0, 1, 2, 3, 4, 5, 101, 102, 103, 104, 105]:
+    for code in [0, 1, 2, 3, 4, 5, 6, 101, 102, 103, 104, 105]:
         assert pa.status_string(code) != "unknown status"
     assert pa.status_string(12345) == "unknown status"
 
