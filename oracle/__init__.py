@@ -29,6 +29,7 @@ from .paged_attention import (  # noqa: F401
     attention_dense,
     decode,
     decode_one,
+    decode_multi,
     decode_blockwise_online,
     partition_states,
     merge_partition_states,

@@ -82,6 +82,38 @@ def decode(q, k_pool, v_pool, block_tables, seq_lens, scale: float, num_kv_heads
     return out
 
 
+def decode_multi(q, k_pool, v_pool, block_tables, seq_lens, scale: float, num_kv_heads: int,
+                 dtype: str) -> np.ndarray:
+    """Attention of q_len new query positions per sequence over the paged
+    cache, causal among them (the speculative-decoding and chunked-prefill
+    items of the CSDN article's "2026年最新进展" list; the attention itself is
+    the vLLM blog's §"关键细节" 2 definition).  q is [S, q_len, Hq, D] bits;
+    seq_lens counts every cached token including the q_len new ones, so
+    position i sees tokens 0 .. seq_lens[s] - q_len + i.  Computed as one
+    masked score matrix per (sequence, head): Z = scale * Q K^T, entries past a
+    row's limit removed, softmax along each row, times V.  A sequence with
+    fewer than q_len tokens gives zeros.  Returns [S, q_len, Hq, D] float64."""
+    S, L, Hq, D = q.shape
+    g = Hq // num_kv_heads
+    B = k_pool.shape[2]
+    out = np.zeros((S, L, Hq, D), dtype=np.float64)
+    for s in range(S):
+        n = int(seq_lens[s])
+        if n < L:
+            continue
+        limit = n - L + np.arange(L)                        # last visible token of each row
+        visible = np.arange(n)[None, :] <= limit[:, None]   # [L, n]
+        for h in range(Hq):
+            K = bits_to_f64(gather_kv(k_pool, block_tables[s], n, h // g, B), dtype)
+            V = bits_to_f64(gather_kv(v_pool, block_tables[s], n, h // g, B), dtype)
+            Z = scale * (bits_to_f64(q[s, :, h], dtype) @ K.T)  # [L, n]
+            Z = np.where(visible, Z, -np.inf)
+            Z = Z - Z.max(axis=1, keepdims=True)
+            W = np.exp(Z)
+            out[s, :, h] = (W / W.sum(axis=1, keepdims=True)) @ V
+    return out
+
+
 def decode_blockwise_online(s: int, h: int, q, k_pool, v_pool, block_tables, seq_lens, scale: float,
                             num_kv_heads: int, dtype: str) -> np.ndarray:
     """The same output computed the way the study notes ch.05 §4 describe it:
