@@ -70,6 +70,7 @@ typedef enum pa_status {
 #define PA_DEV_BAD_SLOT 103    /* slot_mapping entry >= num_blocks * block_size */
 #define PA_DEV_BAD_PAIR 104    /* copy pair with src or dst outside [0, num_blocks) */
 #define PA_DEV_TIMEOUT 105     /* a bounded pipeline wait ran out (kernel returned early) */
+#define PA_DEV_BAD_GROUP 106   /* shared-prefix groups do not partition the sequences, or one is too large */
 
 typedef enum pa_dtype { PA_FP16 = 0, PA_BF16 = 1 } pa_dtype;
 
@@ -194,6 +195,78 @@ PA_API pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const voi
                                     int32_t* dev_status, const pa_pool_desc* pool, void* stream);
 
 /*
+ * pa_decode_multi — paged attention for q_len new query positions per
+ * sequence, causal among them: verifying q_len speculated tokens, or a
+ * short prefill chunk (CSDN "PagedAttention：分页注意力", §"2026年最新进展"
+ * items 1-2: speculative decoding and chunked prefill on the paged cache).
+ * The pages give no formula beyond decode's; the plain reading used here is
+ * causal attention of the new positions over the cache that already holds
+ * them:
+ *   out[s][i][h] = sum_t softmax_t(scale * q[s][i][h] . K_t) V_t,
+ *                  t = 0 .. seq_lens[s] - q_len + i,   i = 0 .. q_len-1,
+ * with K_t / V_t found through block_tables exactly as in pa_decode (the
+ * q_len new tokens must already be in the cache: pa_cache_write first).
+ *   q, out   [num_seqs][q_len][num_q_heads][head_dim]
+ *   others   as pa_decode
+ * q_len == 1 is pa_decode.  For q_len >= 2 the tensor-core kernel runs:
+ * head_dim 128, block_size 16, group size G = num_q_heads / num_kv_heads in
+ * {1, 2, 4, 8} and G * q_len <= 32 (G * q_len rounded up to a power of two);
+ * other shapes return PA_ERR_UNSUPPORTED, as does PA_DECODE_CUDA_CORES_ONLY.
+ * A sequence with seq_lens[s] == 0 gets zero outputs; 0 < seq_lens[s] <
+ * q_len is PA_DEV_BAD_SEQ_LEN (zero outputs).  Workspace: as pa_decode, sized
+ * by pa_decode_multi_workspace_bytes (0 for invalid or unsupported shapes).
+ */
+PA_API size_t pa_decode_multi_workspace_bytes(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                              const pa_pool_desc* pool, const pa_decode_opts* opts);
+PA_API pa_status pa_decode_multi(const void* q, const void* k_pool, const void* v_pool,
+                                 const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                 int32_t num_seqs, int32_t q_len, int32_t num_q_heads, float scale, void* out,
+                                 void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                 const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream);
+
+/*
+ * pa_decode_shared_prefix — pa_decode for batches in which groups of
+ * sequences share their leading blocks (parallel samples or beams of one
+ * prompt, study notes ch.05 §6.1; requests with a cached common prefix,
+ * "vLLM 是什么" §3 Prefix Caching).  Same result as pa_decode (within the
+ * decode tolerance), but each shared block is read from memory once per
+ * group instead of once per member.
+ *
+ * Groups are consecutive sequences: group g holds sequences
+ * [group_starts[g], group_starts[g+1]), and its first group_prefix_blocks[g]
+ * logical blocks are the same physical blocks for every member (as
+ * pa_bm_fork leaves them); the kernel reads them through the first member's
+ * table row and ignores the other members' entries for those blocks.
+ *   group_starts         int32 device [num_groups + 1], group_starts[0] == 0,
+ *                        non-decreasing, group_starts[num_groups] == num_seqs
+ *   group_prefix_blocks  int32 device [num_groups]
+ *   max_group_size       host bound on members per group, >= 1
+ * A group shares nothing (its members are decoded one by one) when its
+ * prefix is 0, or not shorter than every member's block count.
+ * Two launches on `stream`: a prefix pass over (group, kv head) units that
+ * leaves each member's online-softmax state in the workspace, then a pass
+ * over each sequence's own blocks that merges with that state.  Tensor-core
+ * kernel only: head_dim 128, block_size 16, G in {1, 2, 4, 8} and
+ * G * max_group_size <= 32 (rounded up to a power of two), else
+ * PA_ERR_UNSUPPORTED.  Device errors: those of pa_decode, and
+ * PA_DEV_BAD_GROUP when the groups do not partition the sequences (outputs
+ * then unspecified) or a group has more members than max_group_size rounded
+ * up to a power of two (that group is then decoded without sharing).  The
+ * workspace (pa_decode_shared_prefix_workspace_bytes; zeroed before first
+ * use, as for pa_decode) also holds the per-member prefix states.
+ */
+PA_API size_t pa_decode_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t max_group_size,
+                                                      int32_t num_q_heads, const pa_pool_desc* pool,
+                                                      const pa_decode_opts* opts);
+PA_API pa_status pa_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
+                                         const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                         const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                                         const int32_t* group_starts, const int32_t* group_prefix_blocks,
+                                         int32_t num_groups, int32_t max_group_size, float scale, void* out,
+                                         void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                         const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream);
+
+/*
  * pa_cache_write — store the K/V of new tokens into their slots
  * (vLLM blog, plain-language section: each generated token's K/V is
  * written to the cache;
@@ -299,6 +372,21 @@ PA_API pa_status pa_bm_prepare_step(pa_block_manager* bm, const int64_t* seq_ids
                                     int32_t max_blocks_per_seq, int32_t* block_tables, int32_t* seq_lens,
                                     int64_t* slot_mapping, int64_t* copy_pairs, int32_t max_pairs,
                                     int32_t* num_pairs);
+
+/* Plan the groups of pa_decode_shared_prefix from HOST copies of one step's
+ * block tables and lengths (the layout pa_bm_prepare_step writes).
+ * Consecutive sequences whose first table entries are the same physical
+ * block form a group of at most max_group_size members; the group's prefix is
+ * the number of leading entries that every member has in common with the
+ * first one, capped so that each member keeps at least one block of its own
+ * (a group of one, or a prefix under min_prefix_blocks, gets 0: no sharing).
+ * Writes group_starts [*num_groups + 1] and group_prefix_blocks [*num_groups]
+ * (room for num_seqs + 1 and num_seqs entries).  Sequences of length 0 or
+ * with an invalid length are groups of one. */
+PA_API pa_status pa_shared_prefix_groups(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                         const int32_t* seq_lens, int32_t num_seqs, int32_t block_size,
+                                         int32_t max_group_size, int32_t min_prefix_blocks, int32_t* group_starts,
+                                         int32_t* group_prefix_blocks, int32_t* num_groups);
 
 /* Static string for a pa_status or PA_DEV_* code. */
 PA_API const char* pa_status_string(int32_t status);

@@ -4,6 +4,9 @@ The kernels live in ``libpa.so`` (C ABI: ``include/pa.h``), built in-tree by
 ``python -m paged_kv_cache_357_b200.build``.  This package is a thin binding:
 
 * ``pa_decode``       paged decode attention with online softmax
+* ``pa_decode_multi`` q_len causal query positions per sequence (speculative
+                      verification, prefill chunks)
+* ``pa_decode_shared_prefix``  decode reading shared prompt blocks once per group
 * ``pa_cache_write``  slot-mapped write of new tokens' K/V
 * ``pa_copy_blocks``  copy-on-write block copies
 * ``PagedDecodeStep`` one whole step (copy, write, decode) from host buffers
@@ -24,7 +27,14 @@ from ._lib import (  # noqa: F401
     PaError,
     PoolDesc,
     alloc_decode_workspace,
+    alloc_multi_workspace,
+    alloc_shared_prefix_workspace,
     decode_workspace_bytes,
+    multi_workspace_bytes,
+    shared_prefix_workspace_bytes,
+    shared_prefix_groups,
+    pa_decode_multi,
+    pa_decode_shared_prefix,
     load,
     pa_cache_write,
     pa_copy_blocks,

@@ -26,6 +26,7 @@ DEV_STATUS = {
     103: "PA_DEV_BAD_SLOT",
     104: "PA_DEV_BAD_PAIR",
     105: "PA_DEV_TIMEOUT",
+    106: "PA_DEV_BAD_GROUP",
 }
 EXPORTED = (
     "pa_decode_workspace_bytes",
@@ -33,6 +34,11 @@ EXPORTED = (
     "pa_decode",
     "pa_decode_ex",
     "pa_decode_no_alloc",
+    "pa_decode_multi_workspace_bytes",
+    "pa_decode_multi",
+    "pa_decode_shared_prefix_workspace_bytes",
+    "pa_decode_shared_prefix",
+    "pa_shared_prefix_groups",
     "pa_cache_write",
     "pa_copy_blocks",
     "pa_status_string",
@@ -96,6 +102,17 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_ex.restype = i32
     lib.pa_decode_no_alloc.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, f32, vp, vp, pdesc, vp]
     lib.pa_decode_no_alloc.restype = i32
+    lib.pa_decode_multi_workspace_bytes.argtypes = [i32, i32, i32, pdesc, popts]
+    lib.pa_decode_multi_workspace_bytes.restype = sz
+    lib.pa_decode_multi.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp, pdesc, popts, vp]
+    lib.pa_decode_multi.restype = i32
+    lib.pa_decode_shared_prefix_workspace_bytes.argtypes = [i32, i32, i32, pdesc, popts]
+    lib.pa_decode_shared_prefix_workspace_bytes.restype = sz
+    lib.pa_decode_shared_prefix.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, vp, vp, i32, i32, f32, vp, vp, sz,
+                                            vp, pdesc, popts, vp]
+    lib.pa_decode_shared_prefix.restype = i32
+    lib.pa_shared_prefix_groups.argtypes = [vp, i32, vp, i32, i32, i32, i32, vp, vp, vp]
+    lib.pa_shared_prefix_groups.restype = i32
     lib.pa_cache_write.argtypes = [vp, vp, vp, i32, vp, vp, vp, pdesc, vp]
     lib.pa_cache_write.restype = i32
     lib.pa_copy_blocks.argtypes = [vp, i32, vp, vp, vp, pdesc, vp]
@@ -212,6 +229,135 @@ def pa_decode(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, work
     )
     if rc != 0:
         raise PaError(rc, "pa_decode")
+
+
+def _check_attention_args(q, k_pool, v_pool, block_tables, seq_lens, out, workspace, dev_status, q_ndim):
+    torch = _torch()
+    _need(k_pool, "k_pool", ndim=4)
+    dev = k_pool.device
+    _need(v_pool, "v_pool", dtype=k_pool.dtype, ndim=4, device=dev)
+    if v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool and v_pool shapes differ")
+    _need(q, "q", dtype=k_pool.dtype, ndim=q_ndim, device=dev)
+    _need(out, "out", dtype=k_pool.dtype, ndim=q_ndim, device=dev)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2, device=dev)
+    _need(seq_lens, "seq_lens", dtype=torch.int32, ndim=1, device=dev)
+    _need(workspace, "workspace", device=dev)
+    S = q.shape[0]
+    if block_tables.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_tables / seq_lens must have num_seqs rows")
+    if q.shape[-1] != k_pool.shape[3]:
+        raise ValueError("head_dim of q and the pools differ")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", dtype=torch.int32, device=dev)
+
+
+def multi_workspace_bytes(num_seqs: int, q_len: int, num_q_heads: int, k_pool, num_ctas: int = 0,
+                          flags: int = 0) -> int:
+    """Workspace bytes for pa_decode_multi with the same num_ctas and flags."""
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    n = load().pa_decode_multi_workspace_bytes(num_seqs, q_len, num_q_heads, ctypes.byref(desc),
+                                               ctypes.byref(opts))
+    if n == 0:
+        raise PaError(2, "pa_decode_multi_workspace_bytes")
+    return int(n)
+
+
+def alloc_multi_workspace(num_seqs: int, q_len: int, num_q_heads: int, k_pool, num_ctas: int = 0, flags: int = 0):
+    """Zeroed device workspace for pa_decode_multi."""
+    torch = _torch()
+    n = multi_workspace_bytes(num_seqs, q_len, num_q_heads, k_pool, num_ctas, flags)
+    return torch.zeros(n, dtype=torch.uint8, device=k_pool.device)
+
+
+def pa_decode_multi(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, workspace, dev_status=None,
+                    num_ctas: int = 0, flags: int = 0, stream=None) -> None:
+    """Causal attention of q_len new positions per sequence over the paged
+    cache (pa_decode_multi): q, out are [num_seqs, q_len, num_q_heads, head_dim]."""
+    _check_attention_args(q, k_pool, v_pool, block_tables, seq_lens, out, workspace, dev_status, 4)
+    S, L, Hq, D = q.shape
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    rc = load().pa_decode_multi(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), S, L, Hq,
+        float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+        ctypes.byref(desc), ctypes.byref(opts), _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode_multi")
+
+
+def shared_prefix_workspace_bytes(num_seqs: int, max_group_size: int, num_q_heads: int, k_pool, num_ctas: int = 0,
+                                  flags: int = 0) -> int:
+    """Workspace bytes for pa_decode_shared_prefix with the same num_ctas and flags."""
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    n = load().pa_decode_shared_prefix_workspace_bytes(num_seqs, max_group_size, num_q_heads, ctypes.byref(desc),
+                                                       ctypes.byref(opts))
+    if n == 0:
+        raise PaError(2, "pa_decode_shared_prefix_workspace_bytes")
+    return int(n)
+
+
+def alloc_shared_prefix_workspace(num_seqs: int, max_group_size: int, num_q_heads: int, k_pool, num_ctas: int = 0,
+                                  flags: int = 0):
+    """Zeroed device workspace for pa_decode_shared_prefix."""
+    torch = _torch()
+    n = shared_prefix_workspace_bytes(num_seqs, max_group_size, num_q_heads, k_pool, num_ctas, flags)
+    return torch.zeros(n, dtype=torch.uint8, device=k_pool.device)
+
+
+def pa_decode_shared_prefix(q, k_pool, v_pool, block_tables, seq_lens, group_starts, group_prefix_blocks,
+                            max_group_size: int, scale: float, out, workspace, dev_status=None, num_ctas: int = 0,
+                            flags: int = 0, stream=None) -> None:
+    """pa_decode reading each group's shared leading blocks once
+    (pa_decode_shared_prefix); group_starts [G + 1] and group_prefix_blocks [G]
+    are int32 device tensors (see shared_prefix_groups)."""
+    torch = _torch()
+    _check_attention_args(q, k_pool, v_pool, block_tables, seq_lens, out, workspace, dev_status, 3)
+    dev = k_pool.device
+    _need(group_starts, "group_starts", dtype=torch.int32, ndim=1, device=dev)
+    _need(group_prefix_blocks, "group_prefix_blocks", dtype=torch.int32, ndim=1, device=dev)
+    G = group_prefix_blocks.shape[0]
+    if group_starts.shape[0] != G + 1:
+        raise ValueError("group_starts must have num_groups + 1 entries")
+    S, Hq, D = q.shape
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    rc = load().pa_decode_shared_prefix(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), S, Hq,
+        _ptr(group_starts), _ptr(group_prefix_blocks), G, int(max_group_size), float(scale), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), ctypes.byref(desc),
+        ctypes.byref(opts), _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode_shared_prefix")
+
+
+def shared_prefix_groups(block_tables, seq_lens, block_size: int, max_group_size: int, min_prefix_blocks: int = 1):
+    """Groups for pa_decode_shared_prefix from host (numpy int32) tables and
+    lengths (pa_shared_prefix_groups): returns (group_starts, group_prefix_blocks)."""
+    import numpy as np
+
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    if bt.ndim != 2 or sl.ndim != 1 or bt.shape[0] != sl.shape[0]:
+        raise ValueError("block_tables [S, max_nb] and seq_lens [S] expected")
+    S = bt.shape[0]
+    starts = np.zeros(S + 1, np.int32)
+    prefix = np.zeros(max(S, 1), np.int32)
+    ng = ctypes.c_int32(0)
+    rc = load().pa_shared_prefix_groups(
+        bt.ctypes.data, bt.shape[1], sl.ctypes.data, S, block_size, max_group_size, min_prefix_blocks,
+        starts.ctypes.data, prefix.ctypes.data, ctypes.byref(ng),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_shared_prefix_groups")
+    n = ng.value
+    return starts[: n + 1].copy(), prefix[:n].copy()
 
 
 def pa_decode_no_alloc(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, dev_status=None,

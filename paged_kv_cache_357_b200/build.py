@@ -21,8 +21,15 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libpa.so")
-SOURCES = ["pa_decode.cu", "pa_decode_tc.cu", "pa_kv_ops.cu", "pa_block_manager.cpp"]
-HEADERS = ["pa_device.cuh", "pa_internal.h", "pa_decode_common.cuh", "pa_decode_host.h"]
+SOURCES = [
+    "pa_decode.cu",
+    "pa_decode_tc.cu",
+    "pa_attn_tc_multi.cu",
+    "pa_attn_tc_prefix.cu",
+    "pa_kv_ops.cu",
+    "pa_block_manager.cpp",
+]
+HEADERS = ["pa_device.cuh", "pa_internal.h", "pa_decode_common.cuh", "pa_decode_host.h", "pa_attn_tc.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON_FLAGS = ARCH_FLAGS + [

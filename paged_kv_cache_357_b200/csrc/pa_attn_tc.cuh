@@ -1,0 +1,1006 @@
+// Paged attention on tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// What it computes (vLLM blog §"关键细节" 2; PagedAttention study notes
+// ch.05 §4): softmax(scale * q K^T) V over a sequence's paged tokens, the
+// normalisation merged across blocks with a running max and sum.  A unit
+// pairs one kv head with R query rows, which makes both products real (if
+// thin) matrix products:
+//
+//   S^T[token, row] = K_chunk[token, :] . Q^T[:, row]       (M=128, N=16|32, K=128)
+//   O^T[d, row]     = V_chunk^T[d, token] . P^T[token, row] (M=128, N=16|32, K=16 per step)
+//
+// The rows are R = G x RG: the G query heads that share the kv head (GQA),
+// times RG row groups; N is R rounded up to 16.  Three kinds of unit (kMode):
+//   kDecode  one sequence, RG = 1: the decode step.  With per-sequence prefix
+//            lengths given, only the blocks past the prefix are read and the
+//            result is merged with the prefix's state from a kPrefix launch.
+//   kMulti   one sequence, RG >= q_len new query positions, position i seeing
+//            the tokens up to seq_len - q_len + i (causal): speculative
+//            verification and prefill chunks (CSDN "PagedAttention：分页注意力",
+//            §"2026年最新进展" items 1-2).
+//   kPrefix  a group of up to RG sequences whose leading blocks are the same
+//            physical blocks (parallel samples of one prompt, study notes
+//            §6.1; prefix caching, "vLLM 是什么" §3): the shared blocks are read
+//            once for every member's rows, and each row's state (max, sum,
+//            unnormalised output) is stored for the kDecode pass.
+//
+// Work partition and split-unit merge: pa_decode_common.cuh (equal counts of
+// 8-block chunks per persistent CTA).
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      producer: resolves block ids (32 table entries per load, one
+//               batch ahead), issues 2-D TMA loads of the K and V tiles
+//               (64-column boxes, 128-byte swizzle) into separate rings of
+//               32 KB chunk stages — K released when its QK is done, V when
+//               its PV is done — and a 3-D TMA load of the unit's q rows.
+//   warp 1      allocates TMEM; lane 0 issues every tcgen05.mma and
+//               tcgen05.commit, polling which of QK(next) and PV(oldest
+//               pending) is ready and issuing it.
+//   warps 2-5   softmax + epilogue, one TMEM lane (token row, then head_dim
+//               index) per thread: read S^T from TMEM, column maxima and sums
+//               by warp butterfly reduce-scatters, write P^T (bf16/fp16) into
+//               a swizzled buffer, zero V rows past the sequence end inside
+//               the last 16-token step, then read O^T and rescale-accumulate.
+//               The epilogue of chunk i runs after the softmax of chunk i+1.
+// The swizzled layouts written by TMA serve both products directly: the K
+// tile is a K-major A operand for QK, the V tile an MN-major A operand for PV.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pa_decode_host.h"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace tc {
+
+constexpr int D = 128;
+constexpr int B = 16;
+constexpr int kChunkTok = 128;             // tokens per chunk = MMA M of QK
+constexpr int CB = kChunkTok / B;          // blocks per chunk
+constexpr int kKStages = 2;                // K is released as soon as its QK completes
+constexpr int kRowBytes = 128;             // one swizzle row: 64 elements
+constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 tokens
+constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
+constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+constexpr int kSoftmaxBarrier = 1;
+
+enum Mode { kDecode = 0, kMulti = 1, kPrefix = 2 };
+
+// Shapes that follow from the number of query rows R of a unit.
+template <int R>
+struct Rows {
+  static_assert(R >= 1 && R <= 32 && (R & (R - 1)) == 0, "R is a power of two up to 32");
+  static constexpr int N = R < 16 ? 16 : R;                       // MMA N
+  static constexpr int kVStages = N == 32 ? 3 : 4;                // V is held until its PV completes
+  static constexpr int kSlotBytes = 2 * N * kRowBytes;            // a q or P slot: two 64-column halves
+  static constexpr uint32_t kTmemCols = 4 * N <= 64 ? 64 : 128;   // S[0], S[1], O[0], O[1]
+  static constexpr int kPartStride = R * (D + 2);                 // floats per partial slot
+  static constexpr int kLanesPerCol = 32 / R;                     // lanes holding one column after a reduce
+};
+
+template <int R>
+struct TcSmem {
+  using S = Rows<R>;
+  uint8_t kbuf[kKStages][kOperandBytes];  // 1024-aligned regions
+  uint8_t vbuf[S::kVStages][kOperandBytes];
+  uint8_t q[2][S::kSlotBytes];
+  uint8_t p[2][S::kSlotBytes];
+  float red[2][4][R];  // per-warp column maxima, double-buffered by chunk
+  float mbuf[2][R];    // running max after each chunk
+  float abuf[2][R];    // rescale factor of each chunk's running output
+  float lred[4][R];    // per-warp column sums at the end of a segment
+  uint64_t kfull[kKStages];
+  uint64_t kempty[kKStages];
+  uint64_t vfull[S::kVStages];
+  uint64_t vempty[S::kVStages];
+  uint64_t qfull[2];
+  uint64_t qempty[2];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t o_free[2];
+  uint64_t mma_done;
+  RangeSmem range;
+  uint32_t tmem_base;
+  int abort;
+  int is_last;
+  int k_issued;
+  int k_consumed;
+  int v_issued;
+  int v_consumed;
+  int q_issued;
+  int q_consumed;
+};
+
+template <int R>
+constexpr int smem_bytes() {
+  return static_cast<int>(sizeof(TcSmem<R>)) + 1024;  // + alignment slack
+}
+
+// ---- tcgen05 / TMA primitives ------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] . B[smem desc], kind::f16, fp32 accumulate.
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  setp.ne.b32 p, %4, 0;\n"
+      "  tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+      "}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05.mma issued so far by this thread completes.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane (completion is
+// waited for separately, so several loads can be in flight).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Columns [0, NC) of this thread's TMEM lane, NC a multiple of 16.
+template <int NC>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float* v) {
+  uint32_t r[NC];
+#pragma unroll
+  for (int c = 0; c < NC; c += 16) tmem_ld16_nowait(taddr + c, r + c);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < NC; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version 1.
+// lbo/sbo in bytes: lbo = distance between 64-element column groups of an
+// MN-major operand (unused for K-major), sbo = distance between 8-row groups.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulate, A/B both bf16 or both
+// fp16, B K-major, A K-major (QK) or MN-major (PV), M = 128, N = n.
+__host__ __device__ constexpr uint32_t make_idesc(bool bf16, bool a_mn_major, int n) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// Reduce R values per lane over the warp by a butterfly reduce-scatter:
+// afterwards lane l holds, for column l / (32 / R), the max (kMax) or sum of
+// that column over all 32 lanes.  R - 1 + log2(32 / R) shuffles in all,
+// instead of 5 per column.
+template <int R, bool kMax>
+__device__ __forceinline__ float warp_column_reduce(float (&v)[R], int lane) {
+#pragma unroll
+  for (int half = R / 2, o = 16; half >= 1; half /= 2, o /= 2) {
+    const bool upper = (lane & o) != 0;  // keeps columns [half, 2 half) of what it holds
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float send = upper ? v[k] : v[k + half];
+      const float keep = upper ? v[k + half] : v[k];
+      const float got = __shfl_xor_sync(0xffffffffu, send, o);
+      v[k] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int o = 16 / R; o >= 1; o /= 2) {
+    const float got = __shfl_xor_sync(0xffffffffu, r, o);
+    r = kMax ? fmaxf(r, got) : r + got;
+  }
+  return r;
+}
+
+struct ChunkInfo {
+  int j;     // first logical block of the chunk
+  int nblk;  // blocks in the chunk
+  int ntok;  // valid tokens in the chunk
+};
+
+__device__ __forceinline__ ChunkInfo chunk_at(const Seg& sg, int c0) {
+  ChunkInfo c;
+  c.j = sg.j0 + c0;
+  c.nblk = min(CB, sg.n - c0);
+  c.ntok = min(c.nblk * B, sg.len - c.j * B);
+  return c;
+}
+
+// ---- what a unit covers: blocks, table row, q rows -------------------------
+
+template <int kMode, int RG>
+struct Source;
+
+// A sequence: all its blocks, or those past its shared prefix when
+// per-sequence prefix lengths are given.
+template <int RG>
+struct Source<kDecode, RG> {
+  template <int BB>
+  __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int s) const {
+    const int len = checked_len(p, s, BB);
+    const int nb = (len + BB - 1) / BB;
+    int first = 0;
+    if (p.seq_prefix != nullptr) {
+      const int f = __ldcg(p.seq_prefix + s);  // written by the previous launch
+      first = (f > 0 && f < nb) ? f : 0;
+    }
+    return SeqSpan{first, nb, len};
+  }
+  __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
+  __device__ __forceinline__ int table_seq(const DecodeParams&, int s) const { return s; }
+  __device__ __forceinline__ int row_group0(const DecodeParams&, int s) const { return s; }
+  __device__ __forceinline__ int row_groups(const DecodeParams&, int) const { return 1; }
+  __device__ __forceinline__ int limit(const DecodeParams&, int, int len) const { return len - 1; }
+};
+
+// A sequence with q_len query positions, causal among the new tokens.  A
+// sequence shorter than q_len is treated as empty.
+template <int RG>
+struct Source<kMulti, RG> {
+  template <int BB>
+  __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int s) const {
+    int len = checked_len(p, s, BB);
+    if (len < p.q_len) len = 0;
+    return SeqSpan{0, (len + BB - 1) / BB, len};
+  }
+  __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
+  __device__ __forceinline__ int table_seq(const DecodeParams&, int s) const { return s; }
+  __device__ __forceinline__ int row_group0(const DecodeParams& p, int s) const { return s * p.q_len; }
+  __device__ __forceinline__ int row_groups(const DecodeParams& p, int) const { return p.q_len; }
+  __device__ __forceinline__ int limit(const DecodeParams& p, int rg, int len) const { return len - p.q_len + rg; }
+};
+
+// Shared blocks of group g, or 0 when the group cannot share: members are
+// sequences [starts[g], starts[g+1]), at most RG of them, and the prefix must
+// be shorter than every member's block count, so that every member keeps at
+// least one block (its newest token) of its own.
+template <int BB, int RG>
+__device__ __forceinline__ int group_prefix_blocks(const DecodeParams& p, int g) {
+  const int s0 = __ldg(p.group_starts + g), s1 = __ldg(p.group_starts + g + 1);
+  const int pb = __ldg(p.group_prefix + g);
+  if (s0 < 0 || s1 > p.num_seqs || s1 - s0 < 1 || s1 - s0 > RG || pb <= 0) return 0;
+  for (int s = s0; s < s1; ++s) {
+    if (pb >= (checked_len(p, s, BB) + BB - 1) / BB) return 0;
+  }
+  return pb;
+}
+
+// A group of sequences: the leading blocks they share, read through the
+// first member's table.
+template <int RG>
+struct Source<kPrefix, RG> {
+  template <int BB>
+  __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int g) const {
+    const int pb = group_prefix_blocks<BB, RG>(p, g);
+    return SeqSpan{0, pb, pb * BB};
+  }
+  __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_groups; }
+  __device__ __forceinline__ int table_seq(const DecodeParams& p, int g) const { return __ldg(p.group_starts + g); }
+  __device__ __forceinline__ int row_group0(const DecodeParams& p, int g) const { return __ldg(p.group_starts + g); }
+  __device__ __forceinline__ int row_groups(const DecodeParams& p, int g) const {
+    return __ldg(p.group_starts + g + 1) - __ldg(p.group_starts + g);
+  }
+  __device__ __forceinline__ int limit(const DecodeParams&, int, int len) const { return len - 1; }
+};
+
+// kPrefix launches, every CTA before its own work: record each member's
+// shared block count for the kDecode launch that follows (0 where the group
+// cannot share) and check that the groups partition the sequences.  Group g
+// is handled by thread g / gridDim.x of CTA g % gridDim.x.
+template <int BB, int RG>
+__device__ void prefix_bookkeeping(const DecodeParams& p) {
+  const long long stride = static_cast<long long>(gridDim.x) * kThreads;
+  for (long long g = static_cast<long long>(threadIdx.x) * gridDim.x + blockIdx.x; g < p.num_groups; g += stride) {
+    const int s0 = __ldg(p.group_starts + g), s1 = __ldg(p.group_starts + g + 1);
+    if (s0 < 0 || s1 < s0 || s1 > p.num_seqs || s1 - s0 > RG) record_status(p.status, PA_DEV_BAD_GROUP);
+    const int pb = group_prefix_blocks<BB, RG>(p, static_cast<int>(g));
+    for (int s = max(s0, 0); s < min(s1, p.num_seqs); ++s) p.seq_prefix[s] = pb;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (__ldg(p.group_starts) != 0 || __ldg(p.group_starts + p.num_groups) != p.num_seqs) {
+      record_status(p.status, PA_DEV_BAD_GROUP);
+    }
+  }
+}
+
+// kDecode and kMulti: zero the output rows of sequences with nothing to read
+// (length 0, invalid, or shorter than q_len); sequence s by CTA s % gridDim.x.
+template <int kMode, int RG>
+__device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>& src) {
+  const long long nctas = gridDim.x, cta = blockIdx.x;
+  for (int s = threadIdx.x; s < p.num_seqs; s += kThreads) {
+    if ((s % nctas) != cta) continue;
+    if constexpr (kMode == kMulti) {
+      const int raw = __ldg(p.seq_lens + s);
+      if (raw > 0 && raw < p.q_len) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
+    }
+    const SeqSpan sp = src.template span<B>(p, s);
+    if (sp.nb > sp.first) continue;
+    uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(src.row_group0(p, s)) * p.num_q_heads * D);
+    const int n = src.row_groups(p, s) * p.num_q_heads * D / 8;
+    for (int i = 0; i < n; ++i) o[i] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// ---- unit results --------------------------------------------------------------
+
+// Row c of the unit in segment sg, head_dim element d, from its state
+// (m, L, unnormalised a): the normalised output (merged first with the shared
+// prefix's state when the unit skipped one), or, in kPrefix, the state itself.
+template <bool kBf16, int G, int kMode>
+__device__ __forceinline__ void emit_row(const DecodeParams& p, const Seg& sg, int c, int d, float m, float L,
+                                         float a) {
+  const int rg = c / G, g = c % G;
+  const int Hq = p.num_q_heads;
+  const int head = sg.h * G + g;
+  if constexpr (kMode == kPrefix) {
+    const int s = __ldg(p.group_starts + sg.s) + rg;
+    float* pp = p.prefix_part + (static_cast<size_t>(s) * Hq + head) * (D + 2);
+    if (d == 0) {
+      pp[0] = m;
+      pp[1] = L;
+    }
+    pp[2 + d] = a;
+  } else {
+    if constexpr (kMode == kDecode) {
+      if (sg.first > 0) {
+        const float* pp = p.prefix_part + (static_cast<size_t>(sg.s) * Hq + head) * (D + 2);
+        const float pm = __ldcg(pp), pl = __ldcg(pp + 1), pa = __ldcg(pp + 2 + d);
+        const float M = fmaxf(m, pm);
+        const float w0 = fast_exp2(m - M), w1 = fast_exp2(pm - M);
+        a = a * w0 + pa * w1;
+        L = L * w0 + pl * w1;
+      }
+    }
+    const size_t row = (kMode == kMulti) ? static_cast<size_t>(sg.s) * p.q_len + rg : static_cast<size_t>(sg.s);
+    const uint32_t two = pack2<kBf16>(a / L, 0.f);
+    p.out[(row * Hq + head) * D + d] = static_cast<uint16_t>(two & 0xffffu);
+  }
+}
+
+// Called by the 128 softmax threads after this CTA's partial state of a split
+// unit is written and fenced.  The last CTA to arrive merges every partial
+// state of the unit (the rescale rule of the online softmax, per row and
+// head_dim element; thread = element) and emits the rows.
+template <bool kBf16, int G, int R, int kMode, typename Sync>
+__device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, const WorkRange& wr, int rows,
+                                       int ctid, int* is_last, Sync sync) {
+  constexpr int kStride = Rows<R>::kPartStride;
+  const long long F = sg.unit_first;
+  const long long first = cta_of(F, wr.total, wr.nparts);
+  const long long last = cta_of(F + sg.ng - 1, wr.total, wr.nparts);
+  int32_t* counter = p.counters + static_cast<size_t>(sg.s) * p.num_kv_heads + sg.h;
+  sync();
+  if (ctid == 0) {
+    const int prev = atomicAdd(counter, 1);
+    *is_last = (prev == static_cast<int>(last - first));
+  }
+  sync();
+  if (*is_last) {
+    __threadfence();
+    const int d = ctid;
+    for (int c = 0; c < rows; ++c) {
+      float M = -INFINITY;
+      for (long long cc = first; cc <= last; ++cc) {
+        M = fmaxf(M, __ldcg(p.partials + partial_slot(cc, F, wr) * kStride + c));
+      }
+      float L = 0.f, a = 0.f;
+      for (long long cc = first; cc <= last; ++cc) {
+        const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
+        const float w = fast_exp2(__ldcg(pp + c) - M);
+        L = fmaf(__ldcg(pp + R + c), w, L);
+        a = fmaf(__ldcg(pp + 2 * R + c * D + d), w, a);
+      }
+      emit_row<kBf16, G, kMode>(p, sg, c, d, M, L, a);
+    }
+    if (ctid == 0) *counter = 0;
+  }
+}
+
+// ---- the kernel ---------------------------------------------------------------
+
+template <bool kBf16, int G, int RG, int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    pa_decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_q,
+                        const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
+  constexpr int R = G * RG;
+  using Sh = Rows<R>;
+  constexpr int N = Sh::N, kVStages = Sh::kVStages, kLanesPerCol = Sh::kLanesPerCol;
+  static_assert(kMode != kDecode || RG == 1, "a decode unit has one row group");
+  using Smem = TcSmem<R>;
+  const Source<kMode, RG> src;
+  extern __shared__ unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const long long cta = blockIdx.x;
+  const int Hkv = p.num_kv_heads;
+
+  // ---- set-up that reads no input (barriers, TMEM, tensor-map prefetch);
+  // with programmatic dependent launch it overlaps the previous kernel
+  if (tid == 0) {
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sm.kfull[i], 1);
+      mbar_init(&sm.kempty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sm.vfull[i], 1);
+      mbar_init(&sm.vempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.qfull[i], 1);
+      mbar_init(&sm.qempty[i], 1);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_free[i], 4);
+      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.o_full[i], 1);
+      mbar_init(&sm.o_free[i], 4);
+    }
+    mbar_init(&sm.mma_done, 1);
+    sm.abort = 0;
+    sm.k_issued = 0;
+    sm.k_consumed = 0;
+    sm.v_issued = 0;
+    sm.v_consumed = 0;
+    sm.q_issued = 0;
+    sm.q_consumed = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&map_q);
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, Sh::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const volatile int* abort_flag = &sm.abort;
+  constexpr uint32_t kColS = 0, kColO = 2 * N;
+
+  // ---- inputs may come from the previous kernel in the stream
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if constexpr (kMode == kPrefix) {
+    prefix_bookkeeping<B, RG>(p);
+  } else {
+    zero_empty_units(p, src);
+  }
+  WorkRange wr;
+  Cursor cur;
+  const bool has_work = decode_prologue<kThreads, B, CB>(p, sm.range, wr, cur, src);  // uniform across the CTA
+
+  if (!has_work) {
+    // nothing to stream: straight to teardown
+  } else if (warp == 0) {
+    // ===================== producer =========================================
+    const uint64_t pol_stream = l2_policy_evict_first();
+    const uint64_t pol_keep = l2_policy_evict_last();
+    bool ok = true;
+    int ci = 0, qi = 0, k_issued = 0, v_issued = 0, q_issued = 0;
+    if (p.test_flags & kFlagTestWithholdCopies) {
+      if (lane == 0) {
+        const uint64_t t0 = global_timer_ns();
+        while (*abort_flag == 0 && global_timer_ns() - t0 < 4 * p.wait_limit_ns) {
+        }
+      }
+      __syncwarp();
+    } else {
+      Seg sg;
+      while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+        const int qs = qi & 1;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&sm.qempty[qs], ((qi >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+          if (ok) {
+            // q rows: heads [h G, h G + G) of row groups [z, z + RG), one box per 64-column half
+            const int z = src.row_group0(p, sg.s);
+            mbar_arrive_expect_tx(&sm.qfull[qs], 2 * R * kRowBytes);
+            tma_load_3d(sm.q[qs], &map_q, 0, sg.h * G, z, &sm.qfull[qs], pol_keep);
+            tma_load_3d(sm.q[qs] + N * kRowBytes, &map_q, 64, sg.h * G, z, &sm.qfull[qs], pol_keep);
+            ++q_issued;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        ++qi;
+        // Block-table entries 32 at a time (lane l holds entry b0 + l); the
+        // next batch is in flight while the current one is issued.
+        const int32_t* trow = p.block_tables + static_cast<size_t>(src.table_seq(p, sg.s)) * p.max_nb + sg.j0;
+        int e_cur = (lane < sg.n) ? __ldg(trow + lane) : 0;
+        for (int b0 = 0; ok && b0 < sg.n; b0 += 32) {
+          const int e_next = (b0 + 32 + lane < sg.n) ? __ldg(trow + b0 + 32 + lane) : 0;
+          if (b0 + lane < sg.n && (e_cur < 0 || e_cur >= p.num_blocks)) {
+            record_status(p.status, PA_DEV_BAD_BLOCK_ID);
+            e_cur = 0;
+          }
+          const int b_end = min(b0 + 32, sg.n);
+          for (int c0 = b0; c0 < b_end; c0 += CB) {
+            const ChunkInfo ch = chunk_at(sg, c0);
+            const int e = __shfl_sync(0xffffffffu, e_cur, (c0 - b0) + (lane & (CB - 1)));
+            const int ks = ci % kKStages, vs = ci % kVStages;
+            const int y = (e * Hkv + sg.h) * B;
+            if (lane == 0) {
+              ok = mbar_wait_bounded(&sm.kempty[ks], ((ci / kKStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+              if (ok) mbar_arrive_expect_tx(&sm.kfull[ks], ch.nblk * 2 * kBlockBytes);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane < ch.nblk) {
+              uint8_t* base = sm.kbuf[ks] + lane * kBlockBytes;
+              tma_load_2d(base, &map_k, 0, y, &sm.kfull[ks], pol_stream);
+              tma_load_2d(base + kHalfBytes, &map_k, 64, y, &sm.kfull[ks], pol_stream);
+            }
+            __syncwarp();
+            ++k_issued;
+            if (lane == 0) {
+              ok = mbar_wait_bounded(&sm.vempty[vs], ((ci / kVStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+              if (ok) mbar_arrive_expect_tx(&sm.vfull[vs], ch.nblk * 2 * kBlockBytes);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane < ch.nblk) {
+              uint8_t* base = sm.vbuf[vs] + lane * kBlockBytes;
+              tma_load_2d(base, &map_v, 0, y, &sm.vfull[vs], pol_stream);
+              tma_load_2d(base + kHalfBytes, &map_v, 64, y, &sm.vfull[vs], pol_stream);
+            }
+            __syncwarp();
+            ++v_issued;
+            ++ci;
+          }
+          e_cur = e_next;
+        }
+      }
+    }
+    if (lane == 0) {
+      sm.k_issued = k_issued;
+      sm.v_issued = v_issued;
+      sm.q_issued = q_issued;
+      if (!ok) {
+        sm.abort = 1;
+        record_status(p.status, PA_DEV_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================== MMA issuer ========================================
+    // A non-blocking scheduler: each pass tests whether QK of the next chunk
+    // (its K landed, its S buffer free, its q ready) or PV of the oldest chunk
+    // still waiting (its P written, its V landed, its O buffer free) can go,
+    // and issues whichever can, so PV of chunk i never waits for chunk i+1.
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = make_idesc(kBf16, false, N);
+      constexpr uint32_t kIdescPV = make_idesc(kBf16, true, N);
+      bool ok = true;
+      int qk = 0, pv = 0, seg_i = 0, q_consumed = 0;
+      uint32_t ring = 0;  // valid tokens of each pending chunk (index & 3), 8 bits each
+      bool have_seg = false, q_ready = false, walk_done = false;
+      int c0 = 0;
+      Seg sg;
+      uint64_t t_idle = 0;
+      uint32_t idle = 0;
+      while (ok) {
+        bool progress = false;
+        if (!walk_done && !have_seg) {
+          if (next_seg<B, CB>(cur, sg, p, src)) {
+            have_seg = true;
+            c0 = 0;
+          } else {
+            walk_done = true;
+          }
+        }
+        if (have_seg) {
+          const int qs = seg_i & 1;
+          if (!q_ready && mbar_test_wait(&sm.qfull[qs], (seg_i >> 1) & 1)) {
+            q_ready = true;
+            ++q_consumed;
+          }
+          const int ks = qk % kKStages;
+          if (q_ready && qk - pv < 4 && mbar_test_wait(&sm.kfull[ks], (qk / kKStages) & 1) &&
+              mbar_test_wait(&sm.s_free[qk & 1], ((qk >> 1) & 1) ^ 1u)) {
+            tc_fence_after();
+            const uint32_t k0 = smem_u32(sm.kbuf[ks]);
+            const uint32_t q0 = smem_u32(sm.q[qs]);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t a = sw128_desc(k0 + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              const uint64_t b = sw128_desc(q0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              umma(tmem + kColS + (qk & 1) * N, a, b, kIdescQK, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[qk & 1]);
+            umma_commit(&sm.kempty[ks]);
+            const int slot_shift = (qk & 3) * 8;
+            ring = (ring & ~(0xFFu << slot_shift)) | (static_cast<uint32_t>(chunk_at(sg, c0).ntok) << slot_shift);
+            c0 += CB;
+            if (c0 >= sg.n) {  // last chunk of the segment: q may be reloaded after this QK
+              umma_commit(&sm.qempty[qs]);
+              have_seg = false;
+              q_ready = false;
+              ++seg_i;
+            }
+            ++qk;
+            progress = true;
+          }
+        }
+        if (pv < qk) {
+          const int pb = pv & 1;
+          const uint32_t par = (pv >> 1) & 1;
+          const int vs = pv % kVStages;
+          if (mbar_test_wait(&sm.p_full[pb], par) && mbar_test_wait(&sm.o_free[pb], par ^ 1u) &&
+              mbar_test_wait(&sm.vfull[vs], (pv / kVStages) & 1)) {
+            tc_fence_after();
+            const int ntok = static_cast<int>((ring >> ((pv & 3) * 8)) & 0xFFu);
+            const uint32_t v0 = smem_u32(sm.vbuf[vs]);
+            const uint32_t p0 = smem_u32(sm.p[pb]);
+            const int nks = (ntok + 15) / 16;
+            for (int k = 0; k < nks; ++k) {
+              const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
+              const uint64_t b = sw128_desc(p0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              umma(tmem + kColO + pb * N, a, b, kIdescPV, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.o_full[pb]);
+            umma_commit(&sm.vempty[vs]);
+            ++pv;
+            progress = true;
+          }
+        } else if (walk_done) {
+          break;  // every chunk has had its QK and its PV
+        }
+        if (progress) {
+          idle = 0;
+        } else if ((++idle & 63u) == 0) {
+          const uint64_t now = global_timer_ns();
+          if (idle == 64) t_idle = now;
+          if (*abort_flag != 0 || now - t_idle > p.wait_limit_ns) ok = false;
+        }
+      }
+      // every MMA issued above completes before TMEM is released
+      umma_commit(&sm.mma_done);
+      (void)mbar_wait_bounded(&sm.mma_done, 0, nullptr, p.wait_limit_ns);
+      sm.k_consumed = qk;
+      sm.v_consumed = pv;
+      sm.q_consumed = q_consumed;
+      if (!ok) {
+        sm.abort = 1;
+        record_status(p.status, PA_DEV_TIMEOUT);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ===================== softmax + epilogue (warps 2-5) ====================
+    // Per chunk i: softmax(i) then the epilogue of chunk i-1, so the PV of
+    // chunk i-1 runs on the tensor core while the softmax of chunk i runs here.
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+    const int r = quad * 32 + lane;   // token row of the chunk; head_dim index in the epilogue
+    const int ctid = tid - 64;        // 0..127
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int my_col = lane / kLanesPerCol;  // the column this lane holds after a reduce
+    const bool col_writer = (lane % kLanesPerCol) == 0;
+    bool ok = true;
+    int ci = 0;
+    Seg sg;
+    float acc[R];
+    float l_lane = 0.f;  // running sum of p over this warp's tokens, column my_col
+
+    // Online softmax of chunk ci (the first of its segment when `first`):
+    // P^T into the swizzled B operand, the new running max and the rescale
+    // factor of the running output into shared memory.
+    auto softmax_chunk = [&](int ci, const ChunkInfo& ch, bool first, int rows, int len) -> bool {
+      const int vs = ci % kVStages;
+      const int sb = ci & 1;
+      bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      float sN[N];
+      tmem_ld<N>(tmem + lane_base + kColS + sb * N, sN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[sb]);
+
+      // scores of this token row for every query row (log2 domain), masked
+      const int t = ch.j * B + r;  // token index in the sequence
+      float sc[R];
+#pragma unroll
+      for (int c = 0; c < R; ++c) {
+        const bool valid = c < rows && r < ch.ntok && t <= src.limit(p, c / G, len);
+        sc[c] = valid ? sN[c] * p.scale_log2 : -INFINITY;
+      }
+      {
+        float v[R];
+#pragma unroll
+        for (int c = 0; c < R; ++c) v[c] = sc[c];
+        const float wm = warp_column_reduce<R, true>(v, lane);
+        if (col_writer) sm.red[sb][quad][my_col] = wm;
+      }
+      named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+      const float* m_prev = sm.mbuf[(ci - 1) & 1];
+      float pr[R];
+#pragma unroll
+      for (int c = 0; c < R; ++c) {
+        const float cm =
+            fmaxf(fmaxf(sm.red[sb][0][c], sm.red[sb][1][c]), fmaxf(sm.red[sb][2][c], sm.red[sb][3][c]));
+        const float m_new = fmaxf(first ? -INFINITY : m_prev[c], cm);
+        pr[c] = fast_exp2(sc[c] - (m_new == -INFINITY ? 0.f : m_new));
+      }
+      {
+        const float cm = fmaxf(fmaxf(sm.red[sb][0][my_col], sm.red[sb][1][my_col]),
+                               fmaxf(sm.red[sb][2][my_col], sm.red[sb][3][my_col]));
+        const float m_old = first ? -INFINITY : m_prev[my_col];
+        const float m_new = fmaxf(m_old, cm);
+        const float alpha = fast_exp2(m_old - (m_new == -INFINITY ? 0.f : m_new));
+        if (quad == 0 && col_writer) {
+          sm.mbuf[ci & 1][my_col] = m_new;
+          sm.abuf[ci & 1][my_col] = alpha;
+        }
+        float v[R];
+#pragma unroll
+        for (int c = 0; c < R; ++c) v[c] = pr[c];
+        l_lane = fmaf(l_lane, alpha, warp_column_reduce<R, false>(v, lane));
+      }
+      // P^T: row = query row, column = token
+      const int pb = ci & 1;
+      {
+        uint8_t* pbase = sm.p[pb] + (r >> 6) * (N * kRowBytes);
+        const int col = r & 63;
+#pragma unroll
+        for (int c = 0; c < R; ++c) {
+          const int off = (c >> 3) * (8 * kRowBytes) + (c & 7) * kRowBytes + ((((col >> 3) ^ (c & 7)) & 7) << 4) +
+                          (col & 7) * 2;
+          const uint32_t two = pack2<kBf16>(pr[c], 0.f);
+          *reinterpret_cast<uint16_t*>(pbase + off) = static_cast<uint16_t>(two & 0xffffu);
+        }
+      }
+      // V rows past the sequence end inside the last 16-token step are zeroed
+      // so that 0 * (whatever they hold) cannot reach the output
+      if ((ch.ntok & 15) != 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
+        (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
+        uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + r * kRowBytes);
+        uint4* v1 = reinterpret_cast<uint4*>(sm.vbuf[vs] + kHalfBytes + r * kRowBytes);
+#pragma unroll
+        for (int i = 0; i < kRowBytes / 16; ++i) {
+          v0[i] = make_uint4(0, 0, 0, 0);
+          v1[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[pb]);
+      return true;
+    };
+
+    // acc = acc * alpha(ci) + O^T row r of chunk ci.
+    auto epilogue_chunk = [&](int ci) -> bool {
+      const int pb = ci & 1;
+      bool w = mbar_wait_bounded(&sm.o_full[pb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      float oN[N];
+      tmem_ld<N>(tmem + lane_base + kColO + pb * N, oN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free[pb]);
+      const float* alpha = sm.abuf[ci & 1];
+#pragma unroll
+      for (int c = 0; c < R; ++c) acc[c] = fmaf(acc[c], alpha[c], oN[c]);
+      return true;
+    };
+
+    while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+      const int rows = G * src.row_groups(p, sg.s);
+#pragma unroll
+      for (int c = 0; c < R; ++c) acc[c] = 0.f;
+      l_lane = 0.f;
+      bool pending = false;
+      for (int c0 = 0; c0 < sg.n; c0 += CB) {
+        ok = softmax_chunk(ci, chunk_at(sg, c0), c0 == 0, rows, sg.len);
+        if (!ok) break;
+        if (pending) {
+          ok = epilogue_chunk(ci - 1);
+          if (!ok) break;
+        }
+        pending = true;
+        ++ci;
+      }
+      if (ok && pending) ok = epilogue_chunk(ci - 1);
+      if (!ok) break;
+
+      // ---- end of the segment: column sums, then the rows or a partial state
+      if (col_writer) sm.lred[quad][my_col] = l_lane;
+      named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+      const float* m_last = sm.mbuf[(ci - 1) & 1];
+      if (sg.j0 == sg.first && sg.j0 + sg.n == sg.nb) {
+#pragma unroll
+        for (int c = 0; c < R; ++c) {
+          if (c < rows) {
+            const float L = (sm.lred[0][c] + sm.lred[1][c]) + (sm.lred[2][c] + sm.lred[3][c]);
+            emit_row<kBf16, G, kMode>(p, sg, c, r, m_last[c], L, acc[c]);
+          }
+        }
+      } else {
+        float* pp = p.partials + partial_slot(cta, sg.unit_first, wr) * Sh::kPartStride;
+        if (ctid < R) {
+          pp[ctid] = m_last[ctid];
+          pp[R + ctid] = (sm.lred[0][ctid] + sm.lred[1][ctid]) + (sm.lred[2][ctid] + sm.lred[3][ctid]);
+        }
+#pragma unroll
+        for (int c = 0; c < R; ++c) pp[2 * R + c * D + r] = acc[c];
+        __threadfence();
+        finish_split_unit_rows<kBf16, G, R, kMode>(p, sg, wr, rows, ctid, &sm.is_last,
+                                                   [] { named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads); });
+      }
+      named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+    }
+    if (!ok && lane == 0) {
+      sm.abort = 1;
+      record_status(p.status, PA_DEV_TIMEOUT);
+    }
+  }
+
+  // ---- teardown: drain copies after an abort, release TMEM
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0 && sm.abort) {
+    for (int k = sm.k_consumed; k < sm.k_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.kfull[k % kKStages], (k / kKStages) & 1, nullptr, p.wait_limit_ns);
+    }
+    for (int k = sm.v_consumed; k < sm.v_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.vfull[k % kVStages], (k / kVStages) & 1, nullptr, p.wait_limit_ns);
+    }
+    for (int k = sm.q_consumed; k < sm.q_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.qfull[k & 1], (k >> 1) & 1, nullptr, p.wait_limit_ns);
+    }
+  }
+  if (warp == 1) tmem_dealloc(tmem, Sh::kTmemCols);
+}
+
+// ---- host side -----------------------------------------------------------------
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+  });
+  return fn;
+}
+
+// Tensor map over a packed fp16/bf16 tensor whose innermost dimension is
+// head_dim (128) and whose outer dimensions are outer[0..rank-2], innermost
+// first; boxes of 64 columns x outer_box, 128-byte swizzle; coordinates past
+// the end read as zero.
+inline bool make_map(CUtensorMap* map, const void* base, int rank, const unsigned long long* outer,
+                     const uint32_t* outer_box, bool bf16) {
+  auto encode = encode_fn();
+  if (encode == nullptr || rank < 2 || rank > 3) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), 1, 1};
+  cuuint64_t strides[2] = {0, 0};
+  cuuint32_t box[3] = {64, 1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint64_t stride = static_cast<cuuint64_t>(D) * 2;
+  for (int i = 1; i < rank; ++i) {
+    dims[i] = outer[i - 1];
+    box[i] = outer_box[i - 1];
+    strides[i - 1] = stride;
+    stride *= outer[i - 1];
+  }
+  const CUresult r = encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                            static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool kBf16, int G, int RG, int kMode>
+cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv;
+  const unsigned long long q_rows =
+      static_cast<unsigned long long>(prm.num_seqs) * (kMode == kMulti ? prm.q_len : 1);
+  const unsigned long long kv_rows = static_cast<unsigned long long>(prm.num_blocks) * prm.num_kv_heads * B;
+  if (kv_rows >= (1ull << 31) || q_rows >= (1ull << 31)) return cudaErrorInvalidValue;
+  const unsigned long long q_outer[2] = {static_cast<unsigned long long>(prm.num_q_heads), q_rows};
+  const uint32_t q_box[2] = {static_cast<uint32_t>(G), static_cast<uint32_t>(RG)};
+  const unsigned long long kv_outer[1] = {kv_rows};
+  const uint32_t kv_box[1] = {static_cast<uint32_t>(B)};
+  if (!make_map(&mq, prm.q, 3, q_outer, q_box, kBf16) || !make_map(&mk, prm.k_pool, 2, kv_outer, kv_box, kBf16) ||
+      !make_map(&mv, prm.v_pool, 2, kv_outer, kv_box, kBf16)) {
+    return cudaErrorInvalidValue;
+  }
+  return launch_overlapped(pa_decode_tc_kernel<kBf16, G, RG, kMode>, dim3(ctas), dim3(kThreads),
+                           static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
+}
+
+template <bool kBf16, int G, int RG, int kMode>
+Variant tc_variant() {
+  constexpr int R = G * RG;
+  return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode>), kThreads,
+                 smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode>};
+}
+
+inline bool tc_pool_ok(const pa_pool_desc& pool) {
+  return pool.head_dim == D && pool.block_size == B && (pool.dtype == PA_BF16 || pool.dtype == PA_FP16);
+}
+
+// Row-group count a request for rg row groups runs with: the smallest power
+// of two >= rg, or 0 when G * that exceeds 32 rows.
+inline int row_groups_for(int G, int rg) {
+  if (G <= 0 || rg <= 0) return 0;
+  int r = 1;
+  while (r < rg) r *= 2;
+  return G * r <= 32 ? r : 0;
+}
+
+}  // namespace tc
+}  // namespace pa

@@ -240,3 +240,51 @@ extern "C" pa_status pa_bm_prepare_step(pa_block_manager* bm, const int64_t* seq
   *num_pairs = pairs;
   return PA_OK;
 }
+
+// ---- shared-prefix groups of one step's tables (host planning) --------------
+
+extern "C" pa_status pa_shared_prefix_groups(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                             const int32_t* seq_lens, int32_t num_seqs, int32_t block_size,
+                                             int32_t max_group_size, int32_t min_prefix_blocks,
+                                             int32_t* group_starts, int32_t* group_prefix_blocks,
+                                             int32_t* num_groups) {
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || max_group_size < 1 || num_groups == nullptr ||
+      group_starts == nullptr || (num_seqs > 0 && (block_tables == nullptr || seq_lens == nullptr ||
+                                                   group_prefix_blocks == nullptr))) {
+    return PA_ERR_INVALID_ARG;
+  }
+  auto blocks_of = [&](int32_t s) -> int32_t {
+    const int64_t n = seq_lens[s];
+    if (n <= 0 || n > static_cast<int64_t>(max_blocks_per_seq) * block_size) return 0;
+    return static_cast<int32_t>((n + block_size - 1) / block_size);
+  };
+  auto row = [&](int32_t s) { return block_tables + static_cast<size_t>(s) * max_blocks_per_seq; };
+  int32_t g = 0;
+  int32_t s = 0;
+  while (s < num_seqs) {
+    const int32_t first = s;
+    const int32_t nb0 = blocks_of(first);
+    int32_t prefix = nb0;  // common leading entries so far
+    int32_t min_nb = nb0;
+    int32_t end = first + 1;
+    while (nb0 > 0 && end < num_seqs && end - first < max_group_size) {
+      const int32_t nb = blocks_of(end);
+      if (nb == 0 || row(end)[0] != row(first)[0]) break;
+      int32_t c = 0;
+      const int32_t lim = std::min(prefix, nb);
+      while (c < lim && row(end)[c] == row(first)[c]) ++c;
+      prefix = c;
+      min_nb = std::min(min_nb, nb);
+      ++end;
+    }
+    int32_t pb = std::min(prefix, min_nb - 1);
+    if (end - first < 2 || pb < std::max(min_prefix_blocks, 1)) pb = 0;
+    group_starts[g] = first;
+    group_prefix_blocks[g] = pb;
+    ++g;
+    s = end;
+  }
+  group_starts[g] = num_seqs;
+  *num_groups = g;
+  return PA_OK;
+}

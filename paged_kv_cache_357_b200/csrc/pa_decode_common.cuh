@@ -44,6 +44,15 @@ struct DecodeParams {
   float scale_log2;
   unsigned long long wait_limit_ns;
   int test_flags;
+  // multi-query decode: query positions per sequence (q, out are
+  // [num_seqs][q_len][num_q_heads][head_dim]); 1 otherwise
+  int q_len;
+  // shared-prefix decode (both passes; null / 0 otherwise)
+  const int32_t* group_starts;   // [num_groups + 1], consecutive sequences per group
+  const int32_t* group_prefix;   // [num_groups] shared leading blocks of each group
+  int num_groups;
+  int32_t* seq_prefix;           // [num_seqs] prefix blocks per sequence (written by pass 1, read by pass 2)
+  float* prefix_part;            // [num_seqs][num_q_heads][2 + head_dim] prefix states (m, l, acc)
 };
 
 constexpr int kFlagTestWithholdCopies = PA_DECODE_TEST_WITHHOLD_COPIES;  // producer issues nothing
@@ -53,42 +62,63 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, int B) 
   return (n < 0 || n > p.max_nb * B) ? 0 : n;
 }
 
+// The blocks a "sequence" of the work list covers: logical blocks
+// [first, nb) of a sequence of len tokens.  The default span is the whole
+// sequence; other kernels cover only a suffix, or a group's shared prefix.
+struct SeqSpan {
+  int first, nb, len;
+};
+
+struct WholeSequence {
+  template <int B>
+  __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int s) const {
+    const int len = checked_len(p, s, B);
+    return SeqSpan{0, (len + B - 1) / B, len};
+  }
+  __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
+};
+
 struct Cursor {
   int s, h;
-  int jg;   // next granule of unit (s, h)
-  int ng;   // granules of sequence s's units
-  int nb;   // blocks of sequence s's units
-  int len;  // tokens of sequence s
+  int jg;     // next granule of unit (s, h)
+  int ng;     // granules of sequence s's units
+  int first;  // first logical block of the span
+  int nb;     // end of the span (logical blocks)
+  int len;    // tokens of sequence s
   long long x, remaining;  // flattened granule index; granules left in the range
 };
 
 struct Seg {
   int s, h;
   int j0, n;  // logical blocks [j0, j0 + n) of unit (s, h)
-  int nb;     // blocks of the unit
+  int first;  // first logical block of the unit's span
+  int nb;     // end of the unit's span
   int ng;     // granules of the unit
   int len;    // tokens of the sequence
   long long unit_first;  // flattened index of the unit's granule 0
 };
 
-template <int B, int CB>
-__device__ __forceinline__ void load_seq(Cursor& c, const DecodeParams& p) {
-  c.len = checked_len(p, c.s, B);
-  c.nb = (c.len + B - 1) / B;
-  c.ng = (c.nb + CB - 1) / CB;
+template <int B, int CB, class Src>
+__device__ __forceinline__ void load_seq(Cursor& c, const DecodeParams& p, const Src& src) {
+  const SeqSpan sp = src.template span<B>(p, c.s);
+  c.len = sp.len;
+  c.first = sp.first;
+  c.nb = sp.nb;
+  c.ng = sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
 }
 
 // Next segment of the CTA's range; advances the cursor past it.
-template <int B, int CB>
-__device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams& p) {
+template <int B, int CB, class Src = WholeSequence>
+__device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams& p, const Src& src = Src()) {
   if (c.remaining <= 0) return false;
   const long long left = c.ng - c.jg;
   const int k = static_cast<int>(left < c.remaining ? left : c.remaining);
   sg.s = c.s;
   sg.h = c.h;
-  sg.j0 = c.jg * CB;
-  const int j1 = (c.jg + k) * CB;
+  sg.j0 = c.first + c.jg * CB;
+  const int j1 = c.first + (c.jg + k) * CB;
   sg.n = (j1 < c.nb ? j1 : c.nb) - sg.j0;
+  sg.first = c.first;
   sg.nb = c.nb;
   sg.ng = c.ng;
   sg.len = c.len;
@@ -102,11 +132,11 @@ __device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams&
       c.h = 0;
       if (c.remaining > 0) {
         do {
-          if (++c.s >= p.num_seqs) {  // inconsistent lengths: stop cleanly
+          if (++c.s >= src.count(p)) {  // inconsistent lengths: stop cleanly
             c.remaining = 0;
             break;
           }
-          load_seq<B, CB>(c, p);
+          load_seq<B, CB>(c, p, src);
         } while (c.ng == 0);
       }
     }
@@ -158,20 +188,21 @@ struct WorkRange {
 // Every thread of the CTA calls this.  Writes zero outputs of empty
 // sequences (each by one CTA), computes this CTA's range and positions the
 // cursor at its first block.  Returns false when the CTA has no work.
-template <int NT, int B, int CB>
-__device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange& wr, Cursor& cur) {
+template <int NT, int B, int CB, class Src = WholeSequence>
+__device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange& wr, Cursor& cur,
+                                const Src& src = Src()) {
   const int tid = threadIdx.x;
   const long long nctas = gridDim.x, cta = blockIdx.x;
   const int Hkv = p.num_kv_heads;
+  const int nseq = src.count(p);
   long long mine = 0;
   for (int s = tid; s < p.num_seqs; s += NT) {
     const int raw = __ldg(p.seq_lens + s);
-    int n = raw;
-    if (raw < 0 || raw > p.max_nb * B) {
-      if (cta == 0) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
-      n = 0;
-    }
-    mine += ((n + B - 1) / B + CB - 1) / CB;
+    if ((raw < 0 || raw > p.max_nb * B) && cta == 0) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
+  }
+  for (int s = tid; s < nseq; s += NT) {
+    const SeqSpan sp = src.template span<B>(p, s);
+    mine += sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
   }
   long long seq_granules;
   (void)block_inclusive_scan<NT>(mine, rs, seq_granules);
@@ -186,9 +217,13 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
   if (tid == 0) rs.found = 0;
   __syncthreads();
   long long base = 0;
-  for (int chunk = 0; chunk < p.num_seqs; chunk += NT) {
+  for (int chunk = 0; chunk < nseq; chunk += NT) {
     const int s = chunk + tid;
-    const long long ng = (s < p.num_seqs) ? ((checked_len(p, s, B) + B - 1) / B + CB - 1) / CB : 0;
+    long long ng = 0;
+    if (s < nseq) {
+      const SeqSpan sp = src.template span<B>(p, s);
+      ng = sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
+    }
     long long chunk_total;
     const long long incl = block_inclusive_scan<NT>(ng, rs, chunk_total);
     const long long excl = incl - ng;
@@ -203,7 +238,7 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
   }
   if (!rs.found) return false;  // only with lengths changing under the kernel
   cur.s = rs.s0;
-  load_seq<B, CB>(cur, p);
+  load_seq<B, CB>(cur, p, src);
   const long long off = wr.start - rs.pre0 * Hkv;
   cur.h = static_cast<int>(off / cur.ng);
   cur.jg = static_cast<int>(off % cur.ng);

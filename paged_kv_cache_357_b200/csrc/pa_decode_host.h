@@ -16,12 +16,20 @@ struct Variant {
   const void* kernel;  // for occupancy queries and attributes
   int threads;
   int smem_bytes;
-  int part_stride;  // floats per partial slot: G * (D + 2)
+  int part_stride;  // floats per partial slot: query rows per unit * (D + 2)
   LaunchFn launch;
 };
 
-// Tensor-core variant for this pool and group size, if one exists
-// (defined in pa_decode_tc.cu).
+// Tensor-core variants (pa_attn_tc.cuh), if one exists for this pool and
+// shape.  `group` is the number of query heads per kv head.
+// Plain decode (pa_decode_tc.cu): groups of 4 and 8.
 bool select_tc_variant(const pa_pool_desc& pool, int group, Variant& v);
+// Second pass of the shared-prefix decode (pa_decode_tc.cu): groups of 1-8.
+bool select_tc_suffix_variant(const pa_pool_desc& pool, int group, Variant& v);
+// Multi-query decode with q_len >= 2 positions (pa_attn_tc_multi.cu).
+bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v);
+// First pass of the shared-prefix decode, groups of up to max_members
+// sequences (pa_attn_tc_prefix.cu).
+bool select_tc_prefix_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);
 
 }  // namespace pa

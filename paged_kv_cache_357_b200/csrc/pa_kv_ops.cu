@@ -129,6 +129,7 @@ extern "C" const char* pa_status_string(int32_t status) {
     case PA_DEV_BAD_SLOT: return "device: slot_mapping entry beyond the pool";
     case PA_DEV_BAD_PAIR: return "device: copy pair block id outside [0, num_blocks)";
     case PA_DEV_TIMEOUT: return "device: a bounded pipeline wait ran out";
+    case PA_DEV_BAD_GROUP: return "device: shared-prefix groups do not partition the sequences or exceed max_group_size";
     default: return "unknown status";
   }
 }

@@ -1,0 +1,164 @@
+"""GPU parity of multi-query paged attention (pa_decode_multi, the
+tensor-core kernel with q_len causal positions per sequence) against the
+float64 oracle's decode_multi, element by element within
+2e-3 + 1e-2*|oracle|.  Inputs: seeded layouts whose cache already holds every
+token (the q_len new ones included), padding rows and unused blocks NaN."""
+
+import numpy as np
+import pytest
+
+import oracle
+from pa_testlib import assert_attention_close, subproblem, torch_bits, torch_f64
+from workloads import bits_to_torch, config_llama3_8b, f32_to_bits, fill_values_numpy, fill_values_torch, random_layout
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(seed, lens, G, L, dtype, Hkv=2):
+    layout = random_layout(seed, lens, dtype=dtype, block_size=16, num_q_heads=Hkv * G, num_kv_heads=Hkv,
+                           head_dim=128, write_new_token=False)
+    vals = fill_values_numpy(layout)
+    rng = np.random.default_rng([seed, 99])
+    q = f32_to_bits(rng.standard_normal((layout.num_seqs, L, layout.num_q_heads, 128), dtype=np.float32), dtype)
+    return layout, vals, q
+
+
+def _run(device, layout, vals, q_bits, num_ctas=0):
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    dt = layout.dtype
+    kp = bits_to_torch(vals.k_pool, dt).to(device)
+    vp = bits_to_torch(vals.v_pool, dt).to(device)
+    q = bits_to_torch(q_bits, dt).to(device)
+    tables = torch.from_numpy(layout.block_tables).to(device)
+    lens = torch.from_numpy(layout.seq_lens).to(device)
+    S, L, Hq, _ = q.shape
+    out = torch.full_like(q, float("nan"))
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    ws = pa.alloc_multi_workspace(S, L, Hq, kp, num_ctas)
+    pa.pa_decode_multi(q, kp, vp, tables, lens, layout.scale, out, ws, st, num_ctas=num_ctas)
+    torch.cuda.synchronize()
+    return out, int(st.item())
+
+
+def _oracle(layout, vals, q_bits):
+    return oracle.decode_multi(q_bits, vals.k_pool, vals.v_pool, layout.block_tables, layout.seq_lens,
+                               layout.scale, layout.num_kv_heads, layout.dtype)
+
+
+CASES = [(G, L) for G in (1, 2, 4, 8) for L in (2, 3, 4, 5, 8, 16, 32) if G * L <= 32 and L <= 32 // G]
+
+
+@pytest.mark.parametrize("G,L", CASES, ids=[f"G{g}-L{l}" for g, l in CASES])
+def test_multi_shapes(cuda_device, G, L):
+    dtype = "bf16" if (G + L) % 2 else "fp16"
+    lens = [n for n in (L, L + 1, 15, 16, 17, 127, 128, 129, 300, 1000) if n >= L] + [0]
+    layout, vals, q = _inputs(7000 + 40 * G + L, lens, G, L, dtype)
+    out, st = _run(cuda_device, layout, vals, q)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"G={G} q_len={L} {dtype}")
+
+
+@pytest.mark.parametrize("num_ctas", [1, 3, 37, 0])
+def test_multi_split_units(cuda_device, num_ctas):
+    G, L = 4, 4
+    lens = [4, 129, 700, 2049, 3000, 33]
+    layout, vals, q = _inputs(7100 + num_ctas, lens, G, L, "bf16")
+    out, st = _run(cuda_device, layout, vals, q, num_ctas)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"num_ctas={num_ctas}")
+
+
+def test_multi_short_sequence_is_flagged_and_zero(cuda_device):
+    G, L = 2, 4
+    layout, vals, q = _inputs(7200, [40, 3, 0, 100], G, L, "bf16")
+    out, st = _run(cuda_device, layout, vals, q)
+    assert st == 102  # PA_DEV_BAD_SEQ_LEN for the 3-token sequence
+    got = torch_f64(out)
+    assert not got[1].any() and not got[2].any()
+    ref = _oracle(layout, vals, q)
+    assert_attention_close(got[[0, 3]], ref[[0, 3]], "other sequences")
+
+
+def test_single_position_is_the_decode_kernel(cuda_device):
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    layout, vals, q = _inputs(7300, [5, 130, 999], 4, 1, "bf16")
+    out, st = _run(cuda_device, layout, vals, q)
+    assert st == 0
+    dt = layout.dtype
+    kp = bits_to_torch(vals.k_pool, dt).to(cuda_device)
+    vp = bits_to_torch(vals.v_pool, dt).to(cuda_device)
+    q1 = bits_to_torch(q[:, 0], dt).to(cuda_device).contiguous()
+    out1 = torch.empty_like(q1)
+    ws = pa.alloc_decode_workspace(layout.num_seqs, layout.num_q_heads, kp)
+    pa.pa_decode(q1, kp, vp, torch.from_numpy(layout.block_tables).to(cuda_device),
+                 torch.from_numpy(layout.seq_lens).to(cuda_device), layout.scale, out1, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(torch_bits(out[:, 0]), torch_bits(out1))
+
+
+def test_unsupported_shapes_are_refused(cuda_device):
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    layout, vals, q = _inputs(7400, [64, 80], 8, 8, "bf16")  # 8 heads x 8 positions = 64 rows
+    kp = bits_to_torch(vals.k_pool, "bf16").to(cuda_device)
+    with pytest.raises(pa.PaError) as e:
+        pa.multi_workspace_bytes(2, 8, layout.num_q_heads, kp)
+    assert e.value.code == 2
+    qd = bits_to_torch(q, "bf16").to(cuda_device)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device=cuda_device)
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode_multi(qd, kp, kp, torch.from_numpy(layout.block_tables).to(cuda_device),
+                           torch.from_numpy(layout.seq_lens).to(cuda_device), 0.1, torch.empty_like(qd), ws)
+    assert e.value.code == 2
+    q2 = qd[:, :2].contiguous()
+    with pytest.raises(pa.PaError) as e:  # CUDA cores have no multi-query kernel
+        pa.pa_decode_multi(q2, kp, kp, torch.from_numpy(layout.block_tables).to(cuda_device),
+                           torch.from_numpy(layout.seq_lens).to(cuda_device), 0.1, torch.empty_like(q2), ws,
+                           flags=pa.PA_DECODE_CUDA_CORES_ONLY)
+    assert e.value.code == 2
+
+
+def test_llama3_8b_full_size_speculative_verify(cuda_device):
+    """The Llama-3-8B decode workload at full size with 4 positions per
+    sequence (the newest tokens written first), sampled sequences against
+    the oracle; every output finite and inside the range of V."""
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    L = config_llama3_8b()
+    V = fill_values_torch(L, cuda_device)
+    qlen = 4
+    g = torch.Generator(device=cuda_device)
+    g.manual_seed(8081)
+    dt = V.q.dtype
+    q = torch.randn((L.num_seqs, qlen, L.num_q_heads, L.head_dim), generator=g, device=cuda_device).to(dt)
+    rng = np.random.default_rng(5)
+    seqs = sorted({int(np.argmin(L.seq_lens)), int(np.argmax(L.seq_lens)),
+                   *map(int, rng.choice(L.num_seqs, 6, replace=False))})
+    sub = subproblem(L, V, seqs)
+    q_host = torch_bits(q[seqs])
+    tables = torch.from_numpy(L.block_tables).to(cuda_device)
+    lens = torch.from_numpy(L.seq_lens).to(cuda_device)
+    slots = torch.from_numpy(L.slot_mapping).to(cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    pa.pa_cache_write(V.new_k, V.new_v, slots, V.k_pool, V.v_pool, st)
+    out = torch.full_like(q, float("nan"))
+    ws = pa.alloc_multi_workspace(L.num_seqs, qlen, L.num_q_heads, V.k_pool)
+    pa.pa_decode_multi(q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.isfinite(out).all()
+    vmax = max(float(V.v_pool.float().nan_to_num(0).abs().max()), float(V.new_v.float().abs().max()))
+    assert float(out.float().abs().max()) <= vmax * (1 + 1e-2)
+    kp, vp = oracle.cache_write(sub["k_pool"], sub["v_pool"], sub["new_k"], sub["new_v"], sub["slots"])
+    ref = oracle.decode_multi(q_host, kp, vp, sub["tables"], sub["lens"], L.scale, L.num_kv_heads, L.dtype)
+    assert_attention_close(torch_f64(out)[seqs], ref, "llama3_8b q_len=4")

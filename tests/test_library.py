@@ -49,7 +49,7 @@ def test_library_exports_nothing_else(lib):
 
 
 def test_status_strings(lib):
-    for code in [0, 1, 2, 3, 4, 5, 6, 101, 102, 103, 104, 105]:
+    for code in [0, 1, 2, 3, 4, 5, 6, 101, 102, 103, 104, 105, 106]:
         assert pa.status_string(code) != "unknown status"
     assert pa.status_string(12345) == "unknown status"
 
@@ -97,6 +97,53 @@ def test_workspace_query_rejects_bad_arguments(lib):
     # an explicit CTA count needs no device query
     n = lib.pa_decode_workspace_bytes_ex(4, 4, ctypes.byref(d), ctypes.byref(opts))
     assert n >= 7 * 2 * 1 * (64 + 2) * 4 + 4 * 4
+
+
+def _multi(lib, q_len=4, S=4, Hq=16, desc=None, flags=0, ws=FAKE):
+    desc = desc or _desc(head_dim=128)
+    opts = _lib.DecodeOpts(0, flags)
+    return lib.pa_decode_multi(FAKE, FAKE, FAKE, FAKE, 8, FAKE, S, q_len, Hq, 0.1, FAKE, ws, 1 << 20, None,
+                               ctypes.byref(desc), ctypes.byref(opts), None)
+
+
+def test_multi_rejects_bad_arguments_on_host(lib):
+    assert _multi(lib, S=0) == 0
+    assert _multi(lib, q_len=0) == 1
+    assert _multi(lib, q_len=-3) == 1
+    assert _multi(lib, Hq=12) == 2                     # group 3
+    assert _multi(lib, q_len=16) == 2                  # 4 heads x 16 positions > 32 rows
+    assert _multi(lib, desc=_desc(head_dim=64)) == 2   # tensor-core kernel only
+    assert _multi(lib, flags=_lib.PA_DECODE_CUDA_CORES_ONLY) == 2
+    assert _multi(lib, flags=64) == 1                  # unknown flag
+    d = _desc(head_dim=128)
+    opts = _lib.DecodeOpts(7, 0)
+    n = lib.pa_decode_multi_workspace_bytes(4, 4, 16, ctypes.byref(d), ctypes.byref(opts))
+    assert n >= 7 * 2 * 16 * (128 + 2) * 4 + 4 * 4
+    assert lib.pa_decode_multi_workspace_bytes(4, 16, 16, ctypes.byref(d), ctypes.byref(opts)) == 0
+    assert lib.pa_decode_multi_workspace_bytes(4, 0, 16, ctypes.byref(d), ctypes.byref(opts)) == 0
+
+
+def _prefix(lib, S=4, G=2, starts=FAKE, prefix=FAKE, max_group=2, Hq=8, desc=None):
+    desc = desc or _desc(head_dim=128)
+    return lib.pa_decode_shared_prefix(FAKE, FAKE, FAKE, FAKE, 8, FAKE, S, Hq, starts, prefix, G, max_group, 0.1,
+                                       FAKE, FAKE, 1 << 20, None, ctypes.byref(desc), None, None)
+
+
+def test_shared_prefix_rejects_bad_arguments_on_host(lib):
+    assert _prefix(lib, S=0, G=0) == 0
+    assert _prefix(lib, G=0) == 1          # sequences but no groups
+    assert _prefix(lib, G=5) == 1          # more groups than sequences
+    assert _prefix(lib, starts=None) == 1
+    assert _prefix(lib, prefix=None) == 1
+    assert _prefix(lib, max_group=0) == 1
+    assert _prefix(lib, max_group=16, Hq=16) == 2  # 4 heads x 16 members > 32 rows
+    assert _prefix(lib, desc=_desc(head_dim=64)) == 2
+    d = _desc(head_dim=128)
+    opts = _lib.DecodeOpts(5, 0)
+    n = lib.pa_decode_shared_prefix_workspace_bytes(4, 2, 8, ctypes.byref(d), ctypes.byref(opts))
+    # partials (two slots per CTA), counters, prefix lengths, prefix states
+    assert n >= 5 * 2 * 4 * 130 * 4 + 4 * 4 + 4 * 4 + 4 * 8 * 130 * 4
+    assert lib.pa_decode_shared_prefix_workspace_bytes(4, 0, 8, ctypes.byref(d), ctypes.byref(opts)) == 0
 
 
 def test_cache_write_and_copy_reject_bad_arguments(lib):
