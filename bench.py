@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "pa_decode_llama3_8b.md")
 KERNEL_SOURCES = [
     os.path.join(ROOT, "paged_kv_cache_357_b200", "csrc", name)
-    for name in ("pa_decode.cu", "pa_decode_tc.cu", "pa_decode_common.cuh", "pa_device.cuh")
+    for name in ("pa_decode.cu", "pa_decode_tc.cu", "pa_attn_tc.cuh", "pa_decode_common.cuh", "pa_device.cuh")
 ]
 
 
@@ -60,6 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--decode", default="plain", choices=["plain", "shared_prefix"],
+                    help="shared_prefix: pa_decode_shared_prefix over the workload's prompt groups")
+    ap.add_argument("--max-group", type=int, default=4, help="members per shared-prefix group")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per GPU for the llama7b / llama3_8b workloads (0 = the workload's own)")
     return ap.parse_args(argv)
@@ -70,23 +73,28 @@ def parse_args(argv=None):
 # ---------------------------------------------------------------------------
 
 
-def step_bytes(L) -> dict:
+def step_bytes(L, mode: str = "plain") -> dict:
+    """Algorithmic bytes of one step.  The decode reads every (block, kv
+    head) K/V tile its sequences reference — once per sequence, or, with
+    mode "shared_prefix", once per distinct block — plus q, out (q_len rows
+    per sequence), the table entries and lengths."""
     import numpy as np
 
     es = 2
     B, D, Hq, Hkv, S = L.block_size, L.head_dim, L.num_q_heads, L.num_kv_heads, L.num_seqs
     nb = L.total_blocks_touched()
     tile_pair = 2 * B * D * es
-    small = 2 * S * Hq * D * es + nb * 4 + S * 4
-    decode = nb * Hkv * tile_pair + small
+    small = 2 * S * L.q_len * Hq * D * es + nb * 4 + S * 4
+    per_seq = nb * Hkv * tile_pair + small
     exact = int(L.seq_lens.astype(np.int64).sum()) * Hkv * 2 * D * es + small
     unique = L.unique_blocks_touched() * Hkv * tile_pair + small
+    decode = unique if mode == "shared_prefix" else per_seq
     T = L.num_new_tokens
     write = T * Hkv * D * es * 2 * 2 + T * 8
     n = L.copy_pairs.shape[0]
     copy = n * 2 * Hkv * B * D * es * 2 + n * 16
-    return dict(decode=decode, decode_token_exact=exact, decode_unique_blocks=unique, write=write, copy=copy,
-                step=decode + write + copy, tile_pair=tile_pair, tiles=nb * Hkv)
+    return dict(decode=decode, decode_per_sequence=per_seq, decode_token_exact=exact, decode_unique_blocks=unique,
+                write=write, copy=copy, step=decode + write + copy, tile_pair=tile_pair, tiles=nb * Hkv)
 
 
 def measured_hbm_peak():
@@ -106,16 +114,23 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def decode_kernel_name(L) -> str:
-    """Which decode kernel the library runs for this workload by default."""
+def decode_kernel_name(L, mode: str = "plain") -> str:
+    """Which decode kernel(s) the library runs for this workload."""
+    if L.q_len > 1:
+        return "pa_decode_tc_kernel, multi-query (tcgen05)"
+    if mode == "shared_prefix":
+        return "pa_decode_tc_kernel, prefix pass + suffix pass (tcgen05)"
     if L.head_dim == 128 and L.block_size == 16 and L.group in (4, 8):
         return "pa_decode_tc_kernel (tcgen05)"
     return "pa_decode_kernel (CUDA cores)"
 
 
-def profiled_traffic(decode_bytes_per_launch):
-    """dram read+write bytes per decode launch from the committed ncu summary,
-    or None when there is none or the kernel source changed since."""
+def profiled_traffic(L, mode: str = "plain"):
+    """dram read+write bytes per decode launch from the committed ncu summary
+    of the default workload, or None for other workloads, when there is no
+    summary, or when the kernel source changed since it was taken."""
+    if L.name != "llama3_8b" or mode != "plain" or L.num_seqs != 256:
+        return None
     try:
         text = open(PROFILE_SUMMARY).read()
     except OSError:
@@ -222,7 +237,10 @@ def oracle_sample_step(L, seqs):
         kp, vp = oracle.copy_blocks(kp, vp, R.copy_pairs)
     if R.num_new_tokens > 0:
         kp, vp = oracle.cache_write(kp, vp, V.new_k, V.new_v, R.slot_mapping)
-    oracle.decode(V.q, kp, vp, R.block_tables, R.seq_lens, R.scale, R.num_kv_heads, R.dtype)
+    if R.q_len > 1:
+        oracle.decode_multi(V.q, kp, vp, R.block_tables, R.seq_lens, R.scale, R.num_kv_heads, R.dtype)
+    else:
+        oracle.decode(V.q, kp, vp, R.block_tables, R.seq_lens, R.scale, R.num_kv_heads, R.dtype)
     dt = time.perf_counter() - t0
     return dt, step_bytes(R)["step"]
 

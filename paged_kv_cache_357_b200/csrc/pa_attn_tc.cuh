@@ -6,11 +6,13 @@
 // pairs one kv head with R query rows, which makes both products real (if
 // thin) matrix products:
 //
-//   S^T[token, row] = K_chunk[token, :] . Q^T[:, row]       (M=128, N=16|32, K=128)
-//   O^T[d, row]     = V_chunk^T[d, token] . P^T[token, row] (M=128, N=16|32, K=16 per step)
+//   S^T[token, row] = K_chunk[token, :] . Q^T[:, row]       (M=128, N=max(16,R), K=128)
+//   O^T[d, row]     = V_chunk^T[d, token] . P^T[token, row] (M=128, N=max(16,2R), K=16 per step)
 //
 // The rows are R = G x RG: the G query heads that share the kv head (GQA),
-// times RG row groups; N is R rounded up to 16.  Three kinds of unit (kMode):
+// times RG row groups.  P^T carries 2R rows, each probability as a 16-bit
+// head plus a 16-bit residual, summed in the epilogue.  Three kinds of unit
+// (kMode):
 //   kDecode  one sequence, RG = 1: the decode step.  With per-sequence prefix
 //            lengths given, only the blocks past the prefix are read and the
 //            result is merged with the prefix's state from a kPrefix launch.
@@ -76,14 +78,23 @@ constexpr int kSoftmaxBarrier = 1;
 
 enum Mode { kDecode = 0, kMulti = 1, kPrefix = 2 };
 
-// Shapes that follow from the number of query rows R of a unit.
+// Shapes that follow from the number of query rows R of a unit.  P enters
+// the PV product as two 16-bit rows per query row, p = hi + lo (the head and
+// the rounding residual), so PV keeps about 16 significant bits of each
+// probability instead of 8 (bf16); for R <= 8 the tail rows fill columns the
+// MMA computes anyway (N = 16).
 template <int R>
 struct Rows {
   static_assert(R >= 1 && R <= 32 && (R & (R - 1)) == 0, "R is a power of two up to 32");
-  static constexpr int N = R < 16 ? 16 : R;                       // MMA N
-  static constexpr int kVStages = N == 32 ? 3 : 4;                // V is held until its PV completes
-  static constexpr int kSlotBytes = 2 * N * kRowBytes;            // a q or P slot: two 64-column halves
-  static constexpr uint32_t kTmemCols = 4 * N <= 64 ? 64 : 128;   // S[0], S[1], O[0], O[1]
+  static constexpr int Nq = R < 16 ? 16 : R;                      // MMA N of QK (q rows)
+  static constexpr int Np = 2 * R < 16 ? 16 : 2 * R;              // MMA N of PV (P head + tail rows)
+  static constexpr int kVStages = Np == 64 ? 3 : 4;               // V is held until its PV completes
+  static constexpr int kQSlotBytes = 2 * Nq * kRowBytes;          // two 64-column halves
+  static constexpr int kPSlotBytes = 2 * Np * kRowBytes;          // tokens [0, 64) and [64, 128)
+  static constexpr int kColS = 0;                                 // S[0], S[1]: Nq columns each
+  static constexpr int kColO = 2 * Nq;                            // O[0], O[1]: Np columns each
+  static constexpr int kCols = 2 * Nq + 2 * Np;
+  static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : 256;
   static constexpr int kPartStride = R * (D + 2);                 // floats per partial slot
   static constexpr int kLanesPerCol = 32 / R;                     // lanes holding one column after a reduce
 };
@@ -93,12 +104,12 @@ struct TcSmem {
   using S = Rows<R>;
   uint8_t kbuf[kKStages][kOperandBytes];  // 1024-aligned regions
   uint8_t vbuf[S::kVStages][kOperandBytes];
-  uint8_t q[2][S::kSlotBytes];
-  uint8_t p[2][S::kSlotBytes];
-  float red[2][4][R];  // per-warp column maxima, double-buffered by chunk
-  float mbuf[2][R];    // running max after each chunk
-  float abuf[2][R];    // rescale factor of each chunk's running output
-  float lred[4][R];    // per-warp column sums at the end of a segment
+  uint8_t q[2][S::kQSlotBytes];
+  uint8_t p[2][S::kPSlotBytes];
+  alignas(16) float red[2][4][R];  // per-warp column maxima, double-buffered by chunk
+  alignas(16) float mbuf[2][R];    // running max after each chunk
+  alignas(16) float abuf[2][R];    // rescale factor of each chunk's running output
+  alignas(16) float lred[4][R];    // per-warp column sums at the end of a segment
   uint64_t kfull[kKStages];
   uint64_t kempty[kKStages];
   uint64_t vfull[S::kVStages];
@@ -127,6 +138,7 @@ template <int R>
 constexpr int smem_bytes() {
   return static_cast<int>(sizeof(TcSmem<R>)) + 1024;  // + alignment slack
 }
+constexpr int kMaxSmemPerCta = 227 * 1024;
 
 // ---- tcgen05 / TMA primitives ------------------------------------------------
 
@@ -256,6 +268,24 @@ __device__ __forceinline__ float warp_column_reduce(float (&v)[R], int lane) {
     r = kMax ? fmaxf(r, got) : r + got;
   }
   return r;
+}
+
+// R consecutive floats of shared memory (16-byte aligned when R >= 4) into registers.
+template <int R>
+__device__ __forceinline__ void ld_row(const float* src, float (&dst)[R]) {
+  if constexpr (R % 4 == 0) {
+#pragma unroll
+    for (int k = 0; k < R / 4; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(src)[k];
+      dst[4 * k] = v.x;
+      dst[4 * k + 1] = v.y;
+      dst[4 * k + 2] = v.z;
+      dst[4 * k + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < R; ++k) dst[k] = src[k];
+  }
 }
 
 struct ChunkInfo {
@@ -444,20 +474,35 @@ __device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, con
   sync();
   if (*is_last) {
     __threadfence();
+    // every row at once, so each pass over the partial states costs one
+    // memory round trip per CTA piece rather than one per row
     const int d = ctid;
-    for (int c = 0; c < rows; ++c) {
-      float M = -INFINITY;
-      for (long long cc = first; cc <= last; ++cc) {
-        M = fmaxf(M, __ldcg(p.partials + partial_slot(cc, F, wr) * kStride + c));
+    float M[R], L[R], a[R];
+#pragma unroll
+    for (int c = 0; c < R; ++c) {
+      M[c] = -INFINITY;
+      L[c] = 0.f;
+      a[c] = 0.f;
+    }
+    for (long long cc = first; cc <= last; ++cc) {
+      const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
+#pragma unroll
+      for (int c = 0; c < R; ++c) M[c] = fmaxf(M[c], __ldcg(pp + c));
+    }
+    for (long long cc = first; cc <= last; ++cc) {
+      const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
+#pragma unroll
+      for (int c = 0; c < R; ++c) {
+        if (c < rows) {
+          const float w = fast_exp2(__ldcg(pp + c) - M[c]);
+          L[c] = fmaf(__ldcg(pp + R + c), w, L[c]);
+          a[c] = fmaf(__ldcg(pp + 2 * R + c * D + d), w, a[c]);
+        }
       }
-      float L = 0.f, a = 0.f;
-      for (long long cc = first; cc <= last; ++cc) {
-        const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
-        const float w = fast_exp2(__ldcg(pp + c) - M);
-        L = fmaf(__ldcg(pp + R + c), w, L);
-        a = fmaf(__ldcg(pp + 2 * R + c * D + d), w, a);
-      }
-      emit_row<kBf16, G, kMode>(p, sg, c, d, M, L, a);
+    }
+#pragma unroll
+    for (int c = 0; c < R; ++c) {
+      if (c < rows) emit_row<kBf16, G, kMode>(p, sg, c, d, M[c], L[c], a[c]);
     }
     if (ctid == 0) *counter = 0;
   }
@@ -471,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
   constexpr int R = G * RG;
   using Sh = Rows<R>;
-  constexpr int N = Sh::N, kVStages = Sh::kVStages, kLanesPerCol = Sh::kLanesPerCol;
+  constexpr int Nq = Sh::Nq, Np = Sh::Np, kVStages = Sh::kVStages, kLanesPerCol = Sh::kLanesPerCol;
   static_assert(kMode != kDecode || RG == 1, "a decode unit has one row group");
   using Smem = TcSmem<R>;
   const Source<kMode, RG> src;
@@ -525,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const volatile int* abort_flag = &sm.abort;
-  constexpr uint32_t kColS = 0, kColO = 2 * N;
+  constexpr uint32_t kColS = Sh::kColS, kColO = Sh::kColO;
 
   // ---- inputs may come from the previous kernel in the stream
   grid_dependency_wait();
@@ -565,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int z = src.row_group0(p, sg.s);
             mbar_arrive_expect_tx(&sm.qfull[qs], 2 * R * kRowBytes);
             tma_load_3d(sm.q[qs], &map_q, 0, sg.h * G, z, &sm.qfull[qs], pol_keep);
-            tma_load_3d(sm.q[qs] + N * kRowBytes, &map_q, 64, sg.h * G, z, &sm.qfull[qs], pol_keep);
+            tma_load_3d(sm.q[qs] + Nq * kRowBytes, &map_q, 64, sg.h * G, z, &sm.qfull[qs], pol_keep);
             ++q_issued;
           }
         }
@@ -636,8 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // still waiting (its P written, its V landed, its O buffer free) can go,
     // and issues whichever can, so PV of chunk i never waits for chunk i+1.
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = make_idesc(kBf16, false, N);
-      constexpr uint32_t kIdescPV = make_idesc(kBf16, true, N);
+      constexpr uint32_t kIdescQK = make_idesc(kBf16, false, Nq);
+      constexpr uint32_t kIdescPV = make_idesc(kBf16, true, Np);
       bool ok = true;
       int qk = 0, pv = 0, seg_i = 0, q_consumed = 0;
       uint32_t ring = 0;  // valid tokens of each pending chunk (index & 3), 8 bits each
@@ -671,8 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
               const uint64_t a = sw128_desc(k0 + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-              const uint64_t b = sw128_desc(q0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-              umma(tmem + kColS + (qk & 1) * N, a, b, kIdescQK, k > 0 ? 1u : 0u);
+              const uint64_t b = sw128_desc(q0 + (k >> 2) * Nq * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              umma(tmem + kColS + (qk & 1) * Nq, a, b, kIdescQK, k > 0 ? 1u : 0u);
             }
             umma_commit(&sm.s_full[qk & 1]);
             umma_commit(&sm.kempty[ks]);
@@ -702,8 +747,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nks = (ntok + 15) / 16;
             for (int k = 0; k < nks; ++k) {
               const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
-              const uint64_t b = sw128_desc(p0 + (k >> 2) * N * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-              umma(tmem + kColO + pb * N, a, b, kIdescPV, k > 0 ? 1u : 0u);
+              const uint64_t b = sw128_desc(p0 + (k >> 2) * Np * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              umma(tmem + kColO + pb * Np, a, b, kIdescPV, k > 0 ? 1u : 0u);
             }
             umma_commit(&sm.o_full[pb]);
             umma_commit(&sm.vempty[vs]);
@@ -758,8 +803,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      float sN[N];
-      tmem_ld<N>(tmem + lane_base + kColS + sb * N, sN);
+      float sN[Nq];
+      tmem_ld<Nq>(tmem + lane_base + kColS + sb * Nq, sN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[sb]);
@@ -780,41 +825,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (col_writer) sm.red[sb][quad][my_col] = wm;
       }
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+      // new running max of every query row: the chunk's maxima of the four
+      // warps and the running max before the chunk
       const float* m_prev = sm.mbuf[(ci - 1) & 1];
       float pr[R];
-#pragma unroll
-      for (int c = 0; c < R; ++c) {
-        const float cm =
-            fmaxf(fmaxf(sm.red[sb][0][c], sm.red[sb][1][c]), fmaxf(sm.red[sb][2][c], sm.red[sb][3][c]));
-        const float m_new = fmaxf(first ? -INFINITY : m_prev[c], cm);
-        pr[c] = fast_exp2(sc[c] - (m_new == -INFINITY ? 0.f : m_new));
-      }
       {
-        const float cm = fmaxf(fmaxf(sm.red[sb][0][my_col], sm.red[sb][1][my_col]),
-                               fmaxf(sm.red[sb][2][my_col], sm.red[sb][3][my_col]));
-        const float m_old = first ? -INFINITY : m_prev[my_col];
-        const float m_new = fmaxf(m_old, cm);
-        const float alpha = fast_exp2(m_old - (m_new == -INFINITY ? 0.f : m_new));
-        if (quad == 0 && col_writer) {
-          sm.mbuf[ci & 1][my_col] = m_new;
-          sm.abuf[ci & 1][my_col] = alpha;
-        }
-        float v[R];
+        float cm[R], t[R];
+        ld_row<R>(sm.red[sb][0], cm);
 #pragma unroll
-        for (int c = 0; c < R; ++c) v[c] = pr[c];
-        l_lane = fmaf(l_lane, alpha, warp_column_reduce<R, false>(v, lane));
+        for (int w = 1; w < 4; ++w) {
+          ld_row<R>(sm.red[sb][w], t);
+#pragma unroll
+          for (int c = 0; c < R; ++c) cm[c] = fmaxf(cm[c], t[c]);
+        }
+        if (!first) {
+          ld_row<R>(m_prev, t);
+#pragma unroll
+          for (int c = 0; c < R; ++c) cm[c] = fmaxf(cm[c], t[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < R; ++c) pr[c] = fast_exp2(sc[c] - (cm[c] == -INFINITY ? 0.f : cm[c]));
       }
-      // P^T: row = query row, column = token
+      // P^T: row c = head of query row c's probability, row R + c = its
+      // rounding residual; column = token
       const int pb = ci & 1;
       {
-        uint8_t* pbase = sm.p[pb] + (r >> 6) * (N * kRowBytes);
+        uint8_t* pbase = sm.p[pb] + (r >> 6) * (Np * kRowBytes);
         const int col = r & 63;
+        auto put = [&](int row, uint16_t bits) {
+          const int off = (row >> 3) * (8 * kRowBytes) + (row & 7) * kRowBytes +
+                          ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2;
+          *reinterpret_cast<uint16_t*>(pbase + off) = bits;
+        };
 #pragma unroll
         for (int c = 0; c < R; ++c) {
-          const int off = (c >> 3) * (8 * kRowBytes) + (c & 7) * kRowBytes + ((((col >> 3) ^ (c & 7)) & 7) << 4) +
-                          (col & 7) * 2;
-          const uint32_t two = pack2<kBf16>(pr[c], 0.f);
-          *reinterpret_cast<uint16_t*>(pbase + off) = static_cast<uint16_t>(two & 0xffffu);
+          const uint32_t hi = pack2<kBf16>(pr[c], 0.f) & 0xffffu;
+          float hi_f, unused;
+          unpack2<kBf16>(hi, hi_f, unused);
+          const uint32_t lo = pack2<kBf16>(pr[c] - hi_f, 0.f) & 0xffffu;
+          put(c, static_cast<uint16_t>(hi));
+          put(R + c, static_cast<uint16_t>(lo));
         }
       }
       // V rows past the sequence end inside the last 16-token step are zeroed
@@ -832,6 +882,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
+
+      // off the path to PV: the running max and the rescale factor of the
+      // column this lane holds (for the next chunk and the epilogue), and the
+      // running sum of p over this warp's tokens
+      {
+        const float cm = fmaxf(fmaxf(sm.red[sb][0][my_col], sm.red[sb][1][my_col]),
+                               fmaxf(sm.red[sb][2][my_col], sm.red[sb][3][my_col]));
+        const float m_old = first ? -INFINITY : m_prev[my_col];
+        const float m_new = fmaxf(m_old, cm);
+        const float alpha = fast_exp2(m_old - (m_new == -INFINITY ? 0.f : m_new));
+        if (quad == 0 && col_writer) {
+          sm.mbuf[ci & 1][my_col] = m_new;
+          sm.abuf[ci & 1][my_col] = alpha;
+        }
+        float v[R];
+#pragma unroll
+        for (int c = 0; c < R; ++c) v[c] = pr[c];
+        l_lane = fmaf(l_lane, alpha, warp_column_reduce<R, false>(v, lane));
+      }
       return true;
     };
 
@@ -841,14 +910,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool w = mbar_wait_bounded(&sm.o_full[pb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      float oN[N];
-      tmem_ld<N>(tmem + lane_base + kColO + pb * N, oN);
+      float oN[Np];
+      tmem_ld<Np>(tmem + lane_base + kColO + pb * Np, oN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[pb]);
-      const float* alpha = sm.abuf[ci & 1];
+      float alpha[R];
+      ld_row<R>(sm.abuf[ci & 1], alpha);
 #pragma unroll
-      for (int c = 0; c < R; ++c) acc[c] = fmaf(acc[c], alpha[c], oN[c]);
+      for (int c = 0; c < R; ++c) acc[c] = fmaf(acc[c], alpha[c], oN[c] + oN[R + c]);
       return true;
     };
 
@@ -985,6 +1055,7 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
 template <bool kBf16, int G, int RG, int kMode>
 Variant tc_variant() {
   constexpr int R = G * RG;
+  static_assert(smem_bytes<R>() <= kMaxSmemPerCta, "shared memory of one CTA");
   return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode>), kThreads,
                  smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode>};
 }

@@ -196,13 +196,16 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
   const int Hkv = p.num_kv_heads;
   const int nseq = src.count(p);
   long long mine = 0;
-  for (int s = tid; s < p.num_seqs; s += NT) {
-    const int raw = __ldg(p.seq_lens + s);
-    if ((raw < 0 || raw > p.max_nb * B) && cta == 0) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
-  }
-  for (int s = tid; s < nseq; s += NT) {
-    const SeqSpan sp = src.template span<B>(p, s);
-    mine += sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
+  const int nloop = nseq > p.num_seqs ? nseq : p.num_seqs;
+  for (int s = tid; s < nloop; s += NT) {
+    if (s < p.num_seqs && cta == 0) {
+      const int raw = __ldg(p.seq_lens + s);
+      if (raw < 0 || raw > p.max_nb * B) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
+    }
+    if (s < nseq) {
+      const SeqSpan sp = src.template span<B>(p, s);
+      mine += sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
+    }
   }
   long long seq_granules;
   (void)block_inclusive_scan<NT>(mine, rs, seq_granules);

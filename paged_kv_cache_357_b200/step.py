@@ -8,6 +8,8 @@ step runs, in the order the method needs:
 
     H2D copies -> pa_copy_blocks -> pa_cache_write -> pa_decode -> D2H copy
 
+(pa_decode_multi or pa_decode_shared_prefix in place of pa_decode when the
+step is built for them);
 a shared block is copied before a sample writes into it (study notes ch.05
 §6.1), the new token is stored before the decode reads it (vLLM blog,
 plain-language section), and the decode reads every block through the table
@@ -30,8 +32,8 @@ from . import _lib
 
 
 class _BufferSet:
-    def __init__(self, torch, dev, dt, S, Hq, D, Hkv, max_nb, T, P):
-        self.q = torch.empty((S, Hq, D), dtype=dt, device=dev)
+    def __init__(self, torch, dev, dt, S, Hq, D, Hkv, max_nb, T, P, q_len, grouped):
+        self.q = torch.empty((S, Hq, D) if q_len == 1 else (S, q_len, Hq, D), dtype=dt, device=dev)
         self.out = torch.empty_like(self.q)
         self.tables = torch.empty((S, max_nb), dtype=torch.int32, device=dev)
         self.lens = torch.empty((S,), dtype=torch.int32, device=dev)
@@ -39,6 +41,8 @@ class _BufferSet:
         self.new_v = torch.empty_like(self.new_k)
         self.slots = torch.empty((max(T, 1),), dtype=torch.int64, device=dev)
         self.pairs = torch.empty((max(P, 1), 2), dtype=torch.int64, device=dev)
+        self.group_starts = torch.empty((S + 1,), dtype=torch.int32, device=dev) if grouped else None
+        self.group_prefix = torch.empty((max(S, 1),), dtype=torch.int32, device=dev) if grouped else None
         self.out_host = torch.empty(self.out.shape, dtype=dt, pin_memory=True)
         self.uploaded = torch.cuda.Event()
         self.computed = torch.cuda.Event()
@@ -49,7 +53,11 @@ class _BufferSet:
 class PagedDecodeStep:
     def __init__(self, k_pool, v_pool, num_seqs: int, num_q_heads: int, max_blocks_per_seq: int,
                  max_new_tokens: int = 0, max_copy_pairs: int = 0, scale: Optional[float] = None,
-                 num_ctas: int = 0):
+                 num_ctas: int = 0, q_len: int = 1, max_group_size: int = 0):
+        """q_len > 1: each step is a multi-query step (pa_decode_multi, q is
+        [num_seqs, q_len, num_q_heads, head_dim]).  max_group_size > 0: each
+        step decodes with pa_decode_shared_prefix and takes the groups as
+        inputs.  Otherwise pa_decode."""
         import torch
 
         self.torch = torch
@@ -59,23 +67,34 @@ class PagedDecodeStep:
         self.S, self.Hq, self.D, self.Hkv = num_seqs, num_q_heads, D, Hkv
         self.scale = (1.0 / D**0.5) if scale is None else float(scale)
         self.num_ctas = num_ctas
+        if q_len > 1 and max_group_size > 0:
+            raise ValueError("a step is either multi-query or shared-prefix")
+        self.q_len, self.max_group_size = q_len, max_group_size
         self.h2d_stream = torch.cuda.Stream(device=dev)
         self.compute_stream = torch.cuda.Stream(device=dev)
         self.d2h_stream = torch.cuda.Stream(device=dev)
         self.sets = [_BufferSet(torch, dev, k_pool.dtype, num_seqs, num_q_heads, D, Hkv, max_blocks_per_seq,
-                                max_new_tokens, max_copy_pairs) for _ in range(2)]
-        self.workspace = _lib.alloc_decode_workspace(num_seqs, num_q_heads, k_pool, num_ctas)
+                                max_new_tokens, max_copy_pairs, q_len, max_group_size > 0) for _ in range(2)]
+        if q_len > 1:
+            self.workspace = _lib.alloc_multi_workspace(num_seqs, q_len, num_q_heads, k_pool, num_ctas)
+        elif max_group_size > 0:
+            self.workspace = _lib.alloc_shared_prefix_workspace(num_seqs, max_group_size, num_q_heads, k_pool,
+                                                                num_ctas)
+        else:
+            self.workspace = _lib.alloc_decode_workspace(num_seqs, num_q_heads, k_pool, num_ctas)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
         self.steps = 0
         self.last_h2d_bytes = 0
         self.last_d2h_bytes = 0
 
-    def run(self, q, block_tables, seq_lens, new_k=None, new_v=None, slot_mapping=None, copy_pairs=None):
+    def run(self, q, block_tables, seq_lens, new_k=None, new_v=None, slot_mapping=None, copy_pairs=None,
+            group_starts=None, group_prefix_blocks=None):
         """Enqueue one step from host tensors (pinned, so the copies run
         asynchronously; leave them unchanged until the step completes).
         Returns the pinned host output of this step, valid once
         ``wait(result)`` or ``synchronize()`` returns and until the step after
-        next reuses it."""
+        next reuses it.  A shared-prefix step also takes the groups (int32
+        host tensors [num_groups + 1] and [num_groups])."""
         torch = self.torch
         bs = self.sets[self.steps % 2]
         h2d = 0
@@ -85,6 +104,14 @@ class PagedDecodeStep:
             for dst, src in ((bs.q, q), (bs.tables, block_tables), (bs.lens, seq_lens)):
                 dst.copy_(src, non_blocking=True)
                 h2d += src.numel() * src.element_size()
+            n_groups = 0
+            if self.max_group_size > 0:
+                if group_starts is None or group_prefix_blocks is None:
+                    raise ValueError("a shared-prefix step needs group_starts and group_prefix_blocks")
+                n_groups = group_prefix_blocks.shape[0]
+                bs.group_starts[: n_groups + 1].copy_(group_starts, non_blocking=True)
+                bs.group_prefix[:n_groups].copy_(group_prefix_blocks, non_blocking=True)
+                h2d += (2 * n_groups + 1) * 4
             n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
             if n_pairs > 0:
                 bs.pairs[:n_pairs].copy_(copy_pairs, non_blocking=True)
@@ -108,8 +135,17 @@ class PagedDecodeStep:
             if T > 0:
                 _lib.pa_cache_write(bs.new_k[:T], bs.new_v[:T], bs.slots[:T], self.k_pool, self.v_pool, self.status,
                                     stream=self.compute_stream)
-            _lib.pa_decode(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out, self.workspace,
-                           self.status, num_ctas=self.num_ctas, stream=self.compute_stream)
+            if self.q_len > 1:
+                _lib.pa_decode_multi(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out,
+                                     self.workspace, self.status, num_ctas=self.num_ctas, stream=self.compute_stream)
+            elif self.max_group_size > 0:
+                _lib.pa_decode_shared_prefix(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens,
+                                             bs.group_starts[: n_groups + 1], bs.group_prefix[:n_groups],
+                                             self.max_group_size, self.scale, bs.out, self.workspace, self.status,
+                                             num_ctas=self.num_ctas, stream=self.compute_stream)
+            else:
+                _lib.pa_decode(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out,
+                               self.workspace, self.status, num_ctas=self.num_ctas, stream=self.compute_stream)
             bs.computed.record(self.compute_stream)
         with torch.cuda.stream(self.d2h_stream):
             self.d2h_stream.wait_event(bs.computed)

@@ -72,6 +72,7 @@ class PagedLayout:
     refcounts: Optional[np.ndarray] = None  # int32 [num_blocks] after the step (shared-prefix layouts)
     share_groups: List[List[int]] = field(default_factory=list)  # sequences sharing a prompt
     note: str = ""
+    q_len: int = 1  # query positions per sequence; q is [S, Hq, D] if 1 else [S, q_len, Hq, D]
 
     @property
     def num_seqs(self) -> int:
@@ -107,7 +108,7 @@ class PagedLayout:
 class PagedValues:
     """16-bit bit patterns (uint16 numpy) or torch tensors for one layout."""
 
-    q: object  # [S, Hq, D]
+    q: object  # [S, Hq, D], or [S, q_len, Hq, D] for a multi-query layout
     k_pool: object  # [NB, Hkv, B, D]
     v_pool: object
     new_k: object  # [T, Hkv, D]
@@ -125,22 +126,24 @@ def _ceil_div(a: int, b: int) -> int:
 
 def _finish_layout(
     name, seed, dtype, B, NB, Hq, Hkv, D, seq_lens, tables, write_new_token, copy_pairs=None,
-    refcounts=None, share_groups=None, note="", scale=None,
+    refcounts=None, share_groups=None, note="", scale=None, q_len=1,
 ) -> PagedLayout:
+    """With write_new_token, the last q_len tokens of every sequence are the
+    ones this step writes (their rows are unfilled before the step)."""
     S = seq_lens.shape[0]
     copy_pairs = np.zeros((0, 2), np.int64) if copy_pairs is None else np.asarray(copy_pairs, np.int64)
     fill = np.zeros(NB, np.int32)
     slots = []
     for s in range(S):
         n = int(seq_lens[s])
-        before = n - 1 if write_new_token else n
+        before = max(n - q_len, 0) if write_new_token else n
         for j in range(_ceil_div(n, B)):
             b = int(tables[s, j])
             rows = min(B, max(0, before - j * B))
             fill[b] = max(fill[b], rows)
         if write_new_token:
-            t = n - 1
-            slots.append(int(tables[s, t // B]) * B + t % B)
+            for t in range(before, n):
+                slots.append(int(tables[s, t // B]) * B + t % B)
     for _, dst in copy_pairs:
         fill[int(dst)] = 0
     return PagedLayout(
@@ -148,7 +151,7 @@ def _finish_layout(
         num_kv_heads=Hkv, head_dim=D, scale=(1.0 / math.sqrt(D)) if scale is None else scale,
         seq_lens=seq_lens.astype(np.int32), block_tables=tables.astype(np.int32),
         slot_mapping=np.asarray(slots, np.int64), copy_pairs=copy_pairs, block_fill=fill,
-        refcounts=refcounts, share_groups=share_groups or [], note=note,
+        refcounts=refcounts, share_groups=share_groups or [], note=note, q_len=q_len,
     )
 
 
@@ -221,10 +224,13 @@ def config_llama7b(batch: int = 64) -> PagedLayout:
                           note=f"{batch} seqs U[128,2048], 32/32 heads, D=128, B=16, bf16")
 
 
-def config_llama3_8b(batch: int = 256) -> PagedLayout:
+def config_llama3_8b(batch: int = 256, q_len: int = 1) -> PagedLayout:
     """Llama-3-8B-shaped GQA layer: 32 q heads / 8 kv heads, D=128, bf16, B=16,
     256 sequences with lognormal lengths (median 1024, sigma 0.75, clipped to
-    [16, 8192]), shuffled pool of 1.1x, and the cache write of 256 new tokens."""
+    [16, 8192]), shuffled pool of 1.1x, and the cache write of 256 new tokens.
+    With q_len > 1 (speculative verification of q_len tokens): the same
+    lengths, the last q_len tokens of each sequence written this step and
+    attended by q_len causal query positions."""
     seed = 1003
     rng = np.random.default_rng(seed)
     z = rng.standard_normal(batch)
@@ -232,9 +238,11 @@ def config_llama3_8b(batch: int = 256) -> PagedLayout:
     total = sum(_ceil_div(int(n), 16) for n in seq_lens)
     NB = int(math.ceil(1.1 * total))
     tables = _scatter_tables(rng, seq_lens, 16, NB)
-    return _finish_layout("llama3_8b", seed, "bf16", 16, NB, 32, 8, 128, seq_lens, tables, True,
+    name = "llama3_8b" if q_len == 1 else f"llama3_8b_spec{q_len}"
+    what = "cache write" if q_len == 1 else f"cache write, {q_len} causal query positions per sequence"
+    return _finish_layout(name, seed, "bf16", 16, NB, 32, 8, 128, seq_lens, tables, True, q_len=q_len,
                           note=f"{batch} seqs lognormal(median 1024, sigma 0.75) in [16,8192], "
-                               "32/8 heads, D=128, B=16, bf16, 256-token cache write")
+                               f"32/8 heads, D=128, B=16, bf16, {batch * q_len}-token {what}")
 
 
 def config_llama2_70b_shared(
@@ -313,6 +321,7 @@ CONFIGS: Dict[str, Callable[[], PagedLayout]] = {
     "tiny": config_tiny,
     "llama7b": config_llama7b,
     "llama3_8b": config_llama3_8b,
+    "llama3_8b_spec4": lambda: config_llama3_8b(q_len=4),
     "llama2_70b_shared": config_llama2_70b_shared,
     "opt13b_long_b8": lambda: config_opt13b_long(8),
     "opt13b_long_b16": lambda: config_opt13b_long(16),
@@ -336,7 +345,8 @@ def fill_values_numpy(layout: PagedLayout, value_seed: Optional[int] = None) -> 
     L = layout
     rng = np.random.default_rng([L.seed if value_seed is None else value_seed, 7])
     S, Hq, Hkv, D, B, NB = L.num_seqs, L.num_q_heads, L.num_kv_heads, L.head_dim, L.block_size, L.num_blocks
-    q = f32_to_bits(rng.standard_normal((S, Hq, D), dtype=np.float32), L.dtype)
+    q_shape = (S, Hq, D) if L.q_len == 1 else (S, L.q_len, Hq, D)
+    q = f32_to_bits(rng.standard_normal(q_shape, dtype=np.float32), L.dtype)
     nan = np.uint16(NAN_BITS[L.dtype])
     mask = _row_mask(L)[:, None, :, None]  # [NB,1,B,1]
     pools = []
@@ -360,7 +370,8 @@ def fill_values_torch(layout: PagedLayout, device, value_seed: Optional[int] = N
     g = torch.Generator(device=device)
     g.manual_seed(int(L.seed if value_seed is None else value_seed) * 7919 + 13)
     S, Hq, Hkv, D, B, NB = L.num_seqs, L.num_q_heads, L.num_kv_heads, L.head_dim, L.block_size, L.num_blocks
-    q = torch.randn((S, Hq, D), generator=g, device=device, dtype=torch.float32).to(tdt)
+    q_shape = (S, Hq, D) if L.q_len == 1 else (S, L.q_len, Hq, D)
+    q = torch.randn(q_shape, generator=g, device=device, dtype=torch.float32).to(tdt)
     mask_all = torch.from_numpy(_row_mask(L)).to(device)
     nan = float("nan")
     pools = []
@@ -400,10 +411,10 @@ def restrict_layout(layout: PagedLayout, seqs) -> PagedLayout:
         nb = L.blocks_of(s)
         tables[i, :nb] = [remap[int(b)] for b in L.block_tables[s, :nb]]
     slots = []
-    if L.num_new_tokens > 0:
-        for s in seqs:
-            slot = int(L.slot_mapping[s])
-            slots.append(remap[slot // B] * B + slot % B)
+    per = L.num_new_tokens // max(L.num_seqs, 1)  # new tokens per sequence (1, or q_len)
+    for s in seqs:
+        for slot in L.slot_mapping[s * per:(s + 1) * per]:
+            slots.append(remap[int(slot) // B] * B + int(slot) % B)
     fill = np.zeros(len(uniq), np.int32)
     for b, i in remap.items():
         fill[i] = L.block_fill[b]
@@ -412,5 +423,5 @@ def restrict_layout(layout: PagedLayout, seqs) -> PagedLayout:
         num_q_heads=L.num_q_heads, num_kv_heads=L.num_kv_heads, head_dim=L.head_dim, scale=L.scale,
         seq_lens=L.seq_lens[seqs].astype(np.int32), block_tables=tables, slot_mapping=np.asarray(slots, np.int64),
         copy_pairs=np.asarray([(remap[a], remap[b]) for a, b in pairs], np.int64).reshape(-1, 2),
-        block_fill=fill, note=f"sample of {L.name}",
+        block_fill=fill, note=f"sample of {L.name}", q_len=L.q_len,
     )
