@@ -125,6 +125,12 @@ def decode_kernel_name(L, mode: str = "plain") -> str:
     return "pa_decode_kernel (CUDA cores)"
 
 
+def decode_entry(L, mode: str) -> str:
+    if L.q_len > 1:
+        return "pa_decode_multi"
+    return "pa_decode_shared_prefix" if mode == "shared_prefix" else "pa_decode"
+
+
 def profiled_traffic(L, mode: str = "plain"):
     """dram read+write bytes per decode launch from the committed ncu summary
     of the default workload, or None for other workloads, when there is no
@@ -340,18 +346,32 @@ def run_ours(args):
 
     pa.load()
     L = make_layout(args)
+    mode = args.decode
+    if mode == "shared_prefix" and not L.share_groups:
+        raise SystemExit("--decode shared_prefix needs a workload whose sequences share prompt blocks")
+    if mode == "shared_prefix" and L.q_len > 1:
+        raise SystemExit("--decode shared_prefix is a single-position decode")
     V = fill_values_torch(L, dev, value_seed=L.seed + 7 * rank)
-    nbytes = step_bytes(L)
+    nbytes = step_bytes(L, mode)
     tables = torch.from_numpy(L.block_tables).to(dev)
     lens = torch.from_numpy(L.seq_lens).to(dev)
     slots = torch.from_numpy(L.slot_mapping).to(dev)
     pairs = torch.from_numpy(L.copy_pairs.reshape(-1, 2)).to(dev)
     out = torch.empty_like(V.q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, V.k_pool, args.num_ctas)
+    groups = None
+    if L.q_len > 1:
+        ws = pa.alloc_multi_workspace(L.num_seqs, L.q_len, L.num_q_heads, V.k_pool, args.num_ctas)
+    elif mode == "shared_prefix":
+        g_starts, g_prefix = pa.shared_prefix_groups(L.block_tables, L.seq_lens, L.block_size, args.max_group)
+        groups = (torch.from_numpy(g_starts).to(dev), torch.from_numpy(g_prefix).to(dev), g_starts, g_prefix)
+        ws = pa.alloc_shared_prefix_workspace(L.num_seqs, args.max_group, L.num_q_heads, V.k_pool, args.num_ctas)
+    else:
+        ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, V.k_pool, args.num_ctas)
     stream = torch.cuda.Stream(device=dev)
     has_copy, has_write = L.copy_pairs.shape[0] > 0, L.num_new_tokens > 0
-    launches_per_step = 1 + int(has_copy) + int(has_write)
+    decode_launches = 2 if mode == "shared_prefix" else 1
+    launches_per_step = decode_launches + int(has_copy) + int(has_write)
 
     def prologue():
         if has_copy:
@@ -360,8 +380,15 @@ def run_ours(args):
             pa.pa_cache_write(V.new_k, V.new_v, slots, V.k_pool, V.v_pool, status, stream=stream)
 
     def decode():
-        pa.pa_decode(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status, num_ctas=args.num_ctas,
-                     stream=stream)
+        if L.q_len > 1:
+            pa.pa_decode_multi(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status,
+                               num_ctas=args.num_ctas, stream=stream)
+        elif mode == "shared_prefix":
+            pa.pa_decode_shared_prefix(V.q, V.k_pool, V.v_pool, tables, lens, groups[0], groups[1], args.max_group,
+                                       L.scale, out, ws, status, num_ctas=args.num_ctas, stream=stream)
+        else:
+            pa.pa_decode(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status, num_ctas=args.num_ctas,
+                         stream=stream)
 
     def barrier():
         if world > 1:
@@ -405,13 +432,18 @@ def run_ours(args):
         new_k=V.new_k.cpu().pin_memory(), new_v=V.new_v.cpu().pin_memory(), slots=slots.cpu().pin_memory(),
         pairs=pairs.cpu().pin_memory() if has_copy else None,
     )
+    if groups is not None:
+        host["group_starts"] = torch.from_numpy(groups[2]).pin_memory()
+        host["group_prefix"] = torch.from_numpy(groups[3]).pin_memory()
     step = pa.PagedDecodeStep(V.k_pool, V.v_pool, L.num_seqs, L.num_q_heads, L.max_blocks_per_seq,
                               max_new_tokens=L.num_new_tokens, max_copy_pairs=L.copy_pairs.shape[0],
-                              scale=L.scale, num_ctas=args.num_ctas)
+                              scale=L.scale, num_ctas=args.num_ctas, q_len=L.q_len,
+                              max_group_size=args.max_group if groups is not None else 0)
 
     def e2e_step():
         return step.run(host["q"], host["tables"], host["lens"], host["new_k"], host["new_v"],
-                        host["slots"] if has_write else None, host["pairs"])
+                        host["slots"] if has_write else None, host["pairs"],
+                        group_starts=host.get("group_starts"), group_prefix_blocks=host.get("group_prefix"))
 
     for _ in range(args.warmup):
         e2e_step()
@@ -435,7 +467,7 @@ def run_ours(args):
     elapsed_ms, e2e_ms, decode_mean_ms = max_over_ranks([elapsed_ms, e2e_ms, decode_mean_ms], dev)
     ms_per_step = elapsed_ms / K
     value = whole_job_gbs(world, nbytes["step"], ms_per_step)
-    tokens_per_s = world * L.num_seqs / (ms_per_step * 1e-3)
+    tokens_per_s = world * L.num_seqs * L.q_len / (ms_per_step * 1e-3)
     peak, peak_kind = measured_hbm_peak()
     achieved = nbytes["decode"] / (decode_mean_ms * 1e-3) / 1e9
     result = None
@@ -460,17 +492,19 @@ def run_ours(args):
                 "seq_len": {"mean": float(np.mean(L.seq_lens)), "min": int(L.seq_lens.min()),
                             "max": int(L.seq_lens.max())},
                 "step": "+".join((["pa_copy_blocks"] if has_copy else []) + (["pa_cache_write"] if has_write
-                                                                             else []) + ["pa_decode"]),
+                                                                             else []) + [decode_entry(L, mode)]),
+                "q_len": L.q_len,
                 "l2": f"no flush: per-step K/V {nbytes['decode'] / 1e9:.2f} GB > 126 MB L2",
                 "parallelism": f"dp{world} (independent sequence shards, no collective)",
             },
             "tokens_per_s": tokens_per_s,
-            "tokens_per_s_note": "one new token per sequence per single-layer step",
+            "tokens_per_s_note": ("one new token per sequence per single-layer step" if L.q_len == 1 else
+                                  f"{L.q_len} query positions per sequence per single-layer step"),
             "decode_ms": decode_mean_ms,
             "decode_ms_p50": decode_ms[K // 2],
             "bytes": nbytes,
             "roofline": {
-                "kernel": decode_kernel_name(L),
+                "kernel": decode_kernel_name(L, mode),
                 "bound": "hbm",
                 "achieved": achieved,
                 "peak": peak,
@@ -478,7 +512,7 @@ def run_ours(args):
                 "unit": "GB/s",
                 "frac": achieved / peak,
                 "frac_of_8000_nominal": achieved / 8000.0,
-                "traffic": profiled_traffic(nbytes["decode"]),
+                "traffic": profiled_traffic(L, mode),
                 "algorithmic_bytes_per_launch": nbytes["decode"],
             },
             "e2e": {

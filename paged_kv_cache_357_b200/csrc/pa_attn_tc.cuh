@@ -781,7 +781,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ===================== softmax + epilogue (warps 2-5) ====================
     // Per chunk i: softmax(i) then the epilogue of chunk i-1, so the PV of
-    // chunk i-1 runs on the tensor core while the softmax of chunk i runs here.
+    // chunk i-1 runs on the tensor core while the softmax of chunk i runs
+    // here; chunks of consecutive segments form one stream.
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;   // token row of the chunk; head_dim index in the epilogue
     const int ctid = tid - 64;        // 0..127
@@ -922,39 +923,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    while (ok && next_seg<B, CB>(cur, sg, p, src)) {
-      const int rows = G * src.row_groups(p, sg.s);
-#pragma unroll
-      for (int c = 0; c < R; ++c) acc[c] = 0.f;
-      l_lane = 0.f;
-      bool pending = false;
-      for (int c0 = 0; c0 < sg.n; c0 += CB) {
-        ok = softmax_chunk(ci, chunk_at(sg, c0), c0 == 0, rows, sg.len);
-        if (!ok) break;
-        if (pending) {
-          ok = epilogue_chunk(ci - 1);
-          if (!ok) break;
-        }
-        pending = true;
-        ++ci;
-      }
-      if (ok && pending) ok = epilogue_chunk(ci - 1);
-      if (!ok) break;
-
-      // ---- end of the segment: column sums, then the rows or a partial state
-      if (col_writer) sm.lred[quad][my_col] = l_lane;
+    // The finish of a segment (column sums, then its rows or its partial
+    // state) runs after the softmax of the next segment's first chunk, so
+    // the copies and the tensor core keep streaming across unit boundaries.
+    auto finish_segment = [&](const Seg& fs, int rows, float l_sum, int last_ci) {
+      if (col_writer) sm.lred[quad][my_col] = l_sum;
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
-      const float* m_last = sm.mbuf[(ci - 1) & 1];
-      if (sg.j0 == sg.first && sg.j0 + sg.n == sg.nb) {
+      const float* m_last = sm.mbuf[last_ci & 1];
+      if (fs.j0 == fs.first && fs.j0 + fs.n == fs.nb) {
 #pragma unroll
         for (int c = 0; c < R; ++c) {
           if (c < rows) {
             const float L = (sm.lred[0][c] + sm.lred[1][c]) + (sm.lred[2][c] + sm.lred[3][c]);
-            emit_row<kBf16, G, kMode>(p, sg, c, r, m_last[c], L, acc[c]);
+            emit_row<kBf16, G, kMode>(p, fs, c, r, m_last[c], L, acc[c]);
           }
         }
       } else {
-        float* pp = p.partials + partial_slot(cta, sg.unit_first, wr) * Sh::kPartStride;
+        float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * Sh::kPartStride;
         if (ctid < R) {
           pp[ctid] = m_last[ctid];
           pp[R + ctid] = (sm.lred[0][ctid] + sm.lred[1][ctid]) + (sm.lred[2][ctid] + sm.lred[3][ctid]);
@@ -962,11 +947,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < R; ++c) pp[2 * R + c * D + r] = acc[c];
         __threadfence();
-        finish_split_unit_rows<kBf16, G, R, kMode>(p, sg, wr, rows, ctid, &sm.is_last,
+        finish_split_unit_rows<kBf16, G, R, kMode>(p, fs, wr, rows, ctid, &sm.is_last,
                                                    [] { named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads); });
       }
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+#pragma unroll
+      for (int c = 0; c < R; ++c) acc[c] = 0.f;
+    };
+
+#pragma unroll
+    for (int c = 0; c < R; ++c) acc[c] = 0.f;
+    Seg prev;               // the segment whose finish is still due
+    int prev_rows = 0;
+    bool have_prev = false;
+    bool pending = false;   // the epilogue of chunk ci - 1 is still due
+    while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+      const int rows = G * src.row_groups(p, sg.s);
+      for (int c0 = 0; c0 < sg.n; c0 += CB) {
+        const float l_before = l_lane;  // the previous segment's sum, when c0 == 0
+        ok = softmax_chunk(ci, chunk_at(sg, c0), c0 == 0, rows, sg.len);
+        if (!ok) break;
+        if (pending) {
+          ok = epilogue_chunk(ci - 1);
+          if (!ok) break;
+        }
+        if (c0 == 0 && have_prev) {
+          finish_segment(prev, prev_rows, l_before, ci - 1);
+          have_prev = false;
+        }
+        pending = true;
+        ++ci;
+      }
+      if (!ok) break;
+      prev = sg;
+      prev_rows = rows;
+      have_prev = true;
     }
+    if (ok && pending) ok = epilogue_chunk(ci - 1);
+    if (ok && have_prev) finish_segment(prev, prev_rows, l_lane, ci - 1);
     if (!ok && lane == 0) {
       sm.abort = 1;
       record_status(p.status, PA_DEV_TIMEOUT);
