@@ -72,8 +72,6 @@ constexpr int kRowBytes = 128;             // one swizzle row: 64 elements
 constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 tokens
 constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
 constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
 constexpr int kSoftmaxBarrier = 1;
 
 enum Mode { kDecode = 0, kMulti = 1, kPrefix = 2 };
@@ -96,7 +94,13 @@ struct Rows {
   static constexpr int kCols = 2 * Nq + 2 * Np;
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : 256;
   static constexpr int kPartStride = R * (D + 2);                 // floats per partial slot
-  static constexpr int kLanesPerCol = 32 / R;                     // lanes holding one column after a reduce
+  // Softmax warpgroups: one for up to 8 rows; two for 16 or 32, each taking
+  // RC = R / WG of the rows (both read every token row of S and O).
+  static constexpr int WG = R >= 16 ? 2 : 1;
+  static constexpr int RC = R / WG;
+  static constexpr int kSoftmaxThreads = 128 * WG;
+  static constexpr int kThreads = 64 + kSoftmaxThreads;          // + producer warp + MMA warp
+  static constexpr int kLanesPerCol = 32 / RC;                    // lanes holding one column after a reduce
 };
 
 template <int R>
@@ -218,13 +222,32 @@ __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 
-// Columns [0, NC) of this thread's TMEM lane, NC a multiple of 16.
+__device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Columns [0, NC) of this thread's TMEM lane (NC = 8 or a multiple of 16),
+// issued without waiting; tmem_wait_ld() completes them.
+template <int NC>
+__device__ __forceinline__ void tmem_ld_nowait(uint32_t taddr, uint32_t* r) {
+  if constexpr (NC == 8) {
+    tmem_ld8_nowait(taddr, r);
+  } else {
+    static_assert(NC % 16 == 0, "8 or a multiple of 16 columns");
+#pragma unroll
+    for (int c = 0; c < NC; c += 16) tmem_ld16_nowait(taddr + c, r + c);
+  }
+}
+
 template <int NC>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, float* v) {
   uint32_t r[NC];
-#pragma unroll
-  for (int c = 0; c < NC; c += 16) tmem_ld16_nowait(taddr + c, r + c);
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  tmem_ld_nowait<NC>(taddr, r);
+  tmem_wait_ld();
 #pragma unroll
   for (int i = 0; i < NC; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -385,7 +408,7 @@ struct Source<kPrefix, RG> {
 // is handled by thread g / gridDim.x of CTA g % gridDim.x.
 template <int BB, int RG>
 __device__ void prefix_bookkeeping(const DecodeParams& p) {
-  const long long stride = static_cast<long long>(gridDim.x) * kThreads;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long g = static_cast<long long>(threadIdx.x) * gridDim.x + blockIdx.x; g < p.num_groups; g += stride) {
     const int s0 = __ldg(p.group_starts + g), s1 = __ldg(p.group_starts + g + 1);
     if (s0 < 0 || s1 < s0 || s1 > p.num_seqs || s1 - s0 > RG) record_status(p.status, PA_DEV_BAD_GROUP);
@@ -404,7 +427,7 @@ __device__ void prefix_bookkeeping(const DecodeParams& p) {
 template <int kMode, int RG>
 __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>& src) {
   const long long nctas = gridDim.x, cta = blockIdx.x;
-  for (int s = threadIdx.x; s < p.num_seqs; s += kThreads) {
+  for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
     if ((s % nctas) != cta) continue;
     if constexpr (kMode == kMulti) {
       const int raw = __ldg(p.seq_lens + s);
@@ -420,47 +443,73 @@ __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>&
 
 // ---- unit results --------------------------------------------------------------
 
-// Row c of the unit in segment sg, head_dim element d, from its state
-// (m, L, unnormalised a): the normalised output (merged first with the shared
-// prefix's state when the unit skipped one), or, in kPrefix, the state itself.
-template <bool kBf16, int G, int kMode>
-__device__ __forceinline__ void emit_row(const DecodeParams& p, const Seg& sg, int c, int d, float m, float L,
-                                         float a) {
-  const int rg = c / G, g = c % G;
+// Rows col0 .. col0 + RC - 1 of the unit in segment sg (those below `rows`),
+// head_dim element d, from their states (m, L, unnormalised a): the
+// normalised outputs — merged first with the shared prefix's states when the
+// unit skipped a prefix — or, in kPrefix, the states themselves.  Every load
+// is issued before any result is formed, so a thread waits on memory once.
+template <bool kBf16, int G, int RC, int kMode>
+__device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, int col0, int rows, int d,
+                                          const float (&m)[RC], float (&L)[RC], float (&a)[RC]) {
   const int Hq = p.num_q_heads;
-  const int head = sg.h * G + g;
   if constexpr (kMode == kPrefix) {
-    const int s = __ldg(p.group_starts + sg.s) + rg;
-    float* pp = p.prefix_part + (static_cast<size_t>(s) * Hq + head) * (D + 2);
-    if (d == 0) {
-      pp[0] = m;
-      pp[1] = L;
+    const int s0 = __ldg(p.group_starts + sg.s);
+#pragma unroll
+    for (int k = 0; k < RC; ++k) {
+      const int c = col0 + k;
+      if (c < rows) {
+        float* pp = p.prefix_part + (static_cast<size_t>(s0 + c / G) * Hq + sg.h * G + c % G) * (D + 2);
+        if (d == 0) {
+          pp[0] = m[k];
+          pp[1] = L[k];
+        }
+        pp[2 + d] = a[k];
+      }
     }
-    pp[2 + d] = a;
   } else {
     if constexpr (kMode == kDecode) {
       if (sg.first > 0) {
-        const float* pp = p.prefix_part + (static_cast<size_t>(sg.s) * Hq + head) * (D + 2);
-        const float pm = __ldcg(pp), pl = __ldcg(pp + 1), pa = __ldcg(pp + 2 + d);
-        const float M = fmaxf(m, pm);
-        const float w0 = fast_exp2(m - M), w1 = fast_exp2(pm - M);
-        a = a * w0 + pa * w1;
-        L = L * w0 + pl * w1;
+        float pm[RC], pl[RC], pa[RC];
+#pragma unroll
+        for (int k = 0; k < RC; ++k) {
+          const int c = col0 + k;
+          const float* pp = p.prefix_part + (static_cast<size_t>(sg.s) * Hq + sg.h * G + c) * (D + 2);
+          const bool on = c < rows;
+          pm[k] = on ? __ldcg(pp) : 0.f;
+          pl[k] = on ? __ldcg(pp + 1) : 0.f;
+          pa[k] = on ? __ldcg(pp + 2 + d) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < RC; ++k) {
+          const float M = fmaxf(m[k], pm[k]);
+          const float w0 = fast_exp2(m[k] - M), w1 = fast_exp2(pm[k] - M);
+          a[k] = a[k] * w0 + pa[k] * w1;
+          L[k] = L[k] * w0 + pl[k] * w1;
+        }
       }
     }
-    const size_t row = (kMode == kMulti) ? static_cast<size_t>(sg.s) * p.q_len + rg : static_cast<size_t>(sg.s);
-    const uint32_t two = pack2<kBf16>(a / L, 0.f);
-    p.out[(row * Hq + head) * D + d] = static_cast<uint16_t>(two & 0xffffu);
+#pragma unroll
+    for (int k = 0; k < RC; ++k) {
+      const int c = col0 + k;
+      if (c < rows) {
+        const int rg = c / G;
+        const size_t row = (kMode == kMulti) ? static_cast<size_t>(sg.s) * p.q_len + rg : static_cast<size_t>(sg.s);
+        const uint32_t two = pack2<kBf16>(a[k] / L[k], 0.f);
+        p.out[(row * Hq + sg.h * G + c % G) * D + d] = static_cast<uint16_t>(two & 0xffffu);
+      }
+    }
   }
 }
 
-// Called by the 128 softmax threads after this CTA's partial state of a split
+// Called by every softmax thread after this CTA's partial state of a split
 // unit is written and fenced.  The last CTA to arrive merges every partial
 // state of the unit (the rescale rule of the online softmax, per row and
-// head_dim element; thread = element) and emits the rows.
-template <bool kBf16, int G, int R, int kMode, typename Sync>
+// head_dim element) and emits the rows: thread (d, col0) takes element d of
+// rows col0 .. col0 + RC - 1.  Every row is merged at once, so each pass over
+// the partial states costs one memory round trip per CTA piece.
+template <bool kBf16, int G, int R, int RC, int kMode, typename Sync>
 __device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, const WorkRange& wr, int rows,
-                                       int ctid, int* is_last, Sync sync) {
+                                       int ctid, int d, int col0, int* is_last, Sync sync) {
   constexpr int kStride = Rows<R>::kPartStride;
   const long long F = sg.unit_first;
   const long long first = cta_of(F, wr.total, wr.nparts);
@@ -474,36 +523,31 @@ __device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, con
   sync();
   if (*is_last) {
     __threadfence();
-    // every row at once, so each pass over the partial states costs one
-    // memory round trip per CTA piece rather than one per row
-    const int d = ctid;
-    float M[R], L[R], a[R];
+    float M[RC], L[RC], a[RC];
 #pragma unroll
-    for (int c = 0; c < R; ++c) {
-      M[c] = -INFINITY;
-      L[c] = 0.f;
-      a[c] = 0.f;
+    for (int k = 0; k < RC; ++k) {
+      M[k] = -INFINITY;
+      L[k] = 0.f;
+      a[k] = 0.f;
     }
     for (long long cc = first; cc <= last; ++cc) {
       const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
 #pragma unroll
-      for (int c = 0; c < R; ++c) M[c] = fmaxf(M[c], __ldcg(pp + c));
+      for (int k = 0; k < RC; ++k) M[k] = fmaxf(M[k], __ldcg(pp + col0 + k));
     }
     for (long long cc = first; cc <= last; ++cc) {
       const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
 #pragma unroll
-      for (int c = 0; c < R; ++c) {
+      for (int k = 0; k < RC; ++k) {
+        const int c = col0 + k;
         if (c < rows) {
-          const float w = fast_exp2(__ldcg(pp + c) - M[c]);
-          L[c] = fmaf(__ldcg(pp + R + c), w, L[c]);
-          a[c] = fmaf(__ldcg(pp + 2 * R + c * D + d), w, a[c]);
+          const float w = fast_exp2(__ldcg(pp + c) - M[k]);
+          L[k] = fmaf(__ldcg(pp + R + c), w, L[k]);
+          a[k] = fmaf(__ldcg(pp + 2 * R + c * D + d), w, a[k]);
         }
       }
     }
-#pragma unroll
-    for (int c = 0; c < R; ++c) {
-      if (c < rows) emit_row<kBf16, G, kMode>(p, sg, c, d, M[c], L[c], a[c]);
-    }
+    emit_rows<kBf16, G, RC, kMode>(p, sg, col0, rows, d, M, L, a);
     if (ctid == 0) *counter = 0;
   }
 }
@@ -511,12 +555,14 @@ __device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, con
 // ---- the kernel ---------------------------------------------------------------
 
 template <bool kBf16, int G, int RG, int kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     pa_decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_q,
                         const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
   constexpr int R = G * RG;
   using Sh = Rows<R>;
   constexpr int Nq = Sh::Nq, Np = Sh::Np, kVStages = Sh::kVStages, kLanesPerCol = Sh::kLanesPerCol;
+  constexpr int WG = Sh::WG, RC = Sh::RC, kThreads = Sh::kThreads, kSoftmaxThreads = Sh::kSoftmaxThreads;
+  constexpr int RL = RC < 8 ? 8 : RC;  // TMEM columns loaded per row set (x8 is the narrowest load used)
   static_assert(kMode != kDecode || RG == 1, "a decode unit has one row group");
   using Smem = TcSmem<R>;
   const Source<kMode, RG> src;
@@ -543,10 +589,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qempty[i], 1);
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 4);
-      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.s_free[i], 4 * WG);  // one arrival per softmax warp
+      mbar_init(&sm.p_full[i], 4 * WG);
       mbar_init(&sm.o_full[i], 1);
-      mbar_init(&sm.o_free[i], 4);
+      mbar_init(&sm.o_free[i], 4 * WG);
     }
     mbar_init(&sm.mma_done, 1);
     sm.abort = 0;
@@ -785,14 +831,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // here; chunks of consecutive segments form one stream.
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;   // token row of the chunk; head_dim index in the epilogue
-    const int ctid = tid - 64;        // 0..127
+    const int ctid = tid - 64;        // 0 .. kSoftmaxThreads - 1
+    const int col0 = ((warp - 2) / 4) * RC;  // this warpgroup's query rows: col0 .. col0 + RC - 1
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int my_col = lane / kLanesPerCol;  // the column this lane holds after a reduce
+    const int my_col = col0 + lane / kLanesPerCol;  // the row this lane holds after a reduce
     const bool col_writer = (lane % kLanesPerCol) == 0;
     bool ok = true;
     int ci = 0;
     Seg sg;
-    float acc[R];
+    float acc[RC];
     float l_lane = 0.f;  // running sum of p over this warp's tokens, column my_col
 
     // Online softmax of chunk ci (the first of its segment when `first`):
@@ -804,48 +851,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      float sN[Nq];
-      tmem_ld<Nq>(tmem + lane_base + kColS + sb * Nq, sN);
+      float sN[RL];
+      tmem_ld<RL>(tmem + lane_base + kColS + sb * Nq + col0, sN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[sb]);
 
       // scores of this token row for every query row (log2 domain), masked
       const int t = ch.j * B + r;  // token index in the sequence
-      float sc[R];
+      float sc[RC];
 #pragma unroll
-      for (int c = 0; c < R; ++c) {
+      for (int k = 0; k < RC; ++k) {
+        const int c = col0 + k;
         const bool valid = c < rows && r < ch.ntok && t <= src.limit(p, c / G, len);
-        sc[c] = valid ? sN[c] * p.scale_log2 : -INFINITY;
+        sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
       }
       {
-        float v[R];
+        float v[RC];
 #pragma unroll
-        for (int c = 0; c < R; ++c) v[c] = sc[c];
-        const float wm = warp_column_reduce<R, true>(v, lane);
+        for (int k = 0; k < RC; ++k) v[k] = sc[k];
+        const float wm = warp_column_reduce<RC, true>(v, lane);
         if (col_writer) sm.red[sb][quad][my_col] = wm;
       }
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
       // new running max of every query row: the chunk's maxima of the four
       // warps and the running max before the chunk
       const float* m_prev = sm.mbuf[(ci - 1) & 1];
-      float pr[R];
+      float pr[RC];
       {
-        float cm[R], t[R];
-        ld_row<R>(sm.red[sb][0], cm);
+        float cm[RC], t[RC];
+        ld_row<RC>(sm.red[sb][0] + col0, cm);
 #pragma unroll
         for (int w = 1; w < 4; ++w) {
-          ld_row<R>(sm.red[sb][w], t);
+          ld_row<RC>(sm.red[sb][w] + col0, t);
 #pragma unroll
-          for (int c = 0; c < R; ++c) cm[c] = fmaxf(cm[c], t[c]);
+          for (int k = 0; k < RC; ++k) cm[k] = fmaxf(cm[k], t[k]);
         }
         if (!first) {
-          ld_row<R>(m_prev, t);
+          ld_row<RC>(m_prev + col0, t);
 #pragma unroll
-          for (int c = 0; c < R; ++c) cm[c] = fmaxf(cm[c], t[c]);
+          for (int k = 0; k < RC; ++k) cm[k] = fmaxf(cm[k], t[k]);
         }
 #pragma unroll
-        for (int c = 0; c < R; ++c) pr[c] = fast_exp2(sc[c] - (cm[c] == -INFINITY ? 0.f : cm[c]));
+        for (int k = 0; k < RC; ++k) pr[k] = fast_exp2(sc[k] - (cm[k] == -INFINITY ? 0.f : cm[k]));
       }
       // P^T: row c = head of query row c's probability, row R + c = its
       // rounding residual; column = token
@@ -859,18 +907,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint16_t*>(pbase + off) = bits;
         };
 #pragma unroll
-        for (int c = 0; c < R; ++c) {
-          const uint32_t hi = pack2<kBf16>(pr[c], 0.f) & 0xffffu;
+        for (int k = 0; k < RC; ++k) {
+          const uint32_t hi = pack2<kBf16>(pr[k], 0.f) & 0xffffu;
           float hi_f, unused;
           unpack2<kBf16>(hi, hi_f, unused);
-          const uint32_t lo = pack2<kBf16>(pr[c] - hi_f, 0.f) & 0xffffu;
-          put(c, static_cast<uint16_t>(hi));
-          put(R + c, static_cast<uint16_t>(lo));
+          const uint32_t lo = pack2<kBf16>(pr[k] - hi_f, 0.f) & 0xffffu;
+          put(col0 + k, static_cast<uint16_t>(hi));
+          put(R + col0 + k, static_cast<uint16_t>(lo));
         }
       }
       // V rows past the sequence end inside the last 16-token step are zeroed
       // so that 0 * (whatever they hold) cannot reach the output
-      if ((ch.ntok & 15) != 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
+      if (col0 == 0 && (ch.ntok & 15) != 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
         (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
         uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + r * kRowBytes);
         uint4* v1 = reinterpret_cast<uint4*>(sm.vbuf[vs] + kHalfBytes + r * kRowBytes);
@@ -897,10 +945,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm.mbuf[ci & 1][my_col] = m_new;
           sm.abuf[ci & 1][my_col] = alpha;
         }
-        float v[R];
+        float v[RC];
 #pragma unroll
-        for (int c = 0; c < R; ++c) v[c] = pr[c];
-        l_lane = fmaf(l_lane, alpha, warp_column_reduce<R, false>(v, lane));
+        for (int k = 0; k < RC; ++k) v[k] = pr[k];
+        l_lane = fmaf(l_lane, alpha, warp_column_reduce<RC, false>(v, lane));
       }
       return true;
     };
@@ -911,15 +959,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool w = mbar_wait_bounded(&sm.o_full[pb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      float oN[Np];
-      tmem_ld<Np>(tmem + lane_base + kColO + pb * Np, oN);
+      // this warpgroup's rows: head columns col0.., residual columns R + col0..
+      uint32_t oh[RL], ol[RL];
+      tmem_ld_nowait<RL>(tmem + lane_base + kColO + pb * Np + col0, oh);
+      tmem_ld_nowait<RL>(tmem + lane_base + kColO + pb * Np + R + col0, ol);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[pb]);
-      float alpha[R];
-      ld_row<R>(sm.abuf[ci & 1], alpha);
+      float alpha[RC];
+      ld_row<RC>(sm.abuf[ci & 1] + col0, alpha);
 #pragma unroll
-      for (int c = 0; c < R; ++c) acc[c] = fmaf(acc[c], alpha[c], oN[c] + oN[R + c]);
+      for (int k = 0; k < RC; ++k)
+        acc[k] = fmaf(acc[k], alpha[k], __uint_as_float(oh[k]) + __uint_as_float(ol[k]));
       return true;
     };
 
@@ -931,13 +983,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
       const float* m_last = sm.mbuf[last_ci & 1];
       if (fs.j0 == fs.first && fs.j0 + fs.n == fs.nb) {
+        float m[RC], L[RC];
+        ld_row<RC>(m_last + col0, m);
 #pragma unroll
-        for (int c = 0; c < R; ++c) {
-          if (c < rows) {
-            const float L = (sm.lred[0][c] + sm.lred[1][c]) + (sm.lred[2][c] + sm.lred[3][c]);
-            emit_row<kBf16, G, kMode>(p, fs, c, r, m_last[c], L, acc[c]);
-          }
+        for (int k = 0; k < RC; ++k) {
+          const int c = col0 + k;
+          L[k] = (sm.lred[0][c] + sm.lred[1][c]) + (sm.lred[2][c] + sm.lred[3][c]);
         }
+        emit_rows<kBf16, G, RC, kMode>(p, fs, col0, rows, r, m, L, acc);
       } else {
         float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * Sh::kPartStride;
         if (ctid < R) {
@@ -945,18 +998,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           pp[R + ctid] = (sm.lred[0][ctid] + sm.lred[1][ctid]) + (sm.lred[2][ctid] + sm.lred[3][ctid]);
         }
 #pragma unroll
-        for (int c = 0; c < R; ++c) pp[2 * R + c * D + r] = acc[c];
+        for (int k = 0; k < RC; ++k) pp[2 * R + (col0 + k) * D + r] = acc[k];
         __threadfence();
-        finish_split_unit_rows<kBf16, G, R, kMode>(p, fs, wr, rows, ctid, &sm.is_last,
-                                                   [] { named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads); });
+        finish_split_unit_rows<kBf16, G, R, RC, kMode>(
+            p, fs, wr, rows, ctid, r, col0, &sm.is_last,
+            [] { named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads); });
       }
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
 #pragma unroll
-      for (int c = 0; c < R; ++c) acc[c] = 0.f;
+      for (int k = 0; k < RC; ++k) acc[k] = 0.f;
     };
 
 #pragma unroll
-    for (int c = 0; c < R; ++c) acc[c] = 0.f;
+    for (int k = 0; k < RC; ++k) acc[k] = 0.f;
     Seg prev;               // the segment whose finish is still due
     int prev_rows = 0;
     bool have_prev = false;
@@ -1066,7 +1120,7 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
       !make_map(&mv, prm.v_pool, 2, kv_outer, kv_box, kBf16)) {
     return cudaErrorInvalidValue;
   }
-  return launch_overlapped(pa_decode_tc_kernel<kBf16, G, RG, kMode>, dim3(ctas), dim3(kThreads),
+  return launch_overlapped(pa_decode_tc_kernel<kBf16, G, RG, kMode>, dim3(ctas), dim3(Rows<G * RG>::kThreads),
                            static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
 }
 
@@ -1074,7 +1128,7 @@ template <bool kBf16, int G, int RG, int kMode>
 Variant tc_variant() {
   constexpr int R = G * RG;
   static_assert(smem_bytes<R>() <= kMaxSmemPerCta, "shared memory of one CTA");
-  return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode>), kThreads,
+  return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode>), Rows<R>::kThreads,
                  smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode>};
 }
 
