@@ -16,12 +16,12 @@ plain-language section), and the decode reads every block through the table
 (vLLM blog §"关键细节" 2).
 
 Consecutive steps overlap their copies with each other's kernels: the
-per-step device buffers come in two sets used alternately, uploads run on
-one stream, kernels on a second and downloads on a third.  Events order the
-work: a step's kernels wait for its uploads and for the previous step's
-kernels (they share the pools); its download waits for its kernels; the
-upload into a buffer set waits until the kernels that read that set two
-steps earlier are done.
+per-step device buffers come in several sets (three by default) used in
+turn, uploads run on one stream, kernels on a second and downloads on a
+third.  Events order the work: a step's kernels wait for its uploads and for
+the previous step's kernels (they share the pools); its download waits for
+its kernels; the upload into a buffer set waits until the kernels that last
+read that set are done, so an upload has the time of (sets - 1) steps.
 """
 
 from __future__ import annotations
@@ -53,7 +53,7 @@ class _BufferSet:
 class PagedDecodeStep:
     def __init__(self, k_pool, v_pool, num_seqs: int, num_q_heads: int, max_blocks_per_seq: int,
                  max_new_tokens: int = 0, max_copy_pairs: int = 0, scale: Optional[float] = None,
-                 num_ctas: int = 0, q_len: int = 1, max_group_size: int = 0):
+                 num_ctas: int = 0, q_len: int = 1, max_group_size: int = 0, num_buffer_sets: int = 3):
         """q_len > 1: each step is a multi-query step (pa_decode_multi, q is
         [num_seqs, q_len, num_q_heads, head_dim]).  max_group_size > 0: each
         step decodes with pa_decode_shared_prefix and takes the groups as
@@ -73,8 +73,11 @@ class PagedDecodeStep:
         self.h2d_stream = torch.cuda.Stream(device=dev)
         self.compute_stream = torch.cuda.Stream(device=dev)
         self.d2h_stream = torch.cuda.Stream(device=dev)
+        if num_buffer_sets < 2:
+            raise ValueError("at least two buffer sets")
         self.sets = [_BufferSet(torch, dev, k_pool.dtype, num_seqs, num_q_heads, D, Hkv, max_blocks_per_seq,
-                                max_new_tokens, max_copy_pairs, q_len, max_group_size > 0) for _ in range(2)]
+                                max_new_tokens, max_copy_pairs, q_len, max_group_size > 0)
+                     for _ in range(num_buffer_sets)]
         if q_len > 1:
             self.workspace = _lib.alloc_multi_workspace(num_seqs, q_len, num_q_heads, k_pool, num_ctas)
         elif max_group_size > 0:
@@ -92,15 +95,15 @@ class PagedDecodeStep:
         """Enqueue one step from host tensors (pinned, so the copies run
         asynchronously; leave them unchanged until the step completes).
         Returns the pinned host output of this step, valid once
-        ``wait(result)`` or ``synchronize()`` returns and until the step after
-        next reuses it.  A shared-prefix step also takes the groups (int32
+        ``wait(result)`` or ``synchronize()`` returns and until its buffer set
+        comes round again (``len(self.sets)`` steps later).  A shared-prefix step also takes the groups (int32
         host tensors [num_groups + 1] and [num_groups])."""
         torch = self.torch
-        bs = self.sets[self.steps % 2]
+        bs = self.sets[self.steps % len(self.sets)]
         h2d = 0
         with torch.cuda.stream(self.h2d_stream):
             if bs.used:
-                self.h2d_stream.wait_event(bs.computed)  # kernels of two steps ago read this set
+                self.h2d_stream.wait_event(bs.computed)  # the kernels that last read this set
             for dst, src in ((bs.q, q), (bs.tables, block_tables), (bs.lens, seq_lens)):
                 dst.copy_(src, non_blocking=True)
                 h2d += src.numel() * src.element_size()

@@ -7,8 +7,9 @@ Conventions (the same on both sides of every comparison):
   notes ch.05 §3 and §9.2; vLLM blog §"关键细节" 2) "PagedAttention 算子").
 * ``seq_lens[s]`` counts every token the decode step attends, the newest one
   included.  When a layout writes new tokens, token ``seq_lens[s] - 1`` of each
-  sequence is the one written this step: its row is NaN in the pool until the
-  cache write stores it.
+  sequence is the one written this step (the last ``q_len`` tokens for a
+  multi-query layout): its row is NaN in the pool until the cache write
+  stores it.
 * Pool layout is ``[num_blocks, num_kv_heads, block_size, head_dim]``.  Rows
   that hold no token and blocks that no table references are NaN, so a kernel
   that reads past ``seq_lens`` or multiplies a masked V row by zero shows up.
@@ -184,8 +185,11 @@ def random_layout(
     write_new_token: bool = True,
     scale: Optional[float] = None,
     name: str = "random",
+    q_len: int = 1,
 ) -> PagedLayout:
-    """A layout with the given decode lengths scattered over a shuffled pool."""
+    """A layout with the given decode lengths scattered over a shuffled pool
+    (with q_len > 1: q_len query positions per sequence, and the last q_len
+    tokens of each sequence written this step when write_new_token)."""
     rng = np.random.default_rng(seed)
     seq_lens = np.asarray(seq_lens, np.int32)
     B = block_size
@@ -194,7 +198,7 @@ def random_layout(
     tables = _scatter_tables(rng, seq_lens, B, NB, max_blocks_per_seq)
     return _finish_layout(
         name, seed, dtype, B, NB, num_q_heads, num_kv_heads, head_dim, seq_lens, tables,
-        write_new_token and seq_lens.size > 0 and int(seq_lens.min()) > 0, scale=scale,
+        write_new_token and seq_lens.size > 0 and int(seq_lens.min()) >= q_len, scale=scale, q_len=q_len,
     )
 
 
