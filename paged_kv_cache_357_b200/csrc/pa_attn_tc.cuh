@@ -88,7 +88,15 @@ struct Rows {
   static constexpr int Np = 2 * R < 16 ? 16 : 2 * R;              // MMA N of PV (P head + tail rows)
   static constexpr int kVStages = Np == 64 ? 3 : 4;               // V is held until its PV completes
   static constexpr int kQSlotBytes = 2 * Nq * kRowBytes;          // two 64-column halves
-  static constexpr int kPSlotBytes = 2 * Np * kRowBytes;          // tokens [0, 64) and [64, 128)
+  // P^T is stored MN-major: one row of Np 16-bit values per token, swizzled
+  // in 16-byte chunks with the pattern whose width is the row (32, 64 or 128 B)
+  static constexpr int kPRowBytes = Np * 2;
+  static constexpr int kPSlotBytes = kChunkTok * kPRowBytes;
+  static constexpr uint32_t kPLayout = Np == 16 ? 6u : Np == 32 ? 4u : 2u;  // 32B, 64B, 128B swizzle
+  // chunk index XOR for token row t (address bits [4, 4 + b) ^= bits [7, 7 + b))
+  __device__ static __forceinline__ int p_swizzle(int t) {
+    return Np == 16 ? ((t >> 2) & 1) : Np == 32 ? ((t >> 1) & 3) : (t & 7);
+  }
   static constexpr int kColS = 0;                                 // S[0], S[1]: Nq columns each
   static constexpr int kColO = 2 * Nq;                            // O[0], O[1]: Np columns each
   static constexpr int kCols = 2 * Nq + 2 * Np;
@@ -252,19 +260,27 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float* v) {
   for (int i = 0; i < NC; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version 1.
-// lbo/sbo in bytes: lbo = distance between 64-element column groups of an
-// MN-major operand (unused for K-major), sbo = distance between 8-row groups.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor, sm_100 version 1, swizzle layout code
+// `layout` (2 = 128 B, 4 = 64 B, 6 = 32 B).  lbo/sbo in bytes: lbo = distance
+// between swizzle-atom-wide column groups of an MN-major operand (unused for
+// K-major, and when the operand is one atom wide), sbo = distance between
+// 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+         (static_cast<uint64_t>(layout & 7u) << 61);
+}
+
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc(saddr, lbo, sbo, 2u);
 }
 
 // Instruction descriptor of kind::f16: fp32 accumulate, A/B both bf16 or both
-// fp16, B K-major, A K-major (QK) or MN-major (PV), M = 128, N = n.
-__host__ __device__ constexpr uint32_t make_idesc(bool bf16, bool a_mn_major, int n) {
+// fp16, each K-major or MN-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t make_idesc(bool bf16, bool a_mn_major, bool b_mn_major, int n) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
-         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
 // Reduce R values per lane over the warp by a butterfly reduce-scatter:
@@ -727,8 +743,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     // still waiting (its P written, its V landed, its O buffer free) can go,
     // and issues whichever can, so PV of chunk i never waits for chunk i+1.
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = make_idesc(kBf16, false, Nq);
-      constexpr uint32_t kIdescPV = make_idesc(kBf16, true, Np);
+      constexpr uint32_t kIdescQK = make_idesc(kBf16, false, false, Nq);  // K: K-major A, q: K-major B
+      constexpr uint32_t kIdescPV = make_idesc(kBf16, true, true, Np);    // V: MN-major A, P: MN-major B
       bool ok = true;
       int qk = 0, pv = 0, seg_i = 0, q_consumed = 0;
       uint32_t ring = 0;  // valid tokens of each pending chunk (index & 3), 8 bits each
@@ -793,7 +809,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
             const int nks = (ntok + 15) / 16;
             for (int k = 0; k < nks; ++k) {
               const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
-              const uint64_t b = sw128_desc(p0 + (k >> 2) * Np * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+              // tokens [16k, 16k + 16): two groups of 8 token rows; Np fits one swizzle atom
+              const uint64_t b = smem_desc(p0 + k * 16 * Sh::kPRowBytes, 0, 8 * Sh::kPRowBytes, Sh::kPLayout);
               umma(tmem + kColO + pb * Np, a, b, kIdescPV, k > 0 ? 1u : 0u);
             }
             umma_commit(&sm.o_full[pb]);
@@ -895,25 +912,38 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
 #pragma unroll
         for (int k = 0; k < RC; ++k) pr[k] = fast_exp2(sc[k] - (cm[k] == -INFINITY ? 0.f : cm[k]));
       }
-      // P^T: row c = head of query row c's probability, row R + c = its
-      // rounding residual; column = token
+      // P^T, MN-major: token row r holds at position c the head of query row
+      // c's probability and at R + c its rounding residual, written as whole
+      // 16-byte chunks of 8 values (this warpgroup's rows col0 .. col0 + RC)
       const int pb = ci & 1;
       {
-        uint8_t* pbase = sm.p[pb] + (r >> 6) * (Np * kRowBytes);
-        const int col = r & 63;
-        auto put = [&](int row, uint16_t bits) {
-          const int off = (row >> 3) * (8 * kRowBytes) + (row & 7) * kRowBytes +
-                          ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2;
-          *reinterpret_cast<uint16_t*>(pbase + off) = bits;
-        };
+        uint8_t* prow = sm.p[pb] + r * Sh::kPRowBytes;
+        const int swz = Sh::p_swizzle(r);
+        constexpr int kW = (RC + 1) / 2;  // 32-bit words of RC 16-bit values
+        uint32_t hw[kW], lw[kW];
 #pragma unroll
-        for (int k = 0; k < RC; ++k) {
-          const uint32_t hi = pack2<kBf16>(pr[k], 0.f) & 0xffffu;
-          float hi_f, unused;
-          unpack2<kBf16>(hi, hi_f, unused);
-          const uint32_t lo = pack2<kBf16>(pr[k] - hi_f, 0.f) & 0xffffu;
-          put(col0 + k, static_cast<uint16_t>(hi));
-          put(R + col0 + k, static_cast<uint16_t>(lo));
+        for (int k = 0; k < kW; ++k) {
+          const float a0 = pr[2 * k], a1 = (2 * k + 1 < RC) ? pr[2 * k + 1] : 0.f;
+          hw[k] = pack2<kBf16>(a0, a1);
+          float h0, h1;
+          unpack2<kBf16>(hw[k], h0, h1);
+          lw[k] = pack2<kBf16>(a0 - h0, a1 - h1);
+        }
+        auto put = [&](int chunk, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ swz) << 4)) = make_uint4(w0, w1, w2, w3);
+        };
+        if constexpr (RC >= 8) {
+#pragma unroll
+          for (int j = 0; j < RC / 8; ++j) {
+            put(col0 / 8 + j, hw[4 * j], hw[4 * j + 1], hw[4 * j + 2], hw[4 * j + 3]);
+            put((R + col0) / 8 + j, lw[4 * j], lw[4 * j + 1], lw[4 * j + 2], lw[4 * j + 3]);
+          }
+        } else if constexpr (RC == 4) {  // heads 0..3, residuals 4..7
+          put(0, hw[0], hw[1], lw[0], lw[1]);
+        } else if constexpr (RC == 2) {  // heads 0..1, residuals 2..3
+          put(0, hw[0], lw[0], 0u, 0u);
+        } else {  // one row: head 0, residual 1
+          put(0, (hw[0] & 0xffffu) | (lw[0] << 16), 0u, 0u, 0u);
         }
       }
       // V rows past the sequence end inside the last 16-token step are zeroed
