@@ -529,7 +529,7 @@ __device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, con
   constexpr int kStride = Rows<R>::kPartStride;
   const long long F = sg.unit_first;
   const long long first = cta_of(F, wr.total, wr.nparts);
-  const long long last = cta_of(F + sg.ng - 1, wr.total, wr.nparts);
+  const long long last = cta_of(sg.unit_last, wr.total, wr.nparts);
   int32_t* counter = p.counters + static_cast<size_t>(sg.s) * p.num_kv_heads + sg.h;
   sync();
   if (ctid == 0) {
@@ -1154,12 +1154,22 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
                            static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
 }
 
+// Partition cost of finishing a unit, in 1/8 granules: what the finish (row
+// sums, outputs or partial state, the merge) adds to a CTA's time beyond
+// what the pipeline hides; it grows with the rows a unit carries.  Values
+// from sweeps on B200 (Llama-3-8B decode: 2 to 3 best; q_len 4 multi-query
+// at 16 rows: 6; the prefix pass was insensitive).
+constexpr int unit_finish_cost(int kMode, int R) {
+  return kMode == kDecode ? (R <= 4 ? 2 : 4) : kMode == kPrefix ? 8 : (R <= 8 ? 4 : R <= 16 ? 6 : 10);
+}
+
 template <bool kBf16, int G, int RG, int kMode>
 Variant tc_variant() {
   constexpr int R = G * RG;
   static_assert(smem_bytes<R>() <= kMaxSmemPerCta, "shared memory of one CTA");
   return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode>), Rows<R>::kThreads,
-                 smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode>};
+                 smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode>,
+                 unit_finish_cost(kMode, R)};
 }
 
 inline bool tc_pool_ok(const pa_pool_desc& pool) {

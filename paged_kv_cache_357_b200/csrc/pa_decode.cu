@@ -441,7 +441,7 @@ template <bool kBf16, int D, int B, int G>
 Variant make_variant() {
   return Variant{reinterpret_cast<const void*>(&pa_decode_kernel<kBf16, D, B, G>), kThreads,
                  static_cast<int>(sizeof(DecodeSmem<D, B, G>)), Cfg<D, B, G>::kPartStride,
-                 &launch_cuda_cores<kBf16, D, B, G>};
+                 &launch_cuda_cores<kBf16, D, B, G>, 0};
 }
 
 template <bool kBf16, int D, int B>
@@ -599,6 +599,7 @@ static DecodeParams make_params(const void* q, const void* k_pool, const void* v
   prm.num_groups = 0;
   prm.seq_prefix = nullptr;
   prm.prefix_part = nullptr;
+  prm.unit_cost = 0;
   return prm;
 }
 
@@ -701,9 +702,10 @@ extern "C" pa_status pa_decode_ex(const void* q, const void* k_pool, const void*
   if (ctas <= 0) return PA_ERR_CUDA;
   const size_t need = workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
-  const DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+  DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                                        num_q_heads, scale, out, workspace, ctas, v.part_stride, dev_status, pool,
                                        opts_flags(opts));
+  prm.unit_cost = v.unit_cost;
   return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -753,6 +755,7 @@ extern "C" pa_status pa_decode_multi(const void* q, const void* k_pool, const vo
                                  num_q_heads, scale, out, workspace, ctas, v.part_stride, dev_status, pool,
                                  opts_flags(opts));
   prm.q_len = q_len;
+  prm.unit_cost = v.unit_cost;
   return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -808,6 +811,8 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* k_pool, 
                                 pool, flags);
   p2.seq_prefix = seq_prefix;
   p2.prefix_part = prefix_part;
+  p1.unit_cost = pl.pass1.unit_cost;
+  p2.unit_cost = pl.pass2.unit_cost + 12;  // the finish also merges the prefix state (swept on B200)
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pl.pass1.launch(pl.pass1, p1, pl.ctas1, s) != cudaSuccess) return PA_ERR_CUDA;
   return pl.pass2.launch(pl.pass2, p2, pl.ctas2, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -864,7 +869,7 @@ extern "C" pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const
   }
   void* scratch = nullptr;
   if (!no_alloc_scratch_address(&scratch)) return PA_ERR_CUDA;
-  const DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+  DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                                        num_q_heads, scale, out, scratch, ctas, v.part_stride, dev_status, pool, 0);
   // The array keeps whatever the previous call left; the arrival counters
   // must start at zero, so clear them on the caller's stream first.
@@ -872,5 +877,6 @@ extern "C" pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const
                       static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     return PA_ERR_CUDA;
   }
+  prm.unit_cost = v.unit_cost;
   return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -3,16 +3,21 @@
 // the merge of split units through the workspace.
 //
 // Work partition.  Each (sequence, kv head) "unit" is cut into granules of
-// CB consecutive logical blocks (the last one may be shorter); all granules
-// are laid end to end — sequence-major, kv head next, granule innermost —
-// and cut into `nparts` contiguous ranges of equal count, one per CTA, where
-// nparts is the grid size or the total granule count if that is smaller (so
-// no range is empty).  CB is the kernel's processing chunk (1 block for the
-// CUDA-core kernel, 8 for the tensor-core kernel), so every CTA gets the same
-// number of chunks and no range boundary splits a chunk.  A CTA's range
-// falls into segments, one per unit it touches.  A unit covered by one CTA is
-// finished there; a unit split between CTAs is finished by whichever of them
-// arrives last.
+// CB consecutive logical blocks (the last one may be shorter).  CB is the
+// kernel's processing chunk (1 block for the CUDA-core kernel, 8 for the
+// tensor-core kernel).  Every unit is given a cost: kGranuleCost per granule
+// plus `unit_cost` for the fixed work of finishing a unit (sums, output or
+// partial state, merge).  The units are laid end to end on a cost line —
+// sequence-major, kv head next — each as its fixed cost followed by its
+// granules, and the line is cut into `nparts` contiguous ranges of equal
+// cost, one per CTA.  A CTA processes the granules that start in its range,
+// so CTAs get equal expected time whatever the mix of unit lengths, and no
+// range boundary splits a chunk.  nparts is the grid size, or fewer when
+// there is less than one granule of cost per CTA, so that every range that
+// falls inside a unit holds one of its granules.  A CTA's granules fall into
+// segments, one per unit it touches.  A unit covered by one CTA is finished
+// there; a unit split between CTAs is finished by whichever of them arrives
+// last.
 //
 // Merge rule (study notes ch.05 §4, the online-softmax merge applied to
 // partitions): a partial state is (m, l, acc) in the log2 domain — running
@@ -53,7 +58,11 @@ struct DecodeParams {
   int num_groups;
   int32_t* seq_prefix;           // [num_seqs] prefix blocks per sequence (written by pass 1, read by pass 2)
   float* prefix_part;            // [num_seqs][num_q_heads][2 + head_dim] prefix states (m, l, acc)
+  // partition cost of finishing a unit, in 1/kGranuleCost granules
+  int unit_cost;
 };
+
+constexpr long long kGranuleCost = 8;  // partition cost of one granule
 
 constexpr int kFlagTestWithholdCopies = PA_DECODE_TEST_WITHHOLD_COPIES;  // producer issues nothing
 
@@ -85,7 +94,9 @@ struct Cursor {
   int first;  // first logical block of the span
   int nb;     // end of the span (logical blocks)
   int len;    // tokens of sequence s
-  long long x, remaining;  // flattened granule index; granules left in the range
+  long long ucost;  // cost-line position where unit (s, h) starts
+  long long end;    // end of the CTA's cost range
+  bool done;
 };
 
 struct Seg {
@@ -95,8 +106,14 @@ struct Seg {
   int nb;     // end of the unit's span
   int ng;     // granules of the unit
   int len;    // tokens of the sequence
-  long long unit_first;  // flattened index of the unit's granule 0
+  long long unit_first;  // cost-line position of the unit's granule 0
+  long long unit_last;   // cost-line position of its last granule
 };
+
+// Cost of one unit with ng granules (a unit with none costs nothing).
+__device__ __forceinline__ long long unit_cost_of(const DecodeParams& p, int ng) {
+  return ng > 0 ? ng * kGranuleCost + p.unit_cost : 0;
+}
 
 template <int B, int CB, class Src>
 __device__ __forceinline__ void load_seq(Cursor& c, const DecodeParams& p, const Src& src) {
@@ -107,12 +124,35 @@ __device__ __forceinline__ void load_seq(Cursor& c, const DecodeParams& p, const
   c.ng = sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
 }
 
-// Next segment of the CTA's range; advances the cursor past it.
+// Move the cursor to granule 0 of the next unit that has one.
+template <int B, int CB, class Src>
+__device__ __forceinline__ void next_unit(Cursor& c, const DecodeParams& p, const Src& src) {
+  c.ucost += unit_cost_of(p, c.ng);
+  c.jg = 0;
+  if (++c.h == p.num_kv_heads) {
+    c.h = 0;
+    do {
+      if (++c.s >= src.count(p)) {  // past the last sequence
+        c.done = true;
+        break;
+      }
+      load_seq<B, CB>(c, p, src);
+    } while (c.ng == 0);
+  }
+}
+
+// Next segment of the CTA's range (the granules of one unit that start in
+// it); advances the cursor past it.
 template <int B, int CB, class Src = WholeSequence>
 __device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams& p, const Src& src = Src()) {
-  if (c.remaining <= 0) return false;
-  const long long left = c.ng - c.jg;
-  const int k = static_cast<int>(left < c.remaining ? left : c.remaining);
+  if (c.done) return false;
+  const long long g0 = c.ucost + p.unit_cost + c.jg * kGranuleCost;  // where granule jg starts
+  if (g0 >= c.end) {
+    c.done = true;
+    return false;
+  }
+  const long long fit = (c.end - g0 + kGranuleCost - 1) / kGranuleCost;  // granules starting before end
+  const int k = static_cast<int>(fit < c.ng - c.jg ? fit : c.ng - c.jg);
   sg.s = c.s;
   sg.h = c.h;
   sg.j0 = c.first + c.jg * CB;
@@ -122,29 +162,14 @@ __device__ __forceinline__ bool next_seg(Cursor& c, Seg& sg, const DecodeParams&
   sg.nb = c.nb;
   sg.ng = c.ng;
   sg.len = c.len;
-  sg.unit_first = c.x - c.jg;
-  c.remaining -= k;
-  c.x += k;
+  sg.unit_first = c.ucost + p.unit_cost;
+  sg.unit_last = sg.unit_first + (c.ng - 1) * kGranuleCost;
   c.jg += k;
-  if (c.jg == c.ng) {
-    c.jg = 0;
-    if (++c.h == p.num_kv_heads) {
-      c.h = 0;
-      if (c.remaining > 0) {
-        do {
-          if (++c.s >= src.count(p)) {  // inconsistent lengths: stop cleanly
-            c.remaining = 0;
-            break;
-          }
-          load_seq<B, CB>(c, p, src);
-        } while (c.ng == 0);
-      }
-    }
-  }
+  if (c.jg == c.ng) next_unit<B, CB>(c, p, src);
   return true;
 }
 
-// CTA whose range [c*N/C, (c+1)*N/C) holds flattened granule x.
+// CTA whose range [c*N/C, (c+1)*N/C) of the cost line holds position x.
 __device__ __forceinline__ long long cta_of(long long x, long long N, long long C) { return ((x + 1) * C - 1) / N; }
 
 __device__ __forceinline__ long long range_start(long long c, long long N, long long C) { return c * N / C; }
@@ -180,8 +205,8 @@ __device__ __forceinline__ long long block_inclusive_scan(long long v, RangeSmem
 }
 
 struct WorkRange {
-  long long total;   // granules over all units
-  long long nparts;  // CTAs that own a non-empty range
+  long long total;   // length of the cost line
+  long long nparts;  // CTAs that own a range
   long long start, end;
 };
 
@@ -204,33 +229,33 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
     }
     if (s < nseq) {
       const SeqSpan sp = src.template span<B>(p, s);
-      mine += sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
+      mine += Hkv * unit_cost_of(p, sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0);
     }
   }
-  long long seq_granules;
-  (void)block_inclusive_scan<NT>(mine, rs, seq_granules);
-  wr.total = seq_granules * Hkv;
-  wr.nparts = wr.total < nctas ? wr.total : nctas;
-  if (cta >= wr.nparts) return false;  // uniform across the CTA (also covers total == 0)
+  long long line;
+  (void)block_inclusive_scan<NT>(mine, rs, line);
+  wr.total = line;
+  const long long most = line / kGranuleCost;  // at least one granule of cost per range
+  wr.nparts = most < nctas ? most : nctas;
+  if (cta >= wr.nparts) return false;  // uniform across the CTA (also covers an empty line)
   wr.start = range_start(cta, wr.total, wr.nparts);
   wr.end = range_start(cta + 1, wr.total, wr.nparts);
 
-  // locate the sequence holding `start`
-  const long long target = wr.start / Hkv;  // in per-sequence granule units
+  // locate the sequence whose costs hold `start`
   if (tid == 0) rs.found = 0;
   __syncthreads();
   long long base = 0;
   for (int chunk = 0; chunk < nseq; chunk += NT) {
     const int s = chunk + tid;
-    long long ng = 0;
+    long long cost = 0;
     if (s < nseq) {
       const SeqSpan sp = src.template span<B>(p, s);
-      ng = sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0;
+      cost = Hkv * unit_cost_of(p, sp.nb > sp.first ? (sp.nb - sp.first + CB - 1) / CB : 0);
     }
     long long chunk_total;
-    const long long incl = block_inclusive_scan<NT>(ng, rs, chunk_total);
-    const long long excl = incl - ng;
-    if (ng > 0 && base + excl <= target && target < base + incl) {
+    const long long incl = block_inclusive_scan<NT>(cost, rs, chunk_total);
+    const long long excl = incl - cost;
+    if (cost > 0 && base + excl <= wr.start && wr.start < base + incl) {
       rs.s0 = s;
       rs.pre0 = base + excl;
       rs.found = 1;
@@ -242,11 +267,15 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
   if (!rs.found) return false;  // only with lengths changing under the kernel
   cur.s = rs.s0;
   load_seq<B, CB>(cur, p, src);
-  const long long off = wr.start - rs.pre0 * Hkv;
-  cur.h = static_cast<int>(off / cur.ng);
-  cur.jg = static_cast<int>(off % cur.ng);
-  cur.x = wr.start;
-  cur.remaining = wr.end - wr.start;
+  const long long ucost = unit_cost_of(p, cur.ng);
+  const long long off = wr.start - rs.pre0;
+  cur.h = static_cast<int>(off / ucost);
+  cur.ucost = rs.pre0 + cur.h * ucost;
+  const long long rem = off - cur.h * ucost - p.unit_cost;  // past the unit's fixed cost
+  cur.jg = rem <= 0 ? 0 : static_cast<int>((rem + kGranuleCost - 1) / kGranuleCost);
+  cur.end = wr.end;
+  cur.done = false;
+  if (cur.jg >= cur.ng) next_unit<B, CB>(cur, p, src);  // the range starts after the unit's last granule
   return true;
 }
 
@@ -281,7 +310,7 @@ __device__ void finish_split_unit(const DecodeParams& p, const Seg& sg, const Wo
   constexpr int kStride = G * (D + 2);
   const long long F = sg.unit_first;
   const long long first = cta_of(F, wr.total, wr.nparts);
-  const long long last = cta_of(F + sg.ng - 1, wr.total, wr.nparts);
+  const long long last = cta_of(sg.unit_last, wr.total, wr.nparts);
   int32_t* counter = p.counters + static_cast<size_t>(sg.s) * p.num_kv_heads + sg.h;
   sync();
   if (ctid == 0) {

@@ -18,6 +18,7 @@ struct Variant {
   int smem_bytes;
   int part_stride;  // floats per partial slot: query rows per unit * (D + 2)
   LaunchFn launch;
+  int unit_cost;    // partition cost of finishing a unit (DecodeParams::unit_cost)
 };
 
 // Tensor-core variants (pa_attn_tc.cuh), if one exists for this pool and
