@@ -233,7 +233,7 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
     }
   }
   long long line;
-  (void)block_inclusive_scan<NT>(mine, rs, line);
+  const long long incl0 = block_inclusive_scan<NT>(mine, rs, line);
   wr.total = line;
   const long long most = line / kGranuleCost;  // at least one granule of cost per range
   wr.nparts = most < nctas ? most : nctas;
@@ -241,11 +241,20 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
   wr.start = range_start(cta, wr.total, wr.nparts);
   wr.end = range_start(cta + 1, wr.total, wr.nparts);
 
-  // locate the sequence whose costs hold `start`
+  // locate the sequence whose costs hold `start`: with at most one sequence
+  // per thread the scan above already holds every prefix sum
   if (tid == 0) rs.found = 0;
   __syncthreads();
+  if (nseq <= NT) {
+    if (mine > 0 && incl0 - mine <= wr.start && wr.start < incl0) {
+      rs.s0 = tid;
+      rs.pre0 = incl0 - mine;
+      rs.found = 1;
+    }
+    __syncthreads();
+  }
   long long base = 0;
-  for (int chunk = 0; chunk < nseq; chunk += NT) {
+  for (int chunk = 0; chunk < nseq && !rs.found; chunk += NT) {
     const int s = chunk + tid;
     long long cost = 0;
     if (s < nseq) {
@@ -262,7 +271,6 @@ __device__ bool decode_prologue(const DecodeParams& p, RangeSmem& rs, WorkRange&
     }
     base += chunk_total;
     __syncthreads();
-    if (rs.found) break;
   }
   if (!rs.found) return false;  // only with lengths changing under the kernel
   cur.s = rs.s0;

@@ -79,13 +79,14 @@ def _run(device, layout, values, groups, max_group, num_ctas=0):
     return out, int(st.item()), d, ws
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
-def test_forked_samples_match_oracle(cuda_device, G):
+def test_forked_samples_match_oracle(cuda_device, G, dtype):
     import paged_kv_cache_357_b200 as pa
 
     prompts = [(40, [1, 5, 30]), (300, [1, 2, 17, 64]), (17, [1]), (128, [1, 129]), (1000, [3, 40, 200, 7])]
     max_group = 4
-    L = _forked_layout(8000 + G, prompts, G=G)
+    L = _forked_layout(8000 + G, prompts, dtype=dtype, G=G)
     V = fill_values_numpy(L)
     groups = pa.shared_prefix_groups(L.block_tables, L.seq_lens, L.block_size, max_group)
     starts, prefix = groups
@@ -95,7 +96,7 @@ def test_forked_samples_match_oracle(cuda_device, G):
     out, st, _, _ = _run(cuda_device, L, V, groups, max_group)
     assert st == 0
     ref, _, _ = oracle_step(L, V)
-    assert_attention_close(torch_f64(out), ref, f"shared prefix G={G}")
+    assert_attention_close(torch_f64(out), ref, f"shared prefix G={G} {dtype}")
 
 
 @pytest.mark.parametrize("num_ctas", [1, 2, 5, 33, 0])
