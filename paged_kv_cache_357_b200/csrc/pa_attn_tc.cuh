@@ -73,6 +73,11 @@ constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 
 constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
 constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
 constexpr int kSoftmaxBarrier = 1;
+// A row's probabilities are taken relative to a reference max that only moves
+// when a score exceeds it by more than this (log2 units): p <= 2^8 stays
+// exact enough in 16-bit and in the fp32 sums, and most chunks need neither
+// a cross-warp max nor a rescale.
+constexpr float kRescaleGap = 8.f;
 
 enum Mode { kDecode = 0, kMulti = 1, kPrefix = 2 };
 
@@ -119,9 +124,10 @@ struct TcSmem {
   uint8_t q[2][S::kQSlotBytes];
   uint8_t p[2][S::kPSlotBytes];
   alignas(16) float red[2][4][R];  // per-warp column maxima, double-buffered by chunk
-  alignas(16) float mbuf[2][R];    // running max after each chunk
+  alignas(16) float mfin[R];       // reference max of each row of the segment being finished
   alignas(16) float abuf[2][R];    // rescale factor of each chunk's running output
-  alignas(16) float lred[4][R];    // per-warp column sums at the end of a segment
+  alignas(16) float lred[4][R];    // per-warp row sums of the segment being finished
+  int rescaled[2];                 // whether a chunk's rows changed their reference max
   uint64_t kfull[kKStages];
   uint64_t kempty[kKStages];
   uint64_t vfull[S::kVStages];
@@ -857,11 +863,14 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     int ci = 0;
     Seg sg;
     float acc[RC];
-    float l_lane = 0.f;  // running sum of p over this warp's tokens, column my_col
+    float m_ref[RC];  // reference max of each of this thread's rows (the same in every thread)
+    float l_thr[RC];  // sum of p over this thread's token rows, relative to m_ref
 
     // Online softmax of chunk ci (the first of its segment when `first`):
-    // P^T into the swizzled B operand, the new running max and the rescale
-    // factor of the running output into shared memory.
+    // P^T into the swizzled B operand.  The reference maxima move only when
+    // some score exceeds them by more than kRescaleGap (always on a
+    // segment's first chunk); then the chunk's row maxima are reduced across
+    // the warps and the rescale factors are left for the epilogue.
     auto softmax_chunk = [&](int ci, const ChunkInfo& ch, bool first, int rows, int len) -> bool {
       const int vs = ci % kVStages;
       const int sb = ci & 1;
@@ -877,40 +886,54 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       // scores of this token row for every query row (log2 domain), masked
       const int t = ch.j * B + r;  // token index in the sequence
       float sc[RC];
+      bool over = first;
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
         const int c = col0 + k;
         const bool valid = c < rows && r < ch.ntok && t <= src.limit(p, c / G, len);
         sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
+        over |= sc[k] > m_ref[k] + kRescaleGap;
       }
-      {
-        float v[RC];
+      const bool rescale = named_barrier_or(kSoftmaxBarrier, kSoftmaxThreads, over);  // uniform
+      if (rescale) {
+        {
+          float v[RC];
 #pragma unroll
-        for (int k = 0; k < RC; ++k) v[k] = sc[k];
-        const float wm = warp_column_reduce<RC, true>(v, lane);
-        if (col_writer) sm.red[sb][quad][my_col] = wm;
-      }
-      named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
-      // new running max of every query row: the chunk's maxima of the four
-      // warps and the running max before the chunk
-      const float* m_prev = sm.mbuf[(ci - 1) & 1];
-      float pr[RC];
-      {
-        float cm[RC], t[RC];
+          for (int k = 0; k < RC; ++k) v[k] = sc[k];
+          const float wm = warp_column_reduce<RC, true>(v, lane);
+          if (col_writer) sm.red[sb][quad][my_col] = wm;
+        }
+        named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+        float cm[RC], tt[RC], alpha[RC];
         ld_row<RC>(sm.red[sb][0] + col0, cm);
 #pragma unroll
-        for (int w = 1; w < 4; ++w) {
-          ld_row<RC>(sm.red[sb][w] + col0, t);
+        for (int w2 = 1; w2 < 4; ++w2) {
+          ld_row<RC>(sm.red[sb][w2] + col0, tt);
 #pragma unroll
-          for (int k = 0; k < RC; ++k) cm[k] = fmaxf(cm[k], t[k]);
-        }
-        if (!first) {
-          ld_row<RC>(m_prev + col0, t);
-#pragma unroll
-          for (int k = 0; k < RC; ++k) cm[k] = fmaxf(cm[k], t[k]);
+          for (int k = 0; k < RC; ++k) cm[k] = fmaxf(cm[k], tt[k]);
         }
 #pragma unroll
-        for (int k = 0; k < RC; ++k) pr[k] = fast_exp2(sc[k] - (cm[k] == -INFINITY ? 0.f : cm[k]));
+        for (int k = 0; k < RC; ++k) {
+          const float m_old = first ? -INFINITY : m_ref[k];
+          const float m_new = fmaxf(m_old, cm[k]);
+          alpha[k] = fast_exp2(m_old - (m_new == -INFINITY ? 0.f : m_new));
+          m_ref[k] = m_new;
+          l_thr[k] = first ? 0.f : l_thr[k] * alpha[k];
+        }
+        // the epilogue of this chunk rescales the running output
+        if (quad == 0 && lane < RC) {
+          float a = alpha[0];
+#pragma unroll
+          for (int k = 1; k < RC; ++k) a = lane == k ? alpha[k] : a;
+          sm.abuf[ci & 1][col0 + lane] = a;
+        }
+      }
+      if (ctid == 0) sm.rescaled[ci & 1] = rescale ? 1 : 0;
+      float pr[RC];
+#pragma unroll
+      for (int k = 0; k < RC; ++k) {
+        pr[k] = fast_exp2(sc[k] - (m_ref[k] == -INFINITY ? 0.f : m_ref[k]));
+        l_thr[k] += pr[k];
       }
       // P^T, MN-major: token row r holds at position c the head of query row
       // c's probability and at R + c its rounding residual, written as whole
@@ -962,24 +985,6 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
 
-      // off the path to PV: the running max and the rescale factor of the
-      // column this lane holds (for the next chunk and the epilogue), and the
-      // running sum of p over this warp's tokens
-      {
-        const float cm = fmaxf(fmaxf(sm.red[sb][0][my_col], sm.red[sb][1][my_col]),
-                               fmaxf(sm.red[sb][2][my_col], sm.red[sb][3][my_col]));
-        const float m_old = first ? -INFINITY : m_prev[my_col];
-        const float m_new = fmaxf(m_old, cm);
-        const float alpha = fast_exp2(m_old - (m_new == -INFINITY ? 0.f : m_new));
-        if (quad == 0 && col_writer) {
-          sm.mbuf[ci & 1][my_col] = m_new;
-          sm.abuf[ci & 1][my_col] = alpha;
-        }
-        float v[RC];
-#pragma unroll
-        for (int k = 0; k < RC; ++k) v[k] = pr[k];
-        l_lane = fmaf(l_lane, alpha, warp_column_reduce<RC, false>(v, lane));
-      }
       return true;
     };
 
@@ -997,24 +1002,45 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[pb]);
-      float alpha[RC];
-      ld_row<RC>(sm.abuf[ci & 1] + col0, alpha);
+      if (sm.rescaled[ci & 1]) {
+        float alpha[RC];
+        ld_row<RC>(sm.abuf[ci & 1] + col0, alpha);
 #pragma unroll
-      for (int k = 0; k < RC; ++k)
-        acc[k] = fmaf(acc[k], alpha[k], __uint_as_float(oh[k]) + __uint_as_float(ol[k]));
+        for (int k = 0; k < RC; ++k)
+          acc[k] = fmaf(acc[k], alpha[k], __uint_as_float(oh[k]) + __uint_as_float(ol[k]));
+      } else {
+#pragma unroll
+        for (int k = 0; k < RC; ++k) acc[k] += __uint_as_float(oh[k]) + __uint_as_float(ol[k]);
+      }
       return true;
     };
 
-    // The finish of a segment (column sums, then its rows or its partial
-    // state) runs after the softmax of the next segment's first chunk, so
-    // the copies and the tensor core keep streaming across unit boundaries.
-    auto finish_segment = [&](const Seg& fs, int rows, float l_sum, int last_ci) {
-      if (col_writer) sm.lred[quad][my_col] = l_sum;
+    // A segment's row sums and reference maxima, put aside before the next
+    // segment's first softmax resets them: sums reduced over the warp into
+    // lred, maxima into mfin (both read by finish_segment after a barrier).
+    auto stash_segment = [&]() {
+      float v[RC];
+#pragma unroll
+      for (int k = 0; k < RC; ++k) v[k] = l_thr[k];
+      const float ls = warp_column_reduce<RC, false>(v, lane);
+      if (col_writer) sm.lred[quad][my_col] = ls;
+      if (quad == 0 && lane < RC) {
+        float m = m_ref[0];
+#pragma unroll
+        for (int k = 1; k < RC; ++k) m = lane == k ? m_ref[k] : m;
+        sm.mfin[col0 + lane] = m;
+      }
+    };
+
+    // The finish of a segment (its rows or its partial state, and the merge
+    // when it arrives last) runs after the softmax of the next segment's
+    // first chunk, so the copies and the tensor core keep streaming across
+    // unit boundaries.
+    auto finish_segment = [&](const Seg& fs, int rows) {
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
-      const float* m_last = sm.mbuf[last_ci & 1];
       if (fs.j0 == fs.first && fs.j0 + fs.n == fs.nb) {
         float m[RC], L[RC];
-        ld_row<RC>(m_last + col0, m);
+        ld_row<RC>(sm.mfin + col0, m);
 #pragma unroll
         for (int k = 0; k < RC; ++k) {
           const int c = col0 + k;
@@ -1024,7 +1050,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       } else {
         float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * Sh::kPartStride;
         if (ctid < R) {
-          pp[ctid] = m_last[ctid];
+          pp[ctid] = sm.mfin[ctid];
           pp[R + ctid] = (sm.lred[0][ctid] + sm.lred[1][ctid]) + (sm.lred[2][ctid] + sm.lred[3][ctid]);
         }
 #pragma unroll
@@ -1040,7 +1066,11 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     };
 
 #pragma unroll
-    for (int k = 0; k < RC; ++k) acc[k] = 0.f;
+    for (int k = 0; k < RC; ++k) {
+      acc[k] = 0.f;
+      m_ref[k] = -INFINITY;
+      l_thr[k] = 0.f;
+    }
     Seg prev;               // the segment whose finish is still due
     int prev_rows = 0;
     bool have_prev = false;
@@ -1048,7 +1078,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     while (ok && next_seg<B, CB>(cur, sg, p, src)) {
       const int rows = G * src.row_groups(p, sg.s);
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
-        const float l_before = l_lane;  // the previous segment's sum, when c0 == 0
+        if (c0 == 0 && have_prev) stash_segment();
         ok = softmax_chunk(ci, chunk_at(sg, c0), c0 == 0, rows, sg.len);
         if (!ok) break;
         if (pending) {
@@ -1056,7 +1086,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           if (!ok) break;
         }
         if (c0 == 0 && have_prev) {
-          finish_segment(prev, prev_rows, l_before, ci - 1);
+          finish_segment(prev, prev_rows);
           have_prev = false;
         }
         pending = true;
@@ -1068,7 +1098,10 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       have_prev = true;
     }
     if (ok && pending) ok = epilogue_chunk(ci - 1);
-    if (ok && have_prev) finish_segment(prev, prev_rows, l_lane, ci - 1);
+    if (ok && have_prev) {
+      stash_segment();
+      finish_segment(prev, prev_rows);
+    }
     if (!ok && lane == 0) {
       sm.abort = 1;
       record_status(p.status, PA_DEV_TIMEOUT);
