@@ -120,7 +120,7 @@ def decode_kernel_name(L, mode: str = "plain") -> str:
         return "pa_decode_tc_kernel, multi-query (tcgen05)"
     if mode == "shared_prefix":
         return "pa_decode_tc_kernel, prefix pass + suffix pass (tcgen05)"
-    if L.head_dim == 128 and L.block_size == 16 and L.group in (4, 8):
+    if L.head_dim == 128 and L.block_size == 16 and L.group in (1, 2, 4, 8):
         return "pa_decode_tc_kernel (tcgen05)"
     return "pa_decode_kernel (CUDA cores)"
 
@@ -146,6 +146,31 @@ def profiled_traffic(L, mode: str = "plain"):
     if not m_hash or not m_traf or m_hash.group(1) != kernel_source_hash():
         return None
     return float(m_traf.group(1))
+
+
+def host_link_gbs(dev, h2d_bytes: int, d2h_bytes: int, reps: int = 20) -> dict:
+    """Pinned host<->device copy bandwidth for one step's bytes, each
+    direction alone, CUDA events on a side stream."""
+    import torch
+
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+    for name, nbytes, to_dev in (("h2d", h2d_bytes, True), ("d2h", d2h_bytes, False)):
+        host = torch.empty(max(nbytes, 1), dtype=torch.uint8).pin_memory()
+        devbuf = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(reps + 3):
+                if i == 3:
+                    a.record(stream)
+                if to_dev:
+                    devbuf.copy_(host, non_blocking=True)
+                else:
+                    host.copy_(devbuf, non_blocking=True)
+            b.record(stream)
+        stream.synchronize()
+        out[name] = nbytes * reps / (a.elapsed_time(b) * 1e-3) / 1e9
+    return out
 
 
 def max_over_ranks(values, device="cpu"):
@@ -462,6 +487,7 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1) / K2
     if step.device_status() != 0:
         raise SystemExit("device status set in the e2e loop")
+    link = host_link_gbs(dev, step.last_h2d_bytes, step.last_d2h_bytes)
 
     # ---- max over ranks
     elapsed_ms, e2e_ms, decode_mean_ms = max_over_ranks([elapsed_ms, e2e_ms, decode_mean_ms], dev)
@@ -522,6 +548,9 @@ def run_ours(args):
                 "h2d_bytes_per_step": step.last_h2d_bytes,
                 "d2h_bytes_per_step": step.last_d2h_bytes,
                 "steps": K2,
+                "link_gbs": link,
+                "link_note": "this box's pinned-copy bandwidth for one step's input and output bytes, "
+                             "measured outside the timed region (context: e2e is bound by it when slow)",
             },
             "gpu_launches": K * launches_per_step,
             "clocks": clocks,

@@ -96,9 +96,8 @@ typedef struct pa_decode_opts {
 #define PA_DECODE_TEST_WITHHOLD_COPIES 1
 
 /* pa_decode_opts.flags bit: use the CUDA-core kernel even where the
- * tensor-core kernel applies (group size 4 or 8 with head_dim 128 and
- * block_size 16); for comparisons and tests.  Same results within the
- * documented tolerance. */
+ * tensor-core kernel applies (head_dim 128 and block_size 16); for
+ * comparisons and tests.  Same results within the documented tolerance. */
 #define PA_DECODE_CUDA_CORES_ONLY 2
 
 /*

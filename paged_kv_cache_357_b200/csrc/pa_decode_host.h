@@ -23,9 +23,9 @@ struct Variant {
 
 // Tensor-core variants (pa_attn_tc.cuh), if one exists for this pool and
 // shape.  `group` is the number of query heads per kv head.
-// Plain decode (pa_decode_tc.cu): groups of 4 and 8.
+// Plain decode (pa_decode_tc.cu): groups of 1, 2, 4 and 8.
 bool select_tc_variant(const pa_pool_desc& pool, int group, Variant& v);
-// Second pass of the shared-prefix decode (pa_decode_tc.cu): groups of 1-8.
+// Second pass of the shared-prefix decode (pa_decode_tc.cu): the same kernels.
 bool select_tc_suffix_variant(const pa_pool_desc& pool, int group, Variant& v);
 // Multi-query decode with q_len >= 2 positions (pa_attn_tc_multi.cu).
 bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v);

@@ -1,8 +1,11 @@
 // Tensor-core decode (one query row per head): the kDecode instances of the
-// kernel in pa_attn_tc.cuh.  Used for plain decode where a GQA group of 4 or
-// 8 query heads shares each kv head, and for the second pass of the
-// shared-prefix decode (groups of 1, 2, 4 or 8), which reads only each
-// sequence's own blocks and merges the result with the shared prefix's state.
+// kernel in pa_attn_tc.cuh, for groups of 1, 2, 4 or 8 query heads per kv
+// head (head_dim 128, block 16).  Used for plain decode, and for the second
+// pass of the shared-prefix decode, which reads only each sequence's own
+// blocks and merges the result with the shared prefix's state.  Even at one
+// row per kv head, where the products are one real column of 16, its
+// pipeline streams K/V faster than the CUDA-core kernel (B200: 781.9 against
+// 838.3 µs on an 8 x 32k-token MHA layer).
 #include "pa_attn_tc.cuh"
 
 namespace pa {
@@ -22,13 +25,12 @@ static bool pick_decode(int G, Variant& v) {
 }  // namespace tc
 
 bool select_tc_variant(const pa_pool_desc& pool, int group, Variant& v) {
-  if (!tc::tc_pool_ok(pool) || (group != 4 && group != 8)) return false;
+  if (!tc::tc_pool_ok(pool)) return false;
   return pool.dtype == PA_BF16 ? tc::pick_decode<true>(group, v) : tc::pick_decode<false>(group, v);
 }
 
 bool select_tc_suffix_variant(const pa_pool_desc& pool, int group, Variant& v) {
-  if (!tc::tc_pool_ok(pool)) return false;
-  return pool.dtype == PA_BF16 ? tc::pick_decode<true>(group, v) : tc::pick_decode<false>(group, v);
+  return select_tc_variant(pool, group, v);
 }
 
 }  // namespace pa

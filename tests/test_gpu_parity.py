@@ -212,9 +212,9 @@ def test_device_errors_are_reported_not_trapped(pa_mod, cuda_device):
 
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
-@pytest.mark.parametrize("G", [4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_tensor_core_and_cuda_core_paths_agree(pa_mod, cuda_device, dtype, G):
-    """Groups of 4 and 8 at head_dim 128 / block 16 run on the tensor-core
+    """Every group size at head_dim 128 / block 16 runs on the tensor-core
     kernel by default; the CUDA-core kernel is forced with a flag.  Both must
     match the oracle, and each other to within the combined tolerance."""
     import torch
