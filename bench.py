@@ -119,7 +119,7 @@ def decode_kernel_name(L, mode: str = "plain") -> str:
     if L.q_len > 1:
         return "pa_decode_tc_kernel, multi-query (tcgen05)"
     if mode == "shared_prefix":
-        return "pa_decode_tc_kernel, prefix pass + suffix pass (tcgen05)"
+        return "pa_decode_tc_kernel, group units: shared prefix once, then each member's blocks (tcgen05)"
     if L.head_dim == 128 and L.block_size == 16 and L.group in (1, 2, 4, 8):
         return "pa_decode_tc_kernel (tcgen05)"
     return "pa_decode_kernel (CUDA cores)"
@@ -395,8 +395,7 @@ def run_ours(args):
         ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, V.k_pool, args.num_ctas)
     stream = torch.cuda.Stream(device=dev)
     has_copy, has_write = L.copy_pairs.shape[0] > 0, L.num_new_tokens > 0
-    decode_launches = 2 if mode == "shared_prefix" else 1
-    launches_per_step = decode_launches + int(has_copy) + int(has_write)
+    launches_per_step = 1 + int(has_copy) + int(has_write)
 
     def prologue():
         if has_copy:

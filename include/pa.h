@@ -242,17 +242,17 @@ PA_API pa_status pa_decode_multi(const void* q, const void* k_pool, const void* 
  *   max_group_size       host bound on members per group, >= 1
  * A group shares nothing (its members are decoded one by one) when its
  * prefix is 0, or not shorter than every member's block count.
- * Two launches on `stream`: a prefix pass over (group, kv head) units that
- * leaves each member's online-softmax state in the workspace, then a pass
- * over each sequence's own blocks that merges with that state.  Tensor-core
- * kernel only: head_dim 128, block_size 16, G in {1, 2, 4, 8} and
- * G * max_group_size <= 32 (rounded up to a power of two), else
- * PA_ERR_UNSUPPORTED.  Device errors: those of pa_decode, and
- * PA_DEV_BAD_GROUP when the groups do not partition the sequences (outputs
- * then unspecified) or a group has more members than max_group_size rounded
- * up to a power of two (that group is then decoded without sharing).  The
- * workspace (pa_decode_shared_prefix_workspace_bytes; zeroed before first
- * use, as for pa_decode) also holds the per-member prefix states.
+ * One launch of the tensor-core kernel over (group, kv head) units: a unit
+ * streams the group's shared blocks once, seen by every member's query
+ * heads, then each member's own blocks, seen by that member's heads only, and
+ * writes every member's outputs.  Tensor-core kernel only: head_dim 128,
+ * block_size 16, G in {1, 2, 4, 8} and G * max_group_size <= 32 (rounded up
+ * to a power of two), else PA_ERR_UNSUPPORTED.  Device errors: those of
+ * pa_decode, and PA_DEV_BAD_GROUP when the groups do not partition the
+ * sequences or a group has more members than max_group_size rounded up to a
+ * power of two (outputs then unspecified).  The workspace
+ * (pa_decode_shared_prefix_workspace_bytes; zeroed before first use, as for
+ * pa_decode) holds the partial states of units split between CTAs.
  */
 PA_API size_t pa_decode_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t max_group_size,
                                                       int32_t num_q_heads, const pa_pool_desc* pool,

@@ -25,7 +25,7 @@ SOURCES = [
     "pa_decode.cu",
     "pa_decode_tc.cu",
     "pa_attn_tc_multi.cu",
-    "pa_attn_tc_prefix.cu",
+    "pa_attn_tc_group.cu",
     "pa_kv_ops.cu",
     "pa_block_manager.cpp",
 ]

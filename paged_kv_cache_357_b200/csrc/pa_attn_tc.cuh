@@ -13,18 +13,16 @@
 // times RG row groups.  P^T carries 2R rows, each probability as a 16-bit
 // head plus a 16-bit residual, summed in the epilogue.  Three kinds of unit
 // (kMode):
-//   kDecode  one sequence, RG = 1: the decode step.  With per-sequence prefix
-//            lengths given, only the blocks past the prefix are read and the
-//            result is merged with the prefix's state from a kPrefix launch.
+//   kDecode  one sequence, RG = 1: the decode step.
 //   kMulti   one sequence, RG >= q_len new query positions, position i seeing
 //            the tokens up to seq_len - q_len + i (causal): speculative
 //            verification and prefill chunks (CSDN "PagedAttention：分页注意力",
 //            §"2026年最新进展" items 1-2).
-//   kPrefix  a group of up to RG sequences whose leading blocks are the same
+//   kGroup   a group of up to RG sequences whose leading blocks are the same
 //            physical blocks (parallel samples of one prompt, study notes
-//            §6.1; prefix caching, "vLLM 是什么" §3): the shared blocks are read
-//            once for every member's rows, and each row's state (max, sum,
-//            unnormalised output) is stored for the kDecode pass.
+//            §6.1; prefix caching, "vLLM 是什么" §3): the unit streams the
+//            shared blocks once, seen by every member's rows, then each
+//            member's own blocks, seen by that member's rows only.
 //
 // Work partition and split-unit merge: pa_decode_common.cuh (equal counts of
 // 8-block chunks per persistent CTA).
@@ -79,7 +77,7 @@ constexpr int kSoftmaxBarrier = 1;
 // a cross-warp max nor a rescale.
 constexpr float kRescaleGap = 8.f;
 
-enum Mode { kDecode = 0, kMulti = 1, kPrefix = 2 };
+enum Mode { kDecode = 0, kMulti = 1, kGroup = 2 };
 
 // Shapes that follow from the number of query rows R of a unit.  P enters
 // the PV product as two 16-bit rows per query row, p = hi + lo (the head and
@@ -333,45 +331,50 @@ __device__ __forceinline__ void ld_row(const float* src, float (&dst)[R]) {
   }
 }
 
-struct ChunkInfo {
-  int j;     // first logical block of the chunk
-  int nblk;  // blocks in the chunk
-  int ntok;  // valid tokens in the chunk
+// One chunk of a unit: up to CB consecutive blocks of one table row, and the
+// query rows that see its tokens.
+struct ChunkSrc {
+  int seq;             // table row
+  int j;               // first logical block
+  int nblk;            // blocks
+  int ntok;            // valid tokens
+  int len;             // tokens of the row's sequence (the causal limit's reference)
+  int row_lo, row_hi;  // query rows [row_lo, row_hi) that see these tokens
 };
 
-__device__ __forceinline__ ChunkInfo chunk_at(const Seg& sg, int c0) {
-  ChunkInfo c;
-  c.j = sg.j0 + c0;
-  c.nblk = min(CB, sg.n - c0);
-  c.ntok = min(c.nblk * B, sg.len - c.j * B);
-  return c;
+// ---- what a unit covers --------------------------------------------------------
+
+// Shared blocks of group g, or 0 when the group shares none: the prefix must
+// be shorter than every member's block count, so that every member keeps at
+// least one block (its newest token) of its own.
+template <int BB>
+__device__ __forceinline__ int group_prefix_blocks(const DecodeParams& p, int s0, int s1, int g) {
+  const int pb = __ldg(p.group_prefix + g);
+  if (pb <= 0) return 0;
+  for (int s = s0; s < s1; ++s) {
+    if (pb >= (checked_len(p, s, BB) + BB - 1) / BB) return 0;
+  }
+  return pb;
 }
 
-// ---- what a unit covers: blocks, table row, q rows -------------------------
+__device__ __forceinline__ bool group_ok(const DecodeParams& p, int s0, int s1, int max_members) {
+  return s0 >= 0 && s1 <= p.num_seqs && s1 - s0 >= 1 && s1 - s0 <= max_members;
+}
 
 template <int kMode, int RG>
 struct Source;
 
-// A sequence: all its blocks, or those past its shared prefix when
-// per-sequence prefix lengths are given.
+// A sequence: all its blocks.
 template <int RG>
 struct Source<kDecode, RG> {
   template <int BB>
   __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int s) const {
     const int len = checked_len(p, s, BB);
-    const int nb = (len + BB - 1) / BB;
-    int first = 0;
-    if (p.seq_prefix != nullptr) {
-      const int f = __ldcg(p.seq_prefix + s);  // written by the previous launch
-      first = (f > 0 && f < nb) ? f : 0;
-    }
-    return SeqSpan{first, nb, len};
+    return SeqSpan{0, (len + BB - 1) / BB, len};
   }
   __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
-  __device__ __forceinline__ int table_seq(const DecodeParams&, int s) const { return s; }
   __device__ __forceinline__ int row_group0(const DecodeParams&, int s) const { return s; }
   __device__ __forceinline__ int row_groups(const DecodeParams&, int) const { return 1; }
-  __device__ __forceinline__ int limit(const DecodeParams&, int, int len) const { return len - 1; }
 };
 
 // A sequence with q_len query positions, causal among the new tokens.  A
@@ -385,57 +388,138 @@ struct Source<kMulti, RG> {
     return SeqSpan{0, (len + BB - 1) / BB, len};
   }
   __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
-  __device__ __forceinline__ int table_seq(const DecodeParams&, int s) const { return s; }
   __device__ __forceinline__ int row_group0(const DecodeParams& p, int s) const { return s * p.q_len; }
   __device__ __forceinline__ int row_groups(const DecodeParams& p, int) const { return p.q_len; }
-  __device__ __forceinline__ int limit(const DecodeParams& p, int rg, int len) const { return len - p.q_len + rg; }
 };
 
-// Shared blocks of group g, or 0 when the group cannot share: members are
-// sequences [starts[g], starts[g+1]), at most RG of them, and the prefix must
-// be shorter than every member's block count, so that every member keeps at
-// least one block (its newest token) of its own.
-template <int BB, int RG>
-__device__ __forceinline__ int group_prefix_blocks(const DecodeParams& p, int g) {
-  const int s0 = __ldg(p.group_starts + g), s1 = __ldg(p.group_starts + g + 1);
-  const int pb = __ldg(p.group_prefix + g);
-  if (s0 < 0 || s1 > p.num_seqs || s1 - s0 < 1 || s1 - s0 > RG || pb <= 0) return 0;
-  for (int s = s0; s < s1; ++s) {
-    if (pb >= (checked_len(p, s, BB) + BB - 1) / BB) return 0;
-  }
-  return pb;
-}
-
-// A group of sequences: the leading blocks they share, read through the
-// first member's table.
+// A group of sequences [starts[g], starts[g+1]): the shared prefix, then each
+// member's own blocks, each part starting a new granule.  On the work line a
+// group unit is a run of "virtual" blocks, CB per granule; GroupWalk maps
+// them back to table rows.  A group with more than RG members, or outside
+// the batch, covers nothing (and is reported by group_bookkeeping).
 template <int RG>
-struct Source<kPrefix, RG> {
+struct Source<kGroup, RG> {
   template <int BB>
   __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int g) const {
-    const int pb = group_prefix_blocks<BB, RG>(p, g);
-    return SeqSpan{0, pb, pb * BB};
+    const int s0 = __ldg(p.group_starts + g), s1 = __ldg(p.group_starts + g + 1);
+    if (!group_ok(p, s0, s1, RG)) return SeqSpan{0, 0, 0};
+    const int pb = group_prefix_blocks<BB>(p, s0, s1, g);
+    int ng = (pb + CB - 1) / CB;
+    for (int s = s0; s < s1; ++s) {
+      const int nb = (checked_len(p, s, BB) + BB - 1) / BB;
+      ng += (nb - pb + CB - 1) / CB;
+    }
+    return SeqSpan{0, ng * CB, ng * CB * BB};
   }
   __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_groups; }
-  __device__ __forceinline__ int table_seq(const DecodeParams& p, int g) const { return __ldg(p.group_starts + g); }
   __device__ __forceinline__ int row_group0(const DecodeParams& p, int g) const { return __ldg(p.group_starts + g); }
   __device__ __forceinline__ int row_groups(const DecodeParams& p, int g) const {
     return __ldg(p.group_starts + g + 1) - __ldg(p.group_starts + g);
   }
-  __device__ __forceinline__ int limit(const DecodeParams&, int, int len) const { return len - 1; }
 };
 
-// kPrefix launches, every CTA before its own work: record each member's
-// shared block count for the kDecode launch that follows (0 where the group
-// cannot share) and check that the groups partition the sequences.  Group g
-// is handled by thread g / gridDim.x of CTA g % gridDim.x.
-template <int BB, int RG>
-__device__ void prefix_bookkeeping(const DecodeParams& p) {
+// The chunks of one segment, in order, for any kind of unit.  A sequence
+// unit's chunks are consecutive blocks of its row, seen by all its rows.  A
+// group unit's chunks are the shared prefix (through the first member's row,
+// seen by every member's rows) and then each member's own blocks (its row,
+// seen by its own G rows).
+template <int kMode, int G>
+struct ChunkWalk {
+  // current part: table row, next block, end block, sequence tokens, rows
+  int seq, j, jend, len, row_lo, row_hi;
+  // group units only
+  int s0, s1, pb, member;  // member = -1 while in the prefix
+
+  __device__ __forceinline__ void start(const DecodeParams& p, const Seg& sg, int rows) {
+    if constexpr (kMode != kGroup) {
+      seq = sg.s;
+      j = sg.j0;
+      jend = sg.j0 + sg.n;
+      len = sg.len;
+      row_lo = 0;
+      row_hi = rows;
+    } else {
+      s0 = __ldg(p.group_starts + sg.s);
+      s1 = __ldg(p.group_starts + sg.s + 1);
+      pb = group_prefix_blocks<B>(p, s0, s1, sg.s);
+      int skip = sg.j0 / CB;  // granules of the unit before this segment
+      const int gp = (pb + CB - 1) / CB;
+      if (skip < gp) {
+        enter_prefix(skip);
+      } else {
+        skip -= gp;
+        for (member = 0; member < s1 - s0; ++member) {
+          const int nb = (checked_len(p, s0 + member, B) + B - 1) / B;
+          const int gm = (nb - pb + CB - 1) / CB;
+          if (skip < gm) break;
+          skip -= gm;
+        }
+        enter_member(p, skip);
+      }
+    }
+  }
+
+  // The chunk at the walk's position; the walk moves past it.
+  __device__ __forceinline__ ChunkSrc next(const DecodeParams& p) {
+    ChunkSrc c;
+    c.seq = seq;
+    c.j = j;
+    c.nblk = min(CB, jend - j);
+    c.ntok = min(c.nblk * B, len - j * B);
+    c.len = len;
+    c.row_lo = row_lo;
+    c.row_hi = row_hi;
+    j += c.nblk;
+    if constexpr (kMode == kGroup) {
+      if (j >= jend) {  // on to the next member with blocks of its own
+        ++member;
+        enter_member(p, 0);
+      }
+    }
+    return c;
+  }
+
+ private:
+  __device__ __forceinline__ void enter_prefix(int granule) {
+    member = -1;
+    seq = s0;
+    j = granule * CB;
+    jend = pb;
+    len = pb * B;
+    row_lo = 0;
+    row_hi = (s1 - s0) * G;
+  }
+  __device__ __forceinline__ void enter_member(const DecodeParams& p, int granule) {
+    for (; member < s1 - s0; ++member) {
+      len = checked_len(p, s0 + member, B);
+      jend = (len + B - 1) / B;
+      if (jend > pb) break;  // a member without blocks of its own is skipped
+    }
+    seq = s0 + member;
+    j = pb + granule * CB;
+    row_lo = member * G;
+    row_hi = row_lo + G;
+  }
+};
+
+// kGroup launches, every CTA before its own work: check that the groups
+// partition the sequences and fit the kernel, and zero the outputs of groups
+// with nothing to read.  Group g is handled by thread g / gridDim.x of CTA
+// g % gridDim.x.
+template <int RG>
+__device__ void group_bookkeeping(const DecodeParams& p, const Source<kGroup, RG>& src) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long g = static_cast<long long>(threadIdx.x) * gridDim.x + blockIdx.x; g < p.num_groups; g += stride) {
     const int s0 = __ldg(p.group_starts + g), s1 = __ldg(p.group_starts + g + 1);
-    if (s0 < 0 || s1 < s0 || s1 > p.num_seqs || s1 - s0 > RG) record_status(p.status, PA_DEV_BAD_GROUP);
-    const int pb = group_prefix_blocks<BB, RG>(p, static_cast<int>(g));
-    for (int s = max(s0, 0); s < min(s1, p.num_seqs); ++s) p.seq_prefix[s] = pb;
+    if (s0 < 0 || s1 < s0 || s1 > p.num_seqs || s1 - s0 > RG) {
+      record_status(p.status, PA_DEV_BAD_GROUP);
+      continue;
+    }
+    const SeqSpan sp = src.template span<B>(p, static_cast<int>(g));
+    if (sp.nb > 0) continue;
+    uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(s0) * p.num_q_heads * D);
+    const int n = (s1 - s0) * p.num_q_heads * D / 8;
+    for (int i = 0; i < n; ++i) o[i] = make_uint4(0, 0, 0, 0);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (__ldg(p.group_starts) != 0 || __ldg(p.group_starts + p.num_groups) != p.num_seqs) {
@@ -467,58 +551,29 @@ __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>&
 
 // Rows col0 .. col0 + RC - 1 of the unit in segment sg (those below `rows`),
 // head_dim element d, from their states (m, L, unnormalised a): the
-// normalised outputs — merged first with the shared prefix's states when the
-// unit skipped a prefix — or, in kPrefix, the states themselves.  Every load
-// is issued before any result is formed, so a thread waits on memory once.
+// normalised outputs.  A row that saw no token (a group member of length 0)
+// gets zeros.
 template <bool kBf16, int G, int RC, int kMode>
 __device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, int col0, int rows, int d,
-                                          const float (&m)[RC], float (&L)[RC], float (&a)[RC]) {
+                                          const float (&m)[RC], const float (&L)[RC], const float (&a)[RC]) {
+  (void)m;
   const int Hq = p.num_q_heads;
-  if constexpr (kMode == kPrefix) {
-    const int s0 = __ldg(p.group_starts + sg.s);
+  const int s0 = kMode == kGroup ? __ldg(p.group_starts + sg.s) : 0;
 #pragma unroll
-    for (int k = 0; k < RC; ++k) {
-      const int c = col0 + k;
-      if (c < rows) {
-        float* pp = p.prefix_part + (static_cast<size_t>(s0 + c / G) * Hq + sg.h * G + c % G) * (D + 2);
-        if (d == 0) {
-          pp[0] = m[k];
-          pp[1] = L[k];
-        }
-        pp[2 + d] = a[k];
+  for (int k = 0; k < RC; ++k) {
+    const int c = col0 + k;
+    if (c < rows) {
+      const int rg = c / G;
+      size_t row;
+      if constexpr (kMode == kMulti) {
+        row = static_cast<size_t>(sg.s) * p.q_len + rg;
+      } else if constexpr (kMode == kGroup) {
+        row = static_cast<size_t>(s0 + rg);
+      } else {
+        row = static_cast<size_t>(sg.s);
       }
-    }
-  } else {
-    if constexpr (kMode == kDecode) {
-      if (sg.first > 0) {
-        float pm[RC], pl[RC], pa[RC];
-#pragma unroll
-        for (int k = 0; k < RC; ++k) {
-          const int c = col0 + k;
-          const float* pp = p.prefix_part + (static_cast<size_t>(sg.s) * Hq + sg.h * G + c) * (D + 2);
-          const bool on = c < rows;
-          pm[k] = on ? __ldcg(pp) : 0.f;
-          pl[k] = on ? __ldcg(pp + 1) : 0.f;
-          pa[k] = on ? __ldcg(pp + 2 + d) : 0.f;
-        }
-#pragma unroll
-        for (int k = 0; k < RC; ++k) {
-          const float M = fmaxf(m[k], pm[k]);
-          const float w0 = fast_exp2(m[k] - M), w1 = fast_exp2(pm[k] - M);
-          a[k] = a[k] * w0 + pa[k] * w1;
-          L[k] = L[k] * w0 + pl[k] * w1;
-        }
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < RC; ++k) {
-      const int c = col0 + k;
-      if (c < rows) {
-        const int rg = c / G;
-        const size_t row = (kMode == kMulti) ? static_cast<size_t>(sg.s) * p.q_len + rg : static_cast<size_t>(sg.s);
-        const uint32_t two = pack2<kBf16>(a[k] / L[k], 0.f);
-        p.out[(row * Hq + sg.h * G + c % G) * D + d] = static_cast<uint16_t>(two & 0xffffu);
-      }
+      const uint32_t two = pack2<kBf16>(L[k] > 0.f ? a[k] / L[k] : 0.f, 0.f);
+      p.out[(row * Hq + sg.h * G + c % G) * D + d] = static_cast<uint16_t>(two & 0xffffu);
     }
   }
 }
@@ -643,8 +698,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   // ---- inputs may come from the previous kernel in the stream
   grid_dependency_wait();
   grid_launch_dependents();
-  if constexpr (kMode == kPrefix) {
-    prefix_bookkeeping<B, RG>(p);
+  if constexpr (kMode == kGroup) {
+    group_bookkeeping(p, src);
   } else {
     zero_empty_units(p, src);
   }
@@ -685,51 +740,79 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         ++qi;
-        // Block-table entries 32 at a time (lane l holds entry b0 + l); the
-        // next batch is in flight while the current one is issued.
-        const int32_t* trow = p.block_tables + static_cast<size_t>(src.table_seq(p, sg.s)) * p.max_nb + sg.j0;
-        int e_cur = (lane < sg.n) ? __ldg(trow + lane) : 0;
-        for (int b0 = 0; ok && b0 < sg.n; b0 += 32) {
-          const int e_next = (b0 + 32 + lane < sg.n) ? __ldg(trow + b0 + 32 + lane) : 0;
-          if (b0 + lane < sg.n && (e_cur < 0 || e_cur >= p.num_blocks)) {
+        // K and V loads of one chunk of nblk blocks; lane l < nblk holds the
+        // physical block e of the chunk's block l
+        auto issue = [&](int nblk, int e) -> bool {
+          const int ks = ci % kKStages, vs = ci % kVStages;
+          const int y = (e * Hkv + sg.h) * B;
+          bool go = true;
+          if (lane == 0) {
+            go = mbar_wait_bounded(&sm.kempty[ks], ((ci / kKStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+            if (go) mbar_arrive_expect_tx(&sm.kfull[ks], nblk * 2 * kBlockBytes);
+          }
+          if (!__shfl_sync(0xffffffffu, go, 0)) return false;
+          if (lane < nblk) {
+            uint8_t* base = sm.kbuf[ks] + lane * kBlockBytes;
+            tma_load_2d(base, &map_k, 0, y, &sm.kfull[ks], pol_stream);
+            tma_load_2d(base + kHalfBytes, &map_k, 64, y, &sm.kfull[ks], pol_stream);
+          }
+          __syncwarp();
+          ++k_issued;
+          if (lane == 0) {
+            go = mbar_wait_bounded(&sm.vempty[vs], ((ci / kVStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+            if (go) mbar_arrive_expect_tx(&sm.vfull[vs], nblk * 2 * kBlockBytes);
+          }
+          if (!__shfl_sync(0xffffffffu, go, 0)) return false;
+          if (lane < nblk) {
+            uint8_t* base = sm.vbuf[vs] + lane * kBlockBytes;
+            tma_load_2d(base, &map_v, 0, y, &sm.vfull[vs], pol_stream);
+            tma_load_2d(base + kHalfBytes, &map_v, 64, y, &sm.vfull[vs], pol_stream);
+          }
+          __syncwarp();
+          ++v_issued;
+          ++ci;
+          return true;
+        };
+        auto checked = [&](int e, bool used) {
+          if (used && (e < 0 || e >= p.num_blocks)) {
             record_status(p.status, PA_DEV_BAD_BLOCK_ID);
-            e_cur = 0;
+            return 0;
           }
-          const int b_end = min(b0 + 32, sg.n);
-          for (int c0 = b0; c0 < b_end; c0 += CB) {
-            const ChunkInfo ch = chunk_at(sg, c0);
-            const int e = __shfl_sync(0xffffffffu, e_cur, (c0 - b0) + (lane & (CB - 1)));
-            const int ks = ci % kKStages, vs = ci % kVStages;
-            const int y = (e * Hkv + sg.h) * B;
-            if (lane == 0) {
-              ok = mbar_wait_bounded(&sm.kempty[ks], ((ci / kKStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
-              if (ok) mbar_arrive_expect_tx(&sm.kfull[ks], ch.nblk * 2 * kBlockBytes);
+          return e;
+        };
+        if constexpr (kMode != kGroup) {
+          // One table row: entries 32 at a time (lane l holds entry b0 + l),
+          // the next batch in flight while the current one is issued.
+          const int32_t* trow = p.block_tables + static_cast<size_t>(sg.s) * p.max_nb + sg.j0;
+          int e_cur = (lane < sg.n) ? __ldg(trow + lane) : 0;
+          for (int b0 = 0; ok && b0 < sg.n; b0 += 32) {
+            const int e_next = (b0 + 32 + lane < sg.n) ? __ldg(trow + b0 + 32 + lane) : 0;
+            e_cur = checked(e_cur, b0 + lane < sg.n);
+            const int b_end = min(b0 + 32, sg.n);
+            for (int c0 = b0; ok && c0 < b_end; c0 += CB) {
+              const int e = __shfl_sync(0xffffffffu, e_cur, (c0 - b0) + (lane & (CB - 1)));
+              ok = issue(min(CB, sg.n - c0), e);
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            if (lane < ch.nblk) {
-              uint8_t* base = sm.kbuf[ks] + lane * kBlockBytes;
-              tma_load_2d(base, &map_k, 0, y, &sm.kfull[ks], pol_stream);
-              tma_load_2d(base + kHalfBytes, &map_k, 64, y, &sm.kfull[ks], pol_stream);
-            }
-            __syncwarp();
-            ++k_issued;
-            if (lane == 0) {
-              ok = mbar_wait_bounded(&sm.vempty[vs], ((ci / kVStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
-              if (ok) mbar_arrive_expect_tx(&sm.vfull[vs], ch.nblk * 2 * kBlockBytes);
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            if (lane < ch.nblk) {
-              uint8_t* base = sm.vbuf[vs] + lane * kBlockBytes;
-              tma_load_2d(base, &map_v, 0, y, &sm.vfull[vs], pol_stream);
-              tma_load_2d(base + kHalfBytes, &map_v, 64, y, &sm.vfull[vs], pol_stream);
-            }
-            __syncwarp();
-            ++v_issued;
-            ++ci;
+            e_cur = e_next;
           }
-          e_cur = e_next;
+        } else {
+          // Chunks from several rows: each chunk's entries, one chunk ahead.
+          ChunkWalk<kMode, G> walk;
+          walk.start(p, sg, 0);
+          ChunkSrc cs = walk.next(p);
+          int e_cur = (lane < cs.nblk) ? __ldg(p.block_tables + static_cast<size_t>(cs.seq) * p.max_nb + cs.j + lane) : 0;
+          for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
+            ChunkSrc cn = cs;
+            int e_next = 0;
+            if (c0 + CB < sg.n) {
+              cn = walk.next(p);
+              e_next = (lane < cn.nblk) ? __ldg(p.block_tables + static_cast<size_t>(cn.seq) * p.max_nb + cn.j + lane)
+                                        : 0;
+            }
+            ok = issue(cs.nblk, checked(e_cur, lane < cs.nblk));
+            cs = cn;
+            e_cur = e_next;
+          }
         }
       }
     }
@@ -757,6 +840,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       bool have_seg = false, q_ready = false, walk_done = false;
       int c0 = 0;
       Seg sg;
+      ChunkWalk<kMode, G> walk;
       uint64_t t_idle = 0;
       uint32_t idle = 0;
       while (ok) {
@@ -765,6 +849,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           if (next_seg<B, CB>(cur, sg, p, src)) {
             have_seg = true;
             c0 = 0;
+            walk.start(p, sg, 0);
           } else {
             walk_done = true;
           }
@@ -790,7 +875,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
             umma_commit(&sm.s_full[qk & 1]);
             umma_commit(&sm.kempty[ks]);
             const int slot_shift = (qk & 3) * 8;
-            ring = (ring & ~(0xFFu << slot_shift)) | (static_cast<uint32_t>(chunk_at(sg, c0).ntok) << slot_shift);
+            ring = (ring & ~(0xFFu << slot_shift)) | (static_cast<uint32_t>(walk.next(p).ntok) << slot_shift);
             c0 += CB;
             if (c0 >= sg.n) {  // last chunk of the segment: q may be reloaded after this QK
               umma_commit(&sm.qempty[qs]);
@@ -871,14 +956,22 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     // some score exceeds them by more than kRescaleGap (always on a
     // segment's first chunk); then the chunk's row maxima are reduced across
     // the warps and the rescale factors are left for the epilogue.
-    auto softmax_chunk = [&](int ci, const ChunkInfo& ch, bool first, int rows, int len) -> bool {
+    auto softmax_chunk = [&](int ci, const ChunkSrc& ch, bool first) -> bool {
       const int vs = ci % kVStages;
       const int sb = ci & 1;
       bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
+      // whether any of this warpgroup's rows sees the chunk (a group unit's
+      // member chunk is seen by that member's rows only); uniform per warpgroup
+      const bool mine = kMode != kGroup || (ch.row_lo < col0 + RC && ch.row_hi > col0);
       float sN[RL];
-      tmem_ld<RL>(tmem + lane_base + kColS + sb * Nq + col0, sN);
+      if (mine) {
+        tmem_ld<RL>(tmem + lane_base + kColS + sb * Nq + col0, sN);
+      } else {
+#pragma unroll
+        for (int k = 0; k < RL; ++k) sN[k] = 0.f;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[sb]);
@@ -890,13 +983,14 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
         const int c = col0 + k;
-        const bool valid = c < rows && r < ch.ntok && t <= src.limit(p, c / G, len);
+        bool valid = mine && c >= ch.row_lo && c < ch.row_hi && r < ch.ntok;
+        if constexpr (kMode == kMulti) valid = valid && t <= ch.len - p.q_len + c / G;  // causal
         sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
         over |= sc[k] > m_ref[k] + kRescaleGap;
       }
       const bool rescale = named_barrier_or(kSoftmaxBarrier, kSoftmaxThreads, over);  // uniform
       if (rescale) {
-        {
+        if (mine) {
           float v[RC];
 #pragma unroll
           for (int k = 0; k < RC; ++k) v[k] = sc[k];
@@ -905,12 +999,17 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         }
         named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
         float cm[RC], tt[RC], alpha[RC];
-        ld_row<RC>(sm.red[sb][0] + col0, cm);
+        if (mine) {
+          ld_row<RC>(sm.red[sb][0] + col0, cm);
 #pragma unroll
-        for (int w2 = 1; w2 < 4; ++w2) {
-          ld_row<RC>(sm.red[sb][w2] + col0, tt);
+          for (int w2 = 1; w2 < 4; ++w2) {
+            ld_row<RC>(sm.red[sb][w2] + col0, tt);
 #pragma unroll
-          for (int k = 0; k < RC; ++k) cm[k] = fmaxf(cm[k], tt[k]);
+            for (int k = 0; k < RC; ++k) cm[k] = fmaxf(cm[k], tt[k]);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < RC; ++k) cm[k] = -INFINITY;
         }
 #pragma unroll
         for (int k = 0; k < RC; ++k) {
@@ -932,7 +1031,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       float pr[RC];
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
-        pr[k] = fast_exp2(sc[k] - (m_ref[k] == -INFINITY ? 0.f : m_ref[k]));
+        pr[k] = mine ? fast_exp2(sc[k] - (m_ref[k] == -INFINITY ? 0.f : m_ref[k])) : 0.f;
         l_thr[k] += pr[k];
       }
       // P^T, MN-major: token row r holds at position c the head of query row
@@ -1077,9 +1176,11 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     bool pending = false;   // the epilogue of chunk ci - 1 is still due
     while (ok && next_seg<B, CB>(cur, sg, p, src)) {
       const int rows = G * src.row_groups(p, sg.s);
+      ChunkWalk<kMode, G> walk;
+      walk.start(p, sg, rows);
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
         if (c0 == 0 && have_prev) stash_segment();
-        ok = softmax_chunk(ci, chunk_at(sg, c0), c0 == 0, rows, sg.len);
+        ok = softmax_chunk(ci, walk.next(p), c0 == 0);
         if (!ok) break;
         if (pending) {
           ok = epilogue_chunk(ci - 1);
@@ -1191,9 +1292,9 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
 // sums, outputs or partial state, the merge) adds to a CTA's time beyond
 // what the pipeline hides; it grows with the rows a unit carries.  Values
 // from sweeps on B200 (Llama-3-8B decode: 2 to 3 best; q_len 4 multi-query
-// at 16 rows: 6; the prefix pass was insensitive).
+// at 16 rows: 6).
 constexpr int unit_finish_cost(int kMode, int R) {
-  return kMode == kDecode ? (R <= 4 ? 2 : 4) : kMode == kPrefix ? 8 : (R <= 8 ? 4 : R <= 16 ? 6 : 10);
+  return kMode == kDecode ? (R <= 4 ? 2 : 4) : kMode == kGroup ? 10 : (R <= 8 ? 4 : R <= 16 ? 6 : 10);
 }
 
 template <bool kBf16, int G, int RG, int kMode>

@@ -597,8 +597,6 @@ static DecodeParams make_params(const void* q, const void* k_pool, const void* v
   prm.group_starts = nullptr;
   prm.group_prefix = nullptr;
   prm.num_groups = 0;
-  prm.seq_prefix = nullptr;
-  prm.prefix_part = nullptr;
   prm.unit_cost = 0;
   return prm;
 }
@@ -630,39 +628,13 @@ static bool multi_variant(const pa_pool_desc& pool, int num_q_heads, int q_len, 
 }
 
 // ---- shared-prefix decode ----------------------------------------------------
-// Workspace: [partials | counters] sized for the larger of the two passes'
-// needs (both passes put the counters at the same offset, so the second pass
-// finds them zeroed by the first), then the per-sequence prefix block counts
-// and the per-(sequence, query head) prefix states (m, l, acc[head_dim]).
+// One launch over (group, kv head) units; the workspace is a decode
+// workspace sized for the group variant's rows (counters per group fit in the
+// per-sequence counter array since there are no more groups than sequences).
 
-struct PrefixPlan {
-  Variant pass1, pass2;
-  int ctas1, ctas2;
-  int region_ctas, region_stride;
-  size_t counters_end, seq_prefix_off, prefix_part_off, total;
-};
-
-static bool prefix_plan(int num_seqs, int max_group_size, int num_q_heads, const pa_pool_desc& pool,
-                        const pa_decode_opts* opts, bool for_launch, PrefixPlan& pl) {
+static bool group_variant(const pa_pool_desc& pool, int num_q_heads, int max_group_size, Variant& v) {
   int G = 0;
-  if (num_seqs < 0 || max_group_size < 1 || !group_of(pool, num_q_heads, G)) return false;
-  if (!select_tc_prefix_variant(pool, G, max_group_size, pl.pass1)) return false;
-  if (!select_tc_suffix_variant(pool, G, pl.pass2)) return false;
-  if (for_launch) {
-    pl.ctas1 = resolve_ctas(pl.pass1, opts);
-    pl.ctas2 = resolve_ctas(pl.pass2, opts);
-    if (pl.ctas1 <= 0 || pl.ctas2 <= 0) return false;
-  } else if (!query_ctas(pl.pass1, opts, pl.ctas1) || !query_ctas(pl.pass2, opts, pl.ctas2)) {
-    return false;
-  }
-  pl.region_ctas = std::max(pl.ctas1, pl.ctas2);
-  pl.region_stride = std::max(pl.pass1.part_stride, pl.pass2.part_stride);
-  pl.counters_end = workspace_bytes_for(num_seqs, pool.num_kv_heads, pl.region_ctas, pl.region_stride);
-  pl.seq_prefix_off = pl.counters_end;
-  pl.prefix_part_off = pl.seq_prefix_off + align_up(static_cast<size_t>(num_seqs) * sizeof(int32_t), 256);
-  pl.total = pl.prefix_part_off +
-             align_up(static_cast<size_t>(num_seqs) * num_q_heads * (pool.head_dim + 2) * sizeof(float), 256);
-  return true;
+  return max_group_size >= 1 && group_of(pool, num_q_heads, G) && select_tc_group_variant(pool, G, max_group_size, v);
 }
 
 }  // namespace pa
@@ -762,10 +734,11 @@ extern "C" pa_status pa_decode_multi(const void* q, const void* k_pool, const vo
 extern "C" size_t pa_decode_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t max_group_size,
                                                           int32_t num_q_heads, const pa_pool_desc* pool,
                                                           const pa_decode_opts* opts) {
-  if (!pool_shape_ok(pool)) return 0;
-  PrefixPlan pl;
-  if (!prefix_plan(num_seqs, max_group_size, num_q_heads, *pool, opts, false, pl)) return 0;
-  return pl.total;
+  if (num_seqs < 0 || !pool_shape_ok(pool)) return 0;
+  Variant v;
+  int ctas = 0;
+  if (!group_variant(*pool, num_q_heads, max_group_size, v) || !query_ctas(v, opts, ctas)) return 0;
+  return workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
 }
 
 extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
@@ -785,37 +758,20 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* k_pool, 
   if (group_starts == nullptr || group_prefix_blocks == nullptr) return PA_ERR_INVALID_ARG;
   if (!opts_ok(opts)) return PA_ERR_INVALID_ARG;
   if ((opts_flags(opts) & PA_DECODE_CUDA_CORES_ONLY) != 0) return PA_ERR_UNSUPPORTED;
-  PrefixPlan pl;
-  int G = 0;
-  Variant probe1, probe2;
-  if (!group_of(*pool, num_q_heads, G) || !select_tc_prefix_variant(*pool, G, max_group_size, probe1) ||
-      !select_tc_suffix_variant(*pool, G, probe2)) {
-    return PA_ERR_UNSUPPORTED;
-  }
-  if (!prefix_plan(num_seqs, max_group_size, num_q_heads, *pool, opts, true, pl)) return PA_ERR_CUDA;
-  if (workspace == nullptr || workspace_bytes < pl.total || !aligned16(workspace)) return PA_ERR_WORKSPACE;
-  char* ws = static_cast<char*>(workspace);
-  int32_t* seq_prefix = reinterpret_cast<int32_t*>(ws + pl.seq_prefix_off);
-  float* prefix_part = reinterpret_cast<float*>(ws + pl.prefix_part_off);
-  const int flags = opts_flags(opts);
-  DecodeParams p1 = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
-                                num_q_heads, scale, out, workspace, pl.region_ctas, pl.region_stride, dev_status,
-                                pool, flags);
-  p1.group_starts = group_starts;
-  p1.group_prefix = group_prefix_blocks;
-  p1.num_groups = num_groups;
-  p1.seq_prefix = seq_prefix;
-  p1.prefix_part = prefix_part;
-  DecodeParams p2 = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
-                                num_q_heads, scale, out, workspace, pl.region_ctas, pl.region_stride, dev_status,
-                                pool, flags);
-  p2.seq_prefix = seq_prefix;
-  p2.prefix_part = prefix_part;
-  p1.unit_cost = pl.pass1.unit_cost;
-  p2.unit_cost = pl.pass2.unit_cost + 12;  // the finish also merges the prefix state (swept on B200)
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (pl.pass1.launch(pl.pass1, p1, pl.ctas1, s) != cudaSuccess) return PA_ERR_CUDA;
-  return pl.pass2.launch(pl.pass2, p2, pl.ctas2, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  Variant v;
+  if (!group_variant(*pool, num_q_heads, max_group_size, v)) return PA_ERR_UNSUPPORTED;
+  const int ctas = resolve_ctas(v, opts);
+  if (ctas <= 0) return PA_ERR_CUDA;
+  const size_t need = workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+  DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                                 num_q_heads, scale, out, workspace, ctas, v.part_stride, dev_status, pool,
+                                 opts_flags(opts));
+  prm.group_starts = group_starts;
+  prm.group_prefix = group_prefix_blocks;
+  prm.num_groups = num_groups;
+  prm.unit_cost = v.unit_cost;
+  return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

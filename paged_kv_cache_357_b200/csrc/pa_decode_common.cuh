@@ -52,12 +52,10 @@ struct DecodeParams {
   // multi-query decode: query positions per sequence (q, out are
   // [num_seqs][q_len][num_q_heads][head_dim]); 1 otherwise
   int q_len;
-  // shared-prefix decode (both passes; null / 0 otherwise)
+  // shared-prefix decode (null / 0 otherwise)
   const int32_t* group_starts;   // [num_groups + 1], consecutive sequences per group
   const int32_t* group_prefix;   // [num_groups] shared leading blocks of each group
   int num_groups;
-  int32_t* seq_prefix;           // [num_seqs] prefix blocks per sequence (written by pass 1, read by pass 2)
-  float* prefix_part;            // [num_seqs][num_q_heads][2 + head_dim] prefix states (m, l, acc)
   // partition cost of finishing a unit, in 1/kGranuleCost granules
   int unit_cost;
 };

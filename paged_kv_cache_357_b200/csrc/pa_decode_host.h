@@ -25,12 +25,10 @@ struct Variant {
 // shape.  `group` is the number of query heads per kv head.
 // Plain decode (pa_decode_tc.cu): groups of 1, 2, 4 and 8.
 bool select_tc_variant(const pa_pool_desc& pool, int group, Variant& v);
-// Second pass of the shared-prefix decode (pa_decode_tc.cu): the same kernels.
-bool select_tc_suffix_variant(const pa_pool_desc& pool, int group, Variant& v);
 // Multi-query decode with q_len >= 2 positions (pa_attn_tc_multi.cu).
 bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v);
-// First pass of the shared-prefix decode, groups of up to max_members
-// sequences (pa_attn_tc_prefix.cu).
-bool select_tc_prefix_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);
+// Shared-prefix decode over groups of up to max_members sequences
+// (pa_attn_tc_group.cu).
+bool select_tc_group_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);
 
 }  // namespace pa

@@ -1,8 +1,6 @@
 // Tensor-core decode (one query row per head): the kDecode instances of the
 // kernel in pa_attn_tc.cuh, for groups of 1, 2, 4 or 8 query heads per kv
-// head (head_dim 128, block 16).  Used for plain decode, and for the second
-// pass of the shared-prefix decode, which reads only each sequence's own
-// blocks and merges the result with the shared prefix's state.  Even at one
+// head (head_dim 128, block 16).  Even at one
 // row per kv head, where the products are one real column of 16, its
 // pipeline streams K/V faster than the CUDA-core kernel (B200: 781.9 against
 // 838.3 µs on an 8 x 32k-token MHA layer).
@@ -27,10 +25,6 @@ static bool pick_decode(int G, Variant& v) {
 bool select_tc_variant(const pa_pool_desc& pool, int group, Variant& v) {
   if (!tc::tc_pool_ok(pool)) return false;
   return pool.dtype == PA_BF16 ? tc::pick_decode<true>(group, v) : tc::pick_decode<false>(group, v);
-}
-
-bool select_tc_suffix_variant(const pa_pool_desc& pool, int group, Variant& v) {
-  return select_tc_variant(pool, group, v);
 }
 
 }  // namespace pa

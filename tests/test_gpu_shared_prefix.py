@@ -1,9 +1,9 @@
-"""GPU parity of the shared-prefix decode (pa_decode_shared_prefix: a prefix
-pass over each group's shared blocks, then a pass over each sequence's own
-blocks that merges the two states) against the float64 decode oracle — the
-result is plain decode; only the memory reads differ — element by element
-within 2e-3 + 1e-2*|oracle|.  Groups come from pa_shared_prefix_groups on the
-host tables."""
+"""GPU parity of the shared-prefix decode (pa_decode_shared_prefix: one unit
+per (group, kv head) streams the group's shared blocks once for every
+member's heads, then each member's own blocks for its heads) against the
+float64 decode oracle — the result is plain decode; only the memory reads
+differ — element by element within 2e-3 + 1e-2*|oracle|.  Groups come from
+pa_shared_prefix_groups on the host tables."""
 
 import numpy as np
 import pytest
@@ -100,7 +100,7 @@ def test_forked_samples_match_oracle(cuda_device, G, dtype):
 
 
 @pytest.mark.parametrize("num_ctas", [1, 2, 5, 33, 0])
-def test_split_units_in_both_passes(cuda_device, num_ctas):
+def test_split_group_units(cuda_device, num_ctas):
     import paged_kv_cache_357_b200 as pa
 
     prompts = [(2048, [1, 100, 513]), (64, [1, 2]), (700, [260])]

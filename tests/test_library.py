@@ -141,8 +141,8 @@ def test_shared_prefix_rejects_bad_arguments_on_host(lib):
     d = _desc(head_dim=128)
     opts = _lib.DecodeOpts(5, 0)
     n = lib.pa_decode_shared_prefix_workspace_bytes(4, 2, 8, ctypes.byref(d), ctypes.byref(opts))
-    # partials (two slots per CTA), counters, prefix lengths, prefix states
-    assert n >= 5 * 2 * 4 * 130 * 4 + 4 * 4 + 4 * 4 + 4 * 8 * 130 * 4
+    # partial states of 2 members x 2 heads per kv head (two slots per CTA), counters per (seq, kv head)
+    assert n >= 5 * 2 * 4 * 130 * 4 + 4 * 4 * 4
     assert lib.pa_decode_shared_prefix_workspace_bytes(4, 0, 8, ctypes.byref(d), ctypes.byref(opts)) == 0
 
 
