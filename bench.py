@@ -60,11 +60,12 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--num-ctas", type=int, default=0)
-    ap.add_argument("--decode", default="plain", choices=["plain", "shared_prefix"],
-                    help="shared_prefix: pa_decode_shared_prefix over the workload's prompt groups")
+    ap.add_argument("--decode", default="plain", choices=["plain", "shared_prefix", "cuda_cores"],
+                    help="shared_prefix: pa_decode_shared_prefix over the workload's prompt groups; "
+                         "cuda_cores: pa_decode held to its CUDA-core kernel (PA_DECODE_CUDA_CORES_ONLY)")
     ap.add_argument("--max-group", type=int, default=4, help="members per shared-prefix group")
     ap.add_argument("--batch", type=int, default=0,
-                    help="sequences per GPU for the llama7b / llama3_8b workloads (0 = the workload's own)")
+                    help="sequences per GPU for the llama7b / llama3_8b(_spec4) / llama2_70b_shared workloads (0 = the workload's own)")
     return ap.parse_args(argv)
 
 
@@ -120,7 +121,7 @@ def decode_kernel_name(L, mode: str = "plain") -> str:
         return "pa_decode_tc_kernel, multi-query (tcgen05)"
     if mode == "shared_prefix":
         return "pa_decode_tc_kernel, group units: shared prefix once, then each member's blocks (tcgen05)"
-    if L.head_dim == 128 and L.block_size == 16 and L.group in (1, 2, 4, 8):
+    if mode != "cuda_cores" and L.head_dim == 128 and L.block_size == 16 and L.group in (1, 2, 4, 8):
         return "pa_decode_tc_kernel (tcgen05)"
     return "pa_decode_kernel (CUDA cores)"
 
@@ -298,13 +299,20 @@ def cpu_baseline(L, budget_s: float) -> dict:
 
 
 def make_layout(args):
-    from workloads import CONFIGS, config_llama3_8b, config_llama7b
+    from workloads import CONFIGS, config_llama2_70b_shared, config_llama3_8b, config_llama7b
 
     if args.batch:
-        makers = {"llama3_8b": config_llama3_8b, "llama7b": config_llama7b}
+        def shared(batch):
+            if batch % 4:
+                raise SystemExit("llama2_70b_shared forks every prompt into 4 samples: --batch is a multiple of 4")
+            return config_llama2_70b_shared(num_prompts=batch // 4)
+
+        makers = {"llama3_8b": config_llama3_8b, "llama7b": config_llama7b,
+                  "llama3_8b_spec4": lambda batch: config_llama3_8b(batch=batch, q_len=4),
+                  "llama2_70b_shared": shared}
         if args.config not in makers:
             raise SystemExit(f"--batch applies to {sorted(makers)} only")
-        return makers[args.config](batch=args.batch)
+        return makers[args.config](args.batch)
     return CONFIGS[args.config]()
 
 
@@ -374,8 +382,9 @@ def run_ours(args):
     mode = args.decode
     if mode == "shared_prefix" and not L.share_groups:
         raise SystemExit("--decode shared_prefix needs a workload whose sequences share prompt blocks")
-    if mode == "shared_prefix" and L.q_len > 1:
-        raise SystemExit("--decode shared_prefix is a single-position decode")
+    if mode != "plain" and L.q_len > 1:
+        raise SystemExit(f"--decode {mode} is a single-position decode")
+    decode_flags = pa.PA_DECODE_CUDA_CORES_ONLY if mode == "cuda_cores" else 0
     V = fill_values_torch(L, dev, value_seed=L.seed + 7 * rank)
     nbytes = step_bytes(L, mode)
     tables = torch.from_numpy(L.block_tables).to(dev)
@@ -392,7 +401,7 @@ def run_ours(args):
         groups = (torch.from_numpy(g_starts).to(dev), torch.from_numpy(g_prefix).to(dev), g_starts, g_prefix)
         ws = pa.alloc_shared_prefix_workspace(L.num_seqs, args.max_group, L.num_q_heads, V.k_pool, args.num_ctas)
     else:
-        ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, V.k_pool, args.num_ctas)
+        ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, V.k_pool, args.num_ctas, decode_flags)
     stream = torch.cuda.Stream(device=dev)
     has_copy, has_write = L.copy_pairs.shape[0] > 0, L.num_new_tokens > 0
     launches_per_step = 1 + int(has_copy) + int(has_write)
@@ -412,7 +421,7 @@ def run_ours(args):
                                        L.scale, out, ws, status, num_ctas=args.num_ctas, stream=stream)
         else:
             pa.pa_decode(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status, num_ctas=args.num_ctas,
-                         stream=stream)
+                         flags=decode_flags, stream=stream)
 
     def barrier():
         if world > 1:
@@ -462,7 +471,8 @@ def run_ours(args):
     step = pa.PagedDecodeStep(V.k_pool, V.v_pool, L.num_seqs, L.num_q_heads, L.max_blocks_per_seq,
                               max_new_tokens=L.num_new_tokens, max_copy_pairs=L.copy_pairs.shape[0],
                               scale=L.scale, num_ctas=args.num_ctas, q_len=L.q_len,
-                              max_group_size=args.max_group if groups is not None else 0)
+                              max_group_size=args.max_group if groups is not None else 0,
+                              decode_flags=decode_flags)
 
     def e2e_step():
         return step.run(host["q"], host["tables"], host["lens"], host["new_k"], host["new_v"],
@@ -519,6 +529,7 @@ def run_ours(args):
                 "step": "+".join((["pa_copy_blocks"] if has_copy else []) + (["pa_cache_write"] if has_write
                                                                              else []) + [decode_entry(L, mode)]),
                 "q_len": L.q_len,
+                "decode": mode,
                 "l2": f"no flush: per-step K/V {nbytes['decode'] / 1e9:.2f} GB > 126 MB L2",
                 "parallelism": f"dp{world} (independent sequence shards, no collective)",
             },

@@ -53,11 +53,13 @@ class _BufferSet:
 class PagedDecodeStep:
     def __init__(self, k_pool, v_pool, num_seqs: int, num_q_heads: int, max_blocks_per_seq: int,
                  max_new_tokens: int = 0, max_copy_pairs: int = 0, scale: Optional[float] = None,
-                 num_ctas: int = 0, q_len: int = 1, max_group_size: int = 0, num_buffer_sets: int = 3):
+                 num_ctas: int = 0, q_len: int = 1, max_group_size: int = 0, num_buffer_sets: int = 3,
+                 decode_flags: int = 0):
         """q_len > 1: each step is a multi-query step (pa_decode_multi, q is
         [num_seqs, q_len, num_q_heads, head_dim]).  max_group_size > 0: each
         step decodes with pa_decode_shared_prefix and takes the groups as
-        inputs.  Otherwise pa_decode."""
+        inputs.  Otherwise pa_decode, with decode_flags (e.g.
+        PA_DECODE_CUDA_CORES_ONLY)."""
         import torch
 
         self.torch = torch
@@ -67,6 +69,7 @@ class PagedDecodeStep:
         self.S, self.Hq, self.D, self.Hkv = num_seqs, num_q_heads, D, Hkv
         self.scale = (1.0 / D**0.5) if scale is None else float(scale)
         self.num_ctas = num_ctas
+        self.decode_flags = decode_flags
         if q_len > 1 and max_group_size > 0:
             raise ValueError("a step is either multi-query or shared-prefix")
         self.q_len, self.max_group_size = q_len, max_group_size
@@ -84,7 +87,7 @@ class PagedDecodeStep:
             self.workspace = _lib.alloc_shared_prefix_workspace(num_seqs, max_group_size, num_q_heads, k_pool,
                                                                 num_ctas)
         else:
-            self.workspace = _lib.alloc_decode_workspace(num_seqs, num_q_heads, k_pool, num_ctas)
+            self.workspace = _lib.alloc_decode_workspace(num_seqs, num_q_heads, k_pool, num_ctas, decode_flags)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
         self.steps = 0
         self.last_h2d_bytes = 0
@@ -148,7 +151,8 @@ class PagedDecodeStep:
                                              num_ctas=self.num_ctas, stream=self.compute_stream)
             else:
                 _lib.pa_decode(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out,
-                               self.workspace, self.status, num_ctas=self.num_ctas, stream=self.compute_stream)
+                               self.workspace, self.status, num_ctas=self.num_ctas, flags=self.decode_flags,
+                               stream=self.compute_stream)
             bs.computed.record(self.compute_stream)
         with torch.cuda.stream(self.d2h_stream):
             self.d2h_stream.wait_event(bs.computed)
