@@ -27,21 +27,25 @@
 // Work partition and split-unit merge: pa_decode_common.cuh (equal counts of
 // 8-block chunks per persistent CTA).
 //
-// Roles (192 threads, one CTA per SM):
-//   warp 0      producer: resolves block ids (32 table entries per load, one
-//               batch ahead), issues 2-D TMA loads of the K and V tiles
-//               (64-column boxes, 128-byte swizzle) into separate rings of
-//               32 KB chunk stages — K released when its QK is done, V when
-//               its PV is done — and a 3-D TMA load of the unit's q rows.
+// Roles (96 + 128 x WG threads, one CTA per SM):
+//   warp 0      K producer: resolves block ids (32 table entries per load,
+//               one batch ahead), issues 2-D TMA loads of the K tiles
+//               (64-column boxes, 128-byte swizzle) into a ring of 32 KB
+//               chunk stages, released when its QK is done, and a 3-D TMA
+//               load of the unit's q rows.
 //   warp 1      allocates TMEM; lane 0 issues every tcgen05.mma and
 //               tcgen05.commit, polling which of QK(next) and PV(oldest
 //               pending) is ready and issuing it.
-//   warps 2-5   softmax + epilogue, one TMEM lane (token row, then head_dim
-//               index) per thread: read S^T from TMEM, column maxima and sums
-//               by warp butterfly reduce-scatters, write P^T (bf16/fp16) into
-//               a swizzled buffer, zero V rows past the sequence end inside
-//               the last 16-token step, then read O^T and rescale-accumulate.
-//               The epilogue of chunk i runs after the softmax of chunk i+1.
+//   warp 2      V producer: the same walk, V tiles into their own ring,
+//               released when the chunk's PV is done.  A warp issues TMA
+//               boxes one lane at a time, so K and V go out in parallel.
+//   warps 3..   softmax + epilogue (WG warpgroups), one TMEM lane (token row,
+//               then head_dim index) per thread: read S^T from TMEM, column
+//               maxima and sums by warp butterfly reduce-scatters, write P^T
+//               (bf16/fp16) into a swizzled buffer, zero V rows past the
+//               sequence end inside the last 16-token step, then read O^T
+//               and rescale-accumulate.  The epilogue of chunk i runs after
+//               the softmax of chunk i+1.
 // The swizzled layouts written by TMA serve both products directly: the K
 // tile is a K-major A operand for QK, the V tile an MN-major A operand for PV.
 #pragma once
@@ -71,6 +75,7 @@ constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 
 constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
 constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
 constexpr int kSoftmaxBarrier = 1;
+constexpr int kVWarp = 2;                  // the V producer; softmax warps start at 3
 // A row's probabilities are taken relative to a reference max that only moves
 // when a score exceeds it by more than this (log2 units): p <= 2^8 stays
 // exact enough in 16-bit and in the fp32 sums, and most chunks need neither
@@ -110,7 +115,7 @@ struct Rows {
   static constexpr int WG = R >= 16 ? 2 : 1;
   static constexpr int RC = R / WG;
   static constexpr int kSoftmaxThreads = 128 * WG;
-  static constexpr int kThreads = 64 + kSoftmaxThreads;          // + producer warp + MMA warp
+  static constexpr int kThreads = 96 + kSoftmaxThreads;          // + two producer warps + MMA warp
   static constexpr int kLanesPerCol = 32 / RC;                    // lanes holding one column after a reduce
 };
 
@@ -709,8 +714,13 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
 
   if (!has_work) {
     // nothing to stream: straight to teardown
-  } else if (warp == 0) {
-    // ===================== producer =========================================
+  } else if (warp == 0 || warp == kVWarp) {
+    // ===================== producers ========================================
+    // Warp 0 loads q and K, warp 2 loads V, each walking the same chunks.  A
+    // warp issues its TMA boxes one lane at a time (about 70 cycles each), so
+    // one warp issuing all 32 boxes of a chunk would take longer than HBM
+    // takes to deliver the chunk.
+    const bool is_k = warp == 0;
     const uint64_t pol_stream = l2_policy_evict_first();
     const uint64_t pol_keep = l2_policy_evict_last();
     bool ok = true;
@@ -726,7 +736,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       Seg sg;
       while (ok && next_seg<B, CB>(cur, sg, p, src)) {
         const int qs = qi & 1;
-        if (lane == 0) {
+        if (is_k && lane == 0) {
           ok = mbar_wait_bounded(&sm.qempty[qs], ((qi >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
           if (ok) {
             // q rows: heads [h G, h G + G) of row groups [z, z + RG), one box per 64-column half
@@ -742,34 +752,32 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         ++qi;
         // K and V loads of one chunk of nblk blocks; lane l < nblk holds the
         // physical block e of the chunk's block l
+        // This warp's operand of one chunk of nblk blocks; lane l < nblk holds
+        // the physical block e of the chunk's block l
         auto issue = [&](int nblk, int e) -> bool {
-          const int ks = ci % kKStages, vs = ci % kVStages;
+          const int ns = is_k ? kKStages : kVStages;
+          const int st = ci % ns;
+          uint64_t* empty = is_k ? &sm.kempty[st] : &sm.vempty[st];
+          uint64_t* full = is_k ? &sm.kfull[st] : &sm.vfull[st];
+          const CUtensorMap* map = is_k ? &map_k : &map_v;
           const int y = (e * Hkv + sg.h) * B;
           bool go = true;
           if (lane == 0) {
-            go = mbar_wait_bounded(&sm.kempty[ks], ((ci / kKStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
-            if (go) mbar_arrive_expect_tx(&sm.kfull[ks], nblk * 2 * kBlockBytes);
+            go = mbar_wait_bounded(empty, ((ci / ns) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+            if (go) mbar_arrive_expect_tx(full, nblk * 2 * kBlockBytes);
           }
           if (!__shfl_sync(0xffffffffu, go, 0)) return false;
           if (lane < nblk) {
-            uint8_t* base = sm.kbuf[ks] + lane * kBlockBytes;
-            tma_load_2d(base, &map_k, 0, y, &sm.kfull[ks], pol_stream);
-            tma_load_2d(base + kHalfBytes, &map_k, 64, y, &sm.kfull[ks], pol_stream);
+            uint8_t* base = (is_k ? sm.kbuf[st] : sm.vbuf[st]) + lane * kBlockBytes;
+            tma_load_2d(base, map, 0, y, full, pol_stream);
+            tma_load_2d(base + kHalfBytes, map, 64, y, full, pol_stream);
           }
           __syncwarp();
-          ++k_issued;
-          if (lane == 0) {
-            go = mbar_wait_bounded(&sm.vempty[vs], ((ci / kVStages) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
-            if (go) mbar_arrive_expect_tx(&sm.vfull[vs], nblk * 2 * kBlockBytes);
+          if (is_k) {
+            ++k_issued;
+          } else {
+            ++v_issued;
           }
-          if (!__shfl_sync(0xffffffffu, go, 0)) return false;
-          if (lane < nblk) {
-            uint8_t* base = sm.vbuf[vs] + lane * kBlockBytes;
-            tma_load_2d(base, &map_v, 0, y, &sm.vfull[vs], pol_stream);
-            tma_load_2d(base + kHalfBytes, &map_v, 64, y, &sm.vfull[vs], pol_stream);
-          }
-          __syncwarp();
-          ++v_issued;
           ++ci;
           return true;
         };
@@ -817,9 +825,12 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       }
     }
     if (lane == 0) {
-      sm.k_issued = k_issued;
-      sm.v_issued = v_issued;
-      sm.q_issued = q_issued;
+      if (is_k) {
+        sm.k_issued = k_issued;
+        sm.q_issued = q_issued;
+      } else {
+        sm.v_issued = v_issued;
+      }
       if (!ok) {
         sm.abort = 1;
         record_status(p.status, PA_DEV_TIMEOUT);
@@ -933,14 +944,14 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ===================== softmax + epilogue (warps 2-5) ====================
+    // ===================== softmax + epilogue (warps 3..) ====================
     // Per chunk i: softmax(i) then the epilogue of chunk i-1, so the PV of
     // chunk i-1 runs on the tensor core while the softmax of chunk i runs
     // here; chunks of consecutive segments form one stream.
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;   // token row of the chunk; head_dim index in the epilogue
-    const int ctid = tid - 64;        // 0 .. kSoftmaxThreads - 1
-    const int col0 = ((warp - 2) / 4) * RC;  // this warpgroup's query rows: col0 .. col0 + RC - 1
+    const int ctid = tid - 96;        // 0 .. kSoftmaxThreads - 1
+    const int col0 = ((warp - 3) / 4) * RC;  // this warpgroup's query rows: col0 .. col0 + RC - 1
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int my_col = col0 + lane / kLanesPerCol;  // the row this lane holds after a reduce
     const bool col_writer = (lane % kLanesPerCol) == 0;
