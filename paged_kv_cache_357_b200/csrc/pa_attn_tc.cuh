@@ -27,19 +27,21 @@
 // Work partition and split-unit merge: pa_decode_common.cuh (equal counts of
 // 8-block chunks per persistent CTA).
 //
-// Roles (96 + 128 x WG threads, one CTA per SM):
+// Roles (128 + 128 x WG threads, one CTA per SM):
 //   warp 0      K producer: resolves block ids (32 table entries per load,
 //               one batch ahead), issues 2-D TMA loads of the K tiles
 //               (64-column boxes, 128-byte swizzle) into a ring of 32 KB
 //               chunk stages, released when its QK is done, and a 3-D TMA
 //               load of the unit's q rows.
-//   warp 1      allocates TMEM; lane 0 issues every tcgen05.mma and
-//               tcgen05.commit, polling which of QK(next) and PV(oldest
-//               pending) is ready and issuing it.
+//   warp 1      allocates TMEM; lane 0 issues QK of each chunk (tcgen05.mma,
+//               tcgen05.commit) as soon as its K, q and S buffer are ready.
 //   warp 2      V producer: the same walk, V tiles into their own ring,
 //               released when the chunk's PV is done.  A warp issues TMA
 //               boxes one lane at a time, so K and V go out in parallel.
-//   warps 3..   softmax + epilogue (WG warpgroups), one TMEM lane (token row,
+//   warp 3      lane 0 issues PV of each chunk as soon as its P, V and O
+//               buffer are ready; with QK on its own thread neither product
+//               waits for the other's issue.
+//   warps 4..   softmax + epilogue (WG warpgroups), one TMEM lane (token row,
 //               then head_dim index) per thread: read S^T from TMEM, column
 //               maxima and sums by warp butterfly reduce-scatters, write P^T
 //               (bf16/fp16) into a swizzled buffer, zero V rows past the
@@ -75,7 +77,10 @@ constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 
 constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
 constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
 constexpr int kSoftmaxBarrier = 1;
-constexpr int kVWarp = 2;                  // the V producer; softmax warps start at 3
+constexpr int kQKWarp = 1;                 // allocates TMEM, issues QK
+constexpr int kVWarp = 2;                  // the V producer (warp 0 loads q and K)
+constexpr int kPVWarp = 3;                 // issues PV
+constexpr int kSoftmaxWarp0 = 4;           // first softmax warp
 // A row's probabilities are taken relative to a reference max that only moves
 // when a score exceeds it by more than this (log2 units): p <= 2^8 stays
 // exact enough in 16-bit and in the fp32 sums, and most chunks need neither
@@ -115,7 +120,7 @@ struct Rows {
   static constexpr int WG = R >= 16 ? 2 : 1;
   static constexpr int RC = R / WG;
   static constexpr int kSoftmaxThreads = 128 * WG;
-  static constexpr int kThreads = 96 + kSoftmaxThreads;          // + two producer warps + MMA warp
+  static constexpr int kThreads = 128 + kSoftmaxThreads;         // + K, QK, V and PV warps
   static constexpr int kLanesPerCol = 32 / RC;                    // lanes holding one column after a reduce
 };
 
@@ -142,7 +147,7 @@ struct TcSmem {
   uint64_t p_full[2];
   uint64_t o_full[2];
   uint64_t o_free[2];
-  uint64_t mma_done;
+  uint64_t mma_done[2];            // the QK and the PV issuer's last MMAs
   RangeSmem range;
   uint32_t tmem_base;
   int abort;
@@ -349,17 +354,20 @@ struct ChunkSrc {
 
 // ---- what a unit covers --------------------------------------------------------
 
-// Shared blocks of group g, or 0 when the group shares none: the prefix must
-// be shorter than every member's block count, so that every member keeps at
+// Token counts of the members of group g = sequences [s0, s1), at most RG
+// of them, loaded together (0 past s1), and the group's shared blocks: its
+// prefix length, or 0 when the group shares none.  The prefix must be
+// shorter than every member's block count, so that every member keeps at
 // least one block (its newest token) of its own.
-template <int BB>
-__device__ __forceinline__ int group_prefix_blocks(const DecodeParams& p, int s0, int s1, int g) {
+template <int RG, int BB>
+__device__ __forceinline__ int group_members(const DecodeParams& p, int g, int s0, int s1, int (&len)[RG]) {
   const int pb = __ldg(p.group_prefix + g);
-  if (pb <= 0) return 0;
-  for (int s = s0; s < s1; ++s) {
-    if (pb >= (checked_len(p, s, BB) + BB - 1) / BB) return 0;
-  }
-  return pb;
+#pragma unroll
+  for (int m = 0; m < RG; ++m) len[m] = s0 + m < s1 ? checked_len(p, s0 + m, BB) : 0;
+  bool fits = pb > 0;
+#pragma unroll
+  for (int m = 0; m < RG; ++m) fits = fits && (s0 + m >= s1 || pb < (len[m] + BB - 1) / BB);
+  return fits ? pb : 0;
 }
 
 __device__ __forceinline__ bool group_ok(const DecodeParams& p, int s0, int s1, int max_members) {
@@ -408,11 +416,12 @@ struct Source<kGroup, RG> {
   __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int g) const {
     const int s0 = __ldg(p.group_starts + g), s1 = __ldg(p.group_starts + g + 1);
     if (!group_ok(p, s0, s1, RG)) return SeqSpan{0, 0, 0};
-    const int pb = group_prefix_blocks<BB>(p, s0, s1, g);
+    int len[RG];
+    const int pb = group_members<RG, BB>(p, g, s0, s1, len);
     int ng = (pb + CB - 1) / CB;
-    for (int s = s0; s < s1; ++s) {
-      const int nb = (checked_len(p, s, BB) + BB - 1) / BB;
-      ng += (nb - pb + CB - 1) / CB;
+#pragma unroll
+    for (int m = 0; m < RG; ++m) {
+      if (s0 + m < s1) ng += ((len[m] + BB - 1) / BB - pb + CB - 1) / CB;
     }
     return SeqSpan{0, ng * CB, ng * CB * BB};
   }
@@ -427,13 +436,14 @@ struct Source<kGroup, RG> {
 // unit's chunks are consecutive blocks of its row, seen by all its rows.  A
 // group unit's chunks are the shared prefix (through the first member's row,
 // seen by every member's rows) and then each member's own blocks (its row,
-// seen by its own G rows).
-template <int kMode, int G>
+// seen by its own G rows); the members' lengths are read once, at start.
+template <int kMode, int G, int RG>
 struct ChunkWalk {
   // current part: table row, next block, end block, sequence tokens, rows
   int seq, j, jend, len, row_lo, row_hi;
   // group units only
   int s0, s1, pb, member;  // member = -1 while in the prefix
+  int mlen[kMode == kGroup ? RG : 1];
 
   __device__ __forceinline__ void start(const DecodeParams& p, const Seg& sg, int rows) {
     if constexpr (kMode != kGroup) {
@@ -446,26 +456,30 @@ struct ChunkWalk {
     } else {
       s0 = __ldg(p.group_starts + sg.s);
       s1 = __ldg(p.group_starts + sg.s + 1);
-      pb = group_prefix_blocks<B>(p, s0, s1, sg.s);
+      pb = group_members<RG, B>(p, sg.s, s0, s1, mlen);
       int skip = sg.j0 / CB;  // granules of the unit before this segment
       const int gp = (pb + CB - 1) / CB;
       if (skip < gp) {
         enter_prefix(skip);
       } else {
         skip -= gp;
-        for (member = 0; member < s1 - s0; ++member) {
-          const int nb = (checked_len(p, s0 + member, B) + B - 1) / B;
-          const int gm = (nb - pb + CB - 1) / CB;
-          if (skip < gm) break;
-          skip -= gm;
+        member = 0;
+#pragma unroll
+        for (int m = 0; m < RG; ++m) {
+          const int gm = s0 + m < s1 ? ((mlen[m] + B - 1) / B - pb + CB - 1) / CB : 0;
+          if (member == m && skip >= gm) {
+            skip -= gm;
+            member = m + 1;
+          }
         }
-        enter_member(p, skip);
+        enter_member(skip);
       }
     }
   }
 
   // The chunk at the walk's position; the walk moves past it.
   __device__ __forceinline__ ChunkSrc next(const DecodeParams& p) {
+    (void)p;
     ChunkSrc c;
     c.seq = seq;
     c.j = j;
@@ -478,7 +492,7 @@ struct ChunkWalk {
     if constexpr (kMode == kGroup) {
       if (j >= jend) {  // on to the next member with blocks of its own
         ++member;
-        enter_member(p, 0);
+        enter_member(0);
       }
     }
     return c;
@@ -494,12 +508,19 @@ struct ChunkWalk {
     row_lo = 0;
     row_hi = (s1 - s0) * G;
   }
-  __device__ __forceinline__ void enter_member(const DecodeParams& p, int granule) {
-    for (; member < s1 - s0; ++member) {
-      len = checked_len(p, s0 + member, B);
-      jend = (len + B - 1) / B;
-      if (jend > pb) break;  // a member without blocks of its own is skipped
+  // the first member from `member` on with blocks of its own (registers only)
+  __device__ __forceinline__ void enter_member(int granule) {
+    int next = s1 - s0, l = 0;
+#pragma unroll
+    for (int m = RG - 1; m >= 0; --m) {
+      if (m >= member && s0 + m < s1 && (mlen[m] + B - 1) / B > pb) {
+        next = m;
+        l = mlen[m];
+      }
     }
+    member = next;
+    len = l;
+    jend = (l + B - 1) / B;
     seq = s0 + member;
     j = pb + granule * CB;
     row_lo = member * G;
@@ -676,7 +697,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.o_free[i], 4 * WG);
     }
-    mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.mma_done[0], 1);
+    mbar_init(&sm.mma_done[1], 1);
     sm.abort = 0;
     sm.k_issued = 0;
     sm.k_consumed = 0;
@@ -689,7 +711,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
   }
-  if (warp == 1) {
+  if (warp == kQKWarp) {
     tmem_alloc(&sm.tmem_base, Sh::kTmemCols);
     tmem_relinquish();
   }
@@ -716,6 +738,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     // nothing to stream: straight to teardown
   } else if (warp == 0 || warp == kVWarp) {
     // ===================== producers ========================================
+    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
     // Warp 0 loads q and K, warp 2 loads V, each walking the same chunks.  A
     // warp issues its TMA boxes one lane at a time (about 70 cycles each), so
     // one warp issuing all 32 boxes of a chunk would take longer than HBM
@@ -805,7 +828,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           }
         } else {
           // Chunks from several rows: each chunk's entries, one chunk ahead.
-          ChunkWalk<kMode, G> walk;
+          ChunkWalk<kMode, G, RG> walk;
           walk.start(p, sg, 0);
           ChunkSrc cs = walk.next(p);
           int e_cur = (lane < cs.nblk) ? __ldg(p.block_tables + static_cast<size_t>(cs.seq) * p.max_nb + cs.j + lane) : 0;
@@ -836,107 +859,93 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         record_status(p.status, PA_DEV_TIMEOUT);
       }
     }
-  } else if (warp == 1) {
-    // ===================== MMA issuer ========================================
-    // A non-blocking scheduler: each pass tests whether QK of the next chunk
-    // (its K landed, its S buffer free, its q ready) or PV of the oldest chunk
-    // still waiting (its P written, its V landed, its O buffer free) can go,
-    // and issues whichever can, so PV of chunk i never waits for chunk i+1.
+  } else if (warp == kQKWarp) {
+    // ===================== QK issuer =========================================
+    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    // Lane 0 issues QK of each chunk once its K has landed, its S buffer is
+    // free and its q is loaded; it sleeps in the barrier waits in between.
     if (lane == 0) {
       constexpr uint32_t kIdescQK = make_idesc(kBf16, false, false, Nq);  // K: K-major A, q: K-major B
-      constexpr uint32_t kIdescPV = make_idesc(kBf16, true, true, Np);    // V: MN-major A, P: MN-major B
       bool ok = true;
-      int qk = 0, pv = 0, seg_i = 0, q_consumed = 0;
-      uint32_t ring = 0;  // valid tokens of each pending chunk (index & 3), 8 bits each
-      bool have_seg = false, q_ready = false, walk_done = false;
-      int c0 = 0;
+      int qk = 0, seg_i = 0;
       Seg sg;
-      ChunkWalk<kMode, G> walk;
-      uint64_t t_idle = 0;
-      uint32_t idle = 0;
-      while (ok) {
-        bool progress = false;
-        if (!walk_done && !have_seg) {
-          if (next_seg<B, CB>(cur, sg, p, src)) {
-            have_seg = true;
-            c0 = 0;
-            walk.start(p, sg, 0);
-          } else {
-            walk_done = true;
-          }
-        }
-        if (have_seg) {
-          const int qs = seg_i & 1;
-          if (!q_ready && mbar_test_wait(&sm.qfull[qs], (seg_i >> 1) & 1)) {
-            q_ready = true;
-            ++q_consumed;
-          }
+      while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+        const int qs = seg_i & 1;
+        ok = mbar_wait_bounded(&sm.qfull[qs], (seg_i >> 1) & 1, abort_flag, p.wait_limit_ns);
+        const uint32_t q0 = smem_u32(sm.q[qs]);
+        for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
           const int ks = qk % kKStages;
-          if (q_ready && qk - pv < 4 && mbar_test_wait(&sm.kfull[ks], (qk / kKStages) & 1) &&
-              mbar_test_wait(&sm.s_free[qk & 1], ((qk >> 1) & 1) ^ 1u)) {
-            tc_fence_after();
-            const uint32_t k0 = smem_u32(sm.kbuf[ks]);
-            const uint32_t q0 = smem_u32(sm.q[qs]);
+          ok = mbar_wait_bounded(&sm.kfull[ks], (qk / kKStages) & 1, abort_flag, p.wait_limit_ns) &&
+               mbar_wait_bounded(&sm.s_free[qk & 1], ((qk >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k0 = smem_u32(sm.kbuf[ks]);
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint64_t a = sw128_desc(k0 + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-              const uint64_t b = sw128_desc(q0 + (k >> 2) * Nq * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
-              umma(tmem + kColS + (qk & 1) * Nq, a, b, kIdescQK, k > 0 ? 1u : 0u);
-            }
-            umma_commit(&sm.s_full[qk & 1]);
-            umma_commit(&sm.kempty[ks]);
-            const int slot_shift = (qk & 3) * 8;
-            ring = (ring & ~(0xFFu << slot_shift)) | (static_cast<uint32_t>(walk.next(p).ntok) << slot_shift);
-            c0 += CB;
-            if (c0 >= sg.n) {  // last chunk of the segment: q may be reloaded after this QK
-              umma_commit(&sm.qempty[qs]);
-              have_seg = false;
-              q_ready = false;
-              ++seg_i;
-            }
-            ++qk;
-            progress = true;
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t a = sw128_desc(k0 + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+            const uint64_t b = sw128_desc(q0 + (k >> 2) * Nq * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+            umma(tmem + kColS + (qk & 1) * Nq, a, b, kIdescQK, k > 0 ? 1u : 0u);
           }
+          umma_commit(&sm.s_full[qk & 1]);
+          umma_commit(&sm.kempty[ks]);
+          ++qk;
         }
-        if (pv < qk) {
+        if (!ok) break;
+        umma_commit(&sm.qempty[qs]);  // q may be reloaded once the segment's last QK is done
+        ++seg_i;
+      }
+      // every MMA issued above completes before TMEM is released
+      umma_commit(&sm.mma_done[0]);
+      (void)mbar_wait_bounded(&sm.mma_done[0], 0, nullptr, p.wait_limit_ns);
+      sm.k_consumed = qk;
+      sm.q_consumed = seg_i;
+      if (!ok) {
+        sm.abort = 1;
+        record_status(p.status, PA_DEV_TIMEOUT);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kPVWarp) {
+    // ===================== PV issuer =========================================
+    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    // Lane 0 issues PV of each chunk once its P is written, its V has landed
+    // and its O buffer has been read; only the 16-token steps that hold
+    // valid tokens are issued.
+    if (lane == 0) {
+      constexpr uint32_t kIdescPV = make_idesc(kBf16, true, true, Np);  // V: MN-major A, P: MN-major B
+      bool ok = true;
+      int pv = 0;
+      Seg sg;
+      while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+        ChunkWalk<kMode, G, RG> walk;
+        walk.start(p, sg, 0);
+        for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
+          const int ntok = walk.next(p).ntok;
           const int pb = pv & 1;
           const uint32_t par = (pv >> 1) & 1;
           const int vs = pv % kVStages;
-          if (mbar_test_wait(&sm.p_full[pb], par) && mbar_test_wait(&sm.o_free[pb], par ^ 1u) &&
-              mbar_test_wait(&sm.vfull[vs], (pv / kVStages) & 1)) {
-            tc_fence_after();
-            const int ntok = static_cast<int>((ring >> ((pv & 3) * 8)) & 0xFFu);
-            const uint32_t v0 = smem_u32(sm.vbuf[vs]);
-            const uint32_t p0 = smem_u32(sm.p[pb]);
-            const int nks = (ntok + 15) / 16;
-            for (int k = 0; k < nks; ++k) {
-              const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
-              // tokens [16k, 16k + 16): two groups of 8 token rows; Np fits one swizzle atom
-              const uint64_t b = smem_desc(p0 + k * 16 * Sh::kPRowBytes, 0, 8 * Sh::kPRowBytes, Sh::kPLayout);
-              umma(tmem + kColO + pb * Np, a, b, kIdescPV, k > 0 ? 1u : 0u);
-            }
-            umma_commit(&sm.o_full[pb]);
-            umma_commit(&sm.vempty[vs]);
-            ++pv;
-            progress = true;
+          ok = mbar_wait_bounded(&sm.p_full[pb], par, abort_flag, p.wait_limit_ns) &&
+               mbar_wait_bounded(&sm.o_free[pb], par ^ 1u, abort_flag, p.wait_limit_ns) &&
+               mbar_wait_bounded(&sm.vfull[vs], (pv / kVStages) & 1, abort_flag, p.wait_limit_ns);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t v0 = smem_u32(sm.vbuf[vs]);
+          const uint32_t p0 = smem_u32(sm.p[pb]);
+          const int nks = (ntok + 15) / 16;
+          for (int k = 0; k < nks; ++k) {
+            const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
+            // tokens [16k, 16k + 16): two groups of 8 token rows; Np fits one swizzle atom
+            const uint64_t b = smem_desc(p0 + k * 16 * Sh::kPRowBytes, 0, 8 * Sh::kPRowBytes, Sh::kPLayout);
+            umma(tmem + kColO + pb * Np, a, b, kIdescPV, k > 0 ? 1u : 0u);
           }
-        } else if (walk_done) {
-          break;  // every chunk has had its QK and its PV
-        }
-        if (progress) {
-          idle = 0;
-        } else if ((++idle & 63u) == 0) {
-          const uint64_t now = global_timer_ns();
-          if (idle == 64) t_idle = now;
-          if (*abort_flag != 0 || now - t_idle > p.wait_limit_ns) ok = false;
+          umma_commit(&sm.o_full[pb]);
+          umma_commit(&sm.vempty[vs]);
+          ++pv;
         }
       }
-      // every MMA issued above completes before TMEM is released
-      umma_commit(&sm.mma_done);
-      (void)mbar_wait_bounded(&sm.mma_done, 0, nullptr, p.wait_limit_ns);
-      sm.k_consumed = qk;
+      umma_commit(&sm.mma_done[1]);
+      (void)mbar_wait_bounded(&sm.mma_done[1], 0, nullptr, p.wait_limit_ns);
       sm.v_consumed = pv;
-      sm.q_consumed = q_consumed;
       if (!ok) {
         sm.abort = 1;
         record_status(p.status, PA_DEV_TIMEOUT);
@@ -944,14 +953,15 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ===================== softmax + epilogue (warps 3..) ====================
+    // ===================== softmax + epilogue (warps 4..) ====================
+    if constexpr (WG == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
     // Per chunk i: softmax(i) then the epilogue of chunk i-1, so the PV of
     // chunk i-1 runs on the tensor core while the softmax of chunk i runs
     // here; chunks of consecutive segments form one stream.
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;   // token row of the chunk; head_dim index in the epilogue
-    const int ctid = tid - 96;        // 0 .. kSoftmaxThreads - 1
-    const int col0 = ((warp - 3) / 4) * RC;  // this warpgroup's query rows: col0 .. col0 + RC - 1
+    const int ctid = tid - 32 * kSoftmaxWarp0;  // 0 .. kSoftmaxThreads - 1
+    const int col0 = ((warp - kSoftmaxWarp0) / 4) * RC;  // this warpgroup's query rows: col0 .. col0 + RC - 1
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int my_col = col0 + lane / kLanesPerCol;  // the row this lane holds after a reduce
     const bool col_writer = (lane % kLanesPerCol) == 0;
@@ -1187,7 +1197,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     bool pending = false;   // the epilogue of chunk ci - 1 is still due
     while (ok && next_seg<B, CB>(cur, sg, p, src)) {
       const int rows = G * src.row_groups(p, sg.s);
-      ChunkWalk<kMode, G> walk;
+      ChunkWalk<kMode, G, RG> walk;
       walk.start(p, sg, rows);
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
         if (c0 == 0 && have_prev) stash_segment();
@@ -1235,7 +1245,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       (void)mbar_wait_bounded(&sm.qfull[k & 1], (k >> 1) & 1, nullptr, p.wait_limit_ns);
     }
   }
-  if (warp == 1) tmem_dealloc(tmem, Sh::kTmemCols);
+  if (warp == kQKWarp) tmem_dealloc(tmem, Sh::kTmemCols);
 }
 
 // ---- host side -----------------------------------------------------------------
