@@ -35,9 +35,10 @@
 //               load of the unit's q rows.
 //   warp 1      allocates TMEM; lane 0 issues QK of each chunk (tcgen05.mma,
 //               tcgen05.commit) as soon as its K, q and S buffer are ready.
-//   warp 2      V producer: the same walk, V tiles into their own ring,
-//               released when the chunk's PV is done.  A warp issues TMA
-//               boxes one lane at a time, so K and V go out in parallel.
+//   warp 2      V producer: the same walk, V tiles into their own ring
+//               (one 3-D box per block, both 64-column halves), released
+//               when the chunk's PV is done.  A warp issues TMA boxes one
+//               lane at a time, so K and V go out in parallel.
 //   warp 3      lane 0 issues PV of each chunk as soon as its P, V and O
 //               buffer are ready; with QK on its own thread neither product
 //               waits for the other's issue.
@@ -76,6 +77,11 @@ constexpr int kRowBytes = 128;             // one swizzle row: 64 elements
 constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 tokens
 constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
 constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
+// K stage: [half][128 tokens][64 columns], a K-major operand whose 8-row
+// groups are 1 KB apart across all 8 blocks; two boxes per block.
+// V stage: [block][half][16 tokens][64 columns], one 3-D box per block; each
+// 16-token PV step reads one block, halves kBlockBytes apart.
+constexpr int kVBlockBytes = 2 * kBlockBytes;
 constexpr int kSoftmaxBarrier = 1;
 constexpr int kQKWarp = 1;                 // allocates TMEM, issues QK
 constexpr int kVWarp = 2;                  // the V producer (warp 0 loads q and K)
@@ -791,9 +797,13 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           }
           if (!__shfl_sync(0xffffffffu, go, 0)) return false;
           if (lane < nblk) {
-            uint8_t* base = (is_k ? sm.kbuf[st] : sm.vbuf[st]) + lane * kBlockBytes;
-            tma_load_2d(base, map, 0, y, full, pol_stream);
-            tma_load_2d(base + kHalfBytes, map, 64, y, full, pol_stream);
+            if (is_k) {
+              uint8_t* base = sm.kbuf[st] + lane * kBlockBytes;
+              tma_load_2d(base, map, 0, y, full, pol_stream);
+              tma_load_2d(base + kHalfBytes, map, 64, y, full, pol_stream);
+            } else {
+              tma_load_3d(sm.vbuf[st] + lane * kVBlockBytes, map, 0, y, 0, full, pol_stream);
+            }
           }
           __syncwarp();
           if (is_k) {
@@ -933,7 +943,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           const uint32_t p0 = smem_u32(sm.p[pb]);
           const int nks = (ntok + 15) / 16;
           for (int k = 0; k < nks; ++k) {
-            const uint64_t a = sw128_desc(v0 + k * 16 * kRowBytes, kHalfBytes, 8 * kRowBytes);
+            const uint64_t a = sw128_desc(v0 + k * kVBlockBytes, kBlockBytes, 8 * kRowBytes);
             // tokens [16k, 16k + 16): two groups of 8 token rows; Np fits one swizzle atom
             const uint64_t b = smem_desc(p0 + k * 16 * Sh::kPRowBytes, 0, 8 * Sh::kPRowBytes, Sh::kPLayout);
             umma(tmem + kColO + pb * Np, a, b, kIdescPV, k > 0 ? 1u : 0u);
@@ -1093,8 +1103,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       // so that 0 * (whatever they hold) cannot reach the output
       if (col0 == 0 && (ch.ntok & 15) != 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
         (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
-        uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + r * kRowBytes);
-        uint4* v1 = reinterpret_cast<uint4*>(sm.vbuf[vs] + kHalfBytes + r * kRowBytes);
+        uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + (r / B) * kVBlockBytes + (r % B) * kRowBytes);
+        uint4* v1 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(v0) + kBlockBytes);
 #pragma unroll
         for (int i = 0; i < kRowBytes / 16; ++i) {
           v0[i] = make_uint4(0, 0, 0, 0);
@@ -1290,6 +1300,22 @@ inline bool make_map(CUtensorMap* map, const void* base, int rank, const unsigne
   return r == CUDA_SUCCESS;
 }
 
+// V pool as a 3-D tensor (64 columns, rows, 2 halves 128 bytes apart): one
+// box of 64 x 16 x 2 lands a block's rows as [half][16][64] in shared memory.
+inline bool make_map_v(CUtensorMap* map, const void* base, unsigned long long rows, bool bf16) {
+  auto encode = encode_fn();
+  if (encode == nullptr) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), 2};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(B), 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <bool kBf16, int G, int RG, int kMode>
 cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
@@ -1302,7 +1328,7 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
   const unsigned long long kv_outer[1] = {kv_rows};
   const uint32_t kv_box[1] = {static_cast<uint32_t>(B)};
   if (!make_map(&mq, prm.q, 3, q_outer, q_box, kBf16) || !make_map(&mk, prm.k_pool, 2, kv_outer, kv_box, kBf16) ||
-      !make_map(&mv, prm.v_pool, 2, kv_outer, kv_box, kBf16)) {
+      !make_map_v(&mv, prm.v_pool, kv_rows, kBf16)) {
     return cudaErrorInvalidValue;
   }
   return launch_overlapped(pa_decode_tc_kernel<kBf16, G, RG, kMode>, dim3(ctas), dim3(Rows<G * RG>::kThreads),
