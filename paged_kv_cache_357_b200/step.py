@@ -26,6 +26,7 @@ read that set are done, so an upload has the time of (sets - 1) steps.
 
 from __future__ import annotations
 
+import ctypes
 from typing import Optional
 
 from . import _lib
@@ -89,6 +90,18 @@ class PagedDecodeStep:
         else:
             self.workspace = _lib.alloc_decode_workspace(num_seqs, num_q_heads, k_pool, num_ctas, decode_flags)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
+        # Every buffer the kernels touch is fixed above, so the C calls are
+        # bound here once, checked by the same rules as the Python wrappers
+        # (which a first call below goes through); a step then passes only
+        # the counts that change.
+        self._c = _lib.load()
+        self._desc = _lib.pool_desc(k_pool)
+        self._desc_ref = ctypes.byref(self._desc)
+        self._opts = _lib.DecodeOpts(num_ctas, decode_flags)
+        self._opts_ref = ctypes.byref(self._opts)
+        self._cs = self.compute_stream.cuda_stream
+        self._ws = (self.workspace.data_ptr(), self.workspace.numel() * self.workspace.element_size())
+        self._checked = False
         self.steps = 0
         self.last_h2d_bytes = 0
         self.last_d2h_bytes = 0
@@ -135,24 +148,11 @@ class PagedDecodeStep:
             self.compute_stream.wait_event(bs.uploaded)
             if bs.used:
                 self.compute_stream.wait_event(bs.downloaded)  # out of this set was read back
-            if n_pairs > 0:
-                _lib.pa_copy_blocks(bs.pairs[:n_pairs], self.k_pool, self.v_pool, self.status,
-                                    stream=self.compute_stream)
-            if T > 0:
-                _lib.pa_cache_write(bs.new_k[:T], bs.new_v[:T], bs.slots[:T], self.k_pool, self.v_pool, self.status,
-                                    stream=self.compute_stream)
-            if self.q_len > 1:
-                _lib.pa_decode_multi(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out,
-                                     self.workspace, self.status, num_ctas=self.num_ctas, stream=self.compute_stream)
-            elif self.max_group_size > 0:
-                _lib.pa_decode_shared_prefix(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens,
-                                             bs.group_starts[: n_groups + 1], bs.group_prefix[:n_groups],
-                                             self.max_group_size, self.scale, bs.out, self.workspace, self.status,
-                                             num_ctas=self.num_ctas, stream=self.compute_stream)
+            if not self._checked:
+                self._launch_checked(bs, n_pairs, T, n_groups)
+                self._checked = True
             else:
-                _lib.pa_decode(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out,
-                               self.workspace, self.status, num_ctas=self.num_ctas, flags=self.decode_flags,
-                               stream=self.compute_stream)
+                self._launch_bound(bs, n_pairs, T, n_groups)
             bs.computed.record(self.compute_stream)
         with torch.cuda.stream(self.d2h_stream):
             self.d2h_stream.wait_event(bs.computed)
@@ -163,6 +163,54 @@ class PagedDecodeStep:
         self.last_h2d_bytes = h2d
         self.last_d2h_bytes = bs.out.numel() * bs.out.element_size()
         return bs.out_host
+
+    def _launch_checked(self, bs, n_pairs: int, T: int, n_groups: int) -> None:
+        """The step's kernels through the checking Python wrappers."""
+        cs = self.compute_stream
+        if n_pairs > 0:
+            _lib.pa_copy_blocks(bs.pairs[:n_pairs], self.k_pool, self.v_pool, self.status, stream=cs)
+        if T > 0:
+            _lib.pa_cache_write(bs.new_k[:T], bs.new_v[:T], bs.slots[:T], self.k_pool, self.v_pool, self.status,
+                                stream=cs)
+        if self.q_len > 1:
+            _lib.pa_decode_multi(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out,
+                                 self.workspace, self.status, num_ctas=self.num_ctas, flags=self.decode_flags,
+                                 stream=cs)
+        elif self.max_group_size > 0:
+            _lib.pa_decode_shared_prefix(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens,
+                                         bs.group_starts[: n_groups + 1], bs.group_prefix[:n_groups],
+                                         self.max_group_size, self.scale, bs.out, self.workspace, self.status,
+                                         num_ctas=self.num_ctas, flags=self.decode_flags, stream=cs)
+        else:
+            _lib.pa_decode(bs.q, self.k_pool, self.v_pool, bs.tables, bs.lens, self.scale, bs.out, self.workspace,
+                           self.status, num_ctas=self.num_ctas, flags=self.decode_flags, stream=cs)
+
+    def _launch_bound(self, bs, n_pairs: int, T: int, n_groups: int) -> None:
+        """The same kernels through the C entry points with the buffers'
+        addresses (the buffers, pools, workspace and stream never change)."""
+        c, desc, cs, st = self._c, self._desc_ref, self._cs, self.status.data_ptr()
+        kp, vp = self.k_pool.data_ptr(), self.v_pool.data_ptr()
+        if n_pairs > 0:
+            _check(c.pa_copy_blocks(bs.pairs.data_ptr(), n_pairs, kp, vp, st, desc, cs), "pa_copy_blocks")
+        if T > 0:
+            _check(c.pa_cache_write(bs.new_k.data_ptr(), bs.new_v.data_ptr(), bs.slots.data_ptr(), T, kp, vp, st,
+                                    desc, cs), "pa_cache_write")
+        S, max_nb = bs.tables.shape
+        ws, ws_bytes = self._ws
+        if self.q_len > 1:
+            _check(c.pa_decode_multi(bs.q.data_ptr(), kp, vp, bs.tables.data_ptr(), max_nb, bs.lens.data_ptr(), S,
+                                     self.q_len, self.Hq, self.scale, bs.out.data_ptr(), ws, ws_bytes, st, desc,
+                                     self._opts_ref, cs), "pa_decode_multi")
+        elif self.max_group_size > 0:
+            _check(c.pa_decode_shared_prefix(bs.q.data_ptr(), kp, vp, bs.tables.data_ptr(), max_nb,
+                                             bs.lens.data_ptr(), S, self.Hq, bs.group_starts.data_ptr(),
+                                             bs.group_prefix.data_ptr(), n_groups, self.max_group_size, self.scale,
+                                             bs.out.data_ptr(), ws, ws_bytes, st, desc, self._opts_ref, cs),
+                   "pa_decode_shared_prefix")
+        else:
+            _check(c.pa_decode_ex(bs.q.data_ptr(), kp, vp, bs.tables.data_ptr(), max_nb, bs.lens.data_ptr(), S,
+                                  self.Hq, self.scale, bs.out.data_ptr(), ws, ws_bytes, st, desc, self._opts_ref, cs),
+                   "pa_decode")
 
     def wait(self, result) -> None:
         """Block until the step that returned ``result`` has been read back."""
@@ -180,3 +228,8 @@ class PagedDecodeStep:
         """Synchronise every stream of the step and return the device status."""
         self.synchronize()
         return int(self.status.item())
+
+
+def _check(rc: int, name: str) -> None:
+    if rc != 0:
+        raise _lib.PaError(rc, name)
