@@ -24,8 +24,8 @@
 //            shared blocks once, seen by every member's rows, then each
 //            member's own blocks, seen by that member's rows only.
 //
-// Work partition and split-unit merge: pa_decode_common.cuh (equal counts of
-// 8-block chunks per persistent CTA).
+// Work partition and split-unit merge: pa_decode_common.cuh (ranges of equal
+// cost, 8-block chunks plus a fixed finish cost per unit, per CTA).
 //
 // Roles (128 + 128 x WG threads, one CTA per SM):
 //   warp 0      K producer: resolves block ids (32 table entries per load,
