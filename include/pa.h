@@ -89,8 +89,8 @@ typedef struct pa_decode_opts {
   int32_t flags;    /* 0, or PA_DECODE_CUDA_CORES_ONLY and/or PA_DECODE_TEST_WITHHOLD_COPIES */
 } pa_decode_opts;
 
-/* Failure-detection test hook for pa_decode_opts.flags: the producer warp
- * issues no copies, every consumer wait runs out after about 20 ms, and the
+/* Failure-detection test hook for pa_decode_opts.flags: the producer warps
+ * issue no copies, every consumer wait runs out after about 20 ms, and the
  * kernel returns early with PA_DEV_TIMEOUT in *dev_status and the GPU context
  * still usable.  Output is not written.  Never set it outside such tests. */
 #define PA_DECODE_TEST_WITHHOLD_COPIES 1
