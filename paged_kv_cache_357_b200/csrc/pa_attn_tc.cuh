@@ -87,6 +87,10 @@ constexpr int kQKWarp = 1;                 // allocates TMEM, issues QK
 constexpr int kVWarp = 2;                  // the V producer (warp 0 loads q and K)
 constexpr int kPVWarp = 3;                 // issues PV
 constexpr int kSoftmaxWarp0 = 4;           // first softmax warp
+// With two softmax warpgroups the control warpgroup hands registers to them
+// (setmaxnreg): 128 x 72 + 256 x 216 = 384 x 168, the launch's allocation.
+constexpr int kCtrlRegs = 72;
+constexpr int kSoftmaxRegs = 216;
 // A row's probabilities are taken relative to a reference max that only moves
 // when a score exceeds it by more than this (log2 units): p <= 2^8 stays
 // exact enough in 16-bit and in the fp32 sums, and most chunks need neither
@@ -744,7 +748,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     // nothing to stream: straight to teardown
   } else if (warp == 0 || warp == kVWarp) {
     // ===================== producers ========================================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     // Warp 0 loads q and K, warp 2 loads V, each walking the same chunks.  A
     // warp issues its TMA boxes one lane at a time (about 70 cycles each), so
     // one warp issuing all 32 boxes of a chunk would take longer than HBM
@@ -871,7 +875,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     }
   } else if (warp == kQKWarp) {
     // ===================== QK issuer =========================================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     // Lane 0 issues QK of each chunk once its K has landed, its S buffer is
     // free and its q is loaded; it sleeps in the barrier waits in between.
     if (lane == 0) {
@@ -917,7 +921,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     __syncwarp();
   } else if (warp == kPVWarp) {
     // ===================== PV issuer =========================================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     // Lane 0 issues PV of each chunk once its P is written, its V has landed
     // and its O buffer has been read; only the 16-token steps that hold
     // valid tokens are issued.
@@ -964,7 +968,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     __syncwarp();
   } else {
     // ===================== softmax + epilogue (warps 4..) ====================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+    if constexpr (WG == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // Per chunk i: softmax(i) then the epilogue of chunk i-1, so the PV of
     // chunk i-1 runs on the tensor core while the softmax of chunk i runs
     // here; chunks of consecutive segments form one stream.
@@ -1330,6 +1334,17 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
   if (!make_map(&mq, prm.q, 3, q_outer, q_box, kBf16) || !make_map(&mk, prm.k_pool, 2, kv_outer, kv_box, kBf16) ||
       !make_map_v(&mv, prm.v_pool, kv_rows, kBf16)) {
     return cudaErrorInvalidValue;
+  }
+  if constexpr (Rows<G * RG>::WG == 2) {
+    // setmaxnreg only moves registers inside the launch's allocation; should
+    // a build give the kernel fewer than the split needs, the softmax warps'
+    // increase would wait forever, so such a kernel is not launched.
+    static const bool regs_fit = [] {
+      cudaFuncAttributes a{};
+      return cudaFuncGetAttributes(&a, pa_decode_tc_kernel<kBf16, G, RG, kMode>) == cudaSuccess &&
+             a.numRegs * Rows<G * RG>::kThreads >= 128 * kCtrlRegs + 256 * kSoftmaxRegs;
+    }();
+    if (!regs_fit) return cudaErrorInvalidConfiguration;
   }
   return launch_overlapped(pa_decode_tc_kernel<kBf16, G, RG, kMode>, dim3(ctas), dim3(Rows<G * RG>::kThreads),
                            static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
