@@ -177,7 +177,9 @@ PA_API pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_p
  * GPU that loads the library holds that array until the process exits.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it.  Make
- *     that first call on a device before any stream capture.
+ *     that first call on a device before any stream capture.  The cache is
+ *     tied to the device's context: after a cudaDeviceReset the next call
+ *     looks the address up again, and is then a first call once more.
  *   - Each call clears the arrival counters it needs (cudaMemsetAsync on
  *     `stream`) and launches the decode.  Nothing is allocated or freed.
  *   - All calls share the one array and it keeps the last call's contents:

@@ -790,18 +790,54 @@ constexpr int kMaxDevices = 64;
 // symbol, so its device address is looked up below.
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
-// Device address of g_decode_scratch on the current device, looked up on the
-// first call per device (with that device current) and cached.
+// The current context's process-unique id (cuCtxGetId never hands out an id
+// twice in a process), or 0 when no context is current or the driver entry
+// points are missing.  Reached through the runtime's driver entry point
+// table, so libpa needs no link against the driver library.
+static unsigned long long current_context_id() {
+  using GetCurrentFn = int (*)(void**);
+  using GetIdFn = int (*)(void*, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrentFn>(f);
+    }
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess) {
+      get_id = reinterpret_cast<GetIdFn>(f);
+    }
+    looked_up = true;
+  }
+  void* ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != 0 || ctx == nullptr) return 0;
+  return get_id(ctx, &id) == 0 ? id : 0;
+}
+
+// Device address of g_decode_scratch on the current device.  It is looked up
+// with that device current on the first call, and again whenever the
+// device's current context is another one than at the last lookup (after a
+// cudaDeviceReset the module is loaded anew and the array may sit
+// elsewhere); otherwise the cached address is used.
 static bool no_alloc_scratch_address(void** addr) {
   static std::mutex mu;
   static void* cached[kMaxDevices] = {};
+  static unsigned long long cached_ctx[kMaxDevices] = {};
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (cached[dev] == nullptr || ctx == 0 || ctx != cached_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return false;
     cached[dev] = p;
+    // the lookup makes the device's primary context current if none was
+    cached_ctx[dev] = current_context_id();
   }
   *addr = cached[dev];
   return true;

@@ -2,11 +2,17 @@
 run one step through the C-ABI binding, run the oracle step on the same bits,
 and compare.
 
-Tolerance (the reading used throughout): a decode output element passes when
-|gpu - oracle| <= 2e-3 + 1e-2 * |oracle| — max-abs 2e-3 near zero, max-rel
-1e-2 elsewhere, the allclose form; see the design notes for why the two
-bounds combine this way (rounding the output to bf16 alone moves a value of
-magnitude 1 by up to 2^-9 = 1.95e-3).
+Tolerance (the reading used throughout).  The stated bounds are max-abs 2e-3
+and max-rel 1e-2.  Each is asserted where the 16-bit output can meet it:
+
+* max-abs: |gpu - oracle| <= 2e-3 for every element with |oracle| < 0.5.
+  There, rounding to bf16 alone moves a value by at most 2^-10 = 9.8e-4, so
+  the bound leaves about 1e-3 for the arithmetic.  Above 0.5 the rounding
+  alone can reach 2^-9 = 1.95e-3 (and 3.9e-3 in [1, 2)), so an exact answer
+  correctly rounded could fail an absolute bound there.
+* max-rel: |gpu - oracle| / |oracle| <= 1e-2 for every element with
+  |oracle| >= 0.1 (bf16 rounding is at most 2^-9 = 0.39 % relative).
+* and every element, whatever its size, within 2e-3 + 1e-2 * |oracle|.
 """
 
 from __future__ import annotations
@@ -88,14 +94,23 @@ def oracle_step(layout: PagedLayout, values: PagedValues, *, do_copy=True, do_wr
     return out, kp, vp
 
 
+ABS_BELOW = 0.5   # max-abs is asserted for |oracle| below this
+REL_ABOVE = 0.1   # max-rel is asserted for |oracle| at or above this
+
+
 def attention_errors(got: np.ndarray, ref: np.ndarray):
+    """(max abs error over |ref| < ABS_BELOW, max rel error over |ref| >=
+    REL_ABOVE, max abs error over all elements)."""
     err = np.abs(got - ref)
-    big = np.abs(ref) >= 0.1
-    max_rel = float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0
-    return float(err.max()) if err.size else 0.0, max_rel
+    mag = np.abs(ref)
+    small, big = mag < ABS_BELOW, mag >= REL_ABOVE
+    max_abs = float(err[small].max()) if small.any() else 0.0
+    max_rel = float((err[big] / mag[big]).max()) if big.any() else 0.0
+    return max_abs, max_rel, float(err.max()) if err.size else 0.0
 
 
 def assert_attention_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    """Assert the tolerance reading above; returns attention_errors."""
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     err = np.abs(got - ref)
@@ -106,6 +121,10 @@ def assert_attention_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
             f"{what}: {int(bad.sum())} of {bad.size} elements outside 2e-3 + 1e-2*|ref|; "
             f"max abs err {err.max():.3e}; first bad {idx}; got {got[bad][:5]} ref {ref[bad][:5]}"
         )
+    max_abs, max_rel, max_all = attention_errors(got, ref)
+    assert max_abs <= ATOL, f"{what}: max abs err {max_abs:.3e} over |ref| < {ABS_BELOW} exceeds {ATOL}"
+    assert max_rel <= RTOL, f"{what}: max rel err {max_rel:.3e} over |ref| >= {REL_ABOVE} exceeds {RTOL}"
+    return max_abs, max_rel, max_all
 
 
 def subproblem(layout: PagedLayout, values_dev, seqs):

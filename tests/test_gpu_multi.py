@@ -1,7 +1,7 @@
 """GPU parity of multi-query paged attention (pa_decode_multi, the
 tensor-core kernel with q_len causal positions per sequence) against the
-float64 oracle's decode_multi, element by element within
-2e-3 + 1e-2*|oracle|.  Inputs: seeded layouts whose cache already holds every
+float64 oracle's decode_multi, element by element: max-abs
+2e-3 where |oracle| < 0.5, max-rel 1e-2 where |oracle| >= 0.1.  Inputs: seeded layouts whose cache already holds every
 token (the q_len new ones included), padding rows and unused blocks NaN."""
 
 import numpy as np

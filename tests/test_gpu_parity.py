@@ -1,8 +1,8 @@
 """GPU parity of the CUDA path (through the C ABI) against the float64 oracle.
 
 Bit-exact: cache write, block copy, the pools after a step, and everything
-the block tables index.  Decode: within 2e-3 + 1e-2*|oracle| per element
-(see tests/pa_testlib.py).  Inputs are the seeded workloads; padding rows and
+the block tables index.  Decode: max-abs 2e-3 where |oracle| < 0.5
+and max-rel 1e-2 where |oracle| >= 0.1, per element (tests/pa_testlib.py).  Inputs are the seeded workloads; padding rows and
 unused blocks of every pool hold NaN.
 """
 

@@ -2,7 +2,8 @@
 per (group, kv head) streams the group's shared blocks once for every
 member's heads, then each member's own blocks for its heads) against the
 float64 decode oracle — the result is plain decode; only the memory reads
-differ — element by element within 2e-3 + 1e-2*|oracle|.  Groups come from
+differ — element by element: max-abs 2e-3 where |oracle| < 0.5, max-rel
+1e-2 where |oracle| >= 0.1.  Groups come from
 pa_shared_prefix_groups on the host tables."""
 
 import numpy as np
