@@ -46,7 +46,8 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "pa_decode_llama3_8b.md")
 KERNEL_SOURCES = [
     os.path.join(ROOT, "paged_kv_cache_357_b200", "csrc", name)
-    for name in ("pa_decode.cu", "pa_decode_tc.cu", "pa_attn_tc.cuh", "pa_decode_common.cuh", "pa_device.cuh")
+    for name in ("pa_decode.cu", "pa_decode_tc.cu", "pa_decode_tc_blocks.cu", "pa_attn_tc.cuh",
+                 "pa_decode_common.cuh", "pa_device.cuh")
 ]
 
 
@@ -65,7 +66,8 @@ def parse_args(argv=None):
                          "cuda_cores: pa_decode held to its CUDA-core kernel (PA_DECODE_CUDA_CORES_ONLY)")
     ap.add_argument("--max-group", type=int, default=4, help="members per shared-prefix group")
     ap.add_argument("--batch", type=int, default=0,
-                    help="sequences per GPU for the llama7b / llama3_8b(_spec4) / llama2_70b_shared workloads (0 = the workload's own)")
+                    help="sequences per GPU for the llama7b / llama3_8b(_spec4, _prefill256) / llama2_70b_shared "
+                         "workloads (0 = the workload's own)")
     return ap.parse_args(argv)
 
 
@@ -98,6 +100,21 @@ def step_bytes(L, mode: str = "plain") -> dict:
                 write=write, copy=copy, step=decode + write + copy, tile_pair=tile_pair, tiles=nb * Hkv)
 
 
+def decode_flops(L) -> int:
+    """Multiply-add flops of the decode's two products, 2 * D each per
+    (query row, visible token) pair: scores q . K and the weighted sum of V.
+    Position i of a multi-query step sees seq_len - q_len + i + 1 tokens."""
+    import numpy as np
+
+    n = L.seq_lens.astype(np.int64)
+    if L.q_len == 1:
+        pairs = int(n.sum())
+    else:
+        ok = n >= L.q_len
+        pairs = int((L.q_len * (n[ok] - L.q_len) + L.q_len * (L.q_len + 1) // 2).sum())
+    return 4 * pairs * L.num_q_heads * L.head_dim
+
+
 def measured_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -121,7 +138,7 @@ def decode_kernel_name(L, mode: str = "plain") -> str:
         return "pa_decode_tc_kernel, multi-query (tcgen05)"
     if mode == "shared_prefix":
         return "pa_decode_tc_kernel, group units: shared prefix once, then each member's blocks (tcgen05)"
-    if mode != "cuda_cores" and L.head_dim == 128 and L.block_size == 16 and L.group in (1, 2, 4, 8):
+    if mode != "cuda_cores" and L.head_dim == 128 and L.block_size in (8, 16, 32) and L.group in (1, 2, 4, 8):
         return "pa_decode_tc_kernel (tcgen05)"
     return "pa_decode_kernel (CUDA cores)"
 
@@ -378,7 +395,7 @@ def cpu_baseline(L, budget_s: float, args=None) -> dict:
 
 
 def make_layout(args):
-    from workloads import CONFIGS, config_llama2_70b_shared, config_llama3_8b, config_llama7b
+    from workloads import CONFIGS, config_llama2_70b_shared, config_llama3_8b, config_llama3_8b_prefill, config_llama7b
 
     if args.batch:
         def shared(batch):
@@ -388,6 +405,7 @@ def make_layout(args):
 
         makers = {"llama3_8b": config_llama3_8b, "llama7b": config_llama7b,
                   "llama3_8b_spec4": lambda batch: config_llama3_8b(batch=batch, q_len=4),
+                  "llama3_8b_prefill256": lambda batch: config_llama3_8b_prefill(batch=batch),
                   "llama2_70b_shared": shared}
         if args.config not in makers:
             raise SystemExit(f"--batch applies to {sorted(makers)} only")
@@ -554,12 +572,35 @@ def run_ours(args):
                               max_group_size=args.max_group if groups is not None else 0,
                               decode_flags=decode_flags)
 
-    def e2e_step():
-        return step.run(host["q"], host["tables"], host["lens"], host["new_k"], host["new_v"],
-                        host["slots"] if has_write else None, host["pairs"],
-                        group_starts=host.get("group_starts"), group_prefix_blocks=host.get("group_prefix"))
+    # The step's inputs live in the step's pinned staging areas (one per
+    # buffer set, filled once from the host tensors above: a serving loop
+    # would build its batch there), so each step uploads them in one copy.
+    staged = {}
 
-    for _ in range(args.warmup):
+    def e2e_step():
+        k = step.steps % len(step.sets)
+        v = step.staging()
+        if k not in staged:
+            fields = [("q", host["q"]), ("block_tables", host["tables"]), ("seq_lens", host["lens"])]
+            if has_write:
+                fields += [("new_k", host["new_k"]), ("new_v", host["new_v"]), ("slot_mapping", host["slots"])]
+            if has_copy:
+                fields.append(("copy_pairs", host["pairs"]))
+            if groups is not None:
+                fields += [("group_starts", host["group_starts"]), ("group_prefix_blocks", host["group_prefix"])]
+            staged[k] = {}
+            for name, src in fields:
+                dst = v[name][: src.shape[0]]
+                dst.copy_(src)
+                staged[k][name] = dst
+        a = staged[k]
+        return step.run(a["q"], a["block_tables"], a["seq_lens"], a.get("new_k"), a.get("new_v"),
+                        a.get("slot_mapping"), a.get("copy_pairs"), group_starts=a.get("group_starts"),
+                        group_prefix_blocks=a.get("group_prefix_blocks"))
+
+    # untimed: every buffer set's first steps (the first runs through the
+    # checking wrappers, each set's next one captures its graph)
+    for _ in range(max(args.warmup, len(step.sets) + 1)):
         e2e_step()
     step.synchronize()
     K2 = max(1, min(K, 500))
@@ -617,6 +658,7 @@ def run_ours(args):
             "tokens_per_s_note": ("one new token per sequence per single-layer step" if L.q_len == 1 else
                                   f"{L.q_len} query positions per sequence per single-layer step"),
             "decode_ms": decode_mean_ms,
+            "decode_tflops": decode_flops(L) / (decode_mean_ms * 1e-3) / 1e12,
             "decode_ms_p50": decode_ms[K // 2],
             "bytes": nbytes,
             "roofline": {
@@ -638,6 +680,9 @@ def run_ours(args):
                 "h2d_bytes_per_step": step.last_h2d_bytes,
                 "d2h_bytes_per_step": step.last_d2h_bytes,
                 "steps": K2,
+                "how": "PagedDecodeStep from pinned staging buffers: per step one H2D copy of the packed inputs, "
+                       "the step's kernels replayed as a CUDA graph, one D2H copy of the output; three buffer "
+                       "sets overlap neighbouring steps' copies and kernels",
                 "link_gbs": link,
                 "link_note": "this box's pinned-copy bandwidth for one step's input and output bytes, "
                              "measured outside the timed region (context: e2e is bound by it when slow)",

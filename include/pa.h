@@ -211,8 +211,13 @@ PA_API pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const voi
  *   others   as pa_decode
  * q_len == 1 is pa_decode.  For q_len >= 2 the tensor-core kernel runs:
  * head_dim 128, block_size 16, group size G = num_q_heads / num_kv_heads in
- * {1, 2, 4, 8} and G * q_len <= 32 (G * q_len rounded up to a power of two);
- * other shapes return PA_ERR_UNSUPPORTED, as does PA_DECODE_CUDA_CORES_ONLY.
+ * {1, 2, 4, 8}, any q_len.  One unit of work carries up to 32 query rows
+ * (G heads times a power-of-two count of positions); when G * q_len is
+ * larger (a prefill chunk), each sequence is split into row tiles of 32 / G
+ * positions, each tile a unit that reads only the blocks its last position
+ * sees, the tiles of a sequence adjacent so that their reads of the same
+ * blocks mostly hit in L2.  Other shapes return PA_ERR_UNSUPPORTED, as does
+ * PA_DECODE_CUDA_CORES_ONLY.
  * A sequence with seq_lens[s] == 0 gets zero outputs; 0 < seq_lens[s] <
  * q_len is PA_DEV_BAD_SEQ_LEN (zero outputs).  Workspace: as pa_decode, sized
  * by pa_decode_multi_workspace_bytes (0 for invalid or unsupported shapes).

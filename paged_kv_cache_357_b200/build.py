@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(HERE, "libpa.so")
 SOURCES = [
     "pa_decode.cu",
     "pa_decode_tc.cu",
+    "pa_decode_tc_blocks.cu",
     "pa_attn_tc_multi.cu",
     "pa_attn_tc_group.cu",
     "pa_kv_ops.cu",

@@ -69,19 +69,36 @@ namespace pa {
 namespace tc {
 
 constexpr int D = 128;
-constexpr int B = 16;
 constexpr int kChunkTok = 128;             // tokens per chunk = MMA M of QK
-constexpr int CB = kChunkTok / B;          // blocks per chunk
 constexpr int kKStages = 2;                // K is released as soon as its QK completes
 constexpr int kRowBytes = 128;             // one swizzle row: 64 elements
 constexpr int kHalfBytes = kChunkTok * kRowBytes;  // 64 head_dim columns x 128 tokens
 constexpr int kOperandBytes = 2 * kHalfBytes;      // head_dim [0:64) then [64:128)
-constexpr int kBlockBytes = B * kRowBytes;         // one block's rows in one half
-// K stage: [half][128 tokens][64 columns], a K-major operand whose 8-row
-// groups are 1 KB apart across all 8 blocks; two boxes per block.
-// V stage: [block][half][16 tokens][64 columns], one 3-D box per block; each
-// 16-token PV step reads one block, halves kBlockBytes apart.
-constexpr int kVBlockBytes = 2 * kBlockBytes;
+
+// Shapes that follow from the block size BB (8, 16 or 32 tokens).  A chunk
+// is always 128 tokens, so CB = 16, 8 or 4 blocks.
+//   V stage: [block][half][BB tokens][64 columns], one 3-D box per block
+//   (both 64-column halves, kBlockBytes apart).  A 16-token PV step reads
+//   two blocks (BB = 8), one block or half a block.
+//   K stage, a K-major operand whose 8-token groups must sit a uniform
+//   distance apart: for BB = 8 every block is one such group, so the V
+//   layout serves (one 3-D box per block, groups 2 KB apart, halves 1 KB
+//   apart); for BB = 16, 32 [half][128 tokens][64 columns] with two 2-D boxes
+//   per block (groups 1 KB apart, halves kHalfBytes apart).
+template <int BB>
+struct Blk {
+  static_assert(BB == 8 || BB == 16 || BB == 32, "blocks of 8, 16 or 32 tokens");
+  static constexpr int CB = kChunkTok / BB;            // blocks per chunk
+  static constexpr int kBlockBytes = BB * kRowBytes;   // one block's rows in one half
+  static constexpr int kVBlockBytes = 2 * kBlockBytes;  // both halves of one block
+  static constexpr bool kK3D = BB == 8;
+  static constexpr int kKGroupBytes = kK3D ? kVBlockBytes : 8 * kRowBytes;  // K: 8-token group stride
+  static constexpr int kKHalfBytes = kK3D ? kBlockBytes : kHalfBytes;       // K: second 64 columns
+  static constexpr int kKBoxBytes = kK3D ? kVBlockBytes : kBlockBytes;      // K: one box (per block / half)
+  static constexpr int kVGroupBytes = BB == 8 ? kVBlockBytes : 8 * kRowBytes;  // V: 8-token group stride
+  // V stage offset of token t of the chunk (its row in the first half)
+  __host__ __device__ static constexpr int v_offset(int t) { return (t / BB) * kVBlockBytes + (t % BB) * kRowBytes; }
+};
 constexpr int kSoftmaxBarrier = 1;
 constexpr int kQKWarp = 1;                 // allocates TMEM, issues QK
 constexpr int kVWarp = 2;                  // the V producer (warp 0 loads q and K)
@@ -360,6 +377,7 @@ struct ChunkSrc {
   int ntok;            // valid tokens
   int len;             // tokens of the row's sequence (the causal limit's reference)
   int row_lo, row_hi;  // query rows [row_lo, row_hi) that see these tokens
+  int pos0;            // multi-query: position of the unit's first row group
 };
 
 // ---- what a unit covers --------------------------------------------------------
@@ -396,23 +414,36 @@ struct Source<kDecode, RG> {
     return SeqSpan{0, (len + BB - 1) / BB, len};
   }
   __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
+  __device__ __forceinline__ int table_row(const DecodeParams&, int s) const { return s; }
   __device__ __forceinline__ int row_group0(const DecodeParams&, int s) const { return s; }
   __device__ __forceinline__ int row_groups(const DecodeParams&, int) const { return 1; }
 };
 
-// A sequence with q_len query positions, causal among the new tokens.  A
-// sequence shorter than q_len is treated as empty.
+// Query positions of a sequence, causal among the new tokens.  Unit u is row
+// tile t = u % q_tiles of sequence s = u / q_tiles: positions [t RG,
+// min(q_len, (t + 1) RG)), so a sequence with G x q_len query rows past what
+// one unit holds is covered by several units.  A tile reads only the blocks
+// its last position sees.  A sequence shorter than q_len is treated as empty.
 template <int RG>
 struct Source<kMulti, RG> {
   template <int BB>
-  __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int s) const {
+  __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int u) const {
+    const int s = u / p.q_tiles;
     int len = checked_len(p, s, BB);
     if (len < p.q_len) len = 0;
-    return SeqSpan{0, (len + BB - 1) / BB, len};
+    const int end = min(p.q_len, (u - s * p.q_tiles + 1) * RG);  // positions up to the tile's end
+    const int seen = len > 0 ? len - p.q_len + end : 0;           // tokens the tile's last position sees
+    return SeqSpan{0, (seen + BB - 1) / BB, len};
   }
-  __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
-  __device__ __forceinline__ int row_group0(const DecodeParams& p, int s) const { return s * p.q_len; }
-  __device__ __forceinline__ int row_groups(const DecodeParams& p, int) const { return p.q_len; }
+  __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs * p.q_tiles; }
+  __device__ __forceinline__ int table_row(const DecodeParams& p, int u) const { return u / p.q_tiles; }
+  __device__ __forceinline__ int pos0(const DecodeParams& p, int u) const { return (u % p.q_tiles) * RG; }
+  __device__ __forceinline__ int row_group0(const DecodeParams& p, int u) const {
+    return table_row(p, u) * p.q_len + pos0(p, u);
+  }
+  __device__ __forceinline__ int row_groups(const DecodeParams& p, int u) const {
+    return min(RG, p.q_len - pos0(p, u));
+  }
 };
 
 // A group of sequences [starts[g], starts[g+1]): the shared prefix, then each
@@ -428,6 +459,7 @@ struct Source<kGroup, RG> {
     if (!group_ok(p, s0, s1, RG)) return SeqSpan{0, 0, 0};
     int len[RG];
     const int pb = group_members<RG, BB>(p, g, s0, s1, len);
+    constexpr int CB = Blk<BB>::CB;
     int ng = (pb + CB - 1) / CB;
 #pragma unroll
     for (int m = 0; m < RG; ++m) {
@@ -436,6 +468,7 @@ struct Source<kGroup, RG> {
     return SeqSpan{0, ng * CB, ng * CB * BB};
   }
   __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_groups; }
+  __device__ __forceinline__ int table_row(const DecodeParams& p, int g) const { return __ldg(p.group_starts + g); }
   __device__ __forceinline__ int row_group0(const DecodeParams& p, int g) const { return __ldg(p.group_starts + g); }
   __device__ __forceinline__ int row_groups(const DecodeParams& p, int g) const {
     return __ldg(p.group_starts + g + 1) - __ldg(p.group_starts + g);
@@ -447,22 +480,26 @@ struct Source<kGroup, RG> {
 // group unit's chunks are the shared prefix (through the first member's row,
 // seen by every member's rows) and then each member's own blocks (its row,
 // seen by its own G rows); the members' lengths are read once, at start.
-template <int kMode, int G, int RG>
+template <int kMode, int G, int RG, int B>
 struct ChunkWalk {
+  static constexpr int CB = Blk<B>::CB;
   // current part: table row, next block, end block, sequence tokens, rows
   int seq, j, jend, len, row_lo, row_hi;
+  int pos0;  // multi-query: position of the unit's first row group
   // group units only
   int s0, s1, pb, member;  // member = -1 while in the prefix
   int mlen[kMode == kGroup ? RG : 1];
 
   __device__ __forceinline__ void start(const DecodeParams& p, const Seg& sg, int rows) {
+    pos0 = 0;
     if constexpr (kMode != kGroup) {
-      seq = sg.s;
+      seq = kMode == kMulti ? sg.s / p.q_tiles : sg.s;
       j = sg.j0;
       jend = sg.j0 + sg.n;
       len = sg.len;
       row_lo = 0;
       row_hi = rows;
+      if constexpr (kMode == kMulti) pos0 = (sg.s % p.q_tiles) * RG;
     } else {
       s0 = __ldg(p.group_starts + sg.s);
       s1 = __ldg(p.group_starts + sg.s + 1);
@@ -498,6 +535,7 @@ struct ChunkWalk {
     c.len = len;
     c.row_lo = row_lo;
     c.row_hi = row_hi;
+    c.pos0 = pos0;
     j += c.nblk;
     if constexpr (kMode == kGroup) {
       if (j >= jend) {  // on to the next member with blocks of its own
@@ -542,7 +580,7 @@ struct ChunkWalk {
 // partition the sequences and fit the kernel, and zero the outputs of groups
 // with nothing to read.  Group g is handled by thread g / gridDim.x of CTA
 // g % gridDim.x.
-template <int RG>
+template <int RG, int B>
 __device__ void group_bookkeeping(const DecodeParams& p, const Source<kGroup, RG>& src) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long g = static_cast<long long>(threadIdx.x) * gridDim.x + blockIdx.x; g < p.num_groups; g += stride) {
@@ -564,21 +602,22 @@ __device__ void group_bookkeeping(const DecodeParams& p, const Source<kGroup, RG
   }
 }
 
-// kDecode and kMulti: zero the output rows of sequences with nothing to read
-// (length 0, invalid, or shorter than q_len); sequence s by CTA s % gridDim.x.
-template <int kMode, int RG>
+// kDecode and kMulti: zero the output rows of units with nothing to read
+// (length 0, invalid, or shorter than q_len); unit u by CTA u % gridDim.x.
+template <int kMode, int RG, int B>
 __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>& src) {
   const long long nctas = gridDim.x, cta = blockIdx.x;
-  for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
-    if ((s % nctas) != cta) continue;
+  const int units = src.count(p);
+  for (int u = threadIdx.x; u < units; u += blockDim.x) {
+    if ((u % nctas) != cta) continue;
     if constexpr (kMode == kMulti) {
-      const int raw = __ldg(p.seq_lens + s);
-      if (raw > 0 && raw < p.q_len) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
+      const int raw = __ldg(p.seq_lens + src.table_row(p, u));
+      if (src.pos0(p, u) == 0 && raw > 0 && raw < p.q_len) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
     }
-    const SeqSpan sp = src.template span<B>(p, s);
+    const SeqSpan sp = src.template span<B>(p, u);
     if (sp.nb > sp.first) continue;
-    uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(src.row_group0(p, s)) * p.num_q_heads * D);
-    const int n = src.row_groups(p, s) * p.num_q_heads * D / 8;
+    uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(src.row_group0(p, u)) * p.num_q_heads * D);
+    const int n = src.row_groups(p, u) * p.num_q_heads * D / 8;
     for (int i = 0; i < n; ++i) o[i] = make_uint4(0, 0, 0, 0);
   }
 }
@@ -589,7 +628,7 @@ __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>&
 // head_dim element d, from their states (m, L, unnormalised a): the
 // normalised outputs.  A row that saw no token (a group member of length 0)
 // gets zeros.
-template <bool kBf16, int G, int RC, int kMode>
+template <bool kBf16, int G, int RG, int RC, int kMode>
 __device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, int col0, int rows, int d,
                                           const float (&m)[RC], const float (&L)[RC], const float (&a)[RC]) {
   (void)m;
@@ -602,7 +641,8 @@ __device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, 
       const int rg = c / G;
       size_t row;
       if constexpr (kMode == kMulti) {
-        row = static_cast<size_t>(sg.s) * p.q_len + rg;
+        const int s = sg.s / p.q_tiles;
+        row = static_cast<size_t>(s) * p.q_len + (sg.s - s * p.q_tiles) * RG + rg;
       } else if constexpr (kMode == kGroup) {
         row = static_cast<size_t>(s0 + rg);
       } else {
@@ -660,14 +700,14 @@ __device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, con
         }
       }
     }
-    emit_rows<kBf16, G, RC, kMode>(p, sg, col0, rows, d, M, L, a);
+    emit_rows<kBf16, G, R / G, RC, kMode>(p, sg, col0, rows, d, M, L, a);
     if (ctid == 0) *counter = 0;
   }
 }
 
 // ---- the kernel ---------------------------------------------------------------
 
-template <bool kBf16, int G, int RG, int kMode>
+template <bool kBf16, int G, int RG, int kMode, int B>
 __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     pa_decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_q,
                         const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
@@ -677,6 +717,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   constexpr int WG = Sh::WG, RC = Sh::RC, kThreads = Sh::kThreads, kSoftmaxThreads = Sh::kSoftmaxThreads;
   constexpr int RL = RC < 8 ? 8 : RC;  // TMEM columns loaded per row set (x8 is the narrowest load used)
   static_assert(kMode != kDecode || RG == 1, "a decode unit has one row group");
+  using Bk = Blk<B>;
+  constexpr int CB = Bk::CB;
   using Smem = TcSmem<R>;
   const Source<kMode, RG> src;
   extern __shared__ unsigned char smem_raw[];
@@ -736,9 +778,9 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   grid_dependency_wait();
   grid_launch_dependents();
   if constexpr (kMode == kGroup) {
-    group_bookkeeping(p, src);
+    group_bookkeeping<RG, B>(p, src);
   } else {
-    zero_empty_units(p, src);
+    zero_empty_units<kMode, RG, B>(p, src);
   }
   WorkRange wr;
   Cursor cur;
@@ -797,16 +839,17 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           bool go = true;
           if (lane == 0) {
             go = mbar_wait_bounded(empty, ((ci / ns) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
-            if (go) mbar_arrive_expect_tx(full, nblk * 2 * kBlockBytes);
+            if (go) mbar_arrive_expect_tx(full, nblk * Bk::kVBlockBytes);
           }
           if (!__shfl_sync(0xffffffffu, go, 0)) return false;
           if (lane < nblk) {
-            if (is_k) {
-              uint8_t* base = sm.kbuf[st] + lane * kBlockBytes;
+            if (is_k && !Bk::kK3D) {
+              uint8_t* base = sm.kbuf[st] + lane * Bk::kBlockBytes;
               tma_load_2d(base, map, 0, y, full, pol_stream);
               tma_load_2d(base + kHalfBytes, map, 64, y, full, pol_stream);
             } else {
-              tma_load_3d(sm.vbuf[st] + lane * kVBlockBytes, map, 0, y, 0, full, pol_stream);
+              uint8_t* buf = is_k ? sm.kbuf[st] : sm.vbuf[st];
+              tma_load_3d(buf + lane * Bk::kVBlockBytes, map, 0, y, 0, full, pol_stream);
             }
           }
           __syncwarp();
@@ -828,7 +871,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         if constexpr (kMode != kGroup) {
           // One table row: entries 32 at a time (lane l holds entry b0 + l),
           // the next batch in flight while the current one is issued.
-          const int32_t* trow = p.block_tables + static_cast<size_t>(sg.s) * p.max_nb + sg.j0;
+          const int32_t* trow = p.block_tables + static_cast<size_t>(src.table_row(p, sg.s)) * p.max_nb + sg.j0;
           int e_cur = (lane < sg.n) ? __ldg(trow + lane) : 0;
           for (int b0 = 0; ok && b0 < sg.n; b0 += 32) {
             const int e_next = (b0 + 32 + lane < sg.n) ? __ldg(trow + b0 + 32 + lane) : 0;
@@ -842,7 +885,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           }
         } else {
           // Chunks from several rows: each chunk's entries, one chunk ahead.
-          ChunkWalk<kMode, G, RG> walk;
+          ChunkWalk<kMode, G, RG, B> walk;
           walk.start(p, sg, 0);
           ChunkSrc cs = walk.next(p);
           int e_cur = (lane < cs.nblk) ? __ldg(p.block_tables + static_cast<size_t>(cs.seq) * p.max_nb + cs.j + lane) : 0;
@@ -896,7 +939,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           const uint32_t k0 = smem_u32(sm.kbuf[ks]);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint64_t a = sw128_desc(k0 + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 8 * kRowBytes);
+            const uint64_t a = sw128_desc(k0 + (k >> 2) * Bk::kKHalfBytes + (k & 3) * 32, 16, Bk::kKGroupBytes);
             const uint64_t b = sw128_desc(q0 + (k >> 2) * Nq * kRowBytes + (k & 3) * 32, 16, 8 * kRowBytes);
             umma(tmem + kColS + (qk & 1) * Nq, a, b, kIdescQK, k > 0 ? 1u : 0u);
           }
@@ -931,7 +974,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       int pv = 0;
       Seg sg;
       while (ok && next_seg<B, CB>(cur, sg, p, src)) {
-        ChunkWalk<kMode, G, RG> walk;
+        ChunkWalk<kMode, G, RG, B> walk;
         walk.start(p, sg, 0);
         for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
           const int ntok = walk.next(p).ntok;
@@ -947,7 +990,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           const uint32_t p0 = smem_u32(sm.p[pb]);
           const int nks = (ntok + 15) / 16;
           for (int k = 0; k < nks; ++k) {
-            const uint64_t a = sw128_desc(v0 + k * kVBlockBytes, kBlockBytes, 8 * kRowBytes);
+            const uint64_t a = sw128_desc(v0 + Bk::v_offset(16 * k), Bk::kBlockBytes, Bk::kVGroupBytes);
             // tokens [16k, 16k + 16): two groups of 8 token rows; Np fits one swizzle atom
             const uint64_t b = smem_desc(p0 + k * 16 * Sh::kPRowBytes, 0, 8 * Sh::kPRowBytes, Sh::kPLayout);
             umma(tmem + kColO + pb * Np, a, b, kIdescPV, k > 0 ? 1u : 0u);
@@ -1019,7 +1062,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       for (int k = 0; k < RC; ++k) {
         const int c = col0 + k;
         bool valid = mine && c >= ch.row_lo && c < ch.row_hi && r < ch.ntok;
-        if constexpr (kMode == kMulti) valid = valid && t <= ch.len - p.q_len + c / G;  // causal
+        if constexpr (kMode == kMulti) valid = valid && t <= ch.len - p.q_len + ch.pos0 + c / G;  // causal
         sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
         over |= sc[k] > m_ref[k] + kRescaleGap;
       }
@@ -1107,8 +1150,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       // so that 0 * (whatever they hold) cannot reach the output
       if (col0 == 0 && (ch.ntok & 15) != 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
         (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
-        uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + (r / B) * kVBlockBytes + (r % B) * kRowBytes);
-        uint4* v1 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(v0) + kBlockBytes);
+        uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + Bk::v_offset(r));
+        uint4* v1 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(v0) + Bk::kBlockBytes);
 #pragma unroll
         for (int i = 0; i < kRowBytes / 16; ++i) {
           v0[i] = make_uint4(0, 0, 0, 0);
@@ -1180,7 +1223,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           const int c = col0 + k;
           L[k] = (sm.lred[0][c] + sm.lred[1][c]) + (sm.lred[2][c] + sm.lred[3][c]);
         }
-        emit_rows<kBf16, G, RC, kMode>(p, fs, col0, rows, r, m, L, acc);
+        emit_rows<kBf16, G, RG, RC, kMode>(p, fs, col0, rows, r, m, L, acc);
       } else {
         float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * Sh::kPartStride;
         if (ctid < R) {
@@ -1211,7 +1254,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     bool pending = false;   // the epilogue of chunk ci - 1 is still due
     while (ok && next_seg<B, CB>(cur, sg, p, src)) {
       const int rows = G * src.row_groups(p, sg.s);
-      ChunkWalk<kMode, G, RG> walk;
+      ChunkWalk<kMode, G, RG, B> walk;
       walk.start(p, sg, rows);
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
         if (c0 == 0 && have_prev) stash_segment();
@@ -1304,14 +1347,15 @@ inline bool make_map(CUtensorMap* map, const void* base, int rank, const unsigne
   return r == CUDA_SUCCESS;
 }
 
-// V pool as a 3-D tensor (64 columns, rows, 2 halves 128 bytes apart): one
-// box of 64 x 16 x 2 lands a block's rows as [half][16][64] in shared memory.
-inline bool make_map_v(CUtensorMap* map, const void* base, unsigned long long rows, bool bf16) {
+// A pool as a 3-D tensor (64 columns, rows, 2 halves 128 bytes apart): one
+// box of 64 x block x 2 lands a block's rows as [half][block][64] in shared
+// memory.
+inline bool make_map_halves(CUtensorMap* map, const void* base, unsigned long long rows, int block, bool bf16) {
   auto encode = encode_fn();
   if (encode == nullptr) return false;
   cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), 2};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, 128};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(B), 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(block), 2};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1320,33 +1364,89 @@ inline bool make_map_v(CUtensorMap* map, const void* base, unsigned long long ro
   return r == CUDA_SUCCESS;
 }
 
-template <bool kBf16, int G, int RG, int kMode>
+// The three tensor maps of a launch, kept for the launches that follow: a
+// map depends only on the kernel instance (box shapes, element type), the
+// operand addresses and the extents, which make the key, so a cached map is
+// the one a fresh encode would give.  A loop that decodes into the same
+// buffers encodes its maps once.
+struct LaunchMaps {
+  const void* kernel;
+  const void *q, *k, *v;
+  unsigned long long q_rows, kv_rows;
+  int num_q_heads;
+  CUtensorMap mq, mk, mv;
+};
+
+inline bool cached_maps(const LaunchMaps& want, CUtensorMap& mq, CUtensorMap& mk, CUtensorMap& mv,
+                        bool (*encode)(const LaunchMaps&, CUtensorMap&, CUtensorMap&, CUtensorMap&)) {
+  constexpr int kEntries = 16;
+  static std::mutex mu;
+  static LaunchMaps cache[kEntries];
+  static int n_used = 0, next = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_used; ++i) {
+      const LaunchMaps& e = cache[i];
+      if (e.kernel == want.kernel && e.q == want.q && e.k == want.k && e.v == want.v && e.q_rows == want.q_rows &&
+          e.kv_rows == want.kv_rows && e.num_q_heads == want.num_q_heads) {
+        mq = e.mq;
+        mk = e.mk;
+        mv = e.mv;
+        return true;
+      }
+    }
+  }
+  if (!encode(want, mq, mk, mv)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  LaunchMaps& slot = cache[next];
+  slot = want;
+  slot.mq = mq;
+  slot.mk = mk;
+  slot.mv = mv;
+  next = (next + 1) % kEntries;
+  if (n_used < kEntries) ++n_used;
+  return true;
+}
+
+template <bool kBf16, int G, int RG, int B>
+bool encode_launch_maps(const LaunchMaps& w, CUtensorMap& mq, CUtensorMap& mk, CUtensorMap& mv) {
+  const unsigned long long q_outer[2] = {static_cast<unsigned long long>(w.num_q_heads), w.q_rows};
+  const uint32_t q_box[2] = {static_cast<uint32_t>(G), static_cast<uint32_t>(RG)};
+  const unsigned long long kv_outer[1] = {w.kv_rows};
+  const uint32_t kv_box[1] = {static_cast<uint32_t>(B)};
+  const bool k_ok = Blk<B>::kK3D ? make_map_halves(&mk, w.k, w.kv_rows, B, kBf16)
+                                 : make_map(&mk, w.k, 2, kv_outer, kv_box, kBf16);
+  return k_ok && make_map(&mq, w.q, 3, q_outer, q_box, kBf16) && make_map_halves(&mv, w.v, w.kv_rows, B, kBf16);
+}
+
+template <bool kBf16, int G, int RG, int kMode, int B>
 cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   const unsigned long long q_rows =
       static_cast<unsigned long long>(prm.num_seqs) * (kMode == kMulti ? prm.q_len : 1);
   const unsigned long long kv_rows = static_cast<unsigned long long>(prm.num_blocks) * prm.num_kv_heads * B;
   if (kv_rows >= (1ull << 31) || q_rows >= (1ull << 31)) return cudaErrorInvalidValue;
-  const unsigned long long q_outer[2] = {static_cast<unsigned long long>(prm.num_q_heads), q_rows};
-  const uint32_t q_box[2] = {static_cast<uint32_t>(G), static_cast<uint32_t>(RG)};
-  const unsigned long long kv_outer[1] = {kv_rows};
-  const uint32_t kv_box[1] = {static_cast<uint32_t>(B)};
-  if (!make_map(&mq, prm.q, 3, q_outer, q_box, kBf16) || !make_map(&mk, prm.k_pool, 2, kv_outer, kv_box, kBf16) ||
-      !make_map_v(&mv, prm.v_pool, kv_rows, kBf16)) {
-    return cudaErrorInvalidValue;
-  }
+  LaunchMaps want{};
+  want.kernel = reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode, B>);
+  want.q = prm.q;
+  want.k = prm.k_pool;
+  want.v = prm.v_pool;
+  want.q_rows = q_rows;
+  want.kv_rows = kv_rows;
+  want.num_q_heads = prm.num_q_heads;
+  if (!cached_maps(want, mq, mk, mv, &encode_launch_maps<kBf16, G, RG, B>)) return cudaErrorInvalidValue;
   if constexpr (Rows<G * RG>::WG == 2) {
     // setmaxnreg only moves registers inside the launch's allocation; should
     // a build give the kernel fewer than the split needs, the softmax warps'
     // increase would wait forever, so such a kernel is not launched.
     static const bool regs_fit = [] {
       cudaFuncAttributes a{};
-      return cudaFuncGetAttributes(&a, pa_decode_tc_kernel<kBf16, G, RG, kMode>) == cudaSuccess &&
+      return cudaFuncGetAttributes(&a, pa_decode_tc_kernel<kBf16, G, RG, kMode, B>) == cudaSuccess &&
              a.numRegs * Rows<G * RG>::kThreads >= 128 * kCtrlRegs + 256 * kSoftmaxRegs;
     }();
     if (!regs_fit) return cudaErrorInvalidConfiguration;
   }
-  return launch_overlapped(pa_decode_tc_kernel<kBf16, G, RG, kMode>, dim3(ctas), dim3(Rows<G * RG>::kThreads),
+  return launch_overlapped(pa_decode_tc_kernel<kBf16, G, RG, kMode, B>, dim3(ctas), dim3(Rows<G * RG>::kThreads),
                            static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
 }
 
@@ -1359,27 +1459,35 @@ constexpr int unit_finish_cost(int kMode, int R) {
   return kMode == kDecode ? (R <= 4 ? 2 : 4) : kMode == kGroup ? 10 : (R <= 8 ? 4 : R <= 16 ? 6 : 10);
 }
 
-template <bool kBf16, int G, int RG, int kMode>
+template <bool kBf16, int G, int RG, int kMode, int B = 16>
 Variant tc_variant() {
   constexpr int R = G * RG;
   static_assert(smem_bytes<R>() <= kMaxSmemPerCta, "shared memory of one CTA");
-  return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode>), Rows<R>::kThreads,
-                 smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode>,
+  return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode, B>), Rows<R>::kThreads,
+                 smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode, B>,
                  unit_finish_cost(kMode, R)};
 }
 
-inline bool tc_pool_ok(const pa_pool_desc& pool) {
-  return pool.head_dim == D && pool.block_size == B && (pool.dtype == PA_BF16 || pool.dtype == PA_FP16);
+// head_dim 128, a 16-bit pool, and a block size the instances cover: 8, 16
+// or 32 tokens for the decode (any_block), 16 for the other modes.
+inline bool tc_pool_ok(const pa_pool_desc& pool, bool any_block = false) {
+  const bool block_ok = pool.block_size == 16 || (any_block && (pool.block_size == 8 || pool.block_size == 32));
+  return pool.head_dim == D && block_ok && (pool.dtype == PA_BF16 || pool.dtype == PA_FP16);
 }
 
-// Row-group count a request for rg row groups runs with: the smallest power
-// of two >= rg, or 0 when G * that exceeds 32 rows.
-inline int row_groups_for(int G, int rg) {
-  if (G <= 0 || rg <= 0) return 0;
+// Row groups per unit for q_len positions of G heads: the smallest power of
+// two >= q_len while G times that fits 32 rows (one unit per sequence),
+// else 32 / G (several units, row tiles, per sequence); 0 for G outside
+// 1..32.
+inline int row_groups_for(int G, int q_len) {
+  if (G <= 0 || G > 32 || q_len <= 0) return 0;
   int r = 1;
-  while (r < rg) r *= 2;
-  return G * r <= 32 ? r : 0;
+  while (r < q_len && G * r < 32) r *= 2;
+  return r;
 }
+
+// Row tiles (units) per sequence for q_len positions at rg row groups a unit.
+inline int row_tiles_for(int q_len, int rg) { return rg > 0 ? (q_len + rg - 1) / rg : 0; }
 
 }  // namespace tc
 }  // namespace pa

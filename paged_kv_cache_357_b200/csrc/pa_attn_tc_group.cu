@@ -28,8 +28,10 @@ static bool pick_group(int G, int RG, Variant& v) {
 
 bool select_tc_group_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v) {
   if (!tc::tc_pool_ok(pool)) return false;
+  // every member of a group sits in one unit: G x (members rounded up to a
+  // power of two) must fit the 32 rows of a unit
   const int rg = tc::row_groups_for(group, max_members);
-  if (rg == 0) return false;
+  if (rg == 0 || rg < max_members) return false;
   return pool.dtype == PA_BF16 ? tc::pick_group<true>(group, rg, v) : tc::pick_group<false>(group, rg, v);
 }
 

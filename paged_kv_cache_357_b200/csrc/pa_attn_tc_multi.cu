@@ -2,7 +2,9 @@
 // kernel in pa_attn_tc.cuh.  Each sequence brings q_len new query positions
 // (q and out are [num_seqs][q_len][num_q_heads][head_dim]); position i sees
 // the sequence's tokens up to seq_len - q_len + i.  A unit holds the G query
-// heads of a kv head times RG >= q_len positions, G * RG <= 32 rows.
+// heads of a kv head times RG positions, G * RG <= 32 rows: RG >= q_len
+// when they fit, else several units (row tiles of RG = 32 / G positions)
+// per sequence.
 #include "pa_attn_tc.cuh"
 
 namespace pa {
@@ -25,10 +27,11 @@ static bool pick_multi(int G, int RG, Variant& v) {
 
 }  // namespace tc
 
-bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v) {
+bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v, int& tiles) {
   if (!tc::tc_pool_ok(pool) || q_len < 2) return false;
   const int rg = tc::row_groups_for(group, q_len);
   if (rg == 0) return false;
+  tiles = tc::row_tiles_for(q_len, rg);
   return pool.dtype == PA_BF16 ? tc::pick_multi<true>(group, rg, v) : tc::pick_multi<false>(group, rg, v);
 }
 

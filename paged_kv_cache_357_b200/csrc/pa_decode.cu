@@ -594,6 +594,7 @@ static DecodeParams make_params(const void* q, const void* k_pool, const void* v
   prm.wait_limit_ns = test_timeout ? 20ull * 1000 * 1000 : 2ull * 1000 * 1000 * 1000;
   prm.test_flags = test_timeout ? kFlagTestWithholdCopies : 0;
   prm.q_len = 1;
+  prm.q_tiles = 1;
   prm.group_starts = nullptr;
   prm.group_prefix = nullptr;
   prm.num_groups = 0;
@@ -622,9 +623,13 @@ static bool opts_ok(const pa_decode_opts* opts) {
 
 // ---- multi-query decode ------------------------------------------------------
 
-static bool multi_variant(const pa_pool_desc& pool, int num_q_heads, int q_len, Variant& v) {
+// The variant and its row tiles (units) per sequence; false also when the
+// units of the batch overflow the unit index.
+static bool multi_variant(const pa_pool_desc& pool, int num_seqs, int num_q_heads, int q_len, Variant& v,
+                          int& tiles) {
   int G = 0;
-  return group_of(pool, num_q_heads, G) && select_tc_multi_variant(pool, G, q_len, v);
+  if (!group_of(pool, num_q_heads, G) || !select_tc_multi_variant(pool, G, q_len, v, tiles)) return false;
+  return tiles >= 1 && static_cast<long long>(num_seqs) * tiles <= 0x7fffffffLL;
 }
 
 // ---- shared-prefix decode ----------------------------------------------------
@@ -695,9 +700,9 @@ extern "C" size_t pa_decode_multi_workspace_bytes(int32_t num_seqs, int32_t q_le
   if (q_len == 1) return pa_decode_workspace_bytes_ex(num_seqs, num_q_heads, pool, opts);
   if (num_seqs < 0 || q_len < 1 || !pool_shape_ok(pool)) return 0;
   Variant v;
-  int ctas = 0;
-  if (!multi_variant(*pool, num_q_heads, q_len, v) || !query_ctas(v, opts, ctas)) return 0;
-  return workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
+  int ctas = 0, tiles = 0;
+  if (!multi_variant(*pool, num_seqs, num_q_heads, q_len, v, tiles) || !query_ctas(v, opts, ctas)) return 0;
+  return workspace_bytes_for(num_seqs * tiles, pool->num_kv_heads, ctas, v.part_stride);
 }
 
 extern "C" pa_status pa_decode_multi(const void* q, const void* k_pool, const void* v_pool,
@@ -718,15 +723,17 @@ extern "C" pa_status pa_decode_multi(const void* q, const void* k_pool, const vo
   if (static_cast<long long>(num_seqs) * q_len > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
   if ((opts_flags(opts) & PA_DECODE_CUDA_CORES_ONLY) != 0) return PA_ERR_UNSUPPORTED;
   Variant v;
-  if (!multi_variant(*pool, num_q_heads, q_len, v)) return PA_ERR_UNSUPPORTED;
+  int tiles = 0;
+  if (!multi_variant(*pool, num_seqs, num_q_heads, q_len, v, tiles)) return PA_ERR_UNSUPPORTED;
   const int ctas = resolve_ctas(v, opts);
   if (ctas <= 0) return PA_ERR_CUDA;
-  const size_t need = workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
+  const size_t need = workspace_bytes_for(num_seqs * tiles, pool->num_kv_heads, ctas, v.part_stride);
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
   DecodeParams prm = make_params(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                                  num_q_heads, scale, out, workspace, ctas, v.part_stride, dev_status, pool,
                                  opts_flags(opts));
   prm.q_len = q_len;
+  prm.q_tiles = tiles;
   prm.unit_cost = v.unit_cost;
   return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -52,6 +52,9 @@ struct DecodeParams {
   // multi-query decode: query positions per sequence (q, out are
   // [num_seqs][q_len][num_q_heads][head_dim]); 1 otherwise
   int q_len;
+  // multi-query decode: row tiles per sequence (a unit carries the positions
+  // of one tile); 1 otherwise
+  int q_tiles;
   // shared-prefix decode (null / 0 otherwise)
   const int32_t* group_starts;   // [num_groups + 1], consecutive sequences per group
   const int32_t* group_prefix;   // [num_groups] shared leading blocks of each group

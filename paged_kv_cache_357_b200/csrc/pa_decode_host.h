@@ -23,10 +23,15 @@ struct Variant {
 
 // Tensor-core variants (pa_attn_tc.cuh), if one exists for this pool and
 // shape.  `group` is the number of query heads per kv head.
-// Plain decode (pa_decode_tc.cu): groups of 1, 2, 4 and 8.
+// Plain decode (pa_decode_tc.cu): groups of 1, 2, 4 and 8, blocks of 8, 16
+// or 32 tokens.
 bool select_tc_variant(const pa_pool_desc& pool, int group, Variant& v);
-// Multi-query decode with q_len >= 2 positions (pa_attn_tc_multi.cu).
-bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v);
+// The plain decode's instances at blocks of 8 and 32 tokens
+// (pa_decode_tc_blocks.cu).
+bool select_tc_decode_other_block(int block_size, bool bf16, int group, Variant& v);
+// Multi-query decode with q_len >= 2 positions (pa_attn_tc_multi.cu); tiles
+// = units (row tiles) per sequence.
+bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v, int& tiles);
 // Shared-prefix decode over groups of up to max_members sequences
 // (pa_attn_tc_group.cu).
 bool select_tc_group_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);

@@ -16,12 +16,20 @@ plain-language section), and the decode reads every block through the table
 (vLLM blog §"关键细节" 2).
 
 Consecutive steps overlap their copies with each other's kernels: the
-per-step device buffers come in several sets (three by default) used in
-turn, uploads run on one stream, kernels on a second and downloads on a
-third.  Events order the work: a step's kernels wait for its uploads and for
-the previous step's kernels (they share the pools); its download waits for
-its kernels; the upload into a buffer set waits until the kernels that last
-read that set are done, so an upload has the time of (sets - 1) steps.
+per-step buffers come in several sets (three by default) used in turn,
+uploads run on one stream, kernels on a second and downloads on a third.
+Events order the work: a step's kernels wait for its uploads and for the
+previous step's kernels (they share the pools); its download waits for its
+kernels; the upload into a buffer set waits until the kernels that last read
+that set are done, so an upload has the time of (sets - 1) steps.
+
+Per step the host issues little.  Each buffer set is one device allocation
+with a pinned host staging area of the same layout: a caller that builds a
+step's inputs in the staging views (``staging()``) has them go up in one
+copy; other pinned host tensors are copied field by field, straight from
+where they are.  After the first step, a set's kernels (copy, write,
+decode) are replayed as one CUDA graph captured for that set and those
+counts.
 """
 
 from __future__ import annotations
@@ -31,24 +39,57 @@ from typing import Optional
 
 from . import _lib
 
+_ALIGN = 256  # byte alignment of every field inside a buffer set
+
 
 class _BufferSet:
+    """One step's inputs and output: the inputs carved from one device
+    allocation, mirrored by a pinned host staging area of the same layout."""
+
     def __init__(self, torch, dev, dt, S, Hq, D, Hkv, max_nb, T, P, q_len, grouped):
-        self.q = torch.empty((S, Hq, D) if q_len == 1 else (S, q_len, Hq, D), dtype=dt, device=dev)
-        self.out = torch.empty_like(self.q)
-        self.tables = torch.empty((S, max_nb), dtype=torch.int32, device=dev)
-        self.lens = torch.empty((S,), dtype=torch.int32, device=dev)
-        self.new_k = torch.empty((max(T, 1), Hkv, D), dtype=dt, device=dev)
-        self.new_v = torch.empty_like(self.new_k)
-        self.slots = torch.empty((max(T, 1),), dtype=torch.int64, device=dev)
-        self.pairs = torch.empty((max(P, 1), 2), dtype=torch.int64, device=dev)
-        self.group_starts = torch.empty((S + 1,), dtype=torch.int32, device=dev) if grouped else None
-        self.group_prefix = torch.empty((max(S, 1),), dtype=torch.int32, device=dev) if grouped else None
-        self.out_host = torch.empty(self.out.shape, dtype=dt, pin_memory=True)
+        q_shape = (S, Hq, D) if q_len == 1 else (S, q_len, Hq, D)
+        fields = [("q", dt, q_shape), ("tables", torch.int32, (S, max_nb)), ("lens", torch.int32, (S,))]
+        if grouped:
+            fields += [("group_starts", torch.int32, (S + 1,)), ("group_prefix", torch.int32, (max(S, 1),))]
+        fields += [("pairs", torch.int64, (max(P, 1), 2)), ("new_k", dt, (max(T, 1), Hkv, D)),
+                   ("new_v", dt, (max(T, 1), Hkv, D)), ("slots", torch.int64, (max(T, 1),))]
+        self.offsets, off = {}, 0
+        for name, fdt, shape in fields:
+            n = 1
+            for d in shape:
+                n *= d
+            nbytes = n * torch.empty((), dtype=fdt).element_size()
+            self.offsets[name] = (off, off + nbytes, fdt, shape)
+            off = (off + nbytes + _ALIGN - 1) // _ALIGN * _ALIGN
+        self.dev_bytes = torch.empty(off, dtype=torch.uint8, device=dev)
+        self.host_bytes = torch.empty(off, dtype=torch.uint8, pin_memory=True)
+        self.dev = {name: self._view(self.dev_bytes, name) for name in self.offsets}
+        self.host = {name: self._view(self.host_bytes, name) for name in self.offsets}
+        self.q, self.tables, self.lens = self.dev["q"], self.dev["tables"], self.dev["lens"]
+        self.group_starts, self.group_prefix = self.dev.get("group_starts"), self.dev.get("group_prefix")
+        self.pairs, self.new_k, self.new_v, self.slots = (self.dev[n] for n in ("pairs", "new_k", "new_v", "slots"))
+        self.out = torch.empty(q_shape, dtype=dt, device=dev)
+        self.out_host = torch.empty(q_shape, dtype=dt, pin_memory=True)
         self.uploaded = torch.cuda.Event()
         self.computed = torch.cuda.Event()
         self.downloaded = torch.cuda.Event()
+        self.graphs = {}  # (copy pairs, new tokens, groups) -> captured kernels of this set
         self.used = False
+
+    def _view(self, buf, name):
+        a, b, fdt, shape = self.offsets[name]
+        return buf[a:b].view(fdt).view(shape)
+
+    def upload_end(self, n_pairs: int, T: int, n_groups: int) -> int:
+        """Bytes from the start of the layout through the last field this
+        step uses (the whole prefix goes up in one copy)."""
+        if T > 0:
+            return self.offsets["slots"][1]
+        if n_pairs > 0:
+            return self.offsets["pairs"][1]
+        if n_groups > 0:
+            return self.offsets["group_prefix"][1]
+        return self.offsets["lens"][1]
 
 
 class PagedDecodeStep:
@@ -106,41 +147,64 @@ class PagedDecodeStep:
         self.last_h2d_bytes = 0
         self.last_d2h_bytes = 0
 
+    def staging(self):
+        """Pinned host views the next ``run()`` uploads from: q, block_tables,
+        seq_lens, new_k, new_v, slot_mapping, copy_pairs (and group_starts,
+        group_prefix_blocks for a shared-prefix step), each at its maximum
+        size.  A caller that builds its inputs there, and passes them (or
+        their leading rows) to ``run()``, saves the host-side copy.  Waits
+        until the upload that last read this area is done."""
+        bs = self.sets[self.steps % len(self.sets)]
+        if bs.used:
+            bs.uploaded.synchronize()
+        h = bs.host
+        views = dict(q=h["q"], block_tables=h["tables"], seq_lens=h["lens"], new_k=h["new_k"], new_v=h["new_v"],
+                     slot_mapping=h["slots"], copy_pairs=h["pairs"])
+        if self.max_group_size > 0:
+            views.update(group_starts=h["group_starts"], group_prefix_blocks=h["group_prefix"])
+        return views
+
     def run(self, q, block_tables, seq_lens, new_k=None, new_v=None, slot_mapping=None, copy_pairs=None,
             group_starts=None, group_prefix_blocks=None):
-        """Enqueue one step from host tensors (pinned, so the copies run
-        asynchronously; leave them unchanged until the step completes).
+        """Enqueue one step from host tensors (pinned, or the ``staging()``
+        views; leave them unchanged until the step's upload is done).
         Returns the pinned host output of this step, valid once
         ``wait(result)`` or ``synchronize()`` returns and until its buffer set
-        comes round again (``len(self.sets)`` steps later).  A shared-prefix step also takes the groups (int32
-        host tensors [num_groups + 1] and [num_groups])."""
+        comes round again (``len(self.sets)`` steps later).  A shared-prefix
+        step also takes the groups (int32 host tensors [num_groups + 1] and
+        [num_groups])."""
         torch = self.torch
         bs = self.sets[self.steps % len(self.sets)]
-        h2d = 0
+        n_groups = 0
+        if self.max_group_size > 0:
+            if group_starts is None or group_prefix_blocks is None:
+                raise ValueError("a shared-prefix step needs group_starts and group_prefix_blocks")
+            n_groups = group_prefix_blocks.shape[0]
+        n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
+        T = 0 if slot_mapping is None else slot_mapping.shape[0]
+        # (field, leading rows or None for all, host tensor) of this step's inputs
+        inputs = [("q", None, q), ("tables", None, block_tables), ("lens", None, seq_lens)]
+        if n_groups > 0:
+            inputs += [("group_starts", n_groups + 1, group_starts), ("group_prefix", n_groups, group_prefix_blocks)]
+        if n_pairs > 0:
+            inputs.append(("pairs", n_pairs, copy_pairs))
+        if T > 0:
+            inputs += [("new_k", T, new_k), ("new_v", T, new_v), ("slots", T, slot_mapping)]
+        packed = all(src.data_ptr() == bs.host[name].data_ptr() for name, _, src in inputs)
         with torch.cuda.stream(self.h2d_stream):
             if bs.used:
                 self.h2d_stream.wait_event(bs.computed)  # the kernels that last read this set
-            for dst, src in ((bs.q, q), (bs.tables, block_tables), (bs.lens, seq_lens)):
-                dst.copy_(src, non_blocking=True)
-                h2d += src.numel() * src.element_size()
-            n_groups = 0
-            if self.max_group_size > 0:
-                if group_starts is None or group_prefix_blocks is None:
-                    raise ValueError("a shared-prefix step needs group_starts and group_prefix_blocks")
-                n_groups = group_prefix_blocks.shape[0]
-                bs.group_starts[: n_groups + 1].copy_(group_starts, non_blocking=True)
-                bs.group_prefix[:n_groups].copy_(group_prefix_blocks, non_blocking=True)
-                h2d += (2 * n_groups + 1) * 4
-            n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
-            if n_pairs > 0:
-                bs.pairs[:n_pairs].copy_(copy_pairs, non_blocking=True)
-                h2d += copy_pairs.numel() * copy_pairs.element_size()
-            T = 0 if slot_mapping is None else slot_mapping.shape[0]
-            if T > 0:
-                bs.new_k[:T].copy_(new_k, non_blocking=True)
-                bs.new_v[:T].copy_(new_v, non_blocking=True)
-                bs.slots[:T].copy_(slot_mapping, non_blocking=True)
-                h2d += sum(t.numel() * t.element_size() for t in (new_k, new_v, slot_mapping))
+            if packed:
+                # every input sits in this set's staging area: one copy of the used prefix
+                end = bs.upload_end(n_pairs, T, n_groups)
+                bs.dev_bytes[:end].copy_(bs.host_bytes[:end], non_blocking=True)
+                h2d = end
+            else:
+                h2d = 0
+                for name, rows, src in inputs:
+                    dst = bs.dev[name] if rows is None else bs.dev[name][:rows]
+                    dst.copy_(src, non_blocking=True)
+                    h2d += src.numel() * src.element_size()
             bs.uploaded.record(self.h2d_stream)
         with torch.cuda.stream(self.compute_stream):
             # the compute stream is in order, so the previous step's kernels
@@ -152,7 +216,7 @@ class PagedDecodeStep:
                 self._launch_checked(bs, n_pairs, T, n_groups)
                 self._checked = True
             else:
-                self._launch_bound(bs, n_pairs, T, n_groups)
+                self._launch_graph(bs, n_pairs, T, n_groups)
             bs.computed.record(self.compute_stream)
         with torch.cuda.stream(self.d2h_stream):
             self.d2h_stream.wait_event(bs.computed)
@@ -163,6 +227,18 @@ class PagedDecodeStep:
         self.last_h2d_bytes = h2d
         self.last_d2h_bytes = bs.out.numel() * bs.out.element_size()
         return bs.out_host
+
+    def _launch_graph(self, bs, n_pairs: int, T: int, n_groups: int) -> None:
+        """Replay this set's kernels for these counts, capturing them the
+        first time (capture records the launches without running them)."""
+        key = (n_pairs, T, n_groups)
+        g = bs.graphs.get(key)
+        if g is None:
+            g = self.torch.cuda.CUDAGraph()
+            with self.torch.cuda.graph(g, stream=self.compute_stream, capture_error_mode="thread_local"):
+                self._launch_bound(bs, n_pairs, T, n_groups)
+            bs.graphs[key] = g
+        g.replay()
 
     def _launch_checked(self, bs, n_pairs: int, T: int, n_groups: int) -> None:
         """The step's kernels through the checking Python wrappers."""
@@ -187,7 +263,8 @@ class PagedDecodeStep:
 
     def _launch_bound(self, bs, n_pairs: int, T: int, n_groups: int) -> None:
         """The same kernels through the C entry points with the buffers'
-        addresses (the buffers, pools, workspace and stream never change)."""
+        addresses (the buffers, pools, workspace and stream never change);
+        captured into a graph by ``_launch_graph``."""
         c, desc, cs, st = self._c, self._desc_ref, self._cs, self.status.data_ptr()
         kp, vp = self.k_pool.data_ptr(), self.v_pool.data_ptr()
         if n_pairs > 0:

@@ -14,8 +14,8 @@ from workloads import bits_to_torch, config_llama3_8b, f32_to_bits, fill_values_
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(seed, lens, G, L, dtype, Hkv=2):
-    layout = random_layout(seed, lens, dtype=dtype, block_size=16, num_q_heads=Hkv * G, num_kv_heads=Hkv,
+def _inputs(seed, lens, G, L, dtype, Hkv=2, block_size=16):
+    layout = random_layout(seed, lens, dtype=dtype, block_size=block_size, num_q_heads=Hkv * G, num_kv_heads=Hkv,
                            head_dim=128, write_new_token=False)
     vals = fill_values_numpy(layout)
     rng = np.random.default_rng([seed, 99])
@@ -59,6 +59,32 @@ def test_multi_shapes(cuda_device, G, L):
     out, st = _run(cuda_device, layout, vals, q)
     assert st == 0
     assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"G={G} q_len={L} {dtype}")
+
+
+TILED = [(1, 64), (2, 33), (4, 16), (4, 64), (4, 256), (8, 8), (8, 16), (8, 64), (8, 256)]
+
+
+@pytest.mark.parametrize("G,L", TILED, ids=[f"G{g}-L{l}" for g, l in TILED])
+def test_multi_row_tiles(cuda_device, G, L):
+    """G x q_len beyond the 32 rows of one unit (prefill chunks): each
+    sequence's positions are cut into row tiles of 32 / G positions, each a
+    unit reading only the blocks its last position sees; the last tile may
+    be partial."""
+    dtype = "bf16" if L % 2 == 0 else "fp16"
+    lens = [L, L + 1, 2 * L + 3, L + 130, 1000, 2049]
+    layout, vals, q = _inputs(7500 + 40 * G + L, lens, G, L, dtype)
+    out, st = _run(cuda_device, layout, vals, q)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"G={G} q_len={L} {dtype}")
+
+
+@pytest.mark.parametrize("num_ctas", [1, 5, 0])
+def test_multi_row_tiles_split_units(cuda_device, num_ctas):
+    G, L = 4, 64
+    layout, vals, q = _inputs(7600 + num_ctas, [64, 300, 2500, 97], G, L, "bf16")
+    out, st = _run(cuda_device, layout, vals, q, num_ctas)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"tiles num_ctas={num_ctas}")
 
 
 @pytest.mark.parametrize("num_ctas", [1, 3, 37, 0])
@@ -107,7 +133,8 @@ def test_unsupported_shapes_are_refused(cuda_device):
 
     import paged_kv_cache_357_b200 as pa
 
-    layout, vals, q = _inputs(7400, [64, 80], 8, 8, "bf16")  # 8 heads x 8 positions = 64 rows
+    # multi-query runs at block size 16 only
+    layout, vals, q = _inputs(7400, [64, 80], 8, 8, "bf16", block_size=8)
     kp = bits_to_torch(vals.k_pool, "bf16").to(cuda_device)
     with pytest.raises(pa.PaError) as e:
         pa.multi_workspace_bytes(2, 8, layout.num_q_heads, kp)

@@ -58,13 +58,14 @@ def test_shape_sweep(pa_mod, cuda_device, dtype, B, D, G):
     _run_and_check(L, fill_values_numpy(L), cuda_device, what=f"{dtype} B={B} D={D} G={G}")
 
 
+@pytest.mark.parametrize("B", [8, 16, 32])
 @pytest.mark.parametrize("num_ctas", [1, 3, 7, 64, 1000])
-def test_split_counts_agree(pa_mod, cuda_device, num_ctas):
+def test_split_counts_agree(pa_mod, cuda_device, num_ctas, B):
     """One CTA (no split at all) through far more CTAs than blocks: every
-    split of the work list merges to the same result."""
-    L = random_layout(77, [1, 5, 16, 17, 40, 100, 333, 700], dtype="bf16", block_size=16, num_q_heads=8,
+    split of the work list merges to the same result, at every block size."""
+    L = random_layout(77 + B, [1, 5, 16, 17, 40, 100, 333, 700, 1029], dtype="bf16", block_size=B, num_q_heads=8,
                       num_kv_heads=2, head_dim=128)
-    _run_and_check(L, fill_values_numpy(L), cuda_device, num_ctas=num_ctas, what=f"ctas={num_ctas}")
+    _run_and_check(L, fill_values_numpy(L), cuda_device, num_ctas=num_ctas, what=f"B={B} ctas={num_ctas}")
 
 
 def test_physical_placement_does_not_change_bits(pa_mod, cuda_device):
@@ -213,14 +214,16 @@ def test_device_errors_are_reported_not_trapped(pa_mod, cuda_device):
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
-def test_tensor_core_and_cuda_core_paths_agree(pa_mod, cuda_device, dtype, G):
-    """Every group size at head_dim 128 / block 16 runs on the tensor-core
-    kernel by default; the CUDA-core kernel is forced with a flag.  Both must
-    match the oracle, and each other to within the combined tolerance."""
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_tensor_core_and_cuda_core_paths_agree(pa_mod, cuda_device, dtype, G, B):
+    """Every group size at head_dim 128 and blocks of 8, 16 or 32 tokens runs
+    on the tensor-core kernel by default; the CUDA-core kernel is forced with
+    a flag.  Both must match the oracle, and each other to within the
+    combined tolerance."""
     import torch
 
-    lens = [1, 2, 15, 16, 17, 127, 128, 129, 300, 1000, 2049, 5]
-    L = random_layout(4000 + G, lens, dtype=dtype, block_size=16, num_q_heads=2 * G, num_kv_heads=2,
+    lens = [1, 2, B - 1, B, B + 1, 127, 128, 129, 300, 1000, 2049, 5]
+    L = random_layout(4000 + 10 * B + G, lens, dtype=dtype, block_size=B, num_q_heads=2 * G, num_kv_heads=2,
                       head_dim=128, write_new_token=True)
     V = fill_values_numpy(L)
     ref, _, _ = oracle_step(L, V)

@@ -17,6 +17,7 @@ from .generate import (  # noqa: F401
     config_tiny,
     config_llama7b,
     config_llama3_8b,
+    config_llama3_8b_prefill,
     config_llama2_70b_shared,
     config_opt13b_long,
     random_layout,

@@ -249,6 +249,26 @@ def config_llama3_8b(batch: int = 256, q_len: int = 1) -> PagedLayout:
                                f"32/8 heads, D=128, B=16, bf16, {batch * q_len}-token {what}")
 
 
+def config_llama3_8b_prefill(batch: int = 64, q_len: int = 256) -> PagedLayout:
+    """A chunked-prefill step on the Llama-3-8B GQA layer: 64 sequences with
+    the lognormal lengths of the decode workload (median 1024, sigma 0.75,
+    clipped to [q_len, 8192]), each writing its newest q_len tokens (one
+    prefill chunk) and attending them with q_len causal query positions
+    over everything cached before them."""
+    seed = 1006
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal(batch)
+    seq_lens = np.clip(np.rint(1024.0 * np.exp(0.75 * z)), q_len, 8192).astype(np.int32)
+    total = sum(_ceil_div(int(n), 16) for n in seq_lens)
+    NB = int(math.ceil(1.1 * total))
+    tables = _scatter_tables(rng, seq_lens, 16, NB)
+    return _finish_layout(f"llama3_8b_prefill{q_len}", seed, "bf16", 16, NB, 32, 8, 128, seq_lens, tables, True,
+                          q_len=q_len,
+                          note=f"{batch} seqs lognormal(median 1024, sigma 0.75) in [{q_len},8192], 32/8 heads, "
+                               f"D=128, B=16, bf16, a {q_len}-token prefill chunk per sequence "
+                               f"({batch * q_len}-token cache write, {q_len} causal query positions)")
+
+
 def config_llama2_70b_shared(
     prompt_len: int = 2048, num_prompts: int = 32, samples: int = 4, max_tail: int = 512,
     block_size: int = 16,
@@ -326,6 +346,7 @@ CONFIGS: Dict[str, Callable[[], PagedLayout]] = {
     "llama7b": config_llama7b,
     "llama3_8b": config_llama3_8b,
     "llama3_8b_spec4": lambda: config_llama3_8b(q_len=4),
+    "llama3_8b_prefill256": config_llama3_8b_prefill,
     "llama2_70b_shared": config_llama2_70b_shared,
     "opt13b_long_b8": lambda: config_opt13b_long(8),
     "opt13b_long_b16": lambda: config_opt13b_long(16),
