@@ -181,3 +181,64 @@ def oracle_subproblem(layout: PagedLayout, sub, heads=None) -> np.ndarray:
             out[i, k] = oracle.decode_one(i, h, sub["q"], kp, vp, sub["tables"], sub["lens"], layout.scale,
                                           layout.num_kv_heads, layout.dtype)
     return out
+
+
+def oracle_manager_step(mgr, tables, seq_ids, max_nb):
+    """The oracle manager's arrays for one step that appends one token to
+    each of seq_ids: (block_tables, seq_lens, slot_mapping, copy_pairs).
+    tables maps a sequence id to [its oracle block table, its token count]."""
+    n = len(seq_ids)
+    bt = np.full((n, max_nb), -1, np.int32)
+    lens = np.zeros(n, np.int32)
+    slots = np.zeros(n, np.int64)
+    pairs = []
+    for i, s in enumerate(seq_ids):
+        t, ntok = tables[s]
+        slot, cow = mgr.append_slot(t, ntok)
+        tables[s][1] = ntok + 1
+        slots[i] = slot
+        if cow is not None:
+            pairs.append(cow)
+        bt[i, : len(t)] = t
+        lens[i] = ntok + 1
+    return bt, lens, slots, np.asarray(pairs, np.int64).reshape(-1, 2)
+
+
+def run_beam_trace(ours, ref, prompt_len: int, width: int, steps: int, seed: int, max_nb: int, on_step=None,
+                   keep: float = 0.0):
+    """Beam search over one prompt (study notes ch.05 §6.2), driven through
+    the C++ manager `ours` and the oracle manager `ref` side by side: the
+    first step branches the prompt into `width` beams, later steps follow
+    workloads.beam's seeded trace with continuation probability `keep` (free
+    the beams that die, fork the ones that branch, append one token to every
+    live beam).  Every step's kernel
+    arrays must agree between the two managers.  on_step(i, live, arrays)
+    sees each step's arrays.  Returns per step (used blocks, logical
+    blocks), logical = what the live beams would hold without sharing."""
+    from workloads.beam import beam_parents, beam_step
+
+    ours.add(0, prompt_len)
+    tables = {0: [ref.new_sequence(prompt_len), prompt_len]}
+    live, next_id = [0], 1
+    history = []
+    for i, parents in enumerate([[0] * width] + beam_parents(seed, width, steps - 1, keep=keep)):
+        st, next_id = beam_step(live, parents, next_id)
+        for sid in st.frees:
+            ours.free(sid)
+            ref.free_sequence(tables.pop(sid)[0])
+        for parent, child in st.forks:
+            ours.fork(parent, child)
+            tables[child] = [ref.fork(tables[parent][0]), tables[parent][1]]
+        live = st.live
+        arrays = ours.prepare_step(live, max_nb)
+        want = oracle_manager_step(ref, tables, live, max_nb)
+        for got, exp in zip(arrays, want):
+            assert np.array_equal(got, exp), f"beam step {i}: the managers differ"
+        stats = ours.stats()
+        used = len(ref.ref) - len(ref.free)
+        assert stats["used_blocks"] == used
+        assert stats["logical_blocks"] == sum(len(tables[s][0]) for s in live)
+        history.append((stats["used_blocks"], stats["logical_blocks"]))
+        if on_step is not None:
+            on_step(i, live, arrays)
+    return history

@@ -12,6 +12,7 @@ from oracle import BlockManager as OracleBM
 from oracle import block_fills, blocks_needed
 from paged_kv_cache_357_b200 import BlockManager, PaError
 from paged_kv_cache_357_b200 import build as pa_build
+from pa_testlib import run_beam_trace
 
 GOLDEN = json.loads((Path(__file__).parent / "golden" / "bookkeeping.json").read_text())
 
@@ -168,3 +169,48 @@ def test_sharing_statistics_for_beam_style_forks():
     st = bm.stats()
     assert st["tokens"] == 4 * 1024 and st["logical_blocks"] == 4 * 64
     assert st["used_blocks"] == 62 + 4 * 2 and st["shared_blocks"] == 62
+
+
+BEAM_CASES = [(512, 4, 160, 0.0), (64, 8, 256, 0.0), (1000, 6, 96, 0.9), (128, 4, 512, 0.95)]
+
+
+@pytest.mark.parametrize("prompt_len,width,steps,keep", BEAM_CASES)
+def test_beam_search_trace_shares_blocks(prompt_len, width, steps, keep):
+    """Beam search as a process tree (study notes ch.05 §6.2): beams that
+    descend from one beam share the blocks of their common history, dropped
+    beams free theirs, branching beams fork and copy a shared partial block
+    before writing.  The C++ manager follows the oracle manager op by op
+    over a seeded trace; the KV saved by sharing is reported per step."""
+    B = 16
+    max_nb = (prompt_len + steps) // B + 2
+    nb = 4 * width * max_nb
+    hist = run_beam_trace(BlockManager(nb, B), OracleBM(nb, B), prompt_len, width, steps, seed=prompt_len + width,
+                          max_nb=max_nb, keep=keep)
+    saving = [1 - u / l for u, l in hist]
+    mean, final = float(np.mean(saving)), saving[-1]
+    print(f"beam search, prompt {prompt_len}, width {width}, {steps} steps, keep {keep}: KV saved by sharing "
+          f"mean {100 * mean:.1f} %, final {100 * final:.1f} %, "
+          f"blocks stored {hist[-1][0]} vs {hist[-1][1]} unshared")
+    # the prompt alone is shared by every beam at first: at most 1 - 1/width saved
+    assert 0 < saving[0] <= 1 - 1 / width + 1e-12
+    assert all(0 <= s < 1 for s in saving)
+    assert final > 0  # the beams still share at least the prompt's full blocks
+
+
+@pytest.mark.parametrize("prompt_len", [1000, 512, 40])
+def test_beam_search_without_coalescing_shares_the_prompt_only(prompt_len):
+    """keep = 1: every beam continues itself, so after the first step's
+    branching the beams share exactly the prompt's full blocks.  The prompt's
+    partly filled last block is copied by every writer but the last, so the
+    stored blocks are floor(P/B) + width * (ceil(n/B) - floor(P/B)) for n =
+    P + steps tokens per beam."""
+    B, width, steps = 16, 4, 100
+    max_nb = (prompt_len + steps) // B + 2
+    nb = 4 * width * max_nb
+    hist = run_beam_trace(BlockManager(nb, B), OracleBM(nb, B), prompt_len, width, steps, seed=3, max_nb=max_nb,
+                          keep=1.0)
+    for i, (used, logical) in enumerate(hist):
+        n = prompt_len + i + 1
+        shared = prompt_len // B
+        assert logical == width * blocks_needed(n, B)
+        assert used == shared + width * (blocks_needed(n, B) - shared), (i, used)

@@ -9,29 +9,10 @@ import numpy as np
 import pytest
 
 import oracle
-from pa_testlib import assert_attention_close, torch_bits
+from pa_testlib import assert_attention_close, oracle_manager_step, run_beam_trace, torch_bits
 from workloads import bits_to_torch, f32_to_bits
 
 pytestmark = pytest.mark.gpu
-
-
-def _oracle_step(mgr, tables, seq_ids, max_nb, B):
-    """The oracle manager's arrays for one step (appends one token each)."""
-    n = len(seq_ids)
-    bt = np.full((n, max_nb), -1, np.int32)
-    lens = np.zeros(n, np.int32)
-    slots = np.zeros(n, np.int64)
-    pairs = []
-    for i, s in enumerate(seq_ids):
-        t, ntok = tables[s]
-        slot, cow = mgr.append_slot(t, ntok)
-        tables[s][1] = ntok + 1
-        slots[i] = slot
-        if cow is not None:
-            pairs.append(cow)
-        bt[i, : len(t)] = t
-        lens[i] = ntok + 1
-    return bt, lens, slots, np.asarray(pairs, np.int64).reshape(-1, 2)
 
 
 @pytest.mark.parametrize("G", [1, 4])
@@ -76,7 +57,7 @@ def test_block_manager_drives_decode_steps(cuda_device, G):
             new_prompt(30, 70, 2)
             live += [30, 31]
         tables, lens, slots, pairs = ours.prepare_step(live, max_nb)
-        rt, rl, rs, rp = _oracle_step(ref, ref_tables, live, max_nb, B)
+        rt, rl, rs, rp = oracle_manager_step(ref, ref_tables, live, max_nb)
         assert np.array_equal(tables, rt) and np.array_equal(lens, rl)
         assert np.array_equal(slots, rs) and np.array_equal(pairs, rp)
 
@@ -101,3 +82,57 @@ def test_block_manager_drives_decode_steps(cuda_device, G):
     assert np.array_equal(torch_bits(kp), kp_bits) and np.array_equal(torch_bits(vp), vp_bits)
     st_ours = ours.stats()
     assert st_ours["shared_blocks"] > 0 and st_ours["free_blocks"] == len(ref.free)
+
+
+def test_beam_search_drives_decode_steps(cuda_device):
+    """A beam-search trace (study notes ch.05 §6.2: beams share the blocks
+    of their common history, branch by fork, copy a shared partial block
+    before writing, free the beams that die) driven step by step through the
+    copy, write and decode kernels; every step's pools and outputs must
+    match the oracle's."""
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    rng = np.random.default_rng(77)
+    B, Hkv, D, G, dtype = 16, 2, 128, 4, "bf16"
+    Hq, width, steps, prompt = Hkv * G, 6, 24, 203
+    max_nb = (prompt + steps) // B + 2
+    NB = 4 * width * max_nb
+    scale = 1.0 / np.sqrt(D)
+    state = {}
+    state["kb"] = f32_to_bits(rng.standard_normal((NB, Hkv, B, D), dtype=np.float32), dtype)
+    state["vb"] = f32_to_bits(rng.standard_normal((NB, Hkv, B, D), dtype=np.float32), dtype)
+    kp = bits_to_torch(state["kb"], dtype).to(cuda_device)
+    vp = bits_to_torch(state["vb"], dtype).to(cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ws = pa.alloc_decode_workspace(width, Hq, kp)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(cuda_device)  # noqa: E731
+    copies = []
+
+    def on_step(i, live, arrays):
+        tables, lens, slots, pairs = arrays
+        n = len(live)
+        q = f32_to_bits(rng.standard_normal((n, Hq, D), dtype=np.float32), dtype)
+        nk = f32_to_bits(rng.standard_normal((n, Hkv, D), dtype=np.float32), dtype)
+        nv = f32_to_bits(rng.standard_normal((n, Hkv, D), dtype=np.float32), dtype)
+        if pairs.shape[0]:
+            pa.pa_copy_blocks(dev(pairs), kp, vp, st)
+        copies.append(pairs.shape[0])
+        pa.pa_cache_write(bits_to_torch(nk, dtype).to(cuda_device), bits_to_torch(nv, dtype).to(cuda_device),
+                          dev(slots), kp, vp, st)
+        out = torch.full((n, Hq, D), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+        pa.pa_decode(bits_to_torch(q, dtype).to(cuda_device), kp, vp, dev(tables), dev(lens), scale, out, ws, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0, f"beam step {i}"
+        state["kb"], state["vb"] = oracle.copy_blocks(state["kb"], state["vb"], pairs)
+        state["kb"], state["vb"] = oracle.cache_write(state["kb"], state["vb"], nk, nv, slots)
+        ref_out = oracle.decode(q, state["kb"], state["vb"], tables, lens, scale, Hkv, dtype)
+        assert_attention_close(out.double().cpu().numpy(), ref_out, f"beam step {i}")
+
+    hist = run_beam_trace(pa.BlockManager(NB, B), oracle.BlockManager(NB, B), prompt, width, steps, seed=12,
+                          max_nb=max_nb, on_step=on_step, keep=0.5)
+    assert np.array_equal(torch_bits(kp), state["kb"]) and np.array_equal(torch_bits(vp), state["vb"])
+    assert sum(copies) > 0  # branching beams copied shared partial blocks
+    print(f"beam decode: {steps} steps, {sum(copies)} block copies, final KV saved "
+          f"{100 * (1 - hist[-1][0] / hist[-1][1]):.1f} %")
