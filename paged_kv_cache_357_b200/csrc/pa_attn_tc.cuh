@@ -39,16 +39,18 @@
 //               (one 3-D box per block, both 64-column halves), released
 //               when the chunk's PV is done.  A warp issues TMA boxes one
 //               lane at a time, so K and V go out in parallel.
-//   warp 3      lane 0 issues PV of each chunk as soon as its P, V and O
-//               buffer are ready; with QK on its own thread neither product
-//               waits for the other's issue.
-//   warps 4..   softmax + epilogue (WG warpgroups), one TMEM lane (token row,
-//               then head_dim index) per thread: read S^T from TMEM, column
+//   warp 3      lane 0 issues PV of each chunk as soon as its P and V are
+//               ready, accumulating into the O buffer of the chunk's unit
+//               (units alternate between two); with QK on its own thread
+//               neither product waits for the other's issue.
+//   warps 4..   softmax (WG warpgroups), one TMEM lane (token row, then
+//               head_dim index) per thread: read S^T from TMEM, column
 //               maxima and sums by warp butterfly reduce-scatters, write P^T
 //               (bf16/fp16) into a swizzled buffer, zero V rows past the
-//               sequence end inside the last 16-token step, then read O^T
-//               and rescale-accumulate.  The epilogue of chunk i runs after
-//               the softmax of chunk i+1.
+//               sequence end inside the last 16-token step.  O^T stays in
+//               TMEM across a unit's chunks: it is rescaled in place only
+//               when a row's reference max moves (rare past the first
+//               chunk) and read once, when the unit is finished.
 // The swizzled layouts written by TMA serve both products directly: the K
 // tile is a K-major A operand for QK, the V tile an MN-major A operand for PV.
 #pragma once
@@ -99,15 +101,12 @@ struct Blk {
   // V stage offset of token t of the chunk (its row in the first half)
   __host__ __device__ static constexpr int v_offset(int t) { return (t / BB) * kVBlockBytes + (t % BB) * kRowBytes; }
 };
-constexpr int kSoftmaxBarrier = 1;
+constexpr int kSoftmaxBarrier = 1;          // all softmax warps
+constexpr int kWarpgroupBarrier0 = 2;       // + warpgroup index: one softmax warpgroup
 constexpr int kQKWarp = 1;                 // allocates TMEM, issues QK
 constexpr int kVWarp = 2;                  // the V producer (warp 0 loads q and K)
 constexpr int kPVWarp = 3;                 // issues PV
 constexpr int kSoftmaxWarp0 = 4;           // first softmax warp
-// With two softmax warpgroups the control warpgroup hands registers to them
-// (setmaxnreg): 128 x 72 + 256 x 216 = 384 x 168, the launch's allocation.
-constexpr int kCtrlRegs = 72;
-constexpr int kSoftmaxRegs = 216;
 // A row's probabilities are taken relative to a reference max that only moves
 // when a score exceeds it by more than this (log2 units): p <= 2^8 stays
 // exact enough in 16-bit and in the fp32 sums, and most chunks need neither
@@ -142,13 +141,21 @@ struct Rows {
   static constexpr int kCols = 2 * Nq + 2 * Np;
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : 256;
   static constexpr int kPartStride = R * (D + 2);                 // floats per partial slot
-  // Softmax warpgroups: one for up to 8 rows; two for 16 or 32, each taking
+  // Softmax warpgroups: one for up to 8 rows, two for 16 or 32, each taking
   // RC = R / WG of the rows (both read every token row of S and O).
   static constexpr int WG = R >= 16 ? 2 : 1;
   static constexpr int RC = R / WG;
   static constexpr int kSoftmaxThreads = 128 * WG;
   static constexpr int kThreads = 128 + kSoftmaxThreads;         // + K, QK, V and PV warps
   static constexpr int kLanesPerCol = 32 / RC;                    // lanes holding one column after a reduce
+  // With two softmax warpgroups the control warpgroup hands registers to
+  // them (setmaxnreg) inside the launch's allocation of 168 a thread:
+  // 128 x 72 + 256 x 216 = 384 x 168.
+  static constexpr int kCtrlRegs = 72;
+  static constexpr int kSoftmaxRegs = 216;
+  static constexpr int kLaunchRegs = 168;
+  static_assert(WG == 1 || 128 * kCtrlRegs + kSoftmaxThreads * kSoftmaxRegs <= kThreads * kLaunchRegs,
+                "the register split fits the launch's allocation");
 };
 
 template <int R>
@@ -160,9 +167,7 @@ struct TcSmem {
   uint8_t p[2][S::kPSlotBytes];
   alignas(16) float red[2][4][R];  // per-warp column maxima, double-buffered by chunk
   alignas(16) float mfin[R];       // reference max of each row of the segment being finished
-  alignas(16) float abuf[2][R];    // rescale factor of each chunk's running output
   alignas(16) float lred[4][R];    // per-warp row sums of the segment being finished
-  int rescaled[2];                 // whether a chunk's rows changed their reference max
   uint64_t kfull[kKStages];
   uint64_t kempty[kKStages];
   uint64_t vfull[S::kVStages];
@@ -172,8 +177,8 @@ struct TcSmem {
   uint64_t s_full[2];
   uint64_t s_free[2];
   uint64_t p_full[2];
-  uint64_t o_full[2];
-  uint64_t o_free[2];
+  uint64_t pv_done;                // one phase per chunk: its PV has completed
+  uint64_t o_free[2];              // a segment's O buffer has been read by its finish
   uint64_t mma_done[2];            // the QK and the PV issuer's last MMAs
   RangeSmem range;
   uint32_t tmem_base;
@@ -278,6 +283,35 @@ __device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, uint32_t* r) {
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Columns [0, NC) of this thread's TMEM lane from r (NC = 8 or a multiple of 16).
+template <int NC>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t* r) {
+  if constexpr (NC == 8) {
+    tmem_st8(taddr, r);
+  } else {
+    static_assert(NC % 16 == 0, "8 or a multiple of 16 columns");
+#pragma unroll
+    for (int c = 0; c < NC; c += 16) tmem_st16(taddr + c, r + c);
+  }
+}
 
 // Columns [0, NC) of this thread's TMEM lane (NC = 8 or a multiple of 16),
 // issued without waiting; tmem_wait_ld() completes them.
@@ -715,6 +749,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   using Sh = Rows<R>;
   constexpr int Nq = Sh::Nq, Np = Sh::Np, kVStages = Sh::kVStages, kLanesPerCol = Sh::kLanesPerCol;
   constexpr int WG = Sh::WG, RC = Sh::RC, kThreads = Sh::kThreads, kSoftmaxThreads = Sh::kSoftmaxThreads;
+  constexpr int kCtrlRegs = Sh::kCtrlRegs, kSoftmaxRegs = Sh::kSoftmaxRegs;
   constexpr int RL = RC < 8 ? 8 : RC;  // TMEM columns loaded per row set (x8 is the narrowest load used)
   static_assert(kMode != kDecode || RG == 1, "a decode unit has one row group");
   using Bk = Blk<B>;
@@ -746,9 +781,9 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.s_free[i], 4 * WG);  // one arrival per softmax warp
       mbar_init(&sm.p_full[i], 4 * WG);
-      mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.o_free[i], 4 * WG);
     }
+    mbar_init(&sm.pv_done, 1);
     mbar_init(&sm.mma_done[0], 1);
     mbar_init(&sm.mma_done[1], 1);
     sm.abort = 0;
@@ -790,7 +825,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     // nothing to stream: straight to teardown
   } else if (warp == 0 || warp == kVWarp) {
     // ===================== producers ========================================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+    if constexpr (WG > 1) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     // Warp 0 loads q and K, warp 2 loads V, each walking the same chunks.  A
     // warp issues its TMA boxes one lane at a time (about 70 cycles each), so
     // one warp issuing all 32 boxes of a chunk would take longer than HBM
@@ -918,7 +953,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     }
   } else if (warp == kQKWarp) {
     // ===================== QK issuer =========================================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+    if constexpr (WG > 1) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     // Lane 0 issues QK of each chunk once its K has landed, its S buffer is
     // free and its q is loaded; it sleeps in the barrier waits in between.
     if (lane == 0) {
@@ -964,25 +999,27 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     __syncwarp();
   } else if (warp == kPVWarp) {
     // ===================== PV issuer =========================================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
-    // Lane 0 issues PV of each chunk once its P is written, its V has landed
-    // and its O buffer has been read; only the 16-token steps that hold
-    // valid tokens are issued.
+    if constexpr (WG > 1) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+    // Lane 0 issues PV of each chunk once its P is written and its V has
+    // landed; only the 16-token steps that hold valid tokens are issued.  A
+    // segment's products accumulate in one O buffer (segments alternate
+    // between two), started by its first chunk once the finish of the
+    // segment before last has read that buffer.
     if (lane == 0) {
       constexpr uint32_t kIdescPV = make_idesc(kBf16, true, true, Np);  // V: MN-major A, P: MN-major B
       bool ok = true;
-      int pv = 0;
+      int pv = 0, seg_i = 0;
       Seg sg;
       while (ok && next_seg<B, CB>(cur, sg, p, src)) {
         ChunkWalk<kMode, G, RG, B> walk;
         walk.start(p, sg, 0);
+        const int ob = seg_i & 1;
+        ok = mbar_wait_bounded(&sm.o_free[ob], ((seg_i >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
         for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
           const int ntok = walk.next(p).ntok;
           const int pb = pv & 1;
-          const uint32_t par = (pv >> 1) & 1;
           const int vs = pv % kVStages;
-          ok = mbar_wait_bounded(&sm.p_full[pb], par, abort_flag, p.wait_limit_ns) &&
-               mbar_wait_bounded(&sm.o_free[pb], par ^ 1u, abort_flag, p.wait_limit_ns) &&
+          ok = mbar_wait_bounded(&sm.p_full[pb], (pv >> 1) & 1, abort_flag, p.wait_limit_ns) &&
                mbar_wait_bounded(&sm.vfull[vs], (pv / kVStages) & 1, abort_flag, p.wait_limit_ns);
           if (!ok) break;
           tc_fence_after();
@@ -993,12 +1030,13 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
             const uint64_t a = sw128_desc(v0 + Bk::v_offset(16 * k), Bk::kBlockBytes, Bk::kVGroupBytes);
             // tokens [16k, 16k + 16): two groups of 8 token rows; Np fits one swizzle atom
             const uint64_t b = smem_desc(p0 + k * 16 * Sh::kPRowBytes, 0, 8 * Sh::kPRowBytes, Sh::kPLayout);
-            umma(tmem + kColO + pb * Np, a, b, kIdescPV, k > 0 ? 1u : 0u);
+            umma(tmem + kColO + ob * Np, a, b, kIdescPV, (c0 > 0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(&sm.o_full[pb]);
+          umma_commit(&sm.pv_done);
           umma_commit(&sm.vempty[vs]);
           ++pv;
         }
+        ++seg_i;
       }
       umma_commit(&sm.mma_done[1]);
       (void)mbar_wait_bounded(&sm.mma_done[1], 0, nullptr, p.wait_limit_ns);
@@ -1010,31 +1048,99 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ===================== softmax + epilogue (warps 4..) ====================
-    if constexpr (WG == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    // Per chunk i: softmax(i) then the epilogue of chunk i-1, so the PV of
-    // chunk i-1 runs on the tensor core while the softmax of chunk i runs
-    // here; chunks of consecutive segments form one stream.
+    // ===================== softmax (warps 4..) ==============================
+    if constexpr (WG > 1) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    // Per chunk: the scores from TMEM, the online softmax, P^T into shared
+    // memory.  The chunk's PV accumulates into its segment's O buffer in
+    // TMEM, so nothing is read back per chunk: O is read once, by the
+    // segment's finish, and rescaled in place on the rare chunk whose
+    // reference maxima move.  The finish of a segment runs after the softmax
+    // of the next segment's first chunk, so the copies and the tensor core
+    // stream across unit boundaries.
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
-    const int r = quad * 32 + lane;   // token row of the chunk; head_dim index in the epilogue
+    const int r = quad * 32 + lane;   // token row of the chunk; head_dim index of O
     const int ctid = tid - 32 * kSoftmaxWarp0;  // 0 .. kSoftmaxThreads - 1
-    const int col0 = ((warp - kSoftmaxWarp0) / 4) * RC;  // this warpgroup's query rows: col0 .. col0 + RC - 1
+    const int wg = (warp - kSoftmaxWarp0) / 4;
+    const int col0 = wg * RC;         // this warpgroup's query rows: col0 .. col0 + RC - 1
+    const int wg_bar = kWarpgroupBarrier0 + wg;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int my_col = col0 + lane / kLanesPerCol;  // the row this lane holds after a reduce
     const bool col_writer = (lane % kLanesPerCol) == 0;
     bool ok = true;
-    int ci = 0;
+    int ci = 0;       // chunks started
+    int pv_seen = 0;  // pv_done phases consumed: chunks whose PV has completed
+    int si = 0;       // segments started
     Seg sg;
-    float acc[RC];
-    float m_ref[RC];  // reference max of each of this thread's rows (the same in every thread)
+    float m_ref[RC];  // reference max of each of this warpgroup's rows (the same in all its threads)
     float l_thr[RC];  // sum of p over this thread's token rows, relative to m_ref
 
-    // Online softmax of chunk ci (the first of its segment when `first`):
-    // P^T into the swizzled B operand.  The reference maxima move only when
-    // some score exceeds them by more than kRescaleGap (always on a
-    // segment's first chunk); then the chunk's row maxima are reduced across
-    // the warps and the rescale factors are left for the epilogue.
-    auto softmax_chunk = [&](int ci, const ChunkSrc& ch, bool first) -> bool {
+    // Consume the pv_done phases of every chunk before `upto`, in order (a
+    // chunk's PV is only issued after its softmax, so no phase is skipped).
+    auto wait_pv = [&](int upto) -> bool {
+      while (pv_seen < upto) {
+        const bool w = mbar_wait_bounded(&sm.pv_done, pv_seen & 1, abort_flag, p.wait_limit_ns);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        ++pv_seen;
+      }
+      tc_fence_after();
+      return true;
+    };
+
+    // This warpgroup's columns of O buffer ob: the heads (col0 ..) and the
+    // residuals (R + col0 ..); for R <= 8 one 16-column block holds both.
+    auto o_addr = [&](int ob, int part) -> uint32_t {
+      return tmem + lane_base + kColO + ob * Np + (R <= 8 ? 0 : part * R + col0);
+    };
+    auto load_o = [&](int ob, float (&acc)[RC]) {
+      if constexpr (R <= 8) {
+        uint32_t v[16];
+        tmem_ld_nowait<16>(o_addr(ob, 0), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < RC; ++k) acc[k] = __uint_as_float(v[k]) + __uint_as_float(v[R + k]);
+      } else {
+        uint32_t h[RC], l[RC];
+        tmem_ld_nowait<RC>(o_addr(ob, 0), h);
+        tmem_ld_nowait<RC>(o_addr(ob, 1), l);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < RC; ++k) acc[k] = __uint_as_float(h[k]) + __uint_as_float(l[k]);
+      }
+    };
+    // O *= alpha per row, in place (PV of the previous chunk complete, of
+    // this chunk not yet issued).
+    auto rescale_o = [&](int ob, const float (&alpha)[RC]) {
+      if constexpr (R <= 8) {
+        uint32_t v[16];
+        tmem_ld_nowait<16>(o_addr(ob, 0), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 2 * R; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha[j % R]);
+        tmem_st<16>(o_addr(ob, 0), v);
+      } else {
+        uint32_t h[RC], l[RC];
+        tmem_ld_nowait<RC>(o_addr(ob, 0), h);
+        tmem_ld_nowait<RC>(o_addr(ob, 1), l);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < RC; ++k) {
+          h[k] = __float_as_uint(__uint_as_float(h[k]) * alpha[k]);
+          l[k] = __float_as_uint(__uint_as_float(l[k]) * alpha[k]);
+        }
+        tmem_st<RC>(o_addr(ob, 0), h);
+        tmem_st<RC>(o_addr(ob, 1), l);
+      }
+      tmem_wait_st();
+    };
+
+    // Online softmax of chunk ci (the first of its segment when `first`),
+    // whose PV goes to O buffer ob: P^T into the swizzled B operand.  The
+    // reference maxima move only when some score exceeds them by more than
+    // kRescaleGap (always on a segment's first chunk); then the chunk's row
+    // maxima are reduced across the warpgroup's warps and, past the first
+    // chunk, the rows of O are rescaled.  Each warpgroup decides for its own
+    // rows.
+    auto softmax_chunk = [&](int ci, const ChunkSrc& ch, bool first, int ob) -> bool {
       const int vs = ci % kVStages;
       const int sb = ci & 1;
       bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
@@ -1066,7 +1172,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
         over |= sc[k] > m_ref[k] + kRescaleGap;
       }
-      const bool rescale = named_barrier_or(kSoftmaxBarrier, kSoftmaxThreads, over);  // uniform
+      const bool rescale = named_barrier_or(wg_bar, 128, over);  // uniform per warpgroup
+      float alpha[RC];
       if (rescale) {
         if (mine) {
           float v[RC];
@@ -1075,8 +1182,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           const float wm = warp_column_reduce<RC, true>(v, lane);
           if (col_writer) sm.red[sb][quad][my_col] = wm;
         }
-        named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
-        float cm[RC], tt[RC], alpha[RC];
+        named_barrier_sync(wg_bar, 128);
+        float cm[RC], tt[RC];
         if (mine) {
           ld_row<RC>(sm.red[sb][0] + col0, cm);
 #pragma unroll
@@ -1097,15 +1204,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           m_ref[k] = m_new;
           l_thr[k] = first ? 0.f : l_thr[k] * alpha[k];
         }
-        // the epilogue of this chunk rescales the running output
-        if (quad == 0 && lane < RC) {
-          float a = alpha[0];
-#pragma unroll
-          for (int k = 1; k < RC; ++k) a = lane == k ? alpha[k] : a;
-          sm.abuf[ci & 1][col0 + lane] = a;
-        }
       }
-      if (ctid == 0) sm.rescaled[ci & 1] = rescale ? 1 : 0;
       float pr[RC];
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
@@ -1114,7 +1213,9 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       }
       // P^T, MN-major: token row r holds at position c the head of query row
       // c's probability and at R + c its rounding residual, written as whole
-      // 16-byte chunks of 8 values (this warpgroup's rows col0 .. col0 + RC)
+      // 16-byte chunks of 8 values (this warpgroup's rows col0 .. col0 + RC).
+      // The buffer's last reader, PV of chunk ci - 2, completed before chunk
+      // ci - 1 was released.
       const int pb = ci & 1;
       {
         uint8_t* prow = sm.p[pb] + r * Sh::kPRowBytes;
@@ -1159,36 +1260,13 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[pb]);
-
-      return true;
-    };
-
-    // acc = acc * alpha(ci) + O^T row r of chunk ci.
-    auto epilogue_chunk = [&](int ci) -> bool {
-      const int pb = ci & 1;
-      bool w = mbar_wait_bounded(&sm.o_full[pb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
-      if (!__all_sync(0xffffffffu, w)) return false;
-      tc_fence_after();
-      // this warpgroup's rows: head columns col0.., residual columns R + col0..
-      uint32_t oh[RL], ol[RL];
-      tmem_ld_nowait<RL>(tmem + lane_base + kColO + pb * Np + col0, oh);
-      tmem_ld_nowait<RL>(tmem + lane_base + kColO + pb * Np + R + col0, ol);
-      tmem_wait_ld();
+      // the previous chunk's PV must be complete before O is rescaled and
+      // before this chunk's PV may add to it
+      if (!wait_pv(ci)) return false;
+      if (rescale && !first) rescale_o(ob, alpha);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.o_free[pb]);
-      if (sm.rescaled[ci & 1]) {
-        float alpha[RC];
-        ld_row<RC>(sm.abuf[ci & 1] + col0, alpha);
-#pragma unroll
-        for (int k = 0; k < RC; ++k)
-          acc[k] = fmaf(acc[k], alpha[k], __uint_as_float(oh[k]) + __uint_as_float(ol[k]));
-      } else {
-#pragma unroll
-        for (int k = 0; k < RC; ++k) acc[k] += __uint_as_float(oh[k]) + __uint_as_float(ol[k]);
-      }
+      if (lane == 0) mbar_arrive(&sm.p_full[pb]);
       return true;
     };
 
@@ -1209,11 +1287,15 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       }
     };
 
-    // The finish of a segment (its rows or its partial state, and the merge
-    // when it arrives last) runs after the softmax of the next segment's
-    // first chunk, so the copies and the tensor core keep streaming across
-    // unit boundaries.
-    auto finish_segment = [&](const Seg& fs, int rows) {
+    // The finish of a segment whose PVs have all completed: its rows, or its
+    // partial state and the merge when it arrives last.  Its O buffer is
+    // read once and handed back to the PV issuer.
+    auto finish_segment = [&](const Seg& fs, int rows, int ob) {
+      float acc[RC];
+      load_o(ob, acc);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free[ob]);
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
       if (fs.j0 == fs.first && fs.j0 + fs.n == fs.nb) {
         float m[RC], L[RC];
@@ -1238,48 +1320,43 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
             [] { named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads); });
       }
       named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
-#pragma unroll
-      for (int k = 0; k < RC; ++k) acc[k] = 0.f;
     };
 
 #pragma unroll
     for (int k = 0; k < RC; ++k) {
-      acc[k] = 0.f;
       m_ref[k] = -INFINITY;
       l_thr[k] = 0.f;
     }
     Seg prev;               // the segment whose finish is still due
     int prev_rows = 0;
     bool have_prev = false;
-    bool pending = false;   // the epilogue of chunk ci - 1 is still due
     while (ok && next_seg<B, CB>(cur, sg, p, src)) {
       const int rows = G * src.row_groups(p, sg.s);
       ChunkWalk<kMode, G, RG, B> walk;
       walk.start(p, sg, rows);
+      const int ob = si & 1;
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
         if (c0 == 0 && have_prev) stash_segment();
-        ok = softmax_chunk(ci, walk.next(p), c0 == 0);
+        ok = softmax_chunk(ci, walk.next(p), c0 == 0, ob);
         if (!ok) break;
-        if (pending) {
-          ok = epilogue_chunk(ci - 1);
-          if (!ok) break;
-        }
-        if (c0 == 0 && have_prev) {
-          finish_segment(prev, prev_rows);
+        ++ci;
+        if (c0 == 0 && have_prev) {  // every PV of the previous segment is complete
+          finish_segment(prev, prev_rows, ob ^ 1);
           have_prev = false;
         }
-        pending = true;
-        ++ci;
       }
       if (!ok) break;
       prev = sg;
       prev_rows = rows;
       have_prev = true;
+      ++si;
     }
-    if (ok && pending) ok = epilogue_chunk(ci - 1);
     if (ok && have_prev) {
-      stash_segment();
-      finish_segment(prev, prev_rows);
+      ok = wait_pv(ci);
+      if (ok) {
+        stash_segment();
+        finish_segment(prev, prev_rows, (si - 1) & 1);
+      }
     }
     if (!ok && lane == 0) {
       sm.abort = 1;
@@ -1435,14 +1512,15 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
   want.kv_rows = kv_rows;
   want.num_q_heads = prm.num_q_heads;
   if (!cached_maps(want, mq, mk, mv, &encode_launch_maps<kBf16, G, RG, B>)) return cudaErrorInvalidValue;
-  if constexpr (Rows<G * RG>::WG == 2) {
+  if constexpr (Rows<G * RG>::WG > 1) {
     // setmaxnreg only moves registers inside the launch's allocation; should
     // a build give the kernel fewer than the split needs, the softmax warps'
     // increase would wait forever, so such a kernel is not launched.
     static const bool regs_fit = [] {
       cudaFuncAttributes a{};
       return cudaFuncGetAttributes(&a, pa_decode_tc_kernel<kBf16, G, RG, kMode, B>) == cudaSuccess &&
-             a.numRegs * Rows<G * RG>::kThreads >= 128 * kCtrlRegs + 256 * kSoftmaxRegs;
+             a.numRegs * Rows<G * RG>::kThreads >=
+                 128 * Rows<G * RG>::kCtrlRegs + Rows<G * RG>::kSoftmaxThreads * Rows<G * RG>::kSoftmaxRegs;
     }();
     if (!regs_fit) return cudaErrorInvalidConfiguration;
   }
