@@ -394,6 +394,88 @@ PA_API pa_status pa_shared_prefix_groups(const int32_t* block_tables, int32_t ma
                                          int32_t max_group_size, int32_t min_prefix_blocks, int32_t* group_starts,
                                          int32_t* group_prefix_blocks, int32_t* num_groups);
 
+/*
+ * pa_step — one whole step of a paged KV cache driven from pinned host
+ * memory: the host->device copy of the step's inputs, the copy-on-write
+ * block copies (pa_copy_blocks, study notes ch.05 §6.1), the cache write of
+ * the new tokens (pa_cache_write, vLLM blog plain-language section), the
+ * decode (pa_decode, pa_decode_multi or pa_decode_shared_prefix; vLLM blog
+ * §"关键细节" 2) and the device->host copy of the output, in that order.
+ * The pages describe the step, not a runtime; this is the calling
+ * convention of this library for a serving loop.
+ *
+ * Memory is the caller's: for each of num_sets buffer sets, a device input
+ * block and a pinned host input block of pa_step_layout.total bytes each
+ * (16-byte aligned), a device output and a pinned host output of
+ * pa_step_layout.out_bytes; the pools, the decode workspace (sized by the
+ * decode's own *_workspace_bytes for the shape) and dev_status.  The input
+ * blocks are laid out as pa_step_layout_of gives (q, block_tables,
+ * seq_lens, group_starts, group_prefix_blocks, copy_pairs, new k, new v,
+ * slot_mapping; the same layouts as the entry points take, each field at
+ * its maximum size).  The step creates three CUDA streams (uploads,
+ * kernels, downloads), events and, per buffer set and counts, one CUDA
+ * graph of its kernels (the first step runs them directly); it allocates
+ * no memory of its own.
+ *
+ * Per pa_step_run the host issues one copy of the used part of the set's
+ * input block, one graph launch and one copy of the output.  Sets are used
+ * in turn: the upload into a set waits for the kernels that last read it,
+ * the kernels of a step wait for its upload, for the previous step's
+ * kernels (in-order stream: they share the pools) and for the download
+ * that last read the set's output, so neighbouring steps' copies overlap
+ * each other's kernels.  Call pa_step_next_set before writing a set's host
+ * input block: it returns the set the next pa_step_run uses, once that
+ * set's previous upload is done.  pa_step_wait blocks until a set's output
+ * has reached its host block.  Errors: PA_ERR_INVALID_ARG for a bad shape
+ * or pointer, the decode's own return codes from the first step, and
+ * PA_ERR_CUDA for a failed CUDA call.
+ */
+#define PA_STEP_DECODE 0        /* pa_decode (opts.flags may hold PA_DECODE_CUDA_CORES_ONLY) */
+#define PA_STEP_MULTI 1         /* pa_decode_multi with q_len positions per sequence */
+#define PA_STEP_SHARED_PREFIX 2 /* pa_decode_shared_prefix over groups of up to max_group_size */
+#define PA_STEP_MAX_SETS 8
+
+typedef struct pa_step_shape {
+  int32_t kind;               /* PA_STEP_* */
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t max_blocks_per_seq;
+  int32_t q_len;              /* PA_STEP_MULTI: positions per sequence (>= 2); else 1 */
+  int32_t max_group_size;     /* PA_STEP_SHARED_PREFIX: members per group; else 0 */
+  int32_t max_new_tokens;     /* capacity of the new-token fields */
+  int32_t max_copy_pairs;     /* capacity of the copy-pair field */
+  float scale;
+  pa_decode_opts opts;
+} pa_step_shape;
+
+/* Byte offsets of the fields in a set's input block, its size and the
+ * output size.  Fields a shape does not use have size 0 (offset = the next
+ * field's). */
+typedef struct pa_step_layout {
+  size_t q, block_tables, seq_lens, group_starts, group_prefix_blocks, copy_pairs, new_k, new_v, slot_mapping;
+  size_t total;
+  size_t out_bytes;
+} pa_step_layout;
+
+typedef struct pa_step pa_step;
+
+PA_API pa_status pa_step_layout_of(const pa_step_shape* shape, const pa_pool_desc* pool, pa_step_layout* layout);
+PA_API pa_status pa_step_create(const pa_step_shape* shape, const pa_pool_desc* pool, void* k_pool, void* v_pool,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_status, int32_t num_sets,
+                                void* const* dev_inputs, void* const* host_inputs, void* const* dev_outputs,
+                                void* const* host_outputs, pa_step** step);
+/* The set the next pa_step_run uses (its previous upload done). */
+PA_API pa_status pa_step_next_set(pa_step* step, int32_t* set);
+/* Enqueue one step with these counts (copy pairs, new tokens, shared-prefix
+ * groups) from the next set's host input block; *set = the set used. */
+PA_API pa_status pa_step_run(pa_step* step, int32_t num_copy_pairs, int32_t num_new_tokens, int32_t num_groups,
+                             int32_t* set);
+PA_API pa_status pa_step_wait(pa_step* step, int32_t set);
+PA_API pa_status pa_step_synchronize(pa_step* step);
+/* The upload, kernel and download streams (cudaStream_t as void*). */
+PA_API pa_status pa_step_streams(pa_step* step, void** upload, void** kernels, void** download);
+PA_API void pa_step_destroy(pa_step* step);
+
 /* Static string for a pa_status or PA_DEV_* code. */
 PA_API const char* pa_status_string(int32_t status);
 

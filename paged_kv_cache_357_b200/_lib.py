@@ -53,7 +53,18 @@ EXPORTED = (
     "pa_bm_table",
     "pa_bm_get_stats",
     "pa_bm_prepare_step",
+    "pa_step_layout_of",
+    "pa_step_create",
+    "pa_step_next_set",
+    "pa_step_run",
+    "pa_step_wait",
+    "pa_step_synchronize",
+    "pa_step_streams",
+    "pa_step_destroy",
 )
+
+PA_STEP_DECODE, PA_STEP_MULTI, PA_STEP_SHARED_PREFIX = 0, 1, 2
+PA_STEP_MAX_SETS = 8
 
 
 class PoolDesc(ctypes.Structure):
@@ -68,6 +79,30 @@ class PoolDesc(ctypes.Structure):
 
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("num_ctas", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+
+class StepShape(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_int32),
+        ("num_seqs", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32),
+        ("q_len", ctypes.c_int32),
+        ("max_group_size", ctypes.c_int32),
+        ("max_new_tokens", ctypes.c_int32),
+        ("max_copy_pairs", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("opts", DecodeOpts),
+    ]
+
+
+STEP_FIELDS = ("q", "block_tables", "seq_lens", "group_starts", "group_prefix_blocks", "copy_pairs", "new_k", "new_v",
+               "slot_mapping")
+
+
+class StepLayout(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_size_t) for name in STEP_FIELDS] + [("total", ctypes.c_size_t),
+                                                                     ("out_bytes", ctypes.c_size_t)]
 
 
 class PaError(RuntimeError):
@@ -117,6 +152,24 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_cache_write.restype = i32
     lib.pa_copy_blocks.argtypes = [vp, i32, vp, vp, vp, pdesc, vp]
     lib.pa_copy_blocks.restype = i32
+    pshape, playout = ctypes.POINTER(StepShape), ctypes.POINTER(StepLayout)
+    vpp = ctypes.POINTER(ctypes.c_void_p)
+    lib.pa_step_layout_of.argtypes = [pshape, pdesc, playout]
+    lib.pa_step_layout_of.restype = i32
+    lib.pa_step_create.argtypes = [pshape, pdesc, vp, vp, vp, sz, vp, i32, vpp, vpp, vpp, vpp, vpp]
+    lib.pa_step_create.restype = i32
+    lib.pa_step_next_set.argtypes = [vp, ctypes.POINTER(i32)]
+    lib.pa_step_next_set.restype = i32
+    lib.pa_step_run.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32)]
+    lib.pa_step_run.restype = i32
+    lib.pa_step_wait.argtypes = [vp, i32]
+    lib.pa_step_wait.restype = i32
+    lib.pa_step_synchronize.argtypes = [vp]
+    lib.pa_step_synchronize.restype = i32
+    lib.pa_step_streams.argtypes = [vp, vpp, vpp, vpp]
+    lib.pa_step_streams.restype = i32
+    lib.pa_step_destroy.argtypes = [vp]
+    lib.pa_step_destroy.restype = None
     lib.pa_status_string.argtypes = [i32]
     lib.pa_status_string.restype = ctypes.c_char_p
     if path == LIB_PATH:

@@ -29,6 +29,7 @@ SOURCES = [
     "pa_attn_tc_group.cu",
     "pa_kv_ops.cu",
     "pa_block_manager.cpp",
+    "pa_step.cpp",
 ]
 HEADERS = ["pa_device.cuh", "pa_internal.h", "pa_decode_common.cuh", "pa_decode_host.h", "pa_attn_tc.cuh"]
 

@@ -113,7 +113,13 @@ constexpr int kSoftmaxWarp0 = 4;           // first softmax warp
 // a cross-warp max nor a rescale.
 constexpr float kRescaleGap = 8.f;
 
-enum Mode { kDecode = 0, kMulti = 1, kGroup = 2 };
+enum Mode { kDecode = 0, kMulti = 1, kGroup = 2, kMultiTiled = 3 };
+
+// kMulti: one unit per sequence (G x q_len rows fit one unit); kMultiTiled:
+// several units (row tiles) per sequence, for longer q_len.  Two modes
+// rather than one, so that the common single-unit form carries none of the
+// tiling arithmetic.
+__host__ __device__ constexpr bool is_multi(int mode) { return mode == kMulti || mode == kMultiTiled; }
 
 // Shapes that follow from the number of query rows R of a unit.  P enters
 // the PV product as two 16-bit rows per query row, p = hi + lo (the head and
@@ -453,13 +459,30 @@ struct Source<kDecode, RG> {
   __device__ __forceinline__ int row_groups(const DecodeParams&, int) const { return 1; }
 };
 
-// Query positions of a sequence, causal among the new tokens.  Unit u is row
-// tile t = u % q_tiles of sequence s = u / q_tiles: positions [t RG,
-// min(q_len, (t + 1) RG)), so a sequence with G x q_len query rows past what
-// one unit holds is covered by several units.  A tile reads only the blocks
-// its last position sees.  A sequence shorter than q_len is treated as empty.
+// A sequence with q_len query positions, causal among the new tokens, in
+// one unit.  A sequence shorter than q_len is treated as empty.
 template <int RG>
 struct Source<kMulti, RG> {
+  template <int BB>
+  __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int s) const {
+    int len = checked_len(p, s, BB);
+    if (len < p.q_len) len = 0;
+    return SeqSpan{0, (len + BB - 1) / BB, len};
+  }
+  __device__ __forceinline__ int count(const DecodeParams& p) const { return p.num_seqs; }
+  __device__ __forceinline__ int table_row(const DecodeParams&, int s) const { return s; }
+  __device__ __forceinline__ int pos0(const DecodeParams&, int) const { return 0; }
+  __device__ __forceinline__ int row_group0(const DecodeParams& p, int s) const { return s * p.q_len; }
+  __device__ __forceinline__ int row_groups(const DecodeParams& p, int) const { return p.q_len; }
+};
+
+// The same over several units per sequence.  Unit u is row tile t = u %
+// q_tiles of sequence s = u / q_tiles: positions [t RG, min(q_len, (t + 1)
+// RG)), so a sequence with G x q_len query rows past what one unit holds is
+// covered by several units.  A tile reads only the blocks its last position
+// sees.  A sequence shorter than q_len is treated as empty.
+template <int RG>
+struct Source<kMultiTiled, RG> {
   template <int BB>
   __device__ __forceinline__ SeqSpan span(const DecodeParams& p, int u) const {
     const int s = u / p.q_tiles;
@@ -527,13 +550,13 @@ struct ChunkWalk {
   __device__ __forceinline__ void start(const DecodeParams& p, const Seg& sg, int rows) {
     pos0 = 0;
     if constexpr (kMode != kGroup) {
-      seq = kMode == kMulti ? sg.s / p.q_tiles : sg.s;
+      seq = kMode == kMultiTiled ? sg.s / p.q_tiles : sg.s;
       j = sg.j0;
       jend = sg.j0 + sg.n;
       len = sg.len;
       row_lo = 0;
       row_hi = rows;
-      if constexpr (kMode == kMulti) pos0 = (sg.s % p.q_tiles) * RG;
+      if constexpr (kMode == kMultiTiled) pos0 = (sg.s % p.q_tiles) * RG;
     } else {
       s0 = __ldg(p.group_starts + sg.s);
       s1 = __ldg(p.group_starts + sg.s + 1);
@@ -636,7 +659,7 @@ __device__ void group_bookkeeping(const DecodeParams& p, const Source<kGroup, RG
   }
 }
 
-// kDecode and kMulti: zero the output rows of units with nothing to read
+// kDecode and the multi-query modes: zero the output rows of units with nothing to read
 // (length 0, invalid, or shorter than q_len); unit u by CTA u % gridDim.x.
 template <int kMode, int RG, int B>
 __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>& src) {
@@ -644,7 +667,7 @@ __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>&
   const int units = src.count(p);
   for (int u = threadIdx.x; u < units; u += blockDim.x) {
     if ((u % nctas) != cta) continue;
-    if constexpr (kMode == kMulti) {
+    if constexpr (is_multi(kMode)) {
       const int raw = __ldg(p.seq_lens + src.table_row(p, u));
       if (src.pos0(p, u) == 0 && raw > 0 && raw < p.q_len) record_status(p.status, PA_DEV_BAD_SEQ_LEN);
     }
@@ -674,9 +697,11 @@ __device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, 
     if (c < rows) {
       const int rg = c / G;
       size_t row;
-      if constexpr (kMode == kMulti) {
+      if constexpr (kMode == kMultiTiled) {
         const int s = sg.s / p.q_tiles;
         row = static_cast<size_t>(s) * p.q_len + (sg.s - s * p.q_tiles) * RG + rg;
+      } else if constexpr (kMode == kMulti) {
+        row = static_cast<size_t>(sg.s) * p.q_len + rg;
       } else if constexpr (kMode == kGroup) {
         row = static_cast<size_t>(s0 + rg);
       } else {
@@ -1168,7 +1193,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       for (int k = 0; k < RC; ++k) {
         const int c = col0 + k;
         bool valid = mine && c >= ch.row_lo && c < ch.row_hi && r < ch.ntok;
-        if constexpr (kMode == kMulti) valid = valid && t <= ch.len - p.q_len + ch.pos0 + c / G;  // causal
+        if constexpr (kMode == kMulti) valid = valid && t <= ch.len - p.q_len + c / G;  // causal
+        if constexpr (kMode == kMultiTiled) valid = valid && t <= ch.len - p.q_len + ch.pos0 + c / G;
         sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
         over |= sc[k] > m_ref[k] + kRescaleGap;
       }
@@ -1500,7 +1526,7 @@ template <bool kBf16, int G, int RG, int kMode, int B>
 cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   const unsigned long long q_rows =
-      static_cast<unsigned long long>(prm.num_seqs) * (kMode == kMulti ? prm.q_len : 1);
+      static_cast<unsigned long long>(prm.num_seqs) * (is_multi(kMode) ? prm.q_len : 1);
   const unsigned long long kv_rows = static_cast<unsigned long long>(prm.num_blocks) * prm.num_kv_heads * B;
   if (kv_rows >= (1ull << 31) || q_rows >= (1ull << 31)) return cudaErrorInvalidValue;
   LaunchMaps want{};

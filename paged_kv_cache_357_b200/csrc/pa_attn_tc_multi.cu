@@ -11,9 +11,9 @@ namespace pa {
 namespace tc {
 
 template <bool kBf16>
-static bool pick_multi(int G, int RG, Variant& v) {
+static bool pick_multi(int G, int RG, bool tiled, Variant& v) {
 #define PA_MULTI_CASE(g, rg)                         \
-  if (G == g && RG == rg) {                          \
+  if (G == g && RG == rg && !tiled) {                \
     v = tc_variant<kBf16, g, rg, kMulti>();          \
     return true;                                     \
   }
@@ -22,6 +22,14 @@ static bool pick_multi(int G, int RG, Variant& v) {
   PA_MULTI_CASE(4, 2) PA_MULTI_CASE(4, 4) PA_MULTI_CASE(4, 8)
   PA_MULTI_CASE(8, 2) PA_MULTI_CASE(8, 4)
 #undef PA_MULTI_CASE
+  // row tiles: 32 rows a unit
+#define PA_TILED_CASE(g, rg)                         \
+  if (G == g && RG == rg && tiled) {                 \
+    v = tc_variant<kBf16, g, rg, kMultiTiled>();     \
+    return true;                                     \
+  }
+  PA_TILED_CASE(1, 32) PA_TILED_CASE(2, 16) PA_TILED_CASE(4, 8) PA_TILED_CASE(8, 4)
+#undef PA_TILED_CASE
   return false;
 }
 
@@ -32,7 +40,9 @@ bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Var
   const int rg = tc::row_groups_for(group, q_len);
   if (rg == 0) return false;
   tiles = tc::row_tiles_for(q_len, rg);
-  return pool.dtype == PA_BF16 ? tc::pick_multi<true>(group, rg, v) : tc::pick_multi<false>(group, rg, v);
+  const bool tiled = tiles > 1;
+  return pool.dtype == PA_BF16 ? tc::pick_multi<true>(group, rg, tiled, v)
+                               : tc::pick_multi<false>(group, rg, tiled, v);
 }
 
 }  // namespace pa

@@ -132,3 +132,42 @@ def test_shared_prefix_steps_match_oracle(cuda_device):
     for i in range(nsteps):
         ref = oracle.decode(qs[i], k_ref, v_ref, L.block_tables, L.seq_lens, L.scale, L.num_kv_heads, L.dtype)
         assert_attention_close(results[i].double().numpy(), ref, f"shared-prefix step {i}")
+
+
+def test_staged_steps_upload_one_packed_block(cuda_device):
+    """Inputs built in the step's pinned staging views go up as one copy of
+    the used part of the packed block; results match the oracle step by
+    step, and the uploaded byte count is that part's size."""
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    L = random_layout(58, [3, 16, 17, 200, 900, 45, 1], dtype="bf16", block_size=16, num_q_heads=8,
+                      num_kv_heads=2, head_dim=128, write_new_token=True)
+    V = fill_values_numpy(L)
+    rng = np.random.default_rng(12)
+    kp = bits_to_torch(V.k_pool, L.dtype).to(cuda_device)
+    vp = bits_to_torch(V.v_pool, L.dtype).to(cuda_device)
+    step = pa.PagedDecodeStep(kp, vp, L.num_seqs, L.num_q_heads, L.max_blocks_per_seq,
+                              max_new_tokens=L.num_new_tokens, scale=L.scale)
+    k_ref, v_ref = V.k_pool, V.v_pool
+    for i in range(5):
+        q = f32_to_bits(rng.standard_normal(V.q.shape, dtype=np.float32), L.dtype)
+        nk = f32_to_bits(rng.standard_normal(V.new_k.shape, dtype=np.float32), L.dtype)
+        nv = f32_to_bits(rng.standard_normal(V.new_v.shape, dtype=np.float32), L.dtype)
+        s = step.staging()
+        s["q"].copy_(bits_to_torch(q, L.dtype))
+        s["block_tables"].copy_(torch.from_numpy(L.block_tables))
+        s["seq_lens"].copy_(torch.from_numpy(L.seq_lens))
+        s["new_k"].copy_(bits_to_torch(nk, L.dtype))
+        s["new_v"].copy_(bits_to_torch(nv, L.dtype))
+        s["slot_mapping"].copy_(torch.from_numpy(L.slot_mapping))
+        out = step.run(s["q"], s["block_tables"], s["seq_lens"], s["new_k"], s["new_v"], s["slot_mapping"])
+        step.wait(out)
+        assert step.last_h2d_bytes == step.layout.slot_mapping + 8 * L.num_new_tokens
+        k_ref, v_ref = oracle.cache_write(k_ref, v_ref, nk, nv, L.slot_mapping)
+        ref = oracle.decode(q, k_ref, v_ref, L.block_tables, L.seq_lens, L.scale, L.num_kv_heads, L.dtype)
+        assert_attention_close(out.double().numpy(), ref, f"staged step {i}")
+    assert step.device_status() == 0
+    assert np.array_equal(torch_bits(kp), k_ref) and np.array_equal(torch_bits(vp), v_ref)
+    step.close()

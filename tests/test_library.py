@@ -172,3 +172,47 @@ def test_python_binding_checks_tensors_before_calling():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="no fallback"):
         _lib.load(str(tmp_path / "libpa.so"))
+
+
+def _step_shape(kind=0, S=4, Hq=8, max_nb=5, q_len=1, max_group=0, T=4, P=2):
+    return _lib.StepShape(kind, S, Hq, max_nb, q_len, max_group, T, P, 0.125, _lib.DecodeOpts(0, 0))
+
+
+def test_step_layout_packs_the_fields_in_order(lib):
+    """pa_step_layout_of: every field 256-byte aligned, in the documented
+    order, each as large as its shape needs; the output is q's size."""
+    d = _desc(head_dim=128)
+    for kind, q_len, max_group in ((0, 1, 0), (1, 4, 0), (2, 1, 3)):
+        sh = _step_shape(kind=kind, q_len=q_len, max_group=max_group)
+        L = _lib.StepLayout()
+        assert lib.pa_step_layout_of(ctypes.byref(sh), ctypes.byref(d), ctypes.byref(L)) == 0
+        offs = [getattr(L, f) for f in _lib.STEP_FIELDS] + [L.total]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        S, Hq, D, Hkv = sh.num_seqs, sh.num_q_heads, d.head_dim, d.num_kv_heads
+        q_bytes = S * q_len * Hq * D * 2
+        assert L.out_bytes == q_bytes and L.block_tables - L.q >= q_bytes
+        assert L.seq_lens - L.block_tables >= S * sh.max_blocks_per_seq * 4
+        assert L.new_v - L.new_k >= sh.max_new_tokens * Hkv * D * 2
+        assert L.total - L.slot_mapping >= sh.max_new_tokens * 8
+        if kind == 2:
+            assert L.group_prefix_blocks - L.group_starts >= (S + 1) * 4
+        else:
+            assert L.group_starts == L.group_prefix_blocks == L.copy_pairs  # unused fields take no room
+
+
+def test_step_rejects_bad_shapes_and_pointers_on_host(lib):
+    d = _desc(head_dim=128)
+    L = _lib.StepLayout()
+    for bad in (_step_shape(S=0), _step_shape(kind=0, q_len=2), _step_shape(kind=1, q_len=1),
+                _step_shape(kind=2, max_group=0), _step_shape(kind=7), _step_shape(T=-1)):
+        assert lib.pa_step_layout_of(ctypes.byref(bad), ctypes.byref(d), ctypes.byref(L)) == 1
+    sh = _step_shape()
+    ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    bad_ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE + 8)  # misaligned
+    h = ctypes.c_void_p()
+    for n, arrays in ((1, (ptrs,) * 4), (9, (ptrs,) * 4), (2, (ptrs, bad_ptrs, ptrs, ptrs))):
+        rc = lib.pa_step_create(ctypes.byref(sh), ctypes.byref(d), FAKE, FAKE, FAKE, 1 << 20, None, n, *arrays,
+                                ctypes.byref(h))
+        assert rc == 1 and not h.value
+    assert lib.pa_step_run(None, 0, 0, 0, None) == 1
+    lib.pa_step_destroy(None)  # a no-op
