@@ -1199,7 +1199,6 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         over |= sc[k] > m_ref[k] + kRescaleGap;
       }
       const bool rescale = named_barrier_or(wg_bar, 128, over);  // uniform per warpgroup
-      float alpha[RC];
       if (rescale) {
         if (mine) {
           float v[RC];
@@ -1222,6 +1221,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
 #pragma unroll
           for (int k = 0; k < RC; ++k) cm[k] = -INFINITY;
         }
+        float alpha[RC];
 #pragma unroll
         for (int k = 0; k < RC; ++k) {
           const float m_old = first ? -INFINITY : m_ref[k];
@@ -1229,6 +1229,13 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           alpha[k] = fast_exp2(m_old - (m_new == -INFINITY ? 0.f : m_new));
           m_ref[k] = m_new;
           l_thr[k] = first ? 0.f : l_thr[k] * alpha[k];
+        }
+        // the rows of O rescaled in place once the previous chunk's PV has
+        // completed (this chunk's PV is issued only after P is released);
+        // done here so that alpha is dead before the exponentials
+        if (!first) {
+          if (!wait_pv(ci)) return false;
+          rescale_o(ob, alpha);
         }
       }
       float pr[RC];
@@ -1286,10 +1293,9 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      // the previous chunk's PV must be complete before O is rescaled and
-      // before this chunk's PV may add to it
+      // the previous chunk's PV must be complete before this chunk's PV may
+      // add to O (and before P's buffer comes round again)
       if (!wait_pv(ci)) return false;
-      if (rescale && !first) rescale_o(ob, alpha);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
