@@ -112,6 +112,10 @@ constexpr int kSoftmaxWarp0 = 4;           // first softmax warp
 // exact enough in 16-bit and in the fp32 sums, and most chunks need neither
 // a cross-warp max nor a rescale.
 constexpr float kRescaleGap = 8.f;
+// Reference max of a row that has seen no score yet: finite, so that
+// score - reference is -inf for a masked score (p = 0) and never NaN, with no
+// per-row test for an empty row; exp2 of it against any real score is 0.
+constexpr float kNoMax = -1e30f;
 
 enum Mode { kDecode = 0, kMulti = 1, kGroup = 2, kMultiTiled = 3 };
 
@@ -1185,16 +1189,24 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[sb]);
 
-      // scores of this token row for every query row (log2 domain), masked
-      const int t = ch.j * B + r;  // token index in the sequence
+      // scores of this token row for every query row (log2 domain), masked.
+      // The rows of this warpgroup that see the chunk, as a bit mask: all of
+      // them unless a group unit's member chunk, and none past the chunk's
+      // valid tokens.
+      uint32_t vis = 0;
+      if (mine && r < ch.ntok) {
+        const int lo = max(ch.row_lo - col0, 0), hi = min(ch.row_hi - col0, RC);
+        vis = hi > lo ? ((hi >= 32 ? 0xffffffffu : (1u << hi) - 1u) & ~((1u << lo) - 1u)) : 0u;
+      }
+      // causal limit: position c / G of the unit sees tokens up to lim + c / G
+      const int lim = kMode == kMultiTiled ? ch.len - p.q_len + ch.pos0 - (ch.j * B + r)
+                                           : ch.len - p.q_len - (ch.j * B + r);
       float sc[RC];
       bool over = first;
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
-        const int c = col0 + k;
-        bool valid = mine && c >= ch.row_lo && c < ch.row_hi && r < ch.ntok;
-        if constexpr (kMode == kMulti) valid = valid && t <= ch.len - p.q_len + c / G;  // causal
-        if constexpr (kMode == kMultiTiled) valid = valid && t <= ch.len - p.q_len + ch.pos0 + c / G;
+        bool valid = ((vis >> k) & 1u) != 0;
+        if constexpr (is_multi(kMode)) valid = valid && lim + (col0 + k) / G >= 0;  // causal
         sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
         over |= sc[k] > m_ref[k] + kRescaleGap;
       }
@@ -1225,8 +1237,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
 #pragma unroll
         for (int k = 0; k < RC; ++k) {
           const float m_old = first ? -INFINITY : m_ref[k];
-          const float m_new = fmaxf(m_old, cm[k]);
-          alpha[k] = fast_exp2(m_old - (m_new == -INFINITY ? 0.f : m_new));
+          const float m_new = fmaxf(fmaxf(m_old, cm[k]), kNoMax);
+          alpha[k] = fast_exp2(m_old - m_new);
           m_ref[k] = m_new;
           l_thr[k] = first ? 0.f : l_thr[k] * alpha[k];
         }
@@ -1241,7 +1253,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       float pr[RC];
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
-        pr[k] = mine ? fast_exp2(sc[k] - (m_ref[k] == -INFINITY ? 0.f : m_ref[k])) : 0.f;
+        pr[k] = fast_exp2(sc[k] - m_ref[k]);  // 0 for a masked score (m_ref is finite)
         l_thr[k] += pr[k];
       }
       // P^T, MN-major: token row r holds at position c the head of query row
@@ -1356,7 +1368,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
 
 #pragma unroll
     for (int k = 0; k < RC; ++k) {
-      m_ref[k] = -INFINITY;
+      m_ref[k] = kNoMax;
       l_thr[k] = 0.f;
     }
     Seg prev;               // the segment whose finish is still due
