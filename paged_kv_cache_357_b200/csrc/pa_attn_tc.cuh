@@ -1201,21 +1201,26 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       // causal limit: position c / G of the unit sees tokens up to lim + c / G
       const int lim = kMode == kMultiTiled ? ch.len - p.q_len + ch.pos0 - (ch.j * B + r)
                                            : ch.len - p.q_len - (ch.j * B + r);
-      float sc[RC];
+      // d = score - reference max, one FFMA a row; the same d decides the
+      // rescale and, when none is needed, feeds the exponential
+      auto row_valid = [&](int k) {
+        bool valid = ((vis >> k) & 1u) != 0;
+        if constexpr (is_multi(kMode)) valid = valid && lim + (col0 + k) / G >= 0;  // causal
+        return valid;
+      };
+      float d[RC];
       bool over = first;
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
-        bool valid = ((vis >> k) & 1u) != 0;
-        if constexpr (is_multi(kMode)) valid = valid && lim + (col0 + k) / G >= 0;  // causal
-        sc[k] = valid ? sN[k] * p.scale_log2 : -INFINITY;
-        over |= sc[k] > m_ref[k] + kRescaleGap;
+        d[k] = row_valid(k) ? fmaf(sN[k], p.scale_log2, -m_ref[k]) : -INFINITY;
+        over |= d[k] > kRescaleGap;
       }
       const bool rescale = named_barrier_or(wg_bar, 128, over);  // uniform per warpgroup
       if (rescale) {
         if (mine) {
           float v[RC];
 #pragma unroll
-          for (int k = 0; k < RC; ++k) v[k] = sc[k];
+          for (int k = 0; k < RC; ++k) v[k] = row_valid(k) ? sN[k] * p.scale_log2 : -INFINITY;  // the scores
           const float wm = warp_column_reduce<RC, true>(v, lane);
           if (col_writer) sm.red[sb][quad][my_col] = wm;
         }
@@ -1239,6 +1244,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           const float m_old = first ? -INFINITY : m_ref[k];
           const float m_new = fmaxf(fmaxf(m_old, cm[k]), kNoMax);
           alpha[k] = fast_exp2(m_old - m_new);
+          d[k] = row_valid(k) ? fmaf(sN[k], p.scale_log2, -m_new) : -INFINITY;  // against the new reference
           m_ref[k] = m_new;
           l_thr[k] = first ? 0.f : l_thr[k] * alpha[k];
         }
@@ -1253,7 +1259,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       float pr[RC];
 #pragma unroll
       for (int k = 0; k < RC; ++k) {
-        pr[k] = fast_exp2(sc[k] - m_ref[k]);  // 0 for a masked score (m_ref is finite)
+        pr[k] = fast_exp2(d[k]);  // 0 for a masked score
         l_thr[k] += pr[k];
       }
       // P^T, MN-major: token row r holds at position c the head of query row
