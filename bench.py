@@ -611,6 +611,7 @@ def run_ours(args):
     e0.record(step.h2d_stream)
     for _ in range(K2):
         e2e_step()
+    step.flush()  # the last step's download, otherwise held back for a next step
     e1.record(step.d2h_stream)
     step.synchronize()
     barrier()

@@ -418,7 +418,9 @@ PA_API pa_status pa_shared_prefix_groups(const int32_t* block_tables, int32_t ma
  * no memory of its own.
  *
  * Per pa_step_run the host issues one copy of the used part of the set's
- * input block, one graph launch and one copy of the output.  Sets are used
+ * input block, one graph launch, and the copy of the previous step's output
+ * (a step's download is held back to its next step, see pa_step_flush).
+ * Sets are used
  * in turn: the upload into a set waits for the kernels that last read it,
  * the kernels of a step wait for its upload, for the previous step's
  * kernels (in-order stream: they share the pools) and for the download
@@ -470,7 +472,15 @@ PA_API pa_status pa_step_next_set(pa_step* step, int32_t* set);
  * groups) from the next set's host input block; *set = the set used. */
 PA_API pa_status pa_step_run(pa_step* step, int32_t num_copy_pairs, int32_t num_new_tokens, int32_t num_groups,
                              int32_t* set);
+/* Block until that set's output is in its host block (its download is
+ * enqueued first if it is still held back, see pa_step_flush). */
 PA_API pa_status pa_step_wait(pa_step* step, int32_t set);
+/* A step's download is enqueued with the next pa_step_run, behind that
+ * step's upload (a download waits for its kernels, and an upload behind it
+ * on the same copy queue would wait with it).  pa_step_flush enqueues the
+ * held-back download now; pa_step_wait and pa_step_synchronize do so
+ * themselves. */
+PA_API pa_status pa_step_flush(pa_step* step);
 PA_API pa_status pa_step_synchronize(pa_step* step);
 /* The upload, kernel and download streams (cudaStream_t as void*). */
 PA_API pa_status pa_step_streams(pa_step* step, void** upload, void** kernels, void** download);

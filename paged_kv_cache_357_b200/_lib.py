@@ -58,6 +58,7 @@ EXPORTED = (
     "pa_step_next_set",
     "pa_step_run",
     "pa_step_wait",
+    "pa_step_flush",
     "pa_step_synchronize",
     "pa_step_streams",
     "pa_step_destroy",
@@ -164,6 +165,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_step_run.restype = i32
     lib.pa_step_wait.argtypes = [vp, i32]
     lib.pa_step_wait.restype = i32
+    lib.pa_step_flush.argtypes = [vp]
+    lib.pa_step_flush.restype = i32
     lib.pa_step_synchronize.argtypes = [vp]
     lib.pa_step_synchronize.restype = i32
     lib.pa_step_streams.argtypes = [vp, vpp, vpp, vpp]

@@ -99,6 +99,24 @@ struct pa_step {
   Graph graphs[PA_STEP_MAX_SETS][kMaxGraphsPerSet] = {};
   int num_graphs[PA_STEP_MAX_SETS] = {};
   long long steps = 0;
+  int pending = -1;  // the set whose download is still to be enqueued
+
+  // Enqueue the download of the pending set.  A step's download is issued
+  // with the next step (after that step's upload): a download first waits
+  // for its kernels, and an upload queued behind it on the same copy queue
+  // would wait too, putting upload, kernels and download of neighbouring
+  // steps in series.
+  pa_status flush() {
+    if (pending < 0) return PA_OK;
+    const int k = pending;
+    pending = -1;
+    if (cudaStreamWaitEvent(download, computed[k], 0) != cudaSuccess ||
+        cudaMemcpyAsync(hout[k], dout[k], layout.out_bytes, cudaMemcpyDeviceToHost, download) != cudaSuccess ||
+        cudaEventRecord(downloaded[k], download) != cudaSuccess) {
+      return PA_ERR_CUDA;
+    }
+    return PA_OK;
+  }
 
   // The step's kernels on `stream` with set k's buffers (checked by the
   // entry points themselves).
@@ -183,6 +201,7 @@ struct pa_step {
   }
 
   void release() {
+    if (download != nullptr) flush();
     if (upload != nullptr) cudaStreamSynchronize(upload);
     if (kernels != nullptr) cudaStreamSynchronize(kernels);
     if (download != nullptr) cudaStreamSynchronize(download);
@@ -299,27 +318,35 @@ extern "C" pa_status pa_step_run(pa_step* step, int32_t num_copy_pairs, int32_t 
   }
   if (st != PA_OK) return st;
   if (cudaEventRecord(step->computed[k], step->kernels) != cudaSuccess) return PA_ERR_CUDA;
-  // download
-  if (cudaStreamWaitEvent(step->download, step->computed[k], 0) != cudaSuccess ||
-      cudaMemcpyAsync(step->hout[k], step->dout[k], step->layout.out_bytes, cudaMemcpyDeviceToHost,
-                      step->download) != cudaSuccess ||
-      cudaEventRecord(step->downloaded[k], step->download) != cudaSuccess) {
-    return PA_ERR_CUDA;
-  }
+  // the previous step's download now (behind this step's upload); this
+  // step's with the next one, or when its result is waited for
+  st = step->flush();
+  if (st != PA_OK) return st;
+  step->pending = k;
   step->used[k] = true;
   ++step->steps;
   if (set != nullptr) *set = k;
   return PA_OK;
 }
 
+extern "C" pa_status pa_step_flush(pa_step* step) {
+  if (step == nullptr) return PA_ERR_INVALID_ARG;
+  return step->flush();
+}
+
 extern "C" pa_status pa_step_wait(pa_step* step, int32_t set) {
   if (step == nullptr || set < 0 || set >= step->num_sets) return PA_ERR_INVALID_ARG;
   if (!step->used[set]) return PA_OK;
+  if (step->pending == set) {
+    const pa_status st = step->flush();
+    if (st != PA_OK) return st;
+  }
   return cudaEventSynchronize(step->downloaded[set]) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" pa_status pa_step_synchronize(pa_step* step) {
   if (step == nullptr) return PA_ERR_INVALID_ARG;
+  if (step->flush() != PA_OK) return PA_ERR_CUDA;
   const bool ok = cudaStreamSynchronize(step->upload) == cudaSuccess &&
                   cudaStreamSynchronize(step->kernels) == cudaSuccess &&
                   cudaStreamSynchronize(step->download) == cudaSuccess;

@@ -187,6 +187,11 @@ class PagedDecodeStep:
                 return
         raise ValueError("not a result of this PagedDecodeStep")
 
+    def flush(self) -> None:
+        """Enqueue the download of the last step now (it is otherwise issued
+        with the next step, behind that step's upload)."""
+        _check(self._c.pa_step_flush(self._h), "pa_step_flush")
+
     def synchronize(self) -> None:
         _check(self._c.pa_step_synchronize(self._h), "pa_step_synchronize")
 
