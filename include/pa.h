@@ -210,7 +210,7 @@ PA_API pa_status pa_decode_no_alloc(const void* q, const void* k_pool, const voi
  *   q, out   [num_seqs][q_len][num_q_heads][head_dim]
  *   others   as pa_decode
  * q_len == 1 is pa_decode.  For q_len >= 2 the tensor-core kernel runs:
- * head_dim 128, block_size 16, group size G = num_q_heads / num_kv_heads in
+ * head_dim 128, block_size 8, 16 or 32, group size G = num_q_heads / num_kv_heads in
  * {1, 2, 4, 8}, any q_len.  One unit of work carries up to 32 query rows
  * (G heads times a power-of-two count of positions); when G * q_len is
  * larger (a prefill chunk), each sequence is split into row tiles of 32 / G
@@ -414,8 +414,11 @@ PA_API pa_status pa_shared_prefix_groups(const int32_t* block_tables, int32_t ma
  * slot_mapping; the same layouts as the entry points take, each field at
  * its maximum size).  The step creates three CUDA streams (uploads,
  * kernels, downloads), events and, per buffer set and counts, one CUDA
- * graph of its kernels (the first step runs them directly); it allocates
- * no memory of its own.
+ * graph of its kernels (the first step runs them directly; up to four
+ * graphs a set are kept, the oldest replaced).  It makes no allocation of
+ * its own (no cudaMalloc or host allocation); the driver keeps what the
+ * streams, events and graphs need until pa_step_destroy.  A step object is
+ * used from one host thread at a time.
  *
  * Per pa_step_run the host issues one copy of the used part of the set's
  * input block, one graph launch, and the copy of the previous step's output

@@ -1617,5 +1617,29 @@ inline int row_groups_for(int G, int q_len) {
 // Row tiles (units) per sequence for q_len positions at rg row groups a unit.
 inline int row_tiles_for(int q_len, int rg) { return rg > 0 ? (q_len + rg - 1) / rg : 0; }
 
+// The multi-query instances at blocks of B tokens: one unit per sequence for
+// G x RG <= 32 rows (RG a power of two), row tiles of 32 rows beyond.
+template <bool kBf16, int B>
+bool pick_multi(int G, int RG, bool tiled, Variant& v) {
+#define PA_MULTI_CASE(g, rg)                         \
+  if (G == g && RG == rg && !tiled) {                \
+    v = tc_variant<kBf16, g, rg, kMulti, B>();       \
+    return true;                                     \
+  }
+  PA_MULTI_CASE(1, 2) PA_MULTI_CASE(1, 4) PA_MULTI_CASE(1, 8) PA_MULTI_CASE(1, 16) PA_MULTI_CASE(1, 32)
+  PA_MULTI_CASE(2, 2) PA_MULTI_CASE(2, 4) PA_MULTI_CASE(2, 8) PA_MULTI_CASE(2, 16)
+  PA_MULTI_CASE(4, 2) PA_MULTI_CASE(4, 4) PA_MULTI_CASE(4, 8)
+  PA_MULTI_CASE(8, 2) PA_MULTI_CASE(8, 4)
+#undef PA_MULTI_CASE
+#define PA_TILED_CASE(g, rg)                         \
+  if (G == g && RG == rg && tiled) {                 \
+    v = tc_variant<kBf16, g, rg, kMultiTiled, B>();  \
+    return true;                                     \
+  }
+  PA_TILED_CASE(1, 32) PA_TILED_CASE(2, 16) PA_TILED_CASE(4, 8) PA_TILED_CASE(8, 4)
+#undef PA_TILED_CASE
+  return false;
+}
+
 }  // namespace tc
 }  // namespace pa

@@ -32,6 +32,11 @@ bool select_tc_decode_other_block(int block_size, bool bf16, int group, Variant&
 // Multi-query decode with q_len >= 2 positions (pa_attn_tc_multi.cu); tiles
 // = units (row tiles) per sequence.
 bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v, int& tiles);
+// Its instances at blocks of 8 and 32 tokens (pa_attn_tc_multi_b8.cu,
+// pa_attn_tc_multi_b32.cu): rg row groups a unit, tiled = several units a
+// sequence.
+bool select_tc_multi_b8(bool bf16, int group, int rg, bool tiled, Variant& v);
+bool select_tc_multi_b32(bool bf16, int group, int rg, bool tiled, Variant& v);
 // Shared-prefix decode over groups of up to max_members sequences
 // (pa_attn_tc_group.cu).
 bool select_tc_group_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);

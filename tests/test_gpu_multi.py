@@ -14,12 +14,13 @@ from workloads import bits_to_torch, config_llama3_8b, f32_to_bits, fill_values_
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(seed, lens, G, L, dtype, Hkv=2, block_size=16):
+def _inputs(seed, lens, G, L, dtype, Hkv=2, block_size=16, head_dim=128):
     layout = random_layout(seed, lens, dtype=dtype, block_size=block_size, num_q_heads=Hkv * G, num_kv_heads=Hkv,
-                           head_dim=128, write_new_token=False)
+                           head_dim=head_dim, write_new_token=False)
     vals = fill_values_numpy(layout)
     rng = np.random.default_rng([seed, 99])
-    q = f32_to_bits(rng.standard_normal((layout.num_seqs, L, layout.num_q_heads, 128), dtype=np.float32), dtype)
+    q = f32_to_bits(rng.standard_normal((layout.num_seqs, L, layout.num_q_heads, head_dim), dtype=np.float32),
+                    dtype)
     return layout, vals, q
 
 
@@ -78,6 +79,21 @@ def test_multi_row_tiles(cuda_device, G, L):
     assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"G={G} q_len={L} {dtype}")
 
 
+BLOCK_CASES = [(B, G, L) for B in (8, 32) for G, L in ((1, 3), (4, 4), (8, 4), (4, 64))]
+
+
+@pytest.mark.parametrize("B,G,L", BLOCK_CASES, ids=[f"B{b}-G{g}-L{l}" for b, g, l in BLOCK_CASES])
+def test_multi_block_sizes(cuda_device, B, G, L):
+    """Multi-query at blocks of 8 and 32 tokens: a chunk is still 128 tokens
+    (16 or 4 blocks); one unit per sequence up to 32 rows, row tiles beyond."""
+    dtype = "bf16" if (B + L) % 2 == 0 else "fp16"
+    lens = [n for n in (L, L + 1, B - 1, B, B + 1, 129, 300, 1000) if n >= L]
+    layout, vals, q = _inputs(7700 + 10 * B + 3 * G + L, lens, G, L, dtype, block_size=B)
+    out, st = _run(cuda_device, layout, vals, q)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"B={B} G={G} q_len={L} {dtype}")
+
+
 @pytest.mark.parametrize("num_ctas", [1, 5, 0])
 def test_multi_row_tiles_split_units(cuda_device, num_ctas):
     G, L = 4, 64
@@ -133,8 +149,8 @@ def test_unsupported_shapes_are_refused(cuda_device):
 
     import paged_kv_cache_357_b200 as pa
 
-    # multi-query runs at block size 16 only
-    layout, vals, q = _inputs(7400, [64, 80], 8, 8, "bf16", block_size=8)
+    # multi-query runs on the tensor-core kernel only: head_dim 128
+    layout, vals, q = _inputs(7400, [64, 80], 8, 8, "bf16", head_dim=64)
     kp = bits_to_torch(vals.k_pool, "bf16").to(cuda_device)
     with pytest.raises(pa.PaError) as e:
         pa.multi_workspace_bytes(2, 8, layout.num_q_heads, kp)

@@ -171,3 +171,38 @@ def test_staged_steps_upload_one_packed_block(cuda_device):
     assert step.device_status() == 0
     assert np.array_equal(torch_bits(kp), k_ref) and np.array_equal(torch_bits(vp), v_ref)
     step.close()
+
+
+def test_executor_reports_device_errors_and_recovers(cuda_device):
+    """A step whose slot mapping points past the pool: the cache write skips
+    the token and records PA_DEV_BAD_SLOT (103) in the device status, nothing
+    traps, and the next good step on the same executor matches the oracle."""
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    L = random_layout(59, [5, 40, 300], dtype="bf16", block_size=16, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                      write_new_token=True)
+    V = fill_values_numpy(L)
+    kp = bits_to_torch(V.k_pool, L.dtype).to(cuda_device)
+    vp = bits_to_torch(V.v_pool, L.dtype).to(cuda_device)
+    step = pa.PagedDecodeStep(kp, vp, L.num_seqs, L.num_q_heads, L.max_blocks_per_seq,
+                              max_new_tokens=L.num_new_tokens, scale=L.scale)
+    q = bits_to_torch(V.q, L.dtype)
+    nk, nv = bits_to_torch(V.new_k, L.dtype), bits_to_torch(V.new_v, L.dtype)
+    tables, lens = torch.from_numpy(L.block_tables), torch.from_numpy(L.seq_lens)
+    bad = torch.from_numpy(L.slot_mapping.copy())
+    bad[1] = L.num_blocks * L.block_size + 5  # past the pool
+    out = step.run(q, tables, lens, nk, nv, bad)
+    step.wait(out)
+    assert step.device_status() == 103
+    step.status.zero_()
+    torch.cuda.synchronize()  # the reset is on torch's stream, the step's kernels on the executor's
+    out = step.run(q, tables, lens, nk, nv, torch.from_numpy(L.slot_mapping))
+    step.wait(out)
+    assert step.device_status() == 0
+    # the bad step wrote tokens 0 and 2 only; the good step wrote all three
+    k_ref, v_ref = oracle.cache_write(V.k_pool, V.v_pool, V.new_k, V.new_v, L.slot_mapping)
+    ref = oracle.decode(V.q, k_ref, v_ref, L.block_tables, L.seq_lens, L.scale, L.num_kv_heads, L.dtype)
+    assert_attention_close(out.double().numpy(), ref, "after the bad step")
+    step.close()
