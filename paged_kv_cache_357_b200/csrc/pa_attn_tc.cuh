@@ -24,8 +24,10 @@
 //            shared blocks once, seen by every member's rows, then each
 //            member's own blocks, seen by that member's rows only.
 //
-// Work partition and split-unit merge: pa_decode_common.cuh (ranges of equal
-// cost, 8-block chunks plus a fixed finish cost per unit, per CTA).
+// Work partition: pa_decode_common.cuh (ranges of equal cost, 8-block chunks
+// plus a fixed finish cost per unit, per CTA).  A unit split between CTAs is
+// merged by the CTA that holds its first piece (see the split-unit helpers
+// below).
 //
 // Roles (128 + 128 x WG threads, one CTA per SM):
 //   warp 0      K producer: resolves block ids (32 table entries per load,
@@ -101,7 +103,6 @@ struct Blk {
   // V stage offset of token t of the chunk (its row in the first half)
   __host__ __device__ static constexpr int v_offset(int t) { return (t / BB) * kVBlockBytes + (t % BB) * kRowBytes; }
 };
-constexpr int kSoftmaxBarrier = 1;          // all softmax warps
 constexpr int kWarpgroupBarrier0 = 2;       // + warpgroup index: one softmax warpgroup
 constexpr int kQKWarp = 1;                 // allocates TMEM, issues QK
 constexpr int kVWarp = 2;                  // the V producer (warp 0 loads q and K)
@@ -176,8 +177,11 @@ struct TcSmem {
   uint8_t q[2][S::kQSlotBytes];
   uint8_t p[2][S::kPSlotBytes];
   alignas(16) float red[2][4][R];  // per-warp column maxima, double-buffered by chunk
-  alignas(16) float mfin[R];       // reference max of each row of the segment being finished
-  alignas(16) float lred[4][R];    // per-warp row sums of the segment being finished
+  // the reference max and per-warp row sums of a segment being finished,
+  // by the parity of its O buffer (a segment's stash is read while the
+  // next segment's may be written)
+  alignas(16) float mfin[2][R];
+  alignas(16) float lred[2][4][R];
   uint64_t kfull[kKStages];
   uint64_t kempty[kKStages];
   uint64_t vfull[S::kVStages];
@@ -193,7 +197,7 @@ struct TcSmem {
   RangeSmem range;
   uint32_t tmem_base;
   int abort;
-  int is_last;
+  int merge_ok[2];                 // per softmax warpgroup: every other piece of the unit arrived
   int k_issued;
   int k_consumed;
   int v_issued;
@@ -686,15 +690,13 @@ __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>&
 // ---- unit results --------------------------------------------------------------
 
 // Rows col0 .. col0 + RC - 1 of the unit in segment sg (those below `rows`),
-// head_dim element d, from their states (m, L, unnormalised a): the
-// normalised outputs.  A row that saw no token (a group member of length 0)
-// gets zeros.
+// head_dim element d, from their sums L and unnormalised outputs a: the
+// normalised outputs.  s0 is a group unit's first sequence.  A row that saw
+// no token (a group member of length 0) gets zeros.
 template <bool kBf16, int G, int RG, int RC, int kMode>
-__device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, int col0, int rows, int d,
-                                          const float (&m)[RC], const float (&L)[RC], const float (&a)[RC]) {
-  (void)m;
+__device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, int s0, int col0, int rows, int d,
+                                          const float (&L)[RC], const float (&a)[RC]) {
   const int Hq = p.num_q_heads;
-  const int s0 = kMode == kGroup ? __ldg(p.group_starts + sg.s) : 0;
 #pragma unroll
   for (int k = 0; k < RC; ++k) {
     const int c = col0 + k;
@@ -717,55 +719,38 @@ __device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, 
   }
 }
 
-// Called by every softmax thread after this CTA's partial state of a split
-// unit is written and fenced.  The last CTA to arrive merges every partial
-// state of the unit (the rescale rule of the online softmax, per row and
-// head_dim element) and emits the rows: thread (d, col0) takes element d of
-// rows col0 .. col0 + RC - 1.  Every row is merged at once, so each pass over
-// the partial states costs one memory round trip per CTA piece.
-template <bool kBf16, int G, int R, int RC, int kMode, typename Sync>
-__device__ void finish_split_unit_rows(const DecodeParams& p, const Seg& sg, const WorkRange& wr, int rows,
-                                       int ctid, int d, int col0, int* is_last, Sync sync) {
-  constexpr int kStride = Rows<R>::kPartStride;
-  const long long F = sg.unit_first;
-  const long long first = cta_of(F, wr.total, wr.nparts);
-  const long long last = cta_of(sg.unit_last, wr.total, wr.nparts);
-  int32_t* counter = p.counters + static_cast<size_t>(sg.s) * p.num_kv_heads + sg.h;
-  sync();
-  if (ctid == 0) {
-    const int prev = atomicAdd(counter, 1);
-    *is_last = (prev == static_cast<int>(last - first));
+// Split units (study notes ch.05 §4: the online-softmax merge applied to
+// the pieces of a partition).  A unit cut between CTAs is merged by the CTA
+// that holds its first piece: the piece ends that CTA's range, so it is the
+// last thing the CTA does, while the unit's last piece opens the range of
+// the CTA after it and is long finished by then.  Every other piece
+// publishes its partial state (m, l, acc per row) and counts itself in the
+// unit's arrival counter, one 16-bit half per softmax warpgroup (each
+// warpgroup publishes and merges its own rows); the merger waits for the
+// count, merges from its own registers and the published states, and
+// clears its half.  A CTA only waits for CTAs after it whose pieces of the
+// unit open or fill their ranges, so no wait can close a cycle.
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const int32_t* ptr) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+// Spin (bounded by limit_ns) until bits [shift, shift + 16) of *counter
+// reach `need`.
+__device__ __forceinline__ bool wait_arrivals(const int32_t* counter, int shift, uint32_t need,
+                                              unsigned long long limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (((ld_acquire_gpu(counter) >> shift) & 0xffffu) < need) {
+    if (global_timer_ns() - t0 > limit_ns) return false;
+    __nanosleep(32);
   }
-  sync();
-  if (*is_last) {
-    __threadfence();
-    float M[RC], L[RC], a[RC];
-#pragma unroll
-    for (int k = 0; k < RC; ++k) {
-      M[k] = -INFINITY;
-      L[k] = 0.f;
-      a[k] = 0.f;
-    }
-    for (long long cc = first; cc <= last; ++cc) {
-      const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
-#pragma unroll
-      for (int k = 0; k < RC; ++k) M[k] = fmaxf(M[k], __ldcg(pp + col0 + k));
-    }
-    for (long long cc = first; cc <= last; ++cc) {
-      const float* pp = p.partials + partial_slot(cc, F, wr) * kStride;
-#pragma unroll
-      for (int k = 0; k < RC; ++k) {
-        const int c = col0 + k;
-        if (c < rows) {
-          const float w = fast_exp2(__ldcg(pp + c) - M[k]);
-          L[k] = fmaf(__ldcg(pp + R + c), w, L[k]);
-          a[k] = fmaf(__ldcg(pp + 2 * R + c * D + d), w, a[k]);
-        }
-      }
-    }
-    emit_rows<kBf16, G, R / G, RC, kMode>(p, sg, col0, rows, d, M, L, a);
-    if (ctid == 0) *counter = 0;
-  }
+  return true;
+}
+
+__device__ __forceinline__ int32_t* unit_counter(const DecodeParams& p, const Seg& sg) {
+  return p.counters + static_cast<size_t>(sg.s) * p.num_kv_heads + sg.h;
 }
 
 // ---- the kernel ---------------------------------------------------------------
@@ -1320,56 +1305,104 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       return true;
     };
 
-    // A segment's row sums and reference maxima, put aside before the next
-    // segment's first softmax resets them: sums reduced over the warp into
-    // lred, maxima into mfin (both read by finish_segment after a barrier).
-    auto stash_segment = [&]() {
+    // A segment's row sums and reference maxima, put aside (in stash buffer
+    // sb, the parity of its O buffer) before the next segment's first
+    // softmax resets them: sums reduced over the warp into lred, maxima into
+    // mfin.  The warpgroup barrier of the next chunk's softmax orders them
+    // before finish_segment reads them.
+    auto stash_segment = [&](int sb) {
       float v[RC];
 #pragma unroll
       for (int k = 0; k < RC; ++k) v[k] = l_thr[k];
       const float ls = warp_column_reduce<RC, false>(v, lane);
-      if (col_writer) sm.lred[quad][my_col] = ls;
+      if (col_writer) sm.lred[sb][quad][my_col] = ls;
       if (quad == 0 && lane < RC) {
         float m = m_ref[0];
 #pragma unroll
         for (int k = 1; k < RC; ++k) m = lane == k ? m_ref[k] : m;
-        sm.mfin[col0 + lane] = m;
+        sm.mfin[sb][col0 + lane] = m;
       }
     };
 
-    // The finish of a segment whose PVs have all completed: its rows, or its
-    // partial state and the merge when it arrives last.  Its O buffer is
-    // read once and handed back to the PV issuer.
-    auto finish_segment = [&](const Seg& fs, int rows, int ob) {
+    // The finish of a segment whose PVs have all completed, by each
+    // warpgroup for its own rows: the outputs of a whole unit; for a split
+    // unit, its partial state published, or (its first piece) the merge of
+    // every piece.  Its O buffer ob is read once and handed back to the PV
+    // issuer.  s0 is a group unit's first sequence.
+    auto finish_segment = [&](const Seg& fs, int rows, int ob, int s0) {
       float acc[RC];
       load_o(ob, acc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[ob]);
-      named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
-      if (fs.j0 == fs.first && fs.j0 + fs.n == fs.nb) {
-        float m[RC], L[RC];
-        ld_row<RC>(sm.mfin + col0, m);
+      float L[RC];
 #pragma unroll
-        for (int k = 0; k < RC; ++k) {
-          const int c = col0 + k;
-          L[k] = (sm.lred[0][c] + sm.lred[1][c]) + (sm.lred[2][c] + sm.lred[3][c]);
-        }
-        emit_rows<kBf16, G, RG, RC, kMode>(p, fs, col0, rows, r, m, L, acc);
-      } else {
+      for (int k = 0; k < RC; ++k) {
+        const int c = col0 + k;
+        L[k] = (sm.lred[ob][0][c] + sm.lred[ob][1][c]) + (sm.lred[ob][2][c] + sm.lred[ob][3][c]);
+      }
+      const bool opens = fs.j0 == fs.first, closes = fs.j0 + fs.n == fs.nb;
+      if (opens && closes) {
+        emit_rows<kBf16, G, RG, RC, kMode>(p, fs, s0, col0, rows, r, L, acc);
+        return;
+      }
+      int32_t* counter = unit_counter(p, fs);
+      const int shift = 16 * wg;
+      const bool leader = quad == 0 && lane == 0;
+      if (!opens) {
+        // publish: m, l of this warpgroup's rows, then acc; one arrival
         float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * Sh::kPartStride;
-        if (ctid < R) {
-          pp[ctid] = sm.mfin[ctid];
-          pp[R + ctid] = (sm.lred[0][ctid] + sm.lred[1][ctid]) + (sm.lred[2][ctid] + sm.lred[3][ctid]);
+        if (quad == 0 && lane < RC) {
+          pp[col0 + lane] = sm.mfin[ob][col0 + lane];
+          pp[R + col0 + lane] = (sm.lred[ob][0][col0 + lane] + sm.lred[ob][1][col0 + lane]) +
+                                (sm.lred[ob][2][col0 + lane] + sm.lred[ob][3][col0 + lane]);
         }
 #pragma unroll
         for (int k = 0; k < RC; ++k) pp[2 * R + (col0 + k) * D + r] = acc[k];
-        __threadfence();
-        finish_split_unit_rows<kBf16, G, R, RC, kMode>(
-            p, fs, wr, rows, ctid, r, col0, &sm.is_last,
-            [] { named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads); });
+        named_barrier_sync(wg_bar, 128);
+        if (leader) {
+          __threadfence();
+          atomicAdd(reinterpret_cast<unsigned int*>(counter), 1u << shift);
+        }
+        return;
       }
-      named_barrier_sync(kSoftmaxBarrier, kSoftmaxThreads);
+      // merge: this CTA holds the unit's first piece; pieces first + 1 ..
+      // last were published by the CTAs after it
+      const long long first = cta;
+      const long long last = cta_of(fs.unit_last, wr.total, wr.nparts);
+      const uint32_t need = static_cast<uint32_t>(last - first);
+      if (leader) {
+        const bool got = wait_arrivals(counter, shift, need, p.wait_limit_ns);
+        if (got) {
+          atomicSub(reinterpret_cast<unsigned int*>(counter), need << shift);  // back to zero for the next launch
+        } else {
+          record_status(p.status, PA_DEV_TIMEOUT);
+        }
+        sm.merge_ok[wg] = got;
+      }
+      named_barrier_sync(wg_bar, 128);
+      if (!sm.merge_ok[wg]) return;
+      float M[RC];
+      ld_row<RC>(sm.mfin[ob] + col0, M);
+      for (long long cc = first + 1; cc <= last; ++cc) {
+        const float* pp = p.partials + partial_slot(cc, fs.unit_first, wr) * Sh::kPartStride;
+        float mp[RC], lp[RC], ap[RC];
+#pragma unroll
+        for (int k = 0; k < RC; ++k) {
+          mp[k] = __ldcg(pp + col0 + k);
+          lp[k] = __ldcg(pp + R + col0 + k);
+          ap[k] = __ldcg(pp + 2 * R + (col0 + k) * D + r);
+        }
+#pragma unroll
+        for (int k = 0; k < RC; ++k) {
+          const float mn = fmaxf(M[k], mp[k]);
+          const float wa = fast_exp2(M[k] - mn), wb = fast_exp2(mp[k] - mn);
+          L[k] = fmaf(L[k], wa, lp[k] * wb);
+          acc[k] = fmaf(acc[k], wa, ap[k] * wb);
+          M[k] = mn;
+        }
+      }
+      emit_rows<kBf16, G, RG, RC, kMode>(p, fs, s0, col0, rows, r, L, acc);
     };
 
 #pragma unroll
@@ -1378,7 +1411,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       l_thr[k] = 0.f;
     }
     Seg prev;               // the segment whose finish is still due
-    int prev_rows = 0;
+    int prev_rows = 0, prev_s0 = 0;
     bool have_prev = false;
     while (ok && next_seg<B, CB>(cur, sg, p, src)) {
       const int rows = G * src.row_groups(p, sg.s);
@@ -1386,26 +1419,29 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       walk.start(p, sg, rows);
       const int ob = si & 1;
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
-        if (c0 == 0 && have_prev) stash_segment();
+        if (c0 == 0 && have_prev) stash_segment(ob ^ 1);
         ok = softmax_chunk(ci, walk.next(p), c0 == 0, ob);
         if (!ok) break;
         ++ci;
         if (c0 == 0 && have_prev) {  // every PV of the previous segment is complete
-          finish_segment(prev, prev_rows, ob ^ 1);
+          finish_segment(prev, prev_rows, ob ^ 1, prev_s0);
           have_prev = false;
         }
       }
       if (!ok) break;
       prev = sg;
       prev_rows = rows;
+      if constexpr (kMode == kGroup) prev_s0 = walk.s0;
       have_prev = true;
       ++si;
     }
     if (ok && have_prev) {
       ok = wait_pv(ci);
       if (ok) {
-        stash_segment();
-        finish_segment(prev, prev_rows, (si - 1) & 1);
+        const int ob = (si - 1) & 1;
+        stash_segment(ob);
+        named_barrier_sync(wg_bar, 128);
+        finish_segment(prev, prev_rows, ob, prev_s0);
       }
     }
     if (!ok && lane == 0) {
