@@ -161,9 +161,9 @@ struct Rows {
   static constexpr int kLanesPerCol = 32 / RC;                    // lanes holding one column after a reduce
   // With two softmax warpgroups the control warpgroup hands registers to
   // them (setmaxnreg) inside the launch's allocation of 168 a thread:
-  // 128 x 72 + 256 x 216 = 384 x 168.
-  static constexpr int kCtrlRegs = 72;
-  static constexpr int kSoftmaxRegs = 216;
+  // 128 x 80 + 256 x 208 = 384 x 168 (the producers spill below 80).
+  static constexpr int kCtrlRegs = 80;
+  static constexpr int kSoftmaxRegs = 208;
   static constexpr int kLaunchRegs = 168;
   static_assert(WG == 1 || 128 * kCtrlRegs + kSoftmaxThreads * kSoftmaxRegs <= kThreads * kLaunchRegs,
                 "the register split fits the launch's allocation");
@@ -176,6 +176,9 @@ struct TcSmem {
   uint8_t vbuf[S::kVStages][kOperandBytes];
   uint8_t q[2][S::kQSlotBytes];
   uint8_t p[2][S::kPSlotBytes];
+  // a finished unit's outputs, [row][head_dim] 16-bit, written to global
+  // memory by bulk copies (each warpgroup's rows by its leader)
+  alignas(128) uint8_t ostage[R * D * 2];
   alignas(16) float red[2][4][R];  // per-warp column maxima, double-buffered by chunk
   // the reference max and per-warp row sums of a segment being finished,
   // by the parity of its O buffer (a segment's stash is read while the
@@ -689,34 +692,54 @@ __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>&
 
 // ---- unit results --------------------------------------------------------------
 
-// Rows col0 .. col0 + RC - 1 of the unit in segment sg (those below `rows`),
-// head_dim element d, from their sums L and unnormalised outputs a: the
-// normalised outputs.  s0 is a group unit's first sequence.  A row that saw
-// no token (a group member of length 0) gets zeros.
-template <bool kBf16, int G, int RG, int RC, int kMode>
-__device__ __forceinline__ void emit_rows(const DecodeParams& p, const Seg& sg, int s0, int col0, int rows, int d,
-                                          const float (&L)[RC], const float (&a)[RC]) {
-  const int Hq = p.num_q_heads;
+// The output row (in units of num_q_heads x head_dim) of row group rg of
+// the unit in segment sg; s0 is a group unit's first sequence.
+template <int RG, int kMode>
+__device__ __forceinline__ size_t out_row(const DecodeParams& p, const Seg& sg, int s0, int rg) {
+  if constexpr (kMode == kMultiTiled) {
+    const int s = sg.s / p.q_tiles;
+    return static_cast<size_t>(s) * p.q_len + (sg.s - s * p.q_tiles) * RG + rg;
+  } else if constexpr (kMode == kMulti) {
+    return static_cast<size_t>(sg.s) * p.q_len + rg;
+  } else if constexpr (kMode == kGroup) {
+    return static_cast<size_t>(s0 + rg);
+  } else {
+    return static_cast<size_t>(sg.s);
+  }
+}
+
+// Rows col0 .. col0 + RC - 1 of a unit, head_dim element d, from their sums
+// L and unnormalised outputs a: the normalised outputs into this
+// warpgroup's rows of the staging tile.  A row that saw no token (a group
+// member of length 0) gets zeros.  L >= 1 whenever it is positive (the row
+// max contributes 2^0), so the fast quotient keeps 22 or more bits.
+template <bool kBf16, int RC>
+__device__ __forceinline__ void stage_rows(uint8_t* stage, int col0, int d, const float (&L)[RC],
+                                           const float (&a)[RC]) {
 #pragma unroll
   for (int k = 0; k < RC; ++k) {
-    const int c = col0 + k;
+    const uint32_t two = pack2<kBf16>(L[k] > 0.f ? __fdividef(a[k], L[k]) : 0.f, 0.f);
+    *reinterpret_cast<uint16_t*>(stage + ((col0 + k) * D + d) * 2) = static_cast<uint16_t>(two & 0xffffu);
+  }
+}
+
+// By the warpgroup's leader once its rows are staged (and made visible to
+// the async proxy): one bulk copy per row group of G heads (G x head_dim
+// contiguous outputs), for the row groups below `rows`.
+template <int G, int RG, int RC, int kMode>
+__device__ __forceinline__ void issue_rows(const DecodeParams& p, const Seg& sg, int s0, int col0, int rows,
+                                           const uint8_t* stage) {
+  static_assert(RC % G == 0, "a warpgroup holds whole row groups");
+#pragma unroll
+  for (int j = 0; j < RC / G; ++j) {
+    const int c = col0 + j * G;
     if (c < rows) {
-      const int rg = c / G;
-      size_t row;
-      if constexpr (kMode == kMultiTiled) {
-        const int s = sg.s / p.q_tiles;
-        row = static_cast<size_t>(s) * p.q_len + (sg.s - s * p.q_tiles) * RG + rg;
-      } else if constexpr (kMode == kMulti) {
-        row = static_cast<size_t>(sg.s) * p.q_len + rg;
-      } else if constexpr (kMode == kGroup) {
-        row = static_cast<size_t>(s0 + rg);
-      } else {
-        row = static_cast<size_t>(sg.s);
-      }
-      const uint32_t two = pack2<kBf16>(L[k] > 0.f ? a[k] / L[k] : 0.f, 0.f);
-      p.out[(row * Hq + sg.h * G + c % G) * D + d] = static_cast<uint16_t>(two & 0xffffu);
+      const size_t row = out_row<RG, kMode>(p, sg, s0, c / G);
+      bulk_copy_s2g(p.out + (row * p.num_q_heads + static_cast<size_t>(sg.h) * G) * D, stage + c * D * 2,
+                    G * D * 2);
     }
   }
+  bulk_commit();
 }
 
 // Split units (study notes ch.05 §4: the online-softmax merge applied to
@@ -762,7 +785,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   constexpr int R = G * RG;
   using Sh = Rows<R>;
   constexpr int Nq = Sh::Nq, Np = Sh::Np, kVStages = Sh::kVStages, kLanesPerCol = Sh::kLanesPerCol;
-  constexpr int WG = Sh::WG, RC = Sh::RC, kThreads = Sh::kThreads, kSoftmaxThreads = Sh::kSoftmaxThreads;
+  constexpr int WG = Sh::WG, RC = Sh::RC, kThreads = Sh::kThreads;
   constexpr int kCtrlRegs = Sh::kCtrlRegs, kSoftmaxRegs = Sh::kSoftmaxRegs;
   constexpr int RL = RC < 8 ? 8 : RC;  // TMEM columns loaded per row set (x8 is the narrowest load used)
   static_assert(kMode != kDecode || RG == 1, "a decode unit has one row group");
@@ -1073,7 +1096,6 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     // stream across unit boundaries.
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;   // token row of the chunk; head_dim index of O
-    const int ctid = tid - 32 * kSoftmaxWarp0;  // 0 .. kSoftmaxThreads - 1
     const int wg = (warp - kSoftmaxWarp0) / 4;
     const int col0 = wg * RC;         // this warpgroup's query rows: col0 .. col0 + RC - 1
     const int wg_bar = kWarpgroupBarrier0 + wg;
@@ -1305,6 +1327,19 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       return true;
     };
 
+    const bool leader = quad == 0 && lane == 0;  // this warpgroup's first thread
+    // A published partial state's arrival, counted by the leader after the
+    // next chunk (the release fence then finds the stores long done)
+    int32_t* arrival = nullptr;
+    uint32_t arrival_add = 0;
+    auto count_arrival = [&]() {
+      if (arrival != nullptr) {
+        __threadfence();
+        atomicAdd(reinterpret_cast<unsigned int*>(arrival), arrival_add);
+        arrival = nullptr;
+      }
+    };
+
     // A segment's row sums and reference maxima, put aside (in stash buffer
     // sb, the parity of its O buffer) before the next segment's first
     // softmax resets them: sums reduced over the warp into lred, maxima into
@@ -1342,15 +1377,25 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         L[k] = (sm.lred[ob][0][c] + sm.lred[ob][1][c]) + (sm.lred[ob][2][c] + sm.lred[ob][3][c]);
       }
       const bool opens = fs.j0 == fs.first, closes = fs.j0 + fs.n == fs.nb;
+      // the outputs of this warpgroup's rows through the staging tile (the
+      // previous finish's copies have read it by now)
+      auto emit = [&]() {
+        if (leader) bulk_wait_read();
+        named_barrier_sync(wg_bar, 128);
+        stage_rows<kBf16, RC>(sm.ostage, col0, r, L, acc);
+        fence_proxy_async_smem();
+        named_barrier_sync(wg_bar, 128);
+        if (leader) issue_rows<G, RG, RC, kMode>(p, fs, s0, col0, rows, sm.ostage);
+      };
       if (opens && closes) {
-        emit_rows<kBf16, G, RG, RC, kMode>(p, fs, s0, col0, rows, r, L, acc);
+        emit();
         return;
       }
       int32_t* counter = unit_counter(p, fs);
       const int shift = 16 * wg;
-      const bool leader = quad == 0 && lane == 0;
       if (!opens) {
-        // publish: m, l of this warpgroup's rows, then acc; one arrival
+        // publish: m, l of this warpgroup's rows, then acc; the arrival is
+        // counted after the next chunk, once these stores have drained
         float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * Sh::kPartStride;
         if (quad == 0 && lane < RC) {
           pp[col0 + lane] = sm.mfin[ob][col0 + lane];
@@ -1361,8 +1406,8 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         for (int k = 0; k < RC; ++k) pp[2 * R + (col0 + k) * D + r] = acc[k];
         named_barrier_sync(wg_bar, 128);
         if (leader) {
-          __threadfence();
-          atomicAdd(reinterpret_cast<unsigned int*>(counter), 1u << shift);
+          arrival = counter;
+          arrival_add = 1u << shift;
         }
         return;
       }
@@ -1402,7 +1447,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           M[k] = mn;
         }
       }
-      emit_rows<kBf16, G, RG, RC, kMode>(p, fs, s0, col0, rows, r, L, acc);
+      emit();
     };
 
 #pragma unroll
@@ -1423,6 +1468,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         ok = softmax_chunk(ci, walk.next(p), c0 == 0, ob);
         if (!ok) break;
         ++ci;
+        if (leader) count_arrival();
         if (c0 == 0 && have_prev) {  // every PV of the previous segment is complete
           finish_segment(prev, prev_rows, ob ^ 1, prev_s0);
           have_prev = false;
@@ -1443,6 +1489,10 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
         named_barrier_sync(wg_bar, 128);
         finish_segment(prev, prev_rows, ob, prev_s0);
       }
+    }
+    if (leader) {
+      count_arrival();
+      bulk_wait_read();  // the staging tile stays until its copies have read it
     }
     if (!ok && lane == 0) {
       sm.abort = 1;

@@ -101,6 +101,20 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
       : "memory");
 }
 
+// One bulk copy shared -> global, in this thread's current bulk group.
+// Both addresses 16-byte aligned, bytes a multiple of 16; the shared source
+// may be rewritten once bulk_wait_read() has returned.
+__device__ __forceinline__ void bulk_copy_s2g(void* gmem_dst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until this thread's bulk copies have read their shared sources.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // L2 policy for data read exactly once (K/V tiles): evict first.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
