@@ -575,12 +575,15 @@ def run_ours(args):
     # The step's inputs live in the step's pinned staging areas (one per
     # buffer set, filled once from the host tensors above: a serving loop
     # would build its batch there), so each step uploads them in one copy.
-    staged = {}
+    staged = set()
+
+    counts = (int(host["pairs"].shape[0]) if has_copy else 0, int(host["slots"].shape[0]) if has_write else 0,
+              int(host["group_prefix"].shape[0]) if groups is not None else 0)
 
     def e2e_step():
         k = step.steps % len(step.sets)
-        v = step.staging()
-        if k not in staged:
+        if k not in staged:  # a set's inputs are built in its staging block once
+            v = step.staging()
             fields = [("q", host["q"]), ("block_tables", host["tables"]), ("seq_lens", host["lens"])]
             if has_write:
                 fields += [("new_k", host["new_k"]), ("new_v", host["new_v"]), ("slot_mapping", host["slots"])]
@@ -588,15 +591,10 @@ def run_ours(args):
                 fields.append(("copy_pairs", host["pairs"]))
             if groups is not None:
                 fields += [("group_starts", host["group_starts"]), ("group_prefix_blocks", host["group_prefix"])]
-            staged[k] = {}
             for name, src in fields:
-                dst = v[name][: src.shape[0]]
-                dst.copy_(src)
-                staged[k][name] = dst
-        a = staged[k]
-        return step.run(a["q"], a["block_tables"], a["seq_lens"], a.get("new_k"), a.get("new_v"),
-                        a.get("slot_mapping"), a.get("copy_pairs"), group_starts=a.get("group_starts"),
-                        group_prefix_blocks=a.get("group_prefix_blocks"))
+                v[name][: src.shape[0]].copy_(src)
+            staged.add(k)
+        return step.run_staged(*counts)
 
     # untimed: every buffer set's first steps (the first runs through the
     # checking wrappers, each set's next one captures its graph)

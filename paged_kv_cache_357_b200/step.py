@@ -165,15 +165,25 @@ class PagedDecodeStep:
                 raise ValueError(f"{name}: shape {tuple(src.shape)}, the step holds {tuple(dst.shape)}")
             if src.data_ptr() != dst.data_ptr():
                 dst.copy_(src)
-        _check(self._c.pa_step_run(self._h, n_pairs, T, n_groups, ctypes.byref(self._set)), "pa_step_run")
+        return self.run_staged(n_pairs, T, n_groups)
+
+    def run_staged(self, num_copy_pairs: int = 0, num_new_tokens: int = 0, num_groups: int = 0):
+        """Enqueue one step whose inputs already sit in the next buffer
+        set's staging views (written after ``staging()`` returned them, or
+        left there by an earlier step of the same set): the leading
+        num_copy_pairs pairs, num_new_tokens tokens and, for a shared-prefix
+        step, num_groups groups are used.  One C call, no host-side copy or
+        check of the views; returns the pinned host output as ``run()``."""
+        _check(self._c.pa_step_run(self._h, num_copy_pairs, num_new_tokens, num_groups, ctypes.byref(self._set)),
+               "pa_step_run")
         self.steps += 1
         L = self.layout
-        if T > 0:
-            self.last_h2d_bytes = L.slot_mapping + 8 * T
-        elif n_pairs > 0:
-            self.last_h2d_bytes = L.copy_pairs + 16 * n_pairs
-        elif n_groups > 0:
-            self.last_h2d_bytes = L.group_prefix_blocks + 4 * n_groups
+        if num_new_tokens > 0:
+            self.last_h2d_bytes = L.slot_mapping + 8 * num_new_tokens
+        elif num_copy_pairs > 0:
+            self.last_h2d_bytes = L.copy_pairs + 16 * num_copy_pairs
+        elif num_groups > 0:
+            self.last_h2d_bytes = L.group_prefix_blocks + 4 * num_groups
         else:
             self.last_h2d_bytes = L.seq_lens + 4 * self.S
         self.last_d2h_bytes = L.out_bytes

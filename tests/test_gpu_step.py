@@ -137,7 +137,8 @@ def test_shared_prefix_steps_match_oracle(cuda_device):
 def test_staged_steps_upload_one_packed_block(cuda_device):
     """Inputs built in the step's pinned staging views go up as one copy of
     the used part of the packed block; results match the oracle step by
-    step, and the uploaded byte count is that part's size."""
+    step (through run() and through run_staged(), alternately), and the
+    uploaded byte count is that part's size."""
     import torch
 
     import paged_kv_cache_357_b200 as pa
@@ -162,7 +163,10 @@ def test_staged_steps_upload_one_packed_block(cuda_device):
         s["new_k"].copy_(bits_to_torch(nk, L.dtype))
         s["new_v"].copy_(bits_to_torch(nv, L.dtype))
         s["slot_mapping"].copy_(torch.from_numpy(L.slot_mapping))
-        out = step.run(s["q"], s["block_tables"], s["seq_lens"], s["new_k"], s["new_v"], s["slot_mapping"])
+        if i % 2 == 0:
+            out = step.run(s["q"], s["block_tables"], s["seq_lens"], s["new_k"], s["new_v"], s["slot_mapping"])
+        else:
+            out = step.run_staged(num_new_tokens=L.num_new_tokens)
         step.wait(out)
         assert step.last_h2d_bytes == step.layout.slot_mapping + 8 * L.num_new_tokens
         k_ref, v_ref = oracle.cache_write(k_ref, v_ref, nk, nv, L.slot_mapping)
