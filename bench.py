@@ -135,6 +135,8 @@ def kernel_source_hash() -> str:
 def decode_kernel_name(L, mode: str = "plain") -> str:
     """Which decode kernel(s) the library runs for this workload."""
     if L.q_len > 1:
+        if L.head_dim == 128 and L.block_size == 16 and L.group * L.q_len >= 128:
+            return "pa_prefill_tc_kernel, query-major 128-row tiles (tcgen05)"
         return "pa_decode_tc_kernel, multi-query (tcgen05)"
     if mode == "shared_prefix":
         return "pa_decode_tc_kernel, group units: shared prefix once, then each member's blocks (tcgen05)"

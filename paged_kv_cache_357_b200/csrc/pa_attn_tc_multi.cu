@@ -6,7 +6,9 @@
 // when they fit, else several units (row tiles of RG = 32 / G positions)
 // per sequence.  This unit holds the instances at blocks of 16 tokens and
 // the dispatch; blocks of 8 and 32 are instantiated in
-// pa_attn_tc_multi_b8.cu and pa_attn_tc_multi_b32.cu.
+// pa_attn_tc_multi_b8.cu and pa_attn_tc_multi_b32.cu.  Once a sequence's
+// rows fill a 128-row tile, the query-major kernel of
+// pa_attn_tc_prefill.cu takes over.
 #include "pa_attn_tc.cuh"
 
 namespace pa {
@@ -16,6 +18,7 @@ namespace tc {
 
 bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v, int& tiles) {
   if (!tc::tc_pool_ok(pool, true) || q_len < 2) return false;
+  if (select_tc_prefill_variant(pool, group, q_len, v, tiles)) return true;
   const int rg = tc::row_groups_for(group, q_len);
   if (rg == 0) return false;
   tiles = tc::row_tiles_for(q_len, rg);

@@ -1,0 +1,714 @@
+// Multi-query paged attention in query-major tiles (prefill chunks and long
+// speculative runs) on tensor cores, sm_100a.  Each sequence brings q_len
+// new query positions; position i sees the sequence's tokens up to
+// seq_len - q_len + i (CSDN "PagedAttention：分页注意力", §"2026年最新进展"
+// items 1-2), merged over the paged blocks by the online softmax (study
+// notes ch.05 §4; vLLM blog §"关键细节" 2).
+//
+// A unit is 128 query rows: the G heads of one kv head at 128 / G
+// consecutive positions of one sequence (row r = position offset r / G,
+// head r % G).  Per 64-token chunk of the sequence's blocks:
+//
+//   S[row, token] = Q[row, :] . K_chunk[token, :]        (M=128, N=64, K=128)
+//   O[row, d]    += P[row, token] . V_chunk[token, d]     (M=128, N=128, K=16 a step)
+//
+// The rows sit in TMEM lanes, so softmax thread r owns row r of every chunk:
+// its causal limit, running max, sum and rescale are its own, and the
+// softmax needs no reduction or barrier between threads.  P enters PV as a
+// 16-bit head and a 16-bit residual (two MMAs a step), as in the decode
+// kernel.  Against the decode's token-major tile (128 tokens x at most 32
+// rows, pa_attn_tc.cuh) a tile does four times the arithmetic per MMA and
+// per loaded K/V chunk.
+//
+// Roles (256 threads, one CTA per SM): warp 0 loads q and K (TMA, 128-byte
+// swizzle), warp 1 issues QK, warp 2 loads V, warp 3 issues PV, warps 4-7
+// run the softmax, one row per thread.  Work partition, bounded waits and
+// the split-unit merge (by the CTA holding a unit's first piece) follow
+// pa_attn_tc.cuh and pa_decode_common.cuh.
+#include "pa_attn_tc.cuh"
+
+namespace pa {
+namespace tc {
+namespace pf {
+
+constexpr int kRows = 128;                        // query rows of a unit: MMA M
+constexpr int kChunk = 64;                        // tokens per chunk: MMA N of QK
+constexpr int kKStages = 3, kVStages = 3;
+constexpr int kQHalf = kRows * kRowBytes;         // 16 KB: head_dim [0, 64) (or [64, 128)) of the 128 rows
+constexpr int kQBytes = 2 * kQHalf;
+constexpr int kKHalf = kChunk * kRowBytes;        // 8 KB: one head_dim half of a chunk's tokens
+constexpr int kStageBytes = 2 * kKHalf;           // 16 KB: one chunk of K or V
+constexpr int kPBytes = kRows * kRowBytes;        // 16 KB: P[128 rows][64 tokens], 16-bit
+constexpr int kThreads = 256;
+constexpr uint32_t kColS = 0;                     // S[0], S[1]: 64 columns each
+constexpr uint32_t kColO = 128;                   // O[0], O[1]: 128 columns each
+constexpr uint32_t kTmemCols = 512;
+constexpr int kPartStride = kRows * (D + 2);      // floats per partial slot: m, l, acc per row
+
+// Geometry of a 64-token chunk of blocks of B tokens.
+//   K stage: [half][64 tokens][64 columns], two 2-D boxes per block: a
+//            K-major operand whose 8-token groups sit 1 KB apart.
+//   V stage: [block][half][B][64], one 3-D box per block: an MN-major
+//            operand, its head_dim halves kBlockBytes apart.
+template <int B>
+struct Geo {
+  static_assert(B == 16, "blocks of 16 tokens");
+  static constexpr int CB = kChunk / B;                 // blocks per chunk
+  static constexpr int kBlockBytes = B * kRowBytes;     // one block's rows in one half
+  static constexpr int kVBlockBytes = 2 * kBlockBytes;  // both halves of one block
+  __host__ __device__ static constexpr int v_offset(int t) { return (t / B) * kVBlockBytes + (t % B) * kRowBytes; }
+};
+
+struct Smem {
+  uint8_t kbuf[kKStages][kStageBytes];  // 1024-aligned regions
+  uint8_t vbuf[kVStages][kStageBytes];
+  uint8_t q[2][kQBytes];                // [half][128 rows][64]
+  uint8_t p[2][kPBytes];                // P head, P residual: [128 rows][64 tokens]
+  uint64_t kfull[kKStages];
+  uint64_t kempty[kKStages];
+  uint64_t vfull[kVStages];
+  uint64_t vempty[kVStages];
+  uint64_t qfull[2];
+  uint64_t qempty[2];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full;                      // one phase per chunk: its P is written
+  uint64_t pv_done;                     // one phase per chunk: its PV has completed
+  uint64_t o_free[2];                   // a unit's O buffer has been read by its finish
+  uint64_t mma_done[2];
+  RangeSmem range;
+  uint32_t tmem_base;
+  int abort;
+  int merge_ok;
+  int k_issued, k_consumed, v_issued, v_consumed, q_issued, q_consumed;
+};
+
+constexpr int smem_bytes() { return static_cast<int>(sizeof(Smem)) + 1024; }
+static_assert(smem_bytes() <= kMaxSmemPerCta, "shared memory of one CTA");
+
+// The chunks of one segment (a tile's blocks [j0, j0 + n) of its sequence).
+template <int RG, int B>
+struct Walk {
+  static constexpr int CB = Geo<B>::CB;
+  int seq, j, jend, len, pos0;
+  __device__ __forceinline__ void start(const DecodeParams& p, const Source<kMultiTiled, RG>& src, const Seg& sg) {
+    seq = src.table_row(p, sg.s);
+    pos0 = src.pos0(p, sg.s);
+    j = sg.j0;
+    jend = sg.j0 + sg.n;
+    len = sg.len;
+  }
+  struct Chunk {
+    int j, nblk, ntok;
+  };
+  __device__ __forceinline__ Chunk next() {
+    Chunk c;
+    c.j = j;
+    c.nblk = min(CB, jend - j);
+    c.ntok = min(c.nblk * B, len - j * B);
+    j += c.nblk;
+    return c;
+  }
+};
+
+template <bool kBf16, int G, int B>
+__global__ void __launch_bounds__(kThreads, 1)
+    pa_prefill_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_q,
+                         const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
+  constexpr int RG = kRows / G;  // positions per unit
+  using Gm = Geo<B>;
+  constexpr int CB = Gm::CB;
+  const Source<kMultiTiled, RG> src;
+  extern __shared__ unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const long long cta = blockIdx.x;
+  const int Hkv = p.num_kv_heads;
+
+  // ---- set-up that reads no input
+  if (tid == 0) {
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sm.kfull[i], 1);
+      mbar_init(&sm.kempty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sm.vfull[i], 1);
+      mbar_init(&sm.vempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.qfull[i], 1);
+      mbar_init(&sm.qempty[i], 1);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_free[i], 4);  // one arrival per softmax warp
+      mbar_init(&sm.o_free[i], 4);
+      mbar_init(&sm.mma_done[i], 1);
+    }
+    mbar_init(&sm.p_full, 4);
+    mbar_init(&sm.pv_done, 1);
+    sm.abort = 0;
+    sm.merge_ok = 0;
+    sm.k_issued = sm.k_consumed = sm.v_issued = sm.v_consumed = sm.q_issued = sm.q_consumed = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&map_q);
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_v);
+  }
+  if (warp == kQKWarp) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const volatile int* abort_flag = &sm.abort;
+
+  // ---- inputs may come from the previous kernel in the stream
+  grid_dependency_wait();
+  grid_launch_dependents();
+  zero_empty_units<kMultiTiled, RG, B>(p, src);
+  WorkRange wr;
+  Cursor cur;
+  const bool has_work = decode_prologue<kThreads, B, CB>(p, sm.range, wr, cur, src);
+
+  if (!has_work) {
+    // nothing to stream
+  } else if (warp == 0 || warp == kVWarp) {
+    // ===================== producers ========================================
+    const bool is_k = warp == 0;
+    // a sequence's K/V is reread by its other tiles: kept in L2 a while
+    const uint64_t pol_kv = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
+    bool ok = true;
+    int ci = 0, qi = 0, k_issued = 0, v_issued = 0, q_issued = 0;
+    if (p.test_flags & kFlagTestWithholdCopies) {
+      if (lane == 0) {
+        const uint64_t t0 = global_timer_ns();
+        while (*abort_flag == 0 && global_timer_ns() - t0 < 4 * p.wait_limit_ns) {
+        }
+      }
+      __syncwarp();
+    } else {
+      Seg sg;
+      while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+        const int qs = qi & 1;
+        if (is_k && lane == 0) {
+          ok = mbar_wait_bounded(&sm.qempty[qs], ((qi >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+          if (ok) {
+            // q rows: heads [h G, h G + G) of positions [z, z + RG), one box per head_dim half
+            const int z = src.row_group0(p, sg.s);
+            mbar_arrive_expect_tx(&sm.qfull[qs], kQBytes);
+            tma_load_3d(sm.q[qs], &map_q, 0, sg.h * G, z, &sm.qfull[qs], pol_q);
+            tma_load_3d(sm.q[qs] + kQHalf, &map_q, 64, sg.h * G, z, &sm.qfull[qs], pol_q);
+            ++q_issued;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        ++qi;
+        Walk<RG, B> walk;
+        walk.start(p, src, sg);
+        const int32_t* trow = p.block_tables + static_cast<size_t>(walk.seq) * p.max_nb;
+        // lane l < CB: entry of the chunk's block l, one chunk ahead
+        typename Walk<RG, B>::Chunk cs = walk.next();
+        int e_cur = lane < cs.nblk ? __ldg(trow + cs.j + lane) : 0;
+        for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
+          typename Walk<RG, B>::Chunk cn = cs;
+          int e_next = 0;
+          if (c0 + CB < sg.n) {
+            cn = walk.next();
+            e_next = lane < cn.nblk ? __ldg(trow + cn.j + lane) : 0;
+          }
+          int e = e_cur;
+          if (lane < cs.nblk && (e < 0 || e >= p.num_blocks)) {
+            record_status(p.status, PA_DEV_BAD_BLOCK_ID);
+            e = 0;
+          }
+          const int ns = is_k ? kKStages : kVStages;
+          const int st = ci % ns;
+          uint64_t* empty = is_k ? &sm.kempty[st] : &sm.vempty[st];
+          uint64_t* full = is_k ? &sm.kfull[st] : &sm.vfull[st];
+          bool go = true;
+          if (lane == 0) {
+            go = mbar_wait_bounded(empty, ((ci / ns) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+            if (go) mbar_arrive_expect_tx(full, cs.nblk * Gm::kVBlockBytes);
+          }
+          ok = __shfl_sync(0xffffffffu, go, 0);
+          if (!ok) break;
+          if (lane < cs.nblk) {
+            const int y = (e * Hkv + sg.h) * B;
+            if (is_k) {
+              uint8_t* base = sm.kbuf[st] + lane * Gm::kBlockBytes;
+              tma_load_2d(base, &map_k, 0, y, full, pol_kv);
+              tma_load_2d(base + kKHalf, &map_k, 64, y, full, pol_kv);
+            } else {
+              tma_load_3d(sm.vbuf[st] + lane * Gm::kVBlockBytes, &map_v, 0, y, 0, full, pol_kv);
+            }
+          }
+          __syncwarp();
+          if (is_k) {
+            ++k_issued;
+          } else {
+            ++v_issued;
+          }
+          ++ci;
+          cs = cn;
+          e_cur = e_next;
+        }
+      }
+    }
+    if (lane == 0) {
+      if (is_k) {
+        sm.k_issued = k_issued;
+        sm.q_issued = q_issued;
+      } else {
+        sm.v_issued = v_issued;
+      }
+      if (!ok) {
+        sm.abort = 1;
+        record_status(p.status, PA_DEV_TIMEOUT);
+      }
+    }
+  } else if (warp == kQKWarp) {
+    // ===================== QK issuer =========================================
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = make_idesc(kBf16, false, false, kChunk);  // q: K-major A, K: K-major B
+      bool ok = true;
+      int qk = 0, seg_i = 0;
+      Seg sg;
+      while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+        const int qs = seg_i & 1;
+        ok = mbar_wait_bounded(&sm.qfull[qs], (seg_i >> 1) & 1, abort_flag, p.wait_limit_ns);
+        const uint32_t q0 = smem_u32(sm.q[qs]);
+        for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
+          const int ks = qk % kKStages;
+          ok = mbar_wait_bounded(&sm.kfull[ks], (qk / kKStages) & 1, abort_flag, p.wait_limit_ns) &&
+               mbar_wait_bounded(&sm.s_free[qk & 1], ((qk >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k0 = smem_u32(sm.kbuf[ks]);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t a = sw128_desc(q0 + (k >> 2) * kQHalf + (k & 3) * 32, 16, 8 * kRowBytes);
+            const uint64_t b = sw128_desc(k0 + (k >> 2) * kKHalf + (k & 3) * 32, 16, 8 * kRowBytes);
+            umma(tmem + kColS + (qk & 1) * kChunk, a, b, kIdescQK, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&sm.s_full[qk & 1]);
+          umma_commit(&sm.kempty[ks]);
+          ++qk;
+        }
+        if (!ok) break;
+        umma_commit(&sm.qempty[qs]);  // q may be reloaded once the unit's last QK is done
+        ++seg_i;
+      }
+      umma_commit(&sm.mma_done[0]);
+      (void)mbar_wait_bounded(&sm.mma_done[0], 0, nullptr, p.wait_limit_ns);
+      sm.k_consumed = qk;
+      sm.q_consumed = seg_i;
+      if (!ok) {
+        sm.abort = 1;
+        record_status(p.status, PA_DEV_TIMEOUT);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kPVWarp) {
+    // ===================== PV issuer =========================================
+    // Per chunk, once its P is written and its V has landed: P head then P
+    // residual times V, for the 16-token steps that hold valid tokens, into
+    // the unit's O buffer (units alternate between two).
+    if (lane == 0) {
+      constexpr uint32_t kIdescPV = make_idesc(kBf16, false, true, D);  // P: K-major A, V: MN-major B
+      bool ok = true;
+      int pv = 0, seg_i = 0;
+      Seg sg;
+      while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+        Walk<RG, B> walk;
+        walk.start(p, src, sg);
+        const int ob = seg_i & 1;
+        ok = mbar_wait_bounded(&sm.o_free[ob], ((seg_i >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+        for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
+          const int ntok = walk.next().ntok;
+          const int vs = pv % kVStages;
+          ok = mbar_wait_bounded(&sm.p_full, pv & 1, abort_flag, p.wait_limit_ns) &&
+               mbar_wait_bounded(&sm.vfull[vs], (pv / kVStages) & 1, abort_flag, p.wait_limit_ns);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t v0 = smem_u32(sm.vbuf[vs]);
+          const int nks = (ntok + 15) / 16;
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const uint32_t p0 = smem_u32(sm.p[part]);
+            for (int k = 0; k < nks; ++k) {
+              const uint64_t a = sw128_desc(p0 + k * 32, 16, 8 * kRowBytes);
+              const uint64_t b = sw128_desc(v0 + Gm::v_offset(16 * k), Gm::kBlockBytes, 8 * kRowBytes);
+              umma(tmem + kColO + ob * D, a, b, kIdescPV, (c0 > 0 || k > 0 || part > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&sm.pv_done);
+          umma_commit(&sm.vempty[vs]);
+          ++pv;
+        }
+        ++seg_i;
+      }
+      umma_commit(&sm.mma_done[1]);
+      (void)mbar_wait_bounded(&sm.mma_done[1], 0, nullptr, p.wait_limit_ns);
+      sm.v_consumed = pv;
+      if (!ok) {
+        sm.abort = 1;
+        record_status(p.status, PA_DEV_TIMEOUT);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ===================== softmax (warps 4..7) =============================
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // this thread's query row (TMEM lane)
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const bool leader = r == 0;
+    const int G_off = r % G;         // head within the kv head's group
+    const int pos_off = r / G;       // position within the unit
+    bool ok = true;
+    int ci = 0, pv_seen = 0, si = 0;
+    float m_ref = kNoMax, l_sum = 0.f;  // this row's reference max and sum (relative to it)
+    int32_t* arrival = nullptr;         // a published piece's arrival, counted a chunk later
+
+    auto wait_pv = [&](int upto) -> bool {
+      while (pv_seen < upto) {
+        const bool w = mbar_wait_bounded(&sm.pv_done, pv_seen & 1, abort_flag, p.wait_limit_ns);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        ++pv_seen;
+      }
+      tc_fence_after();
+      return true;
+    };
+    auto o_addr = [&](int ob, int c) -> uint32_t { return tmem + lane_base + kColO + ob * D + c; };
+
+    // Online softmax of chunk ci of a unit whose rows start at position
+    // pos0 of a sequence of len tokens; its PV goes to O buffer ob.
+    auto softmax_chunk = [&](int ci, const typename Walk<RG, B>::Chunk& ch, int len, int pos0, bool first,
+                             int ob) -> bool {
+      const int sb = ci & 1;
+      const bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      float s[kChunk];
+      {
+        uint32_t raw[kChunk];
+        tmem_ld_nowait<kChunk>(tmem + lane_base + kColS + sb * kChunk, raw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kChunk; ++c) s[c] = __uint_as_float(raw[c]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[sb]);
+
+      // tokens [t0, t0 + nvis) of the chunk are visible to this row: the
+      // sequence's tokens up to lim (causal), none past the chunk's end
+      const int t0 = ch.j * B;
+      const int lim = len - p.q_len + pos0 + pos_off;
+      const int nvis = max(0, min(ch.ntok, lim - t0 + 1));
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kChunk; ++c) {
+        s[c] = c < nvis ? s[c] * p.scale_log2 : -INFINITY;  // the scores, masked by selection
+        mx = fmaxf(mx, s[c]);
+      }
+      // the reference max moves only when a score passes it by more than
+      // kRescaleGap (always on a unit's first chunk)
+      if (first || mx - m_ref > kRescaleGap) {
+        const float m_old = first ? -INFINITY : m_ref;
+        const float m_new = fmaxf(fmaxf(m_old, mx), kNoMax);
+        const float alpha = fast_exp2(m_old - m_new);
+        l_sum = first ? 0.f : l_sum * alpha;
+        m_ref = m_new;
+        if (!first) {  // O's row rescaled in place once the previous chunk's PV is done
+          if (!wait_pv(ci)) return false;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld_nowait<32>(o_addr(ob, c), o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st<32>(o_addr(ob, c), o);
+          }
+          tmem_wait_st();
+        }
+      }
+      uint32_t hw[kChunk / 2], lw[kChunk / 2];
+#pragma unroll
+      for (int k = 0; k < kChunk / 2; ++k) {
+        const float a0 = fast_exp2(s[2 * k] - m_ref), a1 = fast_exp2(s[2 * k + 1] - m_ref);  // 0 when masked
+        l_sum += a0 + a1;
+        hw[k] = pack2<kBf16>(a0, a1);
+        float h0, h1;
+        unpack2<kBf16>(hw[k], h0, h1);
+        lw[k] = pack2<kBf16>(a0 - h0, a1 - h1);
+      }
+      // V rows past the sequence end inside the last 16-token step are
+      // zeroed so that 0 * (whatever they hold) cannot reach the output
+      // (thread r < 64 takes token row r of the chunk)
+      if (r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
+        const int vs = ci % kVStages;
+        (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
+        uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + Gm::v_offset(r));
+        uint4* v1 = reinterpret_cast<uint4*>(sm.vbuf[vs] + Gm::v_offset(r) + Gm::kBlockBytes);
+#pragma unroll
+        for (int i = 0; i < kRowBytes / 16; ++i) {
+          v0[i] = make_uint4(0, 0, 0, 0);
+          v1[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      // P's buffer is free once the previous chunk's PV has completed
+      if (!wait_pv(ci)) return false;
+      {
+        const int swz = r & 7;
+        uint8_t* ph = sm.p[0] + r * kRowBytes;
+        uint8_t* pl = sm.p[1] + r * kRowBytes;
+#pragma unroll
+        for (int j = 0; j < kRowBytes / 16; ++j) {
+          *reinterpret_cast<uint4*>(ph + ((j ^ swz) << 4)) =
+              make_uint4(hw[4 * j], hw[4 * j + 1], hw[4 * j + 2], hw[4 * j + 3]);
+          *reinterpret_cast<uint4*>(pl + ((j ^ swz) << 4)) =
+              make_uint4(lw[4 * j], lw[4 * j + 1], lw[4 * j + 2], lw[4 * j + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full);
+      return true;
+    };
+
+    // The finish of a unit whose PVs have all completed: its rows' outputs,
+    // its published partial state, or (its first piece) the merge of every
+    // piece.  m, L are the row's reference max and sum; s_seq, pos0 its
+    // sequence and first position; ob its O buffer, handed back after.
+    auto finish_unit = [&](const Seg& fs, float m, float L, int s_seq, int pos0, int ob) {
+      const int pos = pos0 + pos_off;
+      const bool real = pos < p.q_len;
+      uint16_t* out_row =
+          p.out + ((static_cast<size_t>(s_seq) * p.q_len + pos) * p.num_q_heads + fs.h * G + G_off) * D;
+      // O of this row, normalised by inv, a 32-column piece at a time, into out_row
+      auto emit = [&](auto&& piece) {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float a[32];
+          piece(c, a);
+          if (real) {
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) w[k] = pack2<kBf16>(a[2 * k], a[2 * k + 1]);
+            uint4* o = reinterpret_cast<uint4*>(out_row + c);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
+        }
+      };
+      auto load_o = [&](int c, float (&a)[32]) {
+        uint32_t o[32];
+        tmem_ld_nowait<32>(o_addr(ob, c), o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(o[k]);
+      };
+      const bool opens = fs.j0 == fs.first, closes = fs.j0 + fs.n == fs.nb;
+      if (opens && closes) {
+        const float inv = L > 0.f ? __fdividef(1.f, L) : 0.f;  // L >= 1 for a row that saw a token
+        emit([&](int c, float (&a)[32]) {
+          load_o(c, a);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) a[k] *= inv;
+        });
+      } else if (!opens) {
+        // publish m, l and the row of O; the arrival is counted after the
+        // next chunk, once these stores have drained
+        float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * kPartStride;
+        pp[r] = m;
+        pp[kRows + r] = L;
+        float4* pa = reinterpret_cast<float4*>(pp + 2 * kRows + r * D);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float a[32];
+          load_o(c, a);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) pa[c / 4 + k] = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
+        }
+        named_barrier_sync(kWarpgroupBarrier0, 128);
+        if (leader) arrival = unit_counter(p, fs);
+      } else {
+        // merge: pieces first + 1 .. last were published by the CTAs after this one
+        const long long last = cta_of(fs.unit_last, wr.total, wr.nparts);
+        const uint32_t need = static_cast<uint32_t>(last - cta);
+        int32_t* counter = unit_counter(p, fs);
+        if (leader) {
+          const bool got = wait_arrivals(counter, 0, need, p.wait_limit_ns);
+          if (got) {
+            atomicSub(reinterpret_cast<unsigned int*>(counter), need);  // back to zero for the next launch
+          } else {
+            record_status(p.status, PA_DEV_TIMEOUT);
+          }
+          sm.merge_ok = got;
+        }
+        named_barrier_sync(kWarpgroupBarrier0, 128);
+        if (sm.merge_ok) {
+          float M = m;
+          for (long long cc = cta + 1; cc <= last; ++cc) {
+            M = fmaxf(M, __ldcg(p.partials + partial_slot(cc, fs.unit_first, wr) * kPartStride + r));
+          }
+          float Lt = L * fast_exp2(m - M);
+          for (long long cc = cta + 1; cc <= last; ++cc) {
+            const float* pp = p.partials + partial_slot(cc, fs.unit_first, wr) * kPartStride;
+            Lt = fmaf(__ldcg(pp + kRows + r), fast_exp2(__ldcg(pp + r) - M), Lt);
+          }
+          const float inv = Lt > 0.f ? __fdividef(1.f, Lt) : 0.f;
+          const float w_own = fast_exp2(m - M) * inv;
+          emit([&](int c, float (&a)[32]) {
+            load_o(c, a);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) a[k] *= w_own;
+            for (long long cc = cta + 1; cc <= last; ++cc) {
+              const float* pp = p.partials + partial_slot(cc, fs.unit_first, wr) * kPartStride;
+              const float wb = fast_exp2(__ldcg(pp + r) - M) * inv;
+              const float4* pa = reinterpret_cast<const float4*>(pp + 2 * kRows + r * D + c);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float4 v = __ldcg(pa + k);
+                a[4 * k] = fmaf(v.x, wb, a[4 * k]);
+                a[4 * k + 1] = fmaf(v.y, wb, a[4 * k + 1]);
+                a[4 * k + 2] = fmaf(v.z, wb, a[4 * k + 2]);
+                a[4 * k + 3] = fmaf(v.w, wb, a[4 * k + 3]);
+              }
+            }
+          });
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free[ob]);
+    };
+    auto count_arrival = [&]() {
+      if (arrival != nullptr) {
+        __threadfence();
+        atomicAdd(reinterpret_cast<unsigned int*>(arrival), 1u);
+        arrival = nullptr;
+      }
+    };
+
+    Seg sg, prev;
+    float prev_m = 0.f, prev_l = 0.f;
+    int prev_seq = 0, prev_pos0 = 0;
+    bool have_prev = false;
+    while (ok && next_seg<B, CB>(cur, sg, p, src)) {
+      Walk<RG, B> walk;
+      walk.start(p, src, sg);
+      const int ob = si & 1;
+      for (int c0 = 0; c0 < sg.n; c0 += CB) {
+        if (c0 == 0 && have_prev) {  // the previous unit's state, before this one resets it
+          prev_m = m_ref;
+          prev_l = l_sum;
+        }
+        ok = softmax_chunk(ci, walk.next(), walk.len, walk.pos0, c0 == 0, ob);
+        if (!ok) break;
+        ++ci;
+        if (leader) count_arrival();
+        if (c0 == 0 && have_prev) {  // every PV of the previous unit is complete
+          finish_unit(prev, prev_m, prev_l, prev_seq, prev_pos0, ob ^ 1);
+          have_prev = false;
+        }
+      }
+      if (!ok) break;
+      prev = sg;
+      prev_seq = walk.seq;
+      prev_pos0 = walk.pos0;
+      have_prev = true;
+      ++si;
+    }
+    if (ok && have_prev) {
+      ok = wait_pv(ci);
+      if (ok) finish_unit(prev, m_ref, l_sum, prev_seq, prev_pos0, (si - 1) & 1);
+    }
+    if (leader) count_arrival();
+    if (!ok && lane == 0) {
+      sm.abort = 1;
+      record_status(p.status, PA_DEV_TIMEOUT);
+    }
+  }
+
+  // ---- teardown: drain copies after an abort, release TMEM
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0 && sm.abort) {
+    for (int k = sm.k_consumed; k < sm.k_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.kfull[k % kKStages], (k / kKStages) & 1, nullptr, p.wait_limit_ns);
+    }
+    for (int k = sm.v_consumed; k < sm.v_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.vfull[k % kVStages], (k / kVStages) & 1, nullptr, p.wait_limit_ns);
+    }
+    for (int k = sm.q_consumed; k < sm.q_issued; ++k) {
+      (void)mbar_wait_bounded(&sm.qfull[k & 1], (k >> 1) & 1, nullptr, p.wait_limit_ns);
+    }
+  }
+  if (warp == kQKWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---- host side -----------------------------------------------------------------
+
+template <bool kBf16, int G, int B>
+cudaError_t launch_prefill(const Variant& v, const DecodeParams& prm, int ctas, cudaStream_t stream) {
+  constexpr int RG = kRows / G;
+  CUtensorMap mq, mk, mv;
+  const unsigned long long q_rows = static_cast<unsigned long long>(prm.num_seqs) * prm.q_len;
+  const unsigned long long kv_rows = static_cast<unsigned long long>(prm.num_blocks) * prm.num_kv_heads * B;
+  if (kv_rows >= (1ull << 31) || q_rows >= (1ull << 31)) return cudaErrorInvalidValue;
+  LaunchMaps want{};
+  want.kernel = reinterpret_cast<const void*>(&pa_prefill_tc_kernel<kBf16, G, B>);
+  want.q = prm.q;
+  want.k = prm.k_pool;
+  want.v = prm.v_pool;
+  want.q_rows = q_rows;
+  want.kv_rows = kv_rows;
+  want.num_q_heads = prm.num_q_heads;
+  if (!cached_maps(want, mq, mk, mv, &encode_launch_maps<kBf16, G, RG, B>)) return cudaErrorInvalidValue;
+  return launch_overlapped(pa_prefill_tc_kernel<kBf16, G, B>, dim3(ctas), dim3(kThreads),
+                           static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
+}
+
+// Partition cost of finishing a 128-row unit, in 1/8 of a 64-token chunk.
+constexpr int kUnitCost = 8;
+
+template <bool kBf16, int G, int B>
+Variant prefill_variant() {
+  return Variant{reinterpret_cast<const void*>(&pa_prefill_tc_kernel<kBf16, G, B>), kThreads, smem_bytes(),
+                 kPartStride, &launch_prefill<kBf16, G, B>, kUnitCost};
+}
+
+template <bool kBf16>
+bool pick(int G, Variant& v) {
+  switch (G) {
+    case 1: v = prefill_variant<kBf16, 1, 16>(); return true;
+    case 2: v = prefill_variant<kBf16, 2, 16>(); return true;
+    case 4: v = prefill_variant<kBf16, 4, 16>(); return true;
+    case 8: v = prefill_variant<kBf16, 8, 16>(); return true;
+    default: return false;
+  }
+}
+
+}  // namespace pf
+}  // namespace tc
+
+bool select_tc_prefill_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v, int& tiles) {
+  if (pool.head_dim != tc::D || pool.block_size != 16 || (pool.dtype != PA_BF16 && pool.dtype != PA_FP16)) {
+    return false;
+  }
+  if (group <= 0 || tc::pf::kRows % group != 0 || q_len * group < tc::pf::kRows) return false;
+  const int positions = tc::pf::kRows / group;
+  tiles = (q_len + positions - 1) / positions;
+  return pool.dtype == PA_BF16 ? tc::pf::pick<true>(group, v) : tc::pf::pick<false>(group, v);
+}
+
+}  // namespace pa

@@ -37,6 +37,10 @@ bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Var
 // sequence.
 bool select_tc_multi_b8(bool bf16, int group, int rg, bool tiled, Variant& v);
 bool select_tc_multi_b32(bool bf16, int group, int rg, bool tiled, Variant& v);
+// Query-major tiles of 128 rows (pa_attn_tc_prefill.cu) when a sequence's
+// G x q_len rows fill at least one (blocks of 16): tiles = units per
+// sequence and kv head.
+bool select_tc_prefill_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v, int& tiles);
 // Shared-prefix decode over groups of up to max_members sequences
 // (pa_attn_tc_group.cu).
 bool select_tc_group_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);

@@ -103,6 +103,35 @@ def test_multi_row_tiles_split_units(cuda_device, num_ctas):
     assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"tiles num_ctas={num_ctas}")
 
 
+PREFILL = [(1, 128), (1, 200), (2, 64), (2, 100), (4, 32), (4, 40), (4, 256), (8, 16), (8, 33), (8, 256)]
+
+
+@pytest.mark.parametrize("G,L", PREFILL, ids=[f"G{g}-L{l}" for g, l in PREFILL])
+def test_prefill_tiles(cuda_device, G, L):
+    """G x q_len of at least 128 rows: the query-major kernel, one unit per
+    128 rows (128 / G positions x G heads), 64-token chunks, the last tile
+    ragged when q_len is not a multiple of 128 / G; sequences from exactly
+    q_len tokens (the first position sees one) to past two thousand."""
+    dtype = "bf16" if (G + L) % 2 == 0 else "fp16"
+    lens = [L, L + 1, L + 15, L + 64, L + 65, 1000 + L, 2049]
+    layout, vals, q = _inputs(7800 + 50 * G + L, lens, G, L, dtype)
+    out, st = _run(cuda_device, layout, vals, q)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"prefill G={G} q_len={L} {dtype}")
+
+
+@pytest.mark.parametrize("num_ctas", [1, 3, 37, 200, 0])
+def test_prefill_split_units(cuda_device, num_ctas):
+    """Query-major units cut between CTAs: with 200 CTAs a long unit spans
+    several, so the merging CTA combines more than one published piece, and
+    pieces that start past a row's causal limit carry no token for it."""
+    G, L = 4, 128
+    layout, vals, q = _inputs(7900 + num_ctas, [128, 700, 3000, 129, 4100], G, L, "bf16")
+    out, st = _run(cuda_device, layout, vals, q, num_ctas)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"prefill num_ctas={num_ctas}")
+
+
 @pytest.mark.parametrize("num_ctas", [1, 3, 37, 0])
 def test_multi_split_units(cuda_device, num_ctas):
     G, L = 4, 4
