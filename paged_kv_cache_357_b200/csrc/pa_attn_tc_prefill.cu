@@ -12,17 +12,18 @@
 //   S[row, token] = Q[row, :] . K_chunk[token, :]        (M=128, N=64, K=128)
 //   O[row, d]    += P[row, token] . V_chunk[token, d]     (M=128, N=128, K=16 a step)
 //
-// The rows sit in TMEM lanes, so softmax thread r owns row r of every chunk:
-// its causal limit, running max, sum and rescale are its own, and the
-// softmax needs no reduction or barrier between threads.  P enters PV as a
+// The rows sit in TMEM lanes, so a softmax thread owns (half of) row r of
+// every chunk: its causal limit, running sum and rescale are its own; only
+// a chunk's max passes between the two threads that share a row.  P enters PV as a
 // 16-bit head and a 16-bit residual (two MMAs a step), as in the decode
 // kernel.  Against the decode's token-major tile (128 tokens x at most 32
 // rows, pa_attn_tc.cuh) a tile does four times the arithmetic per MMA and
 // per loaded K/V chunk.
 //
-// Roles (256 threads, one CTA per SM): warp 0 loads q and K (TMA, 128-byte
-// swizzle), warp 1 issues QK, warp 2 loads V, warp 3 issues PV, warps 4-7
-// run the softmax, one row per thread.  Work partition, bounded waits and
+// Roles (384 threads, one CTA per SM): warp 0 loads q and K (TMA, 128-byte
+// swizzle), warp 1 issues QK, warp 2 loads V, warp 3 issues PV, warps 4-11
+// run the softmax: two warpgroups, each row split between them by tokens
+// (and O by head_dim columns).  Work partition, bounded waits and
 // the split-unit merge (by the CTA holding a unit's first piece) follow
 // pa_attn_tc.cuh and pa_decode_common.cuh.
 #include "pa_attn_tc.cuh"
@@ -39,7 +40,13 @@ constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKHalf = kChunk * kRowBytes;        // 8 KB: one head_dim half of a chunk's tokens
 constexpr int kStageBytes = 2 * kKHalf;           // 16 KB: one chunk of K or V
 constexpr int kPBytes = kRows * kRowBytes;        // 16 KB: P[128 rows][64 tokens], 16-bit
-constexpr int kThreads = 256;
+constexpr int kHalfChunk = kChunk / 2;          // tokens of a chunk per softmax warpgroup
+constexpr int kThreads = 384;                    // control warpgroup + two softmax warpgroups
+// The control warpgroup hands registers to the softmax warpgroups
+// (setmaxnreg) inside the launch's 168 a thread: 128 x 80 + 256 x 208.
+constexpr int kCtrlRegs = 80, kSoftmaxRegs = 208, kLaunchRegs = 168;
+static_assert(128 * kCtrlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
+constexpr int kPairBarrier = 1;                  // named barrier of the two softmax warpgroups
 constexpr uint32_t kColS = 0;                     // S[0], S[1]: 64 columns each
 constexpr uint32_t kColO = 128;                   // O[0], O[1]: 128 columns each
 constexpr uint32_t kTmemCols = 512;
@@ -76,6 +83,8 @@ struct Smem {
   uint64_t pv_done;                     // one phase per chunk: its PV has completed
   uint64_t o_free[2];                   // a unit's O buffer has been read by its finish
   uint64_t mma_done[2];
+  alignas(16) float red[2][2][kRows];   // per chunk parity and warpgroup: each row's max over its tokens
+  alignas(16) float lsum[2][kRows];     // per warpgroup: a finished unit's row sums
   RangeSmem range;
   uint32_t tmem_base;
   int abort;
@@ -85,6 +94,27 @@ struct Smem {
 
 constexpr int smem_bytes() { return static_cast<int>(sizeof(Smem)) + 1024; }
 static_assert(smem_bytes() <= kMaxSmemPerCta, "shared memory of one CTA");
+
+// Two probabilities as a 16-bit head pair and a 16-bit residual pair (P =
+// head + residual, about 15 significant bits).  bf16 takes the upper half
+// of each fp32 word (truncation: the head then leaves an exact fp32
+// remainder, whose own upper half is the residual), with byte permutes and
+// masks on the integer pipe, not conversions; fp16 rounds with the
+// conversion instruction.
+template <bool kBf16>
+__device__ __forceinline__ void split_pair(float a0, float a1, uint32_t& head, uint32_t& resid) {
+  if constexpr (kBf16) {
+    const uint32_t u0 = __float_as_uint(a0), u1 = __float_as_uint(a1);
+    head = __byte_perm(u0, u1, 0x7632);
+    const float r0 = a0 - __uint_as_float(u0 & 0xffff0000u), r1 = a1 - __uint_as_float(u1 & 0xffff0000u);
+    resid = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+  } else {
+    head = pack2<false>(a0, a1);
+    float h0, h1;
+    unpack2<false>(head, h0, h1);
+    resid = pack2<false>(a0 - h0, a1 - h1);
+  }
+}
 
 // The chunks of one segment (a tile's blocks [j0, j0 + n) of its sequence).
 template <int RG, int B>
@@ -141,11 +171,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qempty[i], 1);
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 4);  // one arrival per softmax warp
-      mbar_init(&sm.o_free[i], 4);
+      mbar_init(&sm.s_free[i], 8);  // one arrival per softmax warp
+      mbar_init(&sm.o_free[i], 8);
       mbar_init(&sm.mma_done[i], 1);
     }
-    mbar_init(&sm.p_full, 4);
+    mbar_init(&sm.p_full, 8);
     mbar_init(&sm.pv_done, 1);
     sm.abort = 0;
     sm.merge_ok = 0;
@@ -177,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // nothing to stream
   } else if (warp == 0 || warp == kVWarp) {
     // ===================== producers ========================================
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     const bool is_k = warp == 0;
     // a sequence's K/V is reread by its other tiles: kept in L2 a while
     const uint64_t pol_kv = l2_policy_evict_last();
@@ -273,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kQKWarp) {
     // ===================== QK issuer =========================================
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     if (lane == 0) {
       constexpr uint32_t kIdescQK = make_idesc(kBf16, false, false, kChunk);  // q: K-major A, K: K-major B
       bool ok = true;
@@ -318,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Per chunk, once its P is written and its V has landed: P head then P
     // residual times V, for the 16-token steps that hold valid tokens, into
     // the unit's O buffer (units alternate between two).
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     if (lane == 0) {
       constexpr uint32_t kIdescPV = make_idesc(kBf16, false, true, D);  // P: K-major A, V: MN-major B
       bool ok = true;
@@ -362,16 +395,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ===================== softmax (warps 4..7) =============================
+    // ===================== softmax (warps 4..11) ============================
+    // Thread r of warpgroup w owns row r: tokens [32 w, 32 w + 32) of each
+    // chunk's S and P, head_dim [64 w, 64 w + 64) of O.  A row's max over a
+    // chunk is put together from its two halves through shared memory, so
+    // both warpgroups take the same reference max; everything else about a
+    // row is the thread's own.
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // this thread's query row (TMEM lane)
+    const int wg = (warp - 4) / 4;
+    const int col0 = wg * kHalfChunk;
+    const int d0 = wg * (D / 2);
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const bool leader = r == 0;
+    const bool leader = warp == 4 && lane == 0;
     const int G_off = r % G;         // head within the kv head's group
     const int pos_off = r / G;       // position within the unit
     bool ok = true;
     int ci = 0, pv_seen = 0, si = 0;
-    float m_ref = kNoMax, l_sum = 0.f;  // this row's reference max and sum (relative to it)
+    float m_ref = kNoMax, l_sum = 0.f;  // the row's reference max; the sum over this warpgroup's tokens
     int32_t* arrival = nullptr;         // a published piece's arrival, counted a chunk later
 
     auto wait_pv = [&](int upto) -> bool {
@@ -393,65 +435,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      float s[kChunk];
+      float s[kHalfChunk];
       {
-        uint32_t raw[kChunk];
-        tmem_ld_nowait<kChunk>(tmem + lane_base + kColS + sb * kChunk, raw);
+        uint32_t raw[kHalfChunk];
+        tmem_ld_nowait<kHalfChunk>(tmem + lane_base + kColS + sb * kChunk + col0, raw);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kChunk; ++c) s[c] = __uint_as_float(raw[c]);
+        for (int c = 0; c < kHalfChunk; ++c) s[c] = __uint_as_float(raw[c]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[sb]);
 
-      // tokens [t0, t0 + nvis) of the chunk are visible to this row: the
-      // sequence's tokens up to lim (causal), none past the chunk's end
-      const int t0 = ch.j * B;
+      // tokens [0, nv) of this warpgroup's half of the chunk are visible to
+      // this row: the sequence's tokens up to lim (causal), none past the
+      // chunk's end
       const int lim = len - p.q_len + pos0 + pos_off;
-      const int nvis = max(0, min(ch.ntok, lim - t0 + 1));
+      const int nv = max(0, min(min(ch.ntok, lim - ch.j * B + 1) - col0, kHalfChunk));
+      // d = score - base, one FFMA a token, masked by selection (most chunks
+      // are whole for every row: no per-token test there).  The base is the
+      // reference max, or 0 on a unit's first chunk, so that the chunk's max
+      // score mx + base never cancels against the no-max-yet sentinel.
+      const float m_base = first ? 0.f : m_ref;
       float mx = -INFINITY;
+      if (nv == kHalfChunk) {
 #pragma unroll
-      for (int c = 0; c < kChunk; ++c) {
-        s[c] = c < nvis ? s[c] * p.scale_log2 : -INFINITY;  // the scores, masked by selection
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kHalfChunk; ++c) {
+          s[c] = fmaf(s[c], p.scale_log2, -m_base);
+          mx = fmaxf(mx, s[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kHalfChunk; ++c) {
+          s[c] = c < nv ? fmaf(s[c], p.scale_log2, -m_base) : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
       }
+      // the row's max over the whole chunk: this half's and the other's
+      sm.red[sb][wg][r] = mx;
+      named_barrier_sync(kPairBarrier, 256);
+      mx = fmaxf(mx, sm.red[sb][wg ^ 1][r]);
       // the reference max moves only when a score passes it by more than
-      // kRescaleGap (always on a unit's first chunk)
-      if (first || mx - m_ref > kRescaleGap) {
+      // kRescaleGap (always on a unit's first chunk); then d is shifted to
+      // the new one.  Both warpgroups decide alike.
+      if (first || mx > kRescaleGap) {
         const float m_old = first ? -INFINITY : m_ref;
-        const float m_new = fmaxf(fmaxf(m_old, mx), kNoMax);
+        const float m_new = fmaxf(fmaxf(m_old, mx + m_base), kNoMax);  // mx + m_base: the chunk's max score
         const float alpha = fast_exp2(m_old - m_new);
         l_sum = first ? 0.f : l_sum * alpha;
+        const float shift = m_base - m_new;
+#pragma unroll
+        for (int c = 0; c < kHalfChunk; ++c) s[c] += shift;
         m_ref = m_new;
-        if (!first) {  // O's row rescaled in place once the previous chunk's PV is done
+        if (!first) {  // this warpgroup's half of O's row, rescaled once the previous PV is done
           if (!wait_pv(ci)) return false;
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
+          for (int c = 0; c < D / 2; c += 32) {
             uint32_t o[32];
-            tmem_ld_nowait<32>(o_addr(ob, c), o);
+            tmem_ld_nowait<32>(o_addr(ob, d0 + c), o);
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st<32>(o_addr(ob, c), o);
+            tmem_st<32>(o_addr(ob, d0 + c), o);
           }
           tmem_wait_st();
         }
       }
-      uint32_t hw[kChunk / 2], lw[kChunk / 2];
+      uint32_t hw[kHalfChunk / 2], lw[kHalfChunk / 2];
 #pragma unroll
-      for (int k = 0; k < kChunk / 2; ++k) {
-        const float a0 = fast_exp2(s[2 * k] - m_ref), a1 = fast_exp2(s[2 * k + 1] - m_ref);  // 0 when masked
+      for (int k = 0; k < kHalfChunk / 2; ++k) {
+        const float a0 = fast_exp2(s[2 * k]), a1 = fast_exp2(s[2 * k + 1]);  // 0 when masked
         l_sum += a0 + a1;
-        hw[k] = pack2<kBf16>(a0, a1);
-        float h0, h1;
-        unpack2<kBf16>(hw[k], h0, h1);
-        lw[k] = pack2<kBf16>(a0 - h0, a1 - h1);
+        split_pair<kBf16>(a0, a1, hw[k], lw[k]);
       }
       // V rows past the sequence end inside the last 16-token step are
       // zeroed so that 0 * (whatever they hold) cannot reach the output
-      // (thread r < 64 takes token row r of the chunk)
-      if (r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
+      // (thread r < 64 of the first warpgroup takes token row r)
+      if (wg == 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
         const int vs = ci % kVStages;
         (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
         uint4* v0 = reinterpret_cast<uint4*>(sm.vbuf[vs] + Gm::v_offset(r));
@@ -465,14 +525,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P's buffer is free once the previous chunk's PV has completed
       if (!wait_pv(ci)) return false;
       {
+        // this half of row r: 16-byte pieces 4 wg .. 4 wg + 3 of the 128-byte row
         const int swz = r & 7;
         uint8_t* ph = sm.p[0] + r * kRowBytes;
         uint8_t* pl = sm.p[1] + r * kRowBytes;
 #pragma unroll
-        for (int j = 0; j < kRowBytes / 16; ++j) {
-          *reinterpret_cast<uint4*>(ph + ((j ^ swz) << 4)) =
+        for (int j = 0; j < 4; ++j) {
+          const int piece = (4 * wg + j) ^ swz;
+          *reinterpret_cast<uint4*>(ph + (piece << 4)) =
               make_uint4(hw[4 * j], hw[4 * j + 1], hw[4 * j + 2], hw[4 * j + 3]);
-          *reinterpret_cast<uint4*>(pl + ((j ^ swz) << 4)) =
+          *reinterpret_cast<uint4*>(pl + (piece << 4)) =
               make_uint4(lw[4 * j], lw[4 * j + 1], lw[4 * j + 2], lw[4 * j + 3]);
         }
       }
@@ -485,17 +547,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // The finish of a unit whose PVs have all completed: its rows' outputs,
     // its published partial state, or (its first piece) the merge of every
-    // piece.  m, L are the row's reference max and sum; s_seq, pos0 its
-    // sequence and first position; ob its O buffer, handed back after.
-    auto finish_unit = [&](const Seg& fs, float m, float L, int s_seq, int pos0, int ob) {
+    // piece.  m is the row's reference max, l this warpgroup's part of its
+    // sum; s_seq, pos0 the unit's sequence and first position; ob its O
+    // buffer, handed back after.  Each warpgroup takes its 64 head_dim
+    // columns.
+    auto finish_unit = [&](const Seg& fs, float m, float l, int s_seq, int pos0, int ob) {
       const int pos = pos0 + pos_off;
       const bool real = pos < p.q_len;
       uint16_t* out_row =
-          p.out + ((static_cast<size_t>(s_seq) * p.q_len + pos) * p.num_q_heads + fs.h * G + G_off) * D;
-      // O of this row, normalised by inv, a 32-column piece at a time, into out_row
+          p.out + ((static_cast<size_t>(s_seq) * p.q_len + pos) * p.num_q_heads + fs.h * G + G_off) * D + d0;
+      sm.lsum[wg][r] = l;
+      named_barrier_sync(kPairBarrier, 256);
+      const float L = sm.lsum[0][r] + sm.lsum[1][r];
+      // this warpgroup's half of O's row, a 32-column piece at a time
       auto emit = [&](auto&& piece) {
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D / 2; c += 32) {
           float a[32];
           piece(c, a);
           if (real) {
@@ -510,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto load_o = [&](int c, float (&a)[32]) {
         uint32_t o[32];
-        tmem_ld_nowait<32>(o_addr(ob, c), o);
+        tmem_ld_nowait<32>(o_addr(ob, d0 + c), o);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(o[k]);
@@ -527,17 +594,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // publish m, l and the row of O; the arrival is counted after the
         // next chunk, once these stores have drained
         float* pp = p.partials + partial_slot(cta, fs.unit_first, wr) * kPartStride;
-        pp[r] = m;
-        pp[kRows + r] = L;
-        float4* pa = reinterpret_cast<float4*>(pp + 2 * kRows + r * D);
+        if (wg == 0) {
+          pp[r] = m;
+          pp[kRows + r] = L;
+        }
+        float4* pa = reinterpret_cast<float4*>(pp + 2 * kRows + r * D + d0);
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D / 2; c += 32) {
           float a[32];
           load_o(c, a);
 #pragma unroll
           for (int k = 0; k < 8; ++k) pa[c / 4 + k] = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
         }
-        named_barrier_sync(kWarpgroupBarrier0, 128);
+        named_barrier_sync(kPairBarrier, 256);
         if (leader) arrival = unit_counter(p, fs);
       } else {
         // merge: pieces first + 1 .. last were published by the CTAs after this one
@@ -553,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           sm.merge_ok = got;
         }
-        named_barrier_sync(kWarpgroupBarrier0, 128);
+        named_barrier_sync(kPairBarrier, 256);
         if (sm.merge_ok) {
           float M = m;
           for (long long cc = cta + 1; cc <= last; ++cc) {
@@ -573,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (long long cc = cta + 1; cc <= last; ++cc) {
               const float* pp = p.partials + partial_slot(cc, fs.unit_first, wr) * kPartStride;
               const float wb = fast_exp2(__ldcg(pp + r) - M) * inv;
-              const float4* pa = reinterpret_cast<const float4*>(pp + 2 * kRows + r * D + c);
+              const float4* pa = reinterpret_cast<const float4*>(pp + 2 * kRows + r * D + d0 + c);
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
                 const float4 v = __ldcg(pa + k);
@@ -674,6 +743,15 @@ cudaError_t launch_prefill(const Variant& v, const DecodeParams& prm, int ctas, 
   want.kv_rows = kv_rows;
   want.num_q_heads = prm.num_q_heads;
   if (!cached_maps(want, mq, mk, mv, &encode_launch_maps<kBf16, G, RG, B>)) return cudaErrorInvalidValue;
+  // setmaxnreg only moves registers inside the launch's allocation; should a
+  // build give the kernel fewer than the split needs, the softmax warps'
+  // increase would wait forever, so such a kernel is not launched
+  static const bool regs_fit = [] {
+    cudaFuncAttributes a{};
+    return cudaFuncGetAttributes(&a, pa_prefill_tc_kernel<kBf16, G, B>) == cudaSuccess &&
+           a.numRegs * kThreads >= 128 * kCtrlRegs + 256 * kSoftmaxRegs;
+  }();
+  if (!regs_fit) return cudaErrorInvalidConfiguration;
   return launch_overlapped(pa_prefill_tc_kernel<kBf16, G, B>, dim3(ctas), dim3(kThreads),
                            static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
 }
