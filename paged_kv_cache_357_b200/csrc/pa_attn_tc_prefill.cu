@@ -39,7 +39,6 @@ constexpr int kQHalf = kRows * kRowBytes;         // 16 KB: head_dim [0, 64) (or
 constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKHalf = kChunk * kRowBytes;        // 8 KB: one head_dim half of a chunk's tokens
 constexpr int kStageBytes = 2 * kKHalf;           // 16 KB: one chunk of K or V
-constexpr int kPBytes = kRows * kRowBytes;        // 16 KB: P[128 rows][64 tokens], 16-bit
 constexpr int kHalfChunk = kChunk / 2;          // tokens of a chunk per softmax warpgroup
 constexpr int kThreads = 384;                    // control warpgroup + two softmax warpgroups
 // The control warpgroup hands registers to the softmax warpgroups
@@ -47,8 +46,9 @@ constexpr int kThreads = 384;                    // control warpgroup + two soft
 constexpr int kCtrlRegs = 80, kSoftmaxRegs = 208, kLaunchRegs = 168;
 static_assert(128 * kCtrlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kPairBarrier = 1;                  // named barrier of the two softmax warpgroups
-constexpr uint32_t kColS = 0;                     // S[0], S[1]: 64 columns each
-constexpr uint32_t kColO = 128;                   // O[0], O[1]: 128 columns each
+constexpr int kSBufs = 3;                         // S / P buffers in TMEM
+constexpr uint32_t kColS = 0;                     // S[0..2]: 64 columns each, P over S once read
+constexpr uint32_t kColO = 256;                   // O[0], O[1]: 128 columns each
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPartStride = kRows * (D + 2);      // floats per partial slot: m, l, acc per row
 
@@ -70,17 +70,19 @@ struct Smem {
   uint8_t kbuf[kKStages][kStageBytes];  // 1024-aligned regions
   uint8_t vbuf[kVStages][kStageBytes];
   uint8_t q[2][kQBytes];                // [half][128 rows][64]
-  uint8_t p[2][kPBytes];                // P head, P residual: [128 rows][64 tokens]
   uint64_t kfull[kKStages];
   uint64_t kempty[kKStages];
   uint64_t vfull[kVStages];
   uint64_t vempty[kVStages];
   uint64_t qfull[2];
   uint64_t qempty[2];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full;                      // one phase per chunk: its P is written
-  uint64_t pv_done;                     // one phase per chunk: its PV has completed
+  // per S buffer (chunk c uses buffer c % 3): S written by QK, P written
+  // over it by the softmax, and the chunk's PV complete (which frees the
+  // buffer for QK of chunk c + 3).  No waiter can fall two phases behind.
+  uint64_t s_full[kSBufs];
+  uint64_t p_full[kSBufs];
+  uint64_t pv_done[kSBufs];
+  uint64_t unit_done[2];                // per O buffer: every PV of its unit has completed
   uint64_t o_free[2];                   // a unit's O buffer has been read by its finish
   uint64_t mma_done[2];
   alignas(16) float red[2][2][kRows];   // per chunk parity and warpgroup: each row's max over its tokens
@@ -114,6 +116,21 @@ __device__ __forceinline__ void split_pair(float a0, float a1, uint32_t& head, u
     unpack2<false>(head, h0, h1);
     resid = pack2<false>(a0 - h0, a1 - h1);
   }
+}
+
+// D[tmem] (+)= A[tmem] . B[smem desc], kind::f16, fp32 accumulate: A is
+// M=128 lanes by K=16 16-bit values, two to a 32-bit column (the lower
+// half holding the even K index).
+__device__ __forceinline__ void umma_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  setp.ne.b32 p, %4, 0;\n"
+      "  tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      "}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // The chunks of one segment (a tile's blocks [j0, j0 + n) of its sequence).
@@ -170,13 +187,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qempty[i], 1);
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 8);  // one arrival per softmax warp
-      mbar_init(&sm.o_free[i], 8);
+      mbar_init(&sm.unit_done[i], 1);
+      mbar_init(&sm.o_free[i], 8);  // one arrival per softmax warp
       mbar_init(&sm.mma_done[i], 1);
     }
-    mbar_init(&sm.p_full, 8);
-    mbar_init(&sm.pv_done, 1);
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 8);
+      mbar_init(&sm.pv_done[i], 1);
+    }
     sm.abort = 0;
     sm.merge_ok = 0;
     sm.k_issued = sm.k_consumed = sm.v_issued = sm.v_consumed = sm.q_issued = sm.q_consumed = 0;
@@ -316,8 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t q0 = smem_u32(sm.q[qs]);
         for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
           const int ks = qk % kKStages;
+          const int sbuf = qk % kSBufs;
           ok = mbar_wait_bounded(&sm.kfull[ks], (qk / kKStages) & 1, abort_flag, p.wait_limit_ns) &&
-               mbar_wait_bounded(&sm.s_free[qk & 1], ((qk >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+               mbar_wait_bounded(&sm.pv_done[sbuf], ((qk / kSBufs) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t k0 = smem_u32(sm.kbuf[ks]);
@@ -325,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < D / 16; ++k) {
             const uint64_t a = sw128_desc(q0 + (k >> 2) * kQHalf + (k & 3) * 32, 16, 8 * kRowBytes);
             const uint64_t b = sw128_desc(k0 + (k >> 2) * kKHalf + (k & 3) * 32, 16, 8 * kRowBytes);
-            umma(tmem + kColS + (qk & 1) * kChunk, a, b, kIdescQK, k > 0 ? 1u : 0u);
+            umma(tmem + kColS + sbuf * kChunk, a, b, kIdescQK, k > 0 ? 1u : 0u);
           }
-          umma_commit(&sm.s_full[qk & 1]);
+          umma_commit(&sm.s_full[sbuf]);
           umma_commit(&sm.kempty[ks]);
           ++qk;
         }
@@ -347,12 +367,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kPVWarp) {
     // ===================== PV issuer =========================================
-    // Per chunk, once its P is written and its V has landed: P head then P
-    // residual times V, for the 16-token steps that hold valid tokens, into
-    // the unit's O buffer (units alternate between two).
+    // Per chunk, once its P is written (over its S, in TMEM) and its V has
+    // landed: P head then P residual times V, for the 16-token steps that
+    // hold valid tokens, into the unit's O buffer (units alternate between
+    // two).  A comes from TMEM: the 16 tokens of step k are 8 columns (two
+    // 16-bit values a column) of the head's or the residual's 16 columns in
+    // the half of the chunk's 64 columns that holds them.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     if (lane == 0) {
-      constexpr uint32_t kIdescPV = make_idesc(kBf16, false, true, D);  // P: K-major A, V: MN-major B
+      constexpr uint32_t kIdescPV = make_idesc(kBf16, false, true, D);  // P: K-major A (TMEM), V: MN-major B
       bool ok = true;
       int pv = 0, seg_i = 0;
       Seg sg;
@@ -364,25 +387,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
           const int ntok = walk.next().ntok;
           const int vs = pv % kVStages;
-          ok = mbar_wait_bounded(&sm.p_full, pv & 1, abort_flag, p.wait_limit_ns) &&
+          const int sbuf = pv % kSBufs;
+          ok = mbar_wait_bounded(&sm.p_full[sbuf], (pv / kSBufs) & 1, abort_flag, p.wait_limit_ns) &&
                mbar_wait_bounded(&sm.vfull[vs], (pv / kVStages) & 1, abort_flag, p.wait_limit_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t v0 = smem_u32(sm.vbuf[vs]);
+          const uint32_t pcol = tmem + kColS + sbuf * kChunk;
           const int nks = (ntok + 15) / 16;
-#pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            const uint32_t p0 = smem_u32(sm.p[part]);
-            for (int k = 0; k < nks; ++k) {
-              const uint64_t a = sw128_desc(p0 + k * 32, 16, 8 * kRowBytes);
-              const uint64_t b = sw128_desc(v0 + Gm::v_offset(16 * k), Gm::kBlockBytes, 8 * kRowBytes);
-              umma(tmem + kColO + ob * D, a, b, kIdescPV, (c0 > 0 || k > 0 || part > 0) ? 1u : 0u);
-            }
+          for (int k = 0; k < nks; ++k) {
+            const uint64_t b = sw128_desc(v0 + Gm::v_offset(16 * k), Gm::kBlockBytes, 8 * kRowBytes);
+            const uint32_t a_head = pcol + (k >> 1) * kHalfChunk + (k & 1) * 8;
+            umma_tmem_a(tmem + kColO + ob * D, a_head, b, kIdescPV, (c0 > 0 || k > 0) ? 1u : 0u);
+            umma_tmem_a(tmem + kColO + ob * D, a_head + kHalfChunk / 2, b, kIdescPV, 1u);
           }
-          umma_commit(&sm.pv_done);
+          umma_commit(&sm.pv_done[sbuf]);
           umma_commit(&sm.vempty[vs]);
           ++pv;
         }
+        if (!ok) break;
+        umma_commit(&sm.unit_done[ob]);
         ++seg_i;
       }
       umma_commit(&sm.mma_done[1]);
@@ -412,16 +436,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int G_off = r % G;         // head within the kv head's group
     const int pos_off = r / G;       // position within the unit
     bool ok = true;
-    int ci = 0, pv_seen = 0, si = 0;
+    int ci = 0, si = 0;
     float m_ref = kNoMax, l_sum = 0.f;  // the row's reference max; the sum over this warpgroup's tokens
     int32_t* arrival = nullptr;         // a published piece's arrival, counted a chunk later
 
-    auto wait_pv = [&](int upto) -> bool {
-      while (pv_seen < upto) {
-        const bool w = mbar_wait_bounded(&sm.pv_done, pv_seen & 1, abort_flag, p.wait_limit_ns);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        ++pv_seen;
-      }
+    // chunk j's PV has completed (its S buffer's barrier; it cannot have
+    // moved on, since chunk j + 3's PV needs a P this thread has not written)
+    auto wait_pv = [&](int j) -> bool {
+      const bool w = mbar_wait_bounded(&sm.pv_done[j % kSBufs], (j / kSBufs) & 1, abort_flag, p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      return true;
+    };
+    // every PV of unit i (O buffer i & 1) has completed
+    auto wait_unit = [&](int i) -> bool {
+      const bool w = mbar_wait_bounded(&sm.unit_done[i & 1], (i >> 1) & 1, abort_flag, p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
       return true;
     };
@@ -431,21 +461,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // pos0 of a sequence of len tokens; its PV goes to O buffer ob.
     auto softmax_chunk = [&](int ci, const typename Walk<RG, B>::Chunk& ch, int len, int pos0, bool first,
                              int ob) -> bool {
-      const int sb = ci & 1;
-      const bool w = mbar_wait_bounded(&sm.s_full[sb], (ci >> 1) & 1, abort_flag, p.wait_limit_ns);
+      const int sbuf = ci % kSBufs;
+      const int sb = ci & 1;  // parity of the max exchange buffer
+      const uint32_t s_addr = tmem + lane_base + kColS + sbuf * kChunk + col0;  // this half of the row
+      const bool w = mbar_wait_bounded(&sm.s_full[sbuf], (ci / kSBufs) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
       float s[kHalfChunk];
       {
         uint32_t raw[kHalfChunk];
-        tmem_ld_nowait<kHalfChunk>(tmem + lane_base + kColS + sb * kChunk + col0, raw);
+        tmem_ld_nowait<kHalfChunk>(s_addr, raw);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kHalfChunk; ++c) s[c] = __uint_as_float(raw[c]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[sb]);
 
       // tokens [0, nv) of this warpgroup's half of the chunk are visible to
       // this row: the sequence's tokens up to lim (causal), none past the
@@ -488,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kHalfChunk; ++c) s[c] += shift;
         m_ref = m_new;
         if (!first) {  // this warpgroup's half of O's row, rescaled once the previous PV is done
-          if (!wait_pv(ci)) return false;
+          if (!wait_pv(ci - 1)) return false;
 #pragma unroll
           for (int c = 0; c < D / 2; c += 32) {
             uint32_t o[32];
@@ -521,27 +550,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           v0[i] = make_uint4(0, 0, 0, 0);
           v1[i] = make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
       }
-      // P's buffer is free once the previous chunk's PV has completed
-      if (!wait_pv(ci)) return false;
-      {
-        // this half of row r: 16-byte pieces 4 wg .. 4 wg + 3 of the 128-byte row
-        const int swz = r & 7;
-        uint8_t* ph = sm.p[0] + r * kRowBytes;
-        uint8_t* pl = sm.p[1] + r * kRowBytes;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int piece = (4 * wg + j) ^ swz;
-          *reinterpret_cast<uint4*>(ph + (piece << 4)) =
-              make_uint4(hw[4 * j], hw[4 * j + 1], hw[4 * j + 2], hw[4 * j + 3]);
-          *reinterpret_cast<uint4*>(pl + (piece << 4)) =
-              make_uint4(lw[4 * j], lw[4 * j + 1], lw[4 * j + 2], lw[4 * j + 3]);
-        }
-      }
-      fence_proxy_async_smem();
+      // P over this half's S columns: the head's 16 columns, then the
+      // residual's
+      tmem_st<16>(s_addr, hw);
+      tmem_st<16>(s_addr + kHalfChunk / 2, lw);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full);
+      if (lane == 0) mbar_arrive(&sm.p_full[sbuf]);
       return true;
     };
 
@@ -684,7 +702,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++ci;
         if (leader) count_arrival();
-        if (c0 == 0 && have_prev) {  // every PV of the previous unit is complete
+        if (c0 == 0 && have_prev) {
+          ok = wait_unit(si - 1);  // every PV of the previous unit
+          if (!ok) break;
           finish_unit(prev, prev_m, prev_l, prev_seq, prev_pos0, ob ^ 1);
           have_prev = false;
         }
@@ -697,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++si;
     }
     if (ok && have_prev) {
-      ok = wait_pv(ci);
+      ok = wait_unit(si - 1);
       if (ok) finish_unit(prev, m_ref, l_sum, prev_seq, prev_pos0, (si - 1) & 1);
     }
     if (leader) count_arrival();
