@@ -7,9 +7,9 @@
 //
 // A unit is 128 query rows: the G heads of one kv head at 128 / G
 // consecutive positions of one sequence (row r = position offset r / G,
-// head r % G).  Per 64-token chunk of the sequence's blocks:
+// head r % G).  Per 128-token chunk of the sequence's blocks:
 //
-//   S[row, token] = Q[row, :] . K_chunk[token, :]        (M=128, N=64, K=128)
+//   S[row, token] = Q[row, :] . K_chunk[token, :]        (M=128, N=128, K=128)
 //   O[row, d]    += P[row, token] . V_chunk[token, d]     (M=128, N=128, K=16 a step)
 //
 // The rows sit in TMEM lanes, so a softmax thread owns (half of) row r of
@@ -33,12 +33,12 @@ namespace tc {
 namespace pf {
 
 constexpr int kRows = 128;                        // query rows of a unit: MMA M
-constexpr int kChunk = 64;                        // tokens per chunk: MMA N of QK
-constexpr int kKStages = 3, kVStages = 3;
+constexpr int kChunk = 128;                       // tokens per chunk: MMA N of QK
+constexpr int kKStages = 2, kVStages = 2;
 constexpr int kQHalf = kRows * kRowBytes;         // 16 KB: head_dim [0, 64) (or [64, 128)) of the 128 rows
 constexpr int kQBytes = 2 * kQHalf;
-constexpr int kKHalf = kChunk * kRowBytes;        // 8 KB: one head_dim half of a chunk's tokens
-constexpr int kStageBytes = 2 * kKHalf;           // 16 KB: one chunk of K or V
+constexpr int kKHalf = kChunk * kRowBytes;        // 16 KB: one head_dim half of a chunk's tokens
+constexpr int kStageBytes = 2 * kKHalf;           // 32 KB: one chunk of K or V
 constexpr int kHalfChunk = kChunk / 2;          // tokens of a chunk per softmax warpgroup
 constexpr int kThreads = 384;                    // control warpgroup + two softmax warpgroups
 // The control warpgroup hands registers to the softmax warpgroups
@@ -46,14 +46,14 @@ constexpr int kThreads = 384;                    // control warpgroup + two soft
 constexpr int kCtrlRegs = 80, kSoftmaxRegs = 208, kLaunchRegs = 168;
 static_assert(128 * kCtrlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kPairBarrier = 1;                  // named barrier of the two softmax warpgroups
-constexpr int kSBufs = 3;                         // S / P buffers in TMEM
-constexpr uint32_t kColS = 0;                     // S[0..2]: 64 columns each, P over S once read
+constexpr int kSBufs = 2;                         // S / P buffers in TMEM
+constexpr uint32_t kColS = 0;                     // S[0], S[1]: 128 columns each, P over S once read
 constexpr uint32_t kColO = 256;                   // O[0], O[1]: 128 columns each
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPartStride = kRows * (D + 2);      // floats per partial slot: m, l, acc per row
 
-// Geometry of a 64-token chunk of blocks of B tokens.
-//   K stage: [half][64 tokens][64 columns], two 2-D boxes per block: a
+// Geometry of a 128-token chunk of blocks of B tokens.
+//   K stage: [half][128 tokens][64 columns], two 2-D boxes per block: a
 //            K-major operand whose 8-token groups sit 1 KB apart.
 //   V stage: [block][half][B][64], one 3-D box per block: an MN-major
 //            operand, its head_dim halves kBlockBytes apart.
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // hold valid tokens, into the unit's O buffer (units alternate between
     // two).  A comes from TMEM: the 16 tokens of step k are 8 columns (two
     // 16-bit values a column) of the head's or the residual's 16 columns in
-    // the half of the chunk's 64 columns that holds them.
+    // the half of the chunk's 128 columns that holds them.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     if (lane == 0) {
       constexpr uint32_t kIdescPV = make_idesc(kBf16, false, true, D);  // P: K-major A (TMEM), V: MN-major B
@@ -397,7 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nks = (ntok + 15) / 16;
           for (int k = 0; k < nks; ++k) {
             const uint64_t b = sw128_desc(v0 + Gm::v_offset(16 * k), Gm::kBlockBytes, 8 * kRowBytes);
-            const uint32_t a_head = pcol + (k >> 1) * kHalfChunk + (k & 1) * 8;
+            constexpr int kSteps = kHalfChunk / 16;  // 16-token steps in a warpgroup's half
+            const uint32_t a_head = pcol + (k / kSteps) * kHalfChunk + (k % kSteps) * 8;
             umma_tmem_a(tmem + kColO + ob * D, a_head, b, kIdescPV, (c0 > 0 || k > 0) ? 1u : 0u);
             umma_tmem_a(tmem + kColO + ob * D, a_head + kHalfChunk / 2, b, kIdescPV, 1u);
           }
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // V rows past the sequence end inside the last 16-token step are
       // zeroed so that 0 * (whatever they hold) cannot reach the output
-      // (thread r < 64 of the first warpgroup takes token row r)
+      // (thread r of the first warpgroup takes token row r)
       if (wg == 0 && r >= ch.ntok && r < ((ch.ntok + 15) & ~15)) {
         const int vs = ci % kVStages;
         (void)mbar_wait_bounded(&sm.vfull[vs], (ci / kVStages) & 1, abort_flag, p.wait_limit_ns);
@@ -554,8 +555,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // P over this half's S columns: the head's 16 columns, then the
       // residual's
-      tmem_st<16>(s_addr, hw);
-      tmem_st<16>(s_addr + kHalfChunk / 2, lw);
+      tmem_st<kHalfChunk / 2>(s_addr, hw);
+      tmem_st<kHalfChunk / 2>(s_addr + kHalfChunk / 2, lw);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -776,7 +777,7 @@ cudaError_t launch_prefill(const Variant& v, const DecodeParams& prm, int ctas, 
                            static_cast<size_t>(v.smem_bytes), stream, prm, mq, mk, mv);
 }
 
-// Partition cost of finishing a 128-row unit, in 1/8 of a 64-token chunk.
+// Partition cost of finishing a 128-row unit, in 1/8 of a 128-token chunk.
 constexpr int kUnitCost = 8;
 
 template <bool kBf16, int G, int B>
