@@ -468,15 +468,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool w = mbar_wait_bounded(&sm.s_full[sbuf], (ci / kSBufs) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      float s[kHalfChunk];
-      {
-        uint32_t raw[kHalfChunk];
-        tmem_ld_nowait<kHalfChunk>(s_addr, raw);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < kHalfChunk; ++c) s[c] = __uint_as_float(raw[c]);
-      }
-
       // tokens [0, nv) of this warpgroup's half of the chunk are visible to
       // this row: the sequence's tokens up to lim (causal), none past the
       // chunk's end
@@ -485,20 +476,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       // d = score - base, one FFMA a token, masked by selection (most chunks
       // are whole for every row: no per-token test there).  The base is the
       // reference max, or 0 on a unit's first chunk, so that the chunk's max
-      // score mx + base never cancels against the no-max-yet sentinel.
+      // score mx + base never cancels against the no-max-yet sentinel.  S
+      // comes in two loads of half the columns, the second in flight while
+      // the first is scaled.
       const float m_base = first ? 0.f : m_ref;
+      constexpr int kQ = kHalfChunk / 2;
+      float s[kHalfChunk];
+      uint32_t raw[kHalfChunk];
       float mx = -INFINITY;
-      if (nv == kHalfChunk) {
+      tmem_ld_nowait<kQ>(s_addr, raw);
+      tmem_wait_ld();
+      tmem_ld_nowait<kQ>(s_addr + kQ, raw + kQ);
 #pragma unroll
-        for (int c = 0; c < kHalfChunk; ++c) {
-          s[c] = fmaf(s[c], p.scale_log2, -m_base);
-          mx = fmaxf(mx, s[c]);
-        }
-      } else {
+      for (int part = 0; part < 2; ++part) {
+        if (part == 1) tmem_wait_ld();
+        if (nv == kHalfChunk) {
 #pragma unroll
-        for (int c = 0; c < kHalfChunk; ++c) {
-          s[c] = c < nv ? fmaf(s[c], p.scale_log2, -m_base) : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+          for (int c = part * kQ; c < (part + 1) * kQ; ++c) {
+            s[c] = fmaf(__uint_as_float(raw[c]), p.scale_log2, -m_base);
+            mx = fmaxf(mx, s[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = part * kQ; c < (part + 1) * kQ; ++c) {
+            s[c] = c < nv ? fmaf(__uint_as_float(raw[c]), p.scale_log2, -m_base) : -INFINITY;
+            mx = fmaxf(mx, s[c]);
+          }
         }
       }
       // the row's max over the whole chunk: this half's and the other's
@@ -531,12 +534,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
       }
+      // probabilities, and P over this half's S columns (read above): the
+      // head in the first half of them, the residual in the second; the
+      // first 32 tokens' columns go out while the rest are computed
       uint32_t hw[kHalfChunk / 2], lw[kHalfChunk / 2];
 #pragma unroll
-      for (int k = 0; k < kHalfChunk / 2; ++k) {
-        const float a0 = fast_exp2(s[2 * k]), a1 = fast_exp2(s[2 * k + 1]);  // 0 when masked
-        l_sum += a0 + a1;
-        split_pair<kBf16>(a0, a1, hw[k], lw[k]);
+      for (int part = 0; part < 2; ++part) {
+#pragma unroll
+        for (int k = part * kQ / 2; k < (part + 1) * kQ / 2; ++k) {
+          const float a0 = fast_exp2(s[2 * k]), a1 = fast_exp2(s[2 * k + 1]);  // 0 when masked
+          l_sum += a0 + a1;
+          split_pair<kBf16>(a0, a1, hw[k], lw[k]);
+        }
+        tmem_st<kQ / 2>(s_addr + part * kQ / 2, hw + part * kQ / 2);
+        tmem_st<kQ / 2>(s_addr + kHalfChunk / 2 + part * kQ / 2, lw + part * kQ / 2);
       }
       // V rows past the sequence end inside the last 16-token step are
       // zeroed so that 0 * (whatever they hold) cannot reach the output
@@ -553,10 +564,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
       }
-      // P over this half's S columns: the head's 16 columns, then the
-      // residual's
-      tmem_st<kHalfChunk / 2>(s_addr, hw);
-      tmem_st<kHalfChunk / 2>(s_addr + kHalfChunk / 2, lw);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
