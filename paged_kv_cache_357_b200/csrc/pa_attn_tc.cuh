@@ -1668,9 +1668,9 @@ cudaError_t launch_tc(const Variant& v, const DecodeParams& prm, int ctas, cudaS
 // sums, outputs or partial state, the merge) adds to a CTA's time beyond
 // what the pipeline hides; it grows with the rows a unit carries.  Values
 // from sweeps on B200 (Llama-3-8B decode: 2 to 3 best; q_len 4 multi-query
-// at 16 rows: 6).
+// at 16 rows: 6; shared-prefix group units: 20, 0.8 % ahead of 10 and 32).
 constexpr int unit_finish_cost(int kMode, int R) {
-  return kMode == kDecode ? (R <= 4 ? 2 : 4) : kMode == kGroup ? 10 : (R <= 8 ? 4 : R <= 16 ? 6 : 10);
+  return kMode == kDecode ? (R <= 4 ? 2 : 4) : kMode == kGroup ? 20 : (R <= 8 ? 4 : R <= 16 ? 6 : 10);
 }
 
 template <bool kBf16, int G, int RG, int kMode, int B = 16>

@@ -16,8 +16,9 @@
 // there is less than one granule of cost per CTA, so that every range that
 // falls inside a unit holds one of its granules.  A CTA's granules fall into
 // segments, one per unit it touches.  A unit covered by one CTA is finished
-// there; a unit split between CTAs is finished by whichever of them arrives
-// last.
+// there.  A unit split between CTAs is merged in the same launch: by
+// whichever CTA arrives last (finish_split_unit, the CUDA-core kernel), or
+// by the CTA holding the unit's first piece (the tensor-core kernels).
 //
 // Merge rule (study notes ch.05 §4, the online-softmax merge applied to
 // partitions): a partial state is (m, l, acc) in the log2 domain — running
