@@ -96,7 +96,7 @@ typedef struct pa_decode_opts {
 #define PA_DECODE_TEST_WITHHOLD_COPIES 1
 
 /* pa_decode_opts.flags bit: use the CUDA-core kernel even where the
- * tensor-core kernel applies (head_dim 128 and block_size 16); for
+ * tensor-core kernel applies (head_dim 128, block_size 8, 16 or 32); for
  * comparisons and tests.  Same results within the documented tolerance. */
 #define PA_DECODE_CUDA_CORES_ONLY 2
 
@@ -253,8 +253,8 @@ PA_API pa_status pa_decode_multi(const void* q, const void* k_pool, const void* 
  * streams the group's shared blocks once, seen by every member's query
  * heads, then each member's own blocks, seen by that member's heads only, and
  * writes every member's outputs.  Tensor-core kernel only: head_dim 128,
- * block_size 16, G in {1, 2, 4, 8} and G * max_group_size <= 32 (rounded up
- * to a power of two), else PA_ERR_UNSUPPORTED.  Device errors: those of
+ * block_size 8, 16 or 32, G in {1, 2, 4, 8} and G * max_group_size <= 32
+ * (rounded up to a power of two), else PA_ERR_UNSUPPORTED.  Device errors: those of
  * pa_decode, and PA_DEV_BAD_GROUP when the groups do not partition the
  * sequences or a group has more members than max_group_size rounded up to a
  * power of two (outputs then unspecified).  The workspace

@@ -44,5 +44,9 @@ bool select_tc_prefill_variant(const pa_pool_desc& pool, int group, int q_len, V
 // Shared-prefix decode over groups of up to max_members sequences
 // (pa_attn_tc_group.cu).
 bool select_tc_group_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);
+// Its instances at blocks of 8 and 32 tokens (pa_attn_tc_group_b8.cu,
+// pa_attn_tc_group_b32.cu), rg row groups (members) a unit.
+bool select_tc_group_b8(bool bf16, int group, int rg, Variant& v);
+bool select_tc_group_b32(bool bf16, int group, int rg, Variant& v);
 
 }  // namespace pa

@@ -100,6 +100,26 @@ def test_forked_samples_match_oracle(cuda_device, G, dtype):
     assert_attention_close(torch_f64(out), ref, f"shared prefix G={G} {dtype}")
 
 
+@pytest.mark.parametrize("B", [8, 32])
+@pytest.mark.parametrize("G", [2, 8])
+def test_forked_samples_other_block_sizes(cuda_device, G, B):
+    """The same forked prompts at blocks of 8 and 32 tokens: 16 or 4 blocks
+    a 128-token chunk, the shared prefix and each member's own blocks in
+    whole granules of them; with 8-token blocks a prompt's partly filled
+    last block is private to every sample more often."""
+    import paged_kv_cache_357_b200 as pa
+
+    prompts = [(40, [1, 5, 30]), (300, [1, 2, 17, 64]), (17, [1]), (128, [1, 129]), (1000, [3, 40, 200, 7])]
+    dtype = "bf16" if B == 8 else "fp16"
+    L = _forked_layout(8050 + 10 * G + B, prompts, dtype=dtype, G=G, B=B)
+    V = fill_values_numpy(L)
+    groups = pa.shared_prefix_groups(L.block_tables, L.seq_lens, L.block_size, 4)
+    out, st, _, _ = _run(cuda_device, L, V, groups, 4)
+    assert st == 0
+    ref, _, _ = oracle_step(L, V)
+    assert_attention_close(torch_f64(out), ref, f"shared prefix G={G} B={B} {dtype}")
+
+
 @pytest.mark.parametrize("num_ctas", [1, 2, 5, 33, 0])
 def test_split_group_units(cuda_device, num_ctas):
     import paged_kv_cache_357_b200 as pa
