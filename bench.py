@@ -139,7 +139,7 @@ def measured_tensor_peak():
 def tensor_bound(L) -> bool:
     """Workloads whose decode runs the query-major prefill kernel: bound by
     the tensor core and the exponentials, not by HBM."""
-    return L.q_len > 1 and L.head_dim == 128 and L.block_size == 16 and L.group * L.q_len >= 128
+    return L.q_len > 1 and L.head_dim == 128 and L.block_size in (8, 16, 32) and L.group * L.q_len >= 128
 
 
 def kernel_source_hash() -> str:

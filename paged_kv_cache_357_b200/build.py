@@ -27,7 +27,7 @@ SOURCES = [
     "pa_decode_tc_blocks.cu",
     "pa_attn_tc_multi.cu",
     "pa_attn_tc_multi_b8.cu",
-    "pa_attn_tc_multi_b32.cu", "pa_attn_tc_prefill.cu",
+    "pa_attn_tc_multi_b32.cu", "pa_attn_tc_prefill.cu", "pa_attn_tc_prefill_b8.cu", "pa_attn_tc_prefill_b32.cu",
     "pa_attn_tc_group.cu", "pa_attn_tc_group_b8.cu", "pa_attn_tc_group_b32.cu",
     "pa_kv_ops.cu",
     "pa_block_manager.cpp",

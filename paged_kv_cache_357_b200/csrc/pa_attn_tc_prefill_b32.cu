@@ -1,0 +1,12 @@
+// Query-major multi-query tiles (prefill chunks) on tensor cores at blocks
+// of 32 tokens: the instances of the kernel in pa_attn_tc_prefill.cuh (the
+// dispatch is in pa_attn_tc_prefill.cu).
+#include "pa_attn_tc_prefill.cuh"
+
+namespace pa {
+
+bool select_tc_prefill_b32(bool bf16, int group, Variant& v) {
+  return bf16 ? tc::pf::pick<true, 32>(group, v) : tc::pf::pick<false, 32>(group, v);
+}
+
+}  // namespace pa

@@ -38,9 +38,12 @@ bool select_tc_multi_variant(const pa_pool_desc& pool, int group, int q_len, Var
 bool select_tc_multi_b8(bool bf16, int group, int rg, bool tiled, Variant& v);
 bool select_tc_multi_b32(bool bf16, int group, int rg, bool tiled, Variant& v);
 // Query-major tiles of 128 rows (pa_attn_tc_prefill.cu) when a sequence's
-// G x q_len rows fill at least one (blocks of 16): tiles = units per
-// sequence and kv head.
+// G x q_len rows fill at least one (blocks of 8, 16 or 32): tiles = units
+// per sequence and kv head.  Its instances at blocks of 8 and 32 tokens:
+// pa_attn_tc_prefill_b8.cu, pa_attn_tc_prefill_b32.cu.
 bool select_tc_prefill_variant(const pa_pool_desc& pool, int group, int q_len, Variant& v, int& tiles);
+bool select_tc_prefill_b8(bool bf16, int group, Variant& v);
+bool select_tc_prefill_b32(bool bf16, int group, Variant& v);
 // Shared-prefix decode over groups of up to max_members sequences
 // (pa_attn_tc_group.cu).
 bool select_tc_group_variant(const pa_pool_desc& pool, int group, int max_members, Variant& v);

@@ -120,6 +120,22 @@ def test_prefill_tiles(cuda_device, G, L):
     assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"prefill G={G} q_len={L} {dtype}")
 
 
+PREFILL_BLOCKS = [(8, 4, 40), (8, 1, 200), (32, 2, 100), (32, 8, 33)]
+
+
+@pytest.mark.parametrize("B,G,L", PREFILL_BLOCKS, ids=[f"B{b}-G{g}-L{l}" for b, g, l in PREFILL_BLOCKS])
+def test_prefill_tiles_other_block_sizes(cuda_device, B, G, L):
+    """The query-major kernel at blocks of 8 and 32 tokens: a 128-token
+    chunk is 16 or 4 blocks (K as one 3-D box per 8-token block, or two
+    2-D boxes per 32-token block); ragged last tiles."""
+    dtype = "bf16" if B == 8 else "fp16"
+    lens = [L, L + 1, L + B - 1, L + 129, 1000 + L, 2049]
+    layout, vals, q = _inputs(7950 + 10 * B + G + L, lens, G, L, dtype, block_size=B)
+    out, st = _run(cuda_device, layout, vals, q)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"prefill B={B} G={G} q_len={L} {dtype}")
+
+
 @pytest.mark.parametrize("num_ctas", [1, 3, 37, 200, 0])
 def test_prefill_split_units(cuda_device, num_ctas):
     """Query-major units cut between CTAs: with 200 CTAs a long unit spans
