@@ -156,12 +156,16 @@ def subproblem(layout: PagedLayout, values_dev, seqs):
     q = torch_bits(values_dev.q[seqs])
     slots, nk, nv = [], [], []
     if layout.num_new_tokens > 0:
-        for s in seqs:
-            slot = int(layout.slot_mapping[s])
+        # every sequence writes the same number of new tokens, in sequence order
+        per = layout.num_new_tokens // layout.num_seqs
+        assert per * layout.num_seqs == layout.num_new_tokens
+        toks = [s * per + i for s in seqs for i in range(per)]
+        for t in toks:
+            slot = int(layout.slot_mapping[t])
             blk, row = slot // B, slot % B
             slots.append(remap[blk] * B + row)
-        nk = torch_bits(values_dev.new_k[seqs])
-        nv = torch_bits(values_dev.new_v[seqs])
+        nk = torch_bits(values_dev.new_k[toks])
+        nv = torch_bits(values_dev.new_v[toks])
     return dict(q=q, k_pool=kp, v_pool=vp, tables=tables, lens=layout.seq_lens[seqs].copy(), pairs=cpairs,
                 slots=np.asarray(slots, np.int64), new_k=nk, new_v=nv)
 

@@ -9,7 +9,8 @@ import pytest
 
 import oracle
 from pa_testlib import assert_attention_close, subproblem, torch_bits, torch_f64
-from workloads import bits_to_torch, config_llama3_8b, f32_to_bits, fill_values_numpy, fill_values_torch, random_layout
+from workloads import (bits_to_torch, config_llama3_8b, config_llama3_8b_prefill, f32_to_bits, fill_values_numpy,
+                       fill_values_torch, random_layout)
 
 pytestmark = pytest.mark.gpu
 
@@ -250,3 +251,38 @@ def test_llama3_8b_full_size_speculative_verify(cuda_device):
     kp, vp = oracle.cache_write(sub["k_pool"], sub["v_pool"], sub["new_k"], sub["new_v"], sub["slots"])
     ref = oracle.decode_multi(q_host, kp, vp, sub["tables"], sub["lens"], L.scale, L.num_kv_heads, L.dtype)
     assert_attention_close(torch_f64(out)[seqs], ref, "llama3_8b q_len=4")
+
+
+def test_llama3_8b_prefill256_full_size(cuda_device):
+    """The 256-token prefill workload at full size, as the bench runs it:
+    the cache write of every sequence's 256 new tokens, then the query-major
+    kernel over all 64 sequences; the shortest sequence (whose first position
+    sees one token), the median and the longest one and three more against
+    the oracle, every output finite and inside the range of V."""
+    import torch
+
+    import paged_kv_cache_357_b200 as pa
+
+    L = config_llama3_8b_prefill()
+    V = fill_values_torch(L, cuda_device)
+    rng = np.random.default_rng(6)
+    order = np.argsort(L.seq_lens)
+    seqs = sorted({int(order[0]), int(order[len(order) // 2]), int(order[-1]),
+                   *map(int, rng.choice(L.num_seqs, 3, replace=False))})
+    sub = subproblem(L, V, seqs)
+    tables = torch.from_numpy(L.block_tables).to(cuda_device)
+    lens = torch.from_numpy(L.seq_lens).to(cuda_device)
+    slots = torch.from_numpy(L.slot_mapping).to(cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    pa.pa_cache_write(V.new_k, V.new_v, slots, V.k_pool, V.v_pool, st)
+    out = torch.full_like(V.q, float("nan"))
+    ws = pa.alloc_multi_workspace(L.num_seqs, L.q_len, L.num_q_heads, V.k_pool)
+    pa.pa_decode_multi(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.isfinite(out).all()
+    vmax = max(float(V.v_pool.float().nan_to_num(0).abs().max()), float(V.new_v.float().abs().max()))
+    assert float(out.float().abs().max()) <= vmax * (1 + 1e-2)
+    kp, vp = oracle.cache_write(sub["k_pool"], sub["v_pool"], sub["new_k"], sub["new_v"], sub["slots"])
+    ref = oracle.decode_multi(sub["q"], kp, vp, sub["tables"], sub["lens"], L.scale, L.num_kv_heads, L.dtype)
+    assert_attention_close(torch_f64(out)[seqs], ref, "llama3_8b prefill q_len=256")
