@@ -33,7 +33,8 @@ SOURCES = [
     "pa_block_manager.cpp",
     "pa_step.cpp",
 ]
-HEADERS = ["pa_device.cuh", "pa_internal.h", "pa_decode_common.cuh", "pa_decode_host.h", "pa_attn_tc.cuh"]
+HEADERS = ["pa_device.cuh", "pa_internal.h", "pa_decode_common.cuh", "pa_decode_host.h", "pa_attn_tc.cuh",
+           "pa_attn_tc_group.cuh", "pa_attn_tc_prefill.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON_FLAGS = ARCH_FLAGS + [

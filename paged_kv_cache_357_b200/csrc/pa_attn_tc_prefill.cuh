@@ -67,9 +67,9 @@ struct Smem {
   uint64_t vempty[kVStages];
   uint64_t qfull[2];
   uint64_t qempty[2];
-  // per S buffer (chunk c uses buffer c % 3): S written by QK, P written
+  // per S buffer (chunk c uses buffer c % 2): S written by QK, P written
   // over it by the softmax, and the chunk's PV complete (which frees the
-  // buffer for QK of chunk c + 3).  No waiter can fall two phases behind.
+  // buffer for QK of chunk c + 2).  No waiter can fall two phases behind.
   uint64_t s_full[kSBufs];
   uint64_t p_full[kSBufs];
   uint64_t pv_done[kSBufs];
@@ -88,6 +88,49 @@ struct Smem {
 constexpr int smem_bytes() { return static_cast<int>(sizeof(Smem)) + 1024; }
 static_assert(smem_bytes() <= kMaxSmemPerCta, "shared memory of one CTA");
 
+// Packed fp32 pairs: sm_100's two-lane FFMA, FADD, FSUB and FMUL each do
+// two independent IEEE single-precision operations (round to nearest, no
+// flush) in one instruction; the three-input max takes two new values a step.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n"
+      "  .reg .b64 ra, rb, rc, rd;\n"
+      "  mov.b64 ra, {%2, %3};\n"
+      "  mov.b64 rb, {%4, %5};\n"
+      "  mov.b64 rc, {%6, %7};\n"
+      "  fma.rn.f32x2 rd, ra, rb, rc;\n"
+      "  mov.b64 {%0, %1}, rd;\n"
+      "}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+#define PA_PF_BINARY_F32X2(name, op)                                          \
+  __device__ __forceinline__ float2 name(float2 a, float2 b) {                \
+    float2 d;                                                                 \
+    asm("{\n"                                                                 \
+        "  .reg .b64 ra, rb, rd;\n"                                           \
+        "  mov.b64 ra, {%2, %3};\n"                                           \
+        "  mov.b64 rb, {%4, %5};\n"                                           \
+        "  " op ".rn.f32x2 rd, ra, rb;\n"                                     \
+        "  mov.b64 {%0, %1}, rd;\n"                                           \
+        "}\n"                                                                 \
+        : "=f"(d.x), "=f"(d.y)                                                \
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));                            \
+    return d;                                                                 \
+  }
+PA_PF_BINARY_F32X2(add2, "add")
+PA_PF_BINARY_F32X2(sub2, "sub")
+PA_PF_BINARY_F32X2(mul2, "mul")
+#undef PA_PF_BINARY_F32X2
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Two probabilities as a 16-bit head pair and a 16-bit residual pair (P =
 // head + residual, about 15 significant bits).  bf16 takes the upper half
 // of each fp32 word (truncation: the head then leaves an exact fp32
@@ -99,8 +142,9 @@ __device__ __forceinline__ void split_pair(float a0, float a1, uint32_t& head, u
   if constexpr (kBf16) {
     const uint32_t u0 = __float_as_uint(a0), u1 = __float_as_uint(a1);
     head = __byte_perm(u0, u1, 0x7632);
-    const float r0 = a0 - __uint_as_float(u0 & 0xffff0000u), r1 = a1 - __uint_as_float(u1 & 0xffff0000u);
-    resid = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+    const float2 r = sub2(make_float2(a0, a1),
+                          make_float2(__uint_as_float(u0 & 0xffff0000u), __uint_as_float(u1 & 0xffff0000u)));
+    resid = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
   } else {
     head = pack2<false>(a0, a1);
     float h0, h1;
@@ -434,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* arrival = nullptr;         // a published piece's arrival, counted a chunk later
 
     // chunk j's PV has completed (its S buffer's barrier; it cannot have
-    // moved on, since chunk j + 3's PV needs a P this thread has not written)
+    // moved on, since chunk j + 2's PV needs a P this thread has not written)
     auto wait_pv = [&](int j) -> bool {
       const bool w = mbar_wait_bounded(&sm.pv_done[j % kSBufs], (j / kSBufs) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
@@ -475,72 +519,98 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int kQ = kHalfChunk / 2;
       float s[kHalfChunk];
       uint32_t raw[kHalfChunk];
-      float mx = -INFINITY;
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nb2 = make_float2(-m_base, -m_base);
+      float mxa = -INFINITY, mxb = -INFINITY;  // two partial maxima: two dependency chains
       tmem_ld_nowait<kQ>(s_addr, raw);
       tmem_wait_ld();
       tmem_ld_nowait<kQ>(s_addr + kQ, raw + kQ);
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         if (part == 1) tmem_wait_ld();
-        if (nv == kHalfChunk) {
 #pragma unroll
-          for (int c = part * kQ; c < (part + 1) * kQ; ++c) {
-            s[c] = fmaf(__uint_as_float(raw[c]), p.scale_log2, -m_base);
-            mx = fmaxf(mx, s[c]);
+        for (int c = part * kQ; c < (part + 1) * kQ; c += 2) {
+          float2 d = fma2(make_float2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), sc2, nb2);
+          if (nv != kHalfChunk) {
+            d.x = c < nv ? d.x : -INFINITY;
+            d.y = c + 1 < nv ? d.y : -INFINITY;
           }
-        } else {
-#pragma unroll
-          for (int c = part * kQ; c < (part + 1) * kQ; ++c) {
-            s[c] = c < nv ? fmaf(__uint_as_float(raw[c]), p.scale_log2, -m_base) : -INFINITY;
-            mx = fmaxf(mx, s[c]);
+          s[c] = d.x;
+          s[c + 1] = d.y;
+          if ((c >> 1) & 1) {
+            mxb = max3(mxb, d.x, d.y);
+          } else {
+            mxa = max3(mxa, d.x, d.y);
           }
         }
       }
+      float mx = fmaxf(mxa, mxb);
       // the row's max over the whole chunk: this half's and the other's
       sm.red[sb][wg][r] = mx;
       named_barrier_sync(kPairBarrier, 256);
       mx = fmaxf(mx, sm.red[sb][wg ^ 1][r]);
       // the reference max moves only when a score passes it by more than
       // kRescaleGap (always on a unit's first chunk); then d is shifted to
-      // the new one.  Both warpgroups decide alike.
-      if (first || mx > kRescaleGap) {
+      // the new one and O's row is scaled by alpha.  Both warpgroups decide
+      // alike for a row.
+      const bool moves = first || mx > kRescaleGap;
+      float alpha = 1.f;
+      if (moves) {
         const float m_old = first ? -INFINITY : m_ref;
         const float m_new = fmaxf(fmaxf(m_old, mx + m_base), kNoMax);  // mx + m_base: the chunk's max score
-        const float alpha = fast_exp2(m_old - m_new);
+        alpha = fast_exp2(m_old - m_new);
         l_sum = first ? 0.f : l_sum * alpha;
-        const float shift = m_base - m_new;
+        const float2 shift = make_float2(m_base - m_new, m_base - m_new);
 #pragma unroll
-        for (int c = 0; c < kHalfChunk; ++c) s[c] += shift;
-        m_ref = m_new;
-        if (!first) {  // this warpgroup's half of O's row, rescaled once the previous PV is done
-          if (!wait_pv(ci - 1)) return false;
-#pragma unroll
-          for (int c = 0; c < D / 2; c += 32) {
-            uint32_t o[32];
-            tmem_ld_nowait<32>(o_addr(ob, d0 + c), o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st<32>(o_addr(ob, d0 + c), o);
-          }
-          tmem_wait_st();
+        for (int c = 0; c < kHalfChunk; c += 2) {
+          const float2 d = add2(make_float2(s[c], s[c + 1]), shift);
+          s[c] = d.x;
+          s[c + 1] = d.y;
         }
+        m_ref = m_new;
+      }
+      // this warpgroup's half of O's rows, once the previous PV is done, by
+      // the warp as a whole (TMEM loads and stores are warp-wide): a row
+      // whose reference stayed takes alpha = 1
+      if (!first && __any_sync(0xffffffffu, moves)) {
+        if (!wait_pv(ci - 1)) return false;
+        const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int c = 0; c < D / 2; c += 32) {
+          uint32_t o[32];
+          tmem_ld_nowait<32>(o_addr(ob, d0 + c), o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float2 d = mul2(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), a2);
+            o[k] = __float_as_uint(d.x);
+            o[k + 1] = __float_as_uint(d.y);
+          }
+          tmem_st<32>(o_addr(ob, d0 + c), o);
+        }
+        tmem_wait_st();
       }
       // probabilities, and P over this half's S columns (read above): the
       // head in the first half of them, the residual in the second; the
       // first 32 tokens' columns go out while the rest are computed
       uint32_t hw[kHalfChunk / 2], lw[kHalfChunk / 2];
+      float2 la = make_float2(0.f, 0.f), lb = la;  // partial row sums, two chains
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
 #pragma unroll
         for (int k = part * kQ / 2; k < (part + 1) * kQ / 2; ++k) {
           const float a0 = fast_exp2(s[2 * k]), a1 = fast_exp2(s[2 * k + 1]);  // 0 when masked
-          l_sum += a0 + a1;
+          if (k & 1) {
+            lb = add2(lb, make_float2(a0, a1));
+          } else {
+            la = add2(la, make_float2(a0, a1));
+          }
           split_pair<kBf16>(a0, a1, hw[k], lw[k]);
         }
         tmem_st<kQ / 2>(s_addr + part * kQ / 2, hw + part * kQ / 2);
         tmem_st<kQ / 2>(s_addr + kHalfChunk / 2 + part * kQ / 2, lw + part * kQ / 2);
       }
+      la = add2(la, lb);
+      l_sum += la.x + la.y;
       // V rows past the sequence end inside the last 16-token step are
       // zeroed so that 0 * (whatever they hold) cannot reach the output
       // (thread r of the first warpgroup takes token row r)

@@ -149,6 +149,40 @@ def test_prefill_split_units(cuda_device, num_ctas):
     assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"prefill num_ctas={num_ctas}")
 
 
+def _bits_to_f32(bits, dtype):
+    if dtype == "fp16":
+        return bits.view(np.float16).astype(np.float32)
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+RISING = [("bf16", 0), ("fp16", 0), ("bf16", 37)]
+
+
+@pytest.mark.parametrize("dtype,num_ctas", RISING, ids=[f"{d}-ctas{n}" for d, n in RISING])
+def test_prefill_rising_scores(cuda_device, dtype, num_ctas):
+    """Keys whose magnitude grows along the sequence (x (1 + t / 256) at
+    token t) and queries of mixed magnitude (x 0.05 .. 1.6 per row): later
+    chunks pass a row's reference max by more than the lazy-rescale gap for
+    some rows of a warp and not for others, so references move, and O is
+    rescaled, in the middle of a unit, row by row; with 37 CTAs also across
+    the pieces of split units."""
+    G, L = 4, 128
+    layout, vals, _ = _inputs(8100 + num_ctas, [L, L + 70, 700, 1500, 3000], G, L, dtype)
+    B = layout.block_size
+    k = _bits_to_f32(vals.k_pool, dtype)
+    for s, n in enumerate(layout.seq_lens):
+        for t in range(int(n)):
+            k[layout.block_tables[s, t // B], :, t % B, :] *= 1.0 + t / 256.0
+    vals.k_pool = f32_to_bits(k, dtype)
+    rng = np.random.default_rng([8100, 5])
+    S, Hq, D = layout.num_seqs, layout.num_q_heads, layout.head_dim
+    q = f32_to_bits(rng.standard_normal((S, L, Hq, D), dtype=np.float32) *
+                    rng.uniform(0.05, 1.6, size=(S, L, Hq, 1)).astype(np.float32), dtype)
+    out, st = _run(cuda_device, layout, vals, q, num_ctas)
+    assert st == 0
+    assert_attention_close(torch_f64(out), _oracle(layout, vals, q), f"rising scores {dtype} num_ctas={num_ctas}")
+
+
 @pytest.mark.parametrize("num_ctas", [1, 3, 37, 0])
 def test_multi_split_units(cuda_device, num_ctas):
     G, L = 4, 4

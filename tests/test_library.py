@@ -216,3 +216,11 @@ def test_step_rejects_bad_shapes_and_pointers_on_host(lib):
         assert rc == 1 and not h.value
     assert lib.pa_step_run(None, 0, 0, 0, None) == 1
     lib.pa_step_destroy(None)  # a no-op
+
+
+def test_build_tracks_every_source_and_header():
+    """An edited kernel header must make the library stale: the build's
+    inputs list every file under csrc/."""
+    csrc = Path(pa_build.CSRC)
+    on_disk = {p.name for p in csrc.iterdir() if p.suffix in (".cu", ".cuh", ".h", ".cpp")}
+    assert on_disk == set(pa_build.SOURCES) | set(pa_build.HEADERS)
