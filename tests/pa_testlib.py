@@ -246,3 +246,42 @@ def run_beam_trace(ours, ref, prompt_len: int, width: int, steps: int, seed: int
         if on_step is not None:
             on_step(i, live, arrays)
     return history
+
+
+def bits_to_f32(bits: np.ndarray, dtype: str) -> np.ndarray:
+    """float32 values of fp16/bf16 bit patterns (exact)."""
+    if dtype == "fp16":
+        return bits.view(np.float16).astype(np.float32)
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def rising_scores(layout: PagedLayout, values: PagedValues, q_bits: np.ndarray, seed: int, rate: float = 1 / 256):
+    """Inputs whose scores rise along each sequence: every cached key (and
+    every new key, at the position it is written to) scaled by 1 + rate * t
+    at token position t, and each query row (a sequence's position and
+    head) scaled by a factor drawn from [0.05, 1.6].  A row's running max is
+    then passed by a wide margin in the middle of a sequence, for some rows
+    of a tile and not for others.  Returns (values with the scaled keys,
+    scaled query bits)."""
+    from dataclasses import replace
+
+    from workloads import f32_to_bits
+
+    dt, B = layout.dtype, layout.block_size
+    k = bits_to_f32(values.k_pool, dt)
+    pos = {}
+    for s, n in enumerate(layout.seq_lens):
+        for t in range(int(n)):
+            pos[(int(layout.block_tables[s, t // B]), t % B)] = t
+    for (blk, off), t in pos.items():  # a shared slot once, at its position
+        k[blk, :, off, :] *= 1.0 + rate * t
+    new_k = values.new_k
+    if layout.num_new_tokens > 0:
+        nk = bits_to_f32(new_k, dt)
+        for i, sl in enumerate(layout.slot_mapping):
+            nk[i] *= 1.0 + rate * pos[(int(sl) // B, int(sl) % B)]
+        new_k = f32_to_bits(nk, dt)
+    rng = np.random.default_rng([seed, 5])
+    qf = bits_to_f32(q_bits, dt)
+    row_scale = rng.uniform(0.05, 1.6, size=qf.shape[:-1] + (1,)).astype(np.float32)
+    return replace(values, k_pool=f32_to_bits(k, dt), new_k=new_k), f32_to_bits(qf * row_scale, dt)
