@@ -49,10 +49,15 @@ constexpr int kThreads = 384;                    // control warpgroup + two soft
 constexpr int kCtrlRegs = 80, kSoftmaxRegs = 208, kLaunchRegs = 168;
 static_assert(128 * kCtrlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kPairBarrier = 1;                  // named barrier of the two softmax warpgroups
-constexpr int kSBufs = 2;                         // S / P buffers in TMEM
-constexpr uint32_t kColS = 0;                     // S[0], S[1]: 128 columns each, P over S once read
-constexpr uint32_t kColO = 256;                   // O[0], O[1]: 128 columns each
+// TMEM: kSBufs S buffers of 128 columns (P written over S once read), then
+// kOBufs O accumulators of 128 columns.  Three S buffers let QK run a chunk
+// further ahead of the softmax than two; one O buffer then makes a unit's
+// first PV wait for the previous unit's finish.
+constexpr int kSBufs = 3, kOBufs = 1;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColO = kSBufs * kChunk;
 constexpr uint32_t kTmemCols = 512;
+static_assert(kColO + kOBufs * D <= kTmemCols, "S and O buffers fit the 512 TMEM columns");
 constexpr int kPartStride = kRows * (D + 2);      // floats per partial slot: m, l, acc per row
 
 static_assert(kChunk == kChunkTok, "a chunk has the decode kernel's block geometry (Blk<B>)");
@@ -67,14 +72,15 @@ struct Smem {
   uint64_t vempty[kVStages];
   uint64_t qfull[2];
   uint64_t qempty[2];
-  // per S buffer (chunk c uses buffer c % 2): S written by QK, P written
-  // over it by the softmax, and the chunk's PV complete (which frees the
-  // buffer for QK of chunk c + 2).  No waiter can fall two phases behind.
+  // per S buffer (chunk c uses buffer c % kSBufs): S written by QK, P
+  // written over it by the softmax, and the chunk's PV complete (which frees
+  // the buffer for QK of chunk c + kSBufs).  No waiter can fall two phases
+  // behind.
   uint64_t s_full[kSBufs];
   uint64_t p_full[kSBufs];
   uint64_t pv_done[kSBufs];
-  uint64_t unit_done[2];                // per O buffer: every PV of its unit has completed
-  uint64_t o_free[2];                   // a unit's O buffer has been read by its finish
+  uint64_t unit_done[kOBufs];           // per O buffer: every PV of its unit has completed
+  uint64_t o_free[kOBufs];              // a unit's O buffer has been read by its finish
   uint64_t mma_done[2];
   alignas(16) float red[2][2][kRows];   // per chunk parity and warpgroup: each row's max over its tokens
   alignas(16) float lsum[2][kRows];     // per warpgroup: a finished unit's row sums
@@ -222,9 +228,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qempty[i], 1);
+      mbar_init(&sm.mma_done[i], 1);
+    }
+    for (int i = 0; i < kOBufs; ++i) {
       mbar_init(&sm.unit_done[i], 1);
       mbar_init(&sm.o_free[i], 8);  // one arrival per softmax warp
-      mbar_init(&sm.mma_done[i], 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&sm.s_full[i], 1);
@@ -405,10 +413,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================== PV issuer =========================================
     // Per chunk, once its P is written (over its S, in TMEM) and its V has
     // landed: P head then P residual times V, for the 16-token steps that
-    // hold valid tokens, into the unit's O buffer (units alternate between
-    // two).  A comes from TMEM: the 16 tokens of step k are 8 columns (two
-    // 16-bit values a column) of the head's or the residual's 16 columns in
-    // the half of the chunk's 128 columns that holds them.
+    // hold valid tokens, into the unit's O buffer (unit i takes buffer
+    // i % kOBufs, once the finish of the unit before has read it).  A comes
+    // from TMEM: the 16 tokens of step k are 8 columns (two 16-bit values a
+    // column) of the head's or the residual's 16 columns in the half of the
+    // chunk's 128 columns that holds them.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     if (lane == 0) {
       constexpr uint32_t kIdescPV = make_idesc(kBf16, false, true, D);  // P: K-major A (TMEM), V: MN-major B
@@ -418,8 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && next_seg<B, CB>(cur, sg, p, src)) {
         Walk<RG, B> walk;
         walk.start(p, src, sg);
-        const int ob = seg_i & 1;
-        ok = mbar_wait_bounded(&sm.o_free[ob], ((seg_i >> 1) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+        const int ob = seg_i % kOBufs;
+        ok = mbar_wait_bounded(&sm.o_free[ob], ((seg_i / kOBufs) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
         for (int c0 = 0; ok && c0 < sg.n; c0 += CB) {
           const int ntok = walk.next().ntok;
           const int vs = pv % kVStages;
@@ -485,9 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       return true;
     };
-    // every PV of unit i (O buffer i & 1) has completed
+    // every PV of unit i (O buffer i % kOBufs) has completed
     auto wait_unit = [&](int i) -> bool {
-      const bool w = mbar_wait_bounded(&sm.unit_done[i & 1], (i >> 1) & 1, abort_flag, p.wait_limit_ns);
+      const bool w = mbar_wait_bounded(&sm.unit_done[i % kOBufs], (i / kOBufs) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
       return true;
@@ -762,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (ok && next_seg<B, CB>(cur, sg, p, src)) {
       Walk<RG, B> walk;
       walk.start(p, src, sg);
-      const int ob = si & 1;
+      const int ob = si % kOBufs;
       for (int c0 = 0; c0 < sg.n; c0 += CB) {
         if (c0 == 0 && have_prev) {  // the previous unit's state, before this one resets it
           prev_m = m_ref;
@@ -775,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c0 == 0 && have_prev) {
           ok = wait_unit(si - 1);  // every PV of the previous unit
           if (!ok) break;
-          finish_unit(prev, prev_m, prev_l, prev_seq, prev_pos0, ob ^ 1);
+          finish_unit(prev, prev_m, prev_l, prev_seq, prev_pos0, (si - 1) % kOBufs);
           have_prev = false;
         }
       }
@@ -788,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && have_prev) {
       ok = wait_unit(si - 1);
-      if (ok) finish_unit(prev, m_ref, l_sum, prev_seq, prev_pos0, (si - 1) & 1);
+      if (ok) finish_unit(prev, m_ref, l_sum, prev_seq, prev_pos0, (si - 1) % kOBufs);
     }
     if (leader) count_arrival();
     if (!ok && lane == 0) {
