@@ -530,25 +530,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t raw[kHalfChunk];
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nb2 = make_float2(-m_base, -m_base);
       float mxa = -INFINITY, mxb = -INFINITY;  // two partial maxima: two dependency chains
+      // whether any row of the warp has masked tokens here (the chunks on a
+      // unit's causal diagonal or at its sequence's end): the masking is
+      // then taken by the whole warp, and skipped by it otherwise
+      const bool masked = __any_sync(0xffffffffu, nv != kHalfChunk);
       tmem_ld_nowait<kQ>(s_addr, raw);
       tmem_wait_ld();
       tmem_ld_nowait<kQ>(s_addr + kQ, raw + kQ);
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         if (part == 1) tmem_wait_ld();
+        if (masked) {
 #pragma unroll
-        for (int c = part * kQ; c < (part + 1) * kQ; c += 2) {
-          float2 d = fma2(make_float2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), sc2, nb2);
-          if (nv != kHalfChunk) {
+          for (int c = part * kQ; c < (part + 1) * kQ; c += 2) {
+            float2 d = fma2(make_float2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), sc2, nb2);
             d.x = c < nv ? d.x : -INFINITY;
             d.y = c + 1 < nv ? d.y : -INFINITY;
+            s[c] = d.x;
+            s[c + 1] = d.y;
+            if ((c >> 1) & 1) {
+              mxb = max3(mxb, d.x, d.y);
+            } else {
+              mxa = max3(mxa, d.x, d.y);
+            }
           }
-          s[c] = d.x;
-          s[c + 1] = d.y;
-          if ((c >> 1) & 1) {
-            mxb = max3(mxb, d.x, d.y);
-          } else {
-            mxa = max3(mxa, d.x, d.y);
+        } else {
+#pragma unroll
+          for (int c = part * kQ; c < (part + 1) * kQ; c += 2) {
+            const float2 d = fma2(make_float2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), sc2, nb2);
+            s[c] = d.x;
+            s[c + 1] = d.y;
+            if ((c >> 1) & 1) {
+              mxb = max3(mxb, d.x, d.y);
+            } else {
+              mxa = max3(mxa, d.x, d.y);
+            }
           }
         }
       }
@@ -560,13 +576,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the reference max moves only when a score passes it by more than
       // kRescaleGap (always on a unit's first chunk); then d is shifted to
       // the new one and O's row is scaled by alpha.  Both warpgroups decide
-      // alike for a row.
+      // alike for a row.  The step is taken by the warp as a whole: a row
+      // that keeps its reference gets a shift of 0 and alpha = 1.
       const bool moves = first || mx > kRescaleGap;
+      const bool any_moves = __any_sync(0xffffffffu, moves);
       float alpha = 1.f;
-      if (moves) {
+      if (any_moves) {
         const float m_old = first ? -INFINITY : m_ref;
-        const float m_new = fmaxf(fmaxf(m_old, mx + m_base), kNoMax);  // mx + m_base: the chunk's max score
-        alpha = fast_exp2(m_old - m_new);
+        const float m_new = moves ? fmaxf(fmaxf(m_old, mx + m_base), kNoMax) : m_ref;  // mx + m_base: the chunk's max
+        alpha = moves ? fast_exp2(m_old - m_new) : 1.f;
         l_sum = first ? 0.f : l_sum * alpha;
         const float2 shift = make_float2(m_base - m_new, m_base - m_new);
 #pragma unroll
@@ -580,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this warpgroup's half of O's rows, once the previous PV is done, by
       // the warp as a whole (TMEM loads and stores are warp-wide): a row
       // whose reference stayed takes alpha = 1
-      if (!first && __any_sync(0xffffffffu, moves)) {
+      if (!first && any_moves) {
         if (!wait_pv(ci - 1)) return false;
         const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
