@@ -14,9 +14,9 @@
 //
 // The rows sit in TMEM lanes, so a softmax thread owns (half of) row r of
 // every chunk: its causal limit, running sum and rescale are its own; only
-// a chunk's max passes between the two threads that share a row.  P enters PV as a
-// 16-bit head and a 16-bit residual (two MMAs a step), as in the decode
-// kernel.  Against the decode's token-major tile (128 tokens x at most 32
+// a chunk's max passes between the two threads that share a row.  P enters
+// PV as a 16-bit head and a 16-bit residual (two MMAs a step), as in the
+// decode kernel.  Against the decode's token-major tile (128 tokens x at most 32
 // rows, pa_attn_tc.cuh) a tile does four times the arithmetic per MMA and
 // per loaded K/V chunk.
 //
@@ -42,13 +42,13 @@ constexpr int kQHalf = kRows * kRowBytes;         // 16 KB: head_dim [0, 64) (or
 constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKHalf = kChunk * kRowBytes;        // 16 KB: one head_dim half of a chunk's tokens
 constexpr int kStageBytes = 2 * kKHalf;           // 32 KB: one chunk of K or V
-constexpr int kHalfChunk = kChunk / 2;          // tokens of a chunk per softmax warpgroup
-constexpr int kThreads = 384;                    // control warpgroup + two softmax warpgroups
+constexpr int kHalfChunk = kChunk / 2;            // tokens of a chunk per softmax warpgroup
+constexpr int kThreads = 384;                     // control warpgroup + two softmax warpgroups
 // The control warpgroup hands registers to the softmax warpgroups
 // (setmaxnreg) inside the launch's 168 a thread: 128 x 80 + 256 x 208.
 constexpr int kCtrlRegs = 80, kSoftmaxRegs = 208, kLaunchRegs = 168;
 static_assert(128 * kCtrlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
-constexpr int kPairBarrier = 1;                  // named barrier of the two softmax warpgroups
+constexpr int kPairBarrier = 1;                   // named barrier of the two softmax warpgroups
 // TMEM: kSBufs S buffers of 128 columns (P written over S once read), then
 // kOBufs O accumulators of 128 columns.  Three S buffers let QK run a chunk
 // further ahead of the softmax than two; one O buffer then makes a unit's
@@ -466,8 +466,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ===================== softmax (warps 4..11) ============================
-    // Thread r of warpgroup w owns row r: tokens [32 w, 32 w + 32) of each
-    // chunk's S and P, head_dim [64 w, 64 w + 64) of O.  A row's max over a
+    // Thread r of warpgroup w owns row r: tokens [64 w, 64 w + 64) of each
+    // chunk's S and P (P's head and residual in the same 64 columns),
+    // head_dim [64 w, 64 w + 64) of O at the unit's finish.  A row's max over a
     // chunk is put together from its two halves through shared memory, so
     // both warpgroups take the same reference max; everything else about a
     // row is the thread's own.
@@ -487,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* arrival = nullptr;         // a published piece's arrival, counted a chunk later
 
     // chunk j's PV has completed (its S buffer's barrier; it cannot have
-    // moved on, since chunk j + 2's PV needs a P this thread has not written)
+    // moved on, since chunk j + kSBufs's PV needs a P this thread has not
+    // written)
     auto wait_pv = [&](int j) -> bool {
       const bool w = mbar_wait_bounded(&sm.pv_done[j % kSBufs], (j / kSBufs) & 1, abort_flag, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
