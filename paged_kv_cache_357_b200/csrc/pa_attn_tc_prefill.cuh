@@ -673,40 +673,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool real = pos < p.q_len;
       uint16_t* out_row =
           p.out + ((static_cast<size_t>(s_seq) * p.q_len + pos) * p.num_q_heads + fs.h * G + G_off) * D + d0;
-      sm.lsum[wg][r] = l;
-      named_barrier_sync(kPairBarrier, 256);
-      const float L = sm.lsum[0][r] + sm.lsum[1][r];
-      // this warpgroup's half of O's row, a 32-column piece at a time
-      auto emit = [&](auto&& piece) {
-#pragma unroll
-        for (int c = 0; c < D / 2; c += 32) {
-          float a[32];
-          piece(c, a);
-          if (real) {
-            uint32_t w[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) w[k] = pack2<kBf16>(a[2 * k], a[2 * k + 1]);
-            uint4* o = reinterpret_cast<uint4*>(out_row + c);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) o[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-          }
-        }
-      };
-      auto load_o = [&](int c, float (&a)[32]) {
-        uint32_t o[32];
-        tmem_ld_nowait<32>(o_addr(ob, d0 + c), o);
+      // this warpgroup's half of O's row, loaded at once (in flight while
+      // the row sums are exchanged); the O buffer is handed back as soon as
+      // it has been read
+      float a[D / 2];
+      {
+        uint32_t o[D / 2];
+        tmem_ld_nowait<32>(o_addr(ob, d0), o);
+        tmem_ld_nowait<32>(o_addr(ob, d0 + 32), o + 32);
+        sm.lsum[wg][r] = l;
+        named_barrier_sync(kPairBarrier, 256);
         tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(o[k]);
+        for (int k = 0; k < D / 2; ++k) a[k] = __uint_as_float(o[k]);
+      }
+      const float L = sm.lsum[0][r] + sm.lsum[1][r];
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free[ob]);
+      // the row's outputs: 64 columns, 16-bit, rounded to nearest even
+      auto store_row = [&]() {
+        if (!real) return;
+        uint32_t w[D / 4];
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) w[k] = pack2<kBf16>(a[2 * k], a[2 * k + 1]);
+        uint4* o = reinterpret_cast<uint4*>(out_row);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) o[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+      };
+      auto scale_row = [&](float f) {
+        const float2 f2 = make_float2(f, f);
+#pragma unroll
+        for (int k = 0; k < D / 2; k += 2) {
+          const float2 v = mul2(make_float2(a[k], a[k + 1]), f2);
+          a[k] = v.x;
+          a[k + 1] = v.y;
+        }
       };
       const bool opens = fs.j0 == fs.first, closes = fs.j0 + fs.n == fs.nb;
       if (opens && closes) {
-        const float inv = L > 0.f ? __fdividef(1.f, L) : 0.f;  // L >= 1 for a row that saw a token
-        emit([&](int c, float (&a)[32]) {
-          load_o(c, a);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) a[k] *= inv;
-        });
+        scale_row(L > 0.f ? __fdividef(1.f, L) : 0.f);  // L >= 1 for a row that saw a token
+        store_row();
       } else if (!opens) {
         // publish m, l and the row of O; the arrival is counted after the
         // next chunk, once these stores have drained
@@ -717,12 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float4* pa = reinterpret_cast<float4*>(pp + 2 * kRows + r * D + d0);
 #pragma unroll
-        for (int c = 0; c < D / 2; c += 32) {
-          float a[32];
-          load_o(c, a);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) pa[c / 4 + k] = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
-        }
+        for (int k = 0; k < D / 8; ++k) pa[k] = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
         named_barrier_sync(kPairBarrier, 256);
         if (leader) arrival = unit_counter(p, fs);
       } else {
@@ -751,30 +753,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             Lt = fmaf(__ldcg(pp + kRows + r), fast_exp2(__ldcg(pp + r) - M), Lt);
           }
           const float inv = Lt > 0.f ? __fdividef(1.f, Lt) : 0.f;
-          const float w_own = fast_exp2(m - M) * inv;
-          emit([&](int c, float (&a)[32]) {
-            load_o(c, a);
+          scale_row(fast_exp2(m - M) * inv);
+          for (long long cc = cta + 1; cc <= last; ++cc) {
+            const float* pp = p.partials + partial_slot(cc, fs.unit_first, wr) * kPartStride;
+            const float wb = fast_exp2(__ldcg(pp + r) - M) * inv;
+            const float4* pa = reinterpret_cast<const float4*>(pp + 2 * kRows + r * D + d0);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) a[k] *= w_own;
-            for (long long cc = cta + 1; cc <= last; ++cc) {
-              const float* pp = p.partials + partial_slot(cc, fs.unit_first, wr) * kPartStride;
-              const float wb = fast_exp2(__ldcg(pp + r) - M) * inv;
-              const float4* pa = reinterpret_cast<const float4*>(pp + 2 * kRows + r * D + d0 + c);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const float4 v = __ldcg(pa + k);
-                a[4 * k] = fmaf(v.x, wb, a[4 * k]);
-                a[4 * k + 1] = fmaf(v.y, wb, a[4 * k + 1]);
-                a[4 * k + 2] = fmaf(v.z, wb, a[4 * k + 2]);
-                a[4 * k + 3] = fmaf(v.w, wb, a[4 * k + 3]);
-              }
+            for (int k = 0; k < D / 8; ++k) {
+              const float4 v = __ldcg(pa + k);
+              a[4 * k] = fmaf(v.x, wb, a[4 * k]);
+              a[4 * k + 1] = fmaf(v.y, wb, a[4 * k + 1]);
+              a[4 * k + 2] = fmaf(v.z, wb, a[4 * k + 2]);
+              a[4 * k + 3] = fmaf(v.w, wb, a[4 * k + 3]);
             }
-          });
+          }
+          store_row();
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.o_free[ob]);
     };
     auto count_arrival = [&]() {
       if (arrival != nullptr) {
