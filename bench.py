@@ -66,6 +66,10 @@ def parse_args(argv=None):
                     help="shared_prefix: pa_decode_shared_prefix over the workload's prompt groups; "
                          "cuda_cores: pa_decode held to its CUDA-core kernel (PA_DECODE_CUDA_CORES_ONLY)")
     ap.add_argument("--max-group", type=int, default=4, help="members per shared-prefix group")
+    ap.add_argument("--step", default="one_launch", choices=["one_launch", "separate"],
+                    help="one_launch: the step's copies and writes inside the tensor-core decode's launch "
+                         "(pa_decode_update and friends) where that kernel runs; separate: pa_copy_blocks, "
+                         "pa_cache_write and the decode as their own launches")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per GPU for the llama7b / llama3_8b(_spec4, _prefill256) / llama2_70b_shared "
                          "workloads (0 = the workload's own)")
@@ -163,8 +167,9 @@ def decode_kernel_name(L, mode: str = "plain") -> str:
     return "pa_decode_kernel (CUDA cores)"
 
 
-def roofline_of(L, mode, achieved_gbs, peak_gbs, peak_kind, nbytes, decode_ms) -> dict:
-    """The decode kernel's roofline: HBM bytes for the decode kernels; for
+def roofline_of(L, mode, achieved_gbs, peak_gbs, peak_kind, nbytes, decode_ms, fused=False) -> dict:
+    """The decode kernel's roofline: HBM bytes for the decode kernels (with
+    the step's copy and write bytes when they run in the same launch); for
     the prefill kernel the algorithmic tensor arithmetic (4 D flops per
     query row and visible token) against the dense 16-bit tensor peak."""
     if tensor_bound(L):
@@ -183,8 +188,11 @@ def roofline_of(L, mode, achieved_gbs, peak_gbs, peak_kind, nbytes, decode_ms) -
             "algorithmic_flops_per_launch": decode_flops(L),
             "hbm_gbs_beside": achieved_gbs,
         }
+    name = decode_kernel_name(L, mode)
+    if fused:
+        name += ", with the step's block copies and new-token writes in the same launch"
     return {
-        "kernel": decode_kernel_name(L, mode),
+        "kernel": name,
         "bound": "hbm",
         "achieved": achieved_gbs,
         "peak": peak_gbs,
@@ -192,8 +200,8 @@ def roofline_of(L, mode, achieved_gbs, peak_gbs, peak_kind, nbytes, decode_ms) -
         "unit": "GB/s",
         "frac": achieved_gbs / peak_gbs,
         "frac_of_8000_nominal": achieved_gbs / 8000.0,
-        "traffic": profiled_traffic(L, mode),
-        "algorithmic_bytes_per_launch": nbytes["decode"],
+        "traffic": profiled_traffic(L, mode, fused),
+        "algorithmic_bytes_per_launch": nbytes["step"] if fused else nbytes["decode"],
     }
 
 
@@ -203,11 +211,22 @@ def decode_entry(L, mode: str) -> str:
     return "pa_decode_shared_prefix" if mode == "shared_prefix" else "pa_decode"
 
 
-def profiled_traffic(L, mode: str = "plain"):
-    """dram read+write bytes per decode launch from the committed ncu summary
-    of the default workload, or None for other workloads, when there is no
-    summary, or when the kernel source changed since it was taken."""
-    if L.name != "llama3_8b" or mode != "plain" or L.num_seqs != 256:
+def one_launch_step(L, mode: str, step: str) -> bool:
+    """Whether the timed step is a single launch of the tensor-core decode
+    with the step's cache update inside it (the *_update entry points): the
+    tensor-core decode family, not the prefill or CUDA-core kernels, which
+    take the update as separate launches."""
+    if step != "one_launch" or mode == "cuda_cores" or tensor_bound(L):
+        return False
+    return L.num_new_tokens > 0 or L.copy_pairs.shape[0] > 0
+
+
+def profiled_traffic(L, mode: str = "plain", fused: bool = True):
+    """dram read+write bytes per launch of the default workload's one-launch
+    step (cache write + decode) from the committed ncu summary, or None for
+    other workloads or launch forms, when there is no summary, or when the
+    kernel source changed since it was taken."""
+    if L.name != "llama3_8b" or mode != "plain" or L.num_seqs != 256 or not fused:
         return None
     try:
         text = open(PROFILE_SUMMARY).read()
@@ -556,16 +575,35 @@ def run_ours(args):
         ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, V.k_pool, args.num_ctas, decode_flags)
     stream = torch.cuda.Stream(device=dev)
     has_copy, has_write = L.copy_pairs.shape[0] > 0, L.num_new_tokens > 0
-    launches_per_step = 1 + int(has_copy) + int(has_write)
+    fused = one_launch_step(L, mode, args.step)
+    launches_per_step = 1 if fused else 1 + int(has_copy) + int(has_write)
+    upd = {}
+    if has_copy:
+        upd["copy_pairs"] = pairs
+    if has_write:
+        upd.update(new_k=V.new_k, new_v=V.new_v, slot_mapping=slots)
 
     def prologue():
+        if fused:
+            return
         if has_copy:
             pa.pa_copy_blocks(pairs, V.k_pool, V.v_pool, status, stream=stream)
         if has_write:
             pa.pa_cache_write(V.new_k, V.new_v, slots, V.k_pool, V.v_pool, status, stream=stream)
 
     def decode():
-        if L.q_len > 1:
+        if fused:  # one launch: the step's copies and writes, then the decode
+            if L.q_len > 1:
+                pa.pa_decode_multi_update(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status,
+                                          num_ctas=args.num_ctas, stream=stream, **upd)
+            elif mode == "shared_prefix":
+                pa.pa_decode_shared_prefix_update(V.q, V.k_pool, V.v_pool, tables, lens, groups[0], groups[1],
+                                                  args.max_group, L.scale, out, ws, status, num_ctas=args.num_ctas,
+                                                  stream=stream, **upd)
+            else:
+                pa.pa_decode_update(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status,
+                                    num_ctas=args.num_ctas, flags=decode_flags, stream=stream, **upd)
+        elif L.q_len > 1:
             pa.pa_decode_multi(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, out, ws, status,
                                num_ctas=args.num_ctas, stream=stream)
         elif mode == "shared_prefix":
@@ -587,8 +625,13 @@ def run_ours(args):
     if int(status.item()) != 0:
         raise SystemExit(f"device status {int(status.item())} during warm-up")
 
+    # Two timed loops of K steps each.  The first gives `value`: events only
+    # at its ends, so consecutive launches overlap as programmatic dependent
+    # launch lets them (an event between two kernels would serialise them).
+    # The second times every decode launch on its own (events around it) for
+    # the roofline.
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(gpu_id_for(local))
     barrier()
@@ -596,17 +639,22 @@ def run_ours(args):
     with torch.cuda.stream(stream):
         t_start.record(stream)
         for k in range(K):
-            ev[k][0].record(stream)
             prologue()
-            ev[k][1].record(stream)
             decode()
-            ev[k][2].record(stream)
         t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            prologue()
+            ev[k][0].record(stream)
+            decode()
+            ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
-    decode_ms = sorted(ev[k][1].elapsed_time(ev[k][2]) for k in range(K))
+    decode_ms = sorted(ev[k][0].elapsed_time(ev[k][1]) for k in range(K))
     decode_mean_ms = sum(decode_ms) / K
     if int(status.item()) != 0:
         raise SystemExit(f"device status {int(status.item())} in the timed region")
@@ -678,7 +726,7 @@ def run_ours(args):
     value = whole_job_gbs(world, nbytes["step"], ms_per_step)
     tokens_per_s = world * L.num_seqs * L.q_len / (ms_per_step * 1e-3)
     peak, peak_kind = measured_hbm_peak()
-    achieved = nbytes["decode"] / (decode_mean_ms * 1e-3) / 1e9
+    achieved = (nbytes["step"] if fused else nbytes["decode"]) / (decode_mean_ms * 1e-3) / 1e9
     result = None
     if rank == 0:
         result = {
@@ -700,8 +748,11 @@ def run_ours(args):
                 "global_batch": L.num_seqs * world,
                 "seq_len": {"mean": float(np.mean(L.seq_lens)), "min": int(L.seq_lens.min()),
                             "max": int(L.seq_lens.max())},
-                "step": "+".join((["pa_copy_blocks"] if has_copy else []) + (["pa_cache_write"] if has_write
-                                                                             else []) + [decode_entry(L, mode)]),
+                "step": (decode_entry(L, mode) + "_update (" + "+".join(
+                    (["block copies"] if has_copy else []) + (["cache write"] if has_write else []) + ["decode"])
+                    + " in one launch)") if fused else "+".join(
+                    (["pa_copy_blocks"] if has_copy else []) + (["pa_cache_write"] if has_write else [])
+                    + [decode_entry(L, mode)]),
                 "q_len": L.q_len,
                 "decode": mode,
                 "l2": f"no flush: per-step K/V {nbytes['decode'] / 1e9:.2f} GB > 126 MB L2",
@@ -711,10 +762,14 @@ def run_ours(args):
             "tokens_per_s_note": ("one new token per sequence per single-layer step" if L.q_len == 1 else
                                   f"{L.q_len} query positions per sequence per single-layer step"),
             "decode_ms": decode_mean_ms,
+            "decode_ms_note": (("CUDA events around each launch of the tensor-core kernel, which also runs the "
+                                "step's cache update" if fused else "CUDA events around each decode launch")
+                               + ", in a second timed loop of K steps; ms_per_step comes from the first loop, "
+                                 "timed by events at its two ends only"),
             "decode_tflops": decode_flops(L) / (decode_mean_ms * 1e-3) / 1e12,
             "decode_ms_p50": decode_ms[K // 2],
             "bytes": nbytes,
-            "roofline": roofline_of(L, mode, achieved, peak, peak_kind, nbytes, decode_mean_ms),
+            "roofline": roofline_of(L, mode, achieved, peak, peak_kind, nbytes, decode_mean_ms, fused),
             "e2e": {
                 "value": whole_job_gbs(world, nbytes["step"], e2e_ms),
                 "unit": "GB/s",
@@ -729,7 +784,8 @@ def run_ours(args):
                 "link_note": "this box's pinned-copy bandwidth for one step's input and output bytes, "
                              "measured outside the timed region (context: e2e is bound by it when slow)",
             },
-            "gpu_launches": K * launches_per_step,
+            "gpu_launches": 2 * K * launches_per_step,
+            "gpu_launches_note": "both timed loops (value's and the per-launch timing's)",
             "clocks": clocks,
         }
     if world > 1:

@@ -86,7 +86,7 @@ typedef struct pa_pool_desc {
 /* Tuning/test options for pa_decode_ex; zero-initialise for the defaults. */
 typedef struct pa_decode_opts {
   int32_t num_ctas; /* persistent CTAs; 0 = SM count x resident CTAs per SM */
-  int32_t flags;    /* 0, or PA_DECODE_CUDA_CORES_ONLY and/or PA_DECODE_TEST_WITHHOLD_COPIES */
+  int32_t flags;    /* 0, or PA_DECODE_CUDA_CORES_ONLY and/or a PA_DECODE_TEST_* hook */
 } pa_decode_opts;
 
 /* Failure-detection test hook for pa_decode_opts.flags: the producer warps
@@ -99,6 +99,13 @@ typedef struct pa_decode_opts {
  * tensor-core kernel applies (head_dim 128, block_size 8, 16 or 32); for
  * comparisons and tests.  Same results within the documented tolerance. */
 #define PA_DECODE_CUDA_CORES_ONLY 2
+
+/* Failure-detection test hook for the *_update entry points: CTA 0 of the
+ * tensor-core kernel never arrives at the cache update's grid-wide
+ * barriers, so every wait for them runs out after about 20 ms and the
+ * kernel returns early with PA_DEV_TIMEOUT (pools and outputs unspecified,
+ * the workspace to be zeroed again).  Never set it outside such tests. */
+#define PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL 4
 
 /*
  * pa_decode_workspace_bytes — bytes of device scratch pa_decode needs.
@@ -304,6 +311,69 @@ PA_API pa_status pa_cache_write(const void* k, const void* v, const int64_t* slo
  */
 PA_API pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs, void* k_pool, void* v_pool,
                          int32_t* dev_status, const pa_pool_desc* pool, void* stream);
+
+/*
+ * One decode step's cache update followed by its attention, in one launch
+ * where the tensor-core kernel runs.  A serving step first copies the
+ * blocks that copy on write gives a writer (study notes ch.05 §6.1), then
+ * stores each new token's K/V in its slot (vLLM blog, plain-language
+ * section), then attends over the cache that now holds it (vLLM blog
+ * §"关键细节" 2).  These entry points take the three as one call:
+ *
+ *   pa_copy_blocks(update->copy_pairs, ...);
+ *   pa_cache_write(update->k, update->v, update->slot_mapping, ...);
+ *   pa_decode_ex / pa_decode_multi / pa_decode_shared_prefix(...);
+ *
+ * with the same results (pools bit for bit, outputs within the decode
+ * tolerance) and the same device errors.  The pool pointers are written.
+ * Where the tensor-core kernel runs (head_dim 128, 16-bit pools, the shapes
+ * listed for each decode), the copies and stores run inside its launch: all
+ * CTAs take a share of them at the start, and a grid-wide barrier (an
+ * arrival count and a generation word in the workspace, every wait bounded)
+ * holds back every K/V load until the last store has landed.  This saves
+ * the two small launches and their gaps per step.  Elsewhere the three
+ * kernels are enqueued in order on `stream`.
+ *
+ * update == NULL, or both counts 0, is the plain decode.  copy_pairs and
+ * slot_mapping follow pa_copy_blocks and pa_cache_write (pairs run in
+ * parallel, and a dst that is also a src is undefined; negative slots are
+ * padding).  k, v are [num_tokens][num_kv_heads][head_dim] like the pools,
+ * 16-byte aligned.  The workspace is the decode's (same size query); its
+ * barrier words are left as found when the device status is PA_DEV_OK.  A
+ * barrier wait that runs out (for instance when other work keeps part of
+ * the grid off the GPU for its whole limit) records PA_DEV_TIMEOUT; the
+ * pools and outputs are then unspecified and the workspace must be zeroed
+ * again, as after any non-zero device status.
+ */
+typedef struct pa_cache_update {
+  const int64_t* copy_pairs;  /* int64 [num_copy_pairs][2] (src, dst) block ids, device; NULL when 0 */
+  int32_t num_copy_pairs;
+  const void* k;              /* new tokens' keys [num_tokens][num_kv_heads][head_dim], device */
+  const void* v;              /* their values, same layout */
+  const int64_t* slot_mapping; /* int64 [num_tokens], device */
+  int32_t num_tokens;
+} pa_cache_update;
+
+PA_API pa_status pa_decode_update(const pa_cache_update* update, const void* q, void* k_pool, void* v_pool,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                  int32_t num_seqs, int32_t num_q_heads, float scale, void* out, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                                  const pa_decode_opts* opts, void* stream);
+PA_API pa_status pa_decode_multi_update(const pa_cache_update* update, const void* q, void* k_pool, void* v_pool,
+                                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t* seq_lens, int32_t num_seqs, int32_t q_len,
+                                        int32_t num_q_heads, float scale, void* out, void* workspace,
+                                        size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                                        const pa_decode_opts* opts, void* stream);
+PA_API pa_status pa_decode_shared_prefix_update(const pa_cache_update* update, const void* q, void* k_pool,
+                                                void* v_pool, const int32_t* block_tables,
+                                                int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                                int32_t num_seqs, int32_t num_q_heads, const int32_t* group_starts,
+                                                const int32_t* group_prefix_blocks, int32_t num_groups,
+                                                int32_t max_group_size, float scale, void* out, void* workspace,
+                                                size_t workspace_bytes, int32_t* dev_status,
+                                                const pa_pool_desc* pool, const pa_decode_opts* opts,
+                                                void* stream);
 
 /*
  * Host block manager — the bookkeeping half of the method (study notes

@@ -9,6 +9,9 @@ The kernels live in ``libpa.so`` (C ABI: ``include/pa.h``), built in-tree by
 * ``pa_decode_shared_prefix``  decode reading shared prompt blocks once per group
 * ``pa_cache_write``  slot-mapped write of new tokens' K/V
 * ``pa_copy_blocks``  copy-on-write block copies
+* ``pa_decode_update`` (and the ``_multi`` / ``_shared_prefix`` forms) a
+                      step's copies, writes and decode as one call, one
+                      launch on the tensor-core kernel
 * ``PagedDecodeStep`` one whole step (copy, write, decode) from host buffers
 * ``BlockManager``    host block manager (free set, ref counts, copy on write)
 
@@ -21,8 +24,10 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     PA_BF16,
     PA_DECODE_CUDA_CORES_ONLY,
+    PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL,
     PA_DECODE_TEST_WITHHOLD_COPIES,
     PA_FP16,
+    CacheUpdate,
     DecodeOpts,
     PaError,
     PoolDesc,
@@ -40,6 +45,9 @@ from ._lib import (  # noqa: F401
     pa_copy_blocks,
     pa_decode,
     pa_decode_no_alloc,
+    pa_decode_multi_update,
+    pa_decode_shared_prefix_update,
+    pa_decode_update,
     pool_desc,
     status_string,
 )

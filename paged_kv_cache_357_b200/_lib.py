@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libpa.so")
 PA_FP16, PA_BF16 = 0, 1
 PA_DECODE_TEST_WITHHOLD_COPIES = 1
 PA_DECODE_CUDA_CORES_ONLY = 2
+PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL = 4
 DEV_STATUS = {
     0: "PA_DEV_OK",
     101: "PA_DEV_BAD_BLOCK_ID",
@@ -41,6 +42,9 @@ EXPORTED = (
     "pa_shared_prefix_groups",
     "pa_cache_write",
     "pa_copy_blocks",
+    "pa_decode_update",
+    "pa_decode_multi_update",
+    "pa_decode_shared_prefix_update",
     "pa_status_string",
     "pa_bm_create",
     "pa_bm_destroy",
@@ -80,6 +84,17 @@ class PoolDesc(ctypes.Structure):
 
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("num_ctas", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+
+class CacheUpdate(ctypes.Structure):
+    _fields_ = [
+        ("copy_pairs", ctypes.c_void_p),
+        ("num_copy_pairs", ctypes.c_int32),
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("slot_mapping", ctypes.c_void_p),
+        ("num_tokens", ctypes.c_int32),
+    ]
 
 
 class StepShape(ctypes.Structure):
@@ -152,6 +167,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_cache_write.argtypes = [vp, vp, vp, i32, vp, vp, vp, pdesc, vp]
     lib.pa_cache_write.restype = i32
     lib.pa_copy_blocks.argtypes = [vp, i32, vp, vp, vp, pdesc, vp]
+    pupd = ctypes.POINTER(CacheUpdate)
+    lib.pa_decode_update.argtypes = [pupd] + lib.pa_decode_ex.argtypes
+    lib.pa_decode_multi_update.argtypes = [pupd] + lib.pa_decode_multi.argtypes
+    lib.pa_decode_shared_prefix_update.argtypes = [pupd] + lib.pa_decode_shared_prefix.argtypes
+    for name in ("pa_decode_update", "pa_decode_multi_update", "pa_decode_shared_prefix_update"):
+        getattr(lib, name).restype = i32
     lib.pa_copy_blocks.restype = i32
     pshape, playout = ctypes.POINTER(StepShape), ctypes.POINTER(StepLayout)
     vpp = ctypes.POINTER(ctypes.c_void_p)
@@ -484,3 +505,102 @@ def pa_copy_blocks(src_dst_pairs, k_pool, v_pool, dev_status=None, stream=None) 
                                _ptr(dev_status), ctypes.byref(desc), _stream(stream))
     if rc != 0:
         raise PaError(rc, "pa_copy_blocks")
+
+
+# ---------------------------------------------------------------------------
+# a step's cache update and its decode in one call (pa_decode_update & co.)
+# ---------------------------------------------------------------------------
+
+
+def _cache_update(k_pool, copy_pairs, new_k, new_v, slot_mapping) -> CacheUpdate:
+    """The pa_cache_update struct of a step: copy-on-write pairs [n, 2] int64,
+    then new tokens' k, v [T, num_kv_heads, head_dim] into slot_mapping [T]
+    int64; either part may be None."""
+    torch = _torch()
+    dev = k_pool.device
+    upd = CacheUpdate()
+    if copy_pairs is not None:
+        _need(copy_pairs, "copy_pairs", dtype=torch.int64, ndim=2, device=dev)
+        if copy_pairs.shape[1] != 2:
+            raise ValueError("copy_pairs must be [n, 2]")
+        upd.copy_pairs, upd.num_copy_pairs = _ptr(copy_pairs), copy_pairs.shape[0]
+    if (new_k is None) != (new_v is None) or (new_k is None) != (slot_mapping is None):
+        raise ValueError("new_k, new_v and slot_mapping go together")
+    if new_k is not None:
+        _need(new_k, "new_k", dtype=k_pool.dtype, ndim=3, device=dev)
+        _need(new_v, "new_v", dtype=k_pool.dtype, ndim=3, device=dev)
+        _need(slot_mapping, "slot_mapping", dtype=torch.int64, ndim=1, device=dev)
+        T = new_k.shape[0]
+        if new_v.shape != new_k.shape or slot_mapping.shape[0] != T:
+            raise ValueError("new_k, new_v and slot_mapping disagree on the token count")
+        if new_k.shape[1:] != (k_pool.shape[1], k_pool.shape[3]):
+            raise ValueError("new tokens must be [T, num_kv_heads, head_dim]")
+        upd.k, upd.v, upd.slot_mapping, upd.num_tokens = _ptr(new_k), _ptr(new_v), _ptr(slot_mapping), T
+    return upd
+
+
+def pa_decode_update(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, workspace, dev_status=None,
+                     copy_pairs=None, new_k=None, new_v=None, slot_mapping=None, num_ctas: int = 0, flags: int = 0,
+                     stream=None) -> None:
+    """pa_copy_blocks, pa_cache_write and pa_decode as one call
+    (pa_decode_update): one launch where the tensor-core kernel runs."""
+    _check_attention_args(q, k_pool, v_pool, block_tables, seq_lens, out, workspace, dev_status, 3)
+    upd = _cache_update(k_pool, copy_pairs, new_k, new_v, slot_mapping)
+    S, Hq, D = q.shape
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    rc = load().pa_decode_update(
+        ctypes.byref(upd), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(seq_lens), S, Hq, float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(dev_status), ctypes.byref(desc), ctypes.byref(opts), _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode_update")
+
+
+def pa_decode_multi_update(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, workspace, dev_status=None,
+                           copy_pairs=None, new_k=None, new_v=None, slot_mapping=None, num_ctas: int = 0,
+                           flags: int = 0, stream=None) -> None:
+    """pa_copy_blocks, pa_cache_write and pa_decode_multi as one call
+    (pa_decode_multi_update)."""
+    _check_attention_args(q, k_pool, v_pool, block_tables, seq_lens, out, workspace, dev_status, 4)
+    upd = _cache_update(k_pool, copy_pairs, new_k, new_v, slot_mapping)
+    S, L, Hq, D = q.shape
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    rc = load().pa_decode_multi_update(
+        ctypes.byref(upd), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(seq_lens), S, L, Hq, float(scale), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), ctypes.byref(desc), ctypes.byref(opts),
+        _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode_multi_update")
+
+
+def pa_decode_shared_prefix_update(q, k_pool, v_pool, block_tables, seq_lens, group_starts, group_prefix_blocks,
+                                   max_group_size: int, scale: float, out, workspace, dev_status=None,
+                                   copy_pairs=None, new_k=None, new_v=None, slot_mapping=None, num_ctas: int = 0,
+                                   flags: int = 0, stream=None) -> None:
+    """pa_copy_blocks, pa_cache_write and pa_decode_shared_prefix as one call
+    (pa_decode_shared_prefix_update)."""
+    torch = _torch()
+    _check_attention_args(q, k_pool, v_pool, block_tables, seq_lens, out, workspace, dev_status, 3)
+    dev = k_pool.device
+    _need(group_starts, "group_starts", dtype=torch.int32, ndim=1, device=dev)
+    _need(group_prefix_blocks, "group_prefix_blocks", dtype=torch.int32, ndim=1, device=dev)
+    G = group_prefix_blocks.shape[0]
+    if group_starts.shape[0] != G + 1:
+        raise ValueError("group_starts must have num_groups + 1 entries")
+    upd = _cache_update(k_pool, copy_pairs, new_k, new_v, slot_mapping)
+    S, Hq, D = q.shape
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    rc = load().pa_decode_shared_prefix_update(
+        ctypes.byref(upd), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(seq_lens), S, Hq, _ptr(group_starts), _ptr(group_prefix_blocks), G, int(max_group_size), float(scale),
+        _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+        ctypes.byref(desc), ctypes.byref(opts), _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode_shared_prefix_update")

@@ -207,6 +207,7 @@ struct TcSmem {
   int v_consumed;
   int q_issued;
   int q_consumed;
+  uint32_t sync_gen[2];            // generation of each cache-update barrier seen before arriving
 };
 
 template <int R>
@@ -760,6 +761,123 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const int32_t* ptr) {
   return v;
 }
 
+// ---- cache update ahead of the decode (pa_decode_update and friends) --------
+// The step's copy-on-write block copies (study notes ch.05 §6.1) and new
+// tokens' K/V stores (vLLM blog, plain-language section) run inside the
+// decode launch: every thread of every CTA takes a grid-stride share of the
+// 16-byte chunks, and a grid-wide barrier closes each phase, so no TMA load
+// of a block can run ahead of a copy or a store into it.  A barrier slot is
+// two words: an arrival count and a generation number.  Each CTA reads the
+// generation, then arrives; the last arrival resets the count to zero (the
+// workspace is left as it was found) and advances the generation, which is
+// what the waiters watch.  Every CTA of the grid arrives, with or without
+// decode work; the grid is persistent (one CTA per SM), so all of it is
+// resident, and every wait is bounded all the same.
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// One thread per CTA, after a CTA barrier that follows the CTA's stores.
+// Returns the generation to wait past.  The failure-detection test hook
+// keeps CTA 0 from arriving.
+__device__ __forceinline__ uint32_t grid_arrive(int32_t* slot, int test_flags) {
+  __threadfence();
+  fence_proxy_async_global();
+  uint32_t gen;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(slot + 1) : "memory");
+  if ((test_flags & kFlagTestSkipUpdateArrival) && blockIdx.x == 0) return gen;
+  uint32_t prev;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(slot) : "memory");
+  if (prev == gridDim.x - 1) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(slot) : "memory");
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(slot + 1) : "memory");
+  }
+  return gen;
+}
+
+// Bounded wait until the slot's generation moves past `gen`; afterwards the
+// pools' new contents are visible to this thread's TMA loads.
+__device__ __forceinline__ bool grid_wait(const int32_t* slot, uint32_t gen, const volatile int* abort_flag,
+                                          unsigned long long limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_gpu(slot + 1) == gen) {
+    if (*abort_flag != 0 || global_timer_ns() - t0 > limit_ns) return false;
+    __nanosleep(64);
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
+// Copy-on-write: block dst of both pools <- block src, for every pair.  A
+// pair with an id outside the pool is reported and skipped; src == dst is a
+// no-op.  Four chunks are loaded before any is stored (a dst is never a src
+// of the same update).
+template <int NT, int B>
+__device__ void update_copy_blocks(const DecodeParams& p) {
+  const long long cpb = static_cast<long long>(p.num_kv_heads) * B * D / 8;  // chunks per pool block
+  const long long total = static_cast<long long>(p.upd_num_pairs) * 2 * cpb;
+  const long long stride = static_cast<long long>(gridDim.x) * NT;
+  uint4* kp = reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.k_pool));
+  uint4* vp = reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.v_pool));
+  for (long long i0 = static_cast<long long>(blockIdx.x) * NT + threadIdx.x; i0 < total; i0 += 4 * stride) {
+    uint4 val[4];
+    size_t dst[4];
+    uint4* pool[4];
+    bool go[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + u * stride;
+      go[u] = false;
+      if (i >= total) continue;
+      const long long chunk = i % cpb;
+      const long long pw = i / cpb;  // pair * 2 + (0: K, 1: V)
+      const long long src = __ldg(p.upd_pairs + 2 * (pw >> 1)), d = __ldg(p.upd_pairs + 2 * (pw >> 1) + 1);
+      if (src < 0 || src >= p.num_blocks || d < 0 || d >= p.num_blocks) {
+        if (chunk == 0 && (pw & 1) == 0) record_status(p.status, PA_DEV_BAD_PAIR);
+        continue;
+      }
+      if (src == d) continue;
+      pool[u] = (pw & 1) ? vp : kp;
+      dst[u] = static_cast<size_t>(d) * cpb + chunk;
+      val[u] = pool[u][static_cast<size_t>(src) * cpb + chunk];
+      go[u] = true;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (go[u]) pool[u][dst[u]] = val[u];
+    }
+  }
+}
+
+// New tokens: chunk i of k/v ([T][Hkv][D], D / 8 chunks a row) goes to row
+// slot % B of block slot / B, same kv head.  A negative slot is a padding
+// token (skipped); a slot past the pool is reported and skipped.
+template <int NT, int B>
+__device__ void update_write_slots(const DecodeParams& p) {
+  constexpr int CPR = D / 8;
+  const int Hkv = p.num_kv_heads;
+  const long long total = static_cast<long long>(p.upd_num_tokens) * Hkv * CPR;
+  const long long num_slots = static_cast<long long>(p.num_blocks) * B;
+  const long long stride = static_cast<long long>(gridDim.x) * NT;
+  uint4* kp = reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.k_pool));
+  uint4* vp = reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.v_pool));
+  for (long long i = static_cast<long long>(blockIdx.x) * NT + threadIdx.x; i < total; i += stride) {
+    const int chunk = static_cast<int>(i % CPR);
+    const long long th = i / CPR;  // token * Hkv + head
+    const int h = static_cast<int>(th % Hkv);
+    const long long slot = __ldg(p.upd_slots + th / Hkv);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (chunk == 0 && h == 0) record_status(p.status, PA_DEV_BAD_SLOT);
+      continue;
+    }
+    const size_t dst = (static_cast<size_t>((slot / B) * Hkv + h) * B + slot % B) * CPR + chunk;
+    kp[dst] = __ldg(p.upd_k + i);
+    vp[dst] = __ldg(p.upd_v + i);
+  }
+}
+
 // Spin (bounded by limit_ns) until bits [shift, shift + 16) of *counter
 // reach `need`.
 __device__ __forceinline__ bool wait_arrivals(const int32_t* counter, int shift, uint32_t need,
@@ -849,6 +967,14 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   // ---- inputs may come from the previous kernel in the stream
   grid_dependency_wait();
   grid_launch_dependents();
+  // Cache update, phase 1: block copies, whose barrier the partition
+  // prologue below hides.
+  const bool upd_copy = p.upd_num_pairs > 0, upd_write = p.upd_num_tokens > 0;
+  if (upd_copy) {
+    update_copy_blocks<kThreads, B>(p);
+    __syncthreads();
+    if (tid == 0) sm.sync_gen[0] = grid_arrive(p.grid_sync, p.test_flags);
+  }
   if constexpr (kMode == kGroup) {
     group_bookkeeping<RG, B>(p, src);
   } else {
@@ -857,6 +983,22 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   WorkRange wr;
   Cursor cur;
   const bool has_work = decode_prologue<kThreads, B, CB>(p, sm.range, wr, cur, src);  // uniform across the CTA
+  // Phase 2: the new tokens' stores, once every copy has landed (a token may
+  // go into a block just copied).  The producers wait for the last phase's
+  // barrier before their first K or V load; a timed-out wait aborts the CTA.
+  if (upd_copy) {
+    if (tid == 0 && !grid_wait(p.grid_sync, sm.sync_gen[0], abort_flag, p.wait_limit_ns)) {
+      sm.abort = 1;
+      record_status(p.status, PA_DEV_TIMEOUT);
+    }
+    __syncthreads();
+  }
+  if (upd_write) {
+    if (*abort_flag == 0) update_write_slots<kThreads, B>(p);
+    __syncthreads();
+    if (tid == 0) sm.sync_gen[1] = grid_arrive(p.grid_sync + 32, p.test_flags);
+    __syncthreads();
+  }
 
   if (!has_work) {
     // nothing to stream: straight to teardown
@@ -872,6 +1014,9 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     const uint64_t pol_keep = l2_policy_evict_last();
     bool ok = true;
     int ci = 0, qi = 0, k_issued = 0, v_issued = 0, q_issued = 0;
+    // The first K or V load waits (again, in this thread, so that its proxy
+    // fence orders the TMA reads) for the last barrier of the cache update.
+    bool gated = upd_write || upd_copy;
     if (p.test_flags & kFlagTestWithholdCopies) {
       if (lane == 0) {
         const uint64_t t0 = global_timer_ns();
@@ -910,7 +1055,12 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           const int y = (e * Hkv + sg.h) * B;
           bool go = true;
           if (lane == 0) {
-            go = mbar_wait_bounded(empty, ((ci / ns) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
+            if (gated) {
+              go = grid_wait(p.grid_sync + (upd_write ? 32 : 0), sm.sync_gen[upd_write ? 1 : 0], abort_flag,
+                             p.wait_limit_ns);
+              gated = false;
+            }
+            if (go) go = mbar_wait_bounded(empty, ((ci / ns) & 1) ^ 1u, abort_flag, p.wait_limit_ns);
             if (go) mbar_arrive_expect_tx(full, nblk * Bk::kVBlockBytes);
           }
           if (!__shfl_sync(0xffffffffu, go, 0)) return false;
@@ -1679,7 +1829,7 @@ Variant tc_variant() {
   static_assert(smem_bytes<R>() <= kMaxSmemPerCta, "shared memory of one CTA");
   return Variant{reinterpret_cast<const void*>(&pa_decode_tc_kernel<kBf16, G, RG, kMode, B>), Rows<R>::kThreads,
                  smem_bytes<R>(), Rows<R>::kPartStride, &launch_tc<kBf16, G, RG, kMode, B>,
-                 unit_finish_cost(kMode, R)};
+                 unit_finish_cost(kMode, R), true};
 }
 
 // head_dim 128, a 16-bit pool, and a block size the instances cover: 8, 16

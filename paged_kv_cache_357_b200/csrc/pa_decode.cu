@@ -527,9 +527,10 @@ static size_t partials_bytes(int ctas, int part_stride) {
   return align_up(static_cast<size_t>(ctas) * 2 * part_stride * sizeof(float), 256);
 }
 
+// [partial states][grid barrier words][arrival counters]
 static size_t workspace_bytes_for(int num_seqs, int num_kv_heads, int ctas, int part_stride) {
   const size_t counters = align_up(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t), 256);
-  return partials_bytes(ctas, part_stride) + counters;
+  return partials_bytes(ctas, part_stride) + kGridSyncBytes + counters;
 }
 
 static bool pool_shape_ok(const pa_pool_desc* pool) {
@@ -548,7 +549,8 @@ static int resolve_ctas(const Variant& v, const pa_decode_opts* opts) {
 
 static int opts_flags(const pa_decode_opts* opts) { return opts != nullptr ? opts->flags : 0; }
 
-constexpr int kKnownFlags = PA_DECODE_TEST_WITHHOLD_COPIES | PA_DECODE_CUDA_CORES_ONLY;
+constexpr int kKnownFlags =
+    PA_DECODE_TEST_WITHHOLD_COPIES | PA_DECODE_CUDA_CORES_ONLY | PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL;
 
 // Shared argument checks of the decode entry points.
 static pa_status check_decode_args(const void* q, const void* k_pool, const void* v_pool,
@@ -582,7 +584,8 @@ static DecodeParams make_params(const void* q, const void* k_pool, const void* v
   prm.seq_lens = seq_lens;
   prm.out = static_cast<uint16_t*>(out);
   prm.partials = static_cast<float*>(scratch);
-  prm.counters = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + partials_bytes(ctas, part_stride));
+  prm.grid_sync = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + partials_bytes(ctas, part_stride));
+  prm.counters = prm.grid_sync + kGridSyncBytes / sizeof(int32_t);
   prm.status = dev_status;
   prm.max_nb = max_blocks_per_seq;
   prm.num_seqs = num_seqs;
@@ -590,16 +593,79 @@ static DecodeParams make_params(const void* q, const void* k_pool, const void* v
   prm.num_kv_heads = pool->num_kv_heads;
   prm.num_blocks = pool->num_blocks;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  const bool test_timeout = (flags & PA_DECODE_TEST_WITHHOLD_COPIES) != 0;
-  prm.wait_limit_ns = test_timeout ? 20ull * 1000 * 1000 : 2ull * 1000 * 1000 * 1000;
-  prm.test_flags = test_timeout ? kFlagTestWithholdCopies : 0;
+  const int test_flags = flags & (PA_DECODE_TEST_WITHHOLD_COPIES | PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL);
+  prm.wait_limit_ns = test_flags != 0 ? 20ull * 1000 * 1000 : 2ull * 1000 * 1000 * 1000;
+  prm.test_flags = test_flags;
   prm.q_len = 1;
   prm.q_tiles = 1;
   prm.group_starts = nullptr;
   prm.group_prefix = nullptr;
   prm.num_groups = 0;
   prm.unit_cost = 0;
+  prm.upd_pairs = nullptr;
+  prm.upd_num_pairs = 0;
+  prm.upd_k = nullptr;
+  prm.upd_v = nullptr;
+  prm.upd_slots = nullptr;
+  prm.upd_num_tokens = 0;
   return prm;
+}
+
+// ---- cache update ahead of a decode (pa_decode_update and friends) -----------
+
+static bool has_update(const pa_cache_update* u) {
+  return u != nullptr && (u->num_copy_pairs > 0 || u->num_tokens > 0);
+}
+
+static bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+// Host-visible checks of an update (NULL is no update).
+static bool update_args_ok(const pa_cache_update* u) {
+  if (u == nullptr) return true;
+  if (u->num_copy_pairs < 0 || u->num_tokens < 0) return false;
+  if (u->num_copy_pairs > 0 && (u->copy_pairs == nullptr || !aligned8(u->copy_pairs))) return false;
+  if (u->num_tokens > 0 && (u->k == nullptr || u->v == nullptr || u->slot_mapping == nullptr ||
+                            !aligned16(u->k) || !aligned16(u->v) || !aligned8(u->slot_mapping))) {
+    return false;
+  }
+  return true;
+}
+
+// The update as its own two kernels, enqueued before the decode.
+static pa_status enqueue_update(const pa_cache_update* u, void* k_pool, void* v_pool, int32_t* dev_status,
+                                const pa_pool_desc* pool, void* stream) {
+  if (!has_update(u)) return PA_OK;
+  pa_status st = PA_OK;
+  if (u->num_copy_pairs > 0) st = pa_copy_blocks(u->copy_pairs, u->num_copy_pairs, k_pool, v_pool, dev_status, pool, stream);
+  if (st == PA_OK && u->num_tokens > 0) {
+    st = pa_cache_write(u->k, u->v, u->slot_mapping, u->num_tokens, k_pool, v_pool, dev_status, pool, stream);
+  }
+  return st;
+}
+
+// Launch a decode variant, with the update inside its launch where the
+// variant runs one and the whole grid can be resident at once (its
+// grid-wide barriers need every CTA on an SM), else after the update's own
+// kernels.
+static pa_status launch_decode(const Variant& v, DecodeParams& prm, int ctas, const pa_cache_update* u,
+                               void* k_pool, void* v_pool, const pa_pool_desc* pool, void* stream) {
+  if (has_update(u)) {
+    int resident = 0;
+    if (v.fuses_update && grid_size_for(v, resident) && ctas <= resident) {
+      prm.upd_pairs = u->num_copy_pairs > 0 ? u->copy_pairs : nullptr;
+      prm.upd_num_pairs = u->num_copy_pairs;
+      if (u->num_tokens > 0) {
+        prm.upd_k = static_cast<const uint4*>(u->k);
+        prm.upd_v = static_cast<const uint4*>(u->v);
+        prm.upd_slots = u->slot_mapping;
+        prm.upd_num_tokens = u->num_tokens;
+      }
+    } else {
+      const pa_status st = enqueue_update(u, k_pool, v_pool, prm.status, pool, stream);
+      if (st != PA_OK) return st;
+    }
+  }
+  return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // CTA count for a workspace-size query: an explicit request needs no device.
@@ -664,14 +730,16 @@ extern "C" size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_head
   return pa_decode_workspace_bytes_ex(num_seqs, num_q_heads, pool, nullptr);
 }
 
-extern "C" pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_pool,
-                                  const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
-                                  int32_t num_seqs, int32_t num_q_heads, float scale, void* out, void* workspace,
-                                  size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
-                                  const pa_decode_opts* opts, void* stream) {
+static pa_status decode_impl(const pa_cache_update* upd, const void* q, const void* k_pool, const void* v_pool,
+                             const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                             int32_t num_seqs, int32_t num_q_heads, float scale, void* out, void* workspace,
+                             size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                             const pa_decode_opts* opts, void* stream) {
   pa_status st = check_decode_args(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                                     num_q_heads, scale, out, pool);
-  if (st != PA_OK || num_seqs == 0) return st;
+  if (st != PA_OK) return st;
+  if (!update_args_ok(upd)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return enqueue_update(upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), dev_status, pool, stream);
   if (opts != nullptr && (opts->num_ctas < 0 || (opts->flags & ~kKnownFlags) != 0)) return PA_ERR_INVALID_ARG;
   Variant v;
   if (!select_variant(*pool, num_q_heads, opts_flags(opts), v)) return PA_ERR_UNSUPPORTED;
@@ -683,7 +751,25 @@ extern "C" pa_status pa_decode_ex(const void* q, const void* k_pool, const void*
                                        num_q_heads, scale, out, workspace, ctas, v.part_stride, dev_status, pool,
                                        opts_flags(opts));
   prm.unit_cost = v.unit_cost;
-  return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return launch_decode(v, prm, ctas, upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), pool, stream);
+}
+
+extern "C" pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_pool,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                  int32_t num_seqs, int32_t num_q_heads, float scale, void* out, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                                  const pa_decode_opts* opts, void* stream) {
+  return decode_impl(nullptr, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                     scale, out, workspace, workspace_bytes, dev_status, pool, opts, stream);
+}
+
+extern "C" pa_status pa_decode_update(const pa_cache_update* update, const void* q, void* k_pool, void* v_pool,
+                                      const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
+                                      void* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                      const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream) {
+  return decode_impl(update, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                     scale, out, workspace, workspace_bytes, dev_status, pool, opts, stream);
 }
 
 extern "C" pa_status pa_decode(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
@@ -705,20 +791,21 @@ extern "C" size_t pa_decode_multi_workspace_bytes(int32_t num_seqs, int32_t q_le
   return workspace_bytes_for(num_seqs * tiles, pool->num_kv_heads, ctas, v.part_stride);
 }
 
-extern "C" pa_status pa_decode_multi(const void* q, const void* k_pool, const void* v_pool,
-                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
-                                     const int32_t* seq_lens, int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
-                                     float scale, void* out, void* workspace, size_t workspace_bytes,
-                                     int32_t* dev_status, const pa_pool_desc* pool, const pa_decode_opts* opts,
-                                     void* stream) {
+static pa_status multi_impl(const pa_cache_update* upd, const void* q, const void* k_pool, const void* v_pool,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                            int32_t num_seqs, int32_t q_len, int32_t num_q_heads, float scale, void* out,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                            const pa_decode_opts* opts, void* stream) {
   if (q_len < 1) return PA_ERR_INVALID_ARG;
   if (q_len == 1) {
-    return pa_decode_ex(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
-                        scale, out, workspace, workspace_bytes, dev_status, pool, opts, stream);
+    return decode_impl(upd, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                       scale, out, workspace, workspace_bytes, dev_status, pool, opts, stream);
   }
   pa_status st = check_decode_args(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                                     num_q_heads, scale, out, pool);
-  if (st != PA_OK || num_seqs == 0) return st;
+  if (st != PA_OK) return st;
+  if (!update_args_ok(upd)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return enqueue_update(upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), dev_status, pool, stream);
   if (!opts_ok(opts)) return PA_ERR_INVALID_ARG;
   if (static_cast<long long>(num_seqs) * q_len > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
   if ((opts_flags(opts) & PA_DECODE_CUDA_CORES_ONLY) != 0) return PA_ERR_UNSUPPORTED;
@@ -735,7 +822,27 @@ extern "C" pa_status pa_decode_multi(const void* q, const void* k_pool, const vo
   prm.q_len = q_len;
   prm.q_tiles = tiles;
   prm.unit_cost = v.unit_cost;
-  return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return launch_decode(v, prm, ctas, upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), pool, stream);
+}
+
+extern "C" pa_status pa_decode_multi(const void* q, const void* k_pool, const void* v_pool,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* seq_lens, int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                     float scale, void* out, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, const pa_pool_desc* pool, const pa_decode_opts* opts,
+                                     void* stream) {
+  return multi_impl(nullptr, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, q_len,
+                    num_q_heads, scale, out, workspace, workspace_bytes, dev_status, pool, opts, stream);
+}
+
+extern "C" pa_status pa_decode_multi_update(const pa_cache_update* update, const void* q, void* k_pool,
+                                            void* v_pool, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                            const int32_t* seq_lens, int32_t num_seqs, int32_t q_len,
+                                            int32_t num_q_heads, float scale, void* out, void* workspace,
+                                            size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                                            const pa_decode_opts* opts, void* stream) {
+  return multi_impl(update, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, q_len,
+                    num_q_heads, scale, out, workspace, workspace_bytes, dev_status, pool, opts, stream);
 }
 
 extern "C" size_t pa_decode_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t max_group_size,
@@ -748,20 +855,21 @@ extern "C" size_t pa_decode_shared_prefix_workspace_bytes(int32_t num_seqs, int3
   return workspace_bytes_for(num_seqs, pool->num_kv_heads, ctas, v.part_stride);
 }
 
-extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
-                                             const int32_t* block_tables, int32_t max_blocks_per_seq,
-                                             const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
-                                             const int32_t* group_starts, const int32_t* group_prefix_blocks,
-                                             int32_t num_groups, int32_t max_group_size, float scale, void* out,
-                                             void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                                             const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream) {
+static pa_status shared_prefix_impl(const pa_cache_update* upd, const void* q, const void* k_pool,
+                                    const void* v_pool, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                                    const int32_t* group_starts, const int32_t* group_prefix_blocks,
+                                    int32_t num_groups, int32_t max_group_size, float scale, void* out,
+                                    void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                    const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream) {
   pa_status st = check_decode_args(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                                     num_q_heads, scale, out, pool);
   if (st != PA_OK) return st;
   if (num_groups < 0 || max_group_size < 1 || (num_seqs > 0 && num_groups == 0) || num_groups > num_seqs) {
     return PA_ERR_INVALID_ARG;
   }
-  if (num_seqs == 0) return PA_OK;
+  if (!update_args_ok(upd)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return enqueue_update(upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), dev_status, pool, stream);
   if (group_starts == nullptr || group_prefix_blocks == nullptr) return PA_ERR_INVALID_ARG;
   if (!opts_ok(opts)) return PA_ERR_INVALID_ARG;
   if ((opts_flags(opts) & PA_DECODE_CUDA_CORES_ONLY) != 0) return PA_ERR_UNSUPPORTED;
@@ -778,7 +886,33 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* k_pool, 
   prm.group_prefix = group_prefix_blocks;
   prm.num_groups = num_groups;
   prm.unit_cost = v.unit_cost;
-  return v.launch(v, prm, ctas, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return launch_decode(v, prm, ctas, upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), pool, stream);
+}
+
+extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
+                                             const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                             const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                                             const int32_t* group_starts, const int32_t* group_prefix_blocks,
+                                             int32_t num_groups, int32_t max_group_size, float scale, void* out,
+                                             void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                             const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream) {
+  return shared_prefix_impl(nullptr, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                            num_q_heads, group_starts, group_prefix_blocks, num_groups, max_group_size, scale, out,
+                            workspace, workspace_bytes, dev_status, pool, opts, stream);
+}
+
+extern "C" pa_status pa_decode_shared_prefix_update(const pa_cache_update* update, const void* q, void* k_pool,
+                                                    void* v_pool, const int32_t* block_tables,
+                                                    int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                                    int32_t num_seqs, int32_t num_q_heads,
+                                                    const int32_t* group_starts, const int32_t* group_prefix_blocks,
+                                                    int32_t num_groups, int32_t max_group_size, float scale,
+                                                    void* out, void* workspace, size_t workspace_bytes,
+                                                    int32_t* dev_status, const pa_pool_desc* pool,
+                                                    const pa_decode_opts* opts, void* stream) {
+  return shared_prefix_impl(update, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                            num_q_heads, group_starts, group_prefix_blocks, num_groups, max_group_size, scale, out,
+                            workspace, workspace_bytes, dev_status, pool, opts, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -119,39 +119,41 @@ struct pa_step {
   }
 
   // The step's kernels on `stream` with set k's buffers (checked by the
-  // entry points themselves).
+  // entry points themselves): the copies and stores of the cache update and
+  // the decode, in one launch where the decode's kernel takes them in.
   pa_status launch(int k, int pairs, int tokens, int groups, cudaStream_t stream) const {
     const char* in = static_cast<const char*>(din[k]);
     const pa_step_layout& L = layout;
-    pa_status st = PA_OK;
+    pa_cache_update upd{};
     if (pairs > 0) {
-      st = pa_copy_blocks(reinterpret_cast<const int64_t*>(in + L.copy_pairs), pairs, k_pool, v_pool, status, &pool,
-                          stream);
-      if (st != PA_OK) return st;
+      upd.copy_pairs = reinterpret_cast<const int64_t*>(in + L.copy_pairs);
+      upd.num_copy_pairs = pairs;
     }
     if (tokens > 0) {
-      st = pa_cache_write(in + L.new_k, in + L.new_v, reinterpret_cast<const int64_t*>(in + L.slot_mapping), tokens,
-                          k_pool, v_pool, status, &pool, stream);
-      if (st != PA_OK) return st;
+      upd.k = in + L.new_k;
+      upd.v = in + L.new_v;
+      upd.slot_mapping = reinterpret_cast<const int64_t*>(in + L.slot_mapping);
+      upd.num_tokens = tokens;
     }
     const auto* tables = reinterpret_cast<const int32_t*>(in + L.block_tables);
     const auto* lens = reinterpret_cast<const int32_t*>(in + L.seq_lens);
     const pa_step_shape& sh = shape;
     switch (sh.kind) {
       case PA_STEP_MULTI:
-        return pa_decode_multi(in + L.q, k_pool, v_pool, tables, sh.max_blocks_per_seq, lens, sh.num_seqs, sh.q_len,
-                               sh.num_q_heads, sh.scale, dout[k], workspace, workspace_bytes, status, &pool,
-                               &sh.opts, stream);
+        return pa_decode_multi_update(&upd, in + L.q, k_pool, v_pool, tables, sh.max_blocks_per_seq, lens,
+                                      sh.num_seqs, sh.q_len, sh.num_q_heads, sh.scale, dout[k], workspace,
+                                      workspace_bytes, status, &pool, &sh.opts, stream);
       case PA_STEP_SHARED_PREFIX:
-        return pa_decode_shared_prefix(in + L.q, k_pool, v_pool, tables, sh.max_blocks_per_seq, lens, sh.num_seqs,
-                                       sh.num_q_heads, reinterpret_cast<const int32_t*>(in + L.group_starts),
-                                       reinterpret_cast<const int32_t*>(in + L.group_prefix_blocks), groups,
-                                       sh.max_group_size, sh.scale, dout[k], workspace, workspace_bytes, status,
-                                       &pool, &sh.opts, stream);
+        return pa_decode_shared_prefix_update(&upd, in + L.q, k_pool, v_pool, tables, sh.max_blocks_per_seq, lens,
+                                              sh.num_seqs, sh.num_q_heads,
+                                              reinterpret_cast<const int32_t*>(in + L.group_starts),
+                                              reinterpret_cast<const int32_t*>(in + L.group_prefix_blocks), groups,
+                                              sh.max_group_size, sh.scale, dout[k], workspace, workspace_bytes,
+                                              status, &pool, &sh.opts, stream);
       default:
-        return pa_decode_ex(in + L.q, k_pool, v_pool, tables, sh.max_blocks_per_seq, lens, sh.num_seqs,
-                            sh.num_q_heads, sh.scale, dout[k], workspace, workspace_bytes, status, &pool, &sh.opts,
-                            stream);
+        return pa_decode_update(&upd, in + L.q, k_pool, v_pool, tables, sh.max_blocks_per_seq, lens, sh.num_seqs,
+                                sh.num_q_heads, sh.scale, dout[k], workspace, workspace_bytes, status, &pool,
+                                &sh.opts, stream);
     }
   }
 
