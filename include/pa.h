@@ -101,8 +101,8 @@ typedef struct pa_decode_opts {
 #define PA_DECODE_CUDA_CORES_ONLY 2
 
 /* Failure-detection test hook for the *_update entry points: CTA 0 of the
- * tensor-core kernel never arrives at the cache update's grid-wide
- * barriers, so every wait for them runs out after about 20 ms and the
+ * tensor-core kernel never arrives at the new tokens' grid-wide barrier,
+ * so every wait for it runs out after about 20 ms and the
  * kernel returns early with PA_DEV_TIMEOUT (pools and outputs unspecified,
  * the workspace to be zeroed again).  Never set it outside such tests. */
 #define PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL 4
@@ -313,12 +313,13 @@ PA_API pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs,
                          int32_t* dev_status, const pa_pool_desc* pool, void* stream);
 
 /*
- * One decode step's cache update followed by its attention, in one launch
- * where the tensor-core kernel runs.  A serving step first copies the
- * blocks that copy on write gives a writer (study notes ch.05 §6.1), then
- * stores each new token's K/V in its slot (vLLM blog, plain-language
- * section), then attends over the cache that now holds it (vLLM blog
- * §"关键细节" 2).  These entry points take the three as one call:
+ * One decode step's cache update followed by its attention, the new tokens'
+ * stores inside the decode's launch where the tensor-core kernel runs.  A
+ * serving step first copies the blocks that copy on write gives a writer
+ * (study notes ch.05 §6.1), then stores each new token's K/V in its slot
+ * (vLLM blog, plain-language section), then attends over the cache that now
+ * holds it (vLLM blog §"关键细节" 2).  These entry points take the three as
+ * one call:
  *
  *   pa_copy_blocks(update->copy_pairs, ...);
  *   pa_cache_write(update->k, update->v, update->slot_mapping, ...);
@@ -326,13 +327,15 @@ PA_API pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs,
  *
  * with the same results (pools bit for bit, outputs within the decode
  * tolerance) and the same device errors.  The pool pointers are written.
- * Where the tensor-core kernel runs (head_dim 128, 16-bit pools, the shapes
- * listed for each decode), the copies and stores run inside its launch: all
+ * Where the tensor-core decode kernel runs (head_dim 128, 16-bit pools, the
+ * shapes listed for each decode; not the query-major prefill kernel) and
+ * the grid fits on the GPU at once, the stores run inside its launch: all
  * CTAs take a share of them at the start, and a grid-wide barrier (an
  * arrival count and a generation word in the workspace, every wait bounded)
- * holds back every K/V load until the last store has landed.  This saves
- * the two small launches and their gaps per step.  Elsewhere the three
- * kernels are enqueued in order on `stream`.
+ * holds back every K/V load until the last store has landed.  That saves a
+ * launch per step.  The block copies always run as pa_copy_blocks' own
+ * kernel ahead of the decode: inside the launch they measured slower.
+ * Elsewhere the three kernels are enqueued in order on `stream`.
  *
  * update == NULL, or both counts 0, is the plain decode.  copy_pairs and
  * slot_mapping follow pa_copy_blocks and pa_cache_write (pairs run in

@@ -207,7 +207,7 @@ struct TcSmem {
   int v_consumed;
   int q_issued;
   int q_consumed;
-  uint32_t sync_gen[2];            // generation of each cache-update barrier seen before arriving
+  uint32_t sync_gen;               // generation of the new-token barrier seen before arriving
 };
 
 template <int R>
@@ -761,18 +761,17 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const int32_t* ptr) {
   return v;
 }
 
-// ---- cache update ahead of the decode (pa_decode_update and friends) --------
-// The step's copy-on-write block copies (study notes ch.05 §6.1) and new
-// tokens' K/V stores (vLLM blog, plain-language section) run inside the
-// decode launch: every thread of every CTA takes a grid-stride share of the
-// 16-byte chunks, and a grid-wide barrier closes each phase, so no TMA load
-// of a block can run ahead of a copy or a store into it.  A barrier slot is
+// ---- new tokens' stores ahead of the decode (pa_decode_update and friends) ---
+// The step's new-token K/V stores (vLLM blog, plain-language section) run
+// inside the decode launch: every thread of every CTA takes a grid-stride
+// share of the 16-byte chunks, and a grid-wide barrier closes the phase, so
+// no TMA load of a block can run ahead of a store into it.  The barrier is
 // two words: an arrival count and a generation number.  Each CTA reads the
 // generation, then arrives; the last arrival resets the count to zero (the
 // workspace is left as it was found) and advances the generation, which is
 // what the waiters watch.  Every CTA of the grid arrives, with or without
-// decode work; the grid is persistent (one CTA per SM), so all of it is
-// resident, and every wait is bounded all the same.
+// decode work; the host launches this form only when the whole grid is
+// resident at once, and every wait is bounded all the same.
 
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -807,47 +806,6 @@ __device__ __forceinline__ bool grid_wait(const int32_t* slot, uint32_t gen, con
   }
   fence_proxy_async_global();
   return true;
-}
-
-// Copy-on-write: block dst of both pools <- block src, for every pair.  A
-// pair with an id outside the pool is reported and skipped; src == dst is a
-// no-op.  Four chunks are loaded before any is stored (a dst is never a src
-// of the same update).
-template <int NT, int B>
-__device__ void update_copy_blocks(const DecodeParams& p) {
-  const long long cpb = static_cast<long long>(p.num_kv_heads) * B * D / 8;  // chunks per pool block
-  const long long total = static_cast<long long>(p.upd_num_pairs) * 2 * cpb;
-  const long long stride = static_cast<long long>(gridDim.x) * NT;
-  uint4* kp = reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.k_pool));
-  uint4* vp = reinterpret_cast<uint4*>(const_cast<uint16_t*>(p.v_pool));
-  for (long long i0 = static_cast<long long>(blockIdx.x) * NT + threadIdx.x; i0 < total; i0 += 4 * stride) {
-    uint4 val[4];
-    size_t dst[4];
-    uint4* pool[4];
-    bool go[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const long long i = i0 + u * stride;
-      go[u] = false;
-      if (i >= total) continue;
-      const long long chunk = i % cpb;
-      const long long pw = i / cpb;  // pair * 2 + (0: K, 1: V)
-      const long long src = __ldg(p.upd_pairs + 2 * (pw >> 1)), d = __ldg(p.upd_pairs + 2 * (pw >> 1) + 1);
-      if (src < 0 || src >= p.num_blocks || d < 0 || d >= p.num_blocks) {
-        if (chunk == 0 && (pw & 1) == 0) record_status(p.status, PA_DEV_BAD_PAIR);
-        continue;
-      }
-      if (src == d) continue;
-      pool[u] = (pw & 1) ? vp : kp;
-      dst[u] = static_cast<size_t>(d) * cpb + chunk;
-      val[u] = pool[u][static_cast<size_t>(src) * cpb + chunk];
-      go[u] = true;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (go[u]) pool[u][dst[u]] = val[u];
-    }
-  }
 }
 
 // New tokens: chunk i of k/v ([T][Hkv][D], D / 8 chunks a row) goes to row
@@ -967,13 +925,14 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   // ---- inputs may come from the previous kernel in the stream
   grid_dependency_wait();
   grid_launch_dependents();
-  // Cache update, phase 1: block copies, whose barrier the partition
-  // prologue below hides.
-  const bool upd_copy = p.upd_num_pairs > 0, upd_write = p.upd_num_tokens > 0;
-  if (upd_copy) {
-    update_copy_blocks<kThreads, B>(p);
+  // The step's new tokens, stored before the partition prologue so that the
+  // prologue hides the barrier; the producers wait for it before their first
+  // K or V load.
+  const bool upd_write = p.upd_num_tokens > 0;
+  if (upd_write) {
+    update_write_slots<kThreads, B>(p);
     __syncthreads();
-    if (tid == 0) sm.sync_gen[0] = grid_arrive(p.grid_sync, p.test_flags);
+    if (tid == 0) sm.sync_gen = grid_arrive(p.grid_sync, p.test_flags);
   }
   if constexpr (kMode == kGroup) {
     group_bookkeeping<RG, B>(p, src);
@@ -983,22 +942,6 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
   WorkRange wr;
   Cursor cur;
   const bool has_work = decode_prologue<kThreads, B, CB>(p, sm.range, wr, cur, src);  // uniform across the CTA
-  // Phase 2: the new tokens' stores, once every copy has landed (a token may
-  // go into a block just copied).  The producers wait for the last phase's
-  // barrier before their first K or V load; a timed-out wait aborts the CTA.
-  if (upd_copy) {
-    if (tid == 0 && !grid_wait(p.grid_sync, sm.sync_gen[0], abort_flag, p.wait_limit_ns)) {
-      sm.abort = 1;
-      record_status(p.status, PA_DEV_TIMEOUT);
-    }
-    __syncthreads();
-  }
-  if (upd_write) {
-    if (*abort_flag == 0) update_write_slots<kThreads, B>(p);
-    __syncthreads();
-    if (tid == 0) sm.sync_gen[1] = grid_arrive(p.grid_sync + 32, p.test_flags);
-    __syncthreads();
-  }
 
   if (!has_work) {
     // nothing to stream: straight to teardown
@@ -1014,9 +957,9 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
     const uint64_t pol_keep = l2_policy_evict_last();
     bool ok = true;
     int ci = 0, qi = 0, k_issued = 0, v_issued = 0, q_issued = 0;
-    // The first K or V load waits (again, in this thread, so that its proxy
-    // fence orders the TMA reads) for the last barrier of the cache update.
-    bool gated = upd_write || upd_copy;
+    // The first K or V load waits for the stores' barrier (in this thread,
+    // so that its proxy fence orders the TMA reads).
+    bool gated = upd_write;
     if (p.test_flags & kFlagTestWithholdCopies) {
       if (lane == 0) {
         const uint64_t t0 = global_timer_ns();
@@ -1056,8 +999,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           bool go = true;
           if (lane == 0) {
             if (gated) {
-              go = grid_wait(p.grid_sync + (upd_write ? 32 : 0), sm.sync_gen[upd_write ? 1 : 0], abort_flag,
-                             p.wait_limit_ns);
+              go = grid_wait(p.grid_sync, sm.sync_gen, abort_flag, p.wait_limit_ns);
               gated = false;
             }
             if (go) go = mbar_wait_bounded(empty, ((ci / ns) & 1) ^ 1u, abort_flag, p.wait_limit_ns);

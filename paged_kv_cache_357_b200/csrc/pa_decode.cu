@@ -602,8 +602,6 @@ static DecodeParams make_params(const void* q, const void* k_pool, const void* v
   prm.group_prefix = nullptr;
   prm.num_groups = 0;
   prm.unit_cost = 0;
-  prm.upd_pairs = nullptr;
-  prm.upd_num_pairs = 0;
   prm.upd_k = nullptr;
   prm.upd_v = nullptr;
   prm.upd_slots = nullptr;
@@ -643,17 +641,22 @@ static pa_status enqueue_update(const pa_cache_update* u, void* k_pool, void* v_
   return st;
 }
 
-// Launch a decode variant, with the update inside its launch where the
-// variant runs one and the whole grid can be resident at once (its
-// grid-wide barriers need every CTA on an SM), else after the update's own
-// kernels.
+// Launch a decode variant after the update.  The block copies run as their
+// own kernel ahead of it (inside the decode launch they measured slower:
+// one CTA per SM keeps fewer copies in flight, and their barrier delayed
+// every CTA's first load).  The new tokens' stores run inside the launch
+// where the variant takes them and the whole grid can be resident at once
+// (its grid-wide barrier needs every CTA on an SM), else as pa_cache_write.
 static pa_status launch_decode(const Variant& v, DecodeParams& prm, int ctas, const pa_cache_update* u,
                                void* k_pool, void* v_pool, const pa_pool_desc* pool, void* stream) {
   if (has_update(u)) {
     int resident = 0;
     if (v.fuses_update && grid_size_for(v, resident) && ctas <= resident) {
-      prm.upd_pairs = u->num_copy_pairs > 0 ? u->copy_pairs : nullptr;
-      prm.upd_num_pairs = u->num_copy_pairs;
+      if (u->num_copy_pairs > 0) {
+        const pa_status st =
+            pa_copy_blocks(u->copy_pairs, u->num_copy_pairs, k_pool, v_pool, prm.status, pool, stream);
+        if (st != PA_OK) return st;
+      }
       if (u->num_tokens > 0) {
         prm.upd_k = static_cast<const uint4*>(u->k);
         prm.upd_v = static_cast<const uint4*>(u->v);

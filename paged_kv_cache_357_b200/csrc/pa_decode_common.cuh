@@ -62,12 +62,9 @@ struct DecodeParams {
   int num_groups;
   // partition cost of finishing a unit, in 1/kGranuleCost granules
   int unit_cost;
-  // cache update run by the tensor-core kernel before it reads the pools
-  // (null / 0 for none): copy-on-write block pairs first, then the new
-  // tokens' K/V into their slots, each phase closed by a grid-wide barrier
-  // whose words sit in grid_sync (two slots of 32 words in the workspace)
-  const int64_t* upd_pairs;   // [upd_num_pairs][2] (src, dst) block ids
-  int upd_num_pairs;
+  // new tokens' K/V stored by the tensor-core kernel before it reads the
+  // pools (null / 0 for none), the phase closed by a grid-wide barrier whose
+  // two words sit at grid_sync in the workspace
   const uint4* upd_k;         // [upd_num_tokens][num_kv_heads][head_dim]
   const uint4* upd_v;
   const int64_t* upd_slots;   // [upd_num_tokens]
@@ -75,14 +72,14 @@ struct DecodeParams {
   int32_t* grid_sync;
 };
 
-// Workspace bytes of the two grid-wide barrier slots, between the partial
-// states and the arrival counters.
+// Workspace bytes of the grid-wide barrier's words (one 128-byte line used),
+// between the partial states and the arrival counters.
 constexpr int kGridSyncBytes = 256;
 
 constexpr long long kGranuleCost = 8;  // partition cost of one granule
 
 constexpr int kFlagTestWithholdCopies = PA_DECODE_TEST_WITHHOLD_COPIES;  // producer issues nothing
-constexpr int kFlagTestSkipUpdateArrival = PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL;  // CTA 0 skips the update barriers
+constexpr int kFlagTestSkipUpdateArrival = PA_DECODE_TEST_SKIP_UPDATE_ARRIVAL;  // CTA 0 skips the stores' barrier
 
 __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, int B) {
   const int n = __ldg(p.seq_lens + s);

@@ -1,9 +1,9 @@
 """GPU parity of the one-call step: pa_decode_update, pa_decode_multi_update
 and pa_decode_shared_prefix_update run the step's copy-on-write block copies
-(study notes ch.05 §6.1), then the new tokens' stores (vLLM blog,
-plain-language section), then the decode, inside one launch of the
-tensor-core kernel (grid-wide barriers between the phases), or as separate
-kernels where that kernel does not run.
+(study notes ch.05 §6.1, a kernel of their own), then the new tokens' stores
+(vLLM blog, plain-language section), then the decode; the stores run inside
+the launch of the tensor-core decode kernel (a grid-wide barrier before its
+first K/V load), or as pa_cache_write where that kernel does not run.
 
 Each case is checked three ways:
 * the pools, bit for bit, against the oracle's copy_blocks and cache_write;
@@ -67,7 +67,7 @@ def _run_plain(L, V, device, *, fused, num_ctas=0, flags=0):
 def test_update_decode_with_copies_and_writes(cuda_device, B, num_ctas):
     """Forked samples at the Llama-2-70B layer shape (64 q / 8 kv heads):
     nine copy-on-write pairs and twelve new tokens, some of them stored into
-    a block copied in the same launch, then the GQA-8 decode."""
+    a block copied by the same call, then the GQA-8 decode."""
     L = config_llama2_70b_shared(prompt_len=256, num_prompts=3, samples=4, max_tail=60, block_size=B)
     assert L.copy_pairs.shape[0] > 0 and L.num_new_tokens > 0
     V = fill_values_numpy(L)
@@ -99,8 +99,8 @@ def test_update_decode_write_only_gqa4(cuda_device, dtype):
 
 
 def test_update_repeated_calls_reuse_the_workspace(cuda_device):
-    """Three one-launch steps in a row on one workspace: the barrier words are
-    left as found (the arrival counts back at zero), so each call completes
+    """Three one-call steps in a row on one workspace: the barrier words are
+    left as found (the arrival count back at zero), so each call completes
     with the same pools and outputs (the update is idempotent here: the
     copies rewrite the same blocks, the stores the same slots)."""
     import torch
@@ -129,7 +129,7 @@ def test_update_repeated_calls_reuse_the_workspace(cuda_device):
 @pytest.mark.parametrize("B", [8, 16, 32])
 def test_update_shared_prefix(cuda_device, B):
     """Shared-prefix decode (group units of 4 members x 8 heads) with its
-    step's copies and stores in the same launch."""
+    step's copies and stores in the same call."""
     import torch
 
     import paged_kv_cache_357_b200 as pa
@@ -165,7 +165,8 @@ def test_update_shared_prefix(cuda_device, B):
 @pytest.mark.parametrize("q_len,G", [(4, 4), (3, 8), (64, 4)])
 def test_update_multi(cuda_device, q_len, G):
     """Multi-query steps whose q_len new tokens are stored by the same call:
-    q_len 4 and 3 run on the tensor-core row-tile kernel (one launch); q_len
+    q_len 4 and 3 run on the tensor-core row-tile kernel (stores in its
+    launch); q_len
     64 at GQA-4 fills 128-row tiles and runs the query-major prefill kernel,
     after the update's own kernels."""
     import torch
@@ -252,7 +253,7 @@ def test_update_reports_bad_slots_and_pairs(cuda_device):
 
 def test_update_barrier_wait_runs_out(cuda_device):
     """Failure detection: with the test hook CTA 0 never arrives at the
-    update's barriers, every wait for them runs out (about 20 ms), the
+    stores' barrier, every wait for it runs out (about 20 ms), the
     kernel returns PA_DEV_TIMEOUT, and the context stays usable: a normal
     step on a zeroed workspace then matches the oracle."""
     import torch
