@@ -205,6 +205,18 @@ def roofline_of(L, mode, achieved_gbs, peak_gbs, peak_kind, nbytes, decode_ms, f
     }
 
 
+# Attention layers of the model whose layer shape a workload takes (the
+# models' published layer counts), for the implied per-model token rate.
+MODEL_LAYERS = {"llama7b": 32, "llama3_8b": 32, "llama2_70b": 80, "opt13b": 40}
+
+
+def model_layers(L):
+    for prefix, n in MODEL_LAYERS.items():
+        if L.name.startswith(prefix):
+            return prefix, n
+    return None, None
+
+
 def decode_entry(L, mode: str) -> str:
     if L.q_len > 1:
         return "pa_decode_multi"
@@ -756,6 +768,10 @@ def run_ours(args):
             "tokens_per_s": tokens_per_s,
             "tokens_per_s_note": ("one new token per sequence per single-layer step" if L.q_len == 1 else
                                   f"{L.q_len} query positions per sequence per single-layer step"),
+            "tokens_per_s_implied_model": (tokens_per_s / model_layers(L)[1]) if model_layers(L)[1] else None,
+            "tokens_per_s_implied_model_note": (
+                f"implied, attention only: the single-layer step repeated for the {model_layers(L)[1]} layers of "
+                f"{model_layers(L)[0]} with nothing else in the model timed" if model_layers(L)[1] else None),
             "decode_ms": decode_mean_ms,
             "decode_ms_note": (("CUDA events around each launch of the tensor-core kernel, which also runs the "
                                 "step's cache update" if fused else "CUDA events around each decode launch")

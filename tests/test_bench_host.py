@@ -58,3 +58,28 @@ def test_profiled_traffic_only_for_the_profiled_workload():
         assert traffic is None  # the kernel changed since the capture
     assert bench.profiled_traffic(full, "shared_prefix") is None
     assert bench.profiled_traffic(_layout("--batch", "64")) is None
+
+
+def test_one_launch_form_and_its_bytes():
+    """The step's new-token writes go inside the tensor-core decode launch
+    for the decode workloads that write, not for the prefill kernel's
+    workload or the CUDA-core kernel, nor without new tokens; that launch's
+    algorithmic bytes add the new tokens' K/V read and written."""
+    full = _layout()
+    assert bench.one_launch_step(full, "plain", "one_launch")
+    assert not bench.one_launch_step(full, "plain", "separate")
+    assert not bench.one_launch_step(full, "cuda_cores", "one_launch")
+    assert not bench.one_launch_step(_layout("--config", "llama3_8b_prefill256", "--batch", "16"), "plain",
+                                     "one_launch")
+    assert not bench.one_launch_step(_layout("--config", "llama7b", "--batch", "16"), "plain", "one_launch")
+    b = bench.step_bytes(full)
+    T = full.num_new_tokens
+    assert b["write"] == T * full.num_kv_heads * full.head_dim * 2 * 2 * 2 + T * 8
+    assert b["step"] == b["decode"] + b["write"] + b["copy"]
+
+
+def test_implied_model_rate_uses_each_models_layer_count():
+    assert bench.model_layers(_layout()) == ("llama3_8b", 32)
+    assert bench.model_layers(_layout("--config", "llama2_70b_shared", "--batch", "64")) == ("llama2_70b", 80)
+    assert bench.model_layers(_layout("--config", "opt13b_long_b8")) == ("opt13b", 40)
+    assert bench.model_layers(_layout("--config", "tiny")) == (None, None)
