@@ -224,3 +224,38 @@ def test_build_tracks_every_source_and_header():
     csrc = Path(pa_build.CSRC)
     on_disk = {p.name for p in csrc.iterdir() if p.suffix in (".cu", ".cuh", ".h", ".cpp")}
     assert on_disk == set(pa_build.SOURCES) | set(pa_build.HEADERS)
+
+
+def _update(copy_pairs=None, num_copy_pairs=0, k=None, v=None, slots=None, num_tokens=0):
+    return _lib.CacheUpdate(copy_pairs, num_copy_pairs, k, v, slots, num_tokens)
+
+
+def test_update_entry_points_reject_bad_updates_on_host(lib):
+    """pa_decode_update and its multi-query and shared-prefix forms check the
+    cache update before anything is enqueued (an empty batch included)."""
+    desc = _desc()
+    opts = _lib.DecodeOpts(0, 0)
+    bad = [
+        _update(num_copy_pairs=-1),
+        _update(num_tokens=-1),
+        _update(num_copy_pairs=2),                                             # pairs missing
+        _update(copy_pairs=FAKE + 4, num_copy_pairs=2),                        # pairs not 8-byte aligned
+        _update(k=FAKE, v=None, slots=FAKE, num_tokens=3),                     # v missing
+        _update(k=FAKE + 8, v=FAKE, slots=FAKE, num_tokens=3),                 # k not 16-byte aligned
+        _update(k=FAKE, v=FAKE, slots=FAKE + 4, num_tokens=3),                 # slots not 8-byte aligned
+    ]
+    for u in bad:
+        for S in (4, 0):
+            rc = lib.pa_decode_update(ctypes.byref(u), FAKE, FAKE, FAKE, FAKE, 8, FAKE, S, 4, 0.125, FAKE, FAKE,
+                                      1 << 20, None, ctypes.byref(desc), ctypes.byref(opts), None)
+            assert rc == 1, (S, rc)
+        rc = lib.pa_decode_multi_update(ctypes.byref(u), FAKE, FAKE, FAKE, FAKE, 8, FAKE, 4, 3, 4, 0.125, FAKE,
+                                        FAKE, 1 << 20, None, ctypes.byref(desc), ctypes.byref(opts), None)
+        assert rc == 1
+        rc = lib.pa_decode_shared_prefix_update(ctypes.byref(u), FAKE, FAKE, FAKE, FAKE, 8, FAKE, 4, 4, FAKE, FAKE,
+                                                2, 4, 0.125, FAKE, FAKE, 1 << 20, None, ctypes.byref(desc),
+                                                ctypes.byref(opts), None)
+        assert rc == 1
+    # bad decode arguments are still caught with a valid (here empty) update
+    assert lib.pa_decode_update(ctypes.byref(_update()), None, FAKE, FAKE, FAKE, 8, FAKE, 4, 4, 0.125, FAKE, FAKE,
+                                1 << 20, None, ctypes.byref(desc), ctypes.byref(opts), None) == 1
