@@ -60,22 +60,36 @@ def torch_f64(t) -> np.ndarray:
 
 
 def gpu_step(dev_t, layout: PagedLayout, *, num_ctas: int = 0, do_copy=True, do_write=True, status=None,
-             workspace=None):
-    """copy -> write -> decode through the C ABI; returns (out tensor, status tensor)."""
+             workspace=None, one_launch=False):
+    """copy -> write -> decode through the C ABI; returns (out tensor, status tensor).
+    With one_launch the three go through pa_decode_update (the writes inside
+    the decode's launch), as the benchmark's step does."""
     import torch
 
     import paged_kv_cache_357_b200 as pa
 
     d = dev_t
     st = torch.zeros(1, dtype=torch.int32, device=d["q"].device) if status is None else status
-    if do_copy and layout.copy_pairs.shape[0] > 0:
-        pa.pa_copy_blocks(d["pairs"], d["k_pool"], d["v_pool"], st)
-    if do_write and layout.num_new_tokens > 0:
-        pa.pa_cache_write(d["new_k"], d["new_v"], d["slots"], d["k_pool"], d["v_pool"], st)
+    copy = do_copy and layout.copy_pairs.shape[0] > 0
+    write = do_write and layout.num_new_tokens > 0
     out = torch.full_like(d["q"], float("nan"))
     ws = workspace
     if ws is None:
         ws = pa.alloc_decode_workspace(layout.num_seqs, layout.num_q_heads, d["k_pool"], num_ctas)
+    if one_launch:
+        upd = {}
+        if copy:
+            upd["copy_pairs"] = d["pairs"]
+        if write:
+            upd.update(new_k=d["new_k"], new_v=d["new_v"], slot_mapping=d["slots"])
+        pa.pa_decode_update(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], layout.scale, out, ws, st,
+                            num_ctas=num_ctas, **upd)
+        torch.cuda.synchronize()
+        return out, st
+    if copy:
+        pa.pa_copy_blocks(d["pairs"], d["k_pool"], d["v_pool"], st)
+    if write:
+        pa.pa_cache_write(d["new_k"], d["new_v"], d["slots"], d["k_pool"], d["v_pool"], st)
     pa.pa_decode(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], layout.scale, out, ws, st,
                  num_ctas=num_ctas)
     torch.cuda.synchronize()

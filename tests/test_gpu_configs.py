@@ -1,5 +1,7 @@
 """The five workloads at full size, in the launch configuration the
-benchmark times (default CTA count).
+benchmark times (default CTA count), in both step forms: the writes inside
+the decode's launch (pa_decode_update, what the benchmark times) and the
+separate pa_copy_blocks / pa_cache_write / pa_decode launches.
 
 * Pools, bit-exact and whole: both pools are copied to the host before the
   step, the oracle applies the step's block copies and cache writes to those
@@ -42,9 +44,10 @@ def _sample(L, k, seed):
     return sorted(pick)
 
 
+@pytest.mark.parametrize("one_launch", [True, False], ids=["one_launch", "separate"])
 @pytest.mark.parametrize("name", ["tiny", "llama7b", "llama3_8b", "llama2_70b_shared", "opt13b_long_b8",
                                   "opt13b_long_b16", "opt13b_long_b32"])
-def test_config_full_size(cuda_device, name):
+def test_config_full_size(cuda_device, name, one_launch):
     import torch
 
     import paged_kv_cache_357_b200 as pa
@@ -70,7 +73,7 @@ def test_config_full_size(cuda_device, name):
     if V.new_v.numel() > 0:
         vmax = max(vmax, float(V.new_v.float().abs().max()))
     d = _device_inputs(L, V, cuda_device)
-    out, st = gpu_step(d, L)
+    out, st = gpu_step(d, L, one_launch=one_launch)
     assert int(st.item()) == 0
 
     # the whole pools after the step, bit for bit, against the oracle's copy and write

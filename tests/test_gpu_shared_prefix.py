@@ -206,9 +206,14 @@ def test_unsupported_group_size_is_refused(cuda_device):
     assert e.value.code == 2
 
 
-def test_llama2_70b_shared_full_size(cuda_device):
+@pytest.mark.parametrize("one_launch", [True, False], ids=["one_launch", "separate"])
+def test_llama2_70b_shared_full_size(cuda_device, one_launch):
     """The 70B shared-prefix workload at full size through the shared-prefix
-    decode: sampled sequences (whole groups among them) against the oracle."""
+    decode: sampled sequences (whole groups among them) against the oracle,
+    with the step's writes inside the decode's launch (what the benchmark
+    times) or as their own launch.  The oracle applies the step's copies and
+    writes to the sampled sequences' blocks before its decode, so a missed
+    or late copy or write shows in their outputs."""
     import torch
 
     import paged_kv_cache_357_b200 as pa
@@ -228,13 +233,18 @@ def test_llama2_70b_shared_full_size(cuda_device):
     starts, prefix = pa.shared_prefix_groups(L.block_tables, L.seq_lens, L.block_size, 4)
     assert len(prefix) == len(L.share_groups) and (prefix == 2048 // 16 - 1).all()
     st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
-    pa.pa_copy_blocks(d["pairs"], d["k_pool"], d["v_pool"], st)
-    pa.pa_cache_write(d["new_k"], d["new_v"], d["slots"], d["k_pool"], d["v_pool"], st)
     out = torch.full_like(d["q"], float("nan"))
     ws = pa.alloc_shared_prefix_workspace(L.num_seqs, 4, L.num_q_heads, d["k_pool"])
-    pa.pa_decode_shared_prefix(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"],
-                               torch.from_numpy(starts).to(cuda_device), torch.from_numpy(prefix).to(cuda_device),
-                               4, L.scale, out, ws, st)
+    gs, gp = torch.from_numpy(starts).to(cuda_device), torch.from_numpy(prefix).to(cuda_device)
+    if one_launch:
+        pa.pa_decode_shared_prefix_update(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], gs, gp, 4,
+                                          L.scale, out, ws, st, copy_pairs=d["pairs"], new_k=d["new_k"],
+                                          new_v=d["new_v"], slot_mapping=d["slots"])
+    else:
+        pa.pa_copy_blocks(d["pairs"], d["k_pool"], d["v_pool"], st)
+        pa.pa_cache_write(d["new_k"], d["new_v"], d["slots"], d["k_pool"], d["v_pool"], st)
+        pa.pa_decode_shared_prefix(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], gs, gp, 4, L.scale,
+                                   out, ws, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert torch.isfinite(out).all()
