@@ -346,7 +346,10 @@ PA_API pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs,
  * barrier wait that runs out (for instance when other work keeps part of
  * the grid off the GPU for its whole limit) records PA_DEV_TIMEOUT; the
  * pools and outputs are then unspecified and the workspace must be zeroed
- * again, as after any non-zero device status.
+ * again, as after any non-zero device status.  The barrier needs every CTA
+ * of the launch on an SM at once: do not run two of these calls at the same
+ * time on different streams (each could hold SMs the other's grid waits
+ * for until its waits run out); order them on one stream.
  */
 typedef struct pa_cache_update {
   const int64_t* copy_pairs;  /* int64 [num_copy_pairs][2] (src, dst) block ids, device; NULL when 0 */
