@@ -28,6 +28,8 @@ from .paged_attention import (  # noqa: F401
     gather_kv,
     attention_dense,
     decode,
+    decode_lse,
+    merge_outputs,
     decode_one,
     decode_multi,
     decode_blockwise_online,

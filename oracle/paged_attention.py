@@ -176,6 +176,51 @@ def merge_partition_states(states) -> np.ndarray:
     return num / den
 
 
+def decode_lse(q, k_pool, v_pool, block_tables, seq_lens, scale: float, num_kv_heads: int, dtype: str):
+    """The decode step's outputs [S, Hq, D] together with, per (s, h), the
+    natural log of the softmax normaliser over the sequence's tokens,
+    lse = log sum_t exp(scale * q . K_t) [S, Hq] (-inf for no token): the
+    quantity that lets decodes of disjoint token ranges be merged afterwards
+    (study notes ch.05 §4, the online-softmax merge).  Written out per row
+    with the shift by the row's maximum, as the softmax itself."""
+    S, Hq, D = q.shape
+    g = Hq // num_kv_heads
+    B = k_pool.shape[2]
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    lse = np.full((S, Hq), -np.inf, dtype=np.float64)
+    for s in range(S):
+        n = int(seq_lens[s])
+        for h in range(Hq):
+            out[s, h] = decode_one(s, h, q, k_pool, v_pool, block_tables, seq_lens, scale, num_kv_heads, dtype)
+            if n == 0:
+                continue
+            K = bits_to_f64(gather_kv(k_pool, block_tables[s], n, h // g, B), dtype)
+            z = scale * (K @ bits_to_f64(q[s, h], dtype))
+            m = z.max()
+            lse[s, h] = m + np.log(np.exp(z - m).sum())
+    return out, lse
+
+
+def merge_outputs(outs, lses):
+    """Merge decodes of disjoint token ranges of the same rows (study notes
+    ch.05 §4: partial results rescaled to a common maximum).  outs
+    [R, ..., D] and lses [R, ...] per range; with M = max_r lse_r and
+    w_r = e^(lse_r - M): out = sum_r w_r out_r / sum_r w_r and
+    lse = M + log sum_r w_r.  A row no range saw (every lse_r = -inf) gets a
+    zero output and -inf.  Returns (out, lse) in float64."""
+    outs = np.asarray(outs, dtype=np.float64)
+    lses = np.asarray(lses, dtype=np.float64)
+    M = lses.max(axis=0)
+    seen = np.isfinite(M)
+    Ms = np.where(seen, M, 0.0)
+    w = np.where(np.isfinite(lses), np.exp(lses - Ms), 0.0)  # [R, ...]
+    wsum = w.sum(axis=0)
+    out = np.zeros(outs.shape[1:], dtype=np.float64)
+    out[seen] = (np.einsum("r...,r...d->...d", w, outs))[seen] / wsum[seen][..., None]
+    lse = np.where(seen, Ms + np.log(np.where(seen, wsum, 1.0)), -np.inf)
+    return out, lse
+
+
 def cache_write(k_pool: np.ndarray, v_pool: np.ndarray, new_k: np.ndarray, new_v: np.ndarray,
                 slot_mapping: np.ndarray):
     """Store each new token's K/V rows in its slot (vLLM blog, plain-language section: each
