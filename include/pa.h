@@ -168,6 +168,45 @@ PA_API pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_p
                        int32_t* dev_status, const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream);
 
 /*
+ * pa_decode_lse — pa_decode that also returns each output row's log
+ * normaliser, so that decodes of disjoint token ranges of the same rows can
+ * be merged afterwards (pa_merge_partials): a sequence too long for one GPU
+ * split by blocks across GPUs, each decoding its own range.  The merge is
+ * the online-softmax rule of study notes ch.05 §4 applied to the ranges.
+ *   lse   float32 device [num_seqs][num_q_heads], 4-byte aligned:
+ *         lse[s][h] = log sum_t exp(scale * q[s][h] . K_t) over the
+ *         sequence's tokens (natural log), -inf for a sequence with no token
+ * Other arguments, results and errors as pa_decode_ex.  The tensor-core
+ * kernel writes it (head_dim 128, 16-bit pools, blocks of 8, 16 or 32);
+ * elsewhere (and under PA_DECODE_CUDA_CORES_ONLY) PA_ERR_UNSUPPORTED.
+ */
+PA_API pa_status pa_decode_lse(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                               int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
+                               int32_t num_q_heads, float scale, void* out, float* lse, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
+                               const pa_decode_opts* opts, void* stream);
+
+/*
+ * pa_merge_partials — merge decodes of disjoint token ranges of the same
+ * query rows (study notes ch.05 §4: the online-softmax merge, rescaling each
+ * part to a common maximum).  For each row i with M = max_r lses[r][i] and
+ * w_r = exp(lses[r][i] - M):
+ *   out[i] = sum_r w_r outs[r][i] / sum_r w_r
+ *   lse_out[i] = M + log sum_r w_r            (lse_out nullable)
+ * A part with lse -inf (no token) adds nothing; a row no part saw gets a
+ * zero output and -inf.  The merge is exact up to fp32 rounding; the parts'
+ * outputs are already rounded to the 16-bit type, so a merged output
+ * carries their rounding (at most one 16-bit rounding step) beside its own.
+ *   outs     [num_parts][num_rows][head_dim], fp16/bf16 (dtype), 16-byte aligned
+ *   lses     float32 [num_parts][num_rows] (as pa_decode_lse writes them)
+ *   out      [num_rows][head_dim], same dtype; lse_out float32 [num_rows]
+ * num_rows is num_seqs * num_q_heads for decode outputs; head_dim 64 or 128.
+ * num_rows == 0 is a no-op.  No device errors.
+ */
+PA_API pa_status pa_merge_partials(const void* outs, const float* lses, int32_t num_parts, int32_t num_rows,
+                                   int32_t head_dim, int32_t dtype, void* out, float* lse_out, void* stream);
+
+/*
  * pa_decode_no_alloc — pa_decode for callers that cannot allocate device
  * memory.  The pages have no counterpart: this is a calling convention of
  * this library, not part of the method.

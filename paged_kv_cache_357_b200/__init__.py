@@ -12,6 +12,10 @@ The kernels live in ``libpa.so`` (C ABI: ``include/pa.h``), built in-tree by
 * ``pa_decode_update`` (and the ``_multi`` / ``_shared_prefix`` forms) a
                       step's copies, writes and decode as one call, one
                       launch on the tensor-core kernel
+* ``pa_decode_lse``, ``pa_merge_partials``  decodes of disjoint token ranges
+                      with their log normalisers, and their merge
+* ``split.gather_partials`` / ``split.decode_split``  a sequence's token ranges
+                      held by different ranks, decoded and merged
 * ``PagedDecodeStep`` one whole step (copy, write, decode) from host buffers
 * ``BlockManager``    host block manager (free set, ref counts, copy on write)
 
@@ -44,7 +48,9 @@ from ._lib import (  # noqa: F401
     pa_cache_write,
     pa_copy_blocks,
     pa_decode,
+    pa_decode_lse,
     pa_decode_no_alloc,
+    pa_merge_partials,
     pa_decode_multi_update,
     pa_decode_shared_prefix_update,
     pa_decode_update,

@@ -43,6 +43,8 @@ EXPORTED = (
     "pa_cache_write",
     "pa_copy_blocks",
     "pa_decode_update",
+    "pa_decode_lse",
+    "pa_merge_partials",
     "pa_decode_multi_update",
     "pa_decode_shared_prefix_update",
     "pa_status_string",
@@ -173,6 +175,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_shared_prefix_update.argtypes = [pupd] + lib.pa_decode_shared_prefix.argtypes
     for name in ("pa_decode_update", "pa_decode_multi_update", "pa_decode_shared_prefix_update"):
         getattr(lib, name).restype = i32
+    lib.pa_decode_lse.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, f32, vp, vp, vp, sz, vp, pdesc, popts, vp]
+    lib.pa_decode_lse.restype = i32
+    lib.pa_merge_partials.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    lib.pa_merge_partials.restype = i32
     lib.pa_copy_blocks.restype = i32
     pshape, playout = ctypes.POINTER(StepShape), ctypes.POINTER(StepLayout)
     vpp = ctypes.POINTER(ctypes.c_void_p)
@@ -604,3 +610,52 @@ def pa_decode_shared_prefix_update(q, k_pool, v_pool, block_tables, seq_lens, gr
     )
     if rc != 0:
         raise PaError(rc, "pa_decode_shared_prefix_update")
+
+
+# ---------------------------------------------------------------------------
+# decodes of disjoint token ranges and their merge (pa_decode_lse, pa_merge_partials)
+# ---------------------------------------------------------------------------
+
+
+def pa_decode_lse(q, k_pool, v_pool, block_tables, seq_lens, scale: float, out, lse, workspace, dev_status=None,
+                  num_ctas: int = 0, flags: int = 0, stream=None) -> None:
+    """pa_decode that also writes lse [num_seqs, num_q_heads] float32, the
+    natural log of each row's softmax normaliser (pa_decode_lse)."""
+    torch = _torch()
+    _check_attention_args(q, k_pool, v_pool, block_tables, seq_lens, out, workspace, dev_status, 3)
+    S, Hq, D = q.shape
+    _need(lse, "lse", dtype=torch.float32, ndim=2, device=k_pool.device)
+    if tuple(lse.shape) != (S, Hq):
+        raise ValueError("lse must be [num_seqs, num_q_heads]")
+    desc = pool_desc(k_pool)
+    opts = DecodeOpts(num_ctas, flags)
+    rc = load().pa_decode_lse(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), S, Hq,
+        float(scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(dev_status), ctypes.byref(desc), ctypes.byref(opts), _stream(stream),
+    )
+    if rc != 0:
+        raise PaError(rc, "pa_decode_lse")
+
+
+def pa_merge_partials(outs, lses, out, lse_out=None, stream=None) -> None:
+    """Merge decodes of disjoint token ranges of the same rows
+    (pa_merge_partials): outs [R, ..., head_dim] fp16/bf16 and lses [R, ...]
+    float32 from pa_decode_lse; out [..., head_dim], lse_out [...] (optional)."""
+    torch = _torch()
+    _need(outs, "outs")
+    dev = outs.device
+    _need(lses, "lses", dtype=torch.float32, device=dev)
+    _need(out, "out", dtype=outs.dtype, device=dev)
+    R, D = outs.shape[0], outs.shape[-1]
+    rows = out.numel() // D if D else 0
+    if tuple(outs.shape[1:]) != tuple(out.shape) or tuple(lses.shape) != (R,) + tuple(out.shape[:-1]):
+        raise ValueError("outs [R, ..., D], lses [R, ...] and out [..., D] disagree")
+    if lse_out is not None:
+        _need(lse_out, "lse_out", dtype=torch.float32, device=dev)
+        if tuple(lse_out.shape) != tuple(out.shape[:-1]):
+            raise ValueError("lse_out must have out's shape without head_dim")
+    rc = load().pa_merge_partials(_ptr(outs), _ptr(lses), R, rows, D, _dtype_code(outs), _ptr(out), _ptr(lse_out),
+                                  _stream(stream))
+    if rc != 0:
+        raise PaError(rc, "pa_merge_partials")

@@ -30,6 +30,7 @@ SOURCES = [
     "pa_attn_tc_multi_b32.cu", "pa_attn_tc_prefill.cu", "pa_attn_tc_prefill_b8.cu", "pa_attn_tc_prefill_b32.cu",
     "pa_attn_tc_group.cu", "pa_attn_tc_group_b8.cu", "pa_attn_tc_group_b32.cu",
     "pa_kv_ops.cu",
+    "pa_merge.cu",
     "pa_block_manager.cpp",
     "pa_step.cpp",
 ]

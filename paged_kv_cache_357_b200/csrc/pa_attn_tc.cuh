@@ -688,6 +688,10 @@ __device__ void zero_empty_units(const DecodeParams& p, const Source<kMode, RG>&
     uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(src.row_group0(p, u)) * p.num_q_heads * D);
     const int n = src.row_groups(p, u) * p.num_q_heads * D / 8;
     for (int i = 0; i < n; ++i) o[i] = make_uint4(0, 0, 0, 0);
+    if (p.lse != nullptr) {
+      float* l = p.lse + static_cast<size_t>(src.row_group0(p, u)) * p.num_q_heads;
+      for (int i = 0; i < src.row_groups(p, u) * p.num_q_heads; ++i) l[i] = -INFINITY;
+    }
   }
 }
 
@@ -1470,17 +1474,37 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
       }
       const bool opens = fs.j0 == fs.first, closes = fs.j0 + fs.n == fs.nb;
       // the outputs of this warpgroup's rows through the staging tile (the
-      // previous finish's copies have read it by now)
-      auto emit = [&]() {
+      // previous finish's copies have read it by now); with p.lse, each row's
+      // log normaliser, m + log2 l in the log2 domain of the scores, as a
+      // natural log, by the thread of the warpgroup's first warp whose lane
+      // is the row
+      auto emit = [&](const float (&Mx)[RC]) {
         if (leader) bulk_wait_read();
         named_barrier_sync(wg_bar, 128);
         stage_rows<kBf16, RC>(sm.ostage, col0, r, L, acc);
         fence_proxy_async_smem();
         named_barrier_sync(wg_bar, 128);
         if (leader) issue_rows<G, RG, RC, kMode>(p, fs, s0, col0, rows, sm.ostage);
+        if constexpr (kMode != kDecode) return;  // pa_decode_lse runs the decode mode only
+        if (p.lse != nullptr && quad == 0 && lane < RC && col0 + lane < rows) {
+          float l = L[0], m = Mx[0];
+#pragma unroll
+          for (int k = 1; k < RC; ++k) {
+            l = lane == k ? L[k] : l;
+            m = lane == k ? Mx[k] : m;
+          }
+          const int c = col0 + lane;
+          const size_t row = out_row<RG, kMode>(p, fs, s0, c / G);
+          p.lse[row * p.num_q_heads + static_cast<size_t>(fs.h) * G + c % G] =
+              l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        }
       };
       if (opens && closes) {
-        emit();
+        float Mw[RC];
+        if constexpr (kMode == kDecode) {
+          if (p.lse != nullptr) ld_row<RC>(sm.mfin[ob] + col0, Mw);
+        }
+        emit(Mw);
         return;
       }
       int32_t* counter = unit_counter(p, fs);
@@ -1539,7 +1563,7 @@ __global__ void __launch_bounds__(Rows<G * RG>::kThreads, 1)
           M[k] = mn;
         }
       }
-      emit();
+      emit(M);
     };
 
 #pragma unroll

@@ -602,6 +602,7 @@ static DecodeParams make_params(const void* q, const void* k_pool, const void* v
   prm.group_prefix = nullptr;
   prm.num_groups = 0;
   prm.unit_cost = 0;
+  prm.lse = nullptr;
   prm.upd_k = nullptr;
   prm.upd_v = nullptr;
   prm.upd_slots = nullptr;
@@ -737,11 +738,12 @@ static pa_status decode_impl(const pa_cache_update* upd, const void* q, const vo
                              const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
                              int32_t num_seqs, int32_t num_q_heads, float scale, void* out, void* workspace,
                              size_t workspace_bytes, int32_t* dev_status, const pa_pool_desc* pool,
-                             const pa_decode_opts* opts, void* stream) {
+                             const pa_decode_opts* opts, void* stream, float* lse = nullptr) {
   pa_status st = check_decode_args(q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
                                     num_q_heads, scale, out, pool);
   if (st != PA_OK) return st;
   if (!update_args_ok(upd)) return PA_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return enqueue_update(upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), dev_status, pool, stream);
   if (opts != nullptr && (opts->num_ctas < 0 || (opts->flags & ~kKnownFlags) != 0)) return PA_ERR_INVALID_ARG;
   Variant v;
@@ -754,7 +756,21 @@ static pa_status decode_impl(const pa_cache_update* upd, const void* q, const vo
                                        num_q_heads, scale, out, workspace, ctas, v.part_stride, dev_status, pool,
                                        opts_flags(opts));
   prm.unit_cost = v.unit_cost;
+  if (lse != nullptr) {
+    if (!v.fuses_update) return PA_ERR_UNSUPPORTED;  // the log normalisers come from the tensor-core kernel
+    prm.lse = lse;
+  }
   return launch_decode(v, prm, ctas, upd, const_cast<void*>(k_pool), const_cast<void*>(v_pool), pool, stream);
+}
+
+extern "C" pa_status pa_decode_lse(const void* q, const void* k_pool, const void* v_pool,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                   int32_t num_seqs, int32_t num_q_heads, float scale, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                   const pa_pool_desc* pool, const pa_decode_opts* opts, void* stream) {
+  if (lse == nullptr && num_seqs > 0) return PA_ERR_INVALID_ARG;
+  return decode_impl(nullptr, q, k_pool, v_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                     scale, out, workspace, workspace_bytes, dev_status, pool, opts, stream, lse);
 }
 
 extern "C" pa_status pa_decode_ex(const void* q, const void* k_pool, const void* v_pool,

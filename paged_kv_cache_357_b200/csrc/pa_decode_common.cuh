@@ -70,6 +70,10 @@ struct DecodeParams {
   const int64_t* upd_slots;   // [upd_num_tokens]
   int upd_num_tokens;
   int32_t* grid_sync;
+  // per output row (num_q_heads per sequence row), the natural log of the
+  // softmax normaliser, log sum_t exp(scale q.K_t); -inf for no token.
+  // Written by the tensor-core kernel when not null.
+  float* lse;
 };
 
 // Workspace bytes of the grid-wide barrier's words (one 128-byte line used),

@@ -19,7 +19,7 @@ struct Variant {
   int part_stride;  // floats per partial slot: query rows per unit * (D + 2)
   LaunchFn launch;
   int unit_cost;    // partition cost of finishing a unit (DecodeParams::unit_cost)
-  bool fuses_update = false;  // runs a cache update (DecodeParams::upd_*) inside the launch
+  bool fuses_update = false;  // tensor-core decode family: takes new tokens (DecodeParams::upd_*) into its launch and writes log normalisers (DecodeParams::lse)
 };
 
 // Tensor-core variants (pa_attn_tc.cuh), if one exists for this pool and

@@ -259,3 +259,23 @@ def test_update_entry_points_reject_bad_updates_on_host(lib):
     # bad decode arguments are still caught with a valid (here empty) update
     assert lib.pa_decode_update(ctypes.byref(_update()), None, FAKE, FAKE, FAKE, 8, FAKE, 4, 4, 0.125, FAKE, FAKE,
                                 1 << 20, None, ctypes.byref(desc), ctypes.byref(opts), None) == 1
+
+
+def test_lse_and_merge_reject_bad_arguments_on_host(lib):
+    desc = _desc(head_dim=128)
+    opts = _lib.DecodeOpts(0, 0)
+    # pa_decode_lse needs its lse output (4-byte aligned)
+    for lse in (None, FAKE + 2):
+        rc = lib.pa_decode_lse(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 4, 4, 0.125, FAKE, lse, FAKE, 1 << 20, None,
+                               ctypes.byref(desc), ctypes.byref(opts), None)
+        assert rc == 1
+    merge = lib.pa_merge_partials
+    assert merge(FAKE, FAKE, 2, 0, 128, _lib.PA_BF16, FAKE, None, None) == 0  # no rows: a no-op
+    assert merge(FAKE, FAKE, 0, 10, 128, _lib.PA_BF16, FAKE, None, None) == 1  # no parts
+    assert merge(FAKE, FAKE, 2, -1, 128, _lib.PA_BF16, FAKE, None, None) == 1
+    assert merge(FAKE, FAKE, 2, 10, 96, _lib.PA_BF16, FAKE, None, None) == 1  # head_dim
+    assert merge(FAKE, FAKE, 2, 10, 128, 7, FAKE, None, None) == 1  # dtype
+    assert merge(None, FAKE, 2, 10, 128, _lib.PA_BF16, FAKE, None, None) == 1
+    assert merge(FAKE + 8, FAKE, 2, 10, 128, _lib.PA_BF16, FAKE, None, None) == 1  # outs misaligned
+    assert merge(FAKE, FAKE + 2, 2, 10, 128, _lib.PA_BF16, FAKE, None, None) == 1  # lses misaligned
+    assert merge(FAKE, FAKE, 2, 10, 128, _lib.PA_BF16, FAKE, FAKE + 1, None) == 1  # lse_out misaligned

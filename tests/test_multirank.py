@@ -66,3 +66,49 @@ def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
                                                "--warmup", "0", "--config", "tiny"]))
     assert rc == 0
     assert capsys.readouterr().out == ""
+
+
+def _split_rank_main(rank, world, port, out):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from paged_kv_cache_357_b200.split import gather_partials
+    from workloads import fill_values_numpy, random_layout
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        L = random_layout(31, [5, 40, 64, 100, 0], dtype="bf16", block_size=8, num_q_heads=4, num_kv_heads=2,
+                          head_dim=16, write_new_token=False)
+        V = fill_values_numpy(L)
+        # rank r holds tokens [32 r, 32 (r + 1)) of every sequence (the last rank the rest)
+        a = 32 * rank
+        b = 32 * (rank + 1) if rank < world - 1 else 1 << 20
+        lens = np.clip(L.seq_lens - a, 0, b - a).astype(np.int32)
+        tables = np.zeros_like(L.block_tables)
+        tables[:, : L.block_tables.shape[1] - a // 8] = L.block_tables[:, a // 8:]
+        part, lse = oracle.decode_lse(V.q, V.k_pool, V.v_pool, tables, lens, L.scale, L.num_kv_heads, L.dtype)
+        outs, lses = gather_partials(torch.from_numpy(part), torch.from_numpy(lse))
+        merged, merged_lse = oracle.merge_outputs(outs.numpy(), lses.numpy())
+        full, full_lse = oracle.decode_lse(V.q, V.k_pool, V.v_pool, L.block_tables, L.seq_lens, L.scale,
+                                           L.num_kv_heads, L.dtype)
+        fin = np.isfinite(full_lse)
+        out[rank] = (float(np.abs(merged - full).max()), float(np.abs(merged_lse[fin] - full_lse[fin]).max()),
+                     bool(np.array_equal(np.isinf(merged_lse), np.isinf(full_lse))), tuple(outs.shape))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_split_sequence_partials_gathered_and_merged_with_two_gloo_ranks():
+    """Two ranks each hold a block range of every sequence: their partial
+    decodes (the oracle's, on CPU) gathered by split.gather_partials and
+    merged equal the whole decode on both ranks."""
+    world = 2
+    out = mp.Manager().dict()
+    mp.spawn(_split_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
+    for rank in range(world):
+        err, lse_err, same_inf, shape = out[rank]
+        assert shape == (world, 5, 4, 16)
+        assert err < 1e-12 and lse_err < 1e-12 and same_inf
