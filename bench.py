@@ -217,6 +217,23 @@ def model_layers(L):
     return None, None
 
 
+def workload_config(L, world: int, mode: str, nbytes) -> dict:
+    """The workload keys of the JSON line's config, the same for both arms."""
+    import numpy as np
+
+    return {
+        "workload": L.name,
+        "note": L.note,
+        "global_batch": L.num_seqs * world,
+        "seq_len": {"mean": float(np.mean(L.seq_lens)), "min": int(L.seq_lens.min()),
+                    "max": int(L.seq_lens.max())},
+        "q_len": L.q_len,
+        "decode": mode,
+        "l2": f"no flush: per-step K/V {nbytes['decode'] / 1e9:.2f} GB > 126 MB L2",
+        "parallelism": f"dp{world} (independent sequence shards, no collective)",
+    }
+
+
 def decode_entry(L, mode: str) -> str:
     if L.q_len > 1:
         return "pa_decode_multi"
@@ -525,7 +542,9 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": L.name, "note": L.note},
+        "config": {**workload_config(L, int(os.environ.get("WORLD_SIZE", "1")), args.decode,
+                                     step_bytes(L, args.decode)),
+                   "step": "the oracle's copy, write and decode of the same step (float64, host cores)"},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "threads": 1, "kind": "oracle",
                          "host_cores": host_cores(), "sample": sample},
@@ -751,19 +770,11 @@ def run_ours(args):
             "dtype": L.dtype,
             "data": "synthetic",
             "config": {
-                "workload": L.name,
-                "note": L.note,
-                "global_batch": L.num_seqs * world,
-                "seq_len": {"mean": float(np.mean(L.seq_lens)), "min": int(L.seq_lens.min()),
-                            "max": int(L.seq_lens.max())},
+                **workload_config(L, world, mode, nbytes),
                 "step": (("pa_copy_blocks+" if has_copy else "") + decode_entry(L, mode)
                          + "_update (cache write + decode in one launch)") if fused else "+".join(
                     (["pa_copy_blocks"] if has_copy else []) + (["pa_cache_write"] if has_write else [])
                     + [decode_entry(L, mode)]),
-                "q_len": L.q_len,
-                "decode": mode,
-                "l2": f"no flush: per-step K/V {nbytes['decode'] / 1e9:.2f} GB > 126 MB L2",
-                "parallelism": f"dp{world} (independent sequence shards, no collective)",
             },
             "tokens_per_s": tokens_per_s,
             "tokens_per_s_note": ("one new token per sequence per single-layer step" if L.q_len == 1 else
