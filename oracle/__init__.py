@@ -18,9 +18,10 @@ Sources (the three pages this project follows):
   LLaMA-7B; its per-block-softmax toy code is NOT followed (it normalises each
   block on its own, which is not attention; the study notes §4 win).
 
-Every function is pinned by tests in ``tests/test_oracle.py`` against values
-the pages print, closed forms, invariants and brute force; none is
-"parity unpinned".
+Every function is pinned by tests in ``tests/test_oracle.py``,
+``tests/test_oracle_multi.py``, ``tests/test_oracle_bits.py`` and
+``tests/test_oracle_lse.py`` against values the pages print, closed forms,
+invariants and brute force; none is "parity unpinned".
 """
 
 from .paged_attention import (  # noqa: F401
