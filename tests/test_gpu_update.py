@@ -62,12 +62,14 @@ def _run_plain(L, V, device, *, fused, num_ctas=0, flags=0):
     return out, int(st.item()), d, ws
 
 
-@pytest.mark.parametrize("num_ctas", [0, 1, 5])
+@pytest.mark.parametrize("num_ctas", [0, 1, 5, 400])
 @pytest.mark.parametrize("B", [8, 16, 32])
 def test_update_decode_with_copies_and_writes(cuda_device, B, num_ctas):
     """Forked samples at the Llama-2-70B layer shape (64 q / 8 kv heads):
     nine copy-on-write pairs and twelve new tokens, some of them stored into
-    a block copied by the same call, then the GQA-8 decode."""
+    a block copied by the same call, then the GQA-8 decode.  With 400 CTAs,
+    more than fit on the GPU at once, the stores run as their own launch
+    (the in-launch barrier needs the whole grid resident)."""
     L = config_llama2_70b_shared(prompt_len=256, num_prompts=3, samples=4, max_tail=60, block_size=B)
     assert L.copy_pairs.shape[0] > 0 and L.num_new_tokens > 0
     V = fill_values_numpy(L)
