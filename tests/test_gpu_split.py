@@ -154,3 +154,46 @@ def test_decode_lse_only_on_tensor_cores(cuda_device):
             pa.pa_decode_lse(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], L.scale,
                              torch.empty_like(d["q"]), lse, ws, flags=flags)
         assert e.value.code == 2
+
+
+def test_decode_split_end_to_end_on_one_nccl_rank(cuda_device):
+    """split.decode_split through a one-rank NCCL process group on this GPU:
+    pa_decode_lse of the rank's range (here the whole sequences), the
+    all-gather, pa_merge_partials; the result is the whole decode."""
+    import datetime
+    import os
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_357_b200 as pa
+    from paged_kv_cache_357_b200.split import decode_split
+
+    L = random_layout(8300, [0, 1, 100, 4097, 777], dtype="bf16", block_size=16, num_q_heads=8, num_kv_heads=2,
+                      head_dim=128, write_new_token=False)
+    V = fill_values_numpy(L)
+    d = to_device(L, V, cuda_device)
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=cuda_device)
+    try:
+        out = torch.full_like(d["q"], float("nan"))
+        lse = torch.full(d["q"].shape[:2], float("nan"), dtype=torch.float32, device=cuda_device)
+        ws = pa.alloc_decode_workspace(L.num_seqs, L.num_q_heads, d["k_pool"])
+        st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+        decode_split(d["q"], d["k_pool"], d["v_pool"], d["tables"], d["lens"], L.scale, out, ws, st, lse_out=lse)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+    finally:
+        dist.destroy_process_group()
+    want_out, want_lse = oracle.decode_lse(V.q, V.k_pool, V.v_pool, L.block_tables, L.seq_lens, L.scale,
+                                           L.num_kv_heads, L.dtype)
+    got = torch_f64(out)
+    err = np.abs(got - want_out)
+    # one part: the merge rescales by exactly 1, so only the part's own rounding and the merge's add up
+    assert (err <= ATOL + RTOL * np.abs(want_out) + 2.0 ** -8 * np.abs(got)).all(), err.max()
+    _assert_lse_close(lse.double().cpu().numpy(), want_lse, "decode_split")
